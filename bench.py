@@ -1,0 +1,431 @@
+"""Benchmark of the TokenGate gated-prefill hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl tokengate|reference]
+                    [--workload c2_32k_k2000] [--layers 1] [--no-cpu-baseline]
+
+One step = one pass of the whole path over one batch of seeded synthetic
+input: gate scoring, top-K selection, compaction, and one token-gated
+attention layer (tg_gated_prefill_layer).  Default workload: Qwen3-1.7B
+shapes at N=32768 with K=2000 kept state tokens (M=2256 kept rows).
+
+Metric: gated-prefill layer tokens/s (N / step time), with the gated
+attention's TFLOP/s and its fraction of the measured bf16 peak reported
+beside it.  Inputs are resident in HBM when timing starts; L2 is flushed by
+a 256 MB write before every timed step (outside the step's events).
+
+Under torchrun (N>1) every rank runs an independent replica of the workload
+(the path is single-GPU; no collective on the data path), the value is the
+tokens of all ranks divided by the slowest rank's time, and scaling is weak.
+
+--impl reference times the fp64 CPU oracle on a bounded sample of the same
+workload, extrapolated to the whole workload; it is a slow program by design.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import re
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import get_config, make_attention_inputs, make_gate_inputs  # noqa: E402
+
+METRIC = "gated-prefill layer tokens/s; gated-attn TFLOP/s (% bf16 peak) at N=32k,K=2000"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "source": "fallback"}
+
+
+# ------------------------------------------------------------------ helpers
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    return dict(FALLBACK_PEAKS)
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def attention_flops(cu_kept, Hq, d):
+    m = np.diff(np.asarray(cu_kept, np.int64))
+    pairs = int(np.sum(m * (m + 1) // 2))
+    return 4.0 * d * Hq * pairs, pairs
+
+
+def stage_bytes(w, M):
+    """Algorithmic HBM bytes per launch of each stage (read + write)."""
+    n_prun = sum(p1 - p0 for p0, p1 in w.spans)
+    return {
+        # hidden rows of the span read once, one fp32 score written, Wg read once
+        "score": n_prun * (2 * w.D + 4) + 2 * w.I * w.D,
+        # scores read, keep flags written, compaction indices written
+        "select": n_prun * 4 + w.T * 1 + M * 16,
+        # kept rows read and written
+        "gather": M * 2 * 2 * w.D,
+    }
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv") \
+            if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else f"/tmp/tg_clocks_{os.getpid()}.csv"
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = max(mx, float(parts[2]))
+                except ValueError:
+                    continue
+                for nm, val in zip(names, parts[5:9]):
+                    if val.lower().startswith("active"):
+                        reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def read_traffic_table():
+    """Per-launch DRAM bytes from the committed ncu summary, keyed by kernel
+    and the sha of the source file it was captured from."""
+    path = os.path.join(ROOT, "profiles", "traffic.md")
+    out = {}
+    if not os.path.exists(path):
+        return out
+    for line in open(path):
+        m = re.match(r"\|\s*(\w+)\s*\|\s*([0-9a-f]{12})\s*\|\s*([\w.]+)\s*\|\s*([0-9.]+)\s*\|", line)
+        if m:
+            out[(m.group(1), m.group(3))] = (m.group(2), float(m.group(4)))
+    return out
+
+
+def source_sha(kernel_file: str) -> str:
+    import hashlib
+    p = os.path.join(ROOT, "learned_token_pruning_rmsnorm_b200", "csrc", kernel_file)
+    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:12]
+
+
+KERNEL_FILES = {"score": "k_gate.cu", "select": "k_select.cu", "gather": "k_select.cu",
+                "attention": "k_attention.cu"}
+
+
+# ------------------------------------------------------------------ oracle (CPU baseline / reference arm)
+
+def oracle_sample_pass(w, gi, Wg_bits, layer, score_rows=1024, attn_rows=48):
+    """One bounded pass of the fp64 oracle over a sample of the workload,
+    extrapolated to the whole workload.  Returns (est_seconds, sample_desc)."""
+    import oracle
+    cu, span, k = w.cu_seqlens(), w.span_array(), w.budget_array()
+    n_prun = int(sum(p1 - p0 for p0, p1 in w.spans))
+    # gate scores on the first `score_rows` prunable rows of sequence 0
+    sub_span = span.copy()
+    sub_span[:, 1] = np.minimum(span[:, 1], span[:, 0] + score_rows)
+    sub_span[1:, 1] = sub_span[1:, 0]
+    t0 = time.perf_counter()
+    s = oracle.score(gi["hidden"], cu, sub_span, Wg_bits, gi["b1"], gi["w2"], gi["b2"], w.eps)
+    t_score = (time.perf_counter() - t0) * n_prun / max(1, int(np.sum(sub_span[:, 1] - sub_span[:, 0])))
+    # selection + compaction on full-length scores (the oracle's real cost)
+    s32 = np.nan_to_num(s, nan=0.0).astype(np.float32)
+    t0 = time.perf_counter()
+    keep = oracle.select_topk(s32, cu, span, k)
+    comp = oracle.compact(gi["hidden"], s32, keep, cu, span)
+    t_sel = time.perf_counter() - t0
+    # attention on evenly spaced query rows; cost of a row is proportional to its causal length
+    cu_kept = comp["cu_kept"]
+    M = int(cu_kept[-1])
+    rows = np.linspace(0, M - 1, attn_rows).astype(np.int64)
+    t0 = time.perf_counter()
+    oracle.gated_attention(layer["q"], layer["k"], layer["v"], cu_kept, comp["pos"], comp["rank"],
+                           comp["gls"].astype(np.float32), layer["g"], layer["c"], rows=rows, want_lse=False)
+    t_attn_sample = time.perf_counter() - t0
+    b_of = np.searchsorted(cu_kept, rows, side="right") - 1
+    sampled_pairs = float(np.sum(rows - cu_kept[b_of] + 1))
+    _, pairs = attention_flops(cu_kept, w.Hq, w.d)
+    t_attn = t_attn_sample * pairs / sampled_pairs
+    desc = (f"oracle fp64: gate on {int(np.sum(sub_span[:, 1] - sub_span[:, 0]))} of {n_prun} prunable rows, "
+            f"full select+compact, attention on {attn_rows} of {M} query rows ({int(sampled_pairs)} of {pairs} "
+            f"causal pairs); times scaled to the whole workload")
+    return t_score + t_sel + t_attn, desc, {"score_s": t_score, "select_compact_s": t_sel, "attention_s": t_attn}
+
+
+def run_reference(args, w):
+    import oracle
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    gi = make_gate_inputs(w)
+    Wg = oracle.gate_fold(gi["gamma"], gi["W1"])
+    M = int(w.cu_kept()[-1])
+    layer = make_attention_inputs(w, M, layer=0)
+    times = []
+    desc = ""
+    for it in range(args.warmup + args.steps):
+        t, desc, _ = oracle_sample_pass(w, gi, Wg, layer, score_rows=1024, attn_rows=64)
+        if it >= args.warmup:
+            times.append(t)
+    t = float(np.mean(times))
+    value = w.T / t
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+            "config": workload_config(w, args.layers),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.get_threads(), "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w, n_layers):
+    M = int(w.cu_kept()[-1])
+    return {"workload": w.name, "B": w.B, "N": list(w.seqlens) if w.B > 1 else w.seqlens[0],
+            "K": list(w.budgets) if w.B > 1 else w.budgets[0], "M": M, "D": w.D, "I": w.I, "Hq": w.Hq,
+            "Hkv": w.Hkv, "head_dim": w.d, "attn_layers_per_step": n_layers,
+            "l2": "flushed (256 MB write) before every timed step", "parallelism": "replicas"}
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def run_gpu(args, w):
+    import torch
+    import torch.distributed as dist
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        dist.init_process_group("nccl", device_id=dev, timeout=__import__("datetime").timedelta(seconds=120))
+
+    import learned_token_pruning_rmsnorm_b200 as tg
+    from learned_token_pruning_rmsnorm_b200 import PrefillBuffers, PrefillCall
+
+    peaks = load_peaks()
+    gi = make_gate_inputs(w)
+    cu, span, k = w.cu_seqlens(), w.span_array(), w.budget_array()
+    M, cu_kept = tg.tg_kept_count(cu, span, k)
+
+    def bf16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+
+    hidden_h = bf16(gi["hidden"]).pin_memory()
+    hidden = hidden_h.to(dev)
+    Wg = tg.tg_gate_prepare(bf16(gi["gamma"]).to(dev), bf16(gi["W1"]).to(dev))
+    b1 = torch.from_numpy(gi["b1"]).to(dev)
+    w2 = torch.from_numpy(gi["w2"]).to(dev)
+    layers_np = [make_attention_inputs(w, M, layer=l) for l in range(args.layers)]
+    layers_h = [{"q": bf16(a["q"]).pin_memory(), "k": bf16(a["k"]).pin_memory(), "v": bf16(a["v"]).pin_memory(),
+                 "g": torch.from_numpy(a["g"]).pin_memory(), "c": torch.from_numpy(a["c"]).pin_memory()}
+                for a in layers_np]
+    layers = [{key: t.to(dev) for key, t in L.items()} for L in layers_h]
+    bufs = PrefillBuffers(w.T, w.D, M, args.layers, w.Hq, w.d, dev, with_hidden=True)
+    call = PrefillCall(hidden, cu, span, k, Wg, b1, w2, gi["b2"], w.eps, layers, bufs, w.Hq, w.Hkv, w.d)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.int32, device=dev)
+    st = torch.cuda.current_stream(dev)
+
+    def barrier():
+        if ws > 1:
+            dist.barrier()
+
+    # warm-up
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize(dev)
+
+    # ---------------- timed region: K whole-path steps
+    clocks = ClockSampler(local)
+    clocks.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.fill_(i)
+        ev[i][0].record(st)
+        call()
+        ev[i][1].record(st)
+    torch.cuda.synchronize(dev)
+    barrier()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+
+    # ---------------- per-stage breakdown over K more steps (same stream)
+    sev = {s: [] for s in ("score", "select", "gather", "attention")}
+    for i in range(args.steps):
+        flush.fill_(i)
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        e[0].record(st)
+        tg.tg_score(hidden, call.cu, call.sp, Wg, b1, w2, gi["b2"], w.eps, scores=bufs.scores)
+        e[1].record(st)
+        tg.tg_select_topk(bufs.scores, call.cu, call.sp, call.kk, keep=bufs.keep)
+        e[2].record(st)
+        tg.tg_compact(hidden, bufs.scores, bufs.keep, call.cu, call.sp, call.ck, M)
+        e[3].record(st)
+        tg.tg_gated_attention(layers[0]["q"], layers[0]["k"], layers[0]["v"], call.ck, call.max_M, bufs.pos,
+                              bufs.rank, bufs.gls, layers[0]["g"], layers[0]["c"], out=bufs.out[0])
+        e[4].record(st)
+        sev["score"].append((e[0], e[1]))
+        sev["select"].append((e[1], e[2]))
+        sev["gather"].append((e[2], e[3]))
+        sev["attention"].append((e[3], e[4]))
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    stage_us = {s: 1e3 * float(np.mean([a.elapsed_time(b) for a, b in v])) for s, v in sev.items()}
+
+    # ---------------- end to end: pinned host inputs in, result out, every step
+    out_h = torch.empty((M, w.Hq, w.d), dtype=torch.bfloat16).pin_memory()
+    idx_h = torch.empty(M, dtype=torch.int32).pin_memory()
+    h2d = hidden_h.numel() * 2 + sum(L[key].numel() * L[key].element_size() for L in layers_h for key in L)
+    d2h = out_h.numel() * 2 + idx_h.numel() * 4
+    e2e_ev = []
+    for i in range(args.warmup + args.steps):
+        flush.fill_(i)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        hidden.copy_(hidden_h, non_blocking=True)
+        for L, Lh in zip(layers, layers_h):
+            for key in L:
+                L[key].copy_(Lh[key], non_blocking=True)
+        call()
+        out_h.copy_(bufs.out[-1], non_blocking=True)
+        idx_h.copy_(bufs.kept_idx, non_blocking=True)
+        b.record(st)
+        if i >= args.warmup:
+            e2e_ev.append((a, b))
+    torch.cuda.synchronize(dev)
+    e2e_ms = float(np.sum([a.elapsed_time(b) for a, b in e2e_ev]))
+
+    # ---------------- max over ranks
+    t_total_ms = float(np.sum(step_ms))
+    vals = torch.tensor([t_total_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if ws > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    t_total_ms, e2e_ms = float(vals[0]), float(vals[1])
+
+    ms_per_step = t_total_ms / args.steps
+    value = ws * w.T * args.steps / (t_total_ms / 1e3)
+    e2e_value = ws * w.T * args.steps / (e2e_ms / 1e3)
+
+    flops, pairs = attention_flops(cu_kept, w.Hq, w.d)
+    attn_tflops = flops / (stage_us["attention"] * 1e-6) / 1e12
+    sb = stage_bytes(w, M)
+    stage_gbs = {s: sb[s] / (stage_us[s] * 1e-6) / 1e9 for s in sb}
+    hbm_peak = float(peaks["hbm_gbs"])
+    tc_peak = float(peaks["bf16_tflops"])
+    # dominant kernel = the stage with the largest share of the step
+    dom = max(stage_us, key=stage_us.get)
+    traffic_tab = read_traffic_table()
+    traffic = None
+    key = (dom, w.name)
+    if key in traffic_tab and traffic_tab[key][0] == source_sha(KERNEL_FILES[dom]):
+        traffic = traffic_tab[key][1]
+    if dom == "attention":
+        roof = {"bound": "tensor", "achieved": attn_tflops, "peak": tc_peak, "unit": "TFLOP/s",
+                "frac": attn_tflops / tc_peak, "traffic": traffic, "kernel": "gated_attention",
+                "algorithmic": f"{flops:.4g} FLOP per launch = 4*d*Hq*{pairs} causal pairs",
+                "peak_source": f"{peaks['source']} bf16_tflops (burst)"}
+    else:
+        roof = {"bound": "hbm", "achieved": stage_gbs[dom], "peak": hbm_peak, "unit": "GB/s",
+                "frac": stage_gbs[dom] / hbm_peak, "traffic": traffic, "kernel": dom,
+                "algorithmic": f"{sb[dom]} bytes per launch", "peak_source": f"{peaks['source']} hbm_gbs"}
+    s13_bytes = sb["score"] + sb["select"] + sb["gather"]
+    s13_us = stage_us["score"] + stage_us["select"] + stage_us["gather"]
+
+    cpu_base = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        import oracle
+        Wg_bits = oracle.gate_fold(gi["gamma"], gi["W1"])
+        t_est, desc, parts = oracle_sample_pass(w, gi, Wg_bits, layers_np[0], score_rows=8192, attn_rows=512)
+        cpu_base = {"value": w.T / t_est, "unit": UNIT, "cores": oracle.get_threads(), "kind": "oracle",
+                    "sample": desc, "est_seconds_per_step": t_est, "parts_s": parts}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; Qwen3-1.7B gate-layer shapes)",
+                "config": workload_config(w, args.layers),
+                "roofline": roof,
+                "gated_attn": {"tflops": attn_tflops, "frac_of_bf16_peak": attn_tflops / tc_peak,
+                               "us": stage_us["attention"], "flops": flops},
+                "score_select_compact": {"us": s13_us, "bytes": s13_bytes, "gbs": s13_bytes / (s13_us * 1e-6) / 1e9,
+                                         "frac_of_hbm": s13_bytes / (s13_us * 1e-6) / 1e9 / hbm_peak},
+                "stage_us": stage_us, "stage_gbs": stage_gbs,
+                "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+                        "d2h_bytes_per_step": int(d2h)},
+                "gpu_launches": args.steps * (3 + args.layers),
+                "cpu_baseline": cpu_base, "clocks": clk, "peaks": {"source": peaks["source"],
+                                                                   "hbm_gbs": hbm_peak, "bf16_tflops": tc_peak}}
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["tokengate", "reference"], default="tokengate")
+    ap.add_argument("--workload", default="c2_32k_k2000")
+    ap.add_argument("--layers", type=int, default=1)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = get_config(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

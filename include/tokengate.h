@@ -1,0 +1,215 @@
+/*
+ * tokengate.h -- C ABI of libtokengate.so, the B200 (sm_100a) implementation
+ * of TokenGate's gated-prefill hot path.
+ *
+ * The method (TokenGate: Adapting LLMs for Fast and Memory-Efficient Prefill
+ * with Learned Token Pruning; AI summary page, "Key Contributions" 1-3 and
+ * "Methodology in Plain English"; README copy, "How it works"):
+ *   1. at gate layer L, score every prunable token with RMSNorm followed by
+ *      a small MLP over its post-attention residual          -> tg_score
+ *   2. keep the K best prunable tokens plus every non-prunable one
+ *                                                           -> tg_select_topk
+ *   3. hand only the kept tokens, in order, to the layers above -> tg_compact
+ *   4. token-gated attention in those layers: causal GQA attention over the
+ *      kept tokens with a per-key, per-head gate bias and a per-query
+ *      temperature                                      -> tg_gated_attention
+ *   tg_gated_prefill_layer chains 1-4 on one stream.
+ *
+ * The pages describe the bias and the temperature only in prose ("a per-key
+ * gate bias", "a learnable per-layer, per-head gain passed through softplus",
+ * "a temperature scaled by the log-ratio of a query's original position to
+ * its rank among kept tokens").  This library defines them as
+ *     b[h,j]   = softplus(g_h) * logsigmoid(s_j)      (0 for non-prunable j)
+ *     tau[q,h] = 1 + c_h * ln(pos_q / rank_q)
+ *     logit    = (q.k_j * sm_scale + b[h,j]) / tau[q,h]
+ * with g_h, c_h caller inputs (one per query head and layer).
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are DEVICE pointers owned by the caller; the library never
+ *     allocates, frees or keeps them.  Host pointers are marked h_.
+ *   - bf16 tensors are passed as uint16_t bit patterns; all layouts are
+ *     row-major and densely packed.
+ *   - Sequences use the varlen layout: B sequences concatenated into T
+ *     tokens, cu_seqlens[B+1] (int32, device) the prefix sums of the lengths.
+ *     span[2*b], span[2*b+1] (int32, device) is sequence b's prunable span
+ *     [p0, p1) in sequence-local token indices (the `{state}` document).
+ *     k[b] (int32, device) is the keep budget; k < 0 keeps every prunable
+ *     token, k >= |P_b| too, k == 0 keeps only the non-prunable tokens.
+ *   - The kept count of sequence b is M_b = (N_b - |P_b|) + min(K_b, |P_b|);
+ *     it depends on no score, so the caller sizes every output on the host
+ *     with tg_kept_count and passes cu_kept (device copy) back in.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream).  Arguments are validated on the host before anything
+ *     is launched; a rejected call launches nothing and returns
+ *     TG_ERR_INVALID_ARG or TG_ERR_UNSUPPORTED.  TG_ERR_CUDA reports a launch
+ *     error.  No exception crosses the ABI.  tg_last_error_string() describes
+ *     the last failure of the calling thread.
+ *   - Supported shapes: D a multiple of 64 (<= 8192); I a multiple of 16 in
+ *     [16, 256]; head_dim 64 or 128; Hq a multiple of Hkv; sm_100 devices.
+ */
+#ifndef TOKENGATE_H
+#define TOKENGATE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* tg_stream_t; /* the same type as cudaStream_t */
+
+typedef enum tg_status {
+    TG_OK = 0,
+    TG_ERR_INVALID_ARG = 1, /* null pointer, bad size, inconsistent shapes */
+    TG_ERR_UNSUPPORTED = 2, /* shape or device outside the supported set */
+    TG_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
+    TG_ERR_TIMEOUT = 4      /* reserved: a bounded device-side wait gave up */
+} tg_status;
+
+/* Version of this ABI (incremented on any signature change). */
+int tg_abi_version(void);
+
+/* Message for the last non-OK status returned on the calling thread. */
+const char* tg_last_error_string(void);
+
+/*
+ * Kept-token count (host only, no device work).
+ * TokenGate README copy, "Quick start": every token outside `{state}` is
+ * kept, plus max_kept_prefill_tokens=K of the state tokens (None = all).
+ * h_cu_seqlens[B+1], h_span[2B], h_k[B] are host arrays; h_cu_kept[B+1]
+ * (host, caller-owned) receives the prefix sums of M_b.  Returns the total
+ * M = sum_b M_b, or -1 on invalid input (see tg_last_error_string).
+ */
+int64_t tg_kept_count(const int32_t* h_cu_seqlens, const int32_t* h_span, const int32_t* h_k, int B,
+                      int32_t* h_cu_kept);
+
+/*
+ * Gate weight preparation (once per gate, not on the per-request path).
+ * The RMSNorm weight gamma [D] is folded into the first gate layer
+ * W1 [D, I]:  Wg[j*D + i] = bf16_rne(gamma[i] * W1[i*I + j])  ->  Wg [I, D].
+ * The product of two bf16 numbers is exact in fp32, so the one rounding is
+ * the final round-to-nearest-even.  RMSNorm's 1/rms factor is applied after
+ * the contraction inside tg_score (AI summary, "Key Contributions" 1: MLP
+ * over the RMSNorm-normalised residual).
+ */
+tg_status tg_gate_prepare(const uint16_t* gamma, const uint16_t* W1, int D, int I, uint16_t* Wg,
+                          tg_stream_t stream);
+
+/*
+ * Stage 1: gate score of every prunable token (AI summary, "Key
+ * Contributions" 1; TokenGate explained blog, "how the gate works").
+ *   r_t = 1 / sqrt(mean_i x_ti^2 + eps)
+ *   s_t = b2 + sum_j w2[j] * SiLU(r_t * (Wg[j,:] . x_t) + b1[j])
+ * hidden [T, D] bf16; Wg [I, D] bf16 from tg_gate_prepare; b1 [I], w2 [I]
+ * fp32; scores [T] fp32 (out).  Only prunable entries are written; the
+ * others keep their previous contents.  The contraction runs on the tensor
+ * cores in fp32 accumulation over the exact bf16 inputs.
+ */
+tg_status tg_score(const uint16_t* hidden, const int32_t* cu_seqlens, const int32_t* span, int B, int64_t T,
+                   int D, const uint16_t* Wg, const float* b1, const float* w2, float b2, int I, float eps,
+                   float* scores, tg_stream_t stream);
+
+/*
+ * Stage 2: deterministic top-K per sequence over the prunable span (AI
+ * summary, "Key Contributions" 1 and "Methodology in Plain English").
+ * Order: higher score first, equal scores by lower token index; -0 equals
+ * +0; NaN ranks below every number.  keep [T] uint8 (out): 1 for every
+ * non-prunable token and for the selected prunable ones, else 0.
+ * Bit-exact and run-to-run deterministic.
+ */
+tg_status tg_select_topk(const float* scores, const int32_t* cu_seqlens, const int32_t* span, const int32_t* k,
+                         int B, int64_t T, uint8_t* keep, tg_stream_t stream);
+
+/*
+ * Stage 3: stable compaction of the kept tokens (AI summary, "Key
+ * Contributions" 1: the layers above L see only kept tokens and create no
+ * KV entries for pruned ones).  For the m-th kept token t of sequence b
+ * (m counted over the whole batch, in original order):
+ *   hidden_kept[m, :] = hidden[t, :]          (bytes copied unchanged)
+ *   pos[m]      = t - cu_seqlens[b] + 1       (1-indexed original position)
+ *   rank[m]     = m - cu_kept[b] + 1          (1-indexed rank among kept)
+ *   gls[m]      = logsigmoid(scores[t]) if t is prunable, else 0
+ *   kept_idx[m] = t                           (source row; the gather map)
+ * cu_kept [B+1] (device) must hold tg_kept_count's prefix sums; M_total is
+ * cu_kept[B].  hidden_kept may be NULL (then only the index outputs are
+ * written); pos, rank, gls, kept_idx are required.
+ */
+tg_status tg_compact(const uint16_t* hidden, const float* scores, const uint8_t* keep, const int32_t* cu_seqlens,
+                     const int32_t* span, int B, int64_t T, int D, const int32_t* cu_kept, int64_t M_total,
+                     uint16_t* hidden_kept, int32_t* pos, int32_t* rank, float* gls, int32_t* kept_idx,
+                     tg_stream_t stream);
+
+/*
+ * Stage 4: token-gated causal GQA attention over the kept tokens, one upper
+ * layer (AI summary, "Key Contributions" 2 and 3; the definitions of b and
+ * tau are at the top of this file).
+ * q [M, Hq, d], k/v [M, Hkv, d] bf16 (M = cu_kept[B]); pos, rank [M] int32
+ * and gls [M] fp32 from tg_compact; g, c [Hq] fp32; out [M, Hq, d] bf16.
+ * Query i of sequence b attends to the kept keys j of b with j <= i (that
+ * is rank_j <= rank_i); query head h reads KV head h / (Hq / Hkv).
+ * lse [M, Hq] fp32 (optional, may be NULL): natural-log softmax
+ * normaliser of each (query, head) row.  max_M is an upper bound of the
+ * longest sequence's M_b (grid sizing).  sm_scale is usually 1/sqrt(d).
+ * tau must stay positive: c_h >= 0 guarantees it since pos >= rank.
+ * Tensor cores: bf16 operands, fp32 accumulation.
+ */
+tg_status tg_gated_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* cu_kept,
+                             int B, int64_t M_total, int max_M, int Hq, int Hkv, int d, const int32_t* pos,
+                             const int32_t* rank, const float* gls, const float* g, const float* c, float sm_scale,
+                             uint16_t* out, float* lse, tg_stream_t stream);
+
+/*
+ * The whole gated prefill at one gate layer: tg_score, tg_select_topk,
+ * tg_compact and then n_layers gated-attention layers above the gate, all
+ * on one stream with no host synchronisation between them.  Fields mirror
+ * the stage arguments above; per-layer tensors are arrays of n_layers
+ * device pointers (the array itself lives in host memory).  The
+ * projections that turn hidden_kept into each layer's q/k/v belong to the
+ * model, not to this method, so q/k/v are inputs sized [M, ...].
+ */
+typedef struct tg_prefill_layer_args {
+    /* stage 1-3 */
+    const uint16_t* hidden;     /* [T, D] */
+    const int32_t* cu_seqlens;  /* [B+1] device */
+    const int32_t* span;        /* [2B] device */
+    const int32_t* k;           /* [B] device */
+    int B;
+    int64_t T;
+    int D;
+    const uint16_t* Wg;         /* [I, D] */
+    const float* b1;            /* [I] */
+    const float* w2;            /* [I] */
+    float b2;
+    int I;
+    float eps;
+    const int32_t* cu_kept;     /* [B+1] device, from tg_kept_count */
+    int64_t M_total;
+    int max_M;
+    float* scores;              /* [T] out */
+    uint8_t* keep;              /* [T] out */
+    uint16_t* hidden_kept;      /* [M, D] out, may be NULL */
+    int32_t* pos;               /* [M] out */
+    int32_t* rank;              /* [M] out */
+    float* gls;                 /* [M] out */
+    int32_t* kept_idx;          /* [M] out */
+    /* stage 4, n_layers times */
+    int n_layers;
+    int Hq, Hkv, d;
+    float sm_scale;
+    const uint16_t* const* q;   /* n_layers x [M, Hq, d] */
+    const uint16_t* const* kk;  /* n_layers x [M, Hkv, d] */
+    const uint16_t* const* v;   /* n_layers x [M, Hkv, d] */
+    const float* const* g;      /* n_layers x [Hq] */
+    const float* const* c;      /* n_layers x [Hq] */
+    uint16_t* const* out;       /* n_layers x [M, Hq, d] out */
+    float* const* lse;          /* n_layers x [M, Hq] out, array or entries may be NULL */
+} tg_prefill_layer_args;
+
+tg_status tg_gated_prefill_layer(const tg_prefill_layer_args* args, tg_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TOKENGATE_H */

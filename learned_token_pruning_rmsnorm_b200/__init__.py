@@ -1,0 +1,247 @@
+"""TokenGate gated-prefill hot path on B200 (sm_100a).
+
+Thin Python binding over the C ABI of libtokengate.so (include/tokengate.h).
+The functions carry the C names; each marshals torch CUDA tensors into raw
+pointers plus the current stream and calls the library.  Nothing here
+computes: scoring, selection, compaction and attention all run in the CUDA
+kernels, and a missing library is an error, not a fallback.
+
+Tensors: bf16 as torch.bfloat16, fp32 as torch.float32, indices as
+torch.int32, keep flags as torch.uint8; all contiguous on one CUDA device.
+"""
+
+from __future__ import annotations
+
+import ctypes as C
+import math
+
+import numpy as np
+import torch
+
+from . import _lib
+from ._lib import TokenGateError, load  # noqa: F401
+
+__all__ = [
+    "TokenGateError", "load", "tg_abi_version", "tg_kept_count", "tg_gate_prepare", "tg_score",
+    "tg_select_topk", "tg_compact", "tg_gated_attention", "tg_gated_prefill_layer",
+]
+
+
+def _dev(t: torch.Tensor, dtype, name: str, shape=None) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    return t
+
+
+def _i32_dev(a, device, name: str) -> torch.Tensor:
+    if isinstance(a, torch.Tensor) and a.is_cuda:
+        return _dev(a, torch.int32, name)
+    return torch.from_numpy(_lib.host_i32(a)).to(device)
+
+
+def tg_abi_version() -> int:
+    return int(load().tg_abi_version())
+
+
+def tg_kept_count(cu_seqlens, span, k):
+    """Host-side kept counts: returns (M_total, cu_kept as a numpy int32 array)."""
+    cu = _lib.host_i32(cu_seqlens)
+    sp = _lib.host_i32(span).reshape(-1)
+    kk = _lib.host_i32(k).reshape(-1)
+    B = len(cu) - 1
+    out = np.zeros(B + 1, dtype=np.int32)
+    tot = load().tg_kept_count(cu.ctypes.data, sp.ctypes.data, kk.ctypes.data, B, out.ctypes.data)
+    if tot < 0:
+        _lib.check(_lib.TG_ERR_INVALID_ARG)
+    return int(tot), out
+
+
+def tg_gate_prepare(gamma: torch.Tensor, W1: torch.Tensor, Wg: torch.Tensor | None = None) -> torch.Tensor:
+    D, I = W1.shape
+    _dev(gamma, torch.bfloat16, "gamma", (D,))
+    _dev(W1, torch.bfloat16, "W1")
+    if Wg is None:
+        Wg = torch.empty((I, D), dtype=torch.bfloat16, device=W1.device)
+    _dev(Wg, torch.bfloat16, "Wg", (I, D))
+    _lib.check(load().tg_gate_prepare(gamma.data_ptr(), W1.data_ptr(), D, I, Wg.data_ptr(),
+                                      _lib.stream_handle(W1.device)))
+    return Wg
+
+
+def tg_score(hidden, cu_seqlens, span, Wg, b1, w2, b2: float, eps: float = 1e-6, scores=None):
+    T, D = hidden.shape
+    I = Wg.shape[0]
+    dev = hidden.device
+    _dev(hidden, torch.bfloat16, "hidden")
+    _dev(Wg, torch.bfloat16, "Wg", (I, D))
+    _dev(b1, torch.float32, "b1", (I,))
+    _dev(w2, torch.float32, "w2", (I,))
+    cu = _i32_dev(cu_seqlens, dev, "cu_seqlens")
+    sp = _i32_dev(span, dev, "span")
+    if scores is None:
+        scores = torch.zeros(T, dtype=torch.float32, device=dev)
+    _dev(scores, torch.float32, "scores", (T,))
+    _lib.check(load().tg_score(hidden.data_ptr(), cu.data_ptr(), sp.data_ptr(), cu.numel() - 1, T, D,
+                               Wg.data_ptr(), b1.data_ptr(), w2.data_ptr(), float(b2), I, float(eps),
+                               scores.data_ptr(), _lib.stream_handle(dev)))
+    return scores
+
+
+def tg_select_topk(scores, cu_seqlens, span, k, keep=None):
+    T = scores.shape[0]
+    dev = scores.device
+    _dev(scores, torch.float32, "scores")
+    cu = _i32_dev(cu_seqlens, dev, "cu_seqlens")
+    sp = _i32_dev(span, dev, "span")
+    kk = _i32_dev(k, dev, "k")
+    if keep is None:
+        keep = torch.empty(T, dtype=torch.uint8, device=dev)
+    _dev(keep, torch.uint8, "keep", (T,))
+    _lib.check(load().tg_select_topk(scores.data_ptr(), cu.data_ptr(), sp.data_ptr(), kk.data_ptr(),
+                                     cu.numel() - 1, T, keep.data_ptr(), _lib.stream_handle(dev)))
+    return keep
+
+
+def tg_compact(hidden, scores, keep, cu_seqlens, span, cu_kept, M_total: int, with_hidden: bool = True):
+    """Returns a dict with hidden_kept (or None), pos, rank, gls, kept_idx."""
+    T = scores.shape[0]
+    dev = scores.device
+    _dev(scores, torch.float32, "scores", (T,))
+    _dev(keep, torch.uint8, "keep", (T,))
+    D = hidden.shape[1] if hidden is not None else 0
+    if hidden is not None:
+        _dev(hidden, torch.bfloat16, "hidden", (T, D))
+    cu = _i32_dev(cu_seqlens, dev, "cu_seqlens")
+    sp = _i32_dev(span, dev, "span")
+    ck = _i32_dev(cu_kept, dev, "cu_kept")
+    M = int(M_total)
+    hk = torch.empty((M, D), dtype=torch.bfloat16, device=dev) if (with_hidden and hidden is not None) else None
+    pos = torch.empty(M, dtype=torch.int32, device=dev)
+    rank = torch.empty(M, dtype=torch.int32, device=dev)
+    gls = torch.empty(M, dtype=torch.float32, device=dev)
+    kept_idx = torch.empty(M, dtype=torch.int32, device=dev)
+    _lib.check(load().tg_compact(_lib.ptr(hidden), scores.data_ptr(), keep.data_ptr(), cu.data_ptr(),
+                                 sp.data_ptr(), cu.numel() - 1, T, D, ck.data_ptr(), M, _lib.ptr(hk),
+                                 pos.data_ptr(), rank.data_ptr(), gls.data_ptr(), kept_idx.data_ptr(),
+                                 _lib.stream_handle(dev)))
+    return {"hidden_kept": hk, "pos": pos, "rank": rank, "gls": gls, "kept_idx": kept_idx}
+
+
+def tg_gated_attention(q, k, v, cu_kept, max_M: int, pos, rank, gls, g, c, sm_scale: float | None = None,
+                       out=None, lse=None, want_lse: bool = False):
+    M, Hq, d = q.shape
+    Hkv = k.shape[1]
+    dev = q.device
+    _dev(q, torch.bfloat16, "q")
+    _dev(k, torch.bfloat16, "k", (M, Hkv, d))
+    _dev(v, torch.bfloat16, "v", (M, Hkv, d))
+    _dev(pos, torch.int32, "pos", (M,))
+    _dev(rank, torch.int32, "rank", (M,))
+    _dev(gls, torch.float32, "gls", (M,))
+    _dev(g, torch.float32, "g", (Hq,))
+    _dev(c, torch.float32, "c", (Hq,))
+    ck = _i32_dev(cu_kept, dev, "cu_kept")
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((M, Hq, d), dtype=torch.bfloat16, device=dev)
+    _dev(out, torch.bfloat16, "out", (M, Hq, d))
+    if lse is None and want_lse:
+        lse = torch.empty((M, Hq), dtype=torch.float32, device=dev)
+    if lse is not None:
+        _dev(lse, torch.float32, "lse", (M, Hq))
+    _lib.check(load().tg_gated_attention(q.data_ptr(), k.data_ptr(), v.data_ptr(), ck.data_ptr(), ck.numel() - 1,
+                                         M, int(max_M), Hq, Hkv, d, pos.data_ptr(), rank.data_ptr(),
+                                         gls.data_ptr(), g.data_ptr(), c.data_ptr(), float(sm_scale),
+                                         out.data_ptr(), _lib.ptr(lse), _lib.stream_handle(dev)))
+    return (out, lse) if want_lse or lse is not None else out
+
+
+class PrefillBuffers:
+    """Device outputs of one gated prefill, sized on the host from (N, span, K)."""
+
+    def __init__(self, T, D, M, n_layers, Hq, d, device, with_hidden=True, with_lse=False):
+        self.scores = torch.zeros(T, dtype=torch.float32, device=device)
+        self.keep = torch.empty(T, dtype=torch.uint8, device=device)
+        self.hidden_kept = torch.empty((M, D), dtype=torch.bfloat16, device=device) if with_hidden else None
+        self.pos = torch.empty(M, dtype=torch.int32, device=device)
+        self.rank = torch.empty(M, dtype=torch.int32, device=device)
+        self.gls = torch.empty(M, dtype=torch.float32, device=device)
+        self.kept_idx = torch.empty(M, dtype=torch.int32, device=device)
+        self.out = [torch.empty((M, Hq, d), dtype=torch.bfloat16, device=device) for _ in range(n_layers)]
+        self.lse = [torch.empty((M, Hq), dtype=torch.float32, device=device) for _ in range(n_layers)] \
+            if with_lse else None
+
+
+class PrefillCall:
+    """A prepared tg_gated_prefill_layer call: the argument struct and the
+    host pointer arrays are built once, so that repeated launches (timing
+    loops, CUDA-graph capture) only cross the ABI."""
+
+    def __init__(self, hidden, cu_seqlens, span, k, Wg, b1, w2, b2, eps, layers, bufs: PrefillBuffers,
+                 Hq, Hkv, d, sm_scale=None):
+        dev = hidden.device
+        T, D = hidden.shape
+        I = Wg.shape[0]
+        self.cu = _i32_dev(cu_seqlens, dev, "cu_seqlens")
+        self.sp = _i32_dev(span, dev, "span")
+        self.kk = _i32_dev(k, dev, "k")
+        M, cu_kept = tg_kept_count(cu_seqlens if not isinstance(cu_seqlens, torch.Tensor) else cu_seqlens.cpu(),
+                                   span if not isinstance(span, torch.Tensor) else span.cpu(),
+                                   k if not isinstance(k, torch.Tensor) else k.cpu())
+        self.M = M
+        self.max_M = int(np.max(np.diff(cu_kept))) if len(cu_kept) > 1 else 0
+        self.ck = torch.from_numpy(cu_kept).to(dev)
+        self.keep_alive = [hidden, Wg, b1, w2, bufs, layers]
+        nl = len(layers)
+        arr = lambda xs: (C.c_void_p * max(nl, 1))(*[x for x in xs])  # noqa: E731
+        self._q = arr([L["q"].data_ptr() for L in layers])
+        self._k = arr([L["k"].data_ptr() for L in layers])
+        self._v = arr([L["v"].data_ptr() for L in layers])
+        self._g = arr([L["g"].data_ptr() for L in layers])
+        self._c = arr([L["c"].data_ptr() for L in layers])
+        self._o = arr([o.data_ptr() for o in bufs.out])
+        self._lse = arr([x.data_ptr() for x in bufs.lse]) if bufs.lse is not None else None
+        a = _lib.PrefillLayerArgs()
+        a.hidden, a.cu_seqlens, a.span, a.k = hidden.data_ptr(), self.cu.data_ptr(), self.sp.data_ptr(), \
+            self.kk.data_ptr()
+        a.B, a.T, a.D = self.cu.numel() - 1, T, D
+        a.Wg, a.b1, a.w2, a.b2, a.I, a.eps = Wg.data_ptr(), b1.data_ptr(), w2.data_ptr(), float(b2), I, float(eps)
+        a.cu_kept, a.M_total, a.max_M = self.ck.data_ptr(), M, self.max_M
+        a.scores, a.keep = bufs.scores.data_ptr(), bufs.keep.data_ptr()
+        a.hidden_kept = _lib.ptr(bufs.hidden_kept)
+        a.pos, a.rank, a.gls, a.kept_idx = bufs.pos.data_ptr(), bufs.rank.data_ptr(), bufs.gls.data_ptr(), \
+            bufs.kept_idx.data_ptr()
+        a.n_layers, a.Hq, a.Hkv, a.d = nl, Hq, Hkv, d
+        a.sm_scale = float(1.0 / math.sqrt(d) if sm_scale is None else sm_scale)
+        cast = lambda x: C.cast(x, C.c_void_p) if x is not None else None  # noqa: E731
+        a.q, a.kk, a.v, a.g, a.c, a.out = (cast(self._q), cast(self._k), cast(self._v), cast(self._g),
+                                           cast(self._c), cast(self._o))
+        a.lse = cast(self._lse)
+        self.args = a
+        self.device = dev
+        self.bufs = bufs
+
+    def __call__(self, stream: int | None = None):
+        st = _lib.stream_handle(self.device) if stream is None else stream
+        _lib.check(load().tg_gated_prefill_layer(C.byref(self.args), st))
+        return self.bufs
+
+
+def tg_gated_prefill_layer(hidden, cu_seqlens, span, k, Wg, b1, w2, b2, eps, layers, Hq, Hkv, d,
+                           sm_scale=None, with_hidden=True, with_lse=False):
+    """One call of the whole gated prefill.  `layers` is a list of dicts with
+    q, k, v (bf16 [M, H, d]) and g, c (fp32 [Hq]).  Returns PrefillBuffers."""
+    T, D = hidden.shape
+    M, _ = tg_kept_count(cu_seqlens if not isinstance(cu_seqlens, torch.Tensor) else cu_seqlens.cpu(),
+                         span if not isinstance(span, torch.Tensor) else span.cpu(),
+                         k if not isinstance(k, torch.Tensor) else k.cpu())
+    bufs = PrefillBuffers(T, D, M, len(layers), Hq, d, hidden.device, with_hidden, with_lse)
+    call = PrefillCall(hidden, cu_seqlens, span, k, Wg, b1, w2, b2, eps, layers, bufs, Hq, Hkv, d, sm_scale)
+    return call()

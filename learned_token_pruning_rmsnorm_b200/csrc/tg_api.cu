@@ -1,0 +1,234 @@
+// C ABI of libtokengate.so: argument validation, then the stage launches.
+// Every entry point checks its arguments on the host and returns before any
+// launch when they are wrong; no exception crosses the ABI.
+
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+
+#include "tg_internal.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+tg_status fail(tg_status st, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    std::vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return st;
+}
+
+tg_status cuda_status(cudaError_t e, const char* where) {
+    if (e == cudaSuccess) return TG_OK;
+    return fail(TG_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+// The kernels are built for sm_100a only.
+tg_status check_device() {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_status(e, "cudaGetDevice");
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (major != 10 || minor != 0)
+        return fail(TG_ERR_UNSUPPORTED, "device %d is sm_%d%d; libtokengate is built for sm_100a only", dev, major,
+                    minor);
+    return TG_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define TG_REQUIRE(cond, ...)                                   \
+    do {                                                        \
+        if (!(cond)) return fail(TG_ERR_INVALID_ARG, __VA_ARGS__); \
+    } while (0)
+
+#define TG_SUPPORT(cond, ...)                                   \
+    do {                                                        \
+        if (!(cond)) return fail(TG_ERR_UNSUPPORTED, __VA_ARGS__); \
+    } while (0)
+
+tg_status check_gate_shape(int D, int I) {
+    TG_SUPPORT(D >= 64 && D <= 8192 && D % 64 == 0, "D=%d must be a multiple of 64 in [64, 8192]", D);
+    TG_SUPPORT(I >= 16 && I <= 256 && I % 16 == 0, "I=%d must be a multiple of 16 in [16, 256]", I);
+    return TG_OK;
+}
+
+tg_status check_attn_shape(int Hq, int Hkv, int d) {
+    TG_SUPPORT(d == 64 || d == 128, "head_dim %d must be 64 or 128", d);
+    TG_REQUIRE(Hq > 0 && Hkv > 0 && Hq % Hkv == 0, "Hq=%d must be a positive multiple of Hkv=%d", Hq, Hkv);
+    TG_SUPPORT(Hq <= 256, "Hq=%d above 256", Hq);
+    return TG_OK;
+}
+
+tg_status do_score(const uint16_t* hidden, const int32_t* cu_seqlens, const int32_t* span, int B, int64_t T, int D,
+                   const uint16_t* Wg, const float* b1, const float* w2, float b2, int I, float eps, float* scores,
+                   cudaStream_t st) {
+    TG_REQUIRE(B >= 0 && T >= 0, "B=%d, T=%lld must be non-negative", B, (long long)T);
+    if (tg_status s = check_gate_shape(D, I)) return s;
+    TG_REQUIRE(eps >= 0.f, "eps must be >= 0");
+    if (B == 0 || T == 0) return TG_OK;
+    TG_REQUIRE(hidden && cu_seqlens && span && Wg && b1 && w2 && scores, "null pointer argument");
+    TG_REQUIRE(aligned16(hidden) && aligned16(Wg), "hidden and Wg must be 16-byte aligned");
+    if (tg_status s = check_device()) return s;
+    return cuda_status(tg::launch_score(hidden, cu_seqlens, span, B, T, D, Wg, b1, w2, b2, I, eps, scores, st),
+                       "tg_score launch");
+}
+
+tg_status do_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* cu_kept, int B,
+                       int64_t M_total, int max_M, int Hq, int Hkv, int d, const int32_t* pos, const int32_t* rank,
+                       const float* gls, const float* g, const float* c, float sm_scale, uint16_t* out, float* lse,
+                       cudaStream_t st) {
+    TG_REQUIRE(B >= 0 && M_total >= 0 && max_M >= 0, "negative size");
+    if (tg_status s = check_attn_shape(Hq, Hkv, d)) return s;
+    TG_REQUIRE(sm_scale > 0.f, "sm_scale must be positive");
+    if (B == 0 || M_total == 0) return TG_OK;
+    TG_REQUIRE(max_M > 0, "max_M must bound the longest sequence");
+    TG_REQUIRE(q && k && v && cu_kept && pos && rank && gls && g && c && out, "null pointer argument");
+    TG_REQUIRE(aligned16(q) && aligned16(k) && aligned16(v) && aligned16(out),
+               "q, k, v and out must be 16-byte aligned");
+    if (tg_status s = check_device()) return s;
+    return cuda_status(tg::launch_gated_attention(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, d, pos, rank, gls, g,
+                                                  c, sm_scale, out, lse, st),
+                       "tg_gated_attention launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+int tg_abi_version(void) { return 1; }
+
+const char* tg_last_error_string(void) { return g_last_error.c_str(); }
+
+int64_t tg_kept_count(const int32_t* h_cu_seqlens, const int32_t* h_span, const int32_t* h_k, int B,
+                      int32_t* h_cu_kept) {
+    if (B < 0 || (B > 0 && (!h_cu_seqlens || !h_span || !h_k)) || !h_cu_kept) {
+        fail(TG_ERR_INVALID_ARG, "tg_kept_count: bad arguments");
+        return -1;
+    }
+    int64_t tot = 0;
+    h_cu_kept[0] = 0;
+    for (int b = 0; b < B; ++b) {
+        const int64_t n = static_cast<int64_t>(h_cu_seqlens[b + 1]) - h_cu_seqlens[b];
+        const int64_t p0 = h_span[2 * b], p1 = h_span[2 * b + 1];
+        if (n < 0 || p0 < 0 || p1 < p0 || p1 > n) {
+            fail(TG_ERR_INVALID_ARG, "tg_kept_count: sequence %d: length %lld, span [%lld, %lld)", b, (long long)n,
+                 (long long)p0, (long long)p1);
+            return -1;
+        }
+        const int64_t P = p1 - p0;
+        const int64_t kk = (h_k[b] < 0 || h_k[b] > P) ? P : h_k[b];
+        tot += (n - P) + kk;
+        if (tot > INT32_MAX) {
+            fail(TG_ERR_INVALID_ARG, "tg_kept_count: total above 2^31-1");
+            return -1;
+        }
+        h_cu_kept[b + 1] = static_cast<int32_t>(tot);
+    }
+    return tot;
+}
+
+tg_status tg_gate_prepare(const uint16_t* gamma, const uint16_t* W1, int D, int I, uint16_t* Wg, tg_stream_t stream) {
+    if (tg_status s = check_gate_shape(D, I)) return s;
+    TG_REQUIRE(gamma && W1 && Wg, "null pointer argument");
+    if (tg_status s = check_device()) return s;
+    return cuda_status(tg::launch_gate_prepare(gamma, W1, D, I, Wg, stream), "tg_gate_prepare launch");
+}
+
+tg_status tg_score(const uint16_t* hidden, const int32_t* cu_seqlens, const int32_t* span, int B, int64_t T, int D,
+                   const uint16_t* Wg, const float* b1, const float* w2, float b2, int I, float eps, float* scores,
+                   tg_stream_t stream) {
+    return do_score(hidden, cu_seqlens, span, B, T, D, Wg, b1, w2, b2, I, eps, scores, stream);
+}
+
+tg_status tg_select_topk(const float* scores, const int32_t* cu_seqlens, const int32_t* span, const int32_t* k, int B,
+                         int64_t T, uint8_t* keep, tg_stream_t stream) {
+    TG_REQUIRE(B >= 0 && T >= 0, "negative size");
+    if (B == 0 || T == 0) return TG_OK;
+    TG_REQUIRE(scores && cu_seqlens && span && k && keep, "null pointer argument");
+    if (tg_status s = check_device()) return s;
+    return cuda_status(tg::launch_select_scan(0, scores, nullptr, cu_seqlens, span, k, nullptr, B, keep, nullptr,
+                                              nullptr, nullptr, nullptr, stream),
+                       "tg_select_topk launch");
+}
+
+tg_status tg_compact(const uint16_t* hidden, const float* scores, const uint8_t* keep, const int32_t* cu_seqlens,
+                     const int32_t* span, int B, int64_t T, int D, const int32_t* cu_kept, int64_t M_total,
+                     uint16_t* hidden_kept, int32_t* pos, int32_t* rank, float* gls, int32_t* kept_idx,
+                     tg_stream_t stream) {
+    TG_REQUIRE(B >= 0 && T >= 0 && M_total >= 0 && M_total <= T, "bad sizes (B=%d T=%lld M=%lld)", B, (long long)T,
+               (long long)M_total);
+    if (B == 0 || T == 0) return TG_OK;
+    TG_REQUIRE(scores && keep && cu_seqlens && span && cu_kept && pos && rank && gls && kept_idx,
+               "null pointer argument");
+    if (hidden_kept) {
+        TG_SUPPORT(D >= 8 && D % 8 == 0, "D=%d must be a multiple of 8 for the row copy", D);
+        TG_REQUIRE(hidden && aligned16(hidden) && aligned16(hidden_kept), "hidden rows must be 16-byte aligned");
+    }
+    if (tg_status s = check_device()) return s;
+    tg_status s = cuda_status(tg::launch_select_scan(1, scores, keep, cu_seqlens, span, nullptr, cu_kept, B, nullptr,
+                                                     kept_idx, pos, rank, gls, stream),
+                              "tg_compact scan launch");
+    if (s != TG_OK || !hidden_kept) return s;
+    return cuda_status(tg::launch_gather_rows(hidden, kept_idx, M_total, T, D, hidden_kept, stream),
+                       "tg_compact gather launch");
+}
+
+tg_status tg_gated_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* cu_kept, int B,
+                             int64_t M_total, int max_M, int Hq, int Hkv, int d, const int32_t* pos,
+                             const int32_t* rank, const float* gls, const float* g, const float* c, float sm_scale,
+                             uint16_t* out, float* lse, tg_stream_t stream) {
+    return do_attention(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, d, pos, rank, gls, g, c, sm_scale, out, lse,
+                        stream);
+}
+
+tg_status tg_gated_prefill_layer(const tg_prefill_layer_args* a, tg_stream_t stream) {
+    TG_REQUIRE(a != nullptr, "null args");
+    TG_REQUIRE(a->B >= 0 && a->T >= 0 && a->M_total >= 0 && a->M_total <= a->T && a->n_layers >= 0, "bad sizes");
+    if (tg_status s = check_gate_shape(a->D, a->I)) return s;
+    if (a->n_layers > 0) {
+        if (tg_status s = check_attn_shape(a->Hq, a->Hkv, a->d)) return s;
+        TG_REQUIRE(a->q && a->kk && a->v && a->g && a->c && a->out, "null per-layer array");
+        for (int l = 0; l < a->n_layers; ++l)
+            TG_REQUIRE(a->q[l] && a->kk[l] && a->v[l] && a->g[l] && a->c[l] && a->out[l],
+                       "null tensor in layer %d", l);
+    }
+    if (a->B == 0 || a->T == 0) return TG_OK;
+    TG_REQUIRE(a->hidden && a->cu_seqlens && a->span && a->k && a->Wg && a->b1 && a->w2 && a->cu_kept && a->scores &&
+                   a->keep && a->pos && a->rank && a->gls && a->kept_idx,
+               "null pointer argument");
+    TG_REQUIRE(aligned16(a->hidden) && aligned16(a->Wg), "hidden and Wg must be 16-byte aligned");
+    if (a->hidden_kept) TG_REQUIRE(aligned16(a->hidden_kept), "hidden_kept must be 16-byte aligned");
+    if (tg_status s = check_device()) return s;
+    cudaStream_t st = stream;
+    if (tg_status s = do_score(a->hidden, a->cu_seqlens, a->span, a->B, a->T, a->D, a->Wg, a->b1, a->w2, a->b2, a->I,
+                               a->eps, a->scores, st))
+        return s;
+    if (tg_status s = cuda_status(tg::launch_select_scan(0, a->scores, nullptr, a->cu_seqlens, a->span, a->k,
+                                                         a->cu_kept, a->B, a->keep, a->kept_idx, a->pos, a->rank,
+                                                         a->gls, st),
+                                  "select launch"))
+        return s;
+    if (a->hidden_kept) {
+        if (tg_status s = cuda_status(tg::launch_gather_rows(a->hidden, a->kept_idx, a->M_total, a->T, a->D,
+                                                             a->hidden_kept, st),
+                                      "gather launch"))
+            return s;
+    }
+    for (int l = 0; l < a->n_layers; ++l) {
+        float* lse = a->lse ? a->lse[l] : nullptr;
+        if (tg_status s = do_attention(a->q[l], a->kk[l], a->v[l], a->cu_kept, a->B, a->M_total, a->max_M, a->Hq,
+                                       a->Hkv, a->d, a->pos, a->rank, a->gls, a->g[l], a->c[l], a->sm_scale,
+                                       a->out[l], lse, st))
+            return s;
+    }
+    return TG_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,54 @@
+// Internal declarations shared by the CUDA translation units of libtokengate.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "tokengate.h"
+
+namespace tg {
+
+// ------------------------------------------------------------------ device helpers
+
+// Order-preserving map of an fp32 score to uint32 (larger score -> larger key).
+// -0 is folded onto +0 so that the two compare equal, as in fp32 comparison;
+// every NaN maps to 0, below the key of -inf (0x007FFFFF).
+__device__ __forceinline__ uint32_t score_key(float s) {
+    if (isnan(s)) return 0u;
+    uint32_t u = __float_as_uint(s);
+    if (u == 0x80000000u) u = 0u;
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
+    return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+// ------------------------------------------------------------------ launchers
+// Each returns cudaSuccess or the launch error; arguments are validated by the
+// C ABI layer before these are called.
+
+cudaError_t launch_gate_prepare(const uint16_t* gamma, const uint16_t* W1, int D, int I, uint16_t* Wg,
+                                cudaStream_t st);
+
+cudaError_t launch_score(const uint16_t* hidden, const int32_t* cu_seqlens, const int32_t* span, int B,
+                         int64_t T, int D, const uint16_t* Wg, const float* b1, const float* w2, float b2, int I,
+                         float eps, float* scores, cudaStream_t st);
+
+// mode 0: select by score (writes keep; the compaction outputs if non-null)
+// mode 1: compaction scan from caller-given keep flags
+cudaError_t launch_select_scan(int mode, const float* scores, const uint8_t* keep_in, const int32_t* cu_seqlens,
+                               const int32_t* span, const int32_t* k, const int32_t* cu_kept, int B,
+                               uint8_t* keep_out, int32_t* kept_idx, int32_t* pos, int32_t* rank, float* gls,
+                               cudaStream_t st);
+
+cudaError_t launch_gather_rows(const uint16_t* hidden, const int32_t* kept_idx, int64_t M_total, int64_t T, int D,
+                               uint16_t* hidden_kept, cudaStream_t st);
+
+cudaError_t launch_gated_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* cu_kept,
+                                   int B, int64_t M_total, int max_M, int Hq, int Hkv, int d, const int32_t* pos,
+                                   const int32_t* rank, const float* gls, const float* g, const float* c,
+                                   float sm_scale, uint16_t* out, float* lse, cudaStream_t st);
+
+}  // namespace tg

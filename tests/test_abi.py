@@ -1,0 +1,115 @@
+"""CPU checks of the C ABI: the library loads, exports every declared symbol,
+its host-only helper is right, and bad arguments are refused before any
+device work.  No call here reaches the GPU."""
+
+import ctypes as C
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tokengate.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from learned_token_pruning_rmsnorm_b200 import build
+    build.build()
+    from learned_token_pruning_rmsnorm_b200 import _lib
+    return _lib.load()
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(tg_[a-z_0-9]+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_five_stage_calls():
+    names = _declared_functions()
+    for n in ("tg_score", "tg_select_topk", "tg_compact", "tg_gated_attention", "tg_gated_prefill_layer"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    from learned_token_pruning_rmsnorm_b200 import _lib
+    names = _declared_functions()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in tokengate.h but not exported"
+        assert n in _lib.SIGNATURES, f"{n} has no binding signature"
+
+
+def test_abi_version(lib):
+    assert lib.tg_abi_version() == 1
+
+
+def test_kept_count_host_helper(lib):
+    from learned_token_pruning_rmsnorm_b200 import tg_kept_count
+    tot, cu_kept = tg_kept_count([0, 10, 10, 25, 40], [[2, 8], [0, 0], [0, 15], [5, 5]], [3, 4, -1, 0])
+    assert tot == 37 and cu_kept.tolist() == [0, 7, 7, 22, 37]
+    # against the workload shape helper for every configured workload
+    from workloads import CONFIGS
+    for w in CONFIGS.values():
+        tot, cu_kept = tg_kept_count(w.cu_seqlens(), w.span_array(), w.budget_array())
+        np.testing.assert_array_equal(cu_kept, w.cu_kept())
+
+
+def test_kept_count_rejects_bad_spans(lib):
+    from learned_token_pruning_rmsnorm_b200 import TokenGateError, tg_kept_count
+    with pytest.raises(TokenGateError):
+        tg_kept_count([0, 10], [[5, 11]], [1])
+    with pytest.raises(TokenGateError):
+        tg_kept_count([0, 10], [[6, 5]], [1])
+
+
+def test_invalid_shapes_are_refused_before_launch(lib):
+    from learned_token_pruning_rmsnorm_b200 import _lib
+    P = C.c_void_p(16)  # never dereferenced: validation fails first
+    # D not a multiple of 64
+    st = lib.tg_score(P, P, P, 1, 128, 100, P, P, P, 0.0, 64, 1e-6, P, None)
+    assert st == _lib.TG_ERR_UNSUPPORTED
+    assert b"D=100" in lib.tg_last_error_string()
+    # I above 256
+    st = lib.tg_score(P, P, P, 1, 128, 256, P, P, P, 0.0, 512, 1e-6, P, None)
+    assert st == _lib.TG_ERR_UNSUPPORTED
+    # head_dim 96
+    st = lib.tg_gated_attention(P, P, P, P, 1, 10, 10, 4, 2, 96, P, P, P, P, P, 0.1, P, None, None)
+    assert st == _lib.TG_ERR_UNSUPPORTED
+    # Hq not a multiple of Hkv
+    st = lib.tg_gated_attention(P, P, P, P, 1, 10, 10, 6, 4, 64, P, P, P, P, P, 0.1, P, None, None)
+    assert st == _lib.TG_ERR_INVALID_ARG
+    # null pointers
+    st = lib.tg_select_topk(None, P, P, P, 1, 10, P, None)
+    assert st == _lib.TG_ERR_INVALID_ARG
+    st = lib.tg_compact(P, P, P, P, P, 1, 10, 64, P, 20, P, P, P, P, P, None)  # M > T
+    assert st == _lib.TG_ERR_INVALID_ARG
+    st = lib.tg_gated_prefill_layer(None, None)
+    assert st == _lib.TG_ERR_INVALID_ARG
+
+
+def test_empty_batches_are_no_ops(lib):
+    from learned_token_pruning_rmsnorm_b200 import _lib
+    assert lib.tg_select_topk(None, None, None, None, 0, 0, None, None) == _lib.TG_OK
+    assert lib.tg_score(None, None, None, 0, 0, 64, None, None, None, 0.0, 16, 1e-6, None, None) == _lib.TG_OK
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    from learned_token_pruning_rmsnorm_b200 import _lib
+    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "LIB_PATH", os.path.join(ROOT, "no_such_dir", "libtokengate.so"))
+    with pytest.raises(ImportError):
+        _lib.load()
+
+
+def test_product_code_never_imports_the_oracle():
+    pkg = os.path.join(ROOT, "learned_token_pruning_rmsnorm_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in src and "from oracle" not in src, f
+                assert "tg_oracle" not in src and "liboracle" not in src, f
