@@ -276,10 +276,45 @@ def run_gpu(args, w):
         if ws > 1:
             dist.barrier()
 
-    # warm-up
+    lib = tg.load()
+    sh = st.cuda_stream
+    B, T, D, I = w.B, w.T, w.D, w.I
+    sm_scale = 1.0 / math.sqrt(w.d)
+    L0 = layers[0]
+    # the product's kernels, one C-ABI call each, arguments bound once (host cost ~1 us per call)
+    stage_calls = {
+        "score": lambda: lib.tg_score(hidden.data_ptr(), call.cu.data_ptr(), call.sp.data_ptr(), B, T, D,
+                                      Wg.data_ptr(), b1.data_ptr(), w2.data_ptr(), float(gi["b2"]), I, float(w.eps),
+                                      bufs.scores.data_ptr(), sh),
+        "select": lambda: lib.tg_select_topk(bufs.scores.data_ptr(), call.cu.data_ptr(), call.sp.data_ptr(),
+                                             call.kk.data_ptr(), B, T, bufs.keep.data_ptr(), call.ck.data_ptr(),
+                                             bufs.kept_idx.data_ptr(), bufs.pos.data_ptr(), bufs.rank.data_ptr(),
+                                             bufs.gls.data_ptr(), sh),
+        "gather": lambda: lib.tg_compact(hidden.data_ptr(), None, None, None, None, B, T, D, None, M,
+                                         bufs.hidden_kept.data_ptr(), None, None, None, bufs.kept_idx.data_ptr(), sh),
+        "attention": lambda: lib.tg_gated_attention(L0["q"].data_ptr(), L0["k"].data_ptr(), L0["v"].data_ptr(),
+                                                    call.ck.data_ptr(), B, M, call.max_M, w.Hq, w.Hkv, w.d,
+                                                    bufs.pos.data_ptr(), bufs.rank.data_ptr(), bufs.gls.data_ptr(),
+                                                    L0["g"].data_ptr(), L0["c"].data_ptr(), sm_scale,
+                                                    bufs.out[0].data_ptr(), None, sh),
+    }
+
+    # warm-up (also sets kernel attributes before any capture)
     for _ in range(args.warmup):
         call()
+        for fn in stage_calls.values():
+            assert fn() == 0
     torch.cuda.synchronize(dev)
+
+    # the step as one CUDA graph: four kernels, no host work between them
+    graph = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            call()
+        graph.replay()
+        torch.cuda.synchronize(dev)
+    step = graph.replay if graph is not None else call
 
     # ---------------- timed region: K whole-path steps
     clocks = ClockSampler(local)
@@ -290,31 +325,24 @@ def run_gpu(args, w):
     for i in range(args.steps):
         flush.fill_(i)
         ev[i][0].record(st)
-        call()
+        step()
         ev[i][1].record(st)
     torch.cuda.synchronize(dev)
     barrier()
     step_ms = [a.elapsed_time(b) for a, b in ev]
 
-    # ---------------- per-stage breakdown over K more steps (same stream)
-    sev = {s: [] for s in ("score", "select", "gather", "attention")}
+    # ---------------- per-stage breakdown over K more steps (same stream, same kernels)
+    names = list(stage_calls)
+    sev = {s: [] for s in names}
     for i in range(args.steps):
         flush.fill_(i)
-        e = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
         e[0].record(st)
-        tg.tg_score(hidden, call.cu, call.sp, Wg, b1, w2, gi["b2"], w.eps, scores=bufs.scores)
-        e[1].record(st)
-        tg.tg_select_topk(bufs.scores, call.cu, call.sp, call.kk, keep=bufs.keep)
-        e[2].record(st)
-        tg.tg_compact(hidden, bufs.scores, bufs.keep, call.cu, call.sp, call.ck, M)
-        e[3].record(st)
-        tg.tg_gated_attention(layers[0]["q"], layers[0]["k"], layers[0]["v"], call.ck, call.max_M, bufs.pos,
-                              bufs.rank, bufs.gls, layers[0]["g"], layers[0]["c"], out=bufs.out[0])
-        e[4].record(st)
-        sev["score"].append((e[0], e[1]))
-        sev["select"].append((e[1], e[2]))
-        sev["gather"].append((e[2], e[3]))
-        sev["attention"].append((e[3], e[4]))
+        for n_i, nm in enumerate(names):
+            stage_calls[nm]()
+            e[n_i + 1].record(st)
+        for n_i, nm in enumerate(names):
+            sev[nm].append((e[n_i], e[n_i + 1]))
     torch.cuda.synchronize(dev)
     clk = clocks.stop()
     stage_us = {s: 1e3 * float(np.mean([a.elapsed_time(b) for a, b in v])) for s, v in sev.items()}
@@ -333,7 +361,7 @@ def run_gpu(args, w):
         for L, Lh in zip(layers, layers_h):
             for key in L:
                 L[key].copy_(Lh[key], non_blocking=True)
-        call()
+        step()
         out_h.copy_(bufs.out[-1], non_blocking=True)
         idx_h.copy_(bufs.kept_idx, non_blocking=True)
         b.record(st)
@@ -399,7 +427,7 @@ def run_gpu(args, w):
                 "stage_us": stage_us, "stage_gbs": stage_gbs,
                 "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                         "d2h_bytes_per_step": int(d2h)},
-                "gpu_launches": args.steps * (3 + args.layers),
+                "gpu_launches": args.steps * (3 + args.layers), "cuda_graph": graph is not None,
                 "cpu_baseline": cpu_base, "clocks": clk, "peaks": {"source": peaks["source"],
                                                                    "hbm_gbs": hbm_peak, "bf16_tflops": tc_peak}}
         print(json.dumps(line), flush=True)
@@ -418,6 +446,7 @@ def main(argv=None):
     ap.add_argument("--workload", default="c2_32k_k2000")
     ap.add_argument("--layers", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch the step directly instead of a CUDA graph")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

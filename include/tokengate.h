@@ -117,9 +117,15 @@ tg_status tg_score(const uint16_t* hidden, const int32_t* cu_seqlens, const int3
  * +0; NaN ranks below every number.  keep [T] uint8 (out): 1 for every
  * non-prunable token and for the selected prunable ones, else 0.
  * Bit-exact and run-to-run deterministic.
+ * Optional fused compaction map: when cu_kept and kept_idx are both
+ * non-NULL, the same pass also writes kept_idx, pos, rank and gls exactly as
+ * tg_compact defines them (pos, rank, gls must then be non-NULL too), so
+ * that tg_compact(keep = NULL) only has to gather the rows.  Pass NULL for
+ * all five to get the flags alone.
  */
 tg_status tg_select_topk(const float* scores, const int32_t* cu_seqlens, const int32_t* span, const int32_t* k,
-                         int B, int64_t T, uint8_t* keep, tg_stream_t stream);
+                         int B, int64_t T, uint8_t* keep, const int32_t* cu_kept, int32_t* kept_idx, int32_t* pos,
+                         int32_t* rank, float* gls, tg_stream_t stream);
 
 /*
  * Stage 3: stable compaction of the kept tokens (AI summary, "Key
@@ -134,6 +140,11 @@ tg_status tg_select_topk(const float* scores, const int32_t* cu_seqlens, const i
  * cu_kept [B+1] (device) must hold tg_kept_count's prefix sums; M_total is
  * cu_kept[B].  hidden_kept may be NULL (then only the index outputs are
  * written); pos, rank, gls, kept_idx are required.
+ * keep == NULL means the compaction map was already written by
+ * tg_select_topk: kept_idx is then an input and only the row gather runs
+ * (scores, pos, rank, gls are not touched and may be NULL).
+ * Keep flags that disagree with cu_kept never make the kernels write or
+ * read outside [0, M_total) and [0, T); the affected rows are unspecified.
  */
 tg_status tg_compact(const uint16_t* hidden, const float* scores, const uint8_t* keep, const int32_t* cu_seqlens,
                      const int32_t* span, int B, int64_t T, int D, const int32_t* cu_kept, int64_t M_total,

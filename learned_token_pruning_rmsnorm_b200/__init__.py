@@ -23,7 +23,7 @@ from ._lib import TokenGateError, load  # noqa: F401
 
 __all__ = [
     "TokenGateError", "load", "tg_abi_version", "tg_kept_count", "tg_gate_prepare", "tg_score",
-    "tg_select_topk", "tg_compact", "tg_gated_attention", "tg_gated_prefill_layer",
+    "tg_select_topk", "tg_compact", "tg_gather_kept", "tg_gated_attention", "tg_gated_prefill_layer",
 ]
 
 
@@ -93,7 +93,9 @@ def tg_score(hidden, cu_seqlens, span, Wg, b1, w2, b2: float, eps: float = 1e-6,
     return scores
 
 
-def tg_select_topk(scores, cu_seqlens, span, k, keep=None):
+def tg_select_topk(scores, cu_seqlens, span, k, keep=None, cu_kept=None, M_total=None):
+    """Keep flags [T] uint8.  With cu_kept and M_total also returns the fused
+    compaction map (kept_idx, pos, rank, gls) written by the same pass."""
     T = scores.shape[0]
     dev = scores.device
     _dev(scores, torch.float32, "scores")
@@ -103,9 +105,42 @@ def tg_select_topk(scores, cu_seqlens, span, k, keep=None):
     if keep is None:
         keep = torch.empty(T, dtype=torch.uint8, device=dev)
     _dev(keep, torch.uint8, "keep", (T,))
+    emit = cu_kept is not None
+    cmap = None
+    if emit:
+        M = int(M_total)
+        ck = _i32_dev(cu_kept, dev, "cu_kept")
+        cmap = {"kept_idx": torch.empty(M, dtype=torch.int32, device=dev),
+                "pos": torch.empty(M, dtype=torch.int32, device=dev),
+                "rank": torch.empty(M, dtype=torch.int32, device=dev),
+                "gls": torch.empty(M, dtype=torch.float32, device=dev)}
+        if M == 0:
+            emit = False
     _lib.check(load().tg_select_topk(scores.data_ptr(), cu.data_ptr(), sp.data_ptr(), kk.data_ptr(),
-                                     cu.numel() - 1, T, keep.data_ptr(), _lib.stream_handle(dev)))
-    return keep
+                                     cu.numel() - 1, T, keep.data_ptr(),
+                                     ck.data_ptr() if emit else None,
+                                     cmap["kept_idx"].data_ptr() if emit else None,
+                                     cmap["pos"].data_ptr() if emit else None,
+                                     cmap["rank"].data_ptr() if emit else None,
+                                     cmap["gls"].data_ptr() if emit else None, _lib.stream_handle(dev)))
+    return keep if cmap is None else (keep, cmap)
+
+
+def tg_gather_kept(hidden, kept_idx, hidden_kept=None):
+    """Row gather of a compaction map written by tg_select_topk (tg_compact
+    with keep = NULL)."""
+    T, D = hidden.shape
+    M = kept_idx.shape[0]
+    dev = hidden.device
+    _dev(hidden, torch.bfloat16, "hidden")
+    _dev(kept_idx, torch.int32, "kept_idx")
+    if hidden_kept is None:
+        hidden_kept = torch.empty((M, D), dtype=torch.bfloat16, device=dev)
+    _dev(hidden_kept, torch.bfloat16, "hidden_kept", (M, D))
+    _lib.check(load().tg_compact(hidden.data_ptr(), None, None, None, None, 1, T, D, None, M,
+                                 hidden_kept.data_ptr(), None, None, None, kept_idx.data_ptr(),
+                                 _lib.stream_handle(dev)))
+    return hidden_kept
 
 
 def tg_compact(hidden, scores, keep, cu_seqlens, span, cu_kept, M_total: int, with_hidden: bool = True):

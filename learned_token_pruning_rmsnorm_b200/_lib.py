@@ -51,7 +51,7 @@ SIGNATURES = {
     "tg_kept_count": ([P, P, P, i32, P], i64),
     "tg_gate_prepare": ([P, P, i32, i32, P, P], i32),
     "tg_score": ([P, P, P, i32, i64, i32, P, P, P, f32, i32, f32, P, P], i32),
-    "tg_select_topk": ([P, P, P, P, i32, i64, P, P], i32),
+    "tg_select_topk": ([P, P, P, P, i32, i64, P, P, P, P, P, P, P], i32),
     "tg_compact": ([P, P, P, P, P, i32, i64, i32, P, i64, P, P, P, P, P, P], i32),
     "tg_gated_attention": ([P, P, P, P, i32, i64, i32, i32, i32, i32, P, P, P, P, P, f32, P, P, P], i32),
     "tg_gated_prefill_layer": ([C.POINTER(PrefillLayerArgs), P], i32),

@@ -1,70 +1,385 @@
 // Stage 4 of the gated prefill: token-gated causal GQA attention over the kept
-// tokens (TokenGate AI summary, "Key Contributions" 2 and 3).
+// tokens (TokenGate AI summary, "Key Contributions" 2 and 3), on the sm_100
+// tensor cores.
 //
 //   logit[q,j] = (q.k_j * sm_scale + softplus(g_h) * gls_j) / tau[q,h]
 //   tau[q,h]   = 1 + c_h * ln(pos_q / rank_q)
 //   o_q        = sum_j softmax_j(logit[q,:]) v_j     over kept j <= q
 //
-// Simple warp-per-(query, head) kernel with an online softmax in fp32.
+// One CTA per (query head, 128-query tile, sequence); heaviest causal tiles
+// are launched first.  Warp roles (192 threads):
+//   warp 4     TMA producer: the Q tile once, then K/V tiles of 128 keys
+//              through a two-stage ring (128-byte swizzled boxes of 64 cols)
+//   warp 5     MMA issuer (one thread): S_j = Q K_j^T into one of two TMEM
+//              S buffers, then O += P_{j-1} V_{j-1} into the TMEM O accumulator
+//   warps 0-3  softmax: thread r owns query row r (TMEM lane r).  It reads
+//              S_j from TMEM, applies scale, gate bias and temperature in the
+//              log2 domain with one FFMA per element, masks the causal
+//              diagonal, keeps a running max that is only moved (and O only
+//              rescaled in TMEM) when it grows by more than 2^8, writes P_j
+//              as bf16 into a swizzled shared-memory tile for the next MMA,
+//              and at the end normalises O and stores it.
+// The bias and temperature therefore cost one extra FFMA per score element
+// on top of plain attention.
 
-#include "tg_internal.cuh"
+#include "tg_sm100.cuh"
 
 namespace tg {
 namespace {
 
-__device__ __forceinline__ float softplus_f(float x) { return fmaxf(x, 0.f) + log1pf(expf(-fabsf(x))); }
+using namespace sm100;
+
+constexpr int BM = 128;           // query rows per tile (TMEM lanes)
+constexpr int BN = 128;           // keys per tile
+constexpr int NUM_THREADS = 192;
+constexpr float LOG2E = 1.4426950408889634f;
+constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: rescale only when the max grows by > 2^8
 
 template <int HD>
-__global__ void __launch_bounds__(128)
-attn_simple_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
-                   const int32_t* __restrict__ cu_kept, int B, int64_t M, int Hq, int Hkv,
-                   const int32_t* __restrict__ pos, const int32_t* __restrict__ rank, const float* __restrict__ gls,
-                   const float* __restrict__ g, const float* __restrict__ c, float sm_scale,
-                   uint16_t* __restrict__ out, float* __restrict__ lse) {
-    constexpr int E = HD / 32;
-    const int lane = threadIdx.x & 31;
-    const int64_t wid = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    if (wid >= M * Hq) return;
-    const int64_t i = wid / Hq;
-    const int h = static_cast<int>(wid - i * Hq);
-    int b = 0;
-    while (b + 1 < B && cu_kept[b + 1] <= i) ++b;
-    const int64_t j0 = cu_kept[b];
-    const int hk = h / (Hq / Hkv);
+struct AttnSmem {
+    static constexpr int TILE_Q = BM * HD * 2;
+    static constexpr int TILE_KV = BN * HD * 2;
+    static constexpr int TILE_P = BM * BN * 2;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = OFF_Q + TILE_Q;
+    static constexpr int OFF_V = OFF_K + 2 * TILE_KV;
+    static constexpr int OFF_P = OFF_V + 2 * TILE_KV;
+    static constexpr int OFF_BIAS = OFF_P + TILE_P;
+    static constexpr int OFF_BAR = OFF_BIAS + 4 * 2 * BN * 4;  // a private bias copy per softmax warp
+    static constexpr int NUM_BARS = 16;
+    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+    static constexpr int BYTES = OFF_MISC + 16;
+    static constexpr int ALLOC = BYTES + 1024;  // slack for 1024-byte alignment
+    static constexpr uint32_t TMEM_COLS = 512;  // S0 | S1 | O
+};
 
-    float qv[E];
-#pragma unroll
-    for (int e = 0; e < E; ++e) qv[e] = bf16_bits_to_float(q[(i * Hq + h) * HD + lane * E + e]);
-    const float gain = softplus_f(g[h]);
-    const float tau = 1.0f + c[h] * logf(static_cast<float>(pos[i]) / static_cast<float>(rank[i]));
-    const float inv_tau = 1.0f / tau;
-    float m = -INFINITY, l = 0.f, acc[E];
-#pragma unroll
-    for (int e = 0; e < E; ++e) acc[e] = 0.f;
-    for (int64_t j = j0; j <= i; ++j) {
-        const uint16_t* kr = k + (j * Hkv + hk) * HD + lane * E;
-        float dot = 0.f;
-#pragma unroll
-        for (int e = 0; e < E; ++e) dot = fmaf(qv[e], bf16_bits_to_float(kr[e]), dot);
-#pragma unroll
-        for (int off = 16; off; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
-        const float logit = (dot * sm_scale + gain * gls[j]) * inv_tau;
-        const float m_new = fmaxf(m, logit);
-        const float corr = expf(m - m_new);
-        const float p = expf(logit - m_new);
-        l = l * corr + p;
-        const uint16_t* vr = v + (j * Hkv + hk) * HD + lane * E;
-#pragma unroll
-        for (int e = 0; e < E; ++e) acc[e] = fmaf(p, bf16_bits_to_float(vr[e]), acc[e] * corr);
-        m = m_new;
+// barrier indices
+enum : int {
+    B_Q_FULL = 0, B_K_FULL = 1, B_K_EMPTY = 3, B_V_FULL = 5, B_V_EMPTY = 7, B_S_FULL = 9, B_S_FREE = 11,
+    B_P_FULL = 13, B_PV_DONE = 14, B_DRAIN = 15
+};
+
+__device__ __forceinline__ float softplus_f(float x) { return fmaxf(x, 0.f) + log1pf(expf(-fabsf(x))); }
+
+__device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity, int* status) {
+    volatile int never = 0;
+    return mbar_wait(bar, parity, &never, status, TG_WHERE_DRAIN);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+template <int HD>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+gated_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, const int32_t* __restrict__ cu_kept,
+                     const int32_t* __restrict__ pos, const int32_t* __restrict__ rank,
+                     const float* __restrict__ gls, const float* __restrict__ g, const float* __restrict__ c,
+                     float sm_scale, int Hq, int Hkv, int n_qt_max, uint16_t* __restrict__ out,
+                     float* __restrict__ lse, int* __restrict__ status) {
+    using L = AttnSmem<HD>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+    const int h = blockIdx.x;
+    const int qt = n_qt_max - 1 - static_cast<int>(blockIdx.y);
+    const int b = blockIdx.z;
+    const int seq0 = cu_kept[b];
+    const int Mb = cu_kept[b + 1] - seq0;
+    if (qt * BM >= Mb) return;
+    const int n_kv = qt + 1;  // BM == BN: the diagonal tile is the last one
+    const int hk = h / (Hq / Hkv);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t sQ = sbase + L::OFF_Q, sK0 = sbase + L::OFF_K, sV0 = sbase + L::OFF_V, sP = sbase + L::OFF_P;
+    auto bar = [&](int i) { return sbase + L::OFF_BAR + 8u * static_cast<uint32_t>(i); };
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+    float* sBias = reinterpret_cast<float*>(smem + L::OFF_BIAS);
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(B_Q_FULL), 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar(B_K_FULL + s), 1);
+            mbar_init(bar(B_K_EMPTY + s), 1);
+            mbar_init(bar(B_V_FULL + s), 1);
+            mbar_init(bar(B_V_EMPTY + s), 1);
+            mbar_init(bar(B_S_FULL + s), 1);
+            mbar_init(bar(B_S_FREE + s), 128);
+        }
+        mbar_init(bar(B_P_FULL), 128);
+        mbar_init(bar(B_PV_DONE), 1);
+        mbar_init(bar(B_DRAIN), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
     }
-    const float inv_l = 1.0f / l;
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-        const __nv_bfloat16 r = __float2bfloat16_rn(acc[e] * inv_l);
-        out[(i * Hq + h) * HD + lane * E + e] = *reinterpret_cast<const uint16_t*>(&r);
+    if (warp == 4) {
+        tmem_alloc(smem_u32(tmem_slot), L::TMEM_COLS);
+        tmem_relinquish();
     }
-    if (lse && lane == 0) lse[i * Hq + h] = m + logf(l);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tmem_O = tmem + 2 * BN;
+
+    if (warp == 4) {
+        // ---------------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            prefetch_tmap(&tmQ);
+            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmV);
+            mbar_expect_tx(bar(B_Q_FULL), BM * HD * 2);
+#pragma unroll
+            for (int hf = 0; hf < HD / 64; ++hf)
+                tma_load_2d(sQ + hf * BM * 128, &tmQ, h * HD + hf * 64, seq0 + qt * BM, bar(B_Q_FULL));
+            int k_issued[2] = {0, 0}, v_issued[2] = {0, 0};
+            for (int j = 0; j < n_kv; ++j) {
+                const int s = j & 1;
+                if (j >= 2 && !mbar_wait(bar(B_K_EMPTY + s), ((j - 2) >> 1) & 1, abort_flag, status,
+                                         TG_WHERE_PRODUCER))
+                    break;
+                mbar_expect_tx(bar(B_K_FULL + s), BN * HD * 2);
+#pragma unroll
+                for (int hf = 0; hf < HD / 64; ++hf)
+                    tma_load_2d(sK0 + s * L::TILE_KV + hf * BN * 128, &tmK, hk * HD + hf * 64, seq0 + j * BN,
+                                bar(B_K_FULL + s));
+                ++k_issued[s];
+                if (j >= 2 && !mbar_wait(bar(B_V_EMPTY + s), ((j - 2) >> 1) & 1, abort_flag, status,
+                                         TG_WHERE_PRODUCER))
+                    break;
+                mbar_expect_tx(bar(B_V_FULL + s), BN * HD * 2);
+#pragma unroll
+                for (int hf = 0; hf < HD / 64; ++hf)
+                    tma_load_2d(sV0 + s * L::TILE_KV + hf * BN * 128, &tmV, hk * HD + hf * 64, seq0 + j * BN,
+                                bar(B_V_FULL + s));
+                ++v_issued[s];
+            }
+            if (*abort_flag) {
+                // let every copy this thread started land before the CTA exits
+                drain_wait(bar(B_Q_FULL), 0, status);
+                for (int s = 0; s < 2; ++s) {
+                    if (k_issued[s]) drain_wait(bar(B_K_FULL + s), (k_issued[s] - 1) & 1, status);
+                    if (v_issued[s]) drain_wait(bar(B_V_FULL + s), (v_issued[s] - 1) & 1, status);
+                }
+            }
+        }
+    } else if (warp == 5) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false);
+            constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, HD, true);
+            bool ok = mbar_wait(bar(B_Q_FULL), 0, abort_flag, status, TG_WHERE_MMA);
+            for (int j = 0; ok && j <= n_kv; ++j) {
+                if (j < n_kv) {
+                    const int s = j & 1;
+                    ok = mbar_wait(bar(B_K_FULL + s), (j >> 1) & 1, abort_flag, status, TG_WHERE_MMA);
+                    if (ok && j >= 2)
+                        ok = mbar_wait(bar(B_S_FREE + s), ((j - 2) >> 1) & 1, abort_flag, status, TG_WHERE_MMA);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t d = tmem + s * BN;
+                    const uint32_t kb = sK0 + s * L::TILE_KV;
+#pragma unroll
+                    for (int kk = 0; kk < HD / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+                        const uint32_t offk = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
+                        mma_bf16_ss(d, smem_desc_sw128(sQ + off, 16, 1024), smem_desc_sw128(kb + offk, 16, 1024),
+                                    idesc_qk, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(bar(B_S_FULL + s));
+                    mma_commit(bar(B_K_EMPTY + s));
+                }
+                if (j >= 1) {
+                    const int jj = j - 1, s = jj & 1;
+                    ok = mbar_wait(bar(B_P_FULL), jj & 1, abort_flag, status, TG_WHERE_MMA);
+                    if (ok) ok = mbar_wait(bar(B_V_FULL + s), (jj >> 1) & 1, abort_flag, status, TG_WHERE_MMA);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t vb = sV0 + s * L::TILE_KV;
+#pragma unroll
+                    for (int kk = 0; kk < BN / 16; ++kk) {
+                        const uint32_t offp = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+                        mma_bf16_ss(tmem_O, smem_desc_sw128(sP + offp, 16, 1024),
+                                    smem_desc_sw128(vb + kk * 16 * 128, BN * 128, 1024), idesc_pv,
+                                    (jj > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    mma_commit(bar(B_PV_DONE));
+                    mma_commit(bar(B_V_EMPTY + s));
+                }
+            }
+            // every MMA (and the barrier arrivals its commits trigger) lands before the CTA exits
+            mma_commit(bar(B_DRAIN));
+            drain_wait(bar(B_DRAIN), 0, status);
+        }
+    } else {
+        // ---------------------------------------------------------------- softmax warps 0-3
+        const int r = threadIdx.x;  // query row within the tile == TMEM lane
+        const int q_local = qt * BM + r;
+        const bool valid_row = q_local < Mb;
+        const int qg = seq0 + q_local;
+        float inv_tau = 1.0f;
+        if (valid_row) inv_tau = 1.0f / (1.0f + c[h] * logf(static_cast<float>(pos[qg]) / static_cast<float>(rank[qg])));
+        const float alpha = sm_scale * LOG2E * inv_tau;
+        const float gscale = softplus_f(g[h]) * LOG2E;
+        const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+        float m_run = -INFINITY, l_run = 0.f;
+        bool ok = true;
+        float* wbias = sBias + warp * (2 * BN);  // this warp's copy, double-buffered
+        for (int j = 0; j < n_kv; ++j) {
+            const int s = j & 1;
+            // gate bias of the tile's 128 keys, log2 domain; each warp keeps its own
+            // copy so that only __syncwarp orders it
+#pragma unroll
+            for (int e = 0; e < BN / 32; ++e) {
+                const int key_local = j * BN + e * 32 + lane;
+                wbias[s * BN + e * 32 + lane] = key_local < Mb ? gscale * gls[seq0 + key_local] : 0.f;
+            }
+            __syncwarp();
+            ok = mbar_wait(bar(B_S_FULL + s), (j >> 1) & 1, abort_flag, status, TG_WHERE_SOFTMAX);
+            if (!ok) break;
+            tc_fence_after();
+            float x[BN];
+#pragma unroll
+            for (int ch = 0; ch < BN / 32; ++ch) tmem_ld32(tmem + lane_addr + s * BN + ch * 32, x + ch * 32);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(bar(B_S_FREE + s));
+
+            const float* bias = wbias + s * BN;
+            float mx = -INFINITY;
+            if (j == n_kv - 1) {
+                const int lim = q_local - j * BN;  // keys with column > lim lie in the causal future
+#pragma unroll
+                for (int cc = 0; cc < BN; ++cc) {
+                    const float v = fmaf(x[cc], alpha, bias[cc] * inv_tau);
+                    x[cc] = cc > lim ? -INFINITY : v;
+                    mx = fmaxf(mx, x[cc]);
+                }
+            } else {
+#pragma unroll
+                for (int cc = 0; cc < BN; ++cc) {
+                    x[cc] = fmaf(x[cc], alpha, bias[cc] * inv_tau);
+                    mx = fmaxf(mx, x[cc]);
+                }
+            }
+            float corr = 1.0f;
+            bool rescale_o = false;
+            if (j == 0 || mx > m_run + RESCALE_THRESHOLD) {
+                const float m_new = fmaxf(m_run, mx);
+                corr = exp2f(m_run - m_new);
+                m_run = m_new;
+                rescale_o = j > 0;
+            }
+            float sum = 0.f;
+#pragma unroll
+            for (int cc = 0; cc < BN; ++cc) {
+                x[cc] = exp2f(x[cc] - m_run);
+                sum += x[cc];
+            }
+            l_run = l_run * corr + sum;
+            // the P tile and O may be touched only once PV_{j-1} has completed
+            if (j >= 1) {
+                ok = mbar_wait(bar(B_PV_DONE), (j - 1) & 1, abort_flag, status, TG_WHERE_SOFTMAX);
+                if (!ok) break;
+                tc_fence_after();
+            }
+            if (rescale_o) {
+#pragma unroll
+                for (int ch = 0; ch < HD / 32; ++ch) {
+                    float o[32];
+                    tmem_ld32(tmem_O + lane_addr + ch * 32, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] *= corr;
+                    tmem_st32(tmem_O + lane_addr + ch * 32, o);
+                }
+                tmem_wait_st();
+            }
+            // P row r as bf16 into the 128-byte-swizzled K-major tile (two 64-key halves)
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                uint8_t* rowp = smem + L::OFF_P + hf * (BM * 128) + r * 128;
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    const float* p = x + hf * 64 + ch * 8;
+                    uint4 v;
+                    v.x = pack_bf16x2(p[0], p[1]);
+                    v.y = pack_bf16x2(p[2], p[3]);
+                    v.z = pack_bf16x2(p[4], p[5]);
+                    v.w = pack_bf16x2(p[6], p[7]);
+                    *reinterpret_cast<uint4*>(rowp + ((ch ^ (r & 7)) << 4)) = v;
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(bar(B_P_FULL));
+        }
+        // ---------------------------------------------------------------- epilogue
+        if (ok) ok = mbar_wait(bar(B_PV_DONE), (n_kv - 1) & 1, abort_flag, status, TG_WHERE_SOFTMAX);
+        if (ok) {
+            tc_fence_after();
+            const float inv_l = 1.0f / l_run;
+            uint16_t* orow = out + (static_cast<size_t>(qg) * Hq + h) * HD;
+#pragma unroll
+            for (int ch = 0; ch < HD / 32; ++ch) {
+                float o[32];
+                tmem_ld32(tmem_O + lane_addr + ch * 32, o);
+                tmem_wait_ld();
+                if (valid_row) {
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        uint4 v;
+                        v.x = pack_bf16x2(o[q4 * 8 + 0] * inv_l, o[q4 * 8 + 1] * inv_l);
+                        v.y = pack_bf16x2(o[q4 * 8 + 2] * inv_l, o[q4 * 8 + 3] * inv_l);
+                        v.z = pack_bf16x2(o[q4 * 8 + 4] * inv_l, o[q4 * 8 + 5] * inv_l);
+                        v.w = pack_bf16x2(o[q4 * 8 + 6] * inv_l, o[q4 * 8 + 7] * inv_l);
+                        *reinterpret_cast<uint4*>(orow + ch * 32 + q4 * 8) = v;
+                    }
+                }
+            }
+            if (valid_row && lse) lse[static_cast<size_t>(qg) * Hq + h] = (m_run + log2f(l_run)) / LOG2E;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 4) {
+        tc_fence_after();
+        tmem_dealloc(tmem, L::TMEM_COLS);
+    }
+}
+
+template <int HD>
+cudaError_t launch_tc(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* cu_kept, int B,
+                      int64_t M_total, int max_M, int Hq, int Hkv, const int32_t* pos, const int32_t* rank,
+                      const float* gls, const float* g, const float* c, float sm_scale, uint16_t* out, float* lse,
+                      cudaStream_t st) {
+    using L = AttnSmem<HD>;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(gated_attn_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             L::ALLOC);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    CUtensorMap tq, tk, tv;
+    if (!encode_tmap_2d_bf16(&tq, q, static_cast<uint64_t>(Hq) * HD, static_cast<uint64_t>(M_total),
+                             static_cast<uint64_t>(Hq) * HD * 2, 64, BM) ||
+        !encode_tmap_2d_bf16(&tk, k, static_cast<uint64_t>(Hkv) * HD, static_cast<uint64_t>(M_total),
+                             static_cast<uint64_t>(Hkv) * HD * 2, 64, BN) ||
+        !encode_tmap_2d_bf16(&tv, v, static_cast<uint64_t>(Hkv) * HD, static_cast<uint64_t>(M_total),
+                             static_cast<uint64_t>(Hkv) * HD * 2, 64, BN))
+        return cudaErrorInvalidValue;
+    int* status = device_status_ptr();
+    const int n_qt_max = (max_M + BM - 1) / BM;
+    dim3 grid(Hq, n_qt_max, B);
+    gated_attn_tc_kernel<HD><<<grid, NUM_THREADS, L::ALLOC, st>>>(tq, tk, tv, cu_kept, pos, rank, gls, g, c, sm_scale,
+                                                                  Hq, Hkv, n_qt_max, out, lse, status);
+    return cudaGetLastError();
 }
 
 }  // namespace
@@ -73,17 +388,12 @@ cudaError_t launch_gated_attention(const uint16_t* q, const uint16_t* k, const u
                                    int B, int64_t M_total, int max_M, int Hq, int Hkv, int d, const int32_t* pos,
                                    const int32_t* rank, const float* gls, const float* g, const float* c,
                                    float sm_scale, uint16_t* out, float* lse, cudaStream_t st) {
-    (void)max_M;
-    const int64_t warps = M_total * Hq;
-    if (warps == 0) return cudaSuccess;
-    const unsigned grid = static_cast<unsigned>((warps + 3) / 4);
+    if (M_total == 0 || B == 0) return cudaSuccess;
     if (d == 64)
-        attn_simple_kernel<64><<<grid, 128, 0, st>>>(q, k, v, cu_kept, B, M_total, Hq, Hkv, pos, rank, gls, g, c,
-                                                     sm_scale, out, lse);
-    else
-        attn_simple_kernel<128><<<grid, 128, 0, st>>>(q, k, v, cu_kept, B, M_total, Hq, Hkv, pos, rank, gls, g, c,
-                                                      sm_scale, out, lse);
-    return cudaGetLastError();
+        return launch_tc<64>(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, pos, rank, gls, g, c, sm_scale, out, lse,
+                             st);
+    return launch_tc<128>(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, pos, rank, gls, g, c, sm_scale, out, lse,
+                          st);
 }
 
 }  // namespace tg

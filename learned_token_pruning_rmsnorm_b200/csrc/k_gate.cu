@@ -5,11 +5,26 @@
 //   r_t = 1 / sqrt(mean_i x_ti^2 + eps)
 //   s_t = b2 + sum_j w2[j] * SiLU(r_t * (Wg[j,:] . x_t) + b1[j])
 // with Wg = bf16(gamma (.) W1^T) prepared once by tg_gate_prepare.
+//
+// Scoring is one pass over the prunable rows of `hidden` on the tensor cores:
+//   - persistent CTAs, each owning tiles of NACC x 128 rows; the NACC
+//     accumulators (128 x I fp32 each, in TMEM) share every Wg tile, so the
+//     gate weight is streamed from L2 once per 128*NACC rows;
+//   - warp 0 streams 64-channel slices of the rows and of Wg with TMA
+//     (128-byte swizzle) through a STAGES-deep ring; warp 1 issues
+//     tcgen05.mma (M=128, N=I, K=16) per accumulator;
+//   - 4*NACC warps read each row's slice from the same shared-memory tiles to
+//     accumulate sum(x^2) while the MMAs run, then apply rsqrt, b1, SiLU and
+//     the w2 dot product to the accumulator rows read from TMEM.
+// HBM traffic is the hidden rows of the span (read once) plus one fp32 score
+// per row; the normalised activations are never rounded before the product.
 
-#include "tg_internal.cuh"
+#include "tg_sm100.cuh"
 
 namespace tg {
 namespace {
+
+using namespace sm100;
 
 __global__ void gate_prepare_kernel(const uint16_t* __restrict__ gamma, const uint16_t* __restrict__ W1, int D, int I,
                                     uint16_t* __restrict__ Wg) {
@@ -23,93 +38,258 @@ __global__ void gate_prepare_kernel(const uint16_t* __restrict__ gamma, const ui
     }
 }
 
-// Simple CUDA-core scoring kernel: ROWS tokens per CTA, one thread per gate
-// unit j (blockDim.x == I), the contraction staged through shared memory in
-// chunks of 64 channels.
-constexpr int SC_ROWS = 16;
-constexpr int SC_KC = 32;
+constexpr int KB = 64;                // channels per pipeline stage (one 128-byte swizzle row)
+constexpr int TILE_A = 128 * KB * 2;  // one 128-row slice: 16 KB
 
-__global__ void __launch_bounds__(256)
-score_simple_kernel(const uint16_t* __restrict__ hidden, const int32_t* __restrict__ cu_seqlens,
-                    const int32_t* __restrict__ span, int B, int D, const uint16_t* __restrict__ Wg,
-                    const float* __restrict__ b1, const float* __restrict__ w2, float b2, int I, float eps,
-                    float* __restrict__ scores) {
-    __shared__ float xs[SC_ROWS][SC_KC + 1];
-    __shared__ float ws[256][SC_KC + 1];
-    __shared__ float rs[SC_ROWS];
-    __shared__ float red[SC_ROWS][8];
-    __shared__ int64_t rows[SC_ROWS];
+template <int NACC>
+struct ScoreCfg {
+    static constexpr int STAGES = NACC == 2 ? 3 : 4;
+    static constexpr int EPI_WARPS = 4 * NACC;
+    static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+    static constexpr uint32_t TMEM_COLS = NACC == 2 ? 512 : 256;
+    static constexpr int ROWS = 128 * NACC;
+};
 
-    // map this CTA's tile to (sequence, first prunable row)
-    int64_t tile = blockIdx.x;
-    int b = 0;
-    int64_t r0 = -1, r1 = -1;
-    for (; b < B; ++b) {
+template <int NACC>
+__host__ __device__ constexpr int score_stage_bytes(int I) { return NACC * TILE_A + I * 128; }
+
+// stages x (NACC row slices + one Wg slice of I rows), b1, w2, 16 barriers, tmem slot + abort flag
+template <int NACC>
+__host__ __device__ constexpr int score_smem_bytes(int I) {
+    return ScoreCfg<NACC>::STAGES * score_stage_bytes<NACC>(I) + 2 * 256 * 4 + 16 * 8 + 16 + 1024;
+}
+
+__device__ __forceinline__ float silu_f(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
+
+// Tile t of the concatenated per-sequence tile lists -> (first row, end of span).
+__device__ __forceinline__ bool map_tile(int64_t t, int rows, const int32_t* cu_seqlens, const int32_t* span, int B,
+                                         int64_t* row0, int64_t* row_end) {
+    for (int b = 0; b < B; ++b) {
         const int64_t s0 = cu_seqlens[b], n = cu_seqlens[b + 1] - s0;
         const int64_t p0 = s0 + min(max(static_cast<int64_t>(span[2 * b]), int64_t(0)), n);
         const int64_t p1 = max(p0, s0 + min(static_cast<int64_t>(span[2 * b + 1]), n));
-        const int64_t nt = (p1 - p0 + SC_ROWS - 1) / SC_ROWS;
-        if (tile < nt) {
-            r0 = p0 + tile * SC_ROWS;
-            r1 = p1;
-            break;
+        const int64_t nt = (p1 - p0 + rows - 1) / rows;
+        if (t < nt) {
+            *row0 = p0 + t * rows;
+            *row_end = p1;
+            return true;
         }
-        tile -= nt;
+        t -= nt;
     }
-    if (r0 < 0) return;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
-    if (tid < SC_ROWS) rows[tid] = (r0 + tid < r1) ? r0 + tid : -1;
+    return false;
+}
+
+template <int NACC>
+__global__ void __launch_bounds__(ScoreCfg<NACC>::THREADS, 1)
+score_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                const int32_t* __restrict__ cu_seqlens, const int32_t* __restrict__ span, int B, int D, int I,
+                const float* __restrict__ b1, const float* __restrict__ w2, float b2, float eps,
+                float* __restrict__ scores, int* __restrict__ status) {
+    using C = ScoreCfg<NACC>;
+    constexpr int STAGES = C::STAGES;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int stage_bytes = score_stage_bytes<NACC>(I);
+    float* s_b1 = reinterpret_cast<float*>(smem + STAGES * stage_bytes);
+    float* s_w2 = s_b1 + 256;
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar0 = sbase + STAGES * stage_bytes + 2 * 256 * 4;
+    // barriers: full[STAGES], empty[STAGES], acc_full, acc_empty, drain
+    auto full = [&](int s) { return bar0 + 8u * s; };
+    auto empty = [&](int s) { return bar0 + 8u * (STAGES + s); };
+    const uint32_t acc_full = bar0 + 8u * (2 * STAGES), acc_empty = bar0 + 8u * (2 * STAGES + 1);
+    const uint32_t drain = bar0 + 8u * (2 * STAGES + 2);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + STAGES * stage_bytes + 2 * 256 * 4 + 16 * 8);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nkb = D / KB;
+
+    for (int j = threadIdx.x; j < I; j += blockDim.x) {
+        s_b1[j] = b1[j];
+        s_w2[j] = w2[j];
+    }
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full(s), 1);
+            mbar_init(empty(s), 1 + C::EPI_WARPS);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, C::EPI_WARPS);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
     __syncthreads();
-    // sum of squares, one warp per row
-    for (int r = warp; r < SC_ROWS; r += nwarps) {
-        float ss = 0.f;
-        if (rows[r] >= 0)
-            for (int i = lane; i < D; i += 32) {
-                const float x = bf16_bits_to_float(hidden[rows[r] * D + i]);
-                ss = fmaf(x, x, ss);
-            }
-        for (int off = 16; off; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-        if (lane == 0) rs[r] = rsqrtf(ss / static_cast<float>(D) + eps);
-    }
-    float acc[SC_ROWS];
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            prefetch_tmap(&tmX);
+            prefetch_tmap(&tmW);
+            int64_t it = 0;
+            int issued[STAGES] = {};
+            bool ok = true;
+            for (int64_t t = blockIdx.x; ok; t += gridDim.x) {
+                int64_t row0, row_end;
+                if (!map_tile(t, C::ROWS, cu_seqlens, span, B, &row0, &row_end)) break;
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    const int s = static_cast<int>(it % STAGES);
+                    const int use = static_cast<int>(it / STAGES);
+                    if (use > 0 && !mbar_wait(empty(s), (use - 1) & 1, abort_flag, status, TG_WHERE_PRODUCER)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t st = sbase + s * stage_bytes;
+                    mbar_expect_tx(full(s), stage_bytes);
 #pragma unroll
-    for (int r = 0; r < SC_ROWS; ++r) acc[r] = 0.f;
-    const int j = tid;
-    for (int k0 = 0; k0 < D; k0 += SC_KC) {
-        __syncthreads();
-        for (int e = tid; e < SC_ROWS * SC_KC; e += blockDim.x) {
-            const int r = e / SC_KC, kk = e % SC_KC;
-            xs[r][kk] = rows[r] >= 0 ? bf16_bits_to_float(hidden[rows[r] * D + k0 + kk]) : 0.f;
-        }
-        for (int e = tid; e < I * SC_KC; e += blockDim.x) {
-            const int jj = e / SC_KC, kk = e % SC_KC;
-            ws[jj][kk] = bf16_bits_to_float(Wg[static_cast<int64_t>(jj) * D + k0 + kk]);
-        }
-        __syncthreads();
-        if (j < I) {
-            for (int kk = 0; kk < SC_KC; ++kk) {
-                const float w = ws[j][kk];
-#pragma unroll
-                for (int r = 0; r < SC_ROWS; ++r) acc[r] = fmaf(w, xs[r][kk], acc[r]);
+                    for (int a = 0; a < NACC; ++a)
+                        tma_load_2d(st + a * TILE_A, &tmX, kb * KB, static_cast<int32_t>(row0 + a * 128), full(s));
+                    tma_load_2d(st + NACC * TILE_A, &tmW, kb * KB, 0, full(s));
+                    ++issued[s];
+                }
+            }
+            if (*abort_flag) {
+                // let every copy this thread started land before the CTA exits
+                volatile int never = 0;
+                for (int s = 0; s < STAGES; ++s)
+                    if (issued[s]) mbar_wait(full(s), (issued[s] - 1) & 1, &never, status, TG_WHERE_DRAIN);
             }
         }
-    }
-    // epilogue: SiLU, output layer, reduction over j
-    for (int r = 0; r < SC_ROWS; ++r) {
-        float v = 0.f;
-        if (j < I) {
-            const float z = fmaf(rs[r], acc[r], b1[j]);
-            v = w2[j] * (z / (1.0f + expf(-z)));
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16_f32(128, I, false);
+            int64_t it = 0;
+            int tcount = 0;
+            bool ok = true;
+            for (int64_t t = blockIdx.x; ok; t += gridDim.x, ++tcount) {
+                int64_t row0, row_end;
+                if (!map_tile(t, C::ROWS, cu_seqlens, span, B, &row0, &row_end)) break;
+                if (tcount > 0 && !mbar_wait(acc_empty, (tcount - 1) & 1, abort_flag, status, TG_WHERE_MMA)) break;
+                tc_fence_after();
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    const int s = static_cast<int>(it % STAGES);
+                    const int use = static_cast<int>(it / STAGES);
+                    if (!mbar_wait(full(s), use & 1, abort_flag, status, TG_WHERE_MMA)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t st = sbase + s * stage_bytes;
+#pragma unroll
+                    for (int kk = 0; kk < KB / 16; ++kk) {
+                        const uint64_t bdesc = smem_desc_sw128(st + NACC * TILE_A + kk * 32, 16, 1024);
+#pragma unroll
+                        for (int a = 0; a < NACC; ++a)
+                            mma_bf16_ss(tmem + a * 256, smem_desc_sw128(st + a * TILE_A + kk * 32, 16, 1024), bdesc,
+                                        idesc, (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    mma_commit(empty(s));
+                }
+                if (ok) mma_commit(acc_full);
+            }
+            // every MMA, and the barrier arrivals its commits trigger, lands before the CTA exits
+            mma_commit(drain);
+            volatile int never = 0;
+            mbar_wait(drain, 0, &never, status, TG_WHERE_DRAIN);
         }
-        for (int off = 16; off; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-        if (lane == 0) red[r][warp] = v;
+    } else {
+        // ---------------------------------------------------------------- sum of squares + epilogue
+        const int e = warp - 2;          // 0 .. EPI_WARPS-1
+        const int a = e >> 2;            // accumulator of this warp
+        const int lg = warp & 3;         // TMEM lane group this warp may access
+        const int r = lg * 32 + lane;    // row within the 128-row slice == TMEM lane
+        const uint32_t lane_addr = static_cast<uint32_t>(lg * 32) << 16;
+        int64_t it = 0;
+        int tcount = 0;
+        bool ok = true;
+        for (int64_t t = blockIdx.x; ok; t += gridDim.x, ++tcount) {
+            int64_t row0, row_end;
+            if (!map_tile(t, C::ROWS, cu_seqlens, span, B, &row0, &row_end)) break;
+            float ss = 0.f;
+            for (int kb = 0; kb < nkb; ++kb, ++it) {
+                const int s = static_cast<int>(it % STAGES);
+                const int use = static_cast<int>(it / STAGES);
+                if (!mbar_wait(full(s), use & 1, abort_flag, status, TG_WHERE_SOFTMAX)) {
+                    ok = false;
+                    break;
+                }
+                // the row's 64 channels of this slice; chunk order is irrelevant for a sum of squares
+                const uint8_t* rowp = smem + s * stage_bytes + a * TILE_A + r * 128;
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(rowp + (ch << 4));
+                    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const float lo = __uint_as_float(wv[q] << 16), hi = __uint_as_float(wv[q] & 0xFFFF0000u);
+                        ss = fmaf(lo, lo, ss);
+                        ss = fmaf(hi, hi, ss);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(empty(s));
+            }
+            if (!ok) break;
+            if (!mbar_wait(acc_full, tcount & 1, abort_flag, status, TG_WHERE_SOFTMAX)) break;
+            tc_fence_after();
+            const float rr = rsqrtf(ss / static_cast<float>(D) + eps);
+            float acc_s = 0.f;
+            for (int c0 = 0; c0 < I; c0 += 32) {
+                float z[32];
+                tmem_ld32(tmem + a * 256 + lane_addr + c0, z);
+                tmem_wait_ld();
+#pragma unroll
+                for (int q = 0; q < 32; ++q) acc_s = fmaf(s_w2[c0 + q], silu_f(fmaf(rr, z[q], s_b1[c0 + q])), acc_s);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty);
+            const int64_t row = row0 + a * 128 + r;
+            if (row < row_end) scores[row] = acc_s + b2;
+        }
     }
+
+    tc_fence_before();
     __syncthreads();
-    if (tid < SC_ROWS && rows[tid] >= 0) {
-        float s = b2;
-        for (int w = 0; w < nwarps; ++w) s += red[tid][w];
-        scores[rows[tid]] = s;
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
     }
+}
+
+template <int NACC>
+cudaError_t launch_score_tc(const uint16_t* hidden, const int32_t* cu_seqlens, const int32_t* span, int B, int64_t T,
+                            int D, const uint16_t* Wg, const float* b1, const float* w2, float b2, int I, float eps,
+                            float* scores, int sms, cudaStream_t st) {
+    using C = ScoreCfg<NACC>;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<NACC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             score_smem_bytes<NACC>(256));
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    CUtensorMap tx, tw;
+    if (!encode_tmap_2d_bf16(&tx, hidden, static_cast<uint64_t>(D), static_cast<uint64_t>(T),
+                             static_cast<uint64_t>(D) * 2, KB, 128) ||
+        !encode_tmap_2d_bf16(&tw, Wg, static_cast<uint64_t>(D), static_cast<uint64_t>(I), static_cast<uint64_t>(D) * 2,
+                             KB, static_cast<uint32_t>(I)))
+        return cudaErrorInvalidValue;
+    const int64_t tiles_bound = (T + C::ROWS - 1) / C::ROWS + B;
+    const int grid = static_cast<int>(tiles_bound < sms ? tiles_bound : sms);
+    score_tc_kernel<NACC><<<grid, C::THREADS, score_smem_bytes<NACC>(I), st>>>(tx, tw, cu_seqlens, span, B, D, I, b1,
+                                                                              w2, b2, eps, scores,
+                                                                              device_status_ptr());
+    return cudaGetLastError();
 }
 
 }  // namespace
@@ -125,11 +305,15 @@ cudaError_t launch_gate_prepare(const uint16_t* gamma, const uint16_t* W1, int D
 cudaError_t launch_score(const uint16_t* hidden, const int32_t* cu_seqlens, const int32_t* span, int B,
                          int64_t T, int D, const uint16_t* Wg, const float* b1, const float* w2, float b2, int I,
                          float eps, float* scores, cudaStream_t st) {
-    const int64_t tiles = (T + SC_ROWS - 1) / SC_ROWS + B;  // upper bound over all spans
-    if (tiles <= 0) return cudaSuccess;
-    score_simple_kernel<<<static_cast<unsigned>(tiles), 256, 0, st>>>(hidden, cu_seqlens, span, B, D, Wg, b1, w2, b2,
-                                                                     I, eps, scores);
-    return cudaGetLastError();
+    if (T == 0 || B == 0) return cudaSuccess;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    // 256-row tiles halve the gate-weight traffic from L2 once there are more
+    // 128-row tiles than SMs; below that, 128-row tiles spread the rows wider.
+    if ((T + 127) / 128 > sms)
+        return launch_score_tc<2>(hidden, cu_seqlens, span, B, T, D, Wg, b1, w2, b2, I, eps, scores, sms, st);
+    return launch_score_tc<1>(hidden, cu_seqlens, span, B, T, D, Wg, b1, w2, b2, I, eps, scores, sms, st);
 }
 
 }  // namespace tg

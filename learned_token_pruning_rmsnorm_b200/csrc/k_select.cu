@@ -27,47 +27,54 @@ namespace {
 
 constexpr int SEL_THREADS = 1024;
 constexpr int SEL_WARPS = SEL_THREADS / 32;
-constexpr int SEL_ITEMS = 8;
-constexpr int SEL_SMEM_KEYS = 36864;  // 144 KB of cached keys
-constexpr int SEL_HIST_BYTES = SEL_WARPS * 256 * 4;
-constexpr int SEL_SMEM_BYTES = SEL_SMEM_KEYS * 4 + SEL_HIST_BYTES;
+constexpr int SEL_ITEMS = 16;                 // consecutive tokens per thread in the ordered scan
+constexpr int SEL_CACHE_KEYS = 40960;         // spans up to this length keep their keys in shared memory
+constexpr int SEL_HIST_BINS = 2048;
+constexpr int SEL_SMEM_BYTES = SEL_CACHE_KEYS * 4 + SEL_HIST_BINS * 4;
 
 struct SelShared {
     int warp_sums[SEL_WARPS];
-    int bcast[4];
+    int total;
+    uint32_t prefix, mask;
+    int remaining, bin_count;
 };
 
-// Exclusive scan of one int per thread over the block; returns the prefix and
-// writes the block total to *total.  All threads must call it.
-__device__ __forceinline__ int block_exclusive_scan(int v, int* total, SelShared& sh) {
+// Inclusive scan of one int per thread over the block; returns the
+// inclusive prefix and writes the block total to *total.  All threads call it.
+__device__ __forceinline__ int block_inclusive_scan(int v, int* total, SelShared& sh) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int x = v;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
-        int y = __shfl_up_sync(0xffffffffu, x, off);
+        const int y = __shfl_up_sync(0xffffffffu, x, off);
         if (lane >= off) x += y;
     }
     if (lane == 31) sh.warp_sums[warp] = x;
     __syncthreads();
     if (warp == 0) {
-        int w = sh.warp_sums[lane];
+        const int w = sh.warp_sums[lane];
         int s = w;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
-            int y = __shfl_up_sync(0xffffffffu, s, off);
+            const int y = __shfl_up_sync(0xffffffffu, s, off);
             if (lane >= off) s += y;
         }
-        sh.warp_sums[lane] = s - w;  // exclusive prefix of warp totals
-        if (lane == 31) sh.bcast[0] = s;
+        sh.warp_sums[lane] = s - w;  // exclusive prefix of the warp totals
+        if (lane == 31) sh.total = s;
     }
     __syncthreads();
-    const int res = sh.warp_sums[warp] + x - v;
-    *total = sh.bcast[0];
+    const int res = sh.warp_sums[warp] + x;
+    *total = sh.total;
     __syncthreads();
     return res;
 }
 
 __device__ __forceinline__ float logsigmoid_f(float s) { return fminf(s, 0.0f) - log1pf(expf(-fabsf(s))); }
+
+// inverse of score_key (every NaN comes back as a NaN, -0 as +0)
+__device__ __forceinline__ float key_to_score(uint32_t key) {
+    return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
 
 __global__ void __launch_bounds__(SEL_THREADS, 1)
 select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __restrict__ keep_in,
@@ -77,13 +84,11 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
                    int32_t* __restrict__ rank, float* __restrict__ gls) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     uint32_t* skeys = reinterpret_cast<uint32_t*>(smem_raw);
-    int* hist = reinterpret_cast<int*>(smem_raw + SEL_SMEM_KEYS * 4);  // [SEL_WARPS][256]
+    int* hist = reinterpret_cast<int*>(smem_raw + SEL_CACHE_KEYS * 4);
     __shared__ SelShared sh;
-    __shared__ uint32_t s_prefix, s_mask;
-    __shared__ int s_remaining;
 
     const int b = blockIdx.x;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x, lane = tid & 31;
     const int64_t s0 = cu_seqlens[b], s1 = cu_seqlens[b + 1];
     // spans are clamped into the sequence so that a malformed span cannot index outside it
     const int64_t p0 = s0 + min(max(static_cast<int64_t>(span[2 * b]), int64_t(0)), s1 - s0);
@@ -93,88 +98,83 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
     const int64_t m0 = emit ? cu_kept[b] : 0, m1 = emit ? cu_kept[b + 1] : 0;
 
     int64_t kk = P;
-    uint32_t thr = 0;       // the K-th largest key (when 0 < kk < P)
-    int64_t need_eq = 0;    // keys equal to thr that are kept
     if (mode == 0) {
         const int32_t kb = kbud[b];
         kk = (kb < 0 || static_cast<int64_t>(kb) > P) ? P : static_cast<int64_t>(kb);
     }
     const bool do_radix = (mode == 0) && kk > 0 && kk < P;
+    const bool cached = do_radix && P <= SEL_CACHE_KEYS;
+
+    uint32_t thr = 0;        // the K-th largest key
+    int64_t need_eq = 0;     // keys equal to thr that are kept (the lowest-indexed ones)
+    bool all_eq_kept = true; // every key equal to thr is kept: no tie ranking needed
 
     if (do_radix) {
-        const bool cached = P <= SEL_SMEM_KEYS;
         if (cached) {
-            for (int64_t i = tid; i < P; i += SEL_THREADS) skeys[i] = score_key(scores[p0 + i]);
+            for (int64_t i = tid; i < P; i += SEL_THREADS) skeys[i] = score_key(__ldg(scores + p0 + i));
         }
         if (tid == 0) {
-            s_prefix = 0u;
-            s_mask = 0u;
-            s_remaining = static_cast<int>(kk);
+            sh.prefix = 0u;
+            sh.mask = 0u;
+            sh.remaining = static_cast<int>(kk);
         }
-        __syncthreads();
-        for (int pass = 0; pass < 4; ++pass) {
-            const int shift = 24 - 8 * pass;
-            for (int i = tid; i < SEL_WARPS * 256; i += SEL_THREADS) hist[i] = 0;
+        // radix select, most significant digits first: 11 + 11 + 10 bits
+        const int shifts[3] = {21, 10, 0};
+        const int widths[3] = {11, 11, 10};
+        const int64_t P_pad = (P + SEL_THREADS - 1) / SEL_THREADS * SEL_THREADS;
+        for (int pass = 0; pass < 3; ++pass) {
+            const int shift = shifts[pass];
+            const int nbins = 1 << widths[pass];
+            const uint32_t dmask = static_cast<uint32_t>(nbins - 1);
+            for (int i = tid; i < nbins; i += SEL_THREADS) hist[i] = 0;
             __syncthreads();
-            const uint32_t prefix = s_prefix, mask = s_mask;
-            int* my_hist = hist + warp * 256;
-            // the loop bound is uniform per warp so that __match_any_sync sees full warps
-            for (int64_t base = 0; base < P; base += SEL_THREADS) {
-                const int64_t i = base + tid;
+            const uint32_t prefix = sh.prefix, mask = sh.mask;
+            for (int64_t i = tid; i < P_pad; i += SEL_THREADS) {
                 bool valid = i < P;
                 uint32_t key = 0;
-                if (valid) key = cached ? skeys[i] : score_key(scores[p0 + i]);
+                if (valid) key = cached ? skeys[i] : score_key(__ldg(scores + p0 + i));
                 valid = valid && ((key & mask) == prefix);
-                const uint32_t digit = valid ? ((key >> shift) & 255u) : 256u;
-                const unsigned peers = __match_any_sync(0xffffffffu, digit);
-                const int leader = __ffs(peers) - 1;
-                if (valid && lane == leader) atomicAdd(&my_hist[digit], __popc(peers));
+                const unsigned act = __ballot_sync(0xffffffffu, valid);
+                if (valid) {
+                    const uint32_t digit = (key >> shift) & dmask;
+                    const unsigned peers = __match_any_sync(act, digit);
+                    if (lane == __ffs(peers) - 1) atomicAdd(&hist[digit], __popc(peers));
+                }
             }
             __syncthreads();
-            // fold the per-warp histograms into warp 0's copy
-            for (int bin = tid; bin < 256; bin += SEL_THREADS) {
-                int sum = 0;
-                for (int w = 0; w < SEL_WARPS; ++w) sum += hist[w * 256 + bin];
-                hist[bin] = sum;
+            // locate the digit holding the remaining-th largest key: thread t owns the
+            // bins of digits nbins-1-t*bpt ... in descending order
+            const int bpt = nbins / SEL_THREADS;  // 2 or 1
+            int cnt[2] = {0, 0};
+            int local = 0;
+            for (int e = 0; e < bpt; ++e) {
+                cnt[e] = hist[nbins - 1 - (tid * bpt + e)];
+                local += cnt[e];
             }
-            __syncthreads();
-            if (warp == 0) {
-                // digits in descending order: lane l covers digits 255-8l ... 248-8l
-                int cnt[8];
-                int lsum = 0;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    cnt[e] = hist[255 - (lane * 8 + e)];
-                    lsum += cnt[e];
-                }
-                int incl = lsum;
-#pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    int y = __shfl_up_sync(0xffffffffu, incl, off);
-                    if (lane >= off) incl += y;
-                }
-                const int excl = incl - lsum;
-                const int rem = s_remaining;
-                __syncwarp();  // every lane has read s_remaining before one lane rewrites it
-                if (excl < rem && incl >= rem) {
-                    int cum = excl;
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        if (cum + cnt[e] >= rem) {
-                            const uint32_t dgt = 255u - static_cast<uint32_t>(lane * 8 + e);
-                            s_prefix = prefix | (dgt << shift);
-                            s_mask = mask | (255u << shift);
-                            s_remaining = rem - cum;
-                            break;
-                        }
-                        cum += cnt[e];
+            int total = 0;
+            const int incl = block_inclusive_scan(local, &total, sh);
+            const int excl = incl - local;
+            const int rem = sh.remaining;
+            __syncthreads();  // every thread has read sh.remaining before it is rewritten
+            if (excl < rem && incl >= rem) {
+                int cum = excl;
+                for (int e = 0; e < bpt; ++e) {
+                    if (cum + cnt[e] >= rem) {
+                        const uint32_t dgt = static_cast<uint32_t>(nbins - 1 - (tid * bpt + e));
+                        sh.prefix = prefix | (dgt << shift);
+                        sh.mask = mask | (dmask << shift);
+                        sh.remaining = rem - cum;
+                        sh.bin_count = cnt[e];
+                        break;
                     }
+                    cum += cnt[e];
                 }
             }
             __syncthreads();
         }
-        thr = s_prefix;
-        need_eq = s_remaining;
+        thr = sh.prefix;
+        need_eq = sh.remaining;
+        all_eq_kept = need_eq == sh.bin_count;  // the last bin holds exactly the keys equal to thr
     }
 
     // ---------------------------------------------------------------- ordered scan
@@ -182,64 +182,70 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
     int64_t eq_carry = 0, kept_carry = 0;
     for (int64_t cbase = 0; cbase < n; cbase += static_cast<int64_t>(SEL_THREADS) * SEL_ITEMS) {
         const int64_t t_first = s0 + cbase + static_cast<int64_t>(tid) * SEL_ITEMS;
-        bool kept[SEL_ITEMS];
-        bool prun[SEL_ITEMS];
-        float sc[SEL_ITEMS];
+        uint32_t kept_bits = 0, eq_bits = 0;
         int n_eq = 0;
-        bool is_eq[SEL_ITEMS];
 #pragma unroll
         for (int e = 0; e < SEL_ITEMS; ++e) {
             const int64_t t = t_first + e;
             const bool in = t < s1;
-            prun[e] = in && t >= p0 && t < p1;
-            sc[e] = prun[e] ? scores[t] : 0.0f;
-            is_eq[e] = false;
+            const bool prun = in && t >= p0 && t < p1;
+            bool kept;
             if (mode == 1) {
-                kept[e] = in && keep_in[t] != 0;
-            } else if (!prun[e]) {
-                kept[e] = in;
-            } else if (kk >= P) {
-                kept[e] = true;
-            } else if (kk == 0) {
-                kept[e] = false;
+                kept = in && keep_in[t] != 0;
+            } else if (!prun) {
+                kept = in;
+            } else if (!do_radix) {
+                kept = kk > 0;  // kk >= P keeps all, kk == 0 keeps none
             } else {
-                const uint32_t key = score_key(sc[e]);
-                kept[e] = key > thr;
-                is_eq[e] = key == thr;
-                n_eq += is_eq[e] ? 1 : 0;
+                const uint32_t key = cached ? skeys[t - p0] : score_key(__ldg(scores + t));
+                const bool eq = key == thr;
+                kept = key > thr || (eq && all_eq_kept);
+                if (eq && !all_eq_kept) {
+                    eq_bits |= 1u << e;
+                    ++n_eq;
+                }
             }
+            kept_bits |= kept ? (1u << e) : 0u;
         }
-        if (do_radix) {
+        if (!all_eq_kept) {
+            // rank the keys equal to thr in index order; the first need_eq are kept
             int eq_total = 0;
-            int64_t eq_rank = eq_carry + block_exclusive_scan(n_eq, &eq_total, sh);
+            int64_t eq_rank = eq_carry + block_inclusive_scan(n_eq, &eq_total, sh) - n_eq;
 #pragma unroll
             for (int e = 0; e < SEL_ITEMS; ++e) {
-                if (is_eq[e]) {
-                    kept[e] = eq_rank < need_eq;
+                if (eq_bits & (1u << e)) {
+                    if (eq_rank < need_eq) kept_bits |= 1u << e;
                     ++eq_rank;
                 }
             }
             eq_carry += eq_total;
         }
-        int n_kept = 0;
-#pragma unroll
-        for (int e = 0; e < SEL_ITEMS; ++e) n_kept += kept[e] ? 1 : 0;
+        const int n_kept = __popc(kept_bits);
         int kept_total = 0;
-        int64_t m = m0 + kept_carry + block_exclusive_scan(n_kept, &kept_total, sh);
+        int64_t m = m0 + kept_carry + block_inclusive_scan(n_kept, &kept_total, sh) - n_kept;
         kept_carry += kept_total;
+        if (mode == 0) {
 #pragma unroll
-        for (int e = 0; e < SEL_ITEMS; ++e) {
-            const int64_t t = t_first + e;
-            if (t >= s1) break;
-            if (mode == 0) keep_out[t] = kept[e] ? 1 : 0;
-            if (kept[e]) {
+            for (int e = 0; e < SEL_ITEMS; ++e) {
+                const int64_t t = t_first + e;
+                if (t < s1) keep_out[t] = (kept_bits >> e) & 1u;
+            }
+        }
+        if (emit && kept_bits) {
+#pragma unroll
+            for (int e = 0; e < SEL_ITEMS; ++e) {
+                if (!((kept_bits >> e) & 1u)) continue;
+                const int64_t t = t_first + e;
                 // a caller-given keep vector that disagrees with cu_kept must
                 // not write outside [m0, m1)
-                if (emit && m < m1) {
+                if (m < m1) {
+                    const bool prun = t >= p0 && t < p1;
+                    float g = 0.0f;
+                    if (prun) g = logsigmoid_f(cached ? key_to_score(skeys[t - p0]) : __ldg(scores + t));
                     kept_idx[m] = static_cast<int32_t>(t);
                     pos[m] = static_cast<int32_t>(t - s0 + 1);
                     rank[m] = static_cast<int32_t>(m - m0 + 1);
-                    gls[m] = prun[e] ? logsigmoid_f(sc[e]) : 0.0f;
+                    gls[m] = g;
                 }
                 ++m;
             }

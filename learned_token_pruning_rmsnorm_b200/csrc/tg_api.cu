@@ -148,13 +148,16 @@ tg_status tg_score(const uint16_t* hidden, const int32_t* cu_seqlens, const int3
 }
 
 tg_status tg_select_topk(const float* scores, const int32_t* cu_seqlens, const int32_t* span, const int32_t* k, int B,
-                         int64_t T, uint8_t* keep, tg_stream_t stream) {
+                         int64_t T, uint8_t* keep, const int32_t* cu_kept, int32_t* kept_idx, int32_t* pos,
+                         int32_t* rank, float* gls, tg_stream_t stream) {
     TG_REQUIRE(B >= 0 && T >= 0, "negative size");
     if (B == 0 || T == 0) return TG_OK;
     TG_REQUIRE(scores && cu_seqlens && span && k && keep, "null pointer argument");
+    const bool emit = cu_kept && kept_idx;
+    TG_REQUIRE(!emit || (pos && rank && gls), "the fused compaction map needs pos, rank and gls");
     if (tg_status s = check_device()) return s;
-    return cuda_status(tg::launch_select_scan(0, scores, nullptr, cu_seqlens, span, k, nullptr, B, keep, nullptr,
-                                              nullptr, nullptr, nullptr, stream),
+    return cuda_status(tg::launch_select_scan(0, scores, nullptr, cu_seqlens, span, k, emit ? cu_kept : nullptr, B,
+                                              keep, emit ? kept_idx : nullptr, pos, rank, gls, stream),
                        "tg_select_topk launch");
 }
 
@@ -164,17 +167,20 @@ tg_status tg_compact(const uint16_t* hidden, const float* scores, const uint8_t*
                      tg_stream_t stream) {
     TG_REQUIRE(B >= 0 && T >= 0 && M_total >= 0 && M_total <= T, "bad sizes (B=%d T=%lld M=%lld)", B, (long long)T,
                (long long)M_total);
-    if (B == 0 || T == 0) return TG_OK;
-    TG_REQUIRE(scores && keep && cu_seqlens && span && cu_kept && pos && rank && gls && kept_idx,
-               "null pointer argument");
+    if (B == 0 || T == 0 || M_total == 0) return TG_OK;  // nothing is kept: no output to write
+    TG_REQUIRE(kept_idx, "null kept_idx");
+    if (keep) TG_REQUIRE(scores && cu_seqlens && span && cu_kept && pos && rank && gls, "null pointer argument");
+    else TG_REQUIRE(hidden_kept, "keep == NULL gathers rows: hidden_kept is required");
     if (hidden_kept) {
         TG_SUPPORT(D >= 8 && D % 8 == 0, "D=%d must be a multiple of 8 for the row copy", D);
         TG_REQUIRE(hidden && aligned16(hidden) && aligned16(hidden_kept), "hidden rows must be 16-byte aligned");
     }
     if (tg_status s = check_device()) return s;
-    tg_status s = cuda_status(tg::launch_select_scan(1, scores, keep, cu_seqlens, span, nullptr, cu_kept, B, nullptr,
-                                                     kept_idx, pos, rank, gls, stream),
-                              "tg_compact scan launch");
+    tg_status s = TG_OK;
+    if (keep)
+        s = cuda_status(tg::launch_select_scan(1, scores, keep, cu_seqlens, span, nullptr, cu_kept, B, nullptr,
+                                               kept_idx, pos, rank, gls, stream),
+                        "tg_compact scan launch");
     if (s != TG_OK || !hidden_kept) return s;
     return cuda_status(tg::launch_gather_rows(hidden, kept_idx, M_total, T, D, hidden_kept, stream),
                        "tg_compact gather launch");
@@ -201,8 +207,9 @@ tg_status tg_gated_prefill_layer(const tg_prefill_layer_args* a, tg_stream_t str
     }
     if (a->B == 0 || a->T == 0) return TG_OK;
     TG_REQUIRE(a->hidden && a->cu_seqlens && a->span && a->k && a->Wg && a->b1 && a->w2 && a->cu_kept && a->scores &&
-                   a->keep && a->pos && a->rank && a->gls && a->kept_idx,
+                   a->keep,
                "null pointer argument");
+    TG_REQUIRE(a->M_total == 0 || (a->pos && a->rank && a->gls && a->kept_idx), "null compaction output");
     TG_REQUIRE(aligned16(a->hidden) && aligned16(a->Wg), "hidden and Wg must be 16-byte aligned");
     if (a->hidden_kept) TG_REQUIRE(aligned16(a->hidden_kept), "hidden_kept must be 16-byte aligned");
     if (tg_status s = check_device()) return s;
@@ -215,6 +222,7 @@ tg_status tg_gated_prefill_layer(const tg_prefill_layer_args* a, tg_stream_t str
                                                          a->gls, st),
                                   "select launch"))
         return s;
+    if (a->M_total == 0) return TG_OK;  // every token pruned: no kept rows, no attention
     if (a->hidden_kept) {
         if (tg_status s = cuda_status(tg::launch_gather_rows(a->hidden, a->kept_idx, a->M_total, a->T, a->D,
                                                              a->hidden_kept, st),

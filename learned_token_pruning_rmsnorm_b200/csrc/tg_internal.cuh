@@ -9,6 +9,13 @@
 
 namespace tg {
 
+// Device status word bits (see tg_device_status in tokengate.h).
+constexpr int TG_DEVICE_TIMEOUT = 1 << 16;   // a bounded wait gave up
+constexpr int TG_WHERE_PRODUCER = 1 << 0;    // ... in the TMA producer
+constexpr int TG_WHERE_MMA = 1 << 1;         // ... in the MMA issuer
+constexpr int TG_WHERE_SOFTMAX = 1 << 2;     // ... in the softmax / epilogue warps
+constexpr int TG_WHERE_DRAIN = 1 << 3;       // ... while draining after an abort
+
 // ------------------------------------------------------------------ device helpers
 
 // Order-preserving map of an fp32 score to uint32 (larger score -> larger key).

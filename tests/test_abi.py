@@ -83,7 +83,9 @@ def test_invalid_shapes_are_refused_before_launch(lib):
     st = lib.tg_gated_attention(P, P, P, P, 1, 10, 10, 6, 4, 64, P, P, P, P, P, 0.1, P, None, None)
     assert st == _lib.TG_ERR_INVALID_ARG
     # null pointers
-    st = lib.tg_select_topk(None, P, P, P, 1, 10, P, None)
+    st = lib.tg_select_topk(None, P, P, P, 1, 10, P, None, None, None, None, None, None)
+    assert st == _lib.TG_ERR_INVALID_ARG
+    st = lib.tg_select_topk(P, P, P, P, 1, 10, P, P, P, None, None, None, None)  # map without pos/rank/gls
     assert st == _lib.TG_ERR_INVALID_ARG
     st = lib.tg_compact(P, P, P, P, P, 1, 10, 64, P, 20, P, P, P, P, P, None)  # M > T
     assert st == _lib.TG_ERR_INVALID_ARG
@@ -93,7 +95,7 @@ def test_invalid_shapes_are_refused_before_launch(lib):
 
 def test_empty_batches_are_no_ops(lib):
     from learned_token_pruning_rmsnorm_b200 import _lib
-    assert lib.tg_select_topk(None, None, None, None, 0, 0, None, None) == _lib.TG_OK
+    assert lib.tg_select_topk(None, None, None, None, 0, 0, None, None, None, None, None, None, None) == _lib.TG_OK
     assert lib.tg_score(None, None, None, 0, 0, 64, None, None, None, 0.0, 16, 1e-6, None, None) == _lib.TG_OK
 
 

@@ -118,10 +118,21 @@ def _select_and_compact(tg, w_cu, w_span, k, scores_f32, hidden_bits=None):
     np.testing.assert_array_equal(comp["rank"].cpu().numpy(), ref["rank"])
     np.testing.assert_array_equal(comp["kept_idx"].cpu().numpy(), ref["src"])
     gls = comp["gls"].cpu().numpy().astype(np.float64)
-    assert np.max(np.abs(gls - ref["gls"]) / np.maximum(1.0, np.abs(ref["gls"])), initial=0.0) <= H.GLS_ABS
+    # a NaN score gives a NaN bias on both sides
+    np.testing.assert_allclose(gls, ref["gls"], rtol=H.GLS_ABS, atol=H.GLS_ABS, equal_nan=True)
     assert (gls[ref["gls"] == 0] == 0).all()
     if hidden_bits is not None:
         np.testing.assert_array_equal(H.bf16_host_bits(comp["hidden_kept"]), ref["hidden_kept"])
+    # the fused path: selection writes the compaction map, then a gather-only compaction
+    keep2, cmap = tg.tg_select_topk(s_dev, cu, span, k, cu_kept=cu_kept, M_total=M)
+    np.testing.assert_array_equal(keep2.cpu().numpy(), keep_ref)
+    np.testing.assert_array_equal(cmap["kept_idx"].cpu().numpy(), ref["src"])
+    np.testing.assert_array_equal(cmap["pos"].cpu().numpy(), ref["pos"])
+    np.testing.assert_array_equal(cmap["rank"].cpu().numpy(), ref["rank"])
+    np.testing.assert_array_equal(cmap["gls"].cpu().numpy(), comp["gls"].cpu().numpy())  # NaN == NaN here
+    if hidden_bits is not None and M > 0:
+        hk = tg.tg_gather_kept(hid, cmap["kept_idx"])
+        np.testing.assert_array_equal(H.bf16_host_bits(hk), ref["hidden_kept"])
     return keep_ref, ref
 
 
