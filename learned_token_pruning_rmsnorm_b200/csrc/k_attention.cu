@@ -353,6 +353,357 @@ gated_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     }
 }
 
+// ---------------------------------------------------------------------------
+// Two query heads of one KV head per CTA (GQA groups of even size).
+//
+// 320 threads: warps 0-3 = softmax of head 0, warps 4-7 = softmax of head 1,
+// warp 8 = TMA producer, warp 9 = MMA issuer.  Both heads share every K/V
+// tile.  TMEM (512 columns): S0 | S1 | O0 | O1; P_h (bf16, two keys per
+// column) is written over the first 64 columns of S_h and read from TMEM as
+// the A operand of the PV MMA.  The MMA issuer interleaves
+//     S0(j) S1(j) | PV0(j) S0(j+1) | PV1(j) S1(j+1) | ...
+// so that one head's softmax overlaps the other head's tensor-core work;
+// tcgen05 operations of one thread execute in issue order, which is what
+// lets S_h(j+1) overwrite P_h(j) right after PV_h(j), and what makes the
+// commit after S_h(j) also cover PV_h(j-1) (so the softmax may rescale O_h
+// as soon as S_h(j) is complete).
+constexpr int G2_THREADS = 320;
+constexpr int G2_ILP = 8;  // independent partial max / sum chains per row
+
+template <int HD>
+struct G2Smem {
+    static constexpr int TILE_Q = BM * HD * 2;
+    static constexpr int TILE_KV = BN * HD * 2;
+    static constexpr int OFF_Q = 0;  // two heads
+    static constexpr int OFF_K = OFF_Q + 2 * TILE_Q;
+    static constexpr int OFF_V = OFF_K + 2 * TILE_KV;
+    static constexpr int OFF_BIAS = OFF_V + 2 * TILE_KV;
+    static constexpr int OFF_BAR = OFF_BIAS + 8 * 2 * BN * 4;  // a private bias copy per softmax warp
+    static constexpr int NUM_BARS = 16;
+    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+    static constexpr int BYTES = OFF_MISC + 16;
+    static constexpr int ALLOC = BYTES + 1024;
+    static constexpr uint32_t TMEM_COLS = 512;
+};
+
+enum : int {
+    G_Q_FULL = 0, G_K_FULL = 1, G_K_EMPTY = 3, G_V_FULL = 5, G_V_EMPTY = 7, G_S_FULL = 9, G_P_FULL = 11,
+    G_O_FULL = 13, G_DRAIN = 14
+};
+
+template <int HD>
+__global__ void __launch_bounds__(G2_THREADS, 1)
+gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const int32_t* __restrict__ cu_kept,
+                       const int32_t* __restrict__ pos, const int32_t* __restrict__ rank,
+                       const float* __restrict__ gls, const float* __restrict__ g, const float* __restrict__ c,
+                       float sm_scale, int Hq, int Hkv, int n_qt_max, uint16_t* __restrict__ out,
+                       float* __restrict__ lse, int* __restrict__ status) {
+    using L = G2Smem<HD>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+    const int pair = blockIdx.x;            // query heads 2*pair and 2*pair+1
+    const int qt = n_qt_max - 1 - static_cast<int>(blockIdx.y);
+    const int b = blockIdx.z;
+    const int seq0 = cu_kept[b];
+    const int Mb = cu_kept[b + 1] - seq0;
+    if (qt * BM >= Mb) return;
+    const int n_kv = qt + 1;
+    const int hk = (2 * pair) / (Hq / Hkv);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t sQ = sbase + L::OFF_Q, sK0 = sbase + L::OFF_K, sV0 = sbase + L::OFF_V;
+    auto bar = [&](int i) { return sbase + L::OFF_BAR + 8u * static_cast<uint32_t>(i); };
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+    float* sBias = reinterpret_cast<float*>(smem + L::OFF_BIAS);
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(G_Q_FULL), 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar(G_K_FULL + s), 1);
+            mbar_init(bar(G_K_EMPTY + s), 1);
+            mbar_init(bar(G_V_FULL + s), 1);
+            mbar_init(bar(G_V_EMPTY + s), 1);
+            mbar_init(bar(G_S_FULL + s), 1);
+            mbar_init(bar(G_P_FULL + s), 128);
+        }
+        mbar_init(bar(G_O_FULL), 1);
+        mbar_init(bar(G_DRAIN), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 8) {
+        tmem_alloc(smem_u32(tmem_slot), L::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 8) {
+        // ---------------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            prefetch_tmap(&tmQ);
+            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmV);
+            mbar_expect_tx(bar(G_Q_FULL), 2 * BM * HD * 2);
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                for (int hf = 0; hf < HD / 64; ++hf)
+                    tma_load_2d(sQ + hh * L::TILE_Q + hf * BM * 128, &tmQ, (2 * pair + hh) * HD + hf * 64,
+                                seq0 + qt * BM, bar(G_Q_FULL));
+            int k_issued[2] = {0, 0}, v_issued[2] = {0, 0};
+            for (int j = 0; j < n_kv; ++j) {
+                const int s = j & 1;
+                if (j >= 2 && !mbar_wait(bar(G_K_EMPTY + s), ((j - 2) >> 1) & 1, abort_flag, status,
+                                         TG_WHERE_PRODUCER))
+                    break;
+                mbar_expect_tx(bar(G_K_FULL + s), BN * HD * 2);
+#pragma unroll
+                for (int hf = 0; hf < HD / 64; ++hf)
+                    tma_load_2d(sK0 + s * L::TILE_KV + hf * BN * 128, &tmK, hk * HD + hf * 64, seq0 + j * BN,
+                                bar(G_K_FULL + s));
+                ++k_issued[s];
+                if (j >= 2 && !mbar_wait(bar(G_V_EMPTY + s), ((j - 2) >> 1) & 1, abort_flag, status,
+                                         TG_WHERE_PRODUCER))
+                    break;
+                mbar_expect_tx(bar(G_V_FULL + s), BN * HD * 2);
+#pragma unroll
+                for (int hf = 0; hf < HD / 64; ++hf)
+                    tma_load_2d(sV0 + s * L::TILE_KV + hf * BN * 128, &tmV, hk * HD + hf * 64, seq0 + j * BN,
+                                bar(G_V_FULL + s));
+                ++v_issued[s];
+            }
+            if (*abort_flag) {
+                drain_wait(bar(G_Q_FULL), 0, status);
+                for (int s = 0; s < 2; ++s) {
+                    if (k_issued[s]) drain_wait(bar(G_K_FULL + s), (k_issued[s] - 1) & 1, status);
+                    if (v_issued[s]) drain_wait(bar(G_V_FULL + s), (v_issued[s] - 1) & 1, status);
+                }
+            }
+        }
+    } else if (warp == 9) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false);
+            constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, HD, true);
+            auto issue_s = [&](int hh, int j) {
+                const uint32_t kb = sK0 + (j & 1) * L::TILE_KV;
+                const uint32_t qb = sQ + hh * L::TILE_Q;
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    const uint32_t off_q = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+                    const uint32_t off_k = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
+                    mma_bf16_ss(tmem + hh * BN, smem_desc_sw128(qb + off_q, 16, 1024),
+                                smem_desc_sw128(kb + off_k, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+                }
+            };
+            auto issue_pv = [&](int hh, int j) {
+                const uint32_t vb = sV0 + (j & 1) * L::TILE_KV;
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk)
+                    mma_bf16_ts(tmem + 2 * BN + hh * HD, tmem + hh * BN + kk * 8,
+                                smem_desc_sw128(vb + kk * 16 * 128, BN * 128, 1024), idesc_pv,
+                                (j > 0 || kk > 0) ? 1u : 0u);
+            };
+            bool ok = mbar_wait(bar(G_Q_FULL), 0, abort_flag, status, TG_WHERE_MMA) &&
+                      mbar_wait(bar(G_K_FULL), 0, abort_flag, status, TG_WHERE_MMA);
+            if (ok) {
+                tc_fence_after();
+                issue_s(0, 0);
+                mma_commit(bar(G_S_FULL + 0));
+                issue_s(1, 0);
+                mma_commit(bar(G_S_FULL + 1));
+                mma_commit(bar(G_K_EMPTY + 0));
+            }
+            for (int j = 0; ok && j < n_kv; ++j) {
+                const int s = j & 1;
+                const bool more = j + 1 < n_kv;
+                ok = mbar_wait(bar(G_V_FULL + s), (j >> 1) & 1, abort_flag, status, TG_WHERE_MMA) &&
+                     mbar_wait(bar(G_P_FULL + 0), j & 1, abort_flag, status, TG_WHERE_MMA);
+                if (!ok) break;
+                tc_fence_after();
+                issue_pv(0, j);
+                if (more) {
+                    ok = mbar_wait(bar(G_K_FULL + (s ^ 1)), ((j + 1) >> 1) & 1, abort_flag, status, TG_WHERE_MMA);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_s(0, j + 1);
+                    mma_commit(bar(G_S_FULL + 0));
+                }
+                ok = mbar_wait(bar(G_P_FULL + 1), j & 1, abort_flag, status, TG_WHERE_MMA);
+                if (!ok) break;
+                tc_fence_after();
+                issue_pv(1, j);
+                mma_commit(bar(G_V_EMPTY + s));
+                if (more) {
+                    issue_s(1, j + 1);
+                    mma_commit(bar(G_S_FULL + 1));
+                    mma_commit(bar(G_K_EMPTY + (s ^ 1)));
+                }
+            }
+            if (ok) mma_commit(bar(G_O_FULL));
+            mma_commit(bar(G_DRAIN));
+            drain_wait(bar(G_DRAIN), 0, status);
+        }
+    } else {
+        // ---------------------------------------------------------------- softmax, warps 0-7
+        const int hh = warp >> 2;             // which of the two heads
+        const int h = 2 * pair + hh;
+        const int r = threadIdx.x & 127;      // query row == TMEM lane
+        const int lg = warp & 3;
+        const int q_local = qt * BM + r;
+        const bool valid_row = q_local < Mb;
+        const int qg = seq0 + q_local;
+        float inv_tau = 1.0f;
+        if (valid_row) inv_tau = 1.0f / (1.0f + c[h] * logf(static_cast<float>(pos[qg]) / static_cast<float>(rank[qg])));
+        const float alpha = sm_scale * LOG2E * inv_tau;
+        const float gscale = softplus_f(g[h]) * LOG2E;
+        const uint32_t lane_addr = static_cast<uint32_t>(lg * 32) << 16;
+        const uint32_t tS = tmem + lane_addr + hh * BN;
+        const uint32_t tO = tmem + lane_addr + 2 * BN + hh * HD;
+        float* wbias = sBias + warp * (2 * BN);
+        float m_run = -INFINITY, l_run = 0.f;
+        bool ok = true;
+        for (int j = 0; j < n_kv; ++j) {
+            const int s = j & 1;
+#pragma unroll
+            for (int e = 0; e < BN / 32; ++e) {
+                const int key_local = j * BN + e * 32 + lane;
+                wbias[s * BN + e * 32 + lane] = key_local < Mb ? gscale * gls[seq0 + key_local] : 0.f;
+            }
+            __syncwarp();
+            ok = mbar_wait(bar(G_S_FULL + hh), j & 1, abort_flag, status, TG_WHERE_SOFTMAX);
+            if (!ok) break;
+            tc_fence_after();
+            float x[BN];
+#pragma unroll
+            for (int ch = 0; ch < BN / 32; ++ch) tmem_ld32(tS + ch * 32, x + ch * 32);
+            tmem_wait_ld();
+            const float* bias = wbias + s * BN;
+            float mp[G2_ILP];
+#pragma unroll
+            for (int i = 0; i < G2_ILP; ++i) mp[i] = -INFINITY;
+            if (j == n_kv - 1) {
+                const int lim = q_local - j * BN;
+#pragma unroll
+                for (int cc = 0; cc < BN; ++cc) {
+                    const float v = fmaf(x[cc], alpha, bias[cc] * inv_tau);
+                    x[cc] = cc > lim ? -INFINITY : v;
+                    mp[cc % G2_ILP] = fmaxf(mp[cc % G2_ILP], x[cc]);
+                }
+            } else {
+#pragma unroll
+                for (int cc = 0; cc < BN; ++cc) {
+                    x[cc] = fmaf(x[cc], alpha, bias[cc] * inv_tau);
+                    mp[cc % G2_ILP] = fmaxf(mp[cc % G2_ILP], x[cc]);
+                }
+            }
+            float mx = mp[0];
+#pragma unroll
+            for (int i = 1; i < G2_ILP; ++i) mx = fmaxf(mx, mp[i]);
+            float corr = 1.0f;
+            bool rescale_o = false;
+            if (j == 0 || mx > m_run + RESCALE_THRESHOLD) {
+                const float m_new = fmaxf(m_run, mx);
+                corr = ex2_approx(m_run - m_new);
+                m_run = m_new;
+                rescale_o = j > 0;
+            }
+            float sp[G2_ILP];
+#pragma unroll
+            for (int i = 0; i < G2_ILP; ++i) sp[i] = 0.f;
+            uint32_t pk[BN / 2];
+#pragma unroll
+            for (int cc = 0; cc < BN; cc += 2) {
+                const float p0 = ex2_approx(x[cc] - m_run), p1 = ex2_approx(x[cc + 1] - m_run);
+                sp[cc % G2_ILP] += p0;
+                sp[(cc + 1) % G2_ILP] += p1;
+                pk[cc / 2] = pack_bf16x2(p0, p1);
+            }
+            // P_h over the first 64 columns of S_h: this thread's own lane, whose S loads are complete
+            tmem_st32u(tS, pk);
+            tmem_st32u(tS + 32, pk + 32);
+            float sum = 0.f;
+#pragma unroll
+            for (int i = 0; i < G2_ILP; ++i) sum += sp[i];
+            l_run = l_run * corr + sum;
+            if (rescale_o) {
+                // O_h is stable: PV_h(j-1) completed before S_h(j), PV_h(j) waits for P_h(j)
+#pragma unroll
+                for (int ch = 0; ch < HD / 32; ++ch) {
+                    float o[32];
+                    tmem_ld32(tO + ch * 32, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] *= corr;
+                    tmem_st32(tO + ch * 32, o);
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(G_P_FULL + hh));
+        }
+        // ---------------------------------------------------------------- epilogue
+        if (ok) ok = mbar_wait(bar(G_O_FULL), 0, abort_flag, status, TG_WHERE_SOFTMAX);
+        if (ok) {
+            tc_fence_after();
+            const float inv_l = 1.0f / l_run;
+            uint16_t* orow = out + (static_cast<size_t>(qg) * Hq + h) * HD;
+#pragma unroll
+            for (int ch = 0; ch < HD / 32; ++ch) {
+                float o[32];
+                tmem_ld32(tO + ch * 32, o);
+                tmem_wait_ld();
+                if (valid_row) {
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        uint4 v;
+                        v.x = pack_bf16x2(o[q4 * 8 + 0] * inv_l, o[q4 * 8 + 1] * inv_l);
+                        v.y = pack_bf16x2(o[q4 * 8 + 2] * inv_l, o[q4 * 8 + 3] * inv_l);
+                        v.z = pack_bf16x2(o[q4 * 8 + 4] * inv_l, o[q4 * 8 + 5] * inv_l);
+                        v.w = pack_bf16x2(o[q4 * 8 + 6] * inv_l, o[q4 * 8 + 7] * inv_l);
+                        *reinterpret_cast<uint4*>(orow + ch * 32 + q4 * 8) = v;
+                    }
+                }
+            }
+            if (valid_row && lse) lse[static_cast<size_t>(qg) * Hq + h] = (m_run + log2f(l_run)) / LOG2E;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 8) {
+        tc_fence_after();
+        tmem_dealloc(tmem, L::TMEM_COLS);
+    }
+}
+
+template <int HD>
+cudaError_t launch_gqa2(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const int32_t* cu_kept,
+                        int B, int max_M, int Hq, int Hkv, const int32_t* pos, const int32_t* rank, const float* gls,
+                        const float* g, const float* c, float sm_scale, uint16_t* out, float* lse, cudaStream_t st) {
+    using L = G2Smem<HD>;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(gated_attn_gqa2_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             L::ALLOC);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    const int n_qt_max = (max_M + BM - 1) / BM;
+    dim3 grid(Hq / 2, n_qt_max, B);
+    gated_attn_gqa2_kernel<HD><<<grid, G2_THREADS, L::ALLOC, st>>>(tq, tk, tv, cu_kept, pos, rank, gls, g, c,
+                                                                   sm_scale, Hq, Hkv, n_qt_max, out, lse,
+                                                                   device_status_ptr());
+    return cudaGetLastError();
+}
+
 template <int HD>
 cudaError_t launch_tc(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* cu_kept, int B,
                       int64_t M_total, int max_M, int Hq, int Hkv, const int32_t* pos, const int32_t* rank,
@@ -374,6 +725,8 @@ cudaError_t launch_tc(const uint16_t* q, const uint16_t* k, const uint16_t* v, c
         !encode_tmap_2d_bf16(&tv, v, static_cast<uint64_t>(Hkv) * HD, static_cast<uint64_t>(M_total),
                              static_cast<uint64_t>(Hkv) * HD * 2, 64, BN))
         return cudaErrorInvalidValue;
+    if ((Hq / Hkv) % 2 == 0)
+        return launch_gqa2<HD>(tq, tk, tv, cu_kept, B, max_M, Hq, Hkv, pos, rank, gls, g, c, sm_scale, out, lse, st);
     int* status = device_status_ptr();
     const int n_qt_max = (max_M + BM - 1) / BM;
     dim3 grid(Hq, n_qt_max, B);

@@ -222,11 +222,14 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                     ok = false;
                     break;
                 }
-                // the row's 64 channels of this slice; chunk order is irrelevant for a sum of squares
+                // the row's 64 channels of this slice.  Lane r starts at physical chunk
+                // (r & 7): the 128-byte swizzle then spreads a warp's 32 rows over all
+                // banks (4 wavefronts per 512-byte access, the minimum); chunk order is
+                // irrelevant for a sum of squares.
                 const uint8_t* rowp = smem + s * stage_bytes + a * TILE_A + r * 128;
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch) {
-                    const uint4 v = *reinterpret_cast<const uint4*>(rowp + (ch << 4));
+                    const uint4 v = *reinterpret_cast<const uint4*>(rowp + ((ch ^ (r & 7)) << 4));
                     const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
