@@ -64,7 +64,7 @@ typedef enum tg_status {
     TG_ERR_INVALID_ARG = 1, /* null pointer, bad size, inconsistent shapes */
     TG_ERR_UNSUPPORTED = 2, /* shape or device outside the supported set */
     TG_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
-    TG_ERR_TIMEOUT = 4      /* reserved: a bounded device-side wait gave up */
+    TG_ERR_TIMEOUT = 4      /* a bounded device-side wait gave up (see tg_device_status) */
 } tg_status;
 
 /* Version of this ABI (incremented on any signature change). */
@@ -218,6 +218,29 @@ typedef struct tg_prefill_layer_args {
 } tg_prefill_layer_args;
 
 tg_status tg_gated_prefill_layer(const tg_prefill_layer_args* args, tg_stream_t stream);
+
+/*
+ * Device status word (failure detection).  Every wait inside the kernels
+ * (on an mbarrier fed by TMA, by the tensor core or by other warps) is
+ * bounded: after 2 s the waiting thread raises its CTA's abort flag, ORs
+ * 0x10000 | <where> into the status word of the current device (where: 1 TMA
+ * producer, 2 MMA issuer, 4 softmax/epilogue warps, 8 draining after an
+ * abort), every role leaves its loop, copies in flight are awaited (again
+ * bounded), TMEM is freed and the kernel returns, leaving the context
+ * usable.  The outputs of such a call are unspecified.
+ * tg_device_status synchronises `stream`, copies the word to *h_word (may be
+ * NULL), clears it when `clear` is non-zero, and returns TG_ERR_TIMEOUT when
+ * a timeout was recorded, else TG_OK.
+ */
+tg_status tg_device_status(int32_t* h_word, int clear, tg_stream_t stream);
+
+/*
+ * Diagnostic: one CTA waits on an mbarrier that nothing ever completes, with
+ * the kernels' bounded-wait routine and a limit of timeout_ns (0 < t <= 10 s).
+ * The wait gives up, records a timeout in the status word and the kernel
+ * returns: no fault and no hang.  Used to test the failure path above.
+ */
+tg_status tg_selftest_bounded_wait(int64_t timeout_ns, tg_stream_t stream);
 
 #ifdef __cplusplus
 }

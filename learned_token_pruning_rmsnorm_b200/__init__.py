@@ -24,6 +24,7 @@ from ._lib import TokenGateError, load  # noqa: F401
 __all__ = [
     "TokenGateError", "load", "tg_abi_version", "tg_kept_count", "tg_gate_prepare", "tg_score",
     "tg_select_topk", "tg_compact", "tg_gather_kept", "tg_gated_attention", "tg_gated_prefill_layer",
+    "tg_device_status", "tg_selftest_bounded_wait",
 ]
 
 
@@ -196,6 +197,20 @@ def tg_gated_attention(q, k, v, cu_kept, max_M: int, pos, rank, gls, g, c, sm_sc
                                          gls.data_ptr(), g.data_ptr(), c.data_ptr(), float(sm_scale),
                                          out.data_ptr(), _lib.ptr(lse), _lib.stream_handle(dev)))
     return (out, lse) if want_lse or lse is not None else out
+
+
+def tg_device_status(clear: bool = True, device=None):
+    """(status, word): the device status word of the current device; status is
+    TG_OK or TG_ERR_TIMEOUT.  Synchronises the current stream."""
+    w = C.c_int32(0)
+    st = load().tg_device_status(C.byref(w), 1 if clear else 0, _lib.stream_handle(device))
+    if st not in (_lib.TG_OK, _lib.TG_ERR_TIMEOUT):
+        _lib.check(st)
+    return st, int(w.value)
+
+
+def tg_selftest_bounded_wait(timeout_ns: int, device=None) -> None:
+    _lib.check(load().tg_selftest_bounded_wait(int(timeout_ns), _lib.stream_handle(device)))
 
 
 class PrefillBuffers:

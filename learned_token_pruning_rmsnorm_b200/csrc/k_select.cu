@@ -5,38 +5,49 @@
 // (TokenGate AI summary, "Key Contributions" 1; README copy, "How it works").
 // Order: higher score first, then lower token index.
 //
-// Design (one CTA of 1024 threads per sequence; the span holds at most a few
-// hundred thousand scores, which sit in L2 right after the scoring kernel):
-//   1. radix select on order-preserving uint32 keys, 8-bit digits, MSB first,
-//      four passes; per-warp shared-memory histograms fed by warp-aggregated
-//      atomics (__match_any_sync), so that the few hot exponent bins of the
-//      first pass do not serialise.  Keys are cached in shared memory when the
-//      span fits (<= SEL_SMEM_KEYS keys), else re-read from global memory.
-//      Result: the K-th key u*, and need_eq = how many keys equal to u* are
-//      kept (the lowest-indexed ones).
-//   2. one ordered pass over the sequence in chunks of 1024 x SEL_ITEMS
-//      tokens: a block scan ranks the keys equal to u*, a second block scan
-//      numbers the kept tokens, and each kept token writes its compaction
-//      outputs (kept_idx, pos, rank, logsigmoid of its score).
+// Design: one cluster of SEL_CL CTAs per sequence.  CTA i owns a contiguous
+// slice of the sequence's tokens and caches the order-preserving uint32 keys
+// of its prunable tokens in shared memory.
+//   1. bucket select: the cluster agrees on the span's [min, max] key range,
+//      then each pass histograms the keys of the current range into <= 2048
+//      buckets of width 2^s (buckets span the data's actual range, so
+//      concentrated exponents still spread), sums the SEL_CL histograms
+//      through distributed shared memory, and narrows the range to the bucket
+//      holding the K-th key.  At most three passes reach a single key value:
+//      thr, with need_eq = how many keys equal to thr are kept (the
+//      lowest-indexed ones).
+//   2. ordered scan, one token per thread per row of 1024 tokens: ballots
+//      and a two-level prefix number the kept tokens, the cluster exchanges
+//      slice totals, and each kept token writes its compaction-map entry
+//      (kept_idx, pos, rank, logsigmoid of its score) with coalesced stores.
 // Everything is deterministic: atomics only build counts.
 
+#include <cooperative_groups.h>
+
 #include "tg_internal.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace tg {
 namespace {
 
+constexpr int SEL_CL = 8;                     // CTAs per sequence (one cluster)
 constexpr int SEL_THREADS = 1024;
 constexpr int SEL_WARPS = SEL_THREADS / 32;
-constexpr int SEL_ITEMS = 16;                 // consecutive tokens per thread in the ordered scan
-constexpr int SEL_CACHE_KEYS = 40960;         // spans up to this length keep their keys in shared memory
-constexpr int SEL_HIST_BINS = 2048;
-constexpr int SEL_SMEM_BYTES = SEL_CACHE_KEYS * 4 + SEL_HIST_BINS * 4;
+constexpr int SEL_CACHE_KEYS = 32768;         // keys cached per CTA (128 KB)
+constexpr int SEL_BINS = 2048;
+constexpr int SEL_SMEM_BYTES = SEL_CACHE_KEYS * 4 + 2 * SEL_BINS * 4;
 
 struct SelShared {
     int warp_sums[SEL_WARPS];
     int total;
-    uint32_t prefix, mask;
-    int remaining, bin_count;
+    uint32_t kmin, kmax;
+    int xchg[4];          // values this CTA publishes to the cluster
+    uint32_t lo;          // current key range [lo, lo + width)
+    uint64_t width;
+    int remaining;        // keys still to take from the current range, counted from its top
+    int bin_count;
+    int64_t above;        // kept keys above the current range
 };
 
 // Inclusive scan of one int per thread over the block; returns the
@@ -76,7 +87,24 @@ __device__ __forceinline__ float key_to_score(uint32_t key) {
     return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
 }
 
-__global__ void __launch_bounds__(SEL_THREADS, 1)
+__device__ __forceinline__ int bit_length(uint64_t v) { return v ? 64 - __clzll(static_cast<long long>(v)) : 0; }
+
+// Sum over the cluster of the int published by every CTA at sh.xchg[slot]
+// (each CTA must have written it before the cluster barrier that precedes the call).
+__device__ __forceinline__ void cluster_prefix(cg::cluster_group& cl, SelShared& sh, int slot, int rank_self,
+                                               int64_t* before, int64_t* total) {
+    int64_t b = 0, t = 0;
+    for (int r = 0; r < SEL_CL; ++r) {
+        const SelShared* o = cl.map_shared_rank(&sh, r);
+        const int v = o->xchg[slot];
+        if (r < rank_self) b += v;
+        t += v;
+    }
+    *before = b;
+    *total = t;
+}
+
+__global__ void __cluster_dims__(SEL_CL, 1, 1) __launch_bounds__(SEL_THREADS, 1)
 select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __restrict__ keep_in,
                    const int32_t* __restrict__ cu_seqlens, const int32_t* __restrict__ span,
                    const int32_t* __restrict__ kbud, const int32_t* __restrict__ cu_kept,
@@ -84,11 +112,13 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
                    int32_t* __restrict__ rank, float* __restrict__ gls) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     uint32_t* skeys = reinterpret_cast<uint32_t*>(smem_raw);
-    int* hist = reinterpret_cast<int*>(smem_raw + SEL_CACHE_KEYS * 4);
+    int* hist_buf = reinterpret_cast<int*>(smem_raw + SEL_CACHE_KEYS * 4);  // [2][SEL_BINS]
     __shared__ SelShared sh;
+    cg::cluster_group cl = cg::this_cluster();
 
-    const int b = blockIdx.x;
-    const int tid = threadIdx.x, lane = tid & 31;
+    const int crank = static_cast<int>(cl.block_rank());
+    const int b = blockIdx.y;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t s0 = cu_seqlens[b], s1 = cu_seqlens[b + 1];
     // spans are clamped into the sequence so that a malformed span cannot index outside it
     const int64_t p0 = s0 + min(max(static_cast<int64_t>(span[2 * b]), int64_t(0)), s1 - s0);
@@ -97,59 +127,89 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
     const bool emit = kept_idx != nullptr;  // cu_kept is only read when emitting
     const int64_t m0 = emit ? cu_kept[b] : 0, m1 = emit ? cu_kept[b + 1] : 0;
 
+    // this CTA's token slice [t0, t1), rows of 1024 tokens
+    const int64_t n = s1 - s0;
+    const int64_t per = ((n + SEL_CL - 1) / SEL_CL + SEL_THREADS - 1) / SEL_THREADS * SEL_THREADS;
+    const int64_t t0 = min(s1, s0 + per * crank), t1 = min(s1, t0 + per);
+    // prunable part of the slice [k0, k1) and whether its keys fit the cache
+    const int64_t k0 = max(t0, p0), k1 = max(k0, min(t1, p1));
+    const bool cached = (k1 - k0) <= SEL_CACHE_KEYS;
+
     int64_t kk = P;
     if (mode == 0) {
         const int32_t kb = kbud[b];
         kk = (kb < 0 || static_cast<int64_t>(kb) > P) ? P : static_cast<int64_t>(kb);
     }
-    const bool do_radix = (mode == 0) && kk > 0 && kk < P;
-    const bool cached = do_radix && P <= SEL_CACHE_KEYS;
+    const bool do_select = (mode == 0) && kk > 0 && kk < P;
 
     uint32_t thr = 0;        // the K-th largest key
-    int64_t need_eq = 0;     // keys equal to thr that are kept (the lowest-indexed ones)
+    int64_t need_eq = 0;     // keys equal to thr that are kept
     bool all_eq_kept = true; // every key equal to thr is kept: no tie ranking needed
 
-    if (do_radix) {
-        if (cached) {
-            for (int64_t i = tid; i < P; i += SEL_THREADS) skeys[i] = score_key(__ldg(scores + p0 + i));
+    if (do_select) {
+        // ------------------------------------------------ cache keys, range of the span
+        uint32_t lmin = 0xFFFFFFFFu, lmax = 0u;
+        for (int64_t t = k0 + tid; t < k1; t += SEL_THREADS) {
+            const uint32_t key = score_key(__ldg(scores + t));
+            if (cached) skeys[t - k0] = key;
+            lmin = min(lmin, key);
+            lmax = max(lmax, key);
+        }
+#pragma unroll
+        for (int off = 16; off; off >>= 1) {
+            lmin = min(lmin, __shfl_xor_sync(0xffffffffu, lmin, off));
+            lmax = max(lmax, __shfl_xor_sync(0xffffffffu, lmax, off));
         }
         if (tid == 0) {
-            sh.prefix = 0u;
-            sh.mask = 0u;
-            sh.remaining = static_cast<int>(kk);
+            sh.kmin = 0xFFFFFFFFu;
+            sh.kmax = 0u;
         }
-        // radix select, most significant digits first: 11 + 11 + 10 bits
-        const int shifts[3] = {21, 10, 0};
-        const int widths[3] = {11, 11, 10};
-        const int64_t P_pad = (P + SEL_THREADS - 1) / SEL_THREADS * SEL_THREADS;
-        for (int pass = 0; pass < 3; ++pass) {
-            const int shift = shifts[pass];
-            const int nbins = 1 << widths[pass];
-            const uint32_t dmask = static_cast<uint32_t>(nbins - 1);
-            for (int i = tid; i < nbins; i += SEL_THREADS) hist[i] = 0;
-            __syncthreads();
-            const uint32_t prefix = sh.prefix, mask = sh.mask;
-            for (int64_t i = tid; i < P_pad; i += SEL_THREADS) {
-                bool valid = i < P;
-                uint32_t key = 0;
-                if (valid) key = cached ? skeys[i] : score_key(__ldg(scores + p0 + i));
-                valid = valid && ((key & mask) == prefix);
-                const unsigned act = __ballot_sync(0xffffffffu, valid);
-                if (valid) {
-                    const uint32_t digit = (key >> shift) & dmask;
-                    const unsigned peers = __match_any_sync(act, digit);
-                    if (lane == __ffs(peers) - 1) atomicAdd(&hist[digit], __popc(peers));
-                }
+        __syncthreads();
+        if (lane == 0) {
+            atomicMin(&sh.kmin, lmin);
+            atomicMax(&sh.kmax, lmax);
+        }
+        cl.sync();  // every CTA's slice min/max is published
+        if (tid == 0) {
+            uint32_t gmin = 0xFFFFFFFFu, gmax = 0u;
+            for (int r = 0; r < SEL_CL; ++r) {
+                const SelShared* o = cl.map_shared_rank(&sh, r);
+                gmin = min(gmin, o->kmin);
+                gmax = max(gmax, o->kmax);
             }
+            sh.lo = gmin;
+            sh.width = static_cast<uint64_t>(gmax) - gmin + 1;
+            sh.remaining = static_cast<int>(kk);
+            sh.above = 0;
+        }
+        __syncthreads();
+        // ------------------------------------------------ bucket passes
+        for (int pass = 0;; ++pass) {
+            const uint32_t lo = sh.lo;
+            const uint64_t width = sh.width;
+            const int sh_bits = max(0, bit_length(width - 1) - 11);  // bucket width 2^sh_bits
+            const int nb = static_cast<int>(((width - 1) >> sh_bits) + 1);
+            int* hist = hist_buf + (pass & 1) * SEL_BINS;
+            for (int i = tid; i < nb; i += SEL_THREADS) hist[i] = 0;
             __syncthreads();
-            // locate the digit holding the remaining-th largest key: thread t owns the
-            // bins of digits nbins-1-t*bpt ... in descending order
-            const int bpt = nbins / SEL_THREADS;  // 2 or 1
+            for (int64_t t = k0 + tid; t < k1; t += SEL_THREADS) {
+                const uint32_t key = cached ? skeys[t - k0] : score_key(__ldg(scores + t));
+                const uint32_t d = key - lo;  // wraps for keys below lo: excluded by the range test
+                if (key >= lo && static_cast<uint64_t>(d) < width) atomicAdd(&hist[d >> sh_bits], 1);
+            }
+            cl.sync();  // every CTA's histogram of this pass is complete
+            // bucket search from the top: thread tid owns buckets nb-1-2*tid and nb-2-2*tid
             int cnt[2] = {0, 0};
             int local = 0;
-            for (int e = 0; e < bpt; ++e) {
-                cnt[e] = hist[nbins - 1 - (tid * bpt + e)];
-                local += cnt[e];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int bin = nb - 1 - (2 * tid + e);
+                if (bin >= 0) {
+                    int v = 0;
+                    for (int r = 0; r < SEL_CL; ++r) v += cl.map_shared_rank(hist, r)[bin];
+                    cnt[e] = v;
+                    local += v;
+                }
             }
             int total = 0;
             const int incl = block_inclusive_scan(local, &total, sh);
@@ -158,99 +218,126 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
             __syncthreads();  // every thread has read sh.remaining before it is rewritten
             if (excl < rem && incl >= rem) {
                 int cum = excl;
-                for (int e = 0; e < bpt; ++e) {
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
                     if (cum + cnt[e] >= rem) {
-                        const uint32_t dgt = static_cast<uint32_t>(nbins - 1 - (tid * bpt + e));
-                        sh.prefix = prefix | (dgt << shift);
-                        sh.mask = mask | (dmask << shift);
+                        const uint32_t bin = static_cast<uint32_t>(nb - 1 - (2 * tid + e));
+                        const uint64_t new_lo = static_cast<uint64_t>(lo) + (static_cast<uint64_t>(bin) << sh_bits);
+                        const uint64_t end = static_cast<uint64_t>(lo) + width;
+                        sh.lo = static_cast<uint32_t>(new_lo);
+                        sh.width = min(static_cast<uint64_t>(1) << sh_bits, end - new_lo);
                         sh.remaining = rem - cum;
                         sh.bin_count = cnt[e];
+                        sh.above += cum;
                         break;
                     }
                     cum += cnt[e];
                 }
             }
             __syncthreads();
+            if (sh_bits == 0) break;  // the bucket is a single key value
         }
-        thr = sh.prefix;
+        thr = sh.lo;
         need_eq = sh.remaining;
-        all_eq_kept = need_eq == sh.bin_count;  // the last bin holds exactly the keys equal to thr
+        all_eq_kept = need_eq == sh.bin_count;
     }
 
     // ---------------------------------------------------------------- ordered scan
-    const int64_t n = s1 - s0;
-    int64_t eq_carry = 0, kept_carry = 0;
-    for (int64_t cbase = 0; cbase < n; cbase += static_cast<int64_t>(SEL_THREADS) * SEL_ITEMS) {
-        const int64_t t_first = s0 + cbase + static_cast<int64_t>(tid) * SEL_ITEMS;
-        uint32_t kept_bits = 0, eq_bits = 0;
-        int n_eq = 0;
-#pragma unroll
-        for (int e = 0; e < SEL_ITEMS; ++e) {
-            const int64_t t = t_first + e;
-            const bool in = t < s1;
-            const bool prun = in && t >= p0 && t < p1;
-            bool kept;
-            if (mode == 1) {
-                kept = in && keep_in[t] != 0;
-            } else if (!prun) {
-                kept = in;
-            } else if (!do_radix) {
-                kept = kk > 0;  // kk >= P keeps all, kk == 0 keeps none
-            } else {
-                const uint32_t key = cached ? skeys[t - p0] : score_key(__ldg(scores + t));
-                const bool eq = key == thr;
-                kept = key > thr || (eq && all_eq_kept);
-                if (eq && !all_eq_kept) {
-                    eq_bits |= 1u << e;
-                    ++n_eq;
-                }
-            }
-            kept_bits |= kept ? (1u << e) : 0u;
+    // kept flag of token t (one per thread per row); eq marks a key equal to thr
+    // that is ranked by index when only some of them are kept
+    auto flags = [&](int64_t t, bool& kept, bool& eq) {
+        kept = false;
+        eq = false;
+        if (t >= t1) return;
+        const bool prun = t >= p0 && t < p1;
+        if (mode == 1) {
+            kept = keep_in[t] != 0;
+        } else if (!prun) {
+            kept = true;
+        } else if (!do_select) {
+            kept = kk > 0;  // kk >= P keeps all, kk == 0 keeps none
+        } else {
+            const uint32_t key = cached ? skeys[t - k0] : score_key(__ldg(scores + t));
+            kept = key > thr || (key == thr && all_eq_kept);
+            eq = key == thr && !all_eq_kept;
         }
-        if (!all_eq_kept) {
-            // rank the keys equal to thr in index order; the first need_eq are kept
-            int eq_total = 0;
-            int64_t eq_rank = eq_carry + block_inclusive_scan(n_eq, &eq_total, sh) - n_eq;
-#pragma unroll
-            for (int e = 0; e < SEL_ITEMS; ++e) {
-                if (eq_bits & (1u << e)) {
-                    if (eq_rank < need_eq) kept_bits |= 1u << e;
-                    ++eq_rank;
-                }
-            }
-            eq_carry += eq_total;
-        }
-        const int n_kept = __popc(kept_bits);
-        int kept_total = 0;
-        int64_t m = m0 + kept_carry + block_inclusive_scan(n_kept, &kept_total, sh) - n_kept;
-        kept_carry += kept_total;
-        if (mode == 0) {
-#pragma unroll
-            for (int e = 0; e < SEL_ITEMS; ++e) {
-                const int64_t t = t_first + e;
-                if (t < s1) keep_out[t] = (kept_bits >> e) & 1u;
-            }
-        }
-        if (emit && kept_bits) {
-#pragma unroll
-            for (int e = 0; e < SEL_ITEMS; ++e) {
-                if (!((kept_bits >> e) & 1u)) continue;
-                const int64_t t = t_first + e;
-                // a caller-given keep vector that disagrees with cu_kept must
-                // not write outside [m0, m1)
-                if (m < m1) {
-                    const bool prun = t >= p0 && t < p1;
-                    float g = 0.0f;
-                    if (prun) g = logsigmoid_f(cached ? key_to_score(skeys[t - p0]) : __ldg(scores + t));
-                    kept_idx[m] = static_cast<int32_t>(t);
-                    pos[m] = static_cast<int32_t>(t - s0 + 1);
-                    rank[m] = static_cast<int32_t>(m - m0 + 1);
-                    gls[m] = g;
-                }
-                ++m;
-            }
-        }
+    };
+    const int nrows = static_cast<int>((t1 - t0 + SEL_THREADS - 1) / SEL_THREADS);
+    const unsigned lt_mask = (1u << lane) - 1u;
+
+    // slice totals: kept tokens and (for the tie ranking) keys equal to thr
+    int my_kept = 0, my_eq = 0;
+    for (int r = 0; r < nrows; ++r) {
+        bool kept, eq;
+        flags(t0 + static_cast<int64_t>(r) * SEL_THREADS + tid, kept, eq);
+        my_kept += kept;
+        my_eq += eq;
     }
+    int tot_kept = 0, tot_eq = 0;
+    block_inclusive_scan(my_kept, &tot_kept, sh);
+    if (!all_eq_kept) block_inclusive_scan(my_eq, &tot_eq, sh);
+    if (tid == 0) {
+        sh.xchg[0] = tot_kept;
+        sh.xchg[1] = tot_eq;
+    }
+    cl.sync();
+    int64_t kept_before = 0, kept_all = 0, eq_before = 0, eq_all = 0;
+    cluster_prefix(cl, sh, 0, crank, &kept_before, &kept_all);
+    if (!all_eq_kept) cluster_prefix(cl, sh, 1, crank, &eq_before, &eq_all);
+    // the keys equal to thr that this slice keeps: ranks [eq_before, eq_before + tot_eq) among all equal keys
+    int64_t eq_seen = eq_before;    // equal keys before the current row, in index order
+    int64_t m = m0 + kept_before;   // compaction index of the first kept token of the current row
+    // kept-before counts the tie-ranked keys as not kept; correct for the ones this CTA's
+    // predecessors keep
+    if (!all_eq_kept) m += min(eq_before, need_eq);
+    __shared__ int row_warp_kept[SEL_WARPS], row_warp_eq[SEL_WARPS];
+    for (int r = 0; r < nrows; ++r) {
+        const int64_t t = t0 + static_cast<int64_t>(r) * SEL_THREADS + tid;
+        bool kept, eq;
+        flags(t, kept, eq);
+        const unsigned eq_ball = __ballot_sync(0xffffffffu, eq);
+        if (!all_eq_kept) {
+            if (lane == 0) row_warp_eq[warp] = __popc(eq_ball);
+            __syncthreads();
+            int eq_prefix = 0, eq_row = 0;
+            for (int w = 0; w < SEL_WARPS; ++w) {
+                const int v = row_warp_eq[w];
+                if (w < warp) eq_prefix += v;
+                eq_row += v;
+            }
+            const int64_t eq_rank = eq_seen + eq_prefix + __popc(eq_ball & lt_mask);
+            if (eq && eq_rank < need_eq) kept = true;
+            eq_seen += eq_row;
+            __syncthreads();
+        }
+        const unsigned kept_ball = __ballot_sync(0xffffffffu, kept);
+        if (lane == 0) row_warp_kept[warp] = __popc(kept_ball);
+        __syncthreads();
+        int kept_prefix = 0, kept_row = 0;
+        for (int w = 0; w < SEL_WARPS; ++w) {
+            const int v = row_warp_kept[w];
+            if (w < warp) kept_prefix += v;
+            kept_row += v;
+        }
+        __syncthreads();
+        if (t < t1) {
+            if (mode == 0) keep_out[t] = kept ? 1 : 0;
+            const int64_t mi = m + kept_prefix + __popc(kept_ball & lt_mask);
+            // a caller-given keep vector that disagrees with cu_kept must not
+            // write outside [m0, m1)
+            if (emit && kept && mi < m1) {
+                const bool prun = t >= p0 && t < p1;
+                float g = 0.0f;
+                if (prun) g = logsigmoid_f(cached && do_select ? key_to_score(skeys[t - k0]) : __ldg(scores + t));
+                kept_idx[mi] = static_cast<int32_t>(t);
+                pos[mi] = static_cast<int32_t>(t - s0 + 1);
+                rank[mi] = static_cast<int32_t>(mi - m0 + 1);
+                gls[mi] = g;
+            }
+        }
+        m += kept_row;
+    }
+    cl.sync();  // no CTA leaves while another may still read its shared memory
 }
 
 // Row gather hidden_kept[m, :] = hidden[kept_idx[m], :], one warp per row,
@@ -297,8 +384,9 @@ cudaError_t launch_select_scan(int mode, const float* scores, const uint8_t* kee
         attr_set = true;
     }
     if (B == 0) return cudaSuccess;
-    select_scan_kernel<<<B, SEL_THREADS, SEL_SMEM_BYTES, st>>>(mode, scores, keep_in, cu_seqlens, span, k, cu_kept,
-                                                               keep_out, kept_idx, pos, rank, gls);
+    select_scan_kernel<<<dim3(SEL_CL, B), SEL_THREADS, SEL_SMEM_BYTES, st>>>(mode, scores, keep_in, cu_seqlens, span,
+                                                                            k, cu_kept, keep_out, kept_idx, pos,
+                                                                            rank, gls);
     return cudaGetLastError();
 }
 

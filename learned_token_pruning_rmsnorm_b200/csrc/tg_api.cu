@@ -194,6 +194,21 @@ tg_status tg_gated_attention(const uint16_t* q, const uint16_t* k, const uint16_
                         stream);
 }
 
+tg_status tg_device_status(int32_t* h_word, int clear, tg_stream_t stream) {
+    if (tg_status s = check_device()) return s;
+    int32_t w = 0;
+    if (tg_status s = cuda_status(tg::read_device_status(&w, clear != 0, stream), "tg_device_status")) return s;
+    if (h_word) *h_word = w;
+    if (w & tg::TG_DEVICE_TIMEOUT) return fail(TG_ERR_TIMEOUT, "a bounded device wait gave up (status word 0x%x)", w);
+    return TG_OK;
+}
+
+tg_status tg_selftest_bounded_wait(int64_t timeout_ns, tg_stream_t stream) {
+    TG_REQUIRE(timeout_ns > 0 && timeout_ns <= 10000000000LL, "timeout_ns must be in (0, 10 s]");
+    if (tg_status s = check_device()) return s;
+    return cuda_status(tg::launch_selftest_wait(timeout_ns, stream), "tg_selftest_bounded_wait launch");
+}
+
 tg_status tg_gated_prefill_layer(const tg_prefill_layer_args* a, tg_stream_t stream) {
     TG_REQUIRE(a != nullptr, "null args");
     TG_REQUIRE(a->B >= 0 && a->T >= 0 && a->M_total >= 0 && a->M_total <= a->T && a->n_layers >= 0, "bad sizes");

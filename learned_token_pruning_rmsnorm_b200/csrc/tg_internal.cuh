@@ -58,4 +58,8 @@ cudaError_t launch_gated_attention(const uint16_t* q, const uint16_t* k, const u
                                    const int32_t* rank, const float* gls, const float* g, const float* c,
                                    float sm_scale, uint16_t* out, float* lse, cudaStream_t st);
 
+cudaError_t launch_selftest_wait(int64_t timeout_ns, cudaStream_t st);
+
+cudaError_t read_device_status(int32_t* word, bool clear, cudaStream_t st);
+
 }  // namespace tg

@@ -63,4 +63,44 @@ int* device_status_ptr() {
     return g_status_ptr[dev];
 }
 
+namespace {
+
+// One CTA whose waiting thread blocks on an mbarrier that nothing ever
+// completes: the bounded wait must give up after timeout_ns, raise the abort
+// flag and record TG_DEVICE_TIMEOUT, and the kernel must then return.
+__global__ void selftest_wait_kernel(uint64_t timeout_ns, int* status) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        sm100::mbar_init(sm100::smem_u32(&bar), 1);
+        abort_flag = 0;
+        sm100::fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0)
+        sm100::mbar_wait(sm100::smem_u32(&bar), 0, &abort_flag, status, TG_WHERE_SOFTMAX, timeout_ns);
+    __syncthreads();
+}
+
+}  // namespace
+
+cudaError_t launch_selftest_wait(int64_t timeout_ns, cudaStream_t st) {
+    int* status = device_status_ptr();
+    if (!status) return cudaErrorInvalidSymbol;
+    selftest_wait_kernel<<<1, 32, 0, st>>>(static_cast<uint64_t>(timeout_ns), status);
+    return cudaGetLastError();
+}
+
+cudaError_t read_device_status(int32_t* word, bool clear, cudaStream_t st) {
+    int* status = device_status_ptr();
+    if (!status) return cudaErrorInvalidSymbol;
+    cudaError_t e = cudaMemcpyAsync(word, status, sizeof(int32_t), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e == cudaSuccess && clear) {
+        e = cudaMemsetAsync(status, 0, sizeof(int32_t), st);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    }
+    return e;
+}
+
 }  // namespace tg

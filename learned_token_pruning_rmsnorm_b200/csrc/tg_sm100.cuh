@@ -63,14 +63,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // false when the CTA is aborting or the wait ran out of time (then the abort
 // flag and the status word are set).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* status,
-                                          int where) {
+                                          int where, uint64_t timeout_ns = TG_WAIT_TIMEOUT_NS) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 63u) == 0) {
             if (*abort_flag) return false;
-            if (globaltimer() - t0 > TG_WAIT_TIMEOUT_NS) {
+            if (globaltimer() - t0 > timeout_ns) {
                 *abort_flag = 1;
                 if (status) atomicOr(status, TG_DEVICE_TIMEOUT | where);
                 return false;
