@@ -281,6 +281,8 @@ def run_gpu(args, w):
     B, T, D, I = w.B, w.T, w.D, w.I
     sm_scale = 1.0 / math.sqrt(w.d)
     L0 = layers[0]
+    _ws_ptr = None if call.ws is None else call.ws.data_ptr()
+    _ws_n = 0 if call.ws is None else call.ws.numel()
     # the product's kernels, one C-ABI call each, arguments bound once (host cost ~1 us per call)
     stage_calls = {
         "score": lambda: lib.tg_score(hidden.data_ptr(), call.cu.data_ptr(), call.sp.data_ptr(), B, T, D,
@@ -296,7 +298,7 @@ def run_gpu(args, w):
                                                     call.ck.data_ptr(), B, M, call.max_M, w.Hq, w.Hkv, w.d,
                                                     bufs.pos.data_ptr(), bufs.rank.data_ptr(), bufs.gls.data_ptr(),
                                                     L0["g"].data_ptr(), L0["c"].data_ptr(), sm_scale,
-                                                    bufs.out[0].data_ptr(), None, sh),
+                                                    bufs.out[0].data_ptr(), None, _ws_ptr, _ws_n, sh),
     }
 
     # warm-up (also sets kernel attributes before any capture)

@@ -164,11 +164,23 @@ tg_status tg_compact(const uint16_t* hidden, const float* scores, const uint8_t*
  * longest sequence's M_b (grid sizing).  sm_scale is usually 1/sqrt(d).
  * tau must stay positive: c_h >= 0 guarantees it since pos >= rank.
  * Tensor cores: bf16 operands, fp32 accumulation.
+ * ws (device, 256-byte aligned, may be NULL) is scratch for the causal work
+ * split: when the longest query tile would dominate the launch, long query
+ * tiles are cut into two KV chunks whose partial results meet in ws, and the
+ * last chunk to finish merges them.  ws_bytes must be at least
+ * tg_gated_attention_workspace_size(B, max_M, Hq, Hkv, d).  ws must be
+ * zero-filled before its first use; every call leaves it zero-filled again.
+ * Calls that share one ws must not run concurrently.  With ws == NULL the
+ * attention runs unsplit (same results, less balanced for small M).
  */
 tg_status tg_gated_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* cu_kept,
                              int B, int64_t M_total, int max_M, int Hq, int Hkv, int d, const int32_t* pos,
                              const int32_t* rank, const float* gls, const float* g, const float* c, float sm_scale,
-                             uint16_t* out, float* lse, tg_stream_t stream);
+                             uint16_t* out, float* lse, void* ws, size_t ws_bytes, tg_stream_t stream);
+
+/* Bytes of scratch tg_gated_attention may use for these sizes (0 when it
+ * never splits, or for unsupported sizes). */
+size_t tg_gated_attention_workspace_size(int B, int max_M, int Hq, int Hkv, int d);
 
 /*
  * The whole gated prefill at one gate layer: tg_score, tg_select_topk,
@@ -215,6 +227,8 @@ typedef struct tg_prefill_layer_args {
     const float* const* c;      /* n_layers x [Hq] */
     uint16_t* const* out;       /* n_layers x [M, Hq, d] out */
     float* const* lse;          /* n_layers x [M, Hq] out, array or entries may be NULL */
+    void* attn_ws;              /* scratch of tg_gated_attention, shared by the layers (may be NULL) */
+    size_t attn_ws_bytes;
 } tg_prefill_layer_args;
 
 tg_status tg_gated_prefill_layer(const tg_prefill_layer_args* args, tg_stream_t stream);

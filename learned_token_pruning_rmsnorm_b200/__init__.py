@@ -169,8 +169,25 @@ def tg_compact(hidden, scores, keep, cu_seqlens, span, cu_kept, M_total: int, wi
     return {"hidden_kept": hk, "pos": pos, "rank": rank, "gls": gls, "kept_idx": kept_idx}
 
 
+_WS_CACHE = {}
+
+
+def attention_workspace(B: int, max_M: int, Hq: int, Hkv: int, d: int, device) -> torch.Tensor | None:
+    """Zero-filled scratch for tg_gated_attention's causal work split (one per
+    device and size, reused; calls sharing it must not run concurrently)."""
+    n = int(load().tg_gated_attention_workspace_size(B, max_M, Hq, Hkv, d))
+    if n == 0:
+        return None
+    key = (torch.device(device), n)
+    ws = _WS_CACHE.get(key)
+    if ws is None:
+        ws = torch.zeros(n, dtype=torch.uint8, device=device)
+        _WS_CACHE[key] = ws
+    return ws
+
+
 def tg_gated_attention(q, k, v, cu_kept, max_M: int, pos, rank, gls, g, c, sm_scale: float | None = None,
-                       out=None, lse=None, want_lse: bool = False):
+                       out=None, lse=None, want_lse: bool = False, ws="auto"):
     M, Hq, d = q.shape
     Hkv = k.shape[1]
     dev = q.device
@@ -192,10 +209,13 @@ def tg_gated_attention(q, k, v, cu_kept, max_M: int, pos, rank, gls, g, c, sm_sc
         lse = torch.empty((M, Hq), dtype=torch.float32, device=dev)
     if lse is not None:
         _dev(lse, torch.float32, "lse", (M, Hq))
+    if isinstance(ws, str):
+        ws = attention_workspace(ck.numel() - 1, int(max_M), Hq, Hkv, d, dev)
     _lib.check(load().tg_gated_attention(q.data_ptr(), k.data_ptr(), v.data_ptr(), ck.data_ptr(), ck.numel() - 1,
                                          M, int(max_M), Hq, Hkv, d, pos.data_ptr(), rank.data_ptr(),
                                          gls.data_ptr(), g.data_ptr(), c.data_ptr(), float(sm_scale),
-                                         out.data_ptr(), _lib.ptr(lse), _lib.stream_handle(dev)))
+                                         out.data_ptr(), _lib.ptr(lse), _lib.ptr(ws),
+                                         0 if ws is None else ws.numel(), _lib.stream_handle(dev)))
     return (out, lse) if want_lse or lse is not None else out
 
 
@@ -274,6 +294,9 @@ class PrefillCall:
         a.q, a.kk, a.v, a.g, a.c, a.out = (cast(self._q), cast(self._k), cast(self._v), cast(self._g),
                                            cast(self._c), cast(self._o))
         a.lse = cast(self._lse)
+        self.ws = attention_workspace(a.B, self.max_M, Hq, Hkv, d, dev) if nl > 0 else None
+        a.attn_ws = _lib.ptr(self.ws)
+        a.attn_ws_bytes = 0 if self.ws is None else self.ws.numel()
         self.args = a
         self.device = dev
         self.bufs = bufs

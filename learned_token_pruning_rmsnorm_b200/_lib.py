@@ -41,6 +41,7 @@ class PrefillLayerArgs(C.Structure):
         ("scores", P), ("keep", P), ("hidden_kept", P), ("pos", P), ("rank", P), ("gls", P), ("kept_idx", P),
         ("n_layers", i32), ("Hq", i32), ("Hkv", i32), ("d", i32), ("sm_scale", f32),
         ("q", P), ("kk", P), ("v", P), ("g", P), ("c", P), ("out", P), ("lse", P),
+        ("attn_ws", P), ("attn_ws_bytes", C.c_size_t),
     ]
 
 
@@ -53,7 +54,9 @@ SIGNATURES = {
     "tg_score": ([P, P, P, i32, i64, i32, P, P, P, f32, i32, f32, P, P], i32),
     "tg_select_topk": ([P, P, P, P, i32, i64, P, P, P, P, P, P, P], i32),
     "tg_compact": ([P, P, P, P, P, i32, i64, i32, P, i64, P, P, P, P, P, P], i32),
-    "tg_gated_attention": ([P, P, P, P, i32, i64, i32, i32, i32, i32, P, P, P, P, P, f32, P, P, P], i32),
+    "tg_gated_attention": ([P, P, P, P, i32, i64, i32, i32, i32, i32, P, P, P, P, P, f32, P, P, P, C.c_size_t, P],
+                           i32),
+    "tg_gated_attention_workspace_size": ([i32, i32, i32, i32, i32], C.c_size_t),
     "tg_gated_prefill_layer": ([C.POINTER(PrefillLayerArgs), P], i32),
     "tg_device_status": ([P, i32, P], i32),
     "tg_selftest_bounded_wait": ([i64, P], i32),

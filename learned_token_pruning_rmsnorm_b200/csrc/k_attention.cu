@@ -59,6 +59,21 @@ enum : int {
     B_P_FULL = 13, B_PV_DONE = 14, B_DRAIN = 15
 };
 
+// Optional device trace (builds with -DTG_TRACE only): clock64 stamps of the
+// pipeline hand-offs of the CTA at blockIdx (0, 0, 0), 64 KV tiles at most.
+#ifdef TG_TRACE
+__device__ unsigned long long g_attn_trace[16 * 64];
+#define TG_TRACE_AT(point, j)                                                              \
+    do {                                                                                   \
+        if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && (j) < 64)             \
+            g_attn_trace[(point) * 64 + (j)] = static_cast<unsigned long long>(clock64()); \
+    } while (0)
+#else
+#define TG_TRACE_AT(point, j) \
+    do {                      \
+    } while (0)
+#endif
+
 __device__ __forceinline__ float softplus_f(float x) { return fmaxf(x, 0.f) + log1pf(expf(-fabsf(x))); }
 
 __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity, int* status) {
@@ -379,7 +394,7 @@ struct G2Smem {
     static constexpr int OFF_V = OFF_K + 2 * TILE_KV;
     static constexpr int OFF_BIAS = OFF_V + 2 * TILE_KV;
     static constexpr int OFF_BAR = OFF_BIAS + 8 * 2 * BN * 4;  // a private bias copy per softmax warp
-    static constexpr int NUM_BARS = 16;
+    static constexpr int NUM_BARS = 18;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int BYTES = OFF_MISC + 16;
     static constexpr int ALLOC = BYTES + 1024;
@@ -388,7 +403,28 @@ struct G2Smem {
 
 enum : int {
     G_Q_FULL = 0, G_K_FULL = 1, G_K_EMPTY = 3, G_V_FULL = 5, G_V_EMPTY = 7, G_S_FULL = 9, G_P_FULL = 11,
-    G_O_FULL = 13, G_DRAIN = 14
+    G_O_FULL = 13, G_DRAIN = 14, G_TOK = 15  // G_TOK + h: head h may run its exponentials
+};
+
+// Causal work split.  Query tile qt of a sequence needs KV tiles 0..qt.  With
+// a chunk length C, it is cut into ceil((qt+1)/C) units of at most C KV
+// tiles; units are numbered heaviest query tile first, so the block
+// scheduler hands out long units first.  units_below(x) counts the units of
+// query tiles 0..x-1:  sum_{L=1..x} ceil(L/C) = C*a*(a+1)/2 + r*(a+1), x = a*C + r.
+__device__ __forceinline__ int64_t units_below(int x, int C) {
+    const int64_t a = x / C, r = x % C;
+    return C * a * (a + 1) / 2 + r * (a + 1);
+}
+
+// Scratch of the KV split, per split query tile (qt >= C) of each (sequence,
+// head pair): nch partial results (O / l in fp32 and m + log2 l per row and
+// head) and one arrival counter that the merging CTA resets to zero.
+struct SplitWs {
+    float* o;       // [slots][max_nch][2][BM][HD]
+    float* lse2;    // [slots][max_nch][2][BM]
+    int* cnt;       // [slots]
+    int max_nch;
+    int slots_per_pair;  // n_qt_max - C (query tiles that may be split)
 };
 
 template <int HD>
@@ -397,19 +433,50 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                        const __grid_constant__ CUtensorMap tmV, const int32_t* __restrict__ cu_kept,
                        const int32_t* __restrict__ pos, const int32_t* __restrict__ rank,
                        const float* __restrict__ gls, const float* __restrict__ g, const float* __restrict__ c,
-                       float sm_scale, int Hq, int Hkv, int n_qt_max, uint16_t* __restrict__ out,
-                       float* __restrict__ lse, int* __restrict__ status) {
+                       float sm_scale, int Hq, int Hkv, int n_qt_max, int kv_chunk, SplitWs ws,
+                       uint16_t* __restrict__ out, float* __restrict__ lse, int* __restrict__ status) {
     using L = G2Smem<HD>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
     const int pair = blockIdx.x;            // query heads 2*pair and 2*pair+1
-    const int qt = n_qt_max - 1 - static_cast<int>(blockIdx.y);
     const int b = blockIdx.z;
     const int seq0 = cu_kept[b];
     const int Mb = cu_kept[b + 1] - seq0;
-    if (qt * BM >= Mb) return;
-    const int n_kv = qt + 1;
+    const int n_qt = (Mb + BM - 1) / BM;
+    const int C = min(kv_chunk, max(n_qt, 1));
+    // unit -> (query tile, chunk) in order of decreasing cost (KV tiles), so that
+    // the block scheduler hands out the longest units first
+    int64_t u = blockIdx.y;
+    const int64_t n_units = units_below(n_qt, C);
+    if (u >= n_units) return;
+    int qt = 0, chunk = 0;
+    if (C >= n_qt) {
+        qt = n_qt - 1 - static_cast<int>(u);  // unsplit: query tile qt costs qt + 1
+    } else {
+        // C >= ceil(n_qt / 2): query tiles C..n_qt-1 split into [0, C) and [C, qt+1).
+        // Cost C first: every first chunk; then for v = C, C-1, ..., 1 the unsplit
+        // query tile v-1 and the second chunk of query tile v-1+C (if it exists).
+        const int a = n_qt - C;
+        if (u < a) {
+            qt = n_qt - 1 - static_cast<int>(u);
+        } else {
+            u -= a;
+            for (int v = C; v >= 1; --v) {
+                if (u == 0) { qt = v - 1; break; }
+                --u;
+                if (v - 1 + C <= n_qt - 1) {
+                    if (u == 0) { qt = v - 1 + C; chunk = 1; break; }
+                    --u;
+                }
+            }
+        }
+    }
+    const int nch = (qt + C) / C;  // ceil((qt + 1) / C), 1 or 2
+    const int kv0 = chunk * C;
+    const int kv1 = min(qt + 1, kv0 + C);
+    const int n_kv = kv1 - kv0;  // the chunk holding the diagonal tile is the last one
+    const bool split = nch > 1;
     const int hk = (2 * pair) / (Hq / Hkv);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -432,6 +499,8 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         }
         mbar_init(bar(G_O_FULL), 1);
         mbar_init(bar(G_DRAIN), 1);
+        mbar_init(bar(G_TOK + 0), 128);
+        mbar_init(bar(G_TOK + 1), 128);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -466,8 +535,8 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 mbar_expect_tx(bar(G_K_FULL + s), BN * HD * 2);
 #pragma unroll
                 for (int hf = 0; hf < HD / 64; ++hf)
-                    tma_load_2d(sK0 + s * L::TILE_KV + hf * BN * 128, &tmK, hk * HD + hf * 64, seq0 + j * BN,
-                                bar(G_K_FULL + s));
+                    tma_load_2d(sK0 + s * L::TILE_KV + hf * BN * 128, &tmK, hk * HD + hf * 64,
+                                seq0 + (kv0 + j) * BN, bar(G_K_FULL + s));
                 ++k_issued[s];
                 if (j >= 2 && !mbar_wait(bar(G_V_EMPTY + s), ((j - 2) >> 1) & 1, abort_flag, status,
                                          TG_WHERE_PRODUCER))
@@ -475,8 +544,8 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 mbar_expect_tx(bar(G_V_FULL + s), BN * HD * 2);
 #pragma unroll
                 for (int hf = 0; hf < HD / 64; ++hf)
-                    tma_load_2d(sV0 + s * L::TILE_KV + hf * BN * 128, &tmV, hk * HD + hf * 64, seq0 + j * BN,
-                                bar(G_V_FULL + s));
+                    tma_load_2d(sV0 + s * L::TILE_KV + hf * BN * 128, &tmV, hk * HD + hf * 64,
+                                seq0 + (kv0 + j) * BN, bar(G_V_FULL + s));
                 ++v_issued[s];
             }
             if (*abort_flag) {
@@ -528,6 +597,7 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                      mbar_wait(bar(G_P_FULL + 0), j & 1, abort_flag, status, TG_WHERE_MMA);
                 if (!ok) break;
                 tc_fence_after();
+                TG_TRACE_AT(0, j);  // P0(j) ready, issuing PV0(j)
                 issue_pv(0, j);
                 if (more) {
                     ok = mbar_wait(bar(G_K_FULL + (s ^ 1)), ((j + 1) >> 1) & 1, abort_flag, status, TG_WHERE_MMA);
@@ -539,6 +609,7 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 ok = mbar_wait(bar(G_P_FULL + 1), j & 1, abort_flag, status, TG_WHERE_MMA);
                 if (!ok) break;
                 tc_fence_after();
+                TG_TRACE_AT(1, j);  // P1(j) ready, issuing PV1(j)
                 issue_pv(1, j);
                 mma_commit(bar(G_V_EMPTY + s));
                 if (more) {
@@ -553,6 +624,11 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         }
     } else {
         // ---------------------------------------------------------------- softmax, warps 0-7
+        // In log2 units the logit is  x = alpha_q * (s + b'_j)  with
+        //   alpha_q = sm_scale * log2(e) / tau_q   and   b'_j = softplus(g_h) * gls_j / sm_scale,
+        // so the gate bias is one FADD per score and the temperature one FFMA.
+        // The two heads take turns on the exponentials (token mbarriers), so that
+        // one head's MUFU work overlaps the other head's tensor-core work.
         const int hh = warp >> 2;             // which of the two heads
         const int h = 2 * pair + hh;
         const int r = threadIdx.x & 127;      // query row == TMEM lane
@@ -563,7 +639,7 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         float inv_tau = 1.0f;
         if (valid_row) inv_tau = 1.0f / (1.0f + c[h] * logf(static_cast<float>(pos[qg]) / static_cast<float>(rank[qg])));
         const float alpha = sm_scale * LOG2E * inv_tau;
-        const float gscale = softplus_f(g[h]) * LOG2E;
+        const float bscale = softplus_f(g[h]) / sm_scale;
         const uint32_t lane_addr = static_cast<uint32_t>(lg * 32) << 16;
         const uint32_t tS = tmem + lane_addr + hh * BN;
         const uint32_t tO = tmem + lane_addr + 2 * BN + hh * HD;
@@ -572,41 +648,45 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         bool ok = true;
         for (int j = 0; j < n_kv; ++j) {
             const int s = j & 1;
+            const int jt = kv0 + j;  // KV tile index within the sequence
 #pragma unroll
             for (int e = 0; e < BN / 32; ++e) {
-                const int key_local = j * BN + e * 32 + lane;
-                wbias[s * BN + e * 32 + lane] = key_local < Mb ? gscale * gls[seq0 + key_local] : 0.f;
+                const int key_local = jt * BN + e * 32 + lane;
+                wbias[s * BN + e * 32 + lane] = key_local < Mb ? bscale * gls[seq0 + key_local] : 0.f;
             }
             __syncwarp();
             ok = mbar_wait(bar(G_S_FULL + hh), j & 1, abort_flag, status, TG_WHERE_SOFTMAX);
             if (!ok) break;
             tc_fence_after();
+            if (r == 0) TG_TRACE_AT(2 + 4 * hh, j);  // S_h(j) ready
             float x[BN];
 #pragma unroll
             for (int ch = 0; ch < BN / 32; ++ch) tmem_ld32(tS + ch * 32, x + ch * 32);
             tmem_wait_ld();
-            const float* bias = wbias + s * BN;
+            if (r == 0) TG_TRACE_AT(3 + 4 * hh, j);  // S_h(j) in registers
+            const float4* bias4 = reinterpret_cast<const float4*>(wbias + s * BN);
+            // Stabiliser: the gate bias is never positive (softplus > 0 times
+            // logsigmoid <= 0), so alpha * max_j s_j bounds every logit alpha * (s_j + b'_j)
+            // from above and the max needs one FMNMX per score.
             float mp[G2_ILP];
 #pragma unroll
             for (int i = 0; i < G2_ILP; ++i) mp[i] = -INFINITY;
-            if (j == n_kv - 1) {
-                const int lim = q_local - j * BN;
+            const bool diag = (jt == qt);
+            const int lim = q_local - jt * BN;  // on the diagonal tile, columns > lim lie in the future
+            if (!diag) {
 #pragma unroll
-                for (int cc = 0; cc < BN; ++cc) {
-                    const float v = fmaf(x[cc], alpha, bias[cc] * inv_tau);
-                    x[cc] = cc > lim ? -INFINITY : v;
-                    mp[cc % G2_ILP] = fmaxf(mp[cc % G2_ILP], x[cc]);
-                }
+                for (int cc = 0; cc < BN; ++cc) mp[cc % G2_ILP] = fmaxf(mp[cc % G2_ILP], x[cc]);
             } else {
 #pragma unroll
                 for (int cc = 0; cc < BN; ++cc) {
-                    x[cc] = fmaf(x[cc], alpha, bias[cc] * inv_tau);
+                    x[cc] = cc > lim ? -INFINITY : x[cc];
                     mp[cc % G2_ILP] = fmaxf(mp[cc % G2_ILP], x[cc]);
                 }
             }
-            float mx = mp[0];
+            float my = mp[0];
 #pragma unroll
-            for (int i = 1; i < G2_ILP; ++i) mx = fmaxf(mx, mp[i]);
+            for (int i = 1; i < G2_ILP; ++i) my = fmaxf(my, mp[i]);
+            const float mx = alpha * my;
             float corr = 1.0f;
             bool rescale_o = false;
             if (j == 0 || mx > m_run + RESCALE_THRESHOLD) {
@@ -615,17 +695,34 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 m_run = m_new;
                 rescale_o = j > 0;
             }
+            if (r == 0) TG_TRACE_AT(4 + 4 * hh, j);  // max done
+            // this head's turn on the exponentials: head 0 goes first in every tile
+            if (hh == 1 || j > 0) {
+                ok = mbar_wait(bar(G_TOK + hh), hh == 1 ? (j & 1) : ((j - 1) & 1), abort_flag, status,
+                               TG_WHERE_SOFTMAX);
+                if (!ok) break;
+            }
+            const float neg_m = -m_run;
             float sp[G2_ILP];
 #pragma unroll
             for (int i = 0; i < G2_ILP; ++i) sp[i] = 0.f;
             uint32_t pk[BN / 2];
 #pragma unroll
-            for (int cc = 0; cc < BN; cc += 2) {
-                const float p0 = ex2_approx(x[cc] - m_run), p1 = ex2_approx(x[cc + 1] - m_run);
+            for (int c4 = 0; c4 < BN / 4; ++c4) {
+                const float4 bv = bias4[c4];
+                const int cc = c4 * 4;
+                const float p0 = ex2_approx(fmaf(alpha, x[cc] + bv.x, neg_m));
+                const float p1 = ex2_approx(fmaf(alpha, x[cc + 1] + bv.y, neg_m));
+                const float p2 = ex2_approx(fmaf(alpha, x[cc + 2] + bv.z, neg_m));
+                const float p3 = ex2_approx(fmaf(alpha, x[cc + 3] + bv.w, neg_m));
                 sp[cc % G2_ILP] += p0;
                 sp[(cc + 1) % G2_ILP] += p1;
+                sp[(cc + 2) % G2_ILP] += p2;
+                sp[(cc + 3) % G2_ILP] += p3;
                 pk[cc / 2] = pack_bf16x2(p0, p1);
+                pk[cc / 2 + 1] = pack_bf16x2(p2, p3);
             }
+            mbar_arrive(bar(G_TOK + (hh ^ 1)));  // the other head's turn
             // P_h over the first 64 columns of S_h: this thread's own lane, whose S loads are complete
             tmem_st32u(tS, pk);
             tmem_st32u(tS + 32, pk + 32);
@@ -648,31 +745,101 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar(G_P_FULL + hh));
+            if (r == 0) TG_TRACE_AT(5 + 4 * hh, j);  // P_h(j) stored and signalled
         }
         // ---------------------------------------------------------------- epilogue
         if (ok) ok = mbar_wait(bar(G_O_FULL), 0, abort_flag, status, TG_WHERE_SOFTMAX);
-        if (ok) {
-            tc_fence_after();
-            const float inv_l = 1.0f / l_run;
-            uint16_t* orow = out + (static_cast<size_t>(qg) * Hq + h) * HD;
+        if (ok) tc_fence_after();
+        const float inv_l = 1.0f / l_run;
+        uint16_t* orow = out + (static_cast<size_t>(qg) * Hq + h) * HD;
+        if (!split) {
+            if (ok) {
 #pragma unroll
-            for (int ch = 0; ch < HD / 32; ++ch) {
-                float o[32];
-                tmem_ld32(tO + ch * 32, o);
-                tmem_wait_ld();
-                if (valid_row) {
+                for (int ch = 0; ch < HD / 32; ++ch) {
+                    float o[32];
+                    tmem_ld32(tO + ch * 32, o);
+                    tmem_wait_ld();
+                    if (valid_row) {
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        uint4 v;
-                        v.x = pack_bf16x2(o[q4 * 8 + 0] * inv_l, o[q4 * 8 + 1] * inv_l);
-                        v.y = pack_bf16x2(o[q4 * 8 + 2] * inv_l, o[q4 * 8 + 3] * inv_l);
-                        v.z = pack_bf16x2(o[q4 * 8 + 4] * inv_l, o[q4 * 8 + 5] * inv_l);
-                        v.w = pack_bf16x2(o[q4 * 8 + 6] * inv_l, o[q4 * 8 + 7] * inv_l);
-                        *reinterpret_cast<uint4*>(orow + ch * 32 + q4 * 8) = v;
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            uint4 v;
+                            v.x = pack_bf16x2(o[q4 * 8 + 0] * inv_l, o[q4 * 8 + 1] * inv_l);
+                            v.y = pack_bf16x2(o[q4 * 8 + 2] * inv_l, o[q4 * 8 + 3] * inv_l);
+                            v.z = pack_bf16x2(o[q4 * 8 + 4] * inv_l, o[q4 * 8 + 5] * inv_l);
+                            v.w = pack_bf16x2(o[q4 * 8 + 6] * inv_l, o[q4 * 8 + 7] * inv_l);
+                            *reinterpret_cast<uint4*>(orow + ch * 32 + q4 * 8) = v;
+                        }
                     }
                 }
+                if (valid_row && lse) lse[static_cast<size_t>(qg) * Hq + h] = (m_run + log2f(l_run)) / LOG2E;
             }
-            if (valid_row && lse) lse[static_cast<size_t>(qg) * Hq + h] = (m_run + log2f(l_run)) / LOG2E;
+        } else {
+            // partial result of this KV chunk -> scratch; the last chunk to arrive merges
+            const int64_t slot = (static_cast<int64_t>(b) * (Hq / 2) + pair) * ws.slots_per_pair + (qt - C);
+            float* po = ws.o + (((slot * ws.max_nch + chunk) * 2 + hh) * BM + r) * HD;
+            float* pl = ws.lse2 + ((slot * ws.max_nch + chunk) * 2 + hh) * BM + r;
+            if (ok) {
+#pragma unroll
+                for (int ch = 0; ch < HD / 32; ++ch) {
+                    float o[32];
+                    tmem_ld32(tO + ch * 32, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int q4 = 0; q4 < 8; ++q4)
+                        *reinterpret_cast<float4*>(po + ch * 32 + q4 * 4) =
+                            make_float4(o[q4 * 4] * inv_l, o[q4 * 4 + 1] * inv_l, o[q4 * 4 + 2] * inv_l,
+                                        o[q4 * 4 + 3] * inv_l);
+                }
+                *pl = m_run + log2f(l_run);
+            }
+            __threadfence();
+            asm volatile("bar.sync 1, 256;" ::: "memory");  // all 256 softmax threads, abort or not
+            int* s_last = reinterpret_cast<int*>(smem + L::OFF_MISC + 8);
+            if (threadIdx.x == 0) {
+                const int prev = atomicAdd(ws.cnt + slot, 1);
+                *s_last = (prev == nch - 1) ? 1 : 0;
+            }
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+            if (*s_last && ok) {
+                __threadfence();
+                // merge: out = sum_k 2^(lse_k - L) o_k,  L = log2 sum_k 2^lse_k
+                float mx = -INFINITY;
+                for (int k = 0; k < nch; ++k)
+                    mx = fmaxf(mx, ws.lse2[((slot * ws.max_nch + k) * 2 + hh) * BM + r]);
+                float wsum = 0.f;
+                for (int k = 0; k < nch; ++k)
+                    wsum += ex2_approx(ws.lse2[((slot * ws.max_nch + k) * 2 + hh) * BM + r] - mx);
+                const float inv_w = 1.0f / wsum;
+#pragma unroll 1
+                for (int ch = 0; ch < HD / 8; ++ch) {
+                    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                    for (int k = 0; k < nch; ++k) {
+                        const float wk =
+                            ex2_approx(ws.lse2[((slot * ws.max_nch + k) * 2 + hh) * BM + r] - mx) * inv_w;
+                        const float* pk_o = ws.o + (((slot * ws.max_nch + k) * 2 + hh) * BM + r) * HD + ch * 8;
+                        const float4 a0 = *reinterpret_cast<const float4*>(pk_o);
+                        const float4 a1 = *reinterpret_cast<const float4*>(pk_o + 4);
+                        acc[0] = fmaf(wk, a0.x, acc[0]);
+                        acc[1] = fmaf(wk, a0.y, acc[1]);
+                        acc[2] = fmaf(wk, a0.z, acc[2]);
+                        acc[3] = fmaf(wk, a0.w, acc[3]);
+                        acc[4] = fmaf(wk, a1.x, acc[4]);
+                        acc[5] = fmaf(wk, a1.y, acc[5]);
+                        acc[6] = fmaf(wk, a1.z, acc[6]);
+                        acc[7] = fmaf(wk, a1.w, acc[7]);
+                    }
+                    if (valid_row) {
+                        uint4 v;
+                        v.x = pack_bf16x2(acc[0], acc[1]);
+                        v.y = pack_bf16x2(acc[2], acc[3]);
+                        v.z = pack_bf16x2(acc[4], acc[5]);
+                        v.w = pack_bf16x2(acc[6], acc[7]);
+                        *reinterpret_cast<uint4*>(orow + ch * 8) = v;
+                    }
+                }
+                if (valid_row && lse) lse[static_cast<size_t>(qg) * Hq + h] = (mx + log2f(wsum)) / LOG2E;
+                if (threadIdx.x == 0) ws.cnt[slot] = 0;  // ready for the next call
+            }
         }
     }
 
@@ -687,7 +854,8 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
 template <int HD>
 cudaError_t launch_gqa2(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const int32_t* cu_kept,
                         int B, int max_M, int Hq, int Hkv, const int32_t* pos, const int32_t* rank, const float* gls,
-                        const float* g, const float* c, float sm_scale, uint16_t* out, float* lse, cudaStream_t st) {
+                        const float* g, const float* c, float sm_scale, uint16_t* out, float* lse, void* ws,
+                        size_t ws_bytes, cudaStream_t st) {
     using L = G2Smem<HD>;
     static bool attr_set = false;
     if (!attr_set) {
@@ -697,9 +865,25 @@ cudaError_t launch_gqa2(const CUtensorMap& tq, const CUtensorMap& tk, const CUte
         attr_set = true;
     }
     const int n_qt_max = (max_M + BM - 1) / BM;
-    dim3 grid(Hq / 2, n_qt_max, B);
+    const int C = attention_kv_chunk(B, max_M, Hq, Hkv, ws != nullptr);
+    SplitWs sw{};
+    if (C < n_qt_max) {
+        const size_t need = attention_workspace_bytes(B, max_M, Hq, Hkv, HD);
+        if (ws_bytes < need) return cudaErrorInvalidValue;
+        sw.max_nch = (n_qt_max + C - 1) / C;
+        sw.slots_per_pair = n_qt_max - C;
+        const int64_t slots = static_cast<int64_t>(B) * (Hq / 2) * sw.slots_per_pair;
+        uint8_t* p = static_cast<uint8_t*>(ws);
+        sw.o = reinterpret_cast<float*>(p);
+        p += slots * sw.max_nch * 2 * BM * HD * sizeof(float);
+        sw.lse2 = reinterpret_cast<float*>(p);
+        p += slots * sw.max_nch * 2 * BM * sizeof(float);
+        sw.cnt = reinterpret_cast<int*>(p);
+    }
+    const int64_t units = units_below_host(n_qt_max, C);
+    dim3 grid(Hq / 2, static_cast<unsigned>(units), B);
     gated_attn_gqa2_kernel<HD><<<grid, G2_THREADS, L::ALLOC, st>>>(tq, tk, tv, cu_kept, pos, rank, gls, g, c,
-                                                                   sm_scale, Hq, Hkv, n_qt_max, out, lse,
+                                                                   sm_scale, Hq, Hkv, n_qt_max, C, sw, out, lse,
                                                                    device_status_ptr());
     return cudaGetLastError();
 }
@@ -708,7 +892,7 @@ template <int HD>
 cudaError_t launch_tc(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* cu_kept, int B,
                       int64_t M_total, int max_M, int Hq, int Hkv, const int32_t* pos, const int32_t* rank,
                       const float* gls, const float* g, const float* c, float sm_scale, uint16_t* out, float* lse,
-                      cudaStream_t st) {
+                      void* ws, size_t ws_bytes, cudaStream_t st) {
     using L = AttnSmem<HD>;
     static bool attr_set = false;
     if (!attr_set) {
@@ -726,7 +910,8 @@ cudaError_t launch_tc(const uint16_t* q, const uint16_t* k, const uint16_t* v, c
                              static_cast<uint64_t>(Hkv) * HD * 2, 64, BN))
         return cudaErrorInvalidValue;
     if ((Hq / Hkv) % 2 == 0)
-        return launch_gqa2<HD>(tq, tk, tv, cu_kept, B, max_M, Hq, Hkv, pos, rank, gls, g, c, sm_scale, out, lse, st);
+        return launch_gqa2<HD>(tq, tk, tv, cu_kept, B, max_M, Hq, Hkv, pos, rank, gls, g, c, sm_scale, out, lse, ws,
+                               ws_bytes, st);
     int* status = device_status_ptr();
     const int n_qt_max = (max_M + BM - 1) / BM;
     dim3 grid(Hq, n_qt_max, B);
@@ -737,16 +922,55 @@ cudaError_t launch_tc(const uint16_t* q, const uint16_t* k, const uint16_t* v, c
 
 }  // namespace
 
+#ifdef TG_TRACE
+extern "C" int tg_trace_read_attention(unsigned long long* host) {
+    return cudaMemcpyFromSymbol(host, g_attn_trace, sizeof(g_attn_trace)) == cudaSuccess ? 0 : 1;
+}
+#endif
+
 cudaError_t launch_gated_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* cu_kept,
                                    int B, int64_t M_total, int max_M, int Hq, int Hkv, int d, const int32_t* pos,
                                    const int32_t* rank, const float* gls, const float* g, const float* c,
-                                   float sm_scale, uint16_t* out, float* lse, cudaStream_t st) {
+                                   float sm_scale, uint16_t* out, float* lse, void* ws, size_t ws_bytes,
+                                   cudaStream_t st) {
     if (M_total == 0 || B == 0) return cudaSuccess;
     if (d == 64)
         return launch_tc<64>(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, pos, rank, gls, g, c, sm_scale, out, lse,
-                             st);
-    return launch_tc<128>(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, pos, rank, gls, g, c, sm_scale, out, lse,
-                          st);
+                             ws, ws_bytes, st);
+    return launch_tc<128>(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, pos, rank, gls, g, c, sm_scale, out, lse, ws,
+                          ws_bytes, st);
+}
+
+int64_t units_below_host(int x, int C) {
+    const int64_t a = x / C, r = x % C;
+    return C * a * (a + 1) / 2 + r * (a + 1);
+}
+
+// KV chunk length (in 128-key tiles) of the causal work split.  The longest
+// query tile of a head pair needs n_qt KV tiles; the whole launch needs
+// B * pairs * n_qt (n_qt + 1) / 2 of them.  When the longest is well above a
+// fair share per SM, long query tiles are cut in halves; otherwise (many
+// waves) the heaviest-first order alone balances the SMs.
+int attention_kv_chunk(int B, int max_M, int Hq, int Hkv, bool have_ws) {
+    const int n_qt = (max_M + BM - 1) / BM;
+    if (!have_ws || (Hq / Hkv) % 2 != 0 || n_qt < 4) return n_qt > 0 ? n_qt : 1;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const double total = static_cast<double>(B) * (Hq / 2) * n_qt * (n_qt + 1) / 2.0;
+    const double share = total / sms;
+    if (n_qt <= 1.3 * share) return n_qt;
+    return (n_qt + 1) / 2;
+}
+
+size_t attention_workspace_bytes(int B, int max_M, int Hq, int Hkv, int d) {
+    const int n_qt = (max_M + BM - 1) / BM;
+    if (B <= 0 || n_qt < 4 || (Hq / Hkv) % 2 != 0) return 0;
+    const int C = (n_qt + 1) / 2;  // the shortest chunk length the split uses
+    const int64_t max_nch = (n_qt + C - 1) / C;
+    const int64_t slots = static_cast<int64_t>(B) * (Hq / 2) * (n_qt - C);
+    return static_cast<size_t>(slots * max_nch * 2 * BM * (static_cast<int64_t>(d) + 1) * sizeof(float) +
+                               slots * sizeof(int));
 }
 
 }  // namespace tg

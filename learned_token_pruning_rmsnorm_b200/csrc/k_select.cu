@@ -31,6 +31,21 @@ namespace cg = cooperative_groups;
 namespace tg {
 namespace {
 
+// Optional device trace (builds with -DTG_TRACE only): clock64 stamps of the
+// phases of the first CTA of the first sequence.
+#ifdef TG_TRACE
+__device__ unsigned long long g_sel_trace[32];
+#define SEL_TRACE(point)                                                                         \
+    do {                                                                                         \
+        if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)                              \
+            g_sel_trace[(point)] = static_cast<unsigned long long>(clock64());                   \
+    } while (0)
+#else
+#define SEL_TRACE(point) \
+    do {                 \
+    } while (0)
+#endif
+
 constexpr int SEL_CL = 8;                     // CTAs per sequence (one cluster)
 constexpr int SEL_THREADS = 1024;
 constexpr int SEL_WARPS = SEL_THREADS / 32;
@@ -93,12 +108,14 @@ __device__ __forceinline__ int bit_length(uint64_t v) { return v ? 64 - __clzll(
 // (each CTA must have written it before the cluster barrier that precedes the call).
 __device__ __forceinline__ void cluster_prefix(cg::cluster_group& cl, SelShared& sh, int slot, int rank_self,
                                                int64_t* before, int64_t* total) {
+    int v[SEL_CL];
+#pragma unroll
+    for (int r = 0; r < SEL_CL; ++r) v[r] = cl.map_shared_rank(&sh, r)->xchg[slot];  // all loads in flight
     int64_t b = 0, t = 0;
+#pragma unroll
     for (int r = 0; r < SEL_CL; ++r) {
-        const SelShared* o = cl.map_shared_rank(&sh, r);
-        const int v = o->xchg[slot];
-        if (r < rank_self) b += v;
-        t += v;
+        if (r < rank_self) b += v[r];
+        t += v[r];
     }
     *before = b;
     *total = t;
@@ -117,6 +134,7 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
     cg::cluster_group cl = cg::this_cluster();
 
     const int crank = static_cast<int>(cl.block_rank());
+    SEL_TRACE(0);
     const int b = blockIdx.y;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t s0 = cu_seqlens[b], s1 = cu_seqlens[b + 1];
@@ -169,18 +187,28 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
             atomicMin(&sh.kmin, lmin);
             atomicMax(&sh.kmax, lmax);
         }
+        SEL_TRACE(1);
         cl.sync();  // every CTA's slice min/max is published
-        if (tid == 0) {
+        SEL_TRACE(2);
+        if (warp == 0) {
+            // lane r < SEL_CL reads CTA r's range; a warp reduction combines them
             uint32_t gmin = 0xFFFFFFFFu, gmax = 0u;
-            for (int r = 0; r < SEL_CL; ++r) {
-                const SelShared* o = cl.map_shared_rank(&sh, r);
-                gmin = min(gmin, o->kmin);
-                gmax = max(gmax, o->kmax);
+            if (lane < SEL_CL) {
+                const SelShared* o = cl.map_shared_rank(&sh, lane);
+                gmin = o->kmin;
+                gmax = o->kmax;
             }
-            sh.lo = gmin;
-            sh.width = static_cast<uint64_t>(gmax) - gmin + 1;
-            sh.remaining = static_cast<int>(kk);
-            sh.above = 0;
+#pragma unroll
+            for (int off = 16; off; off >>= 1) {
+                gmin = min(gmin, __shfl_xor_sync(0xffffffffu, gmin, off));
+                gmax = max(gmax, __shfl_xor_sync(0xffffffffu, gmax, off));
+            }
+            if (lane == 0) sh.lo = gmin;
+            if (lane == 0) {
+                sh.width = static_cast<uint64_t>(gmax) - gmin + 1;
+                sh.remaining = static_cast<int>(kk);
+                sh.above = 0;
+            }
         }
         __syncthreads();
         // ------------------------------------------------ bucket passes
@@ -201,15 +229,22 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
             // bucket search from the top: thread tid owns buckets nb-1-2*tid and nb-2-2*tid
             int cnt[2] = {0, 0};
             int local = 0;
+            {
+                // both buckets of every CTA: all 2 x SEL_CL remote loads in flight at once
+                const int bin0 = nb - 1 - 2 * tid, bin1 = bin0 - 1;
+                int v0[SEL_CL], v1[SEL_CL];
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int bin = nb - 1 - (2 * tid + e);
-                if (bin >= 0) {
-                    int v = 0;
-                    for (int r = 0; r < SEL_CL; ++r) v += cl.map_shared_rank(hist, r)[bin];
-                    cnt[e] = v;
-                    local += v;
+                for (int r = 0; r < SEL_CL; ++r) {
+                    const int* hr = cl.map_shared_rank(hist, r);
+                    v0[r] = bin0 >= 0 ? hr[bin0] : 0;
+                    v1[r] = bin1 >= 0 ? hr[bin1] : 0;
                 }
+#pragma unroll
+                for (int r = 0; r < SEL_CL; ++r) {
+                    cnt[0] += v0[r];
+                    cnt[1] += v1[r];
+                }
+                local = cnt[0] + cnt[1];
             }
             int total = 0;
             const int incl = block_inclusive_scan(local, &total, sh);
@@ -235,6 +270,7 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
                 }
             }
             __syncthreads();
+            SEL_TRACE(3 + pass);
             if (sh_bits == 0) break;  // the bucket is a single key value
         }
         thr = sh.lo;
@@ -280,7 +316,9 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
         sh.xchg[0] = tot_kept;
         sh.xchg[1] = tot_eq;
     }
+    SEL_TRACE(8);
     cl.sync();
+    SEL_TRACE(9);
     int64_t kept_before = 0, kept_all = 0, eq_before = 0, eq_all = 0;
     cluster_prefix(cl, sh, 0, crank, &kept_before, &kept_all);
     if (!all_eq_kept) cluster_prefix(cl, sh, 1, crank, &eq_before, &eq_all);
@@ -337,7 +375,9 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
         }
         m += kept_row;
     }
+    SEL_TRACE(10);
     cl.sync();  // no CTA leaves while another may still read its shared memory
+    SEL_TRACE(11);
 }
 
 // Row gather hidden_kept[m, :] = hidden[kept_idx[m], :], one warp per row,
@@ -371,6 +411,12 @@ gather_rows_kernel(const uint4* __restrict__ hidden, const int32_t* __restrict__
 }
 
 }  // namespace
+
+#ifdef TG_TRACE
+extern "C" int tg_trace_read_select(unsigned long long* host) {
+    return cudaMemcpyFromSymbol(host, g_sel_trace, sizeof(g_sel_trace)) == cudaSuccess ? 0 : 1;
+}
+#endif
 
 cudaError_t launch_select_scan(int mode, const float* scores, const uint8_t* keep_in, const int32_t* cu_seqlens,
                                const int32_t* span, const int32_t* k, const int32_t* cu_kept, int B,

@@ -83,7 +83,7 @@ tg_status do_score(const uint16_t* hidden, const int32_t* cu_seqlens, const int3
 tg_status do_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* cu_kept, int B,
                        int64_t M_total, int max_M, int Hq, int Hkv, int d, const int32_t* pos, const int32_t* rank,
                        const float* gls, const float* g, const float* c, float sm_scale, uint16_t* out, float* lse,
-                       cudaStream_t st) {
+                       void* ws, size_t ws_bytes, cudaStream_t st) {
     TG_REQUIRE(B >= 0 && M_total >= 0 && max_M >= 0, "negative size");
     if (tg_status s = check_attn_shape(Hq, Hkv, d)) return s;
     TG_REQUIRE(sm_scale > 0.f, "sm_scale must be positive");
@@ -92,9 +92,14 @@ tg_status do_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
     TG_REQUIRE(q && k && v && cu_kept && pos && rank && gls && g && c && out, "null pointer argument");
     TG_REQUIRE(aligned16(q) && aligned16(k) && aligned16(v) && aligned16(out),
                "q, k, v and out must be 16-byte aligned");
+    if (ws) {
+        TG_REQUIRE((reinterpret_cast<uintptr_t>(ws) & 255u) == 0, "ws must be 256-byte aligned");
+        const size_t need = tg::attention_workspace_bytes(B, max_M, Hq, Hkv, d);
+        TG_REQUIRE(ws_bytes >= need, "ws holds %zu bytes, the causal split needs %zu", ws_bytes, need);
+    }
     if (tg_status s = check_device()) return s;
     return cuda_status(tg::launch_gated_attention(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, d, pos, rank, gls, g,
-                                                  c, sm_scale, out, lse, st),
+                                                  c, sm_scale, out, lse, ws, ws_bytes, st),
                        "tg_gated_attention launch");
 }
 
@@ -186,12 +191,17 @@ tg_status tg_compact(const uint16_t* hidden, const float* scores, const uint8_t*
                        "tg_compact gather launch");
 }
 
+size_t tg_gated_attention_workspace_size(int B, int max_M, int Hq, int Hkv, int d) {
+    if (B <= 0 || max_M <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || (d != 64 && d != 128)) return 0;
+    return tg::attention_workspace_bytes(B, max_M, Hq, Hkv, d);
+}
+
 tg_status tg_gated_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* cu_kept, int B,
                              int64_t M_total, int max_M, int Hq, int Hkv, int d, const int32_t* pos,
                              const int32_t* rank, const float* gls, const float* g, const float* c, float sm_scale,
-                             uint16_t* out, float* lse, tg_stream_t stream) {
-    return do_attention(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, d, pos, rank, gls, g, c, sm_scale, out, lse,
-                        stream);
+                             uint16_t* out, float* lse, void* ws, size_t ws_bytes, tg_stream_t stream) {
+    return do_attention(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, d, pos, rank, gls, g, c, sm_scale, out, lse, ws,
+                        ws_bytes, stream);
 }
 
 tg_status tg_device_status(int32_t* h_word, int clear, tg_stream_t stream) {
@@ -248,7 +258,7 @@ tg_status tg_gated_prefill_layer(const tg_prefill_layer_args* a, tg_stream_t str
         float* lse = a->lse ? a->lse[l] : nullptr;
         if (tg_status s = do_attention(a->q[l], a->kk[l], a->v[l], a->cu_kept, a->B, a->M_total, a->max_M, a->Hq,
                                        a->Hkv, a->d, a->pos, a->rank, a->gls, a->g[l], a->c[l], a->sm_scale,
-                                       a->out[l], lse, st))
+                                       a->out[l], lse, a->attn_ws, a->attn_ws_bytes, st))
             return s;
     }
     return TG_OK;

@@ -56,7 +56,14 @@ cudaError_t launch_gather_rows(const uint16_t* hidden, const int32_t* kept_idx, 
 cudaError_t launch_gated_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* cu_kept,
                                    int B, int64_t M_total, int max_M, int Hq, int Hkv, int d, const int32_t* pos,
                                    const int32_t* rank, const float* gls, const float* g, const float* c,
-                                   float sm_scale, uint16_t* out, float* lse, cudaStream_t st);
+                                   float sm_scale, uint16_t* out, float* lse, void* ws, size_t ws_bytes,
+                                   cudaStream_t st);
+
+// Causal work split of the attention: KV chunk length chosen for a launch,
+// scratch bytes the split needs (0 when it never splits), unit count.
+int attention_kv_chunk(int B, int max_M, int Hq, int Hkv, bool have_ws);
+size_t attention_workspace_bytes(int B, int max_M, int Hq, int Hkv, int d);
+int64_t units_below_host(int x, int C);
 
 cudaError_t launch_selftest_wait(int64_t timeout_ns, cudaStream_t st);
 

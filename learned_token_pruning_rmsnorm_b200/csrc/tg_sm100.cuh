@@ -49,12 +49,18 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
                  : "memory");
 }
 
+// Suspend limit of one try_wait: the waiting thread is parked (it issues no
+// instructions) until the phase completes or this many ns have passed, so
+// waiting warps do not steal issue slots from the warps doing the work.
+constexpr uint32_t TG_WAIT_SUSPEND_NS = 20000;
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
-        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(bar), "r"(parity)
+        : "r"(bar), "r"(parity), "n"(TG_WAIT_SUSPEND_NS)
         : "memory");
     return ok != 0;
 }
@@ -66,15 +72,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
                                           int where, uint64_t timeout_ns = TG_WAIT_TIMEOUT_NS) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
-    for (uint32_t it = 1;; ++it) {
+    for (;;) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63u) == 0) {
-            if (*abort_flag) return false;
-            if (globaltimer() - t0 > timeout_ns) {
-                *abort_flag = 1;
-                if (status) atomicOr(status, TG_DEVICE_TIMEOUT | where);
-                return false;
-            }
+        if (*abort_flag) return false;
+        if (globaltimer() - t0 > timeout_ns) {
+            *abort_flag = 1;
+            if (status) atomicOr(status, TG_DEVICE_TIMEOUT | where);
+            return false;
         }
     }
 }

@@ -77,10 +77,10 @@ def test_invalid_shapes_are_refused_before_launch(lib):
     st = lib.tg_score(P, P, P, 1, 128, 256, P, P, P, 0.0, 512, 1e-6, P, None)
     assert st == _lib.TG_ERR_UNSUPPORTED
     # head_dim 96
-    st = lib.tg_gated_attention(P, P, P, P, 1, 10, 10, 4, 2, 96, P, P, P, P, P, 0.1, P, None, None)
+    st = lib.tg_gated_attention(P, P, P, P, 1, 10, 10, 4, 2, 96, P, P, P, P, P, 0.1, P, None, None, 0, None)
     assert st == _lib.TG_ERR_UNSUPPORTED
     # Hq not a multiple of Hkv
-    st = lib.tg_gated_attention(P, P, P, P, 1, 10, 10, 6, 4, 64, P, P, P, P, P, 0.1, P, None, None)
+    st = lib.tg_gated_attention(P, P, P, P, 1, 10, 10, 6, 4, 64, P, P, P, P, P, 0.1, P, None, None, 0, None)
     assert st == _lib.TG_ERR_INVALID_ARG
     # null pointers
     st = lib.tg_select_topk(None, P, P, P, 1, 10, P, None, None, None, None, None, None)
