@@ -178,9 +178,35 @@ tg_status tg_gated_attention(const uint16_t* q, const uint16_t* k, const uint16_
                              const int32_t* rank, const float* gls, const float* g, const float* c, float sm_scale,
                              uint16_t* out, float* lse, void* ws, size_t ws_bytes, tg_stream_t stream);
 
-/* Bytes of scratch tg_gated_attention may use for these sizes (0 when it
- * never splits, or for unsupported sizes). */
+/* Bytes of scratch tg_gated_attention may use for these sizes on the
+ * current device (0 when it does not split, or for unsupported sizes). */
 size_t tg_gated_attention_workspace_size(int B, int max_M, int Hq, int Hkv, int d);
+
+/*
+ * tg_gated_attention without a caller workspace: no allocation at all.
+ * (The pages describe no such entry point; it exists for callers that
+ * cannot allocate device memory where they run the attention, such as a
+ * serving engine that reserves all of HBM at start-up and only hands out
+ * fixed buffers, or code inside a host runtime that owns the allocator.)
+ * Same arguments, semantics and results as tg_gated_attention; the scratch
+ * of the causal split is a fixed array of TG_NOALLOC_ATTENTION_SCRATCH_BYTES
+ * in the library's device image, which every GPU that loads the library
+ * keeps until the process exits.  Sizes whose split would need more
+ * (tg_gated_attention_workspace_size above the limit) are rejected with
+ * TG_ERR_UNSUPPORTED and nothing is launched.  The call allocates nothing
+ * (no cudaMalloc, cudaFree or allocating library routine); it clears the
+ * array's arrival counters with cudaMemsetAsync on `stream`.  All calls on
+ * a device share the array and it keeps the last call's contents: calls
+ * whose executions overlap on the GPU (other streams, other threads) race on
+ * it and must be serialised by the caller.  The first call on each device
+ * looks up the array's device address (cudaGetSymbolAddress); make that
+ * first call before any stream capture.
+ */
+#define TG_NOALLOC_ATTENTION_SCRATCH_BYTES (32u * 1024u * 1024u)
+tg_status tg_gated_attention_noalloc(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* cu_kept,
+                                     int B, int64_t M_total, int max_M, int Hq, int Hkv, int d, const int32_t* pos,
+                                     const int32_t* rank, const float* gls, const float* g, const float* c,
+                                     float sm_scale, uint16_t* out, float* lse, tg_stream_t stream);
 
 /*
  * The whole gated prefill at one gate layer: tg_score, tg_select_topk,

@@ -22,6 +22,8 @@
 // The bias and temperature therefore cost one extra FFMA per score element
 // on top of plain attention.
 
+#include <mutex>
+
 #include "tg_sm100.cuh"
 
 namespace tg {
@@ -966,11 +968,72 @@ int attention_kv_chunk(int B, int max_M, int Hq, int Hkv, bool have_ws) {
 size_t attention_workspace_bytes(int B, int max_M, int Hq, int Hkv, int d) {
     const int n_qt = (max_M + BM - 1) / BM;
     if (B <= 0 || n_qt < 4 || (Hq / Hkv) % 2 != 0) return 0;
-    const int C = (n_qt + 1) / 2;  // the shortest chunk length the split uses
+    const int C = attention_kv_chunk(B, max_M, Hq, Hkv, true);
+    if (C >= n_qt) return 0;  // this launch never splits
     const int64_t max_nch = (n_qt + C - 1) / C;
     const int64_t slots = static_cast<int64_t>(B) * (Hq / 2) * (n_qt - C);
     return static_cast<size_t>(slots * max_nch * 2 * BM * (static_cast<int64_t>(d) + 1) * sizeof(float) +
                                slots * sizeof(int));
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of tg_gated_attention.
+//
+// Some callers cannot allocate device memory at the point where they run the
+// attention: a serving engine that reserves every byte of HBM at start-up and
+// hands out only fixed buffers, or code running inside a host runtime that
+// owns the allocator and offers no way to ask it for scratch.  For them the
+// causal-split scratch lives in this fixed array, part of the library's
+// device image: every GPU that loads the library holds it until the process
+// exits.  All calls on a device share it, and it keeps the last call's
+// contents, so calls whose executions overlap on the GPU race on it.
+static __device__ __align__(256) unsigned char g_noalloc_attn_scratch[TG_NOALLOC_ATTENTION_SCRATCH_BYTES];
+
+namespace {
+constexpr int kNoAllocMaxDevices = 64;
+void* g_noalloc_scratch_ptr[kNoAllocMaxDevices] = {};
+std::mutex g_noalloc_mu;
+}  // namespace
+
+// Device address of the array on the current device; the first call on each
+// device resolves it (in host code the array's name is only a stand-in).
+cudaError_t noalloc_attention_scratch(void** ptr) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_scratch_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_attn_scratch);
+        if (e != cudaSuccess) return e;
+        g_noalloc_scratch_ptr[dev] = p;
+    }
+    *ptr = g_noalloc_scratch_ptr[dev];
+    return cudaSuccess;
+}
+
+cudaError_t launch_gated_attention_noalloc(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                           const int32_t* cu_kept, int B, int64_t M_total, int max_M, int Hq, int Hkv,
+                                           int d, const int32_t* pos, const int32_t* rank, const float* gls,
+                                           const float* g, const float* c, float sm_scale, uint16_t* out, float* lse,
+                                           cudaStream_t st) {
+    const size_t need = attention_workspace_bytes(B, max_M, Hq, Hkv, d);
+    if (need > TG_NOALLOC_ATTENTION_SCRATCH_BYTES) return cudaErrorInvalidValue;  // the API rejects it first
+    void* ws = nullptr;
+    cudaError_t e = noalloc_attention_scratch(&ws);
+    if (e != cudaSuccess) return e;
+    if (need > 0) {
+        // the arrival counters must start at zero: the last call may have stopped early
+        const int n_qt = (max_M + BM - 1) / BM;
+        const int C = attention_kv_chunk(B, max_M, Hq, Hkv, true);
+        const int64_t slots = static_cast<int64_t>(B) * (Hq / 2) * (n_qt - C);
+        const size_t cnt_bytes = static_cast<size_t>(slots) * sizeof(int);
+        e = cudaMemsetAsync(static_cast<uint8_t*>(ws) + (need - cnt_bytes), 0, cnt_bytes, st);
+        if (e != cudaSuccess) return e;
+    }
+    return launch_gated_attention(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, d, pos, rank, gls, g, c, sm_scale,
+                                  out, lse, need > 0 ? ws : nullptr, need, st);
 }
 
 }  // namespace tg

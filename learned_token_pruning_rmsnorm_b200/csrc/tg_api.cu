@@ -191,6 +191,29 @@ tg_status tg_compact(const uint16_t* hidden, const float* scores, const uint8_t*
                        "tg_compact gather launch");
 }
 
+tg_status tg_gated_attention_noalloc(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* cu_kept,
+                                     int B, int64_t M_total, int max_M, int Hq, int Hkv, int d, const int32_t* pos,
+                                     const int32_t* rank, const float* gls, const float* g, const float* c,
+                                     float sm_scale, uint16_t* out, float* lse, tg_stream_t stream) {
+    TG_REQUIRE(B >= 0 && M_total >= 0 && max_M >= 0, "negative size");
+    if (tg_status s = check_attn_shape(Hq, Hkv, d)) return s;
+    TG_REQUIRE(sm_scale > 0.f, "sm_scale must be positive");
+    if (B == 0 || M_total == 0) return TG_OK;
+    TG_REQUIRE(max_M > 0, "max_M must bound the longest sequence");
+    TG_REQUIRE(q && k && v && cu_kept && pos && rank && gls && g && c && out, "null pointer argument");
+    TG_REQUIRE(aligned16(q) && aligned16(k) && aligned16(v) && aligned16(out),
+               "q, k, v and out must be 16-byte aligned");
+    if (tg_status s = check_device()) return s;
+    const size_t need = tg::attention_workspace_bytes(B, max_M, Hq, Hkv, d);
+    TG_SUPPORT(need <= TG_NOALLOC_ATTENTION_SCRATCH_BYTES,
+               "tg_gated_attention_noalloc: these sizes need %zu bytes of scratch, above the fixed %zu-byte array; "
+               "use tg_gated_attention with a caller workspace",
+               need, static_cast<size_t>(TG_NOALLOC_ATTENTION_SCRATCH_BYTES));
+    return cuda_status(tg::launch_gated_attention_noalloc(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, d, pos, rank,
+                                                          gls, g, c, sm_scale, out, lse, stream),
+                       "tg_gated_attention_noalloc launch");
+}
+
 size_t tg_gated_attention_workspace_size(int B, int max_M, int Hq, int Hkv, int d) {
     if (B <= 0 || max_M <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || (d != 64 && d != 128)) return 0;
     return tg::attention_workspace_bytes(B, max_M, Hq, Hkv, d);

@@ -62,6 +62,11 @@ cudaError_t launch_gated_attention(const uint16_t* q, const uint16_t* k, const u
 // Causal work split of the attention: KV chunk length chosen for a launch,
 // scratch bytes the split needs (0 when it never splits), unit count.
 int attention_kv_chunk(int B, int max_M, int Hq, int Hkv, bool have_ws);
+cudaError_t launch_gated_attention_noalloc(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                           const int32_t* cu_kept, int B, int64_t M_total, int max_M, int Hq, int Hkv,
+                                           int d, const int32_t* pos, const int32_t* rank, const float* gls,
+                                           const float* g, const float* c, float sm_scale, uint16_t* out, float* lse,
+                                           cudaStream_t st);
 size_t attention_workspace_bytes(int B, int max_M, int Hq, int Hkv, int d);
 int64_t units_below_host(int x, int C);
 
