@@ -209,9 +209,14 @@ tg_status tg_gated_attention_noalloc(const uint16_t* q, const uint16_t* k, const
                                      float sm_scale, uint16_t* out, float* lse, tg_stream_t stream);
 
 /*
- * The whole gated prefill at one gate layer: tg_score, tg_select_topk,
- * tg_compact and then n_layers gated-attention layers above the gate, all
- * on one stream with no host synchronisation between them.  Fields mirror
+ * The whole gated prefill at one gate layer: tg_score, tg_select_topk (which
+ * also writes the compaction map), the row gather of tg_compact and n_layers
+ * gated-attention layers above the gate, with no host synchronisation.  The
+ * row gather runs on a library-owned side stream, forked from and joined
+ * back into `stream` by events (one pair per device, created on first use),
+ * so that it overlaps the attention; everything the call enqueues is
+ * ordered before work enqueued on `stream` afterwards, and the call may be
+ * captured into a CUDA graph.  Fields mirror
  * the stage arguments above; per-layer tensors are arrays of n_layers
  * device pointers (the array itself lives in host memory).  The
  * projections that turn hidden_kept into each layer's q/k/v belong to the

@@ -64,13 +64,22 @@ enum : int {
 // Optional device trace (builds with -DTG_TRACE only): clock64 stamps of the
 // pipeline hand-offs of the CTA at blockIdx (0, 0, 0), 64 KV tiles at most.
 #ifdef TG_TRACE
-__device__ unsigned long long g_attn_trace[16 * 64];
+__device__ unsigned long long g_attn_trace[16 * 64];  // points 0..15 x 64 tiles
+__device__ unsigned long long g_attn_cta[4096 * 12];  // per CTA: phase stamps (ns), SM id | n_kv
 #define TG_TRACE_AT(point, j)                                                              \
     do {                                                                                   \
         if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && (j) < 64)             \
             g_attn_trace[(point) * 64 + (j)] = static_cast<unsigned long long>(clock64()); \
     } while (0)
+#define TG_CTA_STAMP(slot)                                                                            \
+    do {                                                                                              \
+        const unsigned idx_ = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);        \
+        if (idx_ < 4096) g_attn_cta[idx_ * 12 + (slot)] = globaltimer();                              \
+    } while (0)
 #else
+#define TG_CTA_STAMP(slot) \
+    do {                   \
+    } while (0)
 #define TG_TRACE_AT(point, j) \
     do {                      \
     } while (0)
@@ -443,6 +452,9 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
 
     const int pair = blockIdx.x;            // query heads 2*pair and 2*pair+1
     const int b = blockIdx.z;
+#ifdef TG_TRACE
+    const unsigned long long trace_t0 = globaltimer();
+#endif
     const int seq0 = cu_kept[b];
     const int Mb = cu_kept[b + 1] - seq0;
     const int n_qt = (Mb + BM - 1) / BM;
@@ -514,6 +526,7 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    if (threadIdx.x == 0) TG_CTA_STAMP(1);
 
     if (warp == 8) {
         // ---------------------------------------------------------------- TMA producer
@@ -584,6 +597,7 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             };
             bool ok = mbar_wait(bar(G_Q_FULL), 0, abort_flag, status, TG_WHERE_MMA) &&
                       mbar_wait(bar(G_K_FULL), 0, abort_flag, status, TG_WHERE_MMA);
+            TG_CTA_STAMP(2);
             if (ok) {
                 tc_fence_after();
                 issue_s(0, 0);
@@ -648,19 +662,32 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         float* wbias = sBias + warp * (2 * BN);
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
+        // gate bias of the keys of tile j, loaded one tile ahead so that its global-memory
+        // latency hides behind the previous tile's softmax
+        float gnext[BN / 32];
+#pragma unroll
+        for (int e = 0; e < BN / 32; ++e) {
+            const int key_local = kv0 * BN + e * 32 + lane;
+            gnext[e] = key_local < Mb ? gls[seq0 + key_local] : 0.f;
+        }
         for (int j = 0; j < n_kv; ++j) {
             const int s = j & 1;
             const int jt = kv0 + j;  // KV tile index within the sequence
 #pragma unroll
-            for (int e = 0; e < BN / 32; ++e) {
-                const int key_local = jt * BN + e * 32 + lane;
-                wbias[s * BN + e * 32 + lane] = key_local < Mb ? bscale * gls[seq0 + key_local] : 0.f;
+            for (int e = 0; e < BN / 32; ++e) wbias[s * BN + e * 32 + lane] = bscale * gnext[e];
+            if (j + 1 < n_kv) {
+#pragma unroll
+                for (int e = 0; e < BN / 32; ++e) {
+                    const int key_local = (jt + 1) * BN + e * 32 + lane;
+                    gnext[e] = key_local < Mb ? gls[seq0 + key_local] : 0.f;
+                }
             }
             __syncwarp();
             ok = mbar_wait(bar(G_S_FULL + hh), j & 1, abort_flag, status, TG_WHERE_SOFTMAX);
             if (!ok) break;
             tc_fence_after();
             if (r == 0) TG_TRACE_AT(2 + 4 * hh, j);  // S_h(j) ready
+            if (threadIdx.x == 0 && j == 0) TG_CTA_STAMP(3);
             float x[BN];
 #pragma unroll
             for (int ch = 0; ch < BN / 32; ++ch) tmem_ld32(tS + ch * 32, x + ch * 32);
@@ -698,12 +725,15 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 rescale_o = j > 0;
             }
             if (r == 0) TG_TRACE_AT(4 + 4 * hh, j);  // max done
+#ifndef TG_ATTN_NO_PINGPONG
             // this head's turn on the exponentials: head 0 goes first in every tile
             if (hh == 1 || j > 0) {
                 ok = mbar_wait(bar(G_TOK + hh), hh == 1 ? (j & 1) : ((j - 1) & 1), abort_flag, status,
                                TG_WHERE_SOFTMAX);
                 if (!ok) break;
             }
+#endif
+            if (r == 0) TG_TRACE_AT(10 + 3 * hh, j);  // token acquired
             const float neg_m = -m_run;
             float sp[G2_ILP];
 #pragma unroll
@@ -724,10 +754,13 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 pk[cc / 2] = pack_bf16x2(p0, p1);
                 pk[cc / 2 + 1] = pack_bf16x2(p2, p3);
             }
-            mbar_arrive(bar(G_TOK + (hh ^ 1)));  // the other head's turn
             // P_h over the first 64 columns of S_h: this thread's own lane, whose S loads are complete
             tmem_st32u(tS, pk);
             tmem_st32u(tS + 32, pk + 32);
+#ifndef TG_ATTN_NO_PINGPONG
+            mbar_arrive(bar(G_TOK + (hh ^ 1)));  // the other head's turn
+#endif
+            if (r == 0) TG_TRACE_AT(11 + 3 * hh, j);  // exponentials done
             float sum = 0.f;
 #pragma unroll
             for (int i = 0; i < G2_ILP; ++i) sum += sp[i];
@@ -745,15 +778,54 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 }
             }
             tmem_wait_st();
+            if (r == 0) TG_TRACE_AT(12 + 3 * hh, j);  // P and O stores complete
             tc_fence_before();
             mbar_arrive(bar(G_P_FULL + hh));
             if (r == 0) TG_TRACE_AT(5 + 4 * hh, j);  // P_h(j) stored and signalled
         }
         // ---------------------------------------------------------------- epilogue
+        if (threadIdx.x == 0) TG_CTA_STAMP(4);
         if (ok) ok = mbar_wait(bar(G_O_FULL), 0, abort_flag, status, TG_WHERE_SOFTMAX);
         if (ok) tc_fence_after();
+        if (threadIdx.x == 0) TG_CTA_STAMP(5);
         const float inv_l = 1.0f / l_run;
-        uint16_t* orow = out + (static_cast<size_t>(qg) * Hq + h) * HD;
+        // Output rows leave through shared memory: thread r stages its row of this head
+        // in the K buffers (free once every MMA has completed), 16-byte chunks XOR-
+        // swizzled by the row so that the staging is conflict-free, and each warp then
+        // writes whole rows with coalesced stores (rows past the sequence end are skipped).
+        constexpr int CH = HD * 2 / 16;  // 16-byte chunks per bf16 row
+        uint8_t* stage = smem + L::OFF_K + hh * (BM * HD * 2);
+        auto stage_row = [&](const float* o32, int ch32, float w) {  // 32 columns starting at ch32 * 32
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) {
+                const int cidx = ch32 * 4 + k4;
+                uint4 v;
+                v.x = pack_bf16x2(o32[k4 * 8 + 0] * w, o32[k4 * 8 + 1] * w);
+                v.y = pack_bf16x2(o32[k4 * 8 + 2] * w, o32[k4 * 8 + 3] * w);
+                v.z = pack_bf16x2(o32[k4 * 8 + 4] * w, o32[k4 * 8 + 5] * w);
+                v.w = pack_bf16x2(o32[k4 * 8 + 6] * w, o32[k4 * 8 + 7] * w);
+                *reinterpret_cast<uint4*>(stage + r * (HD * 2) + ((cidx ^ (r & (CH - 1))) << 4)) = v;
+            }
+        };
+        auto write_rows = [&]() {  // the 4 warps of this head write its 128 staged rows
+            asm volatile("bar.sync %0, 128;" ::"r"(2 + hh) : "memory");
+#pragma unroll 4
+            for (int i = 0; i < 32; ++i) {
+                const int rr = lg * 32 + i;
+                if (qt * BM + rr >= Mb) break;
+                const uint8_t* src = stage + rr * (HD * 2);
+                uint16_t* dst = out + (static_cast<size_t>(seq0 + qt * BM + rr) * Hq + h) * HD;
+                if (HD == 128) {
+                    const uint2 v = *reinterpret_cast<const uint2*>(src + (((lane >> 1) ^ (rr & (CH - 1))) << 4) +
+                                                                    (lane & 1) * 8);
+                    *reinterpret_cast<uint2*>(dst + lane * 4) = v;
+                } else {
+                    const uint32_t v = *reinterpret_cast<const uint32_t*>(
+                        src + (((lane >> 2) ^ (rr & (CH - 1))) << 4) + (lane & 3) * 4);
+                    *reinterpret_cast<uint32_t*>(dst + lane * 2) = v;
+                }
+            }
+        };
         if (!split) {
             if (ok) {
 #pragma unroll
@@ -761,25 +833,19 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     float o[32];
                     tmem_ld32(tO + ch * 32, o);
                     tmem_wait_ld();
-                    if (valid_row) {
-#pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4) {
-                            uint4 v;
-                            v.x = pack_bf16x2(o[q4 * 8 + 0] * inv_l, o[q4 * 8 + 1] * inv_l);
-                            v.y = pack_bf16x2(o[q4 * 8 + 2] * inv_l, o[q4 * 8 + 3] * inv_l);
-                            v.z = pack_bf16x2(o[q4 * 8 + 4] * inv_l, o[q4 * 8 + 5] * inv_l);
-                            v.w = pack_bf16x2(o[q4 * 8 + 6] * inv_l, o[q4 * 8 + 7] * inv_l);
-                            *reinterpret_cast<uint4*>(orow + ch * 32 + q4 * 8) = v;
-                        }
-                    }
+                    stage_row(o, ch, inv_l);
                 }
                 if (valid_row && lse) lse[static_cast<size_t>(qg) * Hq + h] = (m_run + log2f(l_run)) / LOG2E;
             }
+            write_rows();
         } else {
-            // partial result of this KV chunk -> scratch; the last chunk to arrive merges
+            // partial result of this KV chunk -> scratch, stored [column][row] so that a
+            // warp's 32 rows of one column are one 128-byte write; the last chunk to
+            // arrive merges (a split query tile has exactly two chunks: chunk ^ 1)
             const int64_t slot = (static_cast<int64_t>(b) * (Hq / 2) + pair) * ws.slots_per_pair + (qt - C);
-            float* po = ws.o + (((slot * ws.max_nch + chunk) * 2 + hh) * BM + r) * HD;
+            float* po = ws.o + ((slot * ws.max_nch + chunk) * 2 + hh) * (BM * HD) + r;
             float* pl = ws.lse2 + ((slot * ws.max_nch + chunk) * 2 + hh) * BM + r;
+            const float my_lse = m_run + log2f(l_run);
             if (ok) {
 #pragma unroll
                 for (int ch = 0; ch < HD / 32; ++ch) {
@@ -787,62 +853,53 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     tmem_ld32(tO + ch * 32, o);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int q4 = 0; q4 < 8; ++q4)
-                        *reinterpret_cast<float4*>(po + ch * 32 + q4 * 4) =
-                            make_float4(o[q4 * 4] * inv_l, o[q4 * 4 + 1] * inv_l, o[q4 * 4 + 2] * inv_l,
-                                        o[q4 * 4 + 3] * inv_l);
+                    for (int e = 0; e < 32; ++e) po[(ch * 32 + e) * BM] = o[e] * inv_l;
                 }
-                *pl = m_run + log2f(l_run);
+                *pl = my_lse;
             }
-            __threadfence();
+            if (threadIdx.x == 0) TG_CTA_STAMP(8);
+            // every softmax thread's partial is written before the barrier; one thread then
+            // publishes them with a release fence and the arrival, and the last CTA to
+            // arrive acquires the other chunk's partial the same way
             asm volatile("bar.sync 1, 256;" ::: "memory");  // all 256 softmax threads, abort or not
+            if (threadIdx.x == 0) TG_CTA_STAMP(9);
             int* s_last = reinterpret_cast<int*>(smem + L::OFF_MISC + 8);
             if (threadIdx.x == 0) {
+                asm volatile("fence.acq_rel.gpu;" ::: "memory");
                 const int prev = atomicAdd(ws.cnt + slot, 1);
+                asm volatile("fence.acq_rel.gpu;" ::: "memory");
                 *s_last = (prev == nch - 1) ? 1 : 0;
             }
             asm volatile("bar.sync 1, 256;" ::: "memory");
-            if (*s_last && ok) {
-                __threadfence();
-                // merge: out = sum_k 2^(lse_k - L) o_k,  L = log2 sum_k 2^lse_k
-                float mx = -INFINITY;
-                for (int k = 0; k < nch; ++k)
-                    mx = fmaxf(mx, ws.lse2[((slot * ws.max_nch + k) * 2 + hh) * BM + r]);
-                float wsum = 0.f;
-                for (int k = 0; k < nch; ++k)
-                    wsum += ex2_approx(ws.lse2[((slot * ws.max_nch + k) * 2 + hh) * BM + r] - mx);
-                const float inv_w = 1.0f / wsum;
-#pragma unroll 1
-                for (int ch = 0; ch < HD / 8; ++ch) {
-                    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                    for (int k = 0; k < nch; ++k) {
-                        const float wk =
-                            ex2_approx(ws.lse2[((slot * ws.max_nch + k) * 2 + hh) * BM + r] - mx) * inv_w;
-                        const float* pk_o = ws.o + (((slot * ws.max_nch + k) * 2 + hh) * BM + r) * HD + ch * 8;
-                        const float4 a0 = *reinterpret_cast<const float4*>(pk_o);
-                        const float4 a1 = *reinterpret_cast<const float4*>(pk_o + 4);
-                        acc[0] = fmaf(wk, a0.x, acc[0]);
-                        acc[1] = fmaf(wk, a0.y, acc[1]);
-                        acc[2] = fmaf(wk, a0.z, acc[2]);
-                        acc[3] = fmaf(wk, a0.w, acc[3]);
-                        acc[4] = fmaf(wk, a1.x, acc[4]);
-                        acc[5] = fmaf(wk, a1.y, acc[5]);
-                        acc[6] = fmaf(wk, a1.z, acc[6]);
-                        acc[7] = fmaf(wk, a1.w, acc[7]);
+            if (threadIdx.x == 0) TG_CTA_STAMP(10);
+            if (*s_last) {
+                const float* oo = ws.o + ((slot * ws.max_nch + (chunk ^ 1)) * 2 + hh) * (BM * HD) + r;
+                const float other_lse = ws.lse2[((slot * ws.max_nch + (chunk ^ 1)) * 2 + hh) * BM + r];
+                const float mx = fmaxf(my_lse, other_lse);
+                const float e_me = ex2_approx(my_lse - mx), e_ot = ex2_approx(other_lse - mx);
+                const float inv_w = 1.0f / (e_me + e_ot);
+                const float w_me = e_me * inv_w, w_ot = e_ot * inv_w;
+                if (ok) {
+#pragma unroll
+                    for (int ch = 0; ch < HD / 32; ++ch) {
+                        float ot[32];
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) ot[e] = oo[(ch * 32 + e) * BM];
+                        float o[32];
+                        tmem_ld32(tO + ch * 32, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) o[e] = fmaf(w_me * inv_l, o[e], w_ot * ot[e]);  // own O unnormalised
+                        stage_row(o, ch, 1.0f);
                     }
-                    if (valid_row) {
-                        uint4 v;
-                        v.x = pack_bf16x2(acc[0], acc[1]);
-                        v.y = pack_bf16x2(acc[2], acc[3]);
-                        v.z = pack_bf16x2(acc[4], acc[5]);
-                        v.w = pack_bf16x2(acc[6], acc[7]);
-                        *reinterpret_cast<uint4*>(orow + ch * 8) = v;
-                    }
+                    if (valid_row && lse) lse[static_cast<size_t>(qg) * Hq + h] = (mx + log2f(e_me + e_ot)) / LOG2E;
                 }
-                if (valid_row && lse) lse[static_cast<size_t>(qg) * Hq + h] = (mx + log2f(wsum)) / LOG2E;
+                write_rows();
                 if (threadIdx.x == 0) ws.cnt[slot] = 0;  // ready for the next call
             }
+            if (threadIdx.x == 0) TG_CTA_STAMP(11);
         }
+        if (!split && threadIdx.x == 0) TG_CTA_STAMP(8);
     }
 
     tc_fence_before();
@@ -851,6 +908,19 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         tc_fence_after();
         tmem_dealloc(tmem, L::TMEM_COLS);
     }
+#ifdef TG_TRACE
+    if (threadIdx.x == 0) {
+        const unsigned idx = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+        if (idx < 4096) {
+            unsigned smid;
+            asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+            g_attn_cta[idx * 12 + 0] = trace_t0;
+            g_attn_cta[idx * 12 + 6] = globaltimer();
+            g_attn_cta[idx * 12 + 7] = smid | (static_cast<unsigned long long>(n_kv) << 32) |
+                                      (static_cast<unsigned long long>(split) << 40);
+        }
+    }
+#endif
 }
 
 template <int HD>
@@ -927,6 +997,9 @@ cudaError_t launch_tc(const uint16_t* q, const uint16_t* k, const uint16_t* v, c
 #ifdef TG_TRACE
 extern "C" int tg_trace_read_attention(unsigned long long* host) {
     return cudaMemcpyFromSymbol(host, g_attn_trace, sizeof(g_attn_trace)) == cudaSuccess ? 0 : 1;
+}
+extern "C" int tg_trace_read_attention_ctas(unsigned long long* host) {
+    return cudaMemcpyFromSymbol(host, g_attn_cta, sizeof(g_attn_cta)) == cudaSuccess ? 0 : 1;
 }
 #endif
 

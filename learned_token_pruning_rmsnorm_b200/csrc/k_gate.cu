@@ -41,27 +41,22 @@ __global__ void gate_prepare_kernel(const uint16_t* __restrict__ gamma, const ui
 constexpr int KB = 64;                // channels per pipeline stage (one 128-byte swizzle row)
 constexpr int TILE_A = 128 * KB * 2;  // one 128-row slice: 16 KB
 
-// Two TMA rings: the rows (from HBM, long latency) get STAGES_A stages so that
-// 128 KB per SM are in flight; the gate-weight slices (L2-resident) get two.
 template <int NACC>
 struct ScoreCfg {
-    static constexpr int STAGES_A = 8 / NACC;
-    static constexpr int STAGES_B = 2;
+    static constexpr int STAGES = NACC == 2 ? 3 : 4;
     static constexpr int EPI_WARPS = 4 * NACC;
     static constexpr int THREADS = 64 + 32 * EPI_WARPS;
     static constexpr uint32_t TMEM_COLS = NACC == 2 ? 512 : 256;
     static constexpr int ROWS = 128 * NACC;
-    static constexpr int A_STAGE_BYTES = NACC * TILE_A;
-    static constexpr int A_BYTES = STAGES_A * A_STAGE_BYTES;
 };
 
-__host__ __device__ constexpr int score_b_stage_bytes(int I) { return I * 128; }
-
-// A ring, B ring (sized for I <= 256), b1, w2, 24 barriers, tmem slot + abort flag
 template <int NACC>
-__host__ __device__ constexpr int score_smem_bytes() {
-    return ScoreCfg<NACC>::A_BYTES + ScoreCfg<NACC>::STAGES_B * score_b_stage_bytes(256) + 2 * 256 * 4 + 24 * 8 +
-           16 + 1024;
+__host__ __device__ constexpr int score_stage_bytes(int I) { return NACC * TILE_A + I * 128; }
+
+// stages x (NACC row slices + one Wg slice of I rows), b1, w2, 16 barriers, tmem slot + abort flag
+template <int NACC>
+__host__ __device__ constexpr int score_smem_bytes(int I) {
+    return ScoreCfg<NACC>::STAGES * score_stage_bytes<NACC>(I) + 2 * 256 * 4 + 16 * 8 + 16 + 1024;
 }
 
 __device__ __forceinline__ float silu_f(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
@@ -91,23 +86,20 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                 const float* __restrict__ b1, const float* __restrict__ w2, float b2, float eps,
                 float* __restrict__ scores, int* __restrict__ status) {
     using C = ScoreCfg<NACC>;
-    constexpr int SA = C::STAGES_A, SB = C::STAGES_B;
+    constexpr int STAGES = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int b_stage_bytes = score_b_stage_bytes(I);
-    const int off_b = C::A_BYTES;
-    const int off_misc = C::A_BYTES + SB * score_b_stage_bytes(256);
-    float* s_b1 = reinterpret_cast<float*>(smem + off_misc);
+    const int stage_bytes = score_stage_bytes<NACC>(I);
+    float* s_b1 = reinterpret_cast<float*>(smem + STAGES * stage_bytes);
     float* s_w2 = s_b1 + 256;
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t bar0 = sbase + off_misc + 2 * 256 * 4;
-    // barriers: fullA[SA], emptyA[SA], fullB[SB], emptyB[SB], acc_full, acc_empty, drain
-    auto full_a = [&](int s) { return bar0 + 8u * s; };
-    auto empty_a = [&](int s) { return bar0 + 8u * (SA + s); };
-    auto full_b = [&](int s) { return bar0 + 8u * (2 * SA + s); };
-    auto empty_b = [&](int s) { return bar0 + 8u * (2 * SA + SB + s); };
-    const uint32_t acc_full = bar0 + 8u * (2 * SA + 2 * SB), acc_empty = acc_full + 8u, drain = acc_full + 16u;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + off_misc + 2 * 256 * 4 + 24 * 8);
+    const uint32_t bar0 = sbase + STAGES * stage_bytes + 2 * 256 * 4;
+    // barriers: full[STAGES], empty[STAGES], acc_full, acc_empty, drain
+    auto full = [&](int s) { return bar0 + 8u * s; };
+    auto empty = [&](int s) { return bar0 + 8u * (STAGES + s); };
+    const uint32_t acc_full = bar0 + 8u * (2 * STAGES), acc_empty = bar0 + 8u * (2 * STAGES + 1);
+    const uint32_t drain = bar0 + 8u * (2 * STAGES + 2);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + STAGES * stage_bytes + 2 * 256 * 4 + 16 * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -118,13 +110,9 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
         s_w2[j] = w2[j];
     }
     if (threadIdx.x == 0) {
-        for (int s = 0; s < SA; ++s) {
-            mbar_init(full_a(s), 1);
-            mbar_init(empty_a(s), 1 + C::EPI_WARPS);
-        }
-        for (int s = 0; s < SB; ++s) {
-            mbar_init(full_b(s), 1);
-            mbar_init(empty_b(s), 1);
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full(s), 1);
+            mbar_init(empty(s), 1 + C::EPI_WARPS);
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, C::EPI_WARPS);
@@ -147,40 +135,32 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
             prefetch_tmap(&tmX);
             prefetch_tmap(&tmW);
             int64_t it = 0;
-            int issued_a[SA] = {}, issued_b[SB] = {};
+            int issued[STAGES] = {};
             bool ok = true;
             for (int64_t t = blockIdx.x; ok; t += gridDim.x) {
                 int64_t row0, row_end;
                 if (!map_tile(t, C::ROWS, cu_seqlens, span, B, &row0, &row_end)) break;
                 for (int kb = 0; kb < nkb; ++kb, ++it) {
-                    const int sa = static_cast<int>(it % SA), ua = static_cast<int>(it / SA);
-                    const int sb = static_cast<int>(it % SB), ub = static_cast<int>(it / SB);
-                    if (ua > 0 && !mbar_wait(empty_a(sa), (ua - 1) & 1, abort_flag, status, TG_WHERE_PRODUCER)) {
+                    const int s = static_cast<int>(it % STAGES);
+                    const int use = static_cast<int>(it / STAGES);
+                    if (use > 0 && !mbar_wait(empty(s), (use - 1) & 1, abort_flag, status, TG_WHERE_PRODUCER)) {
                         ok = false;
                         break;
                     }
-                    mbar_expect_tx(full_a(sa), C::A_STAGE_BYTES);
+                    const uint32_t st = sbase + s * stage_bytes;
+                    mbar_expect_tx(full(s), stage_bytes);
 #pragma unroll
                     for (int a = 0; a < NACC; ++a)
-                        tma_load_2d(sbase + sa * C::A_STAGE_BYTES + a * TILE_A, &tmX, kb * KB,
-                                    static_cast<int32_t>(row0 + a * 128), full_a(sa));
-                    ++issued_a[sa];
-                    if (ub > 0 && !mbar_wait(empty_b(sb), (ub - 1) & 1, abort_flag, status, TG_WHERE_PRODUCER)) {
-                        ok = false;
-                        break;
-                    }
-                    mbar_expect_tx(full_b(sb), b_stage_bytes);
-                    tma_load_2d(sbase + off_b + sb * b_stage_bytes, &tmW, kb * KB, 0, full_b(sb));
-                    ++issued_b[sb];
+                        tma_load_2d(st + a * TILE_A, &tmX, kb * KB, static_cast<int32_t>(row0 + a * 128), full(s));
+                    tma_load_2d(st + NACC * TILE_A, &tmW, kb * KB, 0, full(s));
+                    ++issued[s];
                 }
             }
             if (*abort_flag) {
                 // let every copy this thread started land before the CTA exits
                 volatile int never = 0;
-                for (int s = 0; s < SA; ++s)
-                    if (issued_a[s]) mbar_wait(full_a(s), (issued_a[s] - 1) & 1, &never, status, TG_WHERE_DRAIN);
-                for (int s = 0; s < SB; ++s)
-                    if (issued_b[s]) mbar_wait(full_b(s), (issued_b[s] - 1) & 1, &never, status, TG_WHERE_DRAIN);
+                for (int s = 0; s < STAGES; ++s)
+                    if (issued[s]) mbar_wait(full(s), (issued[s] - 1) & 1, &never, status, TG_WHERE_DRAIN);
             }
         }
     } else if (warp == 1) {
@@ -196,26 +176,23 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                 if (tcount > 0 && !mbar_wait(acc_empty, (tcount - 1) & 1, abort_flag, status, TG_WHERE_MMA)) break;
                 tc_fence_after();
                 for (int kb = 0; kb < nkb; ++kb, ++it) {
-                    const int sa = static_cast<int>(it % SA), ua = static_cast<int>(it / SA);
-                    const int sb = static_cast<int>(it % SB), ub = static_cast<int>(it / SB);
-                    if (!mbar_wait(full_a(sa), ua & 1, abort_flag, status, TG_WHERE_MMA) ||
-                        !mbar_wait(full_b(sb), ub & 1, abort_flag, status, TG_WHERE_MMA)) {
+                    const int s = static_cast<int>(it % STAGES);
+                    const int use = static_cast<int>(it / STAGES);
+                    if (!mbar_wait(full(s), use & 1, abort_flag, status, TG_WHERE_MMA)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sta = sbase + sa * C::A_STAGE_BYTES;
-                    const uint32_t stb = sbase + off_b + sb * b_stage_bytes;
+                    const uint32_t st = sbase + s * stage_bytes;
 #pragma unroll
                     for (int kk = 0; kk < KB / 16; ++kk) {
-                        const uint64_t bdesc = smem_desc_sw128(stb + kk * 32, 16, 1024);
+                        const uint64_t bdesc = smem_desc_sw128(st + NACC * TILE_A + kk * 32, 16, 1024);
 #pragma unroll
                         for (int a = 0; a < NACC; ++a)
-                            mma_bf16_ss(tmem + a * 256, smem_desc_sw128(sta + a * TILE_A + kk * 32, 16, 1024), bdesc,
+                            mma_bf16_ss(tmem + a * 256, smem_desc_sw128(st + a * TILE_A + kk * 32, 16, 1024), bdesc,
                                         idesc, (kb | kk) != 0 ? 1u : 0u);
                     }
-                    mma_commit(empty_a(sa));
-                    mma_commit(empty_b(sb));
+                    mma_commit(empty(s));
                 }
                 if (ok) mma_commit(acc_full);
             }
@@ -239,8 +216,9 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
             if (!map_tile(t, C::ROWS, cu_seqlens, span, B, &row0, &row_end)) break;
             float ss = 0.f;
             for (int kb = 0; kb < nkb; ++kb, ++it) {
-                const int sa = static_cast<int>(it % SA), ua = static_cast<int>(it / SA);
-                if (!mbar_wait(full_a(sa), ua & 1, abort_flag, status, TG_WHERE_SOFTMAX)) {
+                const int s = static_cast<int>(it % STAGES);
+                const int use = static_cast<int>(it / STAGES);
+                if (!mbar_wait(full(s), use & 1, abort_flag, status, TG_WHERE_SOFTMAX)) {
                     ok = false;
                     break;
                 }
@@ -248,7 +226,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                 // (r & 7): the 128-byte swizzle then spreads a warp's 32 rows over all
                 // banks (4 wavefronts per 512-byte access, the minimum); chunk order is
                 // irrelevant for a sum of squares.
-                const uint8_t* rowp = smem + sa * C::A_STAGE_BYTES + a * TILE_A + r * 128;
+                const uint8_t* rowp = smem + s * stage_bytes + a * TILE_A + r * 128;
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch) {
                     const uint4 v = *reinterpret_cast<const uint4*>(rowp + ((ch ^ (r & 7)) << 4));
@@ -261,7 +239,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                     }
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(empty_a(sa));
+                if (lane == 0) mbar_arrive(empty(s));
             }
             if (!ok) break;
             if (!mbar_wait(acc_full, tcount & 1, abort_flag, status, TG_WHERE_SOFTMAX)) break;
@@ -299,7 +277,7 @@ cudaError_t launch_score_tc(const uint16_t* hidden, const int32_t* cu_seqlens, c
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<NACC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             score_smem_bytes<NACC>());
+                                             score_smem_bytes<NACC>(256));
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
@@ -311,9 +289,9 @@ cudaError_t launch_score_tc(const uint16_t* hidden, const int32_t* cu_seqlens, c
         return cudaErrorInvalidValue;
     const int64_t tiles_bound = (T + C::ROWS - 1) / C::ROWS + B;
     const int grid = static_cast<int>(tiles_bound < sms ? tiles_bound : sms);
-    score_tc_kernel<NACC><<<grid, C::THREADS, score_smem_bytes<NACC>(), st>>>(tx, tw, cu_seqlens, span, B, D, I, b1,
-                                                                             w2, b2, eps, scores,
-                                                                             device_status_ptr());
+    score_tc_kernel<NACC><<<grid, C::THREADS, score_smem_bytes<NACC>(I), st>>>(tx, tw, cu_seqlens, span, B, D, I, b1,
+                                                                              w2, b2, eps, scores,
+                                                                              device_status_ptr());
     return cudaGetLastError();
 }
 

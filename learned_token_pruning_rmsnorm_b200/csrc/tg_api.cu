@@ -4,6 +4,7 @@
 
 #include <cstdarg>
 #include <cstdio>
+#include <mutex>
 #include <string>
 
 #include "tg_internal.cuh"
@@ -42,6 +43,32 @@ tg_status check_device() {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Per device: a second stream and two events with which tg_gated_prefill_layer
+// runs the row gather beside the attention (both only need the compaction
+// map).  Created on first use; the mutex keeps one fork/join pair at a time.
+struct SideStream {
+    cudaStream_t stream = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+constexpr int kMaxDev = 64;
+SideStream g_side[kMaxDev];
+std::mutex g_side_mu;
+
+cudaError_t side_stream(SideStream** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+    SideStream& ss = g_side[dev];
+    if (!ss.stream) {
+        if ((e = cudaStreamCreateWithFlags(&ss.stream, cudaStreamNonBlocking)) != cudaSuccess) return e;
+        if ((e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming)) != cudaSuccess) return e;
+        if ((e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming)) != cudaSuccess) return e;
+    }
+    *out = &ss;
+    return cudaSuccess;
+}
 
 #define TG_REQUIRE(cond, ...)                                   \
     do {                                                        \
@@ -271,20 +298,36 @@ tg_status tg_gated_prefill_layer(const tg_prefill_layer_args* a, tg_stream_t str
                                   "select launch"))
         return s;
     if (a->M_total == 0) return TG_OK;  // every token pruned: no kept rows, no attention
+    // the row gather (HBM-bound) runs on a side stream beside the attention
+    // layers (tensor-bound); both read only the compaction map
+    std::unique_lock<std::mutex> lk(g_side_mu);
+    SideStream* side = nullptr;
+    const bool fork = a->hidden_kept && a->n_layers > 0;
+    if (fork) {
+        if (tg_status s = cuda_status(side_stream(&side), "side stream")) return s;
+        if (tg_status s = cuda_status(cudaEventRecord(side->fork, st), "fork record")) return s;
+        if (tg_status s = cuda_status(cudaStreamWaitEvent(side->stream, side->fork, 0), "fork wait")) return s;
+    }
     if (a->hidden_kept) {
         if (tg_status s = cuda_status(tg::launch_gather_rows(a->hidden, a->kept_idx, a->M_total, a->T, a->D,
-                                                             a->hidden_kept, st),
+                                                             a->hidden_kept, fork ? side->stream : st),
                                       "gather launch"))
             return s;
     }
-    for (int l = 0; l < a->n_layers; ++l) {
+    tg_status result = TG_OK;
+    for (int l = 0; l < a->n_layers && result == TG_OK; ++l) {
         float* lse = a->lse ? a->lse[l] : nullptr;
-        if (tg_status s = do_attention(a->q[l], a->kk[l], a->v[l], a->cu_kept, a->B, a->M_total, a->max_M, a->Hq,
-                                       a->Hkv, a->d, a->pos, a->rank, a->gls, a->g[l], a->c[l], a->sm_scale,
-                                       a->out[l], lse, a->attn_ws, a->attn_ws_bytes, st))
-            return s;
+        result = do_attention(a->q[l], a->kk[l], a->v[l], a->cu_kept, a->B, a->M_total, a->max_M, a->Hq, a->Hkv,
+                              a->d, a->pos, a->rank, a->gls, a->g[l], a->c[l], a->sm_scale, a->out[l], lse,
+                              a->attn_ws, a->attn_ws_bytes, st);
     }
-    return TG_OK;
+    if (fork) {
+        // join: work queued on `stream` after this call also waits for the gather
+        tg_status s = cuda_status(cudaEventRecord(side->join, side->stream), "join record");
+        if (s == TG_OK) s = cuda_status(cudaStreamWaitEvent(st, side->join, 0), "join wait");
+        if (result == TG_OK) result = s;
+    }
+    return result;
 }
 
 }  // extern "C"
