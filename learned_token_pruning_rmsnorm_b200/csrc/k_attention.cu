@@ -929,13 +929,9 @@ cudaError_t launch_gqa2(const CUtensorMap& tq, const CUtensorMap& tk, const CUte
                         const float* g, const float* c, float sm_scale, uint16_t* out, float* lse, void* ws,
                         size_t ws_bytes, cudaStream_t st) {
     using L = G2Smem<HD>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(gated_attn_gqa2_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             L::ALLOC);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static std::atomic<uint64_t> attr_set{0};
+    if (cudaError_t e = ensure_smem_limit(gated_attn_gqa2_kernel<HD>, L::ALLOC, attr_set); e != cudaSuccess)
+        return e;
     const int n_qt_max = (max_M + BM - 1) / BM;
     const int C = attention_kv_chunk(B, max_M, Hq, Hkv, ws != nullptr);
     SplitWs sw{};
@@ -966,13 +962,9 @@ cudaError_t launch_tc(const uint16_t* q, const uint16_t* k, const uint16_t* v, c
                       const float* gls, const float* g, const float* c, float sm_scale, uint16_t* out, float* lse,
                       void* ws, size_t ws_bytes, cudaStream_t st) {
     using L = AttnSmem<HD>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(gated_attn_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             L::ALLOC);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static std::atomic<uint64_t> attr_set{0};
+    if (cudaError_t e = ensure_smem_limit(gated_attn_tc_kernel<HD>, L::ALLOC, attr_set); e != cudaSuccess)
+        return e;
     CUtensorMap tq, tk, tv;
     if (!encode_tmap_2d_bf16(&tq, q, static_cast<uint64_t>(Hq) * HD, static_cast<uint64_t>(M_total),
                              static_cast<uint64_t>(Hq) * HD * 2, 64, BM) ||

@@ -274,13 +274,9 @@ cudaError_t launch_score_tc(const uint16_t* hidden, const int32_t* cu_seqlens, c
                             int D, const uint16_t* Wg, const float* b1, const float* w2, float b2, int I, float eps,
                             float* scores, int sms, cudaStream_t st) {
     using C = ScoreCfg<NACC>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<NACC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             score_smem_bytes<NACC>(256));
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static std::atomic<uint64_t> attr_set{0};
+    if (cudaError_t e = ensure_smem_limit(score_tc_kernel<NACC>, score_smem_bytes<NACC>(256), attr_set); e != cudaSuccess)
+        return e;
     CUtensorMap tx, tw;
     if (!encode_tmap_2d_bf16(&tx, hidden, static_cast<uint64_t>(D), static_cast<uint64_t>(T),
                              static_cast<uint64_t>(D) * 2, KB, 128) ||

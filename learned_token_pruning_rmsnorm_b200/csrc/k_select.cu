@@ -419,16 +419,12 @@ extern "C" int tg_trace_read_select(unsigned long long* host) {
 #endif
 
 cudaError_t launch_select_scan(int mode, const float* scores, const uint8_t* keep_in, const int32_t* cu_seqlens,
-                               const int32_t* span, const int32_t* k, const int32_t* cu_kept, int B,
+                               const int32_t* span, const int32_t* k, const int32_t* cu_kept, int B, int64_t T,
                                uint8_t* keep_out, int32_t* kept_idx, int32_t* pos, int32_t* rank, float* gls,
                                cudaStream_t st) {
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(select_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             SEL_SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static std::atomic<uint64_t> attr_set{0};
+    if (cudaError_t e = ensure_smem_limit(select_scan_kernel, SEL_SMEM_BYTES, attr_set); e != cudaSuccess)
+        return e;
     if (B == 0) return cudaSuccess;
     select_scan_kernel<<<dim3(SEL_CL, B), SEL_THREADS, SEL_SMEM_BYTES, st>>>(mode, scores, keep_in, cu_seqlens, span,
                                                                             k, cu_kept, keep_out, kept_idx, pos,

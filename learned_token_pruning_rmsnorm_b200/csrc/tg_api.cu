@@ -188,7 +188,7 @@ tg_status tg_select_topk(const float* scores, const int32_t* cu_seqlens, const i
     const bool emit = cu_kept && kept_idx;
     TG_REQUIRE(!emit || (pos && rank && gls), "the fused compaction map needs pos, rank and gls");
     if (tg_status s = check_device()) return s;
-    return cuda_status(tg::launch_select_scan(0, scores, nullptr, cu_seqlens, span, k, emit ? cu_kept : nullptr, B,
+    return cuda_status(tg::launch_select_scan(0, scores, nullptr, cu_seqlens, span, k, emit ? cu_kept : nullptr, B, T,
                                               keep, emit ? kept_idx : nullptr, pos, rank, gls, stream),
                        "tg_select_topk launch");
 }
@@ -210,7 +210,7 @@ tg_status tg_compact(const uint16_t* hidden, const float* scores, const uint8_t*
     if (tg_status s = check_device()) return s;
     tg_status s = TG_OK;
     if (keep)
-        s = cuda_status(tg::launch_select_scan(1, scores, keep, cu_seqlens, span, nullptr, cu_kept, B, nullptr,
+        s = cuda_status(tg::launch_select_scan(1, scores, keep, cu_seqlens, span, nullptr, cu_kept, B, T, nullptr,
                                                kept_idx, pos, rank, gls, stream),
                         "tg_compact scan launch");
     if (s != TG_OK || !hidden_kept) return s;
@@ -293,7 +293,7 @@ tg_status tg_gated_prefill_layer(const tg_prefill_layer_args* a, tg_stream_t str
                                a->eps, a->scores, st))
         return s;
     if (tg_status s = cuda_status(tg::launch_select_scan(0, a->scores, nullptr, a->cu_seqlens, a->span, a->k,
-                                                         a->cu_kept, a->B, a->keep, a->kept_idx, a->pos, a->rank,
+                                                         a->cu_kept, a->B, a->T, a->keep, a->kept_idx, a->pos, a->rank,
                                                          a->gls, st),
                                   "select launch"))
         return s;

@@ -5,9 +5,25 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "tokengate.h"
 
 namespace tg {
+
+// Raises a kernel's dynamic shared-memory limit once per device (the
+// attribute is per device; `done` holds one bit per device ordinal).
+template <typename Kernel>
+inline cudaError_t ensure_smem_limit(Kernel* kernel, int bytes, std::atomic<uint64_t>& done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = dev < 64 ? (uint64_t(1) << dev) : 0;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+    return e;
+}
 
 // Device status word bits (see tg_device_status in tokengate.h).
 constexpr int TG_DEVICE_TIMEOUT = 1 << 16;   // a bounded wait gave up
@@ -46,7 +62,7 @@ cudaError_t launch_score(const uint16_t* hidden, const int32_t* cu_seqlens, cons
 // mode 0: select by score (writes keep; the compaction outputs if non-null)
 // mode 1: compaction scan from caller-given keep flags
 cudaError_t launch_select_scan(int mode, const float* scores, const uint8_t* keep_in, const int32_t* cu_seqlens,
-                               const int32_t* span, const int32_t* k, const int32_t* cu_kept, int B,
+                               const int32_t* span, const int32_t* k, const int32_t* cu_kept, int B, int64_t T,
                                uint8_t* keep_out, int32_t* kept_idx, int32_t* pos, int32_t* rank, float* gls,
                                cudaStream_t st);
 
