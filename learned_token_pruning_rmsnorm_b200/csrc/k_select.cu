@@ -11,15 +11,18 @@
 //   1. bucket select: the cluster agrees on the span's [min, max] key range,
 //      then each pass histograms the keys of the current range into <= 2048
 //      buckets of width 2^s (buckets span the data's actual range, so
-//      concentrated exponents still spread), sums the SEL_CL histograms
-//      through distributed shared memory, and narrows the range to the bucket
-//      holding the K-th key.  At most three passes reach a single key value:
-//      thr, with need_eq = how many keys equal to thr are kept (the
-//      lowest-indexed ones).
-//   2. ordered scan, one token per thread per row of 1024 tokens: ballots
-//      and a two-level prefix number the kept tokens, the cluster exchanges
-//      slice totals, and each kept token writes its compaction-map entry
-//      (kept_idx, pos, rank, logsigmoid of its score) with coalesced stores.
+//      concentrated exponents still spread) and sums them into 64 superbins.
+//      One warp per CTA then reads the 8 x 64 superbin sums and the 8 x 32
+//      buckets of the chosen superbin through distributed shared memory and
+//      narrows the range to the bucket holding the K-th key.  At most three
+//      passes reach a single key value: thr, with need_eq = how many keys
+//      equal to thr are kept (the lowest-indexed ones).
+//   2. ordered scan: every warp owns a contiguous run of the slice and walks
+//      it 32 tokens at a time; ballots count the kept tokens, one block scan
+//      over the warp totals and one exchange of slice totals across the
+//      cluster number them, and each kept token writes its compaction-map
+//      entry (kept_idx, pos, rank, logsigmoid of its score) in coalesced
+//      stores with no further barrier.
 // Everything is deterministic: atomics only build counts.
 
 #include <cooperative_groups.h>
@@ -51,48 +54,35 @@ constexpr int SEL_THREADS = 1024;
 constexpr int SEL_WARPS = SEL_THREADS / 32;
 constexpr int SEL_CACHE_KEYS = 32768;         // keys cached per CTA (128 KB)
 constexpr int SEL_BINS = 2048;
+constexpr int SEL_SUPER = SEL_BINS / 32;      // superbins of 32 buckets
 constexpr int SEL_SMEM_BYTES = SEL_CACHE_KEYS * 4 + 2 * SEL_BINS * 4;
 
 struct SelShared {
-    int warp_sums[SEL_WARPS];
-    int total;
     uint32_t kmin, kmax;
-    int xchg[4];          // values this CTA publishes to the cluster
-    uint32_t lo;          // current key range [lo, lo + width)
+    int coarse[2][SEL_SUPER];  // per pass parity: bucket counts summed over each superbin
+    int xchg[2];               // slice totals published to the cluster: kept, tie-ranked
+    int warp_kept[SEL_WARPS];  // exclusive prefix over the warps of this CTA
+    int warp_eq[SEL_WARPS];
+    uint32_t lo;               // current key range [lo, lo + width)
     uint64_t width;
-    int remaining;        // keys still to take from the current range, counted from its top
+    int remaining;             // keys still to take from the current range, counted from its top
     int bin_count;
-    int64_t above;        // kept keys above the current range
 };
 
-// Inclusive scan of one int per thread over the block; returns the
-// inclusive prefix and writes the block total to *total.  All threads call it.
-__device__ __forceinline__ int block_inclusive_scan(int v, int* total, SelShared& sh) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int x = v;
+__device__ __forceinline__ int warp_sum(int v) {
+#pragma unroll
+    for (int off = 16; off; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    return v;
+}
+
+__device__ __forceinline__ int warp_inclusive_scan(int v) {
+    const int lane = threadIdx.x & 31;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, x, off);
-        if (lane >= off) x += y;
+        const int y = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += y;
     }
-    if (lane == 31) sh.warp_sums[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-        const int w = sh.warp_sums[lane];
-        int s = w;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, s, off);
-            if (lane >= off) s += y;
-        }
-        sh.warp_sums[lane] = s - w;  // exclusive prefix of the warp totals
-        if (lane == 31) sh.total = s;
-    }
-    __syncthreads();
-    const int res = sh.warp_sums[warp] + x;
-    *total = sh.total;
-    __syncthreads();
-    return res;
+    return v;
 }
 
 __device__ __forceinline__ float logsigmoid_f(float s) { return fminf(s, 0.0f) - log1pf(expf(-fabsf(s))); }
@@ -104,21 +94,13 @@ __device__ __forceinline__ float key_to_score(uint32_t key) {
 
 __device__ __forceinline__ int bit_length(uint64_t v) { return v ? 64 - __clzll(static_cast<long long>(v)) : 0; }
 
-// Sum over the cluster of the int published by every CTA at sh.xchg[slot]
-// (each CTA must have written it before the cluster barrier that precedes the call).
-__device__ __forceinline__ void cluster_prefix(cg::cluster_group& cl, SelShared& sh, int slot, int rank_self,
-                                               int64_t* before, int64_t* total) {
-    int v[SEL_CL];
-#pragma unroll
-    for (int r = 0; r < SEL_CL; ++r) v[r] = cl.map_shared_rank(&sh, r)->xchg[slot];  // all loads in flight
-    int64_t b = 0, t = 0;
-#pragma unroll
-    for (int r = 0; r < SEL_CL; ++r) {
-        if (r < rank_self) b += v[r];
-        t += v[r];
-    }
-    *before = b;
-    *total = t;
+// split cluster barrier: arrive once this CTA reads no more remote shared
+// memory, wait before leaving so that no CTA exits while another reads it
+__device__ __forceinline__ void cluster_arrive_release() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 __global__ void __cluster_dims__(SEL_CL, 1, 1) __launch_bounds__(SEL_THREADS, 1)
@@ -145,10 +127,13 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
     const bool emit = kept_idx != nullptr;  // cu_kept is only read when emitting
     const int64_t m0 = emit ? cu_kept[b] : 0, m1 = emit ? cu_kept[b + 1] : 0;
 
-    // this CTA's token slice [t0, t1), rows of 1024 tokens
+    // this CTA's token slice [t0, t1) (a multiple of 1024 tokens long), split
+    // into one contiguous run per warp
     const int64_t n = s1 - s0;
     const int64_t per = ((n + SEL_CL - 1) / SEL_CL + SEL_THREADS - 1) / SEL_THREADS * SEL_THREADS;
     const int64_t t0 = min(s1, s0 + per * crank), t1 = min(s1, t0 + per);
+    const int64_t per_warp = per / SEL_WARPS;
+    const int64_t w0 = min(t1, t0 + per_warp * warp), w1 = min(t1, w0 + per_warp);
     // prunable part of the slice [k0, k1) and whether its keys fit the cache
     const int64_t k0 = max(t0, p0), k1 = max(k0, min(t1, p1));
     const bool cached = (k1 - k0) <= SEL_CACHE_KEYS;
@@ -164,12 +149,36 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
     int64_t need_eq = 0;     // keys equal to thr that are kept
     bool all_eq_kept = true; // every key equal to thr is kept: no tie ranking needed
 
-    if (do_select) {
-        // ------------------------------------------------ cache keys, range of the span
+    // ------------------------------------------------ cache keys (for the selection and for gls)
+    const bool need_gls = emit && kk > 0;  // some prunable token is kept: its logsigmoid is emitted
+    if (cached && (do_select || need_gls)) {
         uint32_t lmin = 0xFFFFFFFFu, lmax = 0u;
         for (int64_t t = k0 + tid; t < k1; t += SEL_THREADS) {
             const uint32_t key = score_key(__ldg(scores + t));
-            if (cached) skeys[t - k0] = key;
+            skeys[t - k0] = key;
+            lmin = min(lmin, key);
+            lmax = max(lmax, key);
+        }
+        if (do_select) {
+#pragma unroll
+            for (int off = 16; off; off >>= 1) {
+                lmin = min(lmin, __shfl_xor_sync(0xffffffffu, lmin, off));
+                lmax = max(lmax, __shfl_xor_sync(0xffffffffu, lmax, off));
+            }
+            if (tid == 0) {
+                sh.kmin = 0xFFFFFFFFu;
+                sh.kmax = 0u;
+            }
+            __syncthreads();
+            if (lane == 0) {
+                atomicMin(&sh.kmin, lmin);
+                atomicMax(&sh.kmax, lmax);
+            }
+        }
+    } else if (do_select) {
+        uint32_t lmin = 0xFFFFFFFFu, lmax = 0u;
+        for (int64_t t = k0 + tid; t < k1; t += SEL_THREADS) {
+            const uint32_t key = score_key(__ldg(scores + t));
             lmin = min(lmin, key);
             lmax = max(lmax, key);
         }
@@ -187,7 +196,10 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
             atomicMin(&sh.kmin, lmin);
             atomicMax(&sh.kmax, lmax);
         }
-        SEL_TRACE(1);
+    }
+    SEL_TRACE(1);
+
+    if (do_select) {  // uniform over the cluster: it depends on the sequence only
         cl.sync();  // every CTA's slice min/max is published
         SEL_TRACE(2);
         if (warp == 0) {
@@ -203,11 +215,11 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
                 gmin = min(gmin, __shfl_xor_sync(0xffffffffu, gmin, off));
                 gmax = max(gmax, __shfl_xor_sync(0xffffffffu, gmax, off));
             }
-            if (lane == 0) sh.lo = gmin;
             if (lane == 0) {
+                sh.lo = gmin;
                 sh.width = static_cast<uint64_t>(gmax) - gmin + 1;
                 sh.remaining = static_cast<int>(kk);
-                sh.above = 0;
+                sh.bin_count = 0;
             }
         }
         __syncthreads();
@@ -215,63 +227,85 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
         for (int pass = 0;; ++pass) {
             const uint32_t lo = sh.lo;
             const uint64_t width = sh.width;
-            const int sh_bits = max(0, bit_length(width - 1) - 11);  // bucket width 2^sh_bits
-            const int nb = static_cast<int>(((width - 1) >> sh_bits) + 1);
+            const int sh_bits = max(0, bit_length(width - 1) - 11);  // bucket width 2^sh_bits, <= 2048 buckets
+            // both buffers alternate by pass: another CTA may still read the previous pass's
             int* hist = hist_buf + (pass & 1) * SEL_BINS;
-            for (int i = tid; i < nb; i += SEL_THREADS) hist[i] = 0;
+            int* coarse = sh.coarse[pass & 1];
+            hist[tid] = 0;
+            hist[tid + SEL_THREADS] = 0;
             __syncthreads();
             for (int64_t t = k0 + tid; t < k1; t += SEL_THREADS) {
                 const uint32_t key = cached ? skeys[t - k0] : score_key(__ldg(scores + t));
                 const uint32_t d = key - lo;  // wraps for keys below lo: excluded by the range test
                 if (key >= lo && static_cast<uint64_t>(d) < width) atomicAdd(&hist[d >> sh_bits], 1);
             }
-            cl.sync();  // every CTA's histogram of this pass is complete
-            // bucket search from the top: thread tid owns buckets nb-1-2*tid and nb-2-2*tid
-            int cnt[2] = {0, 0};
-            int local = 0;
-            {
-                // both buckets of every CTA: all 2 x SEL_CL remote loads in flight at once
-                const int bin0 = nb - 1 - 2 * tid, bin1 = bin0 - 1;
-                int v0[SEL_CL], v1[SEL_CL];
-#pragma unroll
-                for (int r = 0; r < SEL_CL; ++r) {
-                    const int* hr = cl.map_shared_rank(hist, r);
-                    v0[r] = bin0 >= 0 ? hr[bin0] : 0;
-                    v1[r] = bin1 >= 0 ? hr[bin1] : 0;
+            __syncthreads();
+            {   // superbin sums: warp w sums buckets [64w, 64w + 64)
+                const int a = warp_sum(hist[64 * warp + lane]);
+                const int c = warp_sum(hist[64 * warp + 32 + lane]);
+                if (lane == 0) {
+                    coarse[2 * warp] = a;
+                    coarse[2 * warp + 1] = c;
                 }
-#pragma unroll
-                for (int r = 0; r < SEL_CL; ++r) {
-                    cnt[0] += v0[r];
-                    cnt[1] += v1[r];
-                }
-                local = cnt[0] + cnt[1];
             }
-            int total = 0;
-            const int incl = block_inclusive_scan(local, &total, sh);
-            const int excl = incl - local;
-            const int rem = sh.remaining;
-            __syncthreads();  // every thread has read sh.remaining before it is rewritten
-            if (excl < rem && incl >= rem) {
-                int cum = excl;
+            cl.sync();  // every CTA's histogram and superbin sums of this pass are complete
+            if (warp == 0) {
+                // the rem-th key from the top: first its superbin (lane l owns superbins
+                // 63 - 2l and 62 - 2l of all CTAs), then its bucket (lane l owns bucket
+                // 32 S + 31 - l of all CTAs); every CTA finds the same bucket
+                const int rem = sh.remaining;
+                int hi = 0, lo2 = 0;
+                {
+                    int vh[SEL_CL], vl[SEL_CL];
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    if (cum + cnt[e] >= rem) {
-                        const uint32_t bin = static_cast<uint32_t>(nb - 1 - (2 * tid + e));
+                    for (int r = 0; r < SEL_CL; ++r) {
+                        const int* cr = cl.map_shared_rank(coarse, r);
+                        vh[r] = cr[SEL_SUPER - 1 - 2 * lane];
+                        vl[r] = cr[SEL_SUPER - 2 - 2 * lane];
+                    }
+#pragma unroll
+                    for (int r = 0; r < SEL_CL; ++r) {
+                        hi += vh[r];
+                        lo2 += vl[r];
+                    }
+                }
+                const int incl = warp_inclusive_scan(hi + lo2);
+                const int excl = incl - hi - lo2;
+                const unsigned hit = __ballot_sync(0xffffffffu, excl < rem && incl >= rem);
+                if (hit != 0u) {
+                    const int L = __ffs(hit) - 1;
+                    const int excl_L = __shfl_sync(0xffffffffu, excl, L);
+                    const int hi_L = __shfl_sync(0xffffffffu, hi, L);
+                    const bool upper = excl_L + hi_L >= rem;
+                    const int S = upper ? SEL_SUPER - 1 - 2 * L : SEL_SUPER - 2 - 2 * L;
+                    const int rem2 = upper ? rem - excl_L : rem - excl_L - hi_L;
+                    const int bin = 32 * S + 31 - lane;
+                    int v[SEL_CL];
+#pragma unroll
+                    for (int r = 0; r < SEL_CL; ++r) v[r] = cl.map_shared_rank(hist, r)[bin];
+                    int cnt = 0;
+#pragma unroll
+                    for (int r = 0; r < SEL_CL; ++r) cnt += v[r];
+                    const int incl2 = warp_inclusive_scan(cnt);
+                    const int excl2 = incl2 - cnt;
+                    if (excl2 < rem2 && incl2 >= rem2) {
                         const uint64_t new_lo = static_cast<uint64_t>(lo) + (static_cast<uint64_t>(bin) << sh_bits);
                         const uint64_t end = static_cast<uint64_t>(lo) + width;
                         sh.lo = static_cast<uint32_t>(new_lo);
                         sh.width = min(static_cast<uint64_t>(1) << sh_bits, end - new_lo);
-                        sh.remaining = rem - cum;
-                        sh.bin_count = cnt[e];
-                        sh.above += cum;
-                        break;
+                        sh.remaining = rem2 - excl2;
+                        sh.bin_count = cnt;
                     }
-                    cum += cnt[e];
+                } else if (lane == 0) {
+                    // unreachable while the range holds >= rem keys; end the search on lo
+                    sh.width = 1;
+                    sh.remaining = 0;
+                    sh.bin_count = 0;
                 }
             }
             __syncthreads();
             SEL_TRACE(3 + pass);
-            if (sh_bits == 0) break;  // the bucket is a single key value
+            if (sh_bits == 0 || pass >= 3) break;  // the bucket is a single key value
         }
         thr = sh.lo;
         need_eq = sh.remaining;
@@ -279,12 +313,12 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
     }
 
     // ---------------------------------------------------------------- ordered scan
-    // kept flag of token t (one per thread per row); eq marks a key equal to thr
-    // that is ranked by index when only some of them are kept
+    // kept flag of token t; eq marks a key equal to thr that is ranked by index
+    // when only some of them are kept
     auto flags = [&](int64_t t, bool& kept, bool& eq) {
         kept = false;
         eq = false;
-        if (t >= t1) return;
+        if (t >= w1) return;
         const bool prun = t >= p0 && t < p1;
         if (mode == 1) {
             kept = keep_in[t] != 0;
@@ -298,85 +332,83 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
             eq = key == thr && !all_eq_kept;
         }
     };
-    const int nrows = static_cast<int>((t1 - t0 + SEL_THREADS - 1) / SEL_THREADS);
     const unsigned lt_mask = (1u << lane) - 1u;
 
-    // slice totals: kept tokens and (for the tie ranking) keys equal to thr
+    // warp totals: kept tokens and (for the tie ranking) keys equal to thr
     int my_kept = 0, my_eq = 0;
-    for (int r = 0; r < nrows; ++r) {
+    for (int64_t base = w0; base < w1; base += 32) {
         bool kept, eq;
-        flags(t0 + static_cast<int64_t>(r) * SEL_THREADS + tid, kept, eq);
-        my_kept += kept;
-        my_eq += eq;
+        flags(base + lane, kept, eq);
+        my_kept += __popc(__ballot_sync(0xffffffffu, kept));
+        my_eq += __popc(__ballot_sync(0xffffffffu, eq));
     }
-    int tot_kept = 0, tot_eq = 0;
-    block_inclusive_scan(my_kept, &tot_kept, sh);
-    if (!all_eq_kept) block_inclusive_scan(my_eq, &tot_eq, sh);
-    if (tid == 0) {
-        sh.xchg[0] = tot_kept;
-        sh.xchg[1] = tot_eq;
+    if (lane == 0) {
+        sh.warp_kept[warp] = my_kept;
+        sh.warp_eq[warp] = my_eq;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const int vk = sh.warp_kept[lane], ve = sh.warp_eq[lane];
+        const int ik = warp_inclusive_scan(vk), ie = warp_inclusive_scan(ve);
+        sh.warp_kept[lane] = ik - vk;
+        sh.warp_eq[lane] = ie - ve;
+        if (lane == 31) {
+            sh.xchg[0] = ik;
+            sh.xchg[1] = ie;
+        }
     }
     SEL_TRACE(8);
-    cl.sync();
+    cl.sync();  // slice totals published; also orders the key cache before the emission
     SEL_TRACE(9);
-    int64_t kept_before = 0, kept_all = 0, eq_before = 0, eq_all = 0;
-    cluster_prefix(cl, sh, 0, crank, &kept_before, &kept_all);
-    if (!all_eq_kept) cluster_prefix(cl, sh, 1, crank, &eq_before, &eq_all);
-    // the keys equal to thr that this slice keeps: ranks [eq_before, eq_before + tot_eq) among all equal keys
-    int64_t eq_seen = eq_before;    // equal keys before the current row, in index order
-    int64_t m = m0 + kept_before;   // compaction index of the first kept token of the current row
-    // kept-before counts the tie-ranked keys as not kept; correct for the ones this CTA's
-    // predecessors keep
-    if (!all_eq_kept) m += min(eq_before, need_eq);
-    __shared__ int row_warp_kept[SEL_WARPS], row_warp_eq[SEL_WARPS];
-    for (int r = 0; r < nrows; ++r) {
-        const int64_t t = t0 + static_cast<int64_t>(r) * SEL_THREADS + tid;
+    int64_t kept_before = sh.warp_kept[warp], eq_before = sh.warp_eq[warp];
+    {
+        int vk[SEL_CL], ve[SEL_CL];
+#pragma unroll
+        for (int r = 0; r < SEL_CL; ++r) {
+            const SelShared* o = cl.map_shared_rank(&sh, r);
+            vk[r] = o->xchg[0];
+            ve[r] = o->xchg[1];
+        }
+#pragma unroll
+        for (int r = 0; r < SEL_CL; ++r) {
+            if (r < crank) {
+                kept_before += vk[r];
+                eq_before += ve[r];
+            }
+        }
+    }
+    cluster_arrive_release();  // no remote reads after this point
+    // kept_before counts the tie-ranked keys as not kept; min(eq_before, need_eq) of
+    // those before this warp's run are kept
+    int64_t m = m0 + kept_before + (all_eq_kept ? 0 : min(eq_before, need_eq));
+    int64_t eq_seen = eq_before;
+    for (int64_t base = w0; base < w1; base += 32) {
+        const int64_t t = base + lane;
         bool kept, eq;
         flags(t, kept, eq);
         const unsigned eq_ball = __ballot_sync(0xffffffffu, eq);
-        if (!all_eq_kept) {
-            if (lane == 0) row_warp_eq[warp] = __popc(eq_ball);
-            __syncthreads();
-            int eq_prefix = 0, eq_row = 0;
-            for (int w = 0; w < SEL_WARPS; ++w) {
-                const int v = row_warp_eq[w];
-                if (w < warp) eq_prefix += v;
-                eq_row += v;
-            }
-            const int64_t eq_rank = eq_seen + eq_prefix + __popc(eq_ball & lt_mask);
-            if (eq && eq_rank < need_eq) kept = true;
-            eq_seen += eq_row;
-            __syncthreads();
-        }
+        if (eq && eq_seen + __popc(eq_ball & lt_mask) < need_eq) kept = true;
+        eq_seen += __popc(eq_ball);
         const unsigned kept_ball = __ballot_sync(0xffffffffu, kept);
-        if (lane == 0) row_warp_kept[warp] = __popc(kept_ball);
-        __syncthreads();
-        int kept_prefix = 0, kept_row = 0;
-        for (int w = 0; w < SEL_WARPS; ++w) {
-            const int v = row_warp_kept[w];
-            if (w < warp) kept_prefix += v;
-            kept_row += v;
-        }
-        __syncthreads();
-        if (t < t1) {
+        if (t < w1) {
             if (mode == 0) keep_out[t] = kept ? 1 : 0;
-            const int64_t mi = m + kept_prefix + __popc(kept_ball & lt_mask);
+            const int64_t mi = m + __popc(kept_ball & lt_mask);
             // a caller-given keep vector that disagrees with cu_kept must not
             // write outside [m0, m1)
             if (emit && kept && mi < m1) {
                 const bool prun = t >= p0 && t < p1;
                 float g = 0.0f;
-                if (prun) g = logsigmoid_f(cached && do_select ? key_to_score(skeys[t - k0]) : __ldg(scores + t));
+                if (prun) g = logsigmoid_f(cached ? key_to_score(skeys[t - k0]) : __ldg(scores + t));
                 kept_idx[mi] = static_cast<int32_t>(t);
                 pos[mi] = static_cast<int32_t>(t - s0 + 1);
                 rank[mi] = static_cast<int32_t>(mi - m0 + 1);
                 gls[mi] = g;
             }
         }
-        m += kept_row;
+        m += __popc(kept_ball);
     }
     SEL_TRACE(10);
-    cl.sync();  // no CTA leaves while another may still read its shared memory
+    cluster_wait_acquire();
     SEL_TRACE(11);
 }
 
