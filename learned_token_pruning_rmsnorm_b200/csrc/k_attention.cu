@@ -64,7 +64,7 @@ enum : int {
 // Optional device trace (builds with -DTG_TRACE only): clock64 stamps of the
 // pipeline hand-offs of the CTA at blockIdx (0, 0, 0), 64 KV tiles at most.
 #ifdef TG_TRACE
-__device__ unsigned long long g_attn_trace[16 * 64];  // points 0..15 x 64 tiles
+__device__ unsigned long long g_attn_trace[24 * 64];  // points 0..23 x 64 tiles
 __device__ unsigned long long g_attn_cta[4096 * 12];  // per CTA: phase stamps (ns), SM id | n_kv
 #define TG_TRACE_AT(point, j)                                                              \
     do {                                                                                   \
@@ -92,9 +92,64 @@ __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity, int* s
     return mbar_wait(bar, parity, &never, status, TG_WHERE_DRAIN);
 }
 
+// Global load that stays where it is written (volatile asm is not moved across the
+// other volatile asm statements), so that a prefetch issued a tile ahead is not
+// sunk by the compiler to its first use.
+__device__ __forceinline__ float ldg_early(const float* p) {
+    float v;
+    asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v) : "l"(p));
+    return v;
+}
+
+// max of three floats (one instruction on sm_100)
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// Packed fp32 pairs (lo in bits 0-31): two FMAs or adds per instruction on sm_100.
+__device__ __forceinline__ uint64_t f32x2_pack(float lo, float hi) {
+    return static_cast<uint64_t>(__float_as_uint(lo)) | (static_cast<uint64_t>(__float_as_uint(hi)) << 32);
+}
+__device__ __forceinline__ float f32x2_lo(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v)); }
+__device__ __forceinline__ float f32x2_hi(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
+__device__ __forceinline__ uint64_t f32x2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f32x2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// Named barrier `id` over `n` threads that also returns the OR of `pred` over them.
+__device__ __forceinline__ bool bar_red_or(int id, int n, bool pred) {
+    uint32_t res;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(res)
+        : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(n)
+        : "memory");
+    return res != 0;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// (high, low) bf16 split of v packed as a pair: high = bf16(v), low = bf16(v - high).
+// Infinities are clamped to the largest finite magnitude so that products with a zero
+// low part of the other operand stay finite (the sum still overflows to infinity).
+__device__ __forceinline__ uint32_t bf16_hi_lo(float v) {
+    const float c = fminf(fmaxf(v, -3.0e38f), 3.0e38f);  // NaN stays NaN
+    const __nv_bfloat16 hi = __float2bfloat16_rn(isnan(v) ? v : c);
+    const float lo = (isnan(v) ? v : c) - __bfloat162float(hi);
+    return pack_bf16x2(__bfloat162float(hi), lo);
 }
 
 template <int HD>
@@ -265,7 +320,7 @@ gated_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 wbias[s * BN + e * 32 + lane] = key_local < Mb ? gscale * gls[seq0 + key_local] : 0.f;
             }
             __syncwarp();
-            ok = mbar_wait(bar(B_S_FULL + s), (j >> 1) & 1, abort_flag, status, TG_WHERE_SOFTMAX);
+            ok = mbar_wait_warp(bar(B_S_FULL + s), (j >> 1) & 1, abort_flag, status, TG_WHERE_SOFTMAX);
             if (!ok) break;
             tc_fence_after();
             float x[BN];
@@ -309,7 +364,7 @@ gated_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             l_run = l_run * corr + sum;
             // the P tile and O may be touched only once PV_{j-1} has completed
             if (j >= 1) {
-                ok = mbar_wait(bar(B_PV_DONE), (j - 1) & 1, abort_flag, status, TG_WHERE_SOFTMAX);
+                ok = mbar_wait_warp(bar(B_PV_DONE), (j - 1) & 1, abort_flag, status, TG_WHERE_SOFTMAX);
                 if (!ok) break;
                 tc_fence_after();
             }
@@ -345,7 +400,7 @@ gated_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             mbar_arrive(bar(B_P_FULL));
         }
         // ---------------------------------------------------------------- epilogue
-        if (ok) ok = mbar_wait(bar(B_PV_DONE), (n_kv - 1) & 1, abort_flag, status, TG_WHERE_SOFTMAX);
+        if (ok) ok = mbar_wait_warp(bar(B_PV_DONE), (n_kv - 1) & 1, abort_flag, status, TG_WHERE_SOFTMAX);
         if (ok) {
             tc_fence_after();
             const float inv_l = 1.0f / l_run;
@@ -382,19 +437,21 @@ gated_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
 // ---------------------------------------------------------------------------
 // Two query heads of one KV head per CTA (GQA groups of even size).
 //
-// 320 threads: warps 0-3 = softmax of head 0, warps 4-7 = softmax of head 1,
-// warp 8 = TMA producer, warp 9 = MMA issuer.  Both heads share every K/V
-// tile.  TMEM (512 columns): S0 | S1 | O0 | O1; P_h (bf16, two keys per
-// column) is written over the first 64 columns of S_h and read from TMEM as
-// the A operand of the PV MMA.  The MMA issuer interleaves
+// 320 threads: warps 0-7 = softmax of both heads in turn (thread = one row,
+// one half of the columns), warp 8 = TMA producer, warp 9 = MMA issuer.
+// Both heads share every K/V tile.  TMEM (512 columns): S0 | S1 | O0 | O1;
+// P_h (bf16, two keys per column) is written over the first 64 columns of
+// S_h and read from TMEM as the A operand of the PV MMA.  The MMA issuer
+// interleaves
 //     S0(j) S1(j) | PV0(j) S0(j+1) | PV1(j) S1(j+1) | ...
-// so that one head's softmax overlaps the other head's tensor-core work;
+// and the softmax warps take head 0 of tile j, head 1 of tile j, head 0 of
+// tile j+1, ..., so that one head's softmax overlaps the other head's
+// tensor-core work;
 // tcgen05 operations of one thread execute in issue order, which is what
 // lets S_h(j+1) overwrite P_h(j) right after PV_h(j), and what makes the
 // commit after S_h(j) also cover PV_h(j-1) (so the softmax may rescale O_h
 // as soon as S_h(j) is complete).
 constexpr int G2_THREADS = 320;
-constexpr int G2_ILP = 8;  // independent partial max / sum chains per row
 
 template <int HD>
 struct G2Smem {
@@ -403,8 +460,14 @@ struct G2Smem {
     static constexpr int OFF_Q = 0;  // two heads
     static constexpr int OFF_K = OFF_Q + 2 * TILE_Q;
     static constexpr int OFF_V = OFF_K + 2 * TILE_KV;
-    static constexpr int OFF_BIAS = OFF_V + 2 * TILE_KV;
-    static constexpr int OFF_BAR = OFF_BIAS + 8 * 2 * BN * 4;  // a private bias copy per softmax warp
+    // operands of the extra k-step that adds the gate bias to S: 128 rows x 16 bf16,
+    // no swizzle (8-row x 16-byte core matrices, K cores 128 B apart, row groups 256 B)
+    static constexpr int EXT = BM * 16 * 2;
+    static constexpr int OFF_QX = OFF_V + 2 * TILE_KV;  // [head]
+    static constexpr int OFF_KX = OFF_QX + 2 * EXT;      // [stage]
+    // partial row maxima [parity][half][row] (2 KB) and partial row sums [head][half][row] (2 KB)
+    static constexpr int OFF_RED = OFF_KX + 2 * EXT;
+    static constexpr int OFF_BAR = OFF_RED + 2 * 2 * BM * 4 + 2 * 2 * BM * 4;
     static constexpr int NUM_BARS = 18;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int BYTES = OFF_MISC + 16;
@@ -414,7 +477,7 @@ struct G2Smem {
 
 enum : int {
     G_Q_FULL = 0, G_K_FULL = 1, G_K_EMPTY = 3, G_V_FULL = 5, G_V_EMPTY = 7, G_S_FULL = 9, G_P_FULL = 11,
-    G_O_FULL = 13, G_DRAIN = 14, G_TOK = 15  // G_TOK + h: head h may run its exponentials
+    G_O_FULL = 13, G_DRAIN = 14
 };
 
 // Causal work split.  Query tile qt of a sequence needs KV tiles 0..qt.  With
@@ -499,7 +562,27 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     auto bar = [&](int i) { return sbase + L::OFF_BAR + 8u * static_cast<uint32_t>(i); };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
-    float* sBias = reinterpret_cast<float*>(smem + L::OFF_BIAS);
+    const uint32_t sQX = sbase + L::OFF_QX, sKX = sbase + L::OFF_KX;
+
+    // Gate bias as one more k-step of the S = Q K^T product: row q of Q_ext holds
+    // (bh, bl, bh, bl) and row j of K_ext holds (gh, gh, gl, gl), the bf16 high and low
+    // parts of bscale_h = softplus(g_h) / sm_scale and of gls_j, so that the extra products
+    // add bscale_h * gls_j to S with about 2^-16 relative error; the other 12 columns are
+    // zero.  K cores 8..15 of all four tiles are zero throughout; K_ext rows are written by
+    // the producer per KV tile.
+    for (int i = threadIdx.x; i < 4 * (BM / 8) * 8; i += blockDim.x) {
+        const int tile = i / ((BM / 8) * 8), rem = i % ((BM / 8) * 8);
+        *reinterpret_cast<uint4*>(smem + L::OFF_QX + tile * L::EXT + (rem >> 3) * 256 + 128 + (rem & 7) * 16) =
+            make_uint4(0u, 0u, 0u, 0u);
+    }
+    if (threadIdx.x < 2 * BM) {
+        const int hh = threadIdx.x / BM, r = threadIdx.x % BM;
+        const float bscale = softplus_f(g[2 * pair + hh]) / sm_scale;
+        const uint32_t hl = bf16_hi_lo(bscale);
+        *reinterpret_cast<uint4*>(smem + L::OFF_QX + hh * L::EXT + (r >> 3) * 256 + (r & 7) * 16) =
+            make_uint4(hl, hl, 0u, 0u);
+    }
+    fence_proxy_async_smem();
 
     if (threadIdx.x == 0) {
         mbar_init(bar(G_Q_FULL), 1);
@@ -509,12 +592,10 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             mbar_init(bar(G_V_FULL + s), 1);
             mbar_init(bar(G_V_EMPTY + s), 1);
             mbar_init(bar(G_S_FULL + s), 1);
-            mbar_init(bar(G_P_FULL + s), 128);
+            mbar_init(bar(G_P_FULL + s), 256);
         }
         mbar_init(bar(G_O_FULL), 1);
         mbar_init(bar(G_DRAIN), 1);
-        mbar_init(bar(G_TOK + 0), 128);
-        mbar_init(bar(G_TOK + 1), 128);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -530,6 +611,8 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
 
     if (warp == 8) {
         // ---------------------------------------------------------------- TMA producer
+        // The whole warp writes the K_ext rows of each KV tile (lane l: keys 4l .. 4l+3);
+        // lane 0 issues the copies.  K_ext(stage) is released with K(stage).
         if (lane == 0) {
             prefetch_tmap(&tmQ);
             prefetch_tmap(&tmK);
@@ -541,21 +624,50 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 for (int hf = 0; hf < HD / 64; ++hf)
                     tma_load_2d(sQ + hh * L::TILE_Q + hf * BM * 128, &tmQ, (2 * pair + hh) * HD + hf * 64,
                                 seq0 + qt * BM, bar(G_Q_FULL));
-            int k_issued[2] = {0, 0}, v_issued[2] = {0, 0};
-            for (int j = 0; j < n_kv; ++j) {
-                const int s = j & 1;
-                if (j >= 2 && !mbar_wait(bar(G_K_EMPTY + s), ((j - 2) >> 1) & 1, abort_flag, status,
-                                         TG_WHERE_PRODUCER))
-                    break;
+        }
+        int k_issued[2] = {0, 0}, v_issued[2] = {0, 0};
+        float gk[4];  // gls of this lane's keys of the next tile (0 past the sequence end)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int key_local = kv0 * BN + lane * 4 + i;
+            gk[i] = key_local < Mb ? ldg_early(gls + seq0 + key_local) : 0.f;
+        }
+        for (int j = 0; j < n_kv; ++j) {
+            const int s = j & 1;
+            float gcur[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) gcur[i] = gk[i];
+            if (j + 1 < n_kv) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int key_local = (kv0 + j + 1) * BN + lane * 4 + i;
+                    gk[i] = key_local < Mb ? ldg_early(gls + seq0 + key_local) : 0.f;
+                }
+            }
+            if (j >= 2 && !mbar_wait_warp(bar(G_K_EMPTY + s), ((j - 2) >> 1) & 1, abort_flag, status,
+                                          TG_WHERE_PRODUCER))
+                break;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int r = lane * 4 + i;
+                const uint32_t hl = bf16_hi_lo(gcur[i]);
+                *reinterpret_cast<uint4*>(smem + L::OFF_KX + s * L::EXT + (r >> 3) * 256 + (r & 7) * 16) =
+                    make_uint4(__byte_perm(hl, 0u, 0x1010), __byte_perm(hl, 0u, 0x3232), 0u, 0u);
+            }
+            fence_proxy_async_smem();  // K_ext is read by the tensor core (async proxy)
+            __syncwarp();
+            if (lane == 0) {
                 mbar_expect_tx(bar(G_K_FULL + s), BN * HD * 2);
 #pragma unroll
                 for (int hf = 0; hf < HD / 64; ++hf)
                     tma_load_2d(sK0 + s * L::TILE_KV + hf * BN * 128, &tmK, hk * HD + hf * 64,
                                 seq0 + (kv0 + j) * BN, bar(G_K_FULL + s));
                 ++k_issued[s];
-                if (j >= 2 && !mbar_wait(bar(G_V_EMPTY + s), ((j - 2) >> 1) & 1, abort_flag, status,
-                                         TG_WHERE_PRODUCER))
-                    break;
+            }
+            if (j >= 2 && !mbar_wait_warp(bar(G_V_EMPTY + s), ((j - 2) >> 1) & 1, abort_flag, status,
+                                          TG_WHERE_PRODUCER))
+                break;
+            if (lane == 0) {
                 mbar_expect_tx(bar(G_V_FULL + s), BN * HD * 2);
 #pragma unroll
                 for (int hf = 0; hf < HD / 64; ++hf)
@@ -563,12 +675,12 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                                 seq0 + (kv0 + j) * BN, bar(G_V_FULL + s));
                 ++v_issued[s];
             }
-            if (*abort_flag) {
-                drain_wait(bar(G_Q_FULL), 0, status);
-                for (int s = 0; s < 2; ++s) {
-                    if (k_issued[s]) drain_wait(bar(G_K_FULL + s), (k_issued[s] - 1) & 1, status);
-                    if (v_issued[s]) drain_wait(bar(G_V_FULL + s), (v_issued[s] - 1) & 1, status);
-                }
+        }
+        if (lane == 0 && *abort_flag) {
+            drain_wait(bar(G_Q_FULL), 0, status);
+            for (int s = 0; s < 2; ++s) {
+                if (k_issued[s]) drain_wait(bar(G_K_FULL + s), (k_issued[s] - 1) & 1, status);
+                if (v_issued[s]) drain_wait(bar(G_V_FULL + s), (v_issued[s] - 1) & 1, status);
             }
         }
     } else if (warp == 9) {
@@ -586,6 +698,9 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     mma_bf16_ss(tmem + hh * BN, smem_desc_sw128(qb + off_q, 16, 1024),
                                 smem_desc_sw128(kb + off_k, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
                 }
+                // + bscale_h * gls_j: the bias k-step (no-swizzle tiles, K cores 128 B apart)
+                mma_bf16_ss(tmem + hh * BN, smem_desc_noswz(sQX + hh * L::EXT, 128, 256),
+                            smem_desc_noswz(sKX + (j & 1) * L::EXT, 128, 256), idesc_qk, 1u);
             };
             auto issue_pv = [&](int hh, int j) {
                 const uint32_t vb = sV0 + (j & 1) * L::TILE_KV;
@@ -621,6 +736,11 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     tc_fence_after();
                     issue_s(0, j + 1);
                     mma_commit(bar(G_S_FULL + 0));
+                    TG_TRACE_AT(10, j);  // S0(j+1) issued
+#ifdef TG_TRACE
+                    // trace builds only: stamp the completion of S0(j+1) as the tensor core sees it
+                    if (mbar_wait(bar(G_S_FULL + 0), (j + 1) & 1, abort_flag, status, TG_WHERE_MMA)) TG_TRACE_AT(13, j);
+#endif
                 }
                 ok = mbar_wait(bar(G_P_FULL + 1), j & 1, abort_flag, status, TG_WHERE_MMA);
                 if (!ok) break;
@@ -640,162 +760,146 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         }
     } else {
         // ---------------------------------------------------------------- softmax, warps 0-7
-        // In log2 units the logit is  x = alpha_q * (s + b'_j)  with
-        //   alpha_q = sm_scale * log2(e) / tau_q   and   b'_j = softplus(g_h) * gls_j / sm_scale,
-        // so the gate bias is one FADD per score and the temperature one FFMA.
-        // The two heads take turns on the exponentials (token mbarriers), so that
-        // one head's MUFU work overlaps the other head's tensor-core work.
-        const int hh = warp >> 2;             // which of the two heads
-        const int h = 2 * pair + hh;
-        const int r = threadIdx.x & 127;      // query row == TMEM lane
-        const int lg = warp & 3;
+        // Thread (warp w, lane l) owns query row r = 32 (w & 3) + l (TMEM lane r) and the
+        // key / output columns [64 half, 64 half + 64), half = w >> 2, of BOTH heads.  The
+        // eight warps take the heads in turn (head 0 of tile j, head 1 of tile j, head 0 of
+        // tile j + 1, ...): each head's exponentials run on two warps of every SM
+        // sub-partition, which keeps the special-function unit busy, while the tensor core
+        // works on the other head.  The two halves of a row combine their partial maxima
+        // through shared memory at a barrier that also makes any abort decision uniform.
+        // S already holds s + bscale_h * gls_j (the bias k-step), so in log2 units the
+        // logit is  x = alpha_q * S  with  alpha_q = sm_scale * log2(e) / tau_q: one FMA per
+        // score with the running max folded in, issued as f32x2 pairs, and no shared-memory
+        // reads in the loop (those would queue behind the tensor core's operand traffic).
+        const int q4 = warp & 3;
+        const int half = warp >> 2;
+        const int r = q4 * 32 + lane;        // query row == TMEM lane
         const int q_local = qt * BM + r;
         const bool valid_row = q_local < Mb;
         const int qg = seq0 + q_local;
-        float inv_tau = 1.0f;
-        if (valid_row) inv_tau = 1.0f / (1.0f + c[h] * logf(static_cast<float>(pos[qg]) / static_cast<float>(rank[qg])));
-        const float alpha = sm_scale * LOG2E * inv_tau;
-        const float bscale = softplus_f(g[h]) / sm_scale;
-        const uint32_t lane_addr = static_cast<uint32_t>(lg * 32) << 16;
-        const uint32_t tS = tmem + lane_addr + hh * BN;
-        const uint32_t tO = tmem + lane_addr + 2 * BN + hh * HD;
-        float* wbias = sBias + warp * (2 * BN);
-        float m_run = -INFINITY, l_run = 0.f;
+        const float ratio_log = valid_row ? logf(static_cast<float>(pos[qg]) / static_cast<float>(rank[qg])) : 0.f;
+        // per-head values are scalars selected by the head index (no local-memory arrays)
+        const float inv_tau0 = valid_row ? 1.0f / (1.0f + c[2 * pair] * ratio_log) : 1.0f;
+        const float inv_tau1 = valid_row ? 1.0f / (1.0f + c[2 * pair + 1] * ratio_log) : 1.0f;
+        const float alpha0 = sm_scale * LOG2E * inv_tau0, alpha1 = sm_scale * LOG2E * inv_tau1;
+        const uint32_t lane_addr = static_cast<uint32_t>(q4 * 32) << 16;
+        float* red = reinterpret_cast<float*>(smem + L::OFF_RED);  // [parity][half][row] partial maxima
+        float* lred = red + 2 * 2 * BM;                             // [head][half][row] partial sums
+        float m_run0 = -INFINITY, m_run1 = -INFINITY, l_run0 = 0.f, l_run1 = 0.f;
         bool ok = true;
-        // gate bias of the keys of tile j, loaded one tile ahead so that its global-memory
-        // latency hides behind the previous tile's softmax
-        float gnext[BN / 32];
-#pragma unroll
-        for (int e = 0; e < BN / 32; ++e) {
-            const int key_local = kv0 * BN + e * 32 + lane;
-            gnext[e] = key_local < Mb ? gls[seq0 + key_local] : 0.f;
-        }
-        for (int j = 0; j < n_kv; ++j) {
-            const int s = j & 1;
+        for (int j = 0; ok && j < n_kv; ++j) {
             const int jt = kv0 + j;  // KV tile index within the sequence
-#pragma unroll
-            for (int e = 0; e < BN / 32; ++e) wbias[s * BN + e * 32 + lane] = bscale * gnext[e];
-            if (j + 1 < n_kv) {
-#pragma unroll
-                for (int e = 0; e < BN / 32; ++e) {
-                    const int key_local = (jt + 1) * BN + e * 32 + lane;
-                    gnext[e] = key_local < Mb ? gls[seq0 + key_local] : 0.f;
-                }
-            }
-            __syncwarp();
-            ok = mbar_wait(bar(G_S_FULL + hh), j & 1, abort_flag, status, TG_WHERE_SOFTMAX);
-            if (!ok) break;
-            tc_fence_after();
-            if (r == 0) TG_TRACE_AT(2 + 4 * hh, j);  // S_h(j) ready
-            if (threadIdx.x == 0 && j == 0) TG_CTA_STAMP(3);
-            float x[BN];
-#pragma unroll
-            for (int ch = 0; ch < BN / 32; ++ch) tmem_ld32(tS + ch * 32, x + ch * 32);
-            tmem_wait_ld();
-            if (r == 0) TG_TRACE_AT(3 + 4 * hh, j);  // S_h(j) in registers
-            const float4* bias4 = reinterpret_cast<const float4*>(wbias + s * BN);
-            // Stabiliser: the gate bias is never positive (softplus > 0 times
-            // logsigmoid <= 0), so alpha * max_j s_j bounds every logit alpha * (s_j + b'_j)
-            // from above and the max needs one FMNMX per score.
-            float mp[G2_ILP];
-#pragma unroll
-            for (int i = 0; i < G2_ILP; ++i) mp[i] = -INFINITY;
             const bool diag = (jt == qt);
-            const int lim = q_local - jt * BN;  // on the diagonal tile, columns > lim lie in the future
-            if (!diag) {
-#pragma unroll
-                for (int cc = 0; cc < BN; ++cc) mp[cc % G2_ILP] = fmaxf(mp[cc % G2_ILP], x[cc]);
-            } else {
-#pragma unroll
-                for (int cc = 0; cc < BN; ++cc) {
-                    x[cc] = cc > lim ? -INFINITY : x[cc];
-                    mp[cc % G2_ILP] = fmaxf(mp[cc % G2_ILP], x[cc]);
-                }
-            }
-            float my = mp[0];
-#pragma unroll
-            for (int i = 1; i < G2_ILP; ++i) my = fmaxf(my, mp[i]);
-            const float mx = alpha * my;
-            float corr = 1.0f;
-            bool rescale_o = false;
-            if (j == 0 || mx > m_run + RESCALE_THRESHOLD) {
-                const float m_new = fmaxf(m_run, mx);
-                corr = ex2_approx(m_run - m_new);
-                m_run = m_new;
-                rescale_o = j > 0;
-            }
-            if (r == 0) TG_TRACE_AT(4 + 4 * hh, j);  // max done
-#ifndef TG_ATTN_NO_PINGPONG
-            // this head's turn on the exponentials: head 0 goes first in every tile
-            if (hh == 1 || j > 0) {
-                ok = mbar_wait(bar(G_TOK + hh), hh == 1 ? (j & 1) : ((j - 1) & 1), abort_flag, status,
-                               TG_WHERE_SOFTMAX);
-                if (!ok) break;
-            }
-#endif
-            if (r == 0) TG_TRACE_AT(10 + 3 * hh, j);  // token acquired
-            const float neg_m = -m_run;
-            float sp[G2_ILP];
-#pragma unroll
-            for (int i = 0; i < G2_ILP; ++i) sp[i] = 0.f;
-            uint32_t pk[BN / 2];
-#pragma unroll
-            for (int c4 = 0; c4 < BN / 4; ++c4) {
-                const float4 bv = bias4[c4];
-                const int cc = c4 * 4;
-                const float p0 = ex2_approx(fmaf(alpha, x[cc] + bv.x, neg_m));
-                const float p1 = ex2_approx(fmaf(alpha, x[cc + 1] + bv.y, neg_m));
-                const float p2 = ex2_approx(fmaf(alpha, x[cc + 2] + bv.z, neg_m));
-                const float p3 = ex2_approx(fmaf(alpha, x[cc + 3] + bv.w, neg_m));
-                sp[cc % G2_ILP] += p0;
-                sp[(cc + 1) % G2_ILP] += p1;
-                sp[(cc + 2) % G2_ILP] += p2;
-                sp[(cc + 3) % G2_ILP] += p3;
-                pk[cc / 2] = pack_bf16x2(p0, p1);
-                pk[cc / 2 + 1] = pack_bf16x2(p2, p3);
-            }
-            // P_h over the first 64 columns of S_h: this thread's own lane, whose S loads are complete
-            tmem_st32u(tS, pk);
-            tmem_st32u(tS + 32, pk + 32);
-#ifndef TG_ATTN_NO_PINGPONG
-            mbar_arrive(bar(G_TOK + (hh ^ 1)));  // the other head's turn
-#endif
-            if (r == 0) TG_TRACE_AT(11 + 3 * hh, j);  // exponentials done
-            float sum = 0.f;
-#pragma unroll
-            for (int i = 0; i < G2_ILP; ++i) sum += sp[i];
-            l_run = l_run * corr + sum;
-            if (rescale_o) {
-                // O_h is stable: PV_h(j-1) completed before S_h(j), PV_h(j) waits for P_h(j)
-#pragma unroll
-                for (int ch = 0; ch < HD / 32; ++ch) {
-                    float o[32];
-                    tmem_ld32(tO + ch * 32, o);
+            const int lim = q_local - jt * BN - half * 64;  // on the diagonal tile, own columns > lim are future keys
+#pragma unroll 1
+            for (int hh = 0; hh < 2; ++hh) {
+                const int step = 2 * j + hh;
+                const float alpha = hh ? alpha1 : alpha0;
+                float m_h = hh ? m_run1 : m_run0;
+                const uint32_t tS = tmem + lane_addr + hh * BN;
+                const bool okw = mbar_wait_warp(bar(G_S_FULL + hh), j & 1, abort_flag, status, TG_WHERE_SOFTMAX);
+                if (r == 0 && half == 0) TG_TRACE_AT(2 + 4 * hh, j);  // S_h(j) ready
+                if (threadIdx.x == 0 && step == 0) TG_CTA_STAMP(3);
+                float x[64];
+                float my = -INFINITY;
+                if (okw) {
+                    tc_fence_after();
+                    tmem_ld32(tS + half * 64, x);
+                    tmem_ld32(tS + half * 64 + 32, x + 32);
                     tmem_wait_ld();
+                    if (r == 0 && half == 0) TG_TRACE_AT(3 + 4 * hh, j);  // S_h(j) in registers
+                    if (diag) {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] *= corr;
-                    tmem_st32(tO + ch * 32, o);
+                        for (int cc = 0; cc < 64; ++cc) x[cc] = cc > lim ? -INFINITY : x[cc];
+                    }
+                    // stabiliser: the row max of the biased scores
+                    float mp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                    for (int cc = 0; cc < 64; cc += 2) mp[(cc >> 1) & 3] = max3f(mp[(cc >> 1) & 3], x[cc], x[cc + 1]);
+                    my = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
                 }
+                red[(step & 1) * (2 * BM) + half * BM + r] = my;
+                // every S load of both halves is complete past this barrier, so P may overwrite S
+                if (bar_red_or(1, 256, !okw)) {
+                    ok = false;
+                    break;
+                }
+                my = fmaxf(my, red[(step & 1) * (2 * BM) + (half ^ 1) * BM + r]);
+                // floored so that a tile whose keys all carry an infinite negative bias gives
+                // p = 0 instead of 2^(-inf + inf)
+                const float mx = fmaxf(alpha * my, -1.0e30f);
+                float corr = 1.0f;
+                bool rescale_o = false;
+                if (j == 0 || mx > m_h + RESCALE_THRESHOLD) {
+                    const float m_new = fmaxf(m_h, mx);
+                    corr = ex2_approx(m_h - m_new);
+                    m_h = m_new;
+                    rescale_o = j > 0;
+                }
+                if (hh) m_run1 = m_h; else m_run0 = m_h;
+                if (r == 0 && half == 0) TG_TRACE_AT(4 + 4 * hh, j);  // max done
+                const uint64_t al2 = f32x2_pack(alpha, alpha);
+                const uint64_t nm2 = f32x2_pack(-m_h, -m_h);
+                uint64_t sp[4] = {0ull, 0ull, 0ull, 0ull};
+                uint32_t pk[32];
+#pragma unroll
+                for (int c4 = 0; c4 < 16; ++c4) {
+                    const int cc = c4 * 4;
+                    const uint64_t a0 = f32x2_fma(al2, f32x2_pack(x[cc], x[cc + 1]), nm2);
+                    const uint64_t a1 = f32x2_fma(al2, f32x2_pack(x[cc + 2], x[cc + 3]), nm2);
+                    const float p0 = ex2_approx(f32x2_lo(a0)), p1 = ex2_approx(f32x2_hi(a0));
+                    const float p2 = ex2_approx(f32x2_lo(a1)), p3 = ex2_approx(f32x2_hi(a1));
+                    sp[(2 * c4) & 3] = f32x2_add(sp[(2 * c4) & 3], f32x2_pack(p0, p1));
+                    sp[(2 * c4 + 1) & 3] = f32x2_add(sp[(2 * c4 + 1) & 3], f32x2_pack(p2, p3));
+                    pk[cc / 2] = pack_bf16x2(p0, p1);
+                    pk[cc / 2 + 1] = pack_bf16x2(p2, p3);
+                }
+                // P_h: keys 64 half .. 64 half + 63 -> columns 32 half .. 32 half + 31 of S_h
+                tmem_st32u(tS + half * 32, pk);
+                if (r == 0 && half == 0) TG_TRACE_AT(11 + 3 * hh, j);  // exponentials done
+                const uint64_t s01 = f32x2_add(sp[0], sp[1]), s23 = f32x2_add(sp[2], sp[3]);
+                const uint64_t s4 = f32x2_add(s01, s23);
+                const float tile_sum = f32x2_lo(s4) + f32x2_hi(s4);
+                if (hh) l_run1 = l_run1 * corr + tile_sum; else l_run0 = l_run0 * corr + tile_sum;
+                if (rescale_o) {
+                    // O_h is stable: PV_h(j-1) completed before S_h(j), PV_h(j) waits for P_h(j)
+                    const uint32_t tO = tmem + lane_addr + 2 * BN + hh * HD + half * (HD / 2);
+#pragma unroll
+                    for (int ch = 0; ch < HD / 64; ++ch) {
+                        float o[32];
+                        tmem_ld32(tO + ch * 32, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) o[e] *= corr;
+                        tmem_st32(tO + ch * 32, o);
+                    }
+                }
+                tmem_wait_st();
+                if (r == 0 && half == 0) TG_TRACE_AT(12 + 3 * hh, j);  // P and O stores complete
+                tc_fence_before();
+                mbar_arrive(bar(G_P_FULL + hh));
+                if (r == 0 && half == 0) TG_TRACE_AT(5 + 4 * hh, j);  // P_h(j) stored and signalled
             }
-            tmem_wait_st();
-            if (r == 0) TG_TRACE_AT(12 + 3 * hh, j);  // P and O stores complete
-            tc_fence_before();
-            mbar_arrive(bar(G_P_FULL + hh));
-            if (r == 0) TG_TRACE_AT(5 + 4 * hh, j);  // P_h(j) stored and signalled
         }
         // ---------------------------------------------------------------- epilogue
         if (threadIdx.x == 0) TG_CTA_STAMP(4);
-        if (ok) ok = mbar_wait(bar(G_O_FULL), 0, abort_flag, status, TG_WHERE_SOFTMAX);
+        const bool oko = ok && mbar_wait_warp(bar(G_O_FULL), 0, abort_flag, status, TG_WHERE_SOFTMAX);
+        lred[0 * (2 * BM) + half * BM + r] = l_run0;
+        lred[1 * (2 * BM) + half * BM + r] = l_run1;
+        ok = !bar_red_or(1, 256, !oko);  // uniform over the 256 softmax threads
         if (ok) tc_fence_after();
         if (threadIdx.x == 0) TG_CTA_STAMP(5);
-        const float inv_l = 1.0f / l_run;
-        // Output rows leave through shared memory: thread r stages its row of this head
-        // in the K buffers (free once every MMA has completed), 16-byte chunks XOR-
-        // swizzled by the row so that the staging is conflict-free, and each warp then
-        // writes whole rows with coalesced stores (rows past the sequence end are skipped).
+        // per-head values as scalars: the epilogue loops over the heads without unrolling
+        const float l_tot0 = l_run0 + lred[0 * (2 * BM) + (half ^ 1) * BM + r];
+        const float l_tot1 = l_run1 + lred[1 * (2 * BM) + (half ^ 1) * BM + r];
+        const float m_fin0 = m_run0, m_fin1 = m_run1;
+        // Output rows leave through shared memory: each thread stages its half row of both
+        // heads in the K buffers (free once every MMA has completed), 16-byte chunks XOR-
+        // swizzled by the row so that the staging is conflict-free; then each warp writes 32
+        // whole rows of one head with coalesced stores (rows past the sequence end are skipped).
         constexpr int CH = HD * 2 / 16;  // 16-byte chunks per bf16 row
-        uint8_t* stage = smem + L::OFF_K + hh * (BM * HD * 2);
-        auto stage_row = [&](const float* o32, int ch32, float w) {  // 32 columns starting at ch32 * 32
+        auto stage_row = [&](int hh, const float* o32, int ch32, float w) {  // 32 columns from ch32 * 32
+            uint8_t* stage = smem + L::OFF_K + hh * (BM * HD * 2);
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
                 const int cidx = ch32 * 4 + k4;
@@ -807,14 +911,17 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 *reinterpret_cast<uint4*>(stage + r * (HD * 2) + ((cidx ^ (r & (CH - 1))) << 4)) = v;
             }
         };
-        auto write_rows = [&]() {  // the 4 warps of this head write its 128 staged rows
-            asm volatile("bar.sync %0, 128;" ::"r"(2 + hh) : "memory");
+        auto write_rows = [&]() {  // warp w writes rows 32 (w & 3) .. + 31 of head w >> 2
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+            const int wh = warp >> 2;
+            const uint8_t* stg = smem + L::OFF_K + wh * (BM * HD * 2);
+            const int hw = 2 * pair + wh;
 #pragma unroll 4
             for (int i = 0; i < 32; ++i) {
-                const int rr = lg * 32 + i;
+                const int rr = q4 * 32 + i;
                 if (qt * BM + rr >= Mb) break;
-                const uint8_t* src = stage + rr * (HD * 2);
-                uint16_t* dst = out + (static_cast<size_t>(seq0 + qt * BM + rr) * Hq + h) * HD;
+                const uint8_t* src = stg + rr * (HD * 2);
+                uint16_t* dst = out + (static_cast<size_t>(seq0 + qt * BM + rr) * Hq + hw) * HD;
                 if (HD == 128) {
                     const uint2 v = *reinterpret_cast<const uint2*>(src + (((lane >> 1) ^ (rr & (CH - 1))) << 4) +
                                                                     (lane & 1) * 8);
@@ -828,14 +935,21 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         };
         if (!split) {
             if (ok) {
+#pragma unroll 1
+                for (int hh = 0; hh < 2; ++hh) {
+                    const uint32_t tO = tmem + lane_addr + 2 * BN + hh * HD + half * (HD / 2);
+                    const float lt = hh ? l_tot1 : l_tot0, mf = hh ? m_fin1 : m_fin0;
+                    const float inv_l = 1.0f / lt;
 #pragma unroll
-                for (int ch = 0; ch < HD / 32; ++ch) {
-                    float o[32];
-                    tmem_ld32(tO + ch * 32, o);
-                    tmem_wait_ld();
-                    stage_row(o, ch, inv_l);
+                    for (int ch = 0; ch < HD / 64; ++ch) {
+                        float o[32];
+                        tmem_ld32(tO + ch * 32, o);
+                        tmem_wait_ld();
+                        stage_row(hh, o, half * (HD / 64) + ch, inv_l);
+                    }
+                    if (valid_row && lse && half == 0)
+                        lse[static_cast<size_t>(qg) * Hq + 2 * pair + hh] = (mf + log2f(lt)) / LOG2E;
                 }
-                if (valid_row && lse) lse[static_cast<size_t>(qg) * Hq + h] = (m_run + log2f(l_run)) / LOG2E;
             }
             write_rows();
         } else {
@@ -843,19 +957,24 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             // warp's 32 rows of one column are one 128-byte write; the last chunk to
             // arrive merges (a split query tile has exactly two chunks: chunk ^ 1)
             const int64_t slot = (static_cast<int64_t>(b) * (Hq / 2) + pair) * ws.slots_per_pair + (qt - C);
-            float* po = ws.o + ((slot * ws.max_nch + chunk) * 2 + hh) * (BM * HD) + r;
-            float* pl = ws.lse2 + ((slot * ws.max_nch + chunk) * 2 + hh) * BM + r;
-            const float my_lse = m_run + log2f(l_run);
+            const float my_lse0 = m_fin0 + log2f(l_tot0), my_lse1 = m_fin1 + log2f(l_tot1);
             if (ok) {
+#pragma unroll 1
+                for (int hh = 0; hh < 2; ++hh) {
+                    float* po = ws.o + ((slot * ws.max_nch + chunk) * 2 + hh) * (BM * HD) + r;
+                    const uint32_t tO = tmem + lane_addr + 2 * BN + hh * HD + half * (HD / 2);
+                    const float inv_l = 1.0f / (hh ? l_tot1 : l_tot0);
 #pragma unroll
-                for (int ch = 0; ch < HD / 32; ++ch) {
-                    float o[32];
-                    tmem_ld32(tO + ch * 32, o);
-                    tmem_wait_ld();
+                    for (int ch = 0; ch < HD / 64; ++ch) {
+                        float o[32];
+                        tmem_ld32(tO + ch * 32, o);
+                        tmem_wait_ld();
+                        const int col0 = half * (HD / 2) + ch * 32;
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) po[(ch * 32 + e) * BM] = o[e] * inv_l;
+                        for (int e = 0; e < 32; ++e) po[(col0 + e) * BM] = o[e] * inv_l;
+                    }
+                    if (half == 0) ws.lse2[((slot * ws.max_nch + chunk) * 2 + hh) * BM + r] = hh ? my_lse1 : my_lse0;
                 }
-                *pl = my_lse;
             }
             if (threadIdx.x == 0) TG_CTA_STAMP(8);
             // every softmax thread's partial is written before the barrier; one thread then
@@ -873,26 +992,34 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             asm volatile("bar.sync 1, 256;" ::: "memory");
             if (threadIdx.x == 0) TG_CTA_STAMP(10);
             if (*s_last) {
-                const float* oo = ws.o + ((slot * ws.max_nch + (chunk ^ 1)) * 2 + hh) * (BM * HD) + r;
-                const float other_lse = ws.lse2[((slot * ws.max_nch + (chunk ^ 1)) * 2 + hh) * BM + r];
-                const float mx = fmaxf(my_lse, other_lse);
-                const float e_me = ex2_approx(my_lse - mx), e_ot = ex2_approx(other_lse - mx);
-                const float inv_w = 1.0f / (e_me + e_ot);
-                const float w_me = e_me * inv_w, w_ot = e_ot * inv_w;
                 if (ok) {
+#pragma unroll 1
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int64_t oidx = (slot * ws.max_nch + (chunk ^ 1)) * 2 + hh;
+                        const float* oo = ws.o + oidx * (BM * HD) + r;
+                        const float other_lse = ws.lse2[oidx * BM + r];
+                        const float ml = hh ? my_lse1 : my_lse0;
+                        const float mx = fmaxf(ml, other_lse);
+                        const float e_me = ex2_approx(ml - mx), e_ot = ex2_approx(other_lse - mx);
+                        const float inv_w = 1.0f / (e_me + e_ot);
+                        const float w_me = e_me * inv_w / (hh ? l_tot1 : l_tot0), w_ot = e_ot * inv_w;
+                        const uint32_t tO = tmem + lane_addr + 2 * BN + hh * HD + half * (HD / 2);
 #pragma unroll
-                    for (int ch = 0; ch < HD / 32; ++ch) {
-                        float ot[32];
+                        for (int ch = 0; ch < HD / 64; ++ch) {
+                            const int col0 = half * (HD / 2) + ch * 32;
+                            float ot[32];
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) ot[e] = oo[(ch * 32 + e) * BM];
-                        float o[32];
-                        tmem_ld32(tO + ch * 32, o);
-                        tmem_wait_ld();
+                            for (int e = 0; e < 32; ++e) ot[e] = oo[(col0 + e) * BM];
+                            float o[32];
+                            tmem_ld32(tO + ch * 32, o);
+                            tmem_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] = fmaf(w_me * inv_l, o[e], w_ot * ot[e]);  // own O unnormalised
-                        stage_row(o, ch, 1.0f);
+                            for (int e = 0; e < 32; ++e) o[e] = fmaf(w_me, o[e], w_ot * ot[e]);  // own O unnormalised
+                            stage_row(hh, o, half * (HD / 64) + ch, 1.0f);
+                        }
+                        if (valid_row && lse && half == 0)
+                            lse[static_cast<size_t>(qg) * Hq + 2 * pair + hh] = (mx + log2f(e_me + e_ot)) / LOG2E;
                     }
-                    if (valid_row && lse) lse[static_cast<size_t>(qg) * Hq + h] = (mx + log2f(e_me + e_ot)) / LOG2E;
                 }
                 write_rows();
                 if (threadIdx.x == 0) ws.cnt[slot] = 0;  // ready for the next call

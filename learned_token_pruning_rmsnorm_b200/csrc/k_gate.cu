@@ -38,6 +38,30 @@ __global__ void gate_prepare_kernel(const uint16_t* __restrict__ gamma, const ui
     }
 }
 
+// Optional device trace (builds with -DTG_TRACE only): clock64 stamps of the
+// first CTA's pipeline per k-block (producer issue, MMA start, MMA issued,
+// sum of squares done) and globaltimer start/end stamps of every CTA.
+#ifdef TG_TRACE
+__device__ unsigned long long g_score_trace[4 * 128];
+__device__ unsigned long long g_score_cta[512 * 2];
+#define SC_TRACE(point, k)                                                                  \
+    do {                                                                                    \
+        if (blockIdx.x == 0 && (k) < 128)                                                   \
+            g_score_trace[(point) * 128 + (k)] = static_cast<unsigned long long>(clock64()); \
+    } while (0)
+#define SC_CTA(slot)                                                                          \
+    do {                                                                                      \
+        if (blockIdx.x < 512) g_score_cta[blockIdx.x * 2 + (slot)] = globaltimer();            \
+    } while (0)
+#else
+#define SC_TRACE(point, k) \
+    do {                   \
+    } while (0)
+#define SC_CTA(slot) \
+    do {             \
+    } while (0)
+#endif
+
 constexpr int KB = 64;                // channels per pipeline stage (one 128-byte swizzle row)
 constexpr int TILE_A = 128 * KB * 2;  // one 128-row slice: 16 KB
 
@@ -104,6 +128,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nkb = D / KB;
+    if (threadIdx.x == 0) SC_CTA(0);
 
     for (int j = threadIdx.x; j < I; j += blockDim.x) {
         s_b1[j] = b1[j];
@@ -148,6 +173,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                         break;
                     }
                     const uint32_t st = sbase + s * stage_bytes;
+                    SC_TRACE(0, it);
                     mbar_expect_tx(full(s), stage_bytes);
 #pragma unroll
                     for (int a = 0; a < NACC; ++a)
@@ -183,6 +209,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                         break;
                     }
                     tc_fence_after();
+                    SC_TRACE(1, it);
                     const uint32_t st = sbase + s * stage_bytes;
 #pragma unroll
                     for (int kk = 0; kk < KB / 16; ++kk) {
@@ -193,6 +220,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                                         idesc, (kb | kk) != 0 ? 1u : 0u);
                     }
                     mma_commit(empty(s));
+                    SC_TRACE(2, it);
                 }
                 if (ok) mma_commit(acc_full);
             }
@@ -218,7 +246,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
             for (int kb = 0; kb < nkb; ++kb, ++it) {
                 const int s = static_cast<int>(it % STAGES);
                 const int use = static_cast<int>(it / STAGES);
-                if (!mbar_wait(full(s), use & 1, abort_flag, status, TG_WHERE_SOFTMAX)) {
+                if (!mbar_wait_warp(full(s), use & 1, abort_flag, status, TG_WHERE_SOFTMAX)) {
                     ok = false;
                     break;
                 }
@@ -240,9 +268,10 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(empty(s));
+                if (warp == 2 && lane == 0) SC_TRACE(3, it);
             }
             if (!ok) break;
-            if (!mbar_wait(acc_full, tcount & 1, abort_flag, status, TG_WHERE_SOFTMAX)) break;
+            if (!mbar_wait_warp(acc_full, tcount & 1, abort_flag, status, TG_WHERE_SOFTMAX)) break;
             tc_fence_after();
             const float rr = rsqrtf(ss / static_cast<float>(D) + eps);
             float acc_s = 0.f;
@@ -263,6 +292,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
 
     tc_fence_before();
     __syncthreads();
+    if (threadIdx.x == 0) SC_CTA(1);
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
@@ -292,6 +322,13 @@ cudaError_t launch_score_tc(const uint16_t* hidden, const int32_t* cu_seqlens, c
 }
 
 }  // namespace
+
+#ifdef TG_TRACE
+extern "C" int tg_trace_read_score(unsigned long long* pipe, unsigned long long* ctas) {
+    if (cudaMemcpyFromSymbol(pipe, g_score_trace, sizeof(g_score_trace)) != cudaSuccess) return 1;
+    return cudaMemcpyFromSymbol(ctas, g_score_cta, sizeof(g_score_cta)) == cudaSuccess ? 0 : 1;
+}
+#endif
 
 cudaError_t launch_gate_prepare(const uint16_t* gamma, const uint16_t* W1, int D, int I, uint16_t* Wg,
                                 cudaStream_t st) {

@@ -153,6 +153,7 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
     const bool need_gls = emit && kk > 0;  // some prunable token is kept: its logsigmoid is emitted
     if (cached && (do_select || need_gls)) {
         uint32_t lmin = 0xFFFFFFFFu, lmax = 0u;
+#pragma unroll 8
         for (int64_t t = k0 + tid; t < k1; t += SEL_THREADS) {
             const uint32_t key = score_key(__ldg(scores + t));
             skeys[t - k0] = key;
@@ -234,6 +235,7 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
             hist[tid] = 0;
             hist[tid + SEL_THREADS] = 0;
             __syncthreads();
+#pragma unroll 4
             for (int64_t t = k0 + tid; t < k1; t += SEL_THREADS) {
                 const uint32_t key = cached ? skeys[t - k0] : score_key(__ldg(scores + t));
                 const uint32_t d = key - lo;  // wraps for keys below lo: excluded by the range test
@@ -336,6 +338,7 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
 
     // warp totals: kept tokens and (for the tie ranking) keys equal to thr
     int my_kept = 0, my_eq = 0;
+#pragma unroll 4
     for (int64_t base = w0; base < w1; base += 32) {
         bool kept, eq;
         flags(base + lane, kept, eq);
@@ -377,7 +380,9 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
             }
         }
     }
+    SEL_TRACE(6);
     cluster_arrive_release();  // no remote reads after this point
+    SEL_TRACE(7);
     // kept_before counts the tie-ranked keys as not kept; min(eq_before, need_eq) of
     // those before this warp's run are kept
     int64_t m = m0 + kept_before + (all_eq_kept ? 0 : min(eq_before, need_eq));

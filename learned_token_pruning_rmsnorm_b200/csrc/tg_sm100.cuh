@@ -95,6 +95,19 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     }
 }
 
+// mbar_wait for a whole warp: lane 0 polls, the warp synchronises on its
+// result (32 lanes polling one barrier would multiply the shared-memory
+// traffic that competes with the tensor core's operand reads).  Must be
+// called by all 32 lanes.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* status,
+                                               int where) {
+    bool ok = true;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag, status, where);
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    __syncwarp();
+    return ok;
+}
+
 // ------------------------------------------------------------------ TMA
 
 // 2D tiled load of box {x, y} (x innermost, in elements) into shared memory,
@@ -250,6 +263,19 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo_
     d |= static_cast<uint64_t>(1) << 46;  // descriptor version for sm_100
     d |= static_cast<uint64_t>(2) << 61;  // SWIZZLE_128B
     return d;
+}
+
+// Shared-memory matrix descriptor without swizzle (layout type 0), K-major:
+// core matrices of 8 rows x 16 bytes stored contiguously (row i at +16 i);
+// lbo = byte distance between core matrices adjacent in K, sbo = byte
+// distance between 8-row groups.  The start address must be 16-byte aligned.
+__device__ __forceinline__ uint64_t smem_desc_noswz(uint32_t addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((addr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    d |= static_cast<uint64_t>(1) << 46;  // descriptor version for sm_100
+    return d;                             // layout type 0: no swizzle
 }
 
 // Instruction descriptor of tcgen05.mma kind::f16 with bf16 A/B, fp32 D.
