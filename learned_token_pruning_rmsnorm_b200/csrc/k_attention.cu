@@ -592,7 +592,7 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             mbar_init(bar(G_V_FULL + s), 1);
             mbar_init(bar(G_V_EMPTY + s), 1);
             mbar_init(bar(G_S_FULL + s), 1);
-            mbar_init(bar(G_P_FULL + s), 256);
+            mbar_init(bar(G_P_FULL + s), 8);  // one arrival per softmax warp
         }
         mbar_init(bar(G_O_FULL), 1);
         mbar_init(bar(G_DRAIN), 1);
@@ -877,7 +877,8 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 tmem_wait_st();
                 if (r == 0 && half == 0) TG_TRACE_AT(12 + 3 * hh, j);  // P and O stores complete
                 tc_fence_before();
-                mbar_arrive(bar(G_P_FULL + hh));
+                __syncwarp();  // every lane's P and O stores are complete and fenced
+                if (lane == 0) mbar_arrive(bar(G_P_FULL + hh));  // one arrival per warp
                 if (r == 0 && half == 0) TG_TRACE_AT(5 + 4 * hh, j);  // P_h(j) stored and signalled
             }
         }
