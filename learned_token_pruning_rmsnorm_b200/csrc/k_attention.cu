@@ -65,19 +65,16 @@ enum : int {
 // pipeline hand-offs of the CTA at blockIdx (0, 0, 0), 64 KV tiles at most.
 #ifdef TG_TRACE
 __device__ unsigned long long g_attn_trace[24 * 64];  // points 0..23 x 64 tiles
-__device__ unsigned long long g_attn_cta[4096 * 16];  // per CTA: phase stamps (ns), SM id | n_kv
-#ifndef TG_TRACE_CTA
-#define TG_TRACE_CTA 0
-#endif
+__device__ unsigned long long g_attn_cta[4096 * 12];  // per CTA: phase stamps (ns), SM id | n_kv
 #define TG_TRACE_AT(point, j)                                                              \
     do {                                                                                   \
-        if (blockIdx.x == TG_TRACE_CTA && blockIdx.y == 0 && blockIdx.z == 0 && (j) < 64)  \
+        if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && (j) < 64)             \
             g_attn_trace[(point) * 64 + (j)] = static_cast<unsigned long long>(clock64()); \
     } while (0)
 #define TG_CTA_STAMP(slot)                                                                            \
     do {                                                                                              \
         const unsigned idx_ = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);        \
-        if (idx_ < 4096) g_attn_cta[idx_ * 16 + (slot)] = globaltimer();                              \
+        if (idx_ < 4096) g_attn_cta[idx_ * 12 + (slot)] = globaltimer();                              \
     } while (0)
 #else
 #define TG_CTA_STAMP(slot) \
@@ -101,12 +98,6 @@ __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity, int* s
 __device__ __forceinline__ float ldg_early(const float* p) {
     float v;
     asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v) : "l"(p));
-    return v;
-}
-
-__device__ __forceinline__ int ldg_early_i32(const int32_t* p) {
-    int v;
-    asm volatile("ld.global.nc.s32 %0, [%1];" : "=r"(v) : "l"(p));
     return v;
 }
 
@@ -444,30 +435,23 @@ gated_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
 }
 
 // ---------------------------------------------------------------------------
-// Two query heads of one KV head per unit (GQA groups of even size), persistent.
-//
-// One CTA per SM loops over work units: a unit is (sequence, head pair, query
-// tile, causal KV chunk).  Units are ordered by decreasing cost (KV tiles) and
-// dealt to the CTAs in serpentine order (CTA order reversed on every other
-// round), which balances the per-SM totals; each role overlaps the start of
-// the next unit with the end of the current one (the next Q loads once the
-// last S MMA has read the current Q, the next S MMAs follow the last PV, and
-// the next PV waits only until the epilogue has read O out of TMEM).
+// Two query heads of one KV head per CTA (GQA groups of even size).
 //
 // 320 threads: warps 0-7 = softmax of both heads in turn (thread = one row,
-// one half of the columns), warp 8 = TMA producer (+ the bias operands),
-// warp 9 = MMA issuer.  TMEM (512 columns): S0 | S1 | O0 | O1; P_h (bf16, two
-// keys per column) is written over the first 64 columns of S_h and read from
-// TMEM as the A operand of the PV MMA.  The MMA issuer interleaves
+// one half of the columns), warp 8 = TMA producer, warp 9 = MMA issuer.
+// Both heads share every K/V tile.  TMEM (512 columns): S0 | S1 | O0 | O1;
+// P_h (bf16, two keys per column) is written over the first 64 columns of
+// S_h and read from TMEM as the A operand of the PV MMA.  The MMA issuer
+// interleaves
 //     S0(j) S1(j) | PV0(j) S0(j+1) | PV1(j) S1(j+1) | ...
 // and the softmax warps take head 0 of tile j, head 1 of tile j, head 0 of
 // tile j+1, ..., so that one head's softmax overlaps the other head's
-// tensor-core work; tcgen05 operations of one thread execute in issue order,
-// which is what lets S_h(j+1) overwrite P_h(j) right after PV_h(j), and what
-// makes the commit after S_h(j) also cover PV_h(j-1) (so the softmax may
-// rescale O_h as soon as S_h(j) is complete).
+// tensor-core work;
+// tcgen05 operations of one thread execute in issue order, which is what
+// lets S_h(j+1) overwrite P_h(j) right after PV_h(j), and what makes the
+// commit after S_h(j) also cover PV_h(j-1) (so the softmax may rescale O_h
+// as soon as S_h(j) is complete).
 constexpr int G2_THREADS = 320;
-constexpr int G2_CU_CACHE = 256;  // cu_kept entries cached in shared memory
 
 template <int HD>
 struct G2Smem {
@@ -483,10 +467,8 @@ struct G2Smem {
     static constexpr int OFF_KX = OFF_QX + 2 * EXT;      // [stage]
     // partial row maxima [parity][half][row] (2 KB) and partial row sums [head][half][row] (2 KB)
     static constexpr int OFF_RED = OFF_KX + 2 * EXT;
-    static constexpr int OFF_ALPHA = OFF_RED + 2 * 2 * BM * 4 + 2 * 2 * BM * 4;  // [unit parity][head][row]
-    static constexpr int OFF_CU = OFF_ALPHA + 2 * 2 * BM * 4;
-    static constexpr int OFF_BAR = OFF_CU + G2_CU_CACHE * 4;
-    static constexpr int NUM_BARS = 20;
+    static constexpr int OFF_BAR = OFF_RED + 2 * 2 * BM * 4 + 2 * 2 * BM * 4;
+    static constexpr int NUM_BARS = 18;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int BYTES = OFF_MISC + 16;
     static constexpr int ALLOC = BYTES + 1024;
@@ -495,13 +477,14 @@ struct G2Smem {
 
 enum : int {
     G_Q_FULL = 0, G_K_FULL = 1, G_K_EMPTY = 3, G_V_FULL = 5, G_V_EMPTY = 7, G_S_FULL = 9, G_P_FULL = 11,
-    G_O_FULL = 13, G_DRAIN = 14, G_Q_EMPTY = 15, G_O_EMPTY = 16, G_A_FULL = 17  // + unit parity
+    G_O_FULL = 13, G_DRAIN = 14
 };
 
 // Causal work split.  Query tile qt of a sequence needs KV tiles 0..qt.  With
 // a chunk length C, it is cut into ceil((qt+1)/C) units of at most C KV
-// tiles; units are numbered heaviest first.  units_below(x) counts the units
-// of query tiles 0..x-1:  sum_{L=1..x} ceil(L/C) = C*a*(a+1)/2 + r*(a+1), x = a*C + r.
+// tiles; units are numbered heaviest query tile first, so the block
+// scheduler hands out long units first.  units_below(x) counts the units of
+// query tiles 0..x-1:  sum_{L=1..x} ceil(L/C) = C*a*(a+1)/2 + r*(a+1), x = a*C + r.
 __device__ __forceinline__ int64_t units_below(int x, int C) {
     const int64_t a = x / C, r = x % C;
     return C * a * (a + 1) / 2 + r * (a + 1);
@@ -518,32 +501,32 @@ struct SplitWs {
     int slots_per_pair;  // n_qt_max - C (query tiles that may be split)
 };
 
-// One unit of work.  Slot s (0 .. units_max * B * pairs - 1) is y-major:
-// s = (y * B + b) * pairs + pair, y = rank of the unit by cost within its
-// sequence; slots with y beyond the sequence's unit count are empty.
-struct G2Unit {
-    int b, pair, qt, chunk, C, n_kv, kv0, nch, seq0, Mb;
-    bool valid;
-};
+template <int HD>
+__global__ void __launch_bounds__(G2_THREADS, 1)
+gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const int32_t* __restrict__ cu_kept,
+                       const int32_t* __restrict__ pos, const int32_t* __restrict__ rank,
+                       const float* __restrict__ gls, const float* __restrict__ g, const float* __restrict__ c,
+                       float sm_scale, int Hq, int Hkv, int n_qt_max, int kv_chunk, SplitWs ws,
+                       uint16_t* __restrict__ out, float* __restrict__ lse, int* __restrict__ status) {
+    using L = G2Smem<HD>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
-__device__ __forceinline__ G2Unit g2_decode(int64_t slot, int pairs, int B, int kv_chunk, const int32_t* cu_kept,
-                                            const int* s_cu) {
-    G2Unit U{};
-    const int64_t per_y = static_cast<int64_t>(B) * pairs;
-    const int64_t y = slot / per_y;
-    const int rem = static_cast<int>(slot - y * per_y);
-    U.b = rem / pairs;
-    U.pair = rem - U.b * pairs;
-    const int c0 = U.b < G2_CU_CACHE - 1 ? s_cu[U.b] : cu_kept[U.b];
-    const int c1 = U.b < G2_CU_CACHE - 1 ? s_cu[U.b + 1] : cu_kept[U.b + 1];
-    U.seq0 = c0;
-    U.Mb = c1 - c0;
-    const int n_qt = (U.Mb + BM - 1) / BM;
-    U.C = min(kv_chunk, max(n_qt, 1));
-    const int C = U.C;
-    U.valid = n_qt > 0 && y < units_below(n_qt, C);
-    if (!U.valid) return U;
-    int64_t u = y;
+    const int pair = blockIdx.x;            // query heads 2*pair and 2*pair+1
+    const int b = blockIdx.z;
+#ifdef TG_TRACE
+    const unsigned long long trace_t0 = globaltimer();
+#endif
+    const int seq0 = cu_kept[b];
+    const int Mb = cu_kept[b + 1] - seq0;
+    const int n_qt = (Mb + BM - 1) / BM;
+    const int C = min(kv_chunk, max(n_qt, 1));
+    // unit -> (query tile, chunk) in order of decreasing cost (KV tiles), so that
+    // the block scheduler hands out the longest units first
+    int64_t u = blockIdx.y;
+    const int64_t n_units = units_below(n_qt, C);
+    if (u >= n_units) return;
     int qt = 0, chunk = 0;
     if (C >= n_qt) {
         qt = n_qt - 1 - static_cast<int>(u);  // unsplit: query tile qt costs qt + 1
@@ -566,63 +549,43 @@ __device__ __forceinline__ G2Unit g2_decode(int64_t slot, int pairs, int B, int 
             }
         }
     }
-    U.qt = qt;
-    U.chunk = chunk;
-    U.nch = (qt + C) / C;  // ceil((qt + 1) / C), 1 or 2
-    U.kv0 = chunk * C;
-    const int kv1 = min(qt + 1, U.kv0 + C);
-    U.n_kv = kv1 - U.kv0;  // the chunk holding the diagonal tile is the last one
-    return U;
-}
-
-// slot of the CTA's k-th unit in serpentine order (-1 past the end)
-__device__ __forceinline__ int64_t g2_slot(int k, int64_t total) {
-    const int64_t G = gridDim.x;
-    const int64_t s = static_cast<int64_t>(k) * G + ((k & 1) ? (G - 1 - blockIdx.x) : blockIdx.x);
-    return s < total ? s : -1;
-}
-
-template <int HD>
-__global__ void __launch_bounds__(G2_THREADS, 1)
-gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                       const __grid_constant__ CUtensorMap tmV, const int32_t* __restrict__ cu_kept,
-                       const int32_t* __restrict__ pos, const int32_t* __restrict__ rank,
-                       const float* __restrict__ gls, const float* __restrict__ g, const float* __restrict__ c,
-                       float sm_scale, int B, int Hq, int Hkv, int units_max, int kv_chunk, SplitWs ws,
-                       uint16_t* __restrict__ out, float* __restrict__ lse, int* __restrict__ status) {
-    using L = G2Smem<HD>;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-#ifdef TG_TRACE
-    const unsigned long long trace_t0 = globaltimer();
-#endif
-    const int pairs = Hq / 2;
-    const int64_t total = static_cast<int64_t>(units_max) * B * pairs;
+    const int nch = (qt + C) / C;  // ceil((qt + 1) / C), 1 or 2
+    const int kv0 = chunk * C;
+    const int kv1 = min(qt + 1, kv0 + C);
+    const int n_kv = kv1 - kv0;  // the chunk holding the diagonal tile is the last one
+    const bool split = nch > 1;
+    const int hk = (2 * pair) / (Hq / Hkv);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     const uint32_t sbase = smem_u32(smem);
     const uint32_t sQ = sbase + L::OFF_Q, sK0 = sbase + L::OFF_K, sV0 = sbase + L::OFF_V;
-    const uint32_t sQX = sbase + L::OFF_QX, sKX = sbase + L::OFF_KX;
     auto bar = [&](int i) { return sbase + L::OFF_BAR + 8u * static_cast<uint32_t>(i); };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
-    int* s_cu = reinterpret_cast<int*>(smem + L::OFF_CU);
+    const uint32_t sQX = sbase + L::OFF_QX, sKX = sbase + L::OFF_KX;
 
-    for (int i = threadIdx.x; i < min(B + 1, G2_CU_CACHE); i += blockDim.x) s_cu[i] = cu_kept[i];
-    // Gate bias as one more k-step of S = Q K^T: row q of Q_ext holds (bh, bl, bh, bl) and
-    // row j of K_ext holds (gh, gh, gl, gl), the bf16 high and low parts of
-    // bscale_h = softplus(g_h) / sm_scale and of gls_j, so that the extra products add
-    // bscale_h * gls_j to S with about 2^-16 relative error; the other 12 columns are zero.
-    // K cores 8..15 of all four tiles are zero throughout; the producer writes the rest.
+    // Gate bias as one more k-step of the S = Q K^T product: row q of Q_ext holds
+    // (bh, bl, bh, bl) and row j of K_ext holds (gh, gh, gl, gl), the bf16 high and low
+    // parts of bscale_h = softplus(g_h) / sm_scale and of gls_j, so that the extra products
+    // add bscale_h * gls_j to S with about 2^-16 relative error; the other 12 columns are
+    // zero.  K cores 8..15 of all four tiles are zero throughout; K_ext rows are written by
+    // the producer per KV tile.
     for (int i = threadIdx.x; i < 4 * (BM / 8) * 8; i += blockDim.x) {
         const int tile = i / ((BM / 8) * 8), rem = i % ((BM / 8) * 8);
         *reinterpret_cast<uint4*>(smem + L::OFF_QX + tile * L::EXT + (rem >> 3) * 256 + 128 + (rem & 7) * 16) =
             make_uint4(0u, 0u, 0u, 0u);
     }
+    if (threadIdx.x < 2 * BM) {
+        const int hh = threadIdx.x / BM, r = threadIdx.x % BM;
+        const float bscale = softplus_f(g[2 * pair + hh]) / sm_scale;
+        const uint32_t hl = bf16_hi_lo(bscale);
+        *reinterpret_cast<uint4*>(smem + L::OFF_QX + hh * L::EXT + (r >> 3) * 256 + (r & 7) * 16) =
+            make_uint4(hl, hl, 0u, 0u);
+    }
     fence_proxy_async_smem();
+
     if (threadIdx.x == 0) {
         mbar_init(bar(G_Q_FULL), 1);
-        mbar_init(bar(G_Q_EMPTY), 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(bar(G_K_FULL + s), 1);
             mbar_init(bar(G_K_EMPTY + s), 1);
@@ -632,9 +595,6 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             mbar_init(bar(G_P_FULL + s), 8);  // one arrival per softmax warp
         }
         mbar_init(bar(G_O_FULL), 1);
-        mbar_init(bar(G_O_EMPTY), 8);  // one arrival per softmax warp once O is read
-        mbar_init(bar(G_A_FULL + 0), 1);
-        mbar_init(bar(G_A_FULL + 1), 1);
         mbar_init(bar(G_DRAIN), 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -647,173 +607,77 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-#ifdef TG_TRACE
-    if (threadIdx.x == 0 && blockIdx.x < 4096)
-        for (int i = 2; i < 16; ++i) g_attn_cta[blockIdx.x * 16 + i] = 0;
-#endif
     if (threadIdx.x == 0) TG_CTA_STAMP(1);
 
     if (warp == 8) {
         // ---------------------------------------------------------------- TMA producer
-        // The whole warp writes the bias operands (Q_ext per unit, K_ext per KV tile, lane l:
-        // rows 4l .. 4l+3); lane 0 issues the copies.  Q and Q_ext are reloaded once the last
-        // S MMA of the previous unit has completed; K_ext(stage) is released with K(stage).
+        // The whole warp writes the K_ext rows of each KV tile (lane l: keys 4l .. 4l+3);
+        // lane 0 issues the copies.  K_ext(stage) is released with K(stage).
         if (lane == 0) {
             prefetch_tmap(&tmQ);
             prefetch_tmap(&tmK);
             prefetch_tmap(&tmV);
+            mbar_expect_tx(bar(G_Q_FULL), 2 * BM * HD * 2);
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                for (int hf = 0; hf < HD / 64; ++hf)
+                    tma_load_2d(sQ + hh * L::TILE_Q + hf * BM * 128, &tmQ, (2 * pair + hh) * HD + hf * 64,
+                                seq0 + qt * BM, bar(G_Q_FULL));
         }
-        int q_issued = 0, k_issued[2] = {0, 0}, v_issued[2] = {0, 0};
-        uint32_t gt = 0;  // KV tiles streamed by this CTA so far (all units)
-        int nu = 0;       // units started
-        bool okp = true;
-        // the next unit, its gate gains and its first tile's gls are looked up one unit ahead
-        auto next_unit = [&](int& k, G2Unit& U) {
-            for (;; ++k) {
-                const int64_t slot = g2_slot(k, total);
-                if (slot < 0) return false;
-                U = g2_decode(slot, pairs, B, kv_chunk, cu_kept, s_cu);
-                if (U.valid) return true;
+        int k_issued[2] = {0, 0}, v_issued[2] = {0, 0};
+        float gk[4];  // gls of this lane's keys of the next tile (0 past the sequence end)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int key_local = kv0 * BN + lane * 4 + i;
+            gk[i] = key_local < Mb ? ldg_early(gls + seq0 + key_local) : 0.f;
+        }
+        for (int j = 0; j < n_kv; ++j) {
+            const int s = j & 1;
+            float gcur[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) gcur[i] = gk[i];
+            if (j + 1 < n_kv) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int key_local = (kv0 + j + 1) * BN + lane * 4 + i;
+                    gk[i] = key_local < Mb ? ldg_early(gls + seq0 + key_local) : 0.f;
+                }
             }
-        };
-        float gk[4];    // gls of this lane's keys of the next tile (0 past the sequence end)
-        float gg[2];    // g of the next unit's two heads
-        float cc[2];    // c of the next unit's two heads
-        int pr[4][2];   // pos and rank of this lane's query rows 4 lane .. 4 lane + 3 of the next unit
-        auto prefetch_unit = [&](const G2Unit& U) {
+            if (j >= 2 && !mbar_wait_warp(bar(G_K_EMPTY + s), ((j - 2) >> 1) & 1, abort_flag, status,
+                                          TG_WHERE_PRODUCER))
+                break;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const int key_local = U.kv0 * BN + lane * 4 + i;
-                gk[i] = key_local < U.Mb ? ldg_early(gls + U.seq0 + key_local) : 0.f;
-                const int q_local = U.qt * BM + lane * 4 + i;
-                pr[i][0] = q_local < U.Mb ? ldg_early_i32(pos + U.seq0 + q_local) : 1;
-                pr[i][1] = q_local < U.Mb ? ldg_early_i32(rank + U.seq0 + q_local) : 1;
+                const int r = lane * 4 + i;
+                const uint32_t hl = bf16_hi_lo(gcur[i]);
+                *reinterpret_cast<uint4*>(smem + L::OFF_KX + s * L::EXT + (r >> 3) * 256 + (r & 7) * 16) =
+                    make_uint4(__byte_perm(hl, 0u, 0x1010), __byte_perm(hl, 0u, 0x3232), 0u, 0u);
             }
-            gg[0] = ldg_early(g + 2 * U.pair);
-            gg[1] = ldg_early(g + 2 * U.pair + 1);
-            cc[0] = ldg_early(c + 2 * U.pair);
-            cc[1] = ldg_early(c + 2 * U.pair + 1);
-        };
-        int kn = 0;
-        G2Unit Un{};
-        bool have = next_unit(kn, Un);
-        if (have) prefetch_unit(Un);
-        while (okp && have) {
-            const G2Unit U = Un;
-            ++kn;
-            const int hk = (2 * U.pair) / (Hq / Hkv);
-            const uint32_t hl0 = bf16_hi_lo(softplus_f(gg[0]) / sm_scale);
-            const uint32_t hl1 = bf16_hi_lo(softplus_f(gg[1]) / sm_scale);
-            if (nu > 0 && !mbar_wait_warp(bar(G_Q_EMPTY), (nu - 1) & 1, abort_flag, status, TG_WHERE_PRODUCER)) {
-                okp = false;
-                break;
-            }
-            for (int i = lane; i < 2 * BM; i += 32) {
-                const int hh = i / BM, r = i % BM;
-                const uint32_t hl = hh ? hl1 : hl0;
-                *reinterpret_cast<uint4*>(smem + L::OFF_QX + hh * L::EXT + (r >> 3) * 256 + (r & 7) * 16) =
-                    make_uint4(hl, hl, 0u, 0u);
-            }
-            fence_proxy_async_smem();  // Q_ext is read by the tensor core (async proxy)
+            fence_proxy_async_smem();  // K_ext is read by the tensor core (async proxy)
             __syncwarp();
             if (lane == 0) {
-#ifdef TG_TRACE
-                if (nu == 1 && blockIdx.x < 4096) g_attn_cta[blockIdx.x * 16 + 8] = globaltimer();  // Q of unit 2 issued
-#endif
-                mbar_expect_tx(bar(G_Q_FULL), 2 * BM * HD * 2);
+                mbar_expect_tx(bar(G_K_FULL + s), BN * HD * 2);
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-                    for (int hf = 0; hf < HD / 64; ++hf)
-                        tma_load_2d(sQ + hh * L::TILE_Q + hf * BM * 128, &tmQ, (2 * U.pair + hh) * HD + hf * 64,
-                                    U.seq0 + U.qt * BM, bar(G_Q_FULL));
-                ++q_issued;
+                for (int hf = 0; hf < HD / 64; ++hf)
+                    tma_load_2d(sK0 + s * L::TILE_KV + hf * BN * 128, &tmK, hk * HD + hf * 64,
+                                seq0 + (kv0 + j) * BN, bar(G_K_FULL + s));
+                ++k_issued[s];
             }
-            // alpha_q = sm_scale * log2(e) / tau_q of this unit's rows for both heads, for the
-            // softmax warps (its buffer was last read two units ago: this point is past the
-            // previous unit's last S MMA, which the softmax warps had to reach first)
-            {
-                float* s_alpha = reinterpret_cast<float*>(smem + L::OFF_ALPHA) + (nu & 1) * 2 * BM;
+            if (j >= 2 && !mbar_wait_warp(bar(G_V_EMPTY + s), ((j - 2) >> 1) & 1, abort_flag, status,
+                                          TG_WHERE_PRODUCER))
+                break;
+            if (lane == 0) {
+                mbar_expect_tx(bar(G_V_FULL + s), BN * HD * 2);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int row = lane * 4 + i;
-                    const bool valid_row = U.qt * BM + row < U.Mb;
-                    const float ratio_log =
-                        valid_row ? logf(static_cast<float>(pr[i][0]) / static_cast<float>(pr[i][1])) : 0.f;
-                    const float inv_tau0 = valid_row ? 1.0f / (1.0f + cc[0] * ratio_log) : 1.0f;
-                    const float inv_tau1 = valid_row ? 1.0f / (1.0f + cc[1] * ratio_log) : 1.0f;
-                    s_alpha[row] = sm_scale * LOG2E * inv_tau0;
-                    s_alpha[BM + row] = sm_scale * LOG2E * inv_tau1;
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(G_A_FULL + (nu & 1)));
+                for (int hf = 0; hf < HD / 64; ++hf)
+                    tma_load_2d(sV0 + s * L::TILE_KV + hf * BN * 128, &tmV, hk * HD + hf * 64,
+                                seq0 + (kv0 + j) * BN, bar(G_V_FULL + s));
+                ++v_issued[s];
             }
-            for (int j = 0; j < U.n_kv; ++j, ++gt) {
-                const int s = static_cast<int>(gt & 1);
-                const uint32_t use = gt >> 1;
-                float gcur[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) gcur[i] = gk[i];
-                if (j + 1 < U.n_kv) {
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int key_local = (U.kv0 + j + 1) * BN + lane * 4 + i;
-                        gk[i] = key_local < U.Mb ? ldg_early(gls + U.seq0 + key_local) : 0.f;
-                    }
-                } else {
-                    have = next_unit(kn, Un);
-                    if (have) prefetch_unit(Un);
-                }
-                if (use > 0 && !mbar_wait_warp(bar(G_K_EMPTY + s), (use - 1) & 1, abort_flag, status,
-                                               TG_WHERE_PRODUCER)) {
-                    okp = false;
-                    break;
-                }
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int r = lane * 4 + i;
-                    const uint32_t hl = bf16_hi_lo(gcur[i]);
-                    *reinterpret_cast<uint4*>(smem + L::OFF_KX + s * L::EXT + (r >> 3) * 256 + (r & 7) * 16) =
-                        make_uint4(__byte_perm(hl, 0u, 0x1010), __byte_perm(hl, 0u, 0x3232), 0u, 0u);
-                }
-                fence_proxy_async_smem();  // K_ext is read by the tensor core (async proxy)
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_expect_tx(bar(G_K_FULL + s), BN * HD * 2);
-#pragma unroll
-                    for (int hf = 0; hf < HD / 64; ++hf)
-                        tma_load_2d(sK0 + s * L::TILE_KV + hf * BN * 128, &tmK, hk * HD + hf * 64,
-                                    U.seq0 + (U.kv0 + j) * BN, bar(G_K_FULL + s));
-                    ++k_issued[s];
-                }
-                // All CTAs start together: let Q and the first K land before the rest of the
-                // ring is requested, so that the first S MMA does not wait behind every
-                // CTA's V and second K (an observing wait; it consumes nothing).
-                if (nu == 0 && j == 0 &&
-                    !(mbar_wait_warp(bar(G_Q_FULL), 0, abort_flag, status, TG_WHERE_PRODUCER) &&
-                      mbar_wait_warp(bar(G_K_FULL + s), 0, abort_flag, status, TG_WHERE_PRODUCER))) {
-                    okp = false;
-                    break;
-                }
-                if (use > 0 && !mbar_wait_warp(bar(G_V_EMPTY + s), (use - 1) & 1, abort_flag, status,
-                                               TG_WHERE_PRODUCER)) {
-                    okp = false;
-                    break;
-                }
-                if (lane == 0) {
-                    mbar_expect_tx(bar(G_V_FULL + s), BN * HD * 2);
-#pragma unroll
-                    for (int hf = 0; hf < HD / 64; ++hf)
-                        tma_load_2d(sV0 + s * L::TILE_KV + hf * BN * 128, &tmV, hk * HD + hf * 64,
-                                    U.seq0 + (U.kv0 + j) * BN, bar(G_V_FULL + s));
-                    ++v_issued[s];
-                }
-            }
-            ++nu;
         }
         if (lane == 0 && *abort_flag) {
-            // let every copy this warp started land before the CTA exits
-            if (q_issued) drain_wait(bar(G_Q_FULL), (q_issued - 1) & 1, status);
+            drain_wait(bar(G_Q_FULL), 0, status);
             for (int s = 0; s < 2; ++s) {
                 if (k_issued[s]) drain_wait(bar(G_K_FULL + s), (k_issued[s] - 1) & 1, status);
                 if (v_issued[s]) drain_wait(bar(G_V_FULL + s), (v_issued[s] - 1) & 1, status);
@@ -824,8 +688,8 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, HD, true);
-            auto issue_s = [&](int hh, int s) {
-                const uint32_t kb = sK0 + s * L::TILE_KV;
+            auto issue_s = [&](int hh, int j) {
+                const uint32_t kb = sK0 + (j & 1) * L::TILE_KV;
                 const uint32_t qb = sQ + hh * L::TILE_Q;
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk) {
@@ -836,77 +700,61 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 }
                 // + bscale_h * gls_j: the bias k-step (no-swizzle tiles, K cores 128 B apart)
                 mma_bf16_ss(tmem + hh * BN, smem_desc_noswz(sQX + hh * L::EXT, 128, 256),
-                            smem_desc_noswz(sKX + s * L::EXT, 128, 256), idesc_qk, 1u);
+                            smem_desc_noswz(sKX + (j & 1) * L::EXT, 128, 256), idesc_qk, 1u);
             };
-            auto issue_pv = [&](int hh, int s, bool acc) {
-                const uint32_t vb = sV0 + s * L::TILE_KV;
+            auto issue_pv = [&](int hh, int j) {
+                const uint32_t vb = sV0 + (j & 1) * L::TILE_KV;
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk)
                     mma_bf16_ts(tmem + 2 * BN + hh * HD, tmem + hh * BN + kk * 8,
                                 smem_desc_sw128(vb + kk * 16 * 128, BN * 128, 1024), idesc_pv,
-                                (acc || kk > 0) ? 1u : 0u);
+                                (j > 0 || kk > 0) ? 1u : 0u);
             };
-            uint32_t gt = 0;
-            int nu = 0;
-            bool ok = true;
-            for (int k = 0; ok; ++k) {
-                const int64_t slot = g2_slot(k, total);
-                if (slot < 0) break;
-                const G2Unit U = g2_decode(slot, pairs, B, kv_chunk, cu_kept, s_cu);
-                if (!U.valid) continue;
-                const bool tr = (nu < 2);  // trace the first two units (tile index + 16 per unit)
-                ok = mbar_wait(bar(G_Q_FULL), nu & 1, abort_flag, status, TG_WHERE_MMA) &&
-                     mbar_wait(bar(G_K_FULL + (gt & 1)), (gt >> 1) & 1, abort_flag, status, TG_WHERE_MMA);
+            bool ok = mbar_wait(bar(G_Q_FULL), 0, abort_flag, status, TG_WHERE_MMA) &&
+                      mbar_wait(bar(G_K_FULL), 0, abort_flag, status, TG_WHERE_MMA);
+            TG_CTA_STAMP(2);
+            if (ok) {
+                tc_fence_after();
+                issue_s(0, 0);
+                mma_commit(bar(G_S_FULL + 0));
+                issue_s(1, 0);
+                mma_commit(bar(G_S_FULL + 1));
+                mma_commit(bar(G_K_EMPTY + 0));
+            }
+            for (int j = 0; ok && j < n_kv; ++j) {
+                const int s = j & 1;
+                const bool more = j + 1 < n_kv;
+                ok = mbar_wait(bar(G_V_FULL + s), (j >> 1) & 1, abort_flag, status, TG_WHERE_MMA) &&
+                     mbar_wait(bar(G_P_FULL + 0), j & 1, abort_flag, status, TG_WHERE_MMA);
                 if (!ok) break;
                 tc_fence_after();
+                TG_TRACE_AT(0, j);  // P0(j) ready, issuing PV0(j)
+                issue_pv(0, j);
+                if (more) {
+                    ok = mbar_wait(bar(G_K_FULL + (s ^ 1)), ((j + 1) >> 1) & 1, abort_flag, status, TG_WHERE_MMA);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_s(0, j + 1);
+                    mma_commit(bar(G_S_FULL + 0));
+                    TG_TRACE_AT(10, j);  // S0(j+1) issued
 #ifdef TG_TRACE
-                if (nu == 1 && blockIdx.x < 4096) g_attn_cta[blockIdx.x * 16 + 9] = globaltimer();  // S of unit 2 issued
+                    // trace builds only: stamp the completion of S0(j+1) as the tensor core sees it
+                    if (mbar_wait(bar(G_S_FULL + 0), (j + 1) & 1, abort_flag, status, TG_WHERE_MMA)) TG_TRACE_AT(13, j);
 #endif
-                if (tr) TG_TRACE_AT(18, 16 * nu);  // first S of the unit issued
-                issue_s(0, gt & 1);
-                mma_commit(bar(G_S_FULL + 0));
-                issue_s(1, gt & 1);
-                mma_commit(bar(G_S_FULL + 1));
-                mma_commit(bar(G_K_EMPTY + (gt & 1)));
-                if (U.n_kv == 1) mma_commit(bar(G_Q_EMPTY));  // the unit's last S MMA has read Q
-                for (int j = 0; j < U.n_kv; ++j, ++gt) {
-                    const int s = static_cast<int>(gt & 1);
-                    const bool more = j + 1 < U.n_kv;
-                    ok = mbar_wait(bar(G_V_FULL + s), (gt >> 1) & 1, abort_flag, status, TG_WHERE_MMA) &&
-                         mbar_wait(bar(G_P_FULL + 0), gt & 1, abort_flag, status, TG_WHERE_MMA);
-                    // the first PV of a unit overwrites O: wait until the epilogue has read it
-                    if (ok && j == 0 && nu > 0)
-                        ok = mbar_wait(bar(G_O_EMPTY), (nu - 1) & 1, abort_flag, status, TG_WHERE_MMA);
-                    if (!ok) break;
-                    tc_fence_after();
-                    if (tr) TG_TRACE_AT(0, j + 16 * nu);  // P0(j) ready, issuing PV0(j)
-                    issue_pv(0, s, j > 0);
-                    if (more) {
-                        ok = mbar_wait(bar(G_K_FULL + (s ^ 1)), ((gt + 1) >> 1) & 1, abort_flag, status,
-                                       TG_WHERE_MMA);
-                        if (!ok) break;
-                        tc_fence_after();
-                        issue_s(0, s ^ 1);
-                        mma_commit(bar(G_S_FULL + 0));
-                        if (tr) TG_TRACE_AT(10, j + 16 * nu);  // S0(j+1) issued
-                    }
-                    ok = mbar_wait(bar(G_P_FULL + 1), gt & 1, abort_flag, status, TG_WHERE_MMA);
-                    if (!ok) break;
-                    tc_fence_after();
-                    if (tr) TG_TRACE_AT(1, j + 16 * nu);  // P1(j) ready, issuing PV1(j)
-                    issue_pv(1, s, j > 0);
-                    mma_commit(bar(G_V_EMPTY + s));
-                    if (more) {
-                        issue_s(1, s ^ 1);
-                        mma_commit(bar(G_S_FULL + 1));
-                        mma_commit(bar(G_K_EMPTY + (s ^ 1)));
-                        if (j + 2 == U.n_kv) mma_commit(bar(G_Q_EMPTY));
-                    }
                 }
+                ok = mbar_wait(bar(G_P_FULL + 1), j & 1, abort_flag, status, TG_WHERE_MMA);
                 if (!ok) break;
-                mma_commit(bar(G_O_FULL));
-                ++nu;
+                tc_fence_after();
+                TG_TRACE_AT(1, j);  // P1(j) ready, issuing PV1(j)
+                issue_pv(1, j);
+                mma_commit(bar(G_V_EMPTY + s));
+                if (more) {
+                    issue_s(1, j + 1);
+                    mma_commit(bar(G_S_FULL + 1));
+                    mma_commit(bar(G_K_EMPTY + (s ^ 1)));
+                }
             }
+            if (ok) mma_commit(bar(G_O_FULL));
             mma_commit(bar(G_DRAIN));
             drain_wait(bar(G_DRAIN), 0, status);
         }
@@ -925,186 +773,213 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         // reads in the loop (those would queue behind the tensor core's operand traffic).
         const int q4 = warp & 3;
         const int half = warp >> 2;
-        const int r = q4 * 32 + lane;  // query row == TMEM lane
+        const int r = q4 * 32 + lane;        // query row == TMEM lane
+        const int q_local = qt * BM + r;
+        const bool valid_row = q_local < Mb;
+        const int qg = seq0 + q_local;
+        const float ratio_log = valid_row ? logf(static_cast<float>(pos[qg]) / static_cast<float>(rank[qg])) : 0.f;
+        // per-head values are scalars selected by the head index (no local-memory arrays)
+        const float inv_tau0 = valid_row ? 1.0f / (1.0f + c[2 * pair] * ratio_log) : 1.0f;
+        const float inv_tau1 = valid_row ? 1.0f / (1.0f + c[2 * pair + 1] * ratio_log) : 1.0f;
+        const float alpha0 = sm_scale * LOG2E * inv_tau0, alpha1 = sm_scale * LOG2E * inv_tau1;
         const uint32_t lane_addr = static_cast<uint32_t>(q4 * 32) << 16;
         float* red = reinterpret_cast<float*>(smem + L::OFF_RED);  // [parity][half][row] partial maxima
         float* lred = red + 2 * 2 * BM;                             // [head][half][row] partial sums
-        int* s_last = reinterpret_cast<int*>(smem + L::OFF_MISC + 8);
-        uint32_t gt = 0;  // KV tiles consumed so far (all units)
-        int nu = 0;
+        float m_run0 = -INFINITY, m_run1 = -INFINITY, l_run0 = 0.f, l_run1 = 0.f;
         bool ok = true;
-        const float* s_alpha = reinterpret_cast<const float*>(smem + L::OFF_ALPHA);
-        for (int k = 0; ok; ++k) {
-            const int64_t slot = g2_slot(k, total);
-            if (slot < 0) break;
-            const G2Unit U = g2_decode(slot, pairs, B, kv_chunk, cu_kept, s_cu);
-            if (!U.valid) continue;
-            const bool tr = (nu < 2);  // trace the first two units (tile index + 16 per unit)
-            if (tr && r == 0 && half == 0) TG_TRACE_AT(16, 16 * nu);  // unit decoded
-            const int q_local = U.qt * BM + r;
-            const bool valid_row = q_local < U.Mb;
-            const int qg = U.seq0 + q_local;
-            const int h0 = 2 * U.pair;
-            // alpha of this row for both heads, computed by the producer warp ahead of time.  A
-            // failed wait has raised the abort flag; the reducing barrier of the first step then
-            // takes every softmax thread out together (leaving here alone would strand the others).
-            (void)mbar_wait_warp(bar(G_A_FULL + (nu & 1)), (nu >> 1) & 1, abort_flag, status, TG_WHERE_SOFTMAX);
-            if (tr && r == 0 && half == 0) TG_TRACE_AT(17, 16 * nu);  // alpha ready
-            const float alpha0 = s_alpha[((nu & 1) * 2 + 0) * BM + r];
-            const float alpha1 = s_alpha[((nu & 1) * 2 + 1) * BM + r];
-            float m_run0 = -INFINITY, m_run1 = -INFINITY, l_run0 = 0.f, l_run1 = 0.f;
-            int arrival = 0;  // thread 0: the split unit's arrival at its counter (taken a tile early)
-            for (int j = 0; ok && j < U.n_kv; ++j, ++gt) {
-                if (U.nch > 1 && j + 1 == U.n_kv && threadIdx.x == 0) {
-                    // its round trip overlaps the last tile; the value is first used in the epilogue
-                    arrival = atomicAdd(ws.cnt + (static_cast<int64_t>(U.b) * pairs + U.pair) * ws.slots_per_pair +
-                                            (U.qt - U.C),
-                                        1);
-                }
-                const int jt = U.kv0 + j;  // KV tile index within the sequence
-                const bool diag = (jt == U.qt);
-                const int lim = q_local - jt * BN - half * 64;  // on the diagonal tile, own columns > lim are future keys
+        int arrival = 0;  // thread 0: the split unit's arrival at its counter (taken a tile early)
+        for (int j = 0; ok && j < n_kv; ++j) {
+            const int jt = kv0 + j;  // KV tile index within the sequence
+            if (split && j + 1 == n_kv && threadIdx.x == 0) {
+                // its round trip overlaps the last tile; the value is first used in the epilogue
+                arrival = atomicAdd(ws.cnt + (static_cast<int64_t>(b) * (Hq / 2) + pair) * ws.slots_per_pair + (qt - C), 1);
+            }
+            const bool diag = (jt == qt);
+            const int lim = q_local - jt * BN - half * 64;  // on the diagonal tile, own columns > lim are future keys
 #pragma unroll 1
-                for (int hh = 0; hh < 2; ++hh) {
-                    const int step = static_cast<int>(2 * gt) + hh;
-                    const float alpha = hh ? alpha1 : alpha0;
-                    float m_h = hh ? m_run1 : m_run0;
-                    const uint32_t tS = tmem + lane_addr + hh * BN;
-                    const bool okw =
-                        mbar_wait_warp(bar(G_S_FULL + hh), gt & 1, abort_flag, status, TG_WHERE_SOFTMAX);
-                    if (tr && r == 0 && half == 0) TG_TRACE_AT(2 + 4 * hh, j + 16 * nu);  // S_h(j) ready
-#ifdef TG_TRACE
-                    if (nu < 2 && threadIdx.x == 0 && j == 0 && hh == 0 && blockIdx.x < 4096)
-                        g_attn_cta[blockIdx.x * 16 + (nu ? 12 : 2)] = globaltimer();
-#endif
-                    float x[64];
-                    float my = -INFINITY;
-                    if (okw) {
-                        tc_fence_after();
-                        tmem_ld32(tS + half * 64, x);
-                        tmem_ld32(tS + half * 64 + 32, x + 32);
+            for (int hh = 0; hh < 2; ++hh) {
+                const int step = 2 * j + hh;
+                const float alpha = hh ? alpha1 : alpha0;
+                float m_h = hh ? m_run1 : m_run0;
+                const uint32_t tS = tmem + lane_addr + hh * BN;
+                const bool okw = mbar_wait_warp(bar(G_S_FULL + hh), j & 1, abort_flag, status, TG_WHERE_SOFTMAX);
+                if (r == 0 && half == 0) TG_TRACE_AT(2 + 4 * hh, j);  // S_h(j) ready
+                if (threadIdx.x == 0 && step == 0) TG_CTA_STAMP(3);
+                float x[64];
+                float my = -INFINITY;
+                if (okw) {
+                    tc_fence_after();
+                    tmem_ld32(tS + half * 64, x);
+                    tmem_ld32(tS + half * 64 + 32, x + 32);
+                    tmem_wait_ld();
+                    if (r == 0 && half == 0) TG_TRACE_AT(3 + 4 * hh, j);  // S_h(j) in registers
+                    if (diag) {
+#pragma unroll
+                        for (int cc = 0; cc < 64; ++cc) x[cc] = cc > lim ? -INFINITY : x[cc];
+                    }
+                    // stabiliser: the row max of the biased scores
+                    float mp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                    for (int cc = 0; cc < 64; cc += 2) mp[(cc >> 1) & 3] = max3f(mp[(cc >> 1) & 3], x[cc], x[cc + 1]);
+                    my = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
+                }
+                red[(step & 1) * (2 * BM) + half * BM + r] = my;
+                // every S load of both halves is complete past this barrier, so P may overwrite S
+                if (bar_red_or(1, 256, !okw)) {
+                    ok = false;
+                    break;
+                }
+                my = fmaxf(my, red[(step & 1) * (2 * BM) + (half ^ 1) * BM + r]);
+                // floored so that a tile whose keys all carry an infinite negative bias gives
+                // p = 0 instead of 2^(-inf + inf)
+                const float mx = fmaxf(alpha * my, -1.0e30f);
+                float corr = 1.0f;
+                bool rescale_o = false;
+                if (j == 0 || mx > m_h + RESCALE_THRESHOLD) {
+                    const float m_new = fmaxf(m_h, mx);
+                    corr = ex2_approx(m_h - m_new);
+                    m_h = m_new;
+                    rescale_o = j > 0;
+                }
+                if (hh) m_run1 = m_h; else m_run0 = m_h;
+                if (r == 0 && half == 0) TG_TRACE_AT(4 + 4 * hh, j);  // max done
+                const uint64_t al2 = f32x2_pack(alpha, alpha);
+                const uint64_t nm2 = f32x2_pack(-m_h, -m_h);
+                uint64_t sp[4] = {0ull, 0ull, 0ull, 0ull};
+                uint32_t pk[32];
+#pragma unroll
+                for (int c4 = 0; c4 < 16; ++c4) {
+                    const int cc = c4 * 4;
+                    const uint64_t a0 = f32x2_fma(al2, f32x2_pack(x[cc], x[cc + 1]), nm2);
+                    const uint64_t a1 = f32x2_fma(al2, f32x2_pack(x[cc + 2], x[cc + 3]), nm2);
+                    const float p0 = ex2_approx(f32x2_lo(a0)), p1 = ex2_approx(f32x2_hi(a0));
+                    const float p2 = ex2_approx(f32x2_lo(a1)), p3 = ex2_approx(f32x2_hi(a1));
+                    sp[(2 * c4) & 3] = f32x2_add(sp[(2 * c4) & 3], f32x2_pack(p0, p1));
+                    sp[(2 * c4 + 1) & 3] = f32x2_add(sp[(2 * c4 + 1) & 3], f32x2_pack(p2, p3));
+                    pk[cc / 2] = pack_bf16x2(p0, p1);
+                    pk[cc / 2 + 1] = pack_bf16x2(p2, p3);
+                }
+                // P_h: keys 64 half .. 64 half + 63 -> columns 32 half .. 32 half + 31 of S_h
+                tmem_st32u(tS + half * 32, pk);
+                if (r == 0 && half == 0) TG_TRACE_AT(11 + 3 * hh, j);  // exponentials done
+                const uint64_t s01 = f32x2_add(sp[0], sp[1]), s23 = f32x2_add(sp[2], sp[3]);
+                const uint64_t s4 = f32x2_add(s01, s23);
+                const float tile_sum = f32x2_lo(s4) + f32x2_hi(s4);
+                if (hh) l_run1 = l_run1 * corr + tile_sum; else l_run0 = l_run0 * corr + tile_sum;
+                if (rescale_o) {
+                    // O_h is stable: PV_h(j-1) completed before S_h(j), PV_h(j) waits for P_h(j)
+                    const uint32_t tO = tmem + lane_addr + 2 * BN + hh * HD + half * (HD / 2);
+#pragma unroll
+                    for (int ch = 0; ch < HD / 64; ++ch) {
+                        float o[32];
+                        tmem_ld32(tO + ch * 32, o);
                         tmem_wait_ld();
-                        if (tr && r == 0 && half == 0) TG_TRACE_AT(3 + 4 * hh, j + 16 * nu);  // S_h(j) in registers
-                        if (diag) {
 #pragma unroll
-                            for (int cc = 0; cc < 64; ++cc) x[cc] = cc > lim ? -INFINITY : x[cc];
-                        }
-                        // stabiliser: the row max of the biased scores
-                        float mp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-                        for (int cc = 0; cc < 64; cc += 2)
-                            mp[(cc >> 1) & 3] = max3f(mp[(cc >> 1) & 3], x[cc], x[cc + 1]);
-                        my = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
+                        for (int e = 0; e < 32; ++e) o[e] *= corr;
+                        tmem_st32(tO + ch * 32, o);
                     }
-                    red[(step & 1) * (2 * BM) + half * BM + r] = my;
-                    // every S load of both halves is complete past this barrier, so P may overwrite S
-                    if (bar_red_or(1, 256, !okw)) {
-                        ok = false;
-                        break;
-                    }
-                    my = fmaxf(my, red[(step & 1) * (2 * BM) + (half ^ 1) * BM + r]);
-                    // floored so that a tile whose keys all carry an infinite negative bias gives
-                    // p = 0 instead of 2^(-inf + inf)
-                    const float mx = fmaxf(alpha * my, -1.0e30f);
-                    float corr = 1.0f;
-                    bool rescale_o = false;
-                    if (j == 0 || mx > m_h + RESCALE_THRESHOLD) {
-                        const float m_new = fmaxf(m_h, mx);
-                        corr = ex2_approx(m_h - m_new);
-                        m_h = m_new;
-                        rescale_o = j > 0;
-                    }
-                    if (hh) m_run1 = m_h; else m_run0 = m_h;
-                    if (tr && r == 0 && half == 0) TG_TRACE_AT(4 + 4 * hh, j + 16 * nu);  // max done
-                    const uint64_t al2 = f32x2_pack(alpha, alpha);
-                    const uint64_t nm2 = f32x2_pack(-m_h, -m_h);
-                    uint64_t sp[4] = {0ull, 0ull, 0ull, 0ull};
-                    uint32_t pk[32];
-#pragma unroll
-                    for (int c4 = 0; c4 < 16; ++c4) {
-                        const int cc = c4 * 4;
-                        const uint64_t a0 = f32x2_fma(al2, f32x2_pack(x[cc], x[cc + 1]), nm2);
-                        const uint64_t a1 = f32x2_fma(al2, f32x2_pack(x[cc + 2], x[cc + 3]), nm2);
-                        const float p0 = ex2_approx(f32x2_lo(a0)), p1 = ex2_approx(f32x2_hi(a0));
-                        const float p2 = ex2_approx(f32x2_lo(a1)), p3 = ex2_approx(f32x2_hi(a1));
-                        sp[(2 * c4) & 3] = f32x2_add(sp[(2 * c4) & 3], f32x2_pack(p0, p1));
-                        sp[(2 * c4 + 1) & 3] = f32x2_add(sp[(2 * c4 + 1) & 3], f32x2_pack(p2, p3));
-                        pk[cc / 2] = pack_bf16x2(p0, p1);
-                        pk[cc / 2 + 1] = pack_bf16x2(p2, p3);
-                    }
-                    // P_h: keys 64 half .. 64 half + 63 -> columns 32 half .. 32 half + 31 of S_h
-                    tmem_st32u(tS + half * 32, pk);
-                    if (tr && r == 0 && half == 0) TG_TRACE_AT(11 + 3 * hh, j + 16 * nu);  // exponentials done
-                    const uint64_t s01 = f32x2_add(sp[0], sp[1]), s23 = f32x2_add(sp[2], sp[3]);
-                    const uint64_t s4 = f32x2_add(s01, s23);
-                    const float tile_sum = f32x2_lo(s4) + f32x2_hi(s4);
-                    if (hh) l_run1 = l_run1 * corr + tile_sum; else l_run0 = l_run0 * corr + tile_sum;
-                    if (rescale_o) {
-                        // O_h is stable: PV_h(j-1) completed before S_h(j), PV_h(j) waits for P_h(j)
-                        const uint32_t tO = tmem + lane_addr + 2 * BN + hh * HD + half * (HD / 2);
-#pragma unroll
-                        for (int ch = 0; ch < HD / 64; ++ch) {
-                            float o[32];
-                            tmem_ld32(tO + ch * 32, o);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int e = 0; e < 32; ++e) o[e] *= corr;
-                            tmem_st32(tO + ch * 32, o);
-                        }
-                    }
-                    tmem_wait_st();
-                    if (tr && r == 0 && half == 0) TG_TRACE_AT(12 + 3 * hh, j + 16 * nu);  // P and O stores complete
-                    tc_fence_before();
-                    __syncwarp();  // every lane's P and O stores are complete and fenced
-                    if (lane == 0) mbar_arrive(bar(G_P_FULL + hh));  // one arrival per warp
-                    if (tr && r == 0 && half == 0) TG_TRACE_AT(5 + 4 * hh, j + 16 * nu);  // P_h(j) stored and signalled
                 }
-            }
-            if (!ok) break;
-#ifdef TG_TRACE
-            if (nu < 2 && threadIdx.x == 0 && blockIdx.x < 4096) g_attn_cta[blockIdx.x * 16 + (nu ? 13 : 3)] = globaltimer();
-#endif
-            // ---------------------------------------------------------------- epilogue of the unit
-            const bool oko = mbar_wait_warp(bar(G_O_FULL), nu & 1, abort_flag, status, TG_WHERE_SOFTMAX);
-            lred[0 * (2 * BM) + half * BM + r] = l_run0;
-            lred[1 * (2 * BM) + half * BM + r] = l_run1;
-            if (bar_red_or(1, 256, !oko)) {  // uniform over the 256 softmax threads
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-#ifdef TG_TRACE
-            if (nu < 2 && threadIdx.x == 0 && blockIdx.x < 4096) g_attn_cta[blockIdx.x * 16 + (nu ? 14 : 4)] = globaltimer();
-#endif
-            if (tr && r == 0 && half == 0) TG_TRACE_AT(19, 16 * nu);  // O complete
-            const float l_tot0 = l_run0 + lred[0 * (2 * BM) + (half ^ 1) * BM + r];
-            const float l_tot1 = l_run1 + lred[1 * (2 * BM) + (half ^ 1) * BM + r];
-            const bool split = U.nch > 1;
-            const float my_lse0 = m_run0 + log2f(l_tot0), my_lse1 = m_run1 + log2f(l_tot1);
-            // Rows leave from registers: each thread stores its 64 columns (128 contiguous
-            // bytes) per head.  O may be overwritten by the next unit's first PV once every
-            // warp has passed its O_EMPTY arrival.
-            auto store_row = [&](int h, int col0, const float* o, float w) {
-                if (!valid_row) return;
-                uint4* dst = reinterpret_cast<uint4*>(out + (static_cast<size_t>(qg) * Hq + h) * HD + col0);
-#pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4) {
-                    uint4 v;
-                    v.x = pack_bf16x2(o[k4 * 8 + 0] * w, o[k4 * 8 + 1] * w);
-                    v.y = pack_bf16x2(o[k4 * 8 + 2] * w, o[k4 * 8 + 3] * w);
-                    v.z = pack_bf16x2(o[k4 * 8 + 4] * w, o[k4 * 8 + 5] * w);
-                    v.w = pack_bf16x2(o[k4 * 8 + 6] * w, o[k4 * 8 + 7] * w);
-                    dst[k4] = v;
-                }
-            };
-            auto release_o = [&]() {
+                tmem_wait_st();
+                if (r == 0 && half == 0) TG_TRACE_AT(12 + 3 * hh, j);  // P and O stores complete
                 tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(G_O_EMPTY));
-            };
-            if (!split) {
+                __syncwarp();  // every lane's P and O stores are complete and fenced
+                if (lane == 0) mbar_arrive(bar(G_P_FULL + hh));  // one arrival per warp
+                if (r == 0 && half == 0) TG_TRACE_AT(5 + 4 * hh, j);  // P_h(j) stored and signalled
+            }
+        }
+        // ---------------------------------------------------------------- epilogue
+        if (threadIdx.x == 0) TG_CTA_STAMP(4);
+        const bool oko = ok && mbar_wait_warp(bar(G_O_FULL), 0, abort_flag, status, TG_WHERE_SOFTMAX);
+        lred[0 * (2 * BM) + half * BM + r] = l_run0;
+        lred[1 * (2 * BM) + half * BM + r] = l_run1;
+        ok = !bar_red_or(1, 256, !oko);  // uniform over the 256 softmax threads
+        if (ok) tc_fence_after();
+        if (threadIdx.x == 0) TG_CTA_STAMP(5);
+        // per-head values as scalars: the epilogue loops over the heads without unrolling
+        const float l_tot0 = l_run0 + lred[0 * (2 * BM) + (half ^ 1) * BM + r];
+        const float l_tot1 = l_run1 + lred[1 * (2 * BM) + (half ^ 1) * BM + r];
+        const float m_fin0 = m_run0, m_fin1 = m_run1;
+        // Output rows leave through shared memory: each thread stages its half row of both
+        // heads in the K buffers (free once every MMA has completed), 16-byte chunks XOR-
+        // swizzled by the row so that the staging is conflict-free; then each warp writes 32
+        // whole rows of one head with coalesced stores (rows past the sequence end are skipped).
+        constexpr int CH = HD * 2 / 16;  // 16-byte chunks per bf16 row
+        auto stage_row = [&](int hh, const float* o32, int ch32, float w) {  // 32 columns from ch32 * 32
+            uint8_t* stage = smem + L::OFF_K + hh * (BM * HD * 2);
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) {
+                const int cidx = ch32 * 4 + k4;
+                uint4 v;
+                v.x = pack_bf16x2(o32[k4 * 8 + 0] * w, o32[k4 * 8 + 1] * w);
+                v.y = pack_bf16x2(o32[k4 * 8 + 2] * w, o32[k4 * 8 + 3] * w);
+                v.z = pack_bf16x2(o32[k4 * 8 + 4] * w, o32[k4 * 8 + 5] * w);
+                v.w = pack_bf16x2(o32[k4 * 8 + 6] * w, o32[k4 * 8 + 7] * w);
+                *reinterpret_cast<uint4*>(stage + r * (HD * 2) + ((cidx ^ (r & (CH - 1))) << 4)) = v;
+            }
+        };
+        auto write_rows = [&]() {  // warp w writes rows 32 (w & 3) .. + 31 of head w >> 2
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+            const int wh = warp >> 2;
+            const uint8_t* stg = smem + L::OFF_K + wh * (BM * HD * 2);
+            const int hw = 2 * pair + wh;
+#pragma unroll 4
+            for (int i = 0; i < 32; ++i) {
+                const int rr = q4 * 32 + i;
+                if (qt * BM + rr >= Mb) break;
+                const uint8_t* src = stg + rr * (HD * 2);
+                uint16_t* dst = out + (static_cast<size_t>(seq0 + qt * BM + rr) * Hq + hw) * HD;
+                if (HD == 128) {
+                    const uint2 v = *reinterpret_cast<const uint2*>(src + (((lane >> 1) ^ (rr & (CH - 1))) << 4) +
+                                                                    (lane & 1) * 8);
+                    *reinterpret_cast<uint2*>(dst + lane * 4) = v;
+                } else {
+                    const uint32_t v = *reinterpret_cast<const uint32_t*>(
+                        src + (((lane >> 2) ^ (rr & (CH - 1))) << 4) + (lane & 3) * 4);
+                    *reinterpret_cast<uint32_t*>(dst + lane * 2) = v;
+                }
+            }
+        };
+        if (!split) {
+            if (ok) {
 #pragma unroll 1
                 for (int hh = 0; hh < 2; ++hh) {
+                    const uint32_t tO = tmem + lane_addr + 2 * BN + hh * HD + half * (HD / 2);
+                    const float lt = hh ? l_tot1 : l_tot0, mf = hh ? m_fin1 : m_fin0;
+                    const float inv_l = 1.0f / lt;
+#pragma unroll
+                    for (int ch = 0; ch < HD / 64; ++ch) {
+                        float o[32];
+                        tmem_ld32(tO + ch * 32, o);
+                        tmem_wait_ld();
+                        stage_row(hh, o, half * (HD / 64) + ch, inv_l);
+                    }
+                    if (valid_row && lse && half == 0)
+                        lse[static_cast<size_t>(qg) * Hq + 2 * pair + hh] = (mf + log2f(lt)) / LOG2E;
+                }
+            }
+            write_rows();
+        } else {
+            // The two KV chunks of a split query tile meet through one counter (taken by
+            // thread 0 at the start of its last tile): the first to arrive (0 -> 1) writes its
+            // normalised partial (bf16 column pairs, [pair][row] so that a warp's 32 rows are one
+            // 128-byte write) and log-sum-exp, then publishes them (+1, release); the second
+            // (arrival value 1 or 2) waits, if needed, for that publication (the first is
+            // resident and depends on nothing else, so the bounded wait ends), merges the
+            // partial with its own O read straight from TMEM, writes the rows and resets the
+            // counter.
+            const int64_t slot = (static_cast<int64_t>(b) * (Hq / 2) + pair) * ws.slots_per_pair + (qt - C);
+            int* cnt = ws.cnt + slot;
+            const float my_lse0 = m_fin0 + log2f(l_tot0), my_lse1 = m_fin1 + log2f(l_tot1);
+            int* s_last = reinterpret_cast<int*>(smem + L::OFF_MISC + 8);
+            if (threadIdx.x == 0) *s_last = ok ? arrival : -1;
+            asm volatile("bar.sync 1, 256;" ::: "memory");  // all 256 softmax threads, abort or not
+            const int arr = *s_last;
+            asm volatile("bar.sync 1, 256;" ::: "memory");  // s_last is read before it is reused
+            if (arr == 0) {
+#pragma unroll 1
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t* po = reinterpret_cast<uint32_t*>(ws.o) +
+                                   ((slot * ws.max_nch + chunk) * 2 + hh) * (BM * HD / 2) + r;
                     const uint32_t tO = tmem + lane_addr + 2 * BN + hh * HD + half * (HD / 2);
                     const float inv_l = 1.0f / (hh ? l_tot1 : l_tot0);
 #pragma unroll
@@ -1112,132 +987,80 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                         float o[32];
                         tmem_ld32(tO + ch * 32, o);
                         tmem_wait_ld();
-                        store_row(h0 + hh, half * (HD / 2) + ch * 32, o, inv_l);
+                        const int cp0 = (half * (HD / 2) + ch * 32) / 2;  // first column pair
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            po[(cp0 + e) * BM] = pack_bf16x2(o[2 * e] * inv_l, o[2 * e + 1] * inv_l);
                     }
+                    if (half == 0) ws.lse2[((slot * ws.max_nch + chunk) * 2 + hh) * BM + r] = hh ? my_lse1 : my_lse0;
                 }
-                release_o();
-                if (valid_row && lse && half == 0) {
-                    lse[static_cast<size_t>(qg) * Hq + h0] = my_lse0 / LOG2E;
-                    lse[static_cast<size_t>(qg) * Hq + h0 + 1] = my_lse1 / LOG2E;
+                if (threadIdx.x == 0) TG_CTA_STAMP(8);
+                asm volatile("bar.sync 1, 256;" ::: "memory");  // every partial store is issued
+                if (threadIdx.x == 0) {
+                    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+                    atomicAdd(cnt, 1);  // publish
                 }
-            } else {
-                // The two KV chunks of a split query tile meet through one counter: the first
-                // to arrive (0 -> 1) writes its normalised partial and log-sum-exp, then
-                // publishes them (+1, release); the second (arrival value 1 or 2) waits, if
-                // needed, for that publication (the first is resident and depends on nothing
-                // else, so the bounded wait ends), merges the partial with its own O read
-                // straight from TMEM, writes the rows and resets the counter.
-                const int64_t slot_ws =
-                    (static_cast<int64_t>(U.b) * pairs + U.pair) * ws.slots_per_pair + (U.qt - U.C);
-                int* cnt = ws.cnt + slot_ws;
-                if (threadIdx.x == 0) *s_last = arrival;
+            } else if (arr > 0) {
+                if (threadIdx.x == 0) {
+                    int ready = 1;
+                    if (arr == 1) {
+                        const uint64_t t0 = globaltimer();
+                        while (*reinterpret_cast<volatile int*>(cnt) < 3) {
+                            if (globaltimer() - t0 > TG_WAIT_TIMEOUT_NS) {
+                                *abort_flag = 1;
+                                atomicOr(status, TG_DEVICE_TIMEOUT | TG_WHERE_SOFTMAX);
+                                ready = 0;
+                                break;
+                            }
+                        }
+                    }
+                    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+                    *s_last = ready;
+                }
                 asm volatile("bar.sync 1, 256;" ::: "memory");
-                arrival = *s_last;
-                asm volatile("bar.sync 1, 256;" ::: "memory");  // s_last is read before it is reused
-                if (arrival == 0) {
+                if (threadIdx.x == 0) TG_CTA_STAMP(10);
+                if (*s_last) {
 #pragma unroll 1
                     for (int hh = 0; hh < 2; ++hh) {
-                        uint32_t* po = reinterpret_cast<uint32_t*>(ws.o) +
-                                       ((slot_ws * ws.max_nch + U.chunk) * 2 + hh) * (BM * HD / 2) + r;
+                        const int64_t oidx = (slot * ws.max_nch + (chunk ^ 1)) * 2 + hh;
+                        const uint32_t* pt = reinterpret_cast<const uint32_t*>(ws.o) + oidx * (BM * HD / 2) + r;
+                        // the other chunk's half row of this head, all loads in flight at once
+                        uint32_t pw[HD / 4];
+#pragma unroll
+                        for (int e = 0; e < HD / 4; ++e) pw[e] = pt[(half * (HD / 4) + e) * BM];
+                        const float other_lse = ws.lse2[oidx * BM + r];
+                        const float ml = hh ? my_lse1 : my_lse0;
+                        const float mx = fmaxf(ml, other_lse);
+                        const float e_me = ex2_approx(ml - mx), e_ot = ex2_approx(other_lse - mx);
+                        const float inv_w = 1.0f / (e_me + e_ot);
+                        const float w_me = e_me * inv_w / (hh ? l_tot1 : l_tot0), w_ot = e_ot * inv_w;
                         const uint32_t tO = tmem + lane_addr + 2 * BN + hh * HD + half * (HD / 2);
-                        const float inv_l = 1.0f / (hh ? l_tot1 : l_tot0);
 #pragma unroll
                         for (int ch = 0; ch < HD / 64; ++ch) {
+                            float ot[32];
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) {
+                                const uint32_t w = pw[ch * 16 + e];
+                                ot[2 * e] = __uint_as_float(w << 16);
+                                ot[2 * e + 1] = __uint_as_float(w & 0xFFFF0000u);
+                            }
                             float o[32];
                             tmem_ld32(tO + ch * 32, o);
                             tmem_wait_ld();
-                            const int cp0 = (half * (HD / 2) + ch * 32) / 2;  // first column pair
-                            // bf16 pairs stored [column pair][row]: a warp's 32 rows of one pair are
-                            // one 128-byte write
 #pragma unroll
-                            for (int e = 0; e < 16; ++e)
-                                po[(cp0 + e) * BM] = pack_bf16x2(o[2 * e] * inv_l, o[2 * e + 1] * inv_l);
+                            for (int e = 0; e < 32; ++e) o[e] = fmaf(w_me, o[e], w_ot * ot[e]);  // own O unnormalised
+                            stage_row(hh, o, half * (HD / 64) + ch, 1.0f);
                         }
+                        if (valid_row && lse && half == 0)
+                            lse[static_cast<size_t>(qg) * Hq + 2 * pair + hh] = (mx + log2f(e_me + e_ot)) / LOG2E;
                     }
-                    release_o();
-                    if (half == 0) {
-                        ws.lse2[((slot_ws * ws.max_nch + U.chunk) * 2 + 0) * BM + r] = my_lse0;
-                        ws.lse2[((slot_ws * ws.max_nch + U.chunk) * 2 + 1) * BM + r] = my_lse1;
-                    }
-                    asm volatile("bar.sync 1, 256;" ::: "memory");  // every partial store is issued
-                    if (threadIdx.x == 0) {
-                        asm volatile("fence.acq_rel.gpu;" ::: "memory");
-                        atomicAdd(cnt, 1);  // publish
-                    }
-                } else {
-                    if (threadIdx.x == 0) {
-                        int ready = 1;
-                        if (arrival == 1) {
-                            const uint64_t t0 = globaltimer();
-                            while (*reinterpret_cast<volatile int*>(cnt) < 3) {
-                                if (globaltimer() - t0 > TG_WAIT_TIMEOUT_NS) {
-                                    *abort_flag = 1;
-                                    atomicOr(status, TG_DEVICE_TIMEOUT | TG_WHERE_SOFTMAX);
-                                    ready = 0;
-                                    break;
-                                }
-                            }
-                        }
-                        asm volatile("fence.acq_rel.gpu;" ::: "memory");
-                        *s_last = ready;
-                    }
-                    asm volatile("bar.sync 1, 256;" ::: "memory");
-                    const bool ready = *s_last != 0;
-                    if (ready) {
-#pragma unroll 1
-                        for (int hh = 0; hh < 2; ++hh) {
-                            const int64_t oi = (slot_ws * ws.max_nch + (U.chunk ^ 1)) * 2 + hh;
-                            const uint32_t* pt = reinterpret_cast<const uint32_t*>(ws.o) + oi * (BM * HD / 2) + r;
-                            // the other chunk's half row of this head, all loads in flight at once
-                            uint32_t pw[HD / 4];
-#pragma unroll
-                            for (int e = 0; e < HD / 4; ++e) pw[e] = pt[(half * (HD / 4) + e) * BM];
-                            const float ml = hh ? my_lse1 : my_lse0;
-                            const float other_lse = ws.lse2[oi * BM + r];
-                            const float mx = fmaxf(ml, other_lse);
-                            const float e_me = ex2_approx(ml - mx), e_ot = ex2_approx(other_lse - mx);
-                            const float inv_w = 1.0f / (e_me + e_ot);
-                            const float w_me = e_me * inv_w / (hh ? l_tot1 : l_tot0), w_ot = e_ot * inv_w;
-                            const uint32_t tO = tmem + lane_addr + 2 * BN + hh * HD + half * (HD / 2);
-#pragma unroll
-                            for (int ch = 0; ch < HD / 64; ++ch) {
-                                const int col0 = half * (HD / 2) + ch * 32;
-                                float ot[32];
-#pragma unroll
-                                for (int e = 0; e < 16; ++e) {
-                                    const uint32_t w = pw[ch * 16 + e];
-                                    ot[2 * e] = __uint_as_float(w << 16);
-                                    ot[2 * e + 1] = __uint_as_float(w & 0xFFFF0000u);
-                                }
-                                float o[32];
-                                tmem_ld32(tO + ch * 32, o);
-                                tmem_wait_ld();
-#pragma unroll
-                                for (int e = 0; e < 32; ++e) o[e] = fmaf(w_me, o[e], w_ot * ot[e]);  // own O unnormalised
-                                store_row(h0 + hh, col0, o, 1.0f);
-                            }
-                            if (valid_row && lse && half == 0)
-                                lse[static_cast<size_t>(qg) * Hq + h0 + hh] = (mx + log2f(e_me + e_ot)) / LOG2E;
-                        }
-                    }
-                    release_o();
-                    asm volatile("bar.sync 1, 256;" ::: "memory");  // s_last is read before it is reused
-                    if (threadIdx.x == 0) *cnt = 0;  // ready for the next call
                 }
+                write_rows();
+                if (threadIdx.x == 0) *cnt = 0;  // ready for the next call
             }
-#ifdef TG_TRACE
-            if (threadIdx.x == 0 && blockIdx.x < 4096) {
-                // first unit: [2] first S ready, [3] loop done, [4] O complete, [5] epilogue done;
-                // [6], [7]: ends of the second and third units
-                if (nu < 2) g_attn_cta[blockIdx.x * 16 + (nu ? 15 : 5)] = globaltimer();
-                if (nu >= 1 && nu < 3) g_attn_cta[blockIdx.x * 16 + 5 + nu] = globaltimer();
-                g_attn_cta[blockIdx.x * 16 + 10] += 1ull | (static_cast<unsigned long long>(U.n_kv) << 16) |
-                                                    (static_cast<unsigned long long>(U.nch > 1) << 32);
-            }
-#endif
-            if (tr && r == 0 && half == 0) TG_TRACE_AT(20, 16 * nu);  // epilogue done
-            ++nu;
+            if (threadIdx.x == 0) TG_CTA_STAMP(11);
         }
+        if (!split && threadIdx.x == 0) TG_CTA_STAMP(8);
     }
 
     tc_fence_before();
@@ -1247,12 +1070,16 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         tmem_dealloc(tmem, L::TMEM_COLS);
     }
 #ifdef TG_TRACE
-    if (threadIdx.x == 0 && blockIdx.x < 4096) {
-        unsigned smid;
-        asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
-        g_attn_cta[blockIdx.x * 16 + 0] = trace_t0;
-        g_attn_cta[blockIdx.x * 16 + 11] = globaltimer();
-        (void)smid;
+    if (threadIdx.x == 0) {
+        const unsigned idx = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+        if (idx < 4096) {
+            unsigned smid;
+            asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+            g_attn_cta[idx * 12 + 0] = trace_t0;
+            g_attn_cta[idx * 12 + 6] = globaltimer();
+            g_attn_cta[idx * 12 + 7] = smid | (static_cast<unsigned long long>(n_kv) << 32) |
+                                      (static_cast<unsigned long long>(split) << 40);
+        }
     }
 #endif
 }
@@ -1282,19 +1109,11 @@ cudaError_t launch_gqa2(const CUtensorMap& tq, const CUtensorMap& tk, const CUte
         p += slots * sw.max_nch * 2 * BM * sizeof(float);
         sw.cnt = reinterpret_cast<int*>(p);
     }
-    // persistent: one CTA per SM (at most one per unit slot); slots beyond a sequence's
-    // own unit count are skipped by the CTAs
-    const int64_t units_max = units_below_host(n_qt_max, C);
-    const int64_t slots = units_max * B * (Hq / 2);
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return cudaErrorInvalidDevice;
-    if (slots == 0) return cudaSuccess;
-    const unsigned grid = static_cast<unsigned>(slots < sms ? slots : sms);
-    gated_attn_gqa2_kernel<HD><<<grid, G2_THREADS, L::ALLOC, st>>>(
-        tq, tk, tv, cu_kept, pos, rank, gls, g, c, sm_scale, B, Hq, Hkv, static_cast<int>(units_max), C, sw, out, lse,
-        device_status_ptr());
+    const int64_t units = units_below_host(n_qt_max, C);
+    dim3 grid(Hq / 2, static_cast<unsigned>(units), B);
+    gated_attn_gqa2_kernel<HD><<<grid, G2_THREADS, L::ALLOC, st>>>(tq, tk, tv, cu_kept, pos, rank, gls, g, c,
+                                                                   sm_scale, Hq, Hkv, n_qt_max, C, sw, out, lse,
+                                                                   device_status_ptr());
     return cudaGetLastError();
 }
 
