@@ -167,6 +167,8 @@ gated_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     const int h = blockIdx.x;
     const int qt = n_qt_max - 1 - static_cast<int>(blockIdx.y);
     const int b = blockIdx.z;
+    pdl_wait();  // global memory is read only from here on
+    pdl_trigger();
     const int seq0 = cu_kept[b];
     const int Mb = cu_kept[b + 1] - seq0;
     if (qt * BM >= Mb) return;
@@ -518,6 +520,8 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
 #ifdef TG_TRACE
     const unsigned long long trace_t0 = globaltimer();
 #endif
+    pdl_wait();  // global memory is read only from here on
+    pdl_trigger();
     const int seq0 = cu_kept[b];
     const int Mb = cu_kept[b + 1] - seq0;
     const int n_qt = (Mb + BM - 1) / BM;
@@ -1111,10 +1115,9 @@ cudaError_t launch_gqa2(const CUtensorMap& tq, const CUtensorMap& tk, const CUte
     }
     const int64_t units = units_below_host(n_qt_max, C);
     dim3 grid(Hq / 2, static_cast<unsigned>(units), B);
-    gated_attn_gqa2_kernel<HD><<<grid, G2_THREADS, L::ALLOC, st>>>(tq, tk, tv, cu_kept, pos, rank, gls, g, c,
-                                                                   sm_scale, Hq, Hkv, n_qt_max, C, sw, out, lse,
-                                                                   device_status_ptr());
-    return cudaGetLastError();
+    return launch_pdl(gated_attn_gqa2_kernel<HD>, grid, dim3(G2_THREADS), static_cast<size_t>(L::ALLOC), st, tq, tk,
+                      tv, cu_kept, pos, rank, gls, g, c, sm_scale, Hq, Hkv, n_qt_max, C, sw, out, lse,
+                      device_status_ptr());
 }
 
 template <int HD>
@@ -1140,9 +1143,8 @@ cudaError_t launch_tc(const uint16_t* q, const uint16_t* k, const uint16_t* v, c
     int* status = device_status_ptr();
     const int n_qt_max = (max_M + BM - 1) / BM;
     dim3 grid(Hq, n_qt_max, B);
-    gated_attn_tc_kernel<HD><<<grid, NUM_THREADS, L::ALLOC, st>>>(tq, tk, tv, cu_kept, pos, rank, gls, g, c, sm_scale,
-                                                                  Hq, Hkv, n_qt_max, out, lse, status);
-    return cudaGetLastError();
+    return launch_pdl(gated_attn_tc_kernel<HD>, grid, dim3(NUM_THREADS), static_cast<size_t>(L::ALLOC), st, tq, tk, tv,
+                      cu_kept, pos, rank, gls, g, c, sm_scale, Hq, Hkv, n_qt_max, out, lse, status);
 }
 
 }  // namespace

@@ -130,10 +130,6 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
     const int nkb = D / KB;
     if (threadIdx.x == 0) SC_CTA(0);
 
-    for (int j = threadIdx.x; j < I; j += blockDim.x) {
-        s_b1[j] = b1[j];
-        s_w2[j] = w2[j];
-    }
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(full(s), 1);
@@ -153,6 +149,14 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // global memory is read only from here on (see pdl_wait)
+    pdl_wait();
+    pdl_trigger();
+    for (int j = threadIdx.x; j < I; j += blockDim.x) {
+        s_b1[j] = b1[j];
+        s_w2[j] = w2[j];
+    }
+    __syncthreads();
 
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA producer
@@ -315,9 +319,10 @@ cudaError_t launch_score_tc(const uint16_t* hidden, const int32_t* cu_seqlens, c
         return cudaErrorInvalidValue;
     const int64_t tiles_bound = (T + C::ROWS - 1) / C::ROWS + B;
     const int grid = static_cast<int>(tiles_bound < sms ? tiles_bound : sms);
-    score_tc_kernel<NACC><<<grid, C::THREADS, score_smem_bytes<NACC>(I), st>>>(tx, tw, cu_seqlens, span, B, D, I, b1,
-                                                                              w2, b2, eps, scores,
-                                                                              device_status_ptr());
+    const cudaError_t le = launch_pdl(score_tc_kernel<NACC>, dim3(grid), dim3(C::THREADS),
+                                      static_cast<size_t>(score_smem_bytes<NACC>(I)), st, tx, tw, cu_seqlens, span, B,
+                                      D, I, b1, w2, b2, eps, scores, device_status_ptr());
+    if (le != cudaSuccess) return le;
     return cudaGetLastError();
 }
 

@@ -117,6 +117,8 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
 
     const int crank = static_cast<int>(cl.block_rank());
     SEL_TRACE(0);
+    pdl_wait();  // global memory is read only from here on
+    pdl_trigger();
     const int b = blockIdx.y;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t s0 = cu_seqlens[b], s1 = cu_seqlens[b + 1];
@@ -424,6 +426,8 @@ __global__ void __launch_bounds__(256)
 gather_rows_kernel(const uint4* __restrict__ hidden, const int32_t* __restrict__ kept_idx, int64_t M, int64_t T,
                    int vecs_per_row, uint4* __restrict__ out) {
     const int lane = threadIdx.x & 31;
+    pdl_wait();  // global memory is read only from here on
+    pdl_trigger();
     const int64_t warps_total = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
     for (int64_t m = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); m < M;
          m += warps_total) {
@@ -463,10 +467,8 @@ cudaError_t launch_select_scan(int mode, const float* scores, const uint8_t* kee
     if (cudaError_t e = ensure_smem_limit(select_scan_kernel, SEL_SMEM_BYTES, attr_set); e != cudaSuccess)
         return e;
     if (B == 0) return cudaSuccess;
-    select_scan_kernel<<<dim3(SEL_CL, B), SEL_THREADS, SEL_SMEM_BYTES, st>>>(mode, scores, keep_in, cu_seqlens, span,
-                                                                            k, cu_kept, keep_out, kept_idx, pos,
-                                                                            rank, gls);
-    return cudaGetLastError();
+    return launch_pdl(select_scan_kernel, dim3(SEL_CL, B), dim3(SEL_THREADS), static_cast<size_t>(SEL_SMEM_BYTES), st,
+                      mode, scores, keep_in, cu_seqlens, span, k, cu_kept, keep_out, kept_idx, pos, rank, gls);
 }
 
 cudaError_t launch_gather_rows(const uint16_t* hidden, const int32_t* kept_idx, int64_t M_total, int64_t T, int D,
@@ -480,11 +482,8 @@ cudaError_t launch_gather_rows(const uint16_t* hidden, const int32_t* kept_idx, 
     const int grid = static_cast<int>(blocks_needed < static_cast<int64_t>(sms) * 8 ? blocks_needed : sms * 8);
     const uint4* h = reinterpret_cast<const uint4*>(hidden);
     uint4* o = reinterpret_cast<uint4*>(hidden_kept);
-    if (vpr >= 256)
-        gather_rows_kernel<8><<<grid, 256, 0, st>>>(h, kept_idx, M_total, T, vpr, o);
-    else
-        gather_rows_kernel<2><<<grid, 256, 0, st>>>(h, kept_idx, M_total, T, vpr, o);
-    return cudaGetLastError();
+    if (vpr >= 256) return launch_pdl(gather_rows_kernel<8>, dim3(grid), dim3(256), 0, st, h, kept_idx, M_total, T, vpr, o);
+    return launch_pdl(gather_rows_kernel<2>, dim3(grid), dim3(256), 0, st, h, kept_idx, M_total, T, vpr, o);
 }
 
 }  // namespace tg

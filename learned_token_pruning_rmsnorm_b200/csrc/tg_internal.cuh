@@ -11,6 +11,33 @@
 
 namespace tg {
 
+// Programmatic dependent launch.  Kernels of the path are launched with
+// programmatic stream serialisation, so that a kernel can be resident, and
+// through the part of its prologue that reads no global memory (barrier init,
+// TMEM allocation, descriptor prefetch), while the kernel before it in the
+// stream finishes.  Each such kernel executes pdl_wait() before its first read
+// of global memory (the wait returns once the preceding grid has completed and
+// its writes are visible; without the launch attribute it returns at once) and
+// pdl_trigger() after it, which lets the next kernel be scheduled early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // Raises a kernel's dynamic shared-memory limit once per device (the
 // attribute is per device; `done` holds one bit per device ordinal).
 template <typename Kernel>
