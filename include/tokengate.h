@@ -260,9 +260,29 @@ typedef struct tg_prefill_layer_args {
     float* const* lse;          /* n_layers x [M, Hq] out, array or entries may be NULL */
     void* attn_ws;              /* scratch of tg_gated_attention, shared by the layers (may be NULL) */
     size_t attn_ws_bytes;
+    /* optional: more row-major arrays gathered by the same map beside the attention, e.g. the
+       KV cache of the layers below L (see tg_gather_rows); n_gather = 0 for none */
+    int n_gather;
+    const void* const* gather_src;    /* n_gather x [T, row_bytes] */
+    void* const* gather_dst;          /* n_gather x [M, row_bytes] out */
+    const int64_t* gather_row_bytes;  /* n_gather, host */
 } tg_prefill_layer_args;
 
 tg_status tg_gated_prefill_layer(const tg_prefill_layer_args* args, tg_stream_t stream);
+
+/*
+ * Row gather by the compaction map: dst[m, :] = src[kept_idx[m], :] for
+ * m < M, rows of row_bytes bytes (a multiple of 16; src and dst 16-byte
+ * aligned, device).  The serving path of the pages gathers the lower
+ * layers' KV cache to the kept tokens on a separate stream (AI summary,
+ * "Methodology in Plain English"): with src the [T, Hkv, d] K or V cache of
+ * a layer below L (row_bytes = 2 * Hkv * d for bf16) this is that gather.
+ * Entries of kept_idx outside [0, T) leave their row unwritten.
+ * tg_gated_prefill_layer runs the same gather for args->gather_* beside the
+ * attention.
+ */
+tg_status tg_gather_rows(const void* src, int64_t T, int64_t row_bytes, const int32_t* kept_idx, int64_t M,
+                         void* dst, tg_stream_t stream);
 
 /*
  * Device status word (failure detection).  Every wait inside the kernels

@@ -23,7 +23,8 @@ from ._lib import TokenGateError, load  # noqa: F401
 
 __all__ = [
     "TokenGateError", "load", "tg_abi_version", "tg_kept_count", "tg_gate_prepare", "tg_score",
-    "tg_select_topk", "tg_compact", "tg_gather_kept", "tg_gated_attention", "tg_gated_prefill_layer",
+    "tg_select_topk", "tg_compact", "tg_gather_kept", "tg_gather_rows", "tg_gated_attention",
+    "tg_gated_prefill_layer",
     "tg_device_status", "tg_selftest_bounded_wait",
 ]
 
@@ -144,6 +145,25 @@ def tg_gather_kept(hidden, kept_idx, hidden_kept=None):
     return hidden_kept
 
 
+def tg_gather_rows(src, kept_idx, dst=None):
+    """dst[m] = src[kept_idx[m]] for any contiguous device tensor src of shape
+    [T, ...] whose rows are a multiple of 16 bytes (e.g. a layer's [T, Hkv, d]
+    K or V cache).  Returns dst ([M, ...], same dtype)."""
+    if not src.is_cuda or not src.is_contiguous():
+        raise ValueError("src must be a contiguous CUDA tensor")
+    _dev(kept_idx, torch.int32, "kept_idx")
+    T = src.shape[0]
+    M = kept_idx.shape[0]
+    row_bytes = (src[0].numel() if T > 0 else int(np.prod(src.shape[1:]))) * src.element_size()
+    if dst is None:
+        dst = torch.empty((M,) + tuple(src.shape[1:]), dtype=src.dtype, device=src.device)
+    if not dst.is_contiguous() or dst.dtype != src.dtype or tuple(dst.shape) != (M,) + tuple(src.shape[1:]):
+        raise ValueError("dst must be a contiguous [M, ...] tensor of src's dtype")
+    _lib.check(load().tg_gather_rows(src.data_ptr(), T, row_bytes, kept_idx.data_ptr(), M, _lib.ptr(dst),
+                                     _lib.stream_handle(src.device)))
+    return dst
+
+
 def tg_compact(hidden, scores, keep, cu_seqlens, span, cu_kept, M_total: int, with_hidden: bool = True):
     """Returns a dict with hidden_kept (or None), pos, rank, gls, kept_idx."""
     T = scores.shape[0]
@@ -255,7 +275,9 @@ class PrefillCall:
     loops, CUDA-graph capture) only cross the ABI."""
 
     def __init__(self, hidden, cu_seqlens, span, k, Wg, b1, w2, b2, eps, layers, bufs: PrefillBuffers,
-                 Hq, Hkv, d, sm_scale=None):
+                 Hq, Hkv, d, sm_scale=None, gathers=()):
+        """`gathers`: (src [T, ...], dst [M, ...]) pairs of contiguous device tensors that
+        the call gathers by the compaction map beside the attention (tg_gather_rows)."""
         dev = hidden.device
         T, D = hidden.shape
         I = Wg.shape[0]
@@ -297,6 +319,16 @@ class PrefillCall:
         self.ws = attention_workspace(a.B, self.max_M, Hq, Hkv, d, dev) if nl > 0 else None
         a.attn_ws = _lib.ptr(self.ws)
         a.attn_ws_bytes = 0 if self.ws is None else self.ws.numel()
+        gathers = list(gathers)
+        ng = len(gathers)
+        self._gsrc = (C.c_void_p * max(ng, 1))(*[src.data_ptr() for src, _ in gathers])
+        self._gdst = (C.c_void_p * max(ng, 1))(*[dst.data_ptr() for _, dst in gathers])
+        self._grow = (C.c_int64 * max(ng, 1))(*[src[0].numel() * src.element_size() for src, _ in gathers])
+        self.keep_alive.append(gathers)
+        a.n_gather = ng
+        a.gather_src = C.cast(self._gsrc, C.POINTER(C.c_void_p))
+        a.gather_dst = C.cast(self._gdst, C.POINTER(C.c_void_p))
+        a.gather_row_bytes = C.cast(self._grow, C.POINTER(C.c_int64))
         self.args = a
         self.device = dev
         self.bufs = bufs

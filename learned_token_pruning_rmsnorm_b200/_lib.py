@@ -42,6 +42,8 @@ class PrefillLayerArgs(C.Structure):
         ("n_layers", i32), ("Hq", i32), ("Hkv", i32), ("d", i32), ("sm_scale", f32),
         ("q", P), ("kk", P), ("v", P), ("g", P), ("c", P), ("out", P), ("lse", P),
         ("attn_ws", P), ("attn_ws_bytes", C.c_size_t),
+        ("n_gather", C.c_int), ("gather_src", C.POINTER(P)), ("gather_dst", C.POINTER(P)),
+        ("gather_row_bytes", C.POINTER(C.c_int64)),
     ]
 
 
@@ -59,6 +61,7 @@ SIGNATURES = {
     "tg_gated_attention_workspace_size": ([i32, i32, i32, i32, i32], C.c_size_t),
     "tg_gated_attention_noalloc": ([P, P, P, P, i32, i64, i32, i32, i32, i32, P, P, P, P, P, f32, P, P, P], i32),
     "tg_gated_prefill_layer": ([C.POINTER(PrefillLayerArgs), P], i32),
+    "tg_gather_rows": ([P, i64, i64, P, i64, P, P], i32),
     "tg_device_status": ([P, i32, P], i32),
     "tg_selftest_bounded_wait": ([i64, P], i32),
 }

@@ -471,19 +471,26 @@ cudaError_t launch_select_scan(int mode, const float* scores, const uint8_t* kee
                       mode, scores, keep_in, cu_seqlens, span, k, cu_kept, keep_out, kept_idx, pos, rank, gls);
 }
 
-cudaError_t launch_gather_rows(const uint16_t* hidden, const int32_t* kept_idx, int64_t M_total, int64_t T, int D,
-                               uint16_t* hidden_kept, cudaStream_t st) {
+cudaError_t launch_gather_bytes(const void* src, const int32_t* kept_idx, int64_t M_total, int64_t T,
+                                int64_t row_bytes, void* dst, cudaStream_t st) {
     if (M_total == 0) return cudaSuccess;
-    const int vpr = D / 8;
+    const int64_t vpr64 = row_bytes / 16;
+    if (vpr64 <= 0 || vpr64 * 16 != row_bytes || vpr64 > (int64_t(1) << 30)) return cudaErrorInvalidValue;
+    const int vpr = static_cast<int>(vpr64);
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t blocks_needed = (M_total + 7) / 8;
     const int grid = static_cast<int>(blocks_needed < static_cast<int64_t>(sms) * 8 ? blocks_needed : sms * 8);
-    const uint4* h = reinterpret_cast<const uint4*>(hidden);
-    uint4* o = reinterpret_cast<uint4*>(hidden_kept);
+    const uint4* h = static_cast<const uint4*>(src);
+    uint4* o = static_cast<uint4*>(dst);
     if (vpr >= 256) return launch_pdl(gather_rows_kernel<8>, dim3(grid), dim3(256), 0, st, h, kept_idx, M_total, T, vpr, o);
     return launch_pdl(gather_rows_kernel<2>, dim3(grid), dim3(256), 0, st, h, kept_idx, M_total, T, vpr, o);
+}
+
+cudaError_t launch_gather_rows(const uint16_t* hidden, const int32_t* kept_idx, int64_t M_total, int64_t T, int D,
+                               uint16_t* hidden_kept, cudaStream_t st) {
+    return launch_gather_bytes(hidden, kept_idx, M_total, T, static_cast<int64_t>(D) * 2, hidden_kept, st);
 }
 
 }  // namespace tg

@@ -134,7 +134,7 @@ tg_status do_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
 
 extern "C" {
 
-int tg_abi_version(void) { return 1; }
+int tg_abi_version(void) { return 2; }
 
 const char* tg_last_error_string(void) { return g_last_error.c_str(); }
 
@@ -218,6 +218,17 @@ tg_status tg_compact(const uint16_t* hidden, const float* scores, const uint8_t*
                        "tg_compact gather launch");
 }
 
+tg_status tg_gather_rows(const void* src, int64_t T, int64_t row_bytes, const int32_t* kept_idx, int64_t M, void* dst,
+                         tg_stream_t stream) {
+    TG_REQUIRE(T >= 0 && M >= 0 && row_bytes >= 0, "negative size");
+    if (M == 0 || row_bytes == 0) return TG_OK;
+    TG_REQUIRE(src && kept_idx && dst, "null pointer argument");
+    TG_SUPPORT(row_bytes % 16 == 0, "row_bytes=%lld must be a multiple of 16", (long long)row_bytes);
+    TG_REQUIRE(aligned16(src) && aligned16(dst), "src and dst must be 16-byte aligned");
+    if (tg_status s = check_device()) return s;
+    return cuda_status(tg::launch_gather_bytes(src, kept_idx, M, T, row_bytes, dst, stream), "tg_gather_rows launch");
+}
+
 tg_status tg_gated_attention_noalloc(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* cu_kept,
                                      int B, int64_t M_total, int max_M, int Hq, int Hkv, int d, const int32_t* pos,
                                      const int32_t* rank, const float* gls, const float* g, const float* c,
@@ -287,6 +298,18 @@ tg_status tg_gated_prefill_layer(const tg_prefill_layer_args* a, tg_stream_t str
     TG_REQUIRE(a->M_total == 0 || (a->pos && a->rank && a->gls && a->kept_idx), "null compaction output");
     TG_REQUIRE(aligned16(a->hidden) && aligned16(a->Wg), "hidden and Wg must be 16-byte aligned");
     if (a->hidden_kept) TG_REQUIRE(aligned16(a->hidden_kept), "hidden_kept must be 16-byte aligned");
+    TG_REQUIRE(a->n_gather >= 0, "negative n_gather");
+    if (a->n_gather > 0) {
+        TG_REQUIRE(a->gather_src && a->gather_dst && a->gather_row_bytes, "null gather arrays");
+        for (int i = 0; i < a->n_gather; ++i) {
+            TG_REQUIRE(a->gather_src[i] && a->gather_dst[i], "null gather tensor %d", i);
+            TG_SUPPORT(a->gather_row_bytes[i] > 0 && a->gather_row_bytes[i] % 16 == 0,
+                       "gather %d: row_bytes=%lld must be a positive multiple of 16", i,
+                       (long long)a->gather_row_bytes[i]);
+            TG_REQUIRE(aligned16(a->gather_src[i]) && aligned16(a->gather_dst[i]),
+                       "gather %d: tensors must be 16-byte aligned", i);
+        }
+    }
     if (tg_status s = check_device()) return s;
     cudaStream_t st = stream;
     if (tg_status s = do_score(a->hidden, a->cu_seqlens, a->span, a->B, a->T, a->D, a->Wg, a->b1, a->w2, a->b2, a->I,
@@ -302,7 +325,8 @@ tg_status tg_gated_prefill_layer(const tg_prefill_layer_args* a, tg_stream_t str
     // layers (tensor-bound); both read only the compaction map
     std::unique_lock<std::mutex> lk(g_side_mu);
     SideStream* side = nullptr;
-    const bool fork = a->hidden_kept && a->n_layers > 0;
+    const bool gathers = a->hidden_kept || a->n_gather > 0;
+    const bool fork = gathers && a->n_layers > 0;
     if (fork) {
         if (tg_status s = cuda_status(side_stream(&side), "side stream")) return s;
         if (tg_status s = cuda_status(cudaEventRecord(side->fork, st), "fork record")) return s;
@@ -312,6 +336,13 @@ tg_status tg_gated_prefill_layer(const tg_prefill_layer_args* a, tg_stream_t str
         if (tg_status s = cuda_status(tg::launch_gather_rows(a->hidden, a->kept_idx, a->M_total, a->T, a->D,
                                                              a->hidden_kept, fork ? side->stream : st),
                                       "gather launch"))
+            return s;
+    }
+    for (int i = 0; i < a->n_gather; ++i) {
+        if (tg_status s = cuda_status(tg::launch_gather_bytes(a->gather_src[i], a->kept_idx, a->M_total, a->T,
+                                                              a->gather_row_bytes[i], a->gather_dst[i],
+                                                              fork ? side->stream : st),
+                                      "extra gather launch"))
             return s;
     }
     tg_status result = TG_OK;

@@ -93,6 +93,10 @@ cudaError_t launch_select_scan(int mode, const float* scores, const uint8_t* kee
                                uint8_t* keep_out, int32_t* kept_idx, int32_t* pos, int32_t* rank, float* gls,
                                cudaStream_t st);
 
+// dst[m, :] = src[kept_idx[m], :] for rows of row_bytes bytes (a multiple of 16; both
+// pointers 16-byte aligned); rows whose index lies outside [0, T) are left untouched
+cudaError_t launch_gather_bytes(const void* src, const int32_t* kept_idx, int64_t M_total, int64_t T,
+                                int64_t row_bytes, void* dst, cudaStream_t st);
 cudaError_t launch_gather_rows(const uint16_t* hidden, const int32_t* kept_idx, int64_t M_total, int64_t T, int D,
                                uint16_t* hidden_kept, cudaStream_t st);
 

@@ -44,7 +44,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version(lib):
-    assert lib.tg_abi_version() == 1
+    assert lib.tg_abi_version() == 2
 
 
 def test_kept_count_host_helper(lib):
@@ -115,3 +115,14 @@ def test_product_code_never_imports_the_oracle():
                 src = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in src and "from oracle" not in src, f
                 assert "tg_oracle" not in src and "liboracle" not in src, f
+
+
+def test_gather_rows_refuses_bad_rows_before_launch(lib):
+    from learned_token_pruning_rmsnorm_b200 import _lib
+    P = C.c_void_p(16)  # never dereferenced: validation fails first
+    st = lib.tg_gather_rows(P, 10, 24, P, 4, P, None)  # 24-byte rows: not a multiple of 16
+    assert st == _lib.TG_ERR_UNSUPPORTED
+    assert b"row_bytes=24" in lib.tg_last_error_string()
+    st = lib.tg_gather_rows(C.c_void_p(8), 10, 32, P, 4, P, None)  # misaligned source
+    assert st == _lib.TG_ERR_INVALID_ARG
+    assert lib.tg_gather_rows(None, 0, 32, None, 0, None, None) == _lib.TG_OK  # nothing to gather

@@ -310,3 +310,68 @@ def test_prefill_layer_end_to_end(tg, name):
         H.assert_attention_close(bufs.out[l].float().cpu().numpy(), out_ref, f"{name} layer {l}")
         assert np.max(np.abs(bufs.lse[l].cpu().numpy() - lse_ref)) <= H.LSE_ABS
     assert math.isfinite(float(s[m].sum()))
+
+
+# ------------------------------------------------------------------ KV-cache gather (next row f2)
+
+@pytest.mark.parametrize("row_shape", [(8, 128), (2, 64), (8,), (24,), (1, 2056)])
+def test_gather_rows_matches_oracle_gather(tg, row_shape):
+    """dst[m] = src[kept_idx[m]] for rows of any width that is a multiple of 16 bytes
+    (the [T, Hkv, d] K/V cache of a layer below the gate among them), bit-exact against
+    the oracle's compaction gather on the same map."""
+    w = CONFIGS["c1_16k"]
+    cu, span, k = w.cu_seqlens(), w.span_array(), w.budget_array()
+    s32, _ = case_scores("c1_16k")
+    keep = oracle.select_topk(s32, cu, span, k)
+    rng = np.random.default_rng(7)
+    width = int(np.prod(row_shape))
+    src_bits = rng.integers(0, 65536, size=(w.T, width)).astype(np.uint16)
+    ref = oracle.compact(src_bits, s32, keep, cu, span)
+    kept_idx = H.i32_dev(ref["src"])
+    src = H.bf16_dev(src_bits).reshape((w.T,) + tuple(row_shape))
+    dst = tg.tg_gather_rows(src, kept_idx)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(H.bf16_host_bits(dst.reshape(dst.shape[0], -1)), ref["hidden_kept"])
+
+
+def test_gather_rows_skips_indices_outside_the_source(tg):
+    T, width = 64, 16
+    src_bits = np.arange(T * width, dtype=np.uint16).reshape(T, width)
+    idx = np.array([3, -1, T, 0, T - 1, 2 ** 30], np.int32)
+    src = H.bf16_dev(src_bits)
+    dst = torch.full((len(idx), width), 7.0, dtype=torch.bfloat16, device="cuda")
+    sentinel = H.bf16_host_bits(dst).copy()
+    tg.tg_gather_rows(src, H.i32_dev(idx), dst)
+    torch.cuda.synchronize()
+    got = H.bf16_host_bits(dst)
+    for m, t in enumerate(idx):
+        want = src_bits[t] if 0 <= t < T else sentinel[m]
+        np.testing.assert_array_equal(got[m], want)
+
+
+def test_prefill_layer_gathers_kv_cache_beside_attention(tg):
+    """tg_gated_prefill_layer with extra arrays: the K and V cache of a lower layer are
+    gathered by the same map on the side stream, bit-exact."""
+    name = "c0_tiny"
+    w, gi, Wg_ref, s_ref = gate_case(name)
+    cu, span, k = w.cu_seqlens(), w.span_array(), w.budget_array()
+    M, _ = tg.tg_kept_count(cu, span, k)
+    layers_np = [make_attention_inputs(w, M, layer=0)]
+    layers = [{"q": H.bf16_dev(a["q"]), "k": H.bf16_dev(a["k"]), "v": H.bf16_dev(a["v"]),
+               "g": H.f32_dev(a["g"]), "c": H.f32_dev(a["c"])} for a in layers_np]
+    rng = np.random.default_rng(11)
+    kc_bits = rng.integers(0, 65536, size=(w.T, w.Hkv * w.d)).astype(np.uint16)
+    vc_bits = rng.integers(0, 65536, size=(w.T, w.Hkv * w.d)).astype(np.uint16)
+    kc = H.bf16_dev(kc_bits).reshape(w.T, w.Hkv, w.d)
+    vc = H.bf16_dev(vc_bits).reshape(w.T, w.Hkv, w.d)
+    kd = torch.empty((M, w.Hkv, w.d), dtype=torch.bfloat16, device="cuda")
+    vd = torch.empty_like(kd)
+    bufs = tg.PrefillBuffers(w.T, w.D, M, 1, w.Hq, w.d, "cuda")
+    call = tg.PrefillCall(H.bf16_dev(gi["hidden"]), cu, span, k, H.bf16_dev(Wg_ref), H.f32_dev(gi["b1"]),
+                          H.f32_dev(gi["w2"]), gi["b2"], w.eps, layers, bufs, w.Hq, w.Hkv, w.d,
+                          gathers=[(kc, kd), (vc, vd)])
+    call()
+    torch.cuda.synchronize()
+    idx = bufs.kept_idx.cpu().numpy()
+    np.testing.assert_array_equal(H.bf16_host_bits(kd.reshape(M, -1)), kc_bits[idx])
+    np.testing.assert_array_equal(H.bf16_host_bits(vd.reshape(M, -1)), vc_bits[idx])
