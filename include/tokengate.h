@@ -271,6 +271,34 @@ typedef struct tg_prefill_layer_args {
 tg_status tg_gated_prefill_layer(const tg_prefill_layer_args* args, tg_stream_t stream);
 
 /*
+ * Full-length (training-time) token-gated attention for a sampled budget.
+ * The pages train with one full-budget forward and one forward at a smaller
+ * budget drawn per step (AI summary, "Methodology in Plain English"); in the
+ * full-length form of the smaller-budget pass the pruned keys are masked out
+ * of every query's softmax (bias -inf) and the rows of pruned queries are
+ * not computed.  This library defines, for q, k, v of full length
+ * ([T, Hq, d], [T, Hkv, d], [T, Hkv, d] bf16) and the budgets kbud[B]:
+ *   keep = tg_select_topk(scores, cu_seqlens, span, kbud)
+ *   out[t] = 0 for every pruned t; for kept t it is the gated attention of
+ *   tg_gated_attention over the kept keys j <= t of t's sequence, with
+ *   pos/rank/gls from the compaction of `keep`
+ * (the same numbers as compacting, attending and scattering back, which is
+ * also how it runs: select, gather of the kept rows, the compacted kernel,
+ * scatter; every fully masked key tile is skipped).  cu_kept / M_total /
+ * max_M come from tg_kept_count(cu_seqlens, span, kbud) on the host.
+ * keep_out ([T] u8) receives the flags when non-NULL.  ws (256-byte aligned,
+ * zeroed once before first use; the calls leave it reusable) holds
+ * tg_masked_gated_attention_workspace_size(B, T, M_total, max_M, Hq, Hkv, d)
+ * bytes.  sm_scale as in tg_gated_attention.
+ */
+size_t tg_masked_gated_attention_workspace_size(int B, int64_t T, int64_t M_total, int max_M, int Hq, int Hkv, int d);
+tg_status tg_masked_gated_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, const float* scores,
+                                    const int32_t* cu_seqlens, const int32_t* span, const int32_t* kbud,
+                                    const int32_t* cu_kept, int B, int64_t T, int64_t M_total, int max_M, int Hq,
+                                    int Hkv, int d, const float* g, const float* c, float sm_scale, uint16_t* out,
+                                    uint8_t* keep_out, void* ws, size_t ws_bytes, tg_stream_t stream);
+
+/*
  * Row gather by the compaction map: dst[m, :] = src[kept_idx[m], :] for
  * m < M, rows of row_bytes bytes (a multiple of 16; src and dst 16-byte
  * aligned, device).  The serving path of the pages gathers the lower

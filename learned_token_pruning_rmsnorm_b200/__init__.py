@@ -24,6 +24,7 @@ from ._lib import TokenGateError, load  # noqa: F401
 __all__ = [
     "TokenGateError", "load", "tg_abi_version", "tg_kept_count", "tg_gate_prepare", "tg_score",
     "tg_select_topk", "tg_compact", "tg_gather_kept", "tg_gather_rows", "tg_gated_attention",
+    "tg_masked_gated_attention",
     "tg_gated_prefill_layer",
     "tg_device_status", "tg_selftest_bounded_wait",
 ]
@@ -204,6 +205,45 @@ def attention_workspace(B: int, max_M: int, Hq: int, Hkv: int, d: int, device) -
         ws = torch.zeros(n, dtype=torch.uint8, device=device)
         _WS_CACHE[key] = ws
     return ws
+
+
+def tg_masked_gated_attention(q, k, v, scores, cu_seqlens, span, kbud, g, c, sm_scale: float | None = None,
+                              out=None):
+    """Full-length gated attention for the budgets `kbud`: pruned keys masked, rows of
+    pruned queries zero.  q [T, Hq, d], k/v [T, Hkv, d] bf16, scores [T] fp32.
+    Returns (out [T, Hq, d] bf16, keep [T] uint8)."""
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    dev = q.device
+    for t, nm in ((q, "q"), (k, "k"), (v, "v")):
+        _dev(t, torch.bfloat16, nm)
+    _dev(scores, torch.float32, "scores", (T,))
+    _dev(g, torch.float32, "g", (Hq,))
+    _dev(c, torch.float32, "c", (Hq,))
+    to_host = lambda x: x.cpu() if isinstance(x, torch.Tensor) else x  # noqa: E731
+    M, cu_kept = tg_kept_count(to_host(cu_seqlens), to_host(span), to_host(kbud))
+    max_M = int(np.max(np.diff(cu_kept))) if len(cu_kept) > 1 else 0
+    cu = _i32_dev(cu_seqlens, dev, "cu_seqlens")
+    sp = _i32_dev(span, dev, "span")
+    kb = _i32_dev(kbud, dev, "kbud")
+    ck = torch.from_numpy(cu_kept).to(dev)
+    B = cu.numel() - 1
+    if out is None:
+        out = torch.empty((T, Hq, d), dtype=torch.bfloat16, device=dev)
+    keep = torch.empty(T, dtype=torch.uint8, device=dev)
+    n = int(load().tg_masked_gated_attention_workspace_size(B, T, M, max_M, Hq, Hkv, d))
+    key = (torch.device(dev), n, "masked")
+    ws = _WS_CACHE.get(key)
+    if ws is None:
+        ws = torch.zeros(max(n, 256), dtype=torch.uint8, device=dev)
+        _WS_CACHE[key] = ws
+    scale = float(1.0 / math.sqrt(d) if sm_scale is None else sm_scale)
+    _lib.check(load().tg_masked_gated_attention(q.data_ptr(), k.data_ptr(), v.data_ptr(), scores.data_ptr(),
+                                                cu.data_ptr(), sp.data_ptr(), kb.data_ptr(), ck.data_ptr(), B, T, M,
+                                                max_M, Hq, Hkv, d, g.data_ptr(), c.data_ptr(), scale, out.data_ptr(),
+                                                keep.data_ptr(), ws.data_ptr(), ws.numel(),
+                                                _lib.stream_handle(dev)))
+    return out, keep
 
 
 def tg_gated_attention(q, k, v, cu_kept, max_M: int, pos, rank, gls, g, c, sm_scale: float | None = None,

@@ -451,6 +451,38 @@ gather_rows_kernel(const uint4* __restrict__ hidden, const int32_t* __restrict__
     }
 }
 
+// Row scatter out[idx[m], :] = in[m, :] (the inverse of the gather), one warp per
+// row; indices outside [0, T) write nothing.
+template <int VPL>
+__global__ void __launch_bounds__(256)
+scatter_rows_kernel(const uint4* __restrict__ in, const int32_t* __restrict__ idx, int64_t M, int64_t T,
+                    int vecs_per_row, uint4* __restrict__ out) {
+    const int lane = threadIdx.x & 31;
+    pdl_wait();  // global memory is read only from here on
+    pdl_trigger();
+    const int64_t warps_total = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+    for (int64_t m = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); m < M;
+         m += warps_total) {
+        const int64_t dst = idx[m];
+        if (dst < 0 || dst >= T) continue;
+        const uint4* s = in + m * vecs_per_row;
+        uint4* d = out + dst * vecs_per_row;
+        for (int c0 = 0; c0 < vecs_per_row; c0 += 32 * VPL) {
+            uint4 r[VPL];
+#pragma unroll
+            for (int e = 0; e < VPL; ++e) {
+                const int c = c0 + e * 32 + lane;
+                if (c < vecs_per_row) r[e] = __ldg(s + c);
+            }
+#pragma unroll
+            for (int e = 0; e < VPL; ++e) {
+                const int c = c0 + e * 32 + lane;
+                if (c < vecs_per_row) d[c] = r[e];
+            }
+        }
+    }
+}
+
 }  // namespace
 
 #ifdef TG_TRACE
@@ -486,6 +518,23 @@ cudaError_t launch_gather_bytes(const void* src, const int32_t* kept_idx, int64_
     uint4* o = static_cast<uint4*>(dst);
     if (vpr >= 256) return launch_pdl(gather_rows_kernel<8>, dim3(grid), dim3(256), 0, st, h, kept_idx, M_total, T, vpr, o);
     return launch_pdl(gather_rows_kernel<2>, dim3(grid), dim3(256), 0, st, h, kept_idx, M_total, T, vpr, o);
+}
+
+cudaError_t launch_scatter_bytes(const void* src, const int32_t* idx, int64_t M, int64_t T, int64_t row_bytes,
+                                 void* dst, cudaStream_t st) {
+    if (M == 0) return cudaSuccess;
+    const int64_t vpr64 = row_bytes / 16;
+    if (vpr64 <= 0 || vpr64 * 16 != row_bytes || vpr64 > (int64_t(1) << 30)) return cudaErrorInvalidValue;
+    const int vpr = static_cast<int>(vpr64);
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t blocks_needed = (M + 7) / 8;
+    const int grid = static_cast<int>(blocks_needed < static_cast<int64_t>(sms) * 8 ? blocks_needed : sms * 8);
+    const uint4* h = static_cast<const uint4*>(src);
+    uint4* o = static_cast<uint4*>(dst);
+    if (vpr >= 256) return launch_pdl(scatter_rows_kernel<8>, dim3(grid), dim3(256), 0, st, h, idx, M, T, vpr, o);
+    return launch_pdl(scatter_rows_kernel<2>, dim3(grid), dim3(256), 0, st, h, idx, M, T, vpr, o);
 }
 
 cudaError_t launch_gather_rows(const uint16_t* hidden, const int32_t* kept_idx, int64_t M_total, int64_t T, int D,

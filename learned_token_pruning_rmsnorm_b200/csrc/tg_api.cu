@@ -130,9 +130,91 @@ tg_status do_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
                        "tg_gated_attention launch");
 }
 
+// Scratch of tg_masked_gated_attention: keep flags, compaction map, the gathered
+// Q/K/V rows, the compacted output and the attention's own split scratch, each
+// 256-byte aligned.
+struct MaskedWs {
+    size_t keep, idx, pos, rank, gls, qc, kc, vc, oc, attn, attn_bytes, total;
+};
+
+MaskedWs masked_layout(int B, int64_t T, int64_t M, int max_M, int Hq, int Hkv, int d) {
+    auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+    MaskedWs L{};
+    size_t o = 0;
+    L.keep = o; o += al(static_cast<size_t>(T));
+    L.idx = o; o += al(4 * static_cast<size_t>(M));
+    L.pos = o; o += al(4 * static_cast<size_t>(M));
+    L.rank = o; o += al(4 * static_cast<size_t>(M));
+    L.gls = o; o += al(4 * static_cast<size_t>(M));
+    L.qc = o; o += al(2 * static_cast<size_t>(M) * Hq * d);
+    L.kc = o; o += al(2 * static_cast<size_t>(M) * Hkv * d);
+    L.vc = o; o += al(2 * static_cast<size_t>(M) * Hkv * d);
+    L.oc = o; o += al(2 * static_cast<size_t>(M) * Hq * d);
+    L.attn = o;
+    L.attn_bytes = B > 0 && max_M > 0 ? tg::attention_workspace_bytes(B, max_M, Hq, Hkv, d) : 0;
+    o += al(L.attn_bytes);
+    L.total = o;
+    return L;
+}
+
 }  // namespace
 
 extern "C" {
+
+size_t tg_masked_gated_attention_workspace_size(int B, int64_t T, int64_t M_total, int max_M, int Hq, int Hkv, int d) {
+    if (B <= 0 || T <= 0 || M_total < 0 || max_M < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 ||
+        (d != 64 && d != 128))
+        return 0;
+    return masked_layout(B, T, M_total, max_M, Hq, Hkv, d).total;
+}
+
+tg_status tg_masked_gated_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, const float* scores,
+                                    const int32_t* cu_seqlens, const int32_t* span, const int32_t* kbud,
+                                    const int32_t* cu_kept, int B, int64_t T, int64_t M_total, int max_M, int Hq,
+                                    int Hkv, int d, const float* g, const float* c, float sm_scale, uint16_t* out,
+                                    uint8_t* keep_out, void* ws, size_t ws_bytes, tg_stream_t stream) {
+    TG_REQUIRE(B >= 0 && T >= 0 && M_total >= 0 && M_total <= T && max_M >= 0, "bad sizes");
+    if (tg_status s = check_attn_shape(Hq, Hkv, d)) return s;
+    TG_REQUIRE(sm_scale > 0.f, "sm_scale must be positive");
+    if (B == 0 || T == 0) return TG_OK;
+    TG_REQUIRE(q && k && v && scores && cu_seqlens && span && kbud && cu_kept && g && c && out && ws,
+               "null pointer argument");
+    TG_REQUIRE(aligned16(q) && aligned16(k) && aligned16(v) && aligned16(out),
+               "q, k, v and out must be 16-byte aligned");
+    TG_REQUIRE((reinterpret_cast<uintptr_t>(ws) & 255u) == 0, "ws must be 256-byte aligned");
+    TG_REQUIRE(M_total == 0 || max_M > 0, "max_M must bound the longest kept sequence");
+    const MaskedWs L = masked_layout(B, T, M_total, max_M, Hq, Hkv, d);
+    TG_REQUIRE(ws_bytes >= L.total, "ws holds %zu bytes, this call needs %zu", ws_bytes, L.total);
+    if (tg_status s = check_device()) return s;
+    cudaStream_t st = stream;
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    uint8_t* keep = keep_out ? keep_out : base + L.keep;
+    int32_t* idx = reinterpret_cast<int32_t*>(base + L.idx);
+    int32_t* pos = reinterpret_cast<int32_t*>(base + L.pos);
+    int32_t* rank = reinterpret_cast<int32_t*>(base + L.rank);
+    float* gls = reinterpret_cast<float*>(base + L.gls);
+    uint16_t* qc = reinterpret_cast<uint16_t*>(base + L.qc);
+    uint16_t* kc = reinterpret_cast<uint16_t*>(base + L.kc);
+    uint16_t* vc = reinterpret_cast<uint16_t*>(base + L.vc);
+    uint16_t* oc = reinterpret_cast<uint16_t*>(base + L.oc);
+    // rows of pruned queries are zero; the kept rows are overwritten below
+    if (tg_status s = cuda_status(cudaMemsetAsync(out, 0, static_cast<size_t>(T) * Hq * d * 2, st), "out clear"))
+        return s;
+    if (tg_status s = cuda_status(tg::launch_select_scan(0, scores, nullptr, cu_seqlens, span, kbud, cu_kept, B, T,
+                                                         keep, idx, pos, rank, gls, st),
+                                  "masked select launch"))
+        return s;
+    if (M_total == 0) return TG_OK;
+    const int64_t qrow = static_cast<int64_t>(Hq) * d * 2, kvrow = static_cast<int64_t>(Hkv) * d * 2;
+    if (tg_status s = cuda_status(tg::launch_gather_bytes(q, idx, M_total, T, qrow, qc, st), "q gather")) return s;
+    if (tg_status s = cuda_status(tg::launch_gather_bytes(k, idx, M_total, T, kvrow, kc, st), "k gather")) return s;
+    if (tg_status s = cuda_status(tg::launch_gather_bytes(v, idx, M_total, T, kvrow, vc, st), "v gather")) return s;
+    if (tg_status s = do_attention(qc, kc, vc, cu_kept, B, M_total, max_M, Hq, Hkv, d, pos, rank, gls, g, c, sm_scale,
+                                   oc, nullptr, L.attn_bytes ? base + L.attn : nullptr, L.attn_bytes, st))
+        return s;
+    return cuda_status(tg::launch_scatter_bytes(oc, idx, M_total, T, qrow, out, st), "out scatter");
+}
+
 
 int tg_abi_version(void) { return 2; }
 

@@ -97,6 +97,9 @@ cudaError_t launch_select_scan(int mode, const float* scores, const uint8_t* kee
 // pointers 16-byte aligned); rows whose index lies outside [0, T) are left untouched
 cudaError_t launch_gather_bytes(const void* src, const int32_t* kept_idx, int64_t M_total, int64_t T,
                                 int64_t row_bytes, void* dst, cudaStream_t st);
+// dst[idx[m], :] = src[m, :] (rows of row_bytes bytes, as for launch_gather_bytes)
+cudaError_t launch_scatter_bytes(const void* src, const int32_t* idx, int64_t M, int64_t T, int64_t row_bytes,
+                                 void* dst, cudaStream_t st);
 cudaError_t launch_gather_rows(const uint16_t* hidden, const int32_t* kept_idx, int64_t M_total, int64_t T, int D,
                                uint16_t* hidden_kept, cudaStream_t st);
 

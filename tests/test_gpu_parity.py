@@ -375,3 +375,73 @@ def test_prefill_layer_gathers_kv_cache_beside_attention(tg):
     idx = bufs.kept_idx.cpu().numpy()
     np.testing.assert_array_equal(H.bf16_host_bits(kd.reshape(M, -1)), kc_bits[idx])
     np.testing.assert_array_equal(H.bf16_host_bits(vd.reshape(M, -1)), vc_bits[idx])
+
+
+# ------------------------------------------------------------------ full-length masked attention (next row f1)
+
+def _masked_case(name, seed):
+    from workloads import masked_budgets
+    w = CONFIGS[name]
+    cu, span = w.cu_seqlens(), w.span_array()
+    kb = np.array(masked_budgets(w, seed), np.int32)
+    s = make_scores(w.T, std=2.0, seed=21 + seed)
+    ai = make_attention_inputs(w, w.T, layer=seed)  # full-length q, k, v
+    return w, cu, span, kb, s, ai
+
+
+@pytest.mark.parametrize("name,seed,rows_step", [("c0_tiny", 0, None), ("c0_tiny", 1, None),
+                                                 ("c3_full_budget_16k", 0, 128), ("c3_full_budget_16k", 1, 128)])
+def test_masked_attention_matches_oracle(tg, name, seed, rows_step):
+    """Full-length gated attention at a sampled budget (log-uniform in [1, |P|/2]) against
+    the oracle's masked form: keep flags bit-exact, rows of pruned queries exactly zero,
+    kept rows within the attention tolerance."""
+    w, cu, span, kb, s, ai = _masked_case(name, seed)
+    keep_ref = oracle.select_topk(s, cu, span, kb)
+    rows = None
+    if rows_step:
+        rows = np.unique(np.concatenate([np.arange(0, w.T, rows_step), np.arange(w.T - 64, w.T)])).astype(np.int64)
+    out_ref = oracle.masked_gated_attention(ai["q"], ai["k"], ai["v"], cu, span, keep_ref, s, ai["g"], ai["c"],
+                                            rows=rows)
+    out, keep = tg.tg_masked_gated_attention(H.bf16_dev(ai["q"]), H.bf16_dev(ai["k"]), H.bf16_dev(ai["v"]),
+                                             H.f32_dev(s), cu, span, kb, H.f32_dev(ai["g"]), H.f32_dev(ai["c"]))
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(keep.cpu().numpy(), keep_ref)
+    got = out.float().cpu().numpy()
+    if rows is not None:
+        got = got[rows]
+        pruned = keep_ref[rows] == 0
+    else:
+        pruned = keep_ref == 0
+    assert pruned.any() and (~pruned).any()
+    assert (got[pruned] == 0).all()
+    H.assert_attention_close(got, out_ref, f"masked {name} seed {seed}")
+
+
+def test_masked_attention_equals_compacted_path(tg):
+    """The masked call is the compacted kernel on the kept rows: bitwise equal to
+    tg_gated_attention fed the same compaction map."""
+    w, cu, span, kb, s, ai = _masked_case("c3_full_budget_16k", 2)
+    q, k, v = H.bf16_dev(ai["q"]), H.bf16_dev(ai["k"]), H.bf16_dev(ai["v"])
+    g, c = H.f32_dev(ai["g"]), H.f32_dev(ai["c"])
+    s_dev = H.f32_dev(s)
+    out, keep = tg.tg_masked_gated_attention(q, k, v, s_dev, cu, span, kb, g, c)
+    M, cu_kept = tg.tg_kept_count(cu, span, kb)
+    _, cmap = tg.tg_select_topk(s_dev, cu, span, kb, cu_kept=cu_kept, M_total=M)
+    idx = cmap["kept_idx"].long()
+    max_M = int(np.max(np.diff(cu_kept)))
+    outc, _ = tg.tg_gated_attention(q[idx].contiguous(), k[idx].contiguous(), v[idx].contiguous(), cu_kept, max_M,
+                                    cmap["pos"], cmap["rank"], cmap["gls"], g, c, want_lse=True)
+    torch.cuda.synchronize()
+    assert torch.equal(out[idx], outc)
+    pruned = keep == 0
+    assert int(pruned.sum()) == w.T - M
+    assert bool((out[pruned] == 0).all())
+
+
+def test_attention_is_deterministic_with_the_causal_split(tg):
+    """Split query tiles merge in chunk order with both halves at the same precision:
+    repeated calls give identical bits whichever chunk finishes first."""
+    w, comp, ai, gls32, rows, out_ref, lse_ref = attn_case("c2_32k_k2000")
+    outs = [_run_attention(tg, w, comp, ai, gls32) for _ in range(3)]
+    for o, l in outs[1:]:
+        assert np.array_equal(o, outs[0][0]) and np.array_equal(l, outs[0][1])

@@ -6,7 +6,7 @@ so both the CPU oracle and the CUDA path can take their inputs from it without
 sharing any computation.
 """
 
-from .configs import CONFIGS, Workload, get_config  # noqa: F401
+from .configs import CONFIGS, Workload, get_config, masked_budgets  # noqa: F401
 from .gen import (  # noqa: F401
     bf16_bits_to_f32,
     f32_to_bf16_bits,

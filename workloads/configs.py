@@ -90,6 +90,16 @@ def _varlen_budgets(seed: int, n: int, lo: float, hi: float) -> list:
     return [int(round(math.exp(math.log(lo) + x * (math.log(hi) - math.log(lo))))) for x in u]
 
 
+def masked_budgets(w: "Workload", seed: int = 0) -> list:
+    """The smaller budget of a training step, one per sequence: log-uniform in
+    [1, |P_b| / 2] (the pages sample it that way), seeded."""
+    out = []
+    for b, (p0, p1) in enumerate(w.spans):
+        hi = max(1.0, (p1 - p0) / 2.0)
+        out.append(_varlen_budgets(1000 + seed * 97 + b, 1, 1.0, hi)[0])
+    return out
+
+
 def _build() -> dict:
     cfg = {}
     cfg["c0_tiny"] = Workload(
