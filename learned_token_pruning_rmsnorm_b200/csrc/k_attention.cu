@@ -1035,13 +1035,13 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                         const float other_lse = ws.lse2[oidx * BM + r];
                         const float ml = hh ? my_lse1 : my_lse0;
                         // Order-independent merge: this chunk's row is rounded to bf16 exactly as
-                        // the partial of the other was, and the two terms are combined in chunk
-                        // order, so the result does not depend on which chunk arrived first.
-                        const float lse_c0 = chunk == 0 ? ml : other_lse, lse_c1 = chunk == 0 ? other_lse : ml;
-                        const float mx = fmaxf(lse_c0, lse_c1);
-                        const float e0 = ex2_approx(lse_c0 - mx), e1 = ex2_approx(lse_c1 - mx);
-                        const float inv_w = 1.0f / (e0 + e1);
-                        const float w0 = e0 * inv_w, w1 = e1 * inv_w;
+                        // the other's partial was, each weight depends only on its own chunk's
+                        // log-sum-exp and the (commutative) sum, and the two products are added,
+                        // so the result does not depend on which chunk arrived first.
+                        const float mx = fmaxf(ml, other_lse);
+                        const float e_me = ex2_approx(ml - mx), e_ot = ex2_approx(other_lse - mx);
+                        const float inv_w = 1.0f / (e_me + e_ot);
+                        const float w_me = e_me * inv_w, w_ot = e_ot * inv_w;
                         const float inv_l = 1.0f / (hh ? l_tot1 : l_tot0);
                         const uint32_t tO = tmem + lane_addr + 2 * BN + hh * HD + half * (HD / 2);
 #pragma unroll
@@ -1053,15 +1053,15 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                             for (int e = 0; e < 16; ++e) {
                                 const uint32_t w = pw[ch * 16 + e];
                                 const uint32_t mine = pack_bf16x2(o[2 * e] * inv_l, o[2 * e + 1] * inv_l);
-                                const uint32_t a = chunk == 0 ? mine : w, b = chunk == 0 ? w : mine;
-                                o[2 * e] = fmaf(w0, __uint_as_float(a << 16), w1 * __uint_as_float(b << 16));
-                                o[2 * e + 1] = fmaf(w0, __uint_as_float(a & 0xFFFF0000u),
-                                                    w1 * __uint_as_float(b & 0xFFFF0000u));
+                                o[2 * e] = __fadd_rn(__fmul_rn(w_me, __uint_as_float(mine << 16)),
+                                                     __fmul_rn(w_ot, __uint_as_float(w << 16)));
+                                o[2 * e + 1] = __fadd_rn(__fmul_rn(w_me, __uint_as_float(mine & 0xFFFF0000u)),
+                                                         __fmul_rn(w_ot, __uint_as_float(w & 0xFFFF0000u)));
                             }
                             stage_row(hh, o, half * (HD / 64) + ch, 1.0f);
                         }
                         if (valid_row && lse && half == 0)
-                            lse[static_cast<size_t>(qg) * Hq + 2 * pair + hh] = (mx + log2f(e0 + e1)) / LOG2E;
+                            lse[static_cast<size_t>(qg) * Hq + 2 * pair + hh] = (mx + log2f(e_me + e_ot)) / LOG2E;
                     }
                 }
                 write_rows();
