@@ -178,6 +178,39 @@ tg_status tg_gated_attention(const uint16_t* q, const uint16_t* k, const uint16_
                              const int32_t* rank, const float* gls, const float* g, const float* c, float sm_scale,
                              uint16_t* out, float* lse, void* ws, size_t ws_bytes, tg_stream_t stream);
 
+/*
+ * Several gate modules (AI summary, "Future Directions": gates at several
+ * layers, each selecting from what the lower ones kept and each contributing
+ * to the token-gated attention above it).  Same as tg_gated_attention with
+ * the bias summed over the gates:
+ *     b[h,j] = sum_i softplus(g[i][h]) * gls[i][j],  i < n_gates
+ * gls and g are HOST arrays of n_gates DEVICE pointers: gls[i] [M] fp32 is
+ * gate i's logsigmoid per kept row (0 for rows that gate could not prune),
+ * g[i] [Hq] fp32 its gain parameters for this layer.  pos must hold the
+ * ORIGINAL 1-indexed positions and rank the rank among the tokens finally
+ * kept (compose them with tg_gather_rows over the later gates' kept_idx).
+ * 1 <= n_gates <= 4, else TG_ERR_UNSUPPORTED; n_gates = 1 is
+ * tg_gated_attention.  The gates ride in the same extra k-step of the
+ * tensor-core product that carries one gate's bias, so more gates cost no
+ * softmax work.
+ */
+tg_status tg_gated_attention_gates(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* cu_kept,
+                                   int B, int64_t M_total, int max_M, int Hq, int Hkv, int d, const int32_t* pos,
+                                   const int32_t* rank, int n_gates, const float* const* gls, const float* const* g,
+                                   const float* c, float sm_scale, uint16_t* out, float* lse, void* ws,
+                                   size_t ws_bytes, tg_stream_t stream);
+
+/*
+ * Host only: the prunable span of the NEXT gate, in the kept order of this
+ * one.  All tokens before a span are kept, so sequence b's surviving span
+ * tokens sit at kept indices [p0_b, p0_b + min(k_b, |P_b|)) (k_b < 0 = all).
+ * h_span and h_span_next are [B, 2] int32 (may alias); h_k is [B].  With
+ * cu_kept as the next gate's cu_seqlens, tg_score / tg_select_topk /
+ * tg_compact run the next gate unchanged.  Returns TG_ERR_INVALID_ARG for a
+ * negative or reversed span.
+ */
+tg_status tg_next_gate_span(const int32_t* h_span, const int32_t* h_k, int B, int32_t* h_span_next);
+
 /* Bytes of scratch tg_gated_attention may use for these sizes on the
  * current device (0 when it does not split, or for unsupported sizes). */
 size_t tg_gated_attention_workspace_size(int B, int max_M, int Hq, int Hkv, int d);
@@ -300,14 +333,17 @@ tg_status tg_masked_gated_attention(const uint16_t* q, const uint16_t* k, const 
 
 /*
  * Row gather by the compaction map: dst[m, :] = src[kept_idx[m], :] for
- * m < M, rows of row_bytes bytes (a multiple of 16; src and dst 16-byte
- * aligned, device).  The serving path of the pages gathers the lower
+ * m < M, rows of row_bytes bytes (4, 8 or a multiple of 16; src and dst
+ * aligned to min(row_bytes, 16) bytes, device; anything else is
+ * TG_ERR_UNSUPPORTED or TG_ERR_INVALID_ARG before any launch).  The serving path of the pages gathers the lower
  * layers' KV cache to the kept tokens on a separate stream (AI summary,
  * "Methodology in Plain English"): with src the [T, Hkv, d] K or V cache of
  * a layer below L (row_bytes = 2 * Hkv * d for bf16) this is that gather.
  * Entries of kept_idx outside [0, T) leave their row unwritten.
  * tg_gated_prefill_layer runs the same gather for args->gather_* beside the
- * attention.
+ * attention.  With 4-byte rows it composes the maps of two gates: the
+ * original positions of the tokens the second gate keeps are
+ * pos1[kept_idx2], their first-gate logsigmoids gls1[kept_idx2].
  */
 tg_status tg_gather_rows(const void* src, int64_t T, int64_t row_bytes, const int32_t* kept_idx, int64_t M,
                          void* dst, tg_stream_t stream);

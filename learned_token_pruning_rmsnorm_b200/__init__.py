@@ -24,7 +24,7 @@ from ._lib import TokenGateError, load  # noqa: F401
 __all__ = [
     "TokenGateError", "load", "tg_abi_version", "tg_kept_count", "tg_gate_prepare", "tg_score",
     "tg_select_topk", "tg_compact", "tg_gather_kept", "tg_gather_rows", "tg_gated_attention",
-    "tg_masked_gated_attention",
+    "tg_gated_attention_gates", "tg_next_gate_span", "tg_masked_gated_attention",
     "tg_gated_prefill_layer",
     "tg_device_status", "tg_selftest_bounded_wait",
 ]
@@ -148,8 +148,9 @@ def tg_gather_kept(hidden, kept_idx, hidden_kept=None):
 
 def tg_gather_rows(src, kept_idx, dst=None):
     """dst[m] = src[kept_idx[m]] for any contiguous device tensor src of shape
-    [T, ...] whose rows are a multiple of 16 bytes (e.g. a layer's [T, Hkv, d]
-    K or V cache).  Returns dst ([M, ...], same dtype)."""
+    [T, ...] whose rows are 4 or 8 bytes or a multiple of 16 bytes (e.g. a
+    layer's [T, Hkv, d] K or V cache, or a [T] int32 position map).  Returns
+    dst ([M, ...], same dtype)."""
     if not src.is_cuda or not src.is_contiguous():
         raise ValueError("src must be a contiguous CUDA tensor")
     _dev(kept_idx, torch.int32, "kept_idx")
@@ -276,6 +277,61 @@ def tg_gated_attention(q, k, v, cu_kept, max_M: int, pos, rank, gls, g, c, sm_sc
                                          gls.data_ptr(), g.data_ptr(), c.data_ptr(), float(sm_scale),
                                          out.data_ptr(), _lib.ptr(lse), _lib.ptr(ws),
                                          0 if ws is None else ws.numel(), _lib.stream_handle(dev)))
+    return (out, lse) if want_lse or lse is not None else out
+
+
+def tg_next_gate_span(span, k):
+    """Host-side: the next gate's prunable span in this gate's kept order
+    ([B, 2] int32 numpy array)."""
+    sp = _lib.host_i32(span).reshape(-1)
+    kk = _lib.host_i32(k).reshape(-1)
+    B = len(kk)
+    if len(sp) != 2 * B:
+        raise ValueError("span must be [B, 2] for B budgets")
+    out = np.zeros(2 * B, dtype=np.int32)
+    _lib.check(load().tg_next_gate_span(sp.ctypes.data, kk.ctypes.data, B, out.ctypes.data))
+    return out.reshape(B, 2)
+
+
+def tg_gated_attention_gates(q, k, v, cu_kept, max_M: int, pos, rank, gls, g, c, sm_scale: float | None = None,
+                             out=None, lse=None, want_lse: bool = False, ws="auto"):
+    """tg_gated_attention with the bias summed over several gates: gls and g are
+    sequences of [M] and [Hq] fp32 device tensors, one per gate (1 to 4)."""
+    M, Hq, d = q.shape
+    Hkv = k.shape[1]
+    dev = q.device
+    _dev(q, torch.bfloat16, "q")
+    _dev(k, torch.bfloat16, "k", (M, Hkv, d))
+    _dev(v, torch.bfloat16, "v", (M, Hkv, d))
+    _dev(pos, torch.int32, "pos", (M,))
+    _dev(rank, torch.int32, "rank", (M,))
+    gls, g = list(gls), list(g)
+    if len(gls) != len(g):
+        raise ValueError("one gls and one g per gate")
+    for i, (a, b) in enumerate(zip(gls, g)):
+        _dev(a, torch.float32, f"gls[{i}]", (M,))
+        _dev(b, torch.float32, f"g[{i}]", (Hq,))
+    _dev(c, torch.float32, "c", (Hq,))
+    ck = _i32_dev(cu_kept, dev, "cu_kept")
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((M, Hq, d), dtype=torch.bfloat16, device=dev)
+    _dev(out, torch.bfloat16, "out", (M, Hq, d))
+    if lse is None and want_lse:
+        lse = torch.empty((M, Hq), dtype=torch.float32, device=dev)
+    if lse is not None:
+        _dev(lse, torch.float32, "lse", (M, Hq))
+    if isinstance(ws, str):
+        ws = attention_workspace(ck.numel() - 1, int(max_M), Hq, Hkv, d, dev)
+    n = len(gls)
+    gls_arr = (C.c_void_p * max(n, 1))(*[t.data_ptr() for t in gls])
+    g_arr = (C.c_void_p * max(n, 1))(*[t.data_ptr() for t in g])
+    _lib.check(load().tg_gated_attention_gates(q.data_ptr(), k.data_ptr(), v.data_ptr(), ck.data_ptr(),
+                                               ck.numel() - 1, M, int(max_M), Hq, Hkv, d, pos.data_ptr(),
+                                               rank.data_ptr(), n, gls_arr, g_arr, c.data_ptr(), float(sm_scale),
+                                               out.data_ptr(), _lib.ptr(lse), _lib.ptr(ws),
+                                               0 if ws is None else ws.numel(), _lib.stream_handle(dev)))
     return (out, lse) if want_lse or lse is not None else out
 
 

@@ -156,10 +156,9 @@ template <int HD>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gated_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const int32_t* __restrict__ cu_kept,
-                     const int32_t* __restrict__ pos, const int32_t* __restrict__ rank,
-                     const float* __restrict__ gls, const float* __restrict__ g, const float* __restrict__ c,
-                     float sm_scale, int Hq, int Hkv, int n_qt_max, uint16_t* __restrict__ out,
-                     float* __restrict__ lse, int* __restrict__ status) {
+                     const int32_t* __restrict__ pos, const int32_t* __restrict__ rank, const GateSet gates,
+                     const float* __restrict__ c, float sm_scale, int Hq, int Hkv, int n_qt_max,
+                     uint16_t* __restrict__ out, float* __restrict__ lse, int* __restrict__ status) {
     using L = AttnSmem<HD>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -307,19 +306,28 @@ gated_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         float inv_tau = 1.0f;
         if (valid_row) inv_tau = 1.0f / (1.0f + c[h] * logf(static_cast<float>(pos[qg]) / static_cast<float>(rank[qg])));
         const float alpha = sm_scale * LOG2E * inv_tau;
-        const float gscale = softplus_f(g[h]) * LOG2E;
+        float gscale[kMaxGates];  // per gate: softplus(g_h) in log2 units (0 past the last gate)
+#pragma unroll
+        for (int gi = 0; gi < kMaxGates; ++gi) gscale[gi] = gi < gates.n ? softplus_f(gates.g[gi][h]) * LOG2E : 0.f;
         const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
         float* wbias = sBias + warp * (2 * BN);  // this warp's copy, double-buffered
         for (int j = 0; j < n_kv; ++j) {
             const int s = j & 1;
-            // gate bias of the tile's 128 keys, log2 domain; each warp keeps its own
-            // copy so that only __syncwarp orders it
+            // gate bias of the tile's 128 keys (summed over the gates), log2 domain; each
+            // warp keeps its own copy so that only __syncwarp orders it
 #pragma unroll
             for (int e = 0; e < BN / 32; ++e) {
                 const int key_local = j * BN + e * 32 + lane;
-                wbias[s * BN + e * 32 + lane] = key_local < Mb ? gscale * gls[seq0 + key_local] : 0.f;
+                float bsum = 0.f;
+                if (key_local < Mb) {
+                    bsum = gscale[0] * gates.gls[0][seq0 + key_local];
+#pragma unroll
+                    for (int gi = 1; gi < kMaxGates; ++gi)
+                        if (gi < gates.n) bsum += gscale[gi] * gates.gls[gi][seq0 + key_local];
+                }
+                wbias[s * BN + e * 32 + lane] = bsum;
             }
             __syncwarp();
             ok = mbar_wait_warp(bar(B_S_FULL + s), (j >> 1) & 1, abort_flag, status, TG_WHERE_SOFTMAX);
@@ -503,13 +511,31 @@ struct SplitWs {
     int slots_per_pair;  // n_qt_max - C (query tiles that may be split)
 };
 
+// Q_ext columns 4..15 (gates 2..n) of both heads' rows, out of line so that the
+// one-gate kernel body stays as it is without them.  Called by every thread of the
+// CTA: the barrier orders these writes after the zeroing of cores 8..15.
+template <typename L>
+__device__ __noinline__ void g2_extra_gates_q(uint8_t* smem, int n, const float* g1, const float* g2,
+                                              const float* g3, int pair, float sm_scale) {
+    __syncthreads();
+    if (threadIdx.x < 2 * BM) {
+        const int hh = threadIdx.x / BM, r = threadIdx.x % BM;
+        uint8_t* row = smem + L::OFF_QX + hh * L::EXT + (r >> 3) * 256 + (r & 7) * 16;
+        for (int gi = 1; gi < n; ++gi) {
+            const float* gg = gi == 1 ? g1 : (gi == 2 ? g2 : g3);
+            const uint32_t hl = bf16_hi_lo(softplus_f(gg[2 * pair + hh]) / sm_scale);
+            *reinterpret_cast<uint2*>(row + (gi >> 1) * 128 + (gi & 1) * 8) = make_uint2(hl, hl);
+        }
+    }
+}
+
 template <int HD>
 __global__ void __launch_bounds__(G2_THREADS, 1)
 gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const int32_t* __restrict__ cu_kept,
-                       const int32_t* __restrict__ pos, const int32_t* __restrict__ rank,
-                       const float* __restrict__ gls, const float* __restrict__ g, const float* __restrict__ c,
-                       float sm_scale, int Hq, int Hkv, int n_qt_max, int kv_chunk, SplitWs ws,
+                       const int32_t* __restrict__ pos, const int32_t* __restrict__ rank, const GateSet gates,
+                       const float* __restrict__ c, float sm_scale, int Hq, int Hkv, int n_qt_max, int kv_chunk,
+                       SplitWs ws,
                        uint16_t* __restrict__ out, float* __restrict__ lse, int* __restrict__ status) {
     using L = G2Smem<HD>;
     extern __shared__ uint8_t smem_raw[];
@@ -568,12 +594,14 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
     const uint32_t sQX = sbase + L::OFF_QX, sKX = sbase + L::OFF_KX;
 
-    // Gate bias as one more k-step of the S = Q K^T product: row q of Q_ext holds
-    // (bh, bl, bh, bl) and row j of K_ext holds (gh, gh, gl, gl), the bf16 high and low
-    // parts of bscale_h = softplus(g_h) / sm_scale and of gls_j, so that the extra products
-    // add bscale_h * gls_j to S with about 2^-16 relative error; the other 12 columns are
-    // zero.  K cores 8..15 of all four tiles are zero throughout; K_ext rows are written by
-    // the producer per KV tile.
+    // Gate bias as one more k-step of the S = Q K^T product.  Gate i owns columns
+    // 4i .. 4i+3 of the step: row q of Q_ext holds (bh, bl, bh, bl) and row j of K_ext
+    // holds (gh, gh, gl, gl), the bf16 high and low parts of bscale_h = softplus(g_h) /
+    // sm_scale and of gls_j, so that the four products add bscale_h * gls_j to S with
+    // about 2^-16 relative error.  Columns of absent gates are zero: K cores 8..15 of all
+    // four tiles are zeroed here and columns 4..7 are written as zeros with the first
+    // gate's; further gates (rare) are filled in by out-of-line code, which keeps the
+    // one-gate kernel body unchanged.
     for (int i = threadIdx.x; i < 4 * (BM / 8) * 8; i += blockDim.x) {
         const int tile = i / ((BM / 8) * 8), rem = i % ((BM / 8) * 8);
         *reinterpret_cast<uint4*>(smem + L::OFF_QX + tile * L::EXT + (rem >> 3) * 256 + 128 + (rem & 7) * 16) =
@@ -581,11 +609,13 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     }
     if (threadIdx.x < 2 * BM) {
         const int hh = threadIdx.x / BM, r = threadIdx.x % BM;
-        const float bscale = softplus_f(g[2 * pair + hh]) / sm_scale;
+        const float bscale = softplus_f(gates.g[0][2 * pair + hh]) / sm_scale;
         const uint32_t hl = bf16_hi_lo(bscale);
         *reinterpret_cast<uint4*>(smem + L::OFF_QX + hh * L::EXT + (r >> 3) * 256 + (r & 7) * 16) =
             make_uint4(hl, hl, 0u, 0u);
     }
+    if (gates.n > 1)  // uniform: all threads
+        g2_extra_gates_q<L>(smem, gates.n, gates.g[1], gates.g[2], gates.g[3], pair, sm_scale);
     fence_proxy_async_smem();
 
     if (threadIdx.x == 0) {
@@ -630,11 +660,11 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                                 seq0 + qt * BM, bar(G_Q_FULL));
         }
         int k_issued[2] = {0, 0}, v_issued[2] = {0, 0};
-        float gk[4];  // gls of this lane's keys of the next tile (0 past the sequence end)
+        float gk[4];  // first gate's gls of this lane's keys of the next tile (0 past the end)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int key_local = kv0 * BN + lane * 4 + i;
-            gk[i] = key_local < Mb ? ldg_early(gls + seq0 + key_local) : 0.f;
+            gk[i] = key_local < Mb ? ldg_early(gates.gls[0] + seq0 + key_local) : 0.f;
         }
         for (int j = 0; j < n_kv; ++j) {
             const int s = j & 1;
@@ -645,7 +675,7 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int key_local = (kv0 + j + 1) * BN + lane * 4 + i;
-                    gk[i] = key_local < Mb ? ldg_early(gls + seq0 + key_local) : 0.f;
+                    gk[i] = key_local < Mb ? ldg_early(gates.gls[0] + seq0 + key_local) : 0.f;
                 }
             }
             if (j >= 2 && !mbar_wait_warp(bar(G_K_EMPTY + s), ((j - 2) >> 1) & 1, abort_flag, status,
@@ -657,6 +687,23 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 const uint32_t hl = bf16_hi_lo(gcur[i]);
                 *reinterpret_cast<uint4*>(smem + L::OFF_KX + s * L::EXT + (r >> 3) * 256 + (r & 7) * 16) =
                     make_uint4(__byte_perm(hl, 0u, 0x1010), __byte_perm(hl, 0u, 0x3232), 0u, 0u);
+            }
+            // further gates (rare): the same lane rewrites its rows' slots of those gates
+#pragma unroll 1
+            for (int gi = 1; gi < gates.n; ++gi) {
+                // (a select chain, not gates.gls[gi]: a run-time index into the parameter
+                // block would copy it to local memory)
+                const float* gsrc = (gi == 1 ? gates.gls[1] : (gi == 2 ? gates.gls[2] : gates.gls[3])) + seq0 +
+                                    (kv0 + j) * BN;
+                const int valid = Mb - (kv0 + j) * BN;
+                uint8_t* kx = smem + L::OFF_KX + s * L::EXT;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int r = lane * 4 + i;
+                    const uint32_t hl = bf16_hi_lo(r < valid ? gsrc[r] : 0.f);
+                    *reinterpret_cast<uint2*>(kx + (r >> 3) * 256 + (gi >> 1) * 128 + (r & 7) * 16 + (gi & 1) * 8) =
+                        make_uint2(__byte_perm(hl, 0u, 0x1010), __byte_perm(hl, 0u, 0x3232));
+                }
             }
             fence_proxy_async_smem();  // K_ext is read by the tensor core (async proxy)
             __syncwarp();
@@ -1095,8 +1142,8 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
 
 template <int HD>
 cudaError_t launch_gqa2(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const int32_t* cu_kept,
-                        int B, int max_M, int Hq, int Hkv, const int32_t* pos, const int32_t* rank, const float* gls,
-                        const float* g, const float* c, float sm_scale, uint16_t* out, float* lse, void* ws,
+                        int B, int max_M, int Hq, int Hkv, const int32_t* pos, const int32_t* rank,
+                        const GateSet& gates, const float* c, float sm_scale, uint16_t* out, float* lse, void* ws,
                         size_t ws_bytes, cudaStream_t st) {
     using L = G2Smem<HD>;
     static std::atomic<uint64_t> attr_set{0};
@@ -1121,15 +1168,15 @@ cudaError_t launch_gqa2(const CUtensorMap& tq, const CUtensorMap& tk, const CUte
     const int64_t units = units_below_host(n_qt_max, C);
     dim3 grid(Hq / 2, static_cast<unsigned>(units), B);
     return launch_pdl(gated_attn_gqa2_kernel<HD>, grid, dim3(G2_THREADS), static_cast<size_t>(L::ALLOC), st, tq, tk,
-                      tv, cu_kept, pos, rank, gls, g, c, sm_scale, Hq, Hkv, n_qt_max, C, sw, out, lse,
+                      tv, cu_kept, pos, rank, gates, c, sm_scale, Hq, Hkv, n_qt_max, C, sw, out, lse,
                       device_status_ptr());
 }
 
 template <int HD>
 cudaError_t launch_tc(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* cu_kept, int B,
                       int64_t M_total, int max_M, int Hq, int Hkv, const int32_t* pos, const int32_t* rank,
-                      const float* gls, const float* g, const float* c, float sm_scale, uint16_t* out, float* lse,
-                      void* ws, size_t ws_bytes, cudaStream_t st) {
+                      const GateSet& gates, const float* c, float sm_scale, uint16_t* out, float* lse, void* ws,
+                      size_t ws_bytes, cudaStream_t st) {
     using L = AttnSmem<HD>;
     static std::atomic<uint64_t> attr_set{0};
     if (cudaError_t e = ensure_smem_limit(gated_attn_tc_kernel<HD>, L::ALLOC, attr_set); e != cudaSuccess)
@@ -1143,13 +1190,13 @@ cudaError_t launch_tc(const uint16_t* q, const uint16_t* k, const uint16_t* v, c
                              static_cast<uint64_t>(Hkv) * HD * 2, 64, BN))
         return cudaErrorInvalidValue;
     if ((Hq / Hkv) % 2 == 0)
-        return launch_gqa2<HD>(tq, tk, tv, cu_kept, B, max_M, Hq, Hkv, pos, rank, gls, g, c, sm_scale, out, lse, ws,
+        return launch_gqa2<HD>(tq, tk, tv, cu_kept, B, max_M, Hq, Hkv, pos, rank, gates, c, sm_scale, out, lse, ws,
                                ws_bytes, st);
     int* status = device_status_ptr();
     const int n_qt_max = (max_M + BM - 1) / BM;
     dim3 grid(Hq, n_qt_max, B);
     return launch_pdl(gated_attn_tc_kernel<HD>, grid, dim3(NUM_THREADS), static_cast<size_t>(L::ALLOC), st, tq, tk, tv,
-                      cu_kept, pos, rank, gls, g, c, sm_scale, Hq, Hkv, n_qt_max, out, lse, status);
+                      cu_kept, pos, rank, gates, c, sm_scale, Hq, Hkv, n_qt_max, out, lse, status);
 }
 
 }  // namespace
@@ -1165,14 +1212,14 @@ extern "C" int tg_trace_read_attention_ctas(unsigned long long* host) {
 
 cudaError_t launch_gated_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* cu_kept,
                                    int B, int64_t M_total, int max_M, int Hq, int Hkv, int d, const int32_t* pos,
-                                   const int32_t* rank, const float* gls, const float* g, const float* c,
-                                   float sm_scale, uint16_t* out, float* lse, void* ws, size_t ws_bytes,
-                                   cudaStream_t st) {
+                                   const int32_t* rank, const GateSet& gates, const float* c, float sm_scale,
+                                   uint16_t* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t st) {
     if (M_total == 0 || B == 0) return cudaSuccess;
+    if (gates.n < 1 || gates.n > kMaxGates) return cudaErrorInvalidValue;
     if (d == 64)
-        return launch_tc<64>(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, pos, rank, gls, g, c, sm_scale, out, lse,
+        return launch_tc<64>(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, pos, rank, gates, c, sm_scale, out, lse,
                              ws, ws_bytes, st);
-    return launch_tc<128>(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, pos, rank, gls, g, c, sm_scale, out, lse, ws,
+    return launch_tc<128>(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, pos, rank, gates, c, sm_scale, out, lse, ws,
                           ws_bytes, st);
 }
 
@@ -1248,8 +1295,8 @@ cudaError_t noalloc_attention_scratch(void** ptr) {
 
 cudaError_t launch_gated_attention_noalloc(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                            const int32_t* cu_kept, int B, int64_t M_total, int max_M, int Hq, int Hkv,
-                                           int d, const int32_t* pos, const int32_t* rank, const float* gls,
-                                           const float* g, const float* c, float sm_scale, uint16_t* out, float* lse,
+                                           int d, const int32_t* pos, const int32_t* rank, const GateSet& gates,
+                                           const float* c, float sm_scale, uint16_t* out, float* lse,
                                            cudaStream_t st) {
     const size_t need = attention_workspace_bytes(B, max_M, Hq, Hkv, d);
     if (need > TG_NOALLOC_ATTENTION_SCRATCH_BYTES) return cudaErrorInvalidValue;  // the API rejects it first
@@ -1265,7 +1312,7 @@ cudaError_t launch_gated_attention_noalloc(const uint16_t* q, const uint16_t* k,
         e = cudaMemsetAsync(static_cast<uint8_t*>(ws) + (need - cnt_bytes), 0, cnt_bytes, st);
         if (e != cudaSuccess) return e;
     }
-    return launch_gated_attention(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, d, pos, rank, gls, g, c, sm_scale,
+    return launch_gated_attention(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, d, pos, rank, gates, c, sm_scale,
                                   out, lse, need > 0 ? ws : nullptr, need, st);
 }
 

@@ -451,6 +451,21 @@ gather_rows_kernel(const uint4* __restrict__ hidden, const int32_t* __restrict__
     }
 }
 
+// Gather of narrow rows (one 4- or 8-byte word each, e.g. a position or a gate's
+// logsigmoid per kept row): dst[m] = src[kept_idx[m]], one thread per row.
+template <typename W>
+__global__ void __launch_bounds__(256)
+gather_words_kernel(const W* __restrict__ src, const int32_t* __restrict__ kept_idx, int64_t M, int64_t T,
+                    W* __restrict__ out) {
+    pdl_wait();  // global memory is read only from here on
+    pdl_trigger();
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t m = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; m < M; m += stride) {
+        const int64_t i = kept_idx[m];
+        if (i >= 0 && i < T) out[m] = src[i];
+    }
+}
+
 // Row scatter out[idx[m], :] = in[m, :] (the inverse of the gather), one warp per
 // row; indices outside [0, T) write nothing.
 template <int VPL>
@@ -506,12 +521,22 @@ cudaError_t launch_select_scan(int mode, const float* scores, const uint8_t* kee
 cudaError_t launch_gather_bytes(const void* src, const int32_t* kept_idx, int64_t M_total, int64_t T,
                                 int64_t row_bytes, void* dst, cudaStream_t st) {
     if (M_total == 0) return cudaSuccess;
-    const int64_t vpr64 = row_bytes / 16;
-    if (vpr64 <= 0 || vpr64 * 16 != row_bytes || vpr64 > (int64_t(1) << 30)) return cudaErrorInvalidValue;
-    const int vpr = static_cast<int>(vpr64);
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (row_bytes == 4 || row_bytes == 8) {
+        const int64_t need = (M_total + 255) / 256;
+        const int grid = static_cast<int>(need < static_cast<int64_t>(sms) * 8 ? need : sms * 8);
+        if (row_bytes == 4)
+            return launch_pdl(gather_words_kernel<uint32_t>, dim3(grid), dim3(256), 0, st,
+                              static_cast<const uint32_t*>(src), kept_idx, M_total, T, static_cast<uint32_t*>(dst));
+        return launch_pdl(gather_words_kernel<unsigned long long>, dim3(grid), dim3(256), 0, st,
+                          static_cast<const unsigned long long*>(src), kept_idx, M_total, T,
+                          static_cast<unsigned long long*>(dst));
+    }
+    const int64_t vpr64 = row_bytes / 16;
+    if (vpr64 <= 0 || vpr64 * 16 != row_bytes || vpr64 > (int64_t(1) << 30)) return cudaErrorInvalidValue;
+    const int vpr = static_cast<int>(vpr64);
     const int64_t blocks_needed = (M_total + 7) / 8;
     const int grid = static_cast<int>(blocks_needed < static_cast<int64_t>(sms) * 8 ? blocks_needed : sms * 8);
     const uint4* h = static_cast<const uint4*>(src);

@@ -109,14 +109,16 @@ tg_status do_score(const uint16_t* hidden, const int32_t* cu_seqlens, const int3
 
 tg_status do_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* cu_kept, int B,
                        int64_t M_total, int max_M, int Hq, int Hkv, int d, const int32_t* pos, const int32_t* rank,
-                       const float* gls, const float* g, const float* c, float sm_scale, uint16_t* out, float* lse,
+                       const tg::GateSet& gates, const float* c, float sm_scale, uint16_t* out, float* lse,
                        void* ws, size_t ws_bytes, cudaStream_t st) {
     TG_REQUIRE(B >= 0 && M_total >= 0 && max_M >= 0, "negative size");
     if (tg_status s = check_attn_shape(Hq, Hkv, d)) return s;
     TG_REQUIRE(sm_scale > 0.f, "sm_scale must be positive");
+    TG_SUPPORT(gates.n >= 1 && gates.n <= tg::kMaxGates, "n_gates=%d must be in [1, %d]", gates.n, tg::kMaxGates);
     if (B == 0 || M_total == 0) return TG_OK;
     TG_REQUIRE(max_M > 0, "max_M must bound the longest sequence");
-    TG_REQUIRE(q && k && v && cu_kept && pos && rank && gls && g && c && out, "null pointer argument");
+    for (int i = 0; i < gates.n; ++i) TG_REQUIRE(gates.gls[i] && gates.g[i], "null gls or g of gate %d", i);
+    TG_REQUIRE(q && k && v && cu_kept && pos && rank && c && out, "null pointer argument");
     TG_REQUIRE(aligned16(q) && aligned16(k) && aligned16(v) && aligned16(out),
                "q, k, v and out must be 16-byte aligned");
     if (ws) {
@@ -125,7 +127,7 @@ tg_status do_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
         TG_REQUIRE(ws_bytes >= need, "ws holds %zu bytes, the causal split needs %zu", ws_bytes, need);
     }
     if (tg_status s = check_device()) return s;
-    return cuda_status(tg::launch_gated_attention(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, d, pos, rank, gls, g,
+    return cuda_status(tg::launch_gated_attention(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, d, pos, rank, gates,
                                                   c, sm_scale, out, lse, ws, ws_bytes, st),
                        "tg_gated_attention launch");
 }
@@ -209,14 +211,15 @@ tg_status tg_masked_gated_attention(const uint16_t* q, const uint16_t* k, const 
     if (tg_status s = cuda_status(tg::launch_gather_bytes(q, idx, M_total, T, qrow, qc, st), "q gather")) return s;
     if (tg_status s = cuda_status(tg::launch_gather_bytes(k, idx, M_total, T, kvrow, kc, st), "k gather")) return s;
     if (tg_status s = cuda_status(tg::launch_gather_bytes(v, idx, M_total, T, kvrow, vc, st), "v gather")) return s;
-    if (tg_status s = do_attention(qc, kc, vc, cu_kept, B, M_total, max_M, Hq, Hkv, d, pos, rank, gls, g, c, sm_scale,
-                                   oc, nullptr, L.attn_bytes ? base + L.attn : nullptr, L.attn_bytes, st))
+    if (tg_status s = do_attention(qc, kc, vc, cu_kept, B, M_total, max_M, Hq, Hkv, d, pos, rank,
+                                   tg::single_gate(gls, g), c, sm_scale, oc, nullptr,
+                                   L.attn_bytes ? base + L.attn : nullptr, L.attn_bytes, st))
         return s;
     return cuda_status(tg::launch_scatter_bytes(oc, idx, M_total, T, qrow, out, st), "out scatter");
 }
 
 
-int tg_abi_version(void) { return 2; }
+int tg_abi_version(void) { return 3; }
 
 const char* tg_last_error_string(void) { return g_last_error.c_str(); }
 
@@ -305,8 +308,11 @@ tg_status tg_gather_rows(const void* src, int64_t T, int64_t row_bytes, const in
     TG_REQUIRE(T >= 0 && M >= 0 && row_bytes >= 0, "negative size");
     if (M == 0 || row_bytes == 0) return TG_OK;
     TG_REQUIRE(src && kept_idx && dst, "null pointer argument");
-    TG_SUPPORT(row_bytes % 16 == 0, "row_bytes=%lld must be a multiple of 16", (long long)row_bytes);
-    TG_REQUIRE(aligned16(src) && aligned16(dst), "src and dst must be 16-byte aligned");
+    TG_SUPPORT(row_bytes == 4 || row_bytes == 8 || row_bytes % 16 == 0,
+               "row_bytes=%lld must be 4, 8 or a multiple of 16", (long long)row_bytes);
+    const uintptr_t amask = static_cast<uintptr_t>(row_bytes < 16 ? row_bytes : 16) - 1;
+    TG_REQUIRE(((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & amask) == 0,
+               "src and dst must be aligned to %d bytes", static_cast<int>(amask + 1));
     if (tg_status s = check_device()) return s;
     return cuda_status(tg::launch_gather_bytes(src, kept_idx, M, T, row_bytes, dst, stream), "tg_gather_rows launch");
 }
@@ -324,13 +330,14 @@ tg_status tg_gated_attention_noalloc(const uint16_t* q, const uint16_t* k, const
     TG_REQUIRE(aligned16(q) && aligned16(k) && aligned16(v) && aligned16(out),
                "q, k, v and out must be 16-byte aligned");
     if (tg_status s = check_device()) return s;
+    const tg::GateSet gates = tg::single_gate(gls, g);
     const size_t need = tg::attention_workspace_bytes(B, max_M, Hq, Hkv, d);
     TG_SUPPORT(need <= TG_NOALLOC_ATTENTION_SCRATCH_BYTES,
                "tg_gated_attention_noalloc: these sizes need %zu bytes of scratch, above the fixed %zu-byte array; "
                "use tg_gated_attention with a caller workspace",
                need, static_cast<size_t>(TG_NOALLOC_ATTENTION_SCRATCH_BYTES));
     return cuda_status(tg::launch_gated_attention_noalloc(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, d, pos, rank,
-                                                          gls, g, c, sm_scale, out, lse, stream),
+                                                          gates, c, sm_scale, out, lse, stream),
                        "tg_gated_attention_noalloc launch");
 }
 
@@ -343,8 +350,42 @@ tg_status tg_gated_attention(const uint16_t* q, const uint16_t* k, const uint16_
                              int64_t M_total, int max_M, int Hq, int Hkv, int d, const int32_t* pos,
                              const int32_t* rank, const float* gls, const float* g, const float* c, float sm_scale,
                              uint16_t* out, float* lse, void* ws, size_t ws_bytes, tg_stream_t stream) {
-    return do_attention(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, d, pos, rank, gls, g, c, sm_scale, out, lse, ws,
+    return do_attention(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, d, pos, rank, tg::single_gate(gls, g), c,
+                        sm_scale, out, lse, ws, ws_bytes, stream);
+}
+
+tg_status tg_gated_attention_gates(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* cu_kept,
+                                   int B, int64_t M_total, int max_M, int Hq, int Hkv, int d, const int32_t* pos,
+                                   const int32_t* rank, int n_gates, const float* const* gls, const float* const* g,
+                                   const float* c, float sm_scale, uint16_t* out, float* lse, void* ws,
+                                   size_t ws_bytes, tg_stream_t stream) {
+    TG_SUPPORT(n_gates >= 1 && n_gates <= tg::kMaxGates, "n_gates=%d must be in [1, %d]", n_gates, tg::kMaxGates);
+    TG_REQUIRE(gls && g, "null gate arrays");
+    tg::GateSet gates{};
+    gates.n = n_gates;
+    for (int i = 0; i < n_gates; ++i) {
+        gates.gls[i] = gls[i];
+        gates.g[i] = g[i];
+    }
+    return do_attention(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, d, pos, rank, gates, c, sm_scale, out, lse, ws,
                         ws_bytes, stream);
+}
+
+tg_status tg_next_gate_span(const int32_t* h_span, const int32_t* h_k, int B, int32_t* h_span_next) {
+    TG_REQUIRE(B >= 0, "negative B");
+    if (B == 0) return TG_OK;
+    TG_REQUIRE(h_span && h_k && h_span_next, "null pointer argument");
+    for (int b = 0; b < B; ++b) {
+        const int64_t p0 = h_span[2 * b], p1 = h_span[2 * b + 1];
+        TG_REQUIRE(p0 >= 0 && p1 >= p0, "sequence %d: span [%lld, %lld)", b, (long long)p0, (long long)p1);
+        const int64_t P = p1 - p0;
+        const int64_t kk = (h_k[b] < 0 || h_k[b] > P) ? P : h_k[b];
+        // every token before the span is kept, so the kept part of the span starts at p0
+        // in kept order and holds the kk survivors
+        h_span_next[2 * b] = static_cast<int32_t>(p0);
+        h_span_next[2 * b + 1] = static_cast<int32_t>(p0 + kk);
+    }
+    return TG_OK;
 }
 
 tg_status tg_device_status(int32_t* h_word, int clear, tg_stream_t stream) {
@@ -431,8 +472,8 @@ tg_status tg_gated_prefill_layer(const tg_prefill_layer_args* a, tg_stream_t str
     for (int l = 0; l < a->n_layers && result == TG_OK; ++l) {
         float* lse = a->lse ? a->lse[l] : nullptr;
         result = do_attention(a->q[l], a->kk[l], a->v[l], a->cu_kept, a->B, a->M_total, a->max_M, a->Hq, a->Hkv,
-                              a->d, a->pos, a->rank, a->gls, a->g[l], a->c[l], a->sm_scale, a->out[l], lse,
-                              a->attn_ws, a->attn_ws_bytes, st);
+                              a->d, a->pos, a->rank, tg::single_gate(a->gls, a->g[l]), a->c[l], a->sm_scale,
+                              a->out[l], lse, a->attn_ws, a->attn_ws_bytes, st);
     }
     if (fork) {
         // join: work queued on `stream` after this call also waits for the gather

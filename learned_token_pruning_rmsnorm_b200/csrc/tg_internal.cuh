@@ -93,8 +93,9 @@ cudaError_t launch_select_scan(int mode, const float* scores, const uint8_t* kee
                                uint8_t* keep_out, int32_t* kept_idx, int32_t* pos, int32_t* rank, float* gls,
                                cudaStream_t st);
 
-// dst[m, :] = src[kept_idx[m], :] for rows of row_bytes bytes (a multiple of 16; both
-// pointers 16-byte aligned); rows whose index lies outside [0, T) are left untouched
+// dst[m, :] = src[kept_idx[m], :] for rows of row_bytes bytes (4, 8 or a multiple of 16;
+// both pointers aligned to min(row_bytes, 16)); rows whose index lies outside [0, T) are
+// left untouched
 cudaError_t launch_gather_bytes(const void* src, const int32_t* kept_idx, int64_t M_total, int64_t T,
                                 int64_t row_bytes, void* dst, cudaStream_t st);
 // dst[idx[m], :] = src[m, :] (rows of row_bytes bytes, as for launch_gather_bytes)
@@ -103,19 +104,35 @@ cudaError_t launch_scatter_bytes(const void* src, const int32_t* idx, int64_t M,
 cudaError_t launch_gather_rows(const uint16_t* hidden, const int32_t* kept_idx, int64_t M_total, int64_t T, int D,
                                uint16_t* hidden_kept, cudaStream_t st);
 
+// The gate modules whose biases add up on the attention logits: gate i
+// contributes softplus(g[i][h]) * gls[i][j] (one gate is n = 1).  gls[i] is
+// indexed by kept row, g[i] by query head.
+constexpr int kMaxGates = 4;
+struct GateSet {
+    const float* gls[kMaxGates];
+    const float* g[kMaxGates];
+    int n;
+};
+inline GateSet single_gate(const float* gls, const float* g) {
+    GateSet s{};
+    s.gls[0] = gls;
+    s.g[0] = g;
+    s.n = 1;
+    return s;
+}
+
 cudaError_t launch_gated_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* cu_kept,
                                    int B, int64_t M_total, int max_M, int Hq, int Hkv, int d, const int32_t* pos,
-                                   const int32_t* rank, const float* gls, const float* g, const float* c,
-                                   float sm_scale, uint16_t* out, float* lse, void* ws, size_t ws_bytes,
-                                   cudaStream_t st);
+                                   const int32_t* rank, const GateSet& gates, const float* c, float sm_scale,
+                                   uint16_t* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t st);
 
 // Causal work split of the attention: KV chunk length chosen for a launch,
 // scratch bytes the split needs (0 when it never splits), unit count.
 int attention_kv_chunk(int B, int max_M, int Hq, int Hkv, bool have_ws);
 cudaError_t launch_gated_attention_noalloc(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                            const int32_t* cu_kept, int B, int64_t M_total, int max_M, int Hq, int Hkv,
-                                           int d, const int32_t* pos, const int32_t* rank, const float* gls,
-                                           const float* g, const float* c, float sm_scale, uint16_t* out, float* lse,
+                                           int d, const int32_t* pos, const int32_t* rank, const GateSet& gates,
+                                           const float* c, float sm_scale, uint16_t* out, float* lse,
                                            cudaStream_t st);
 size_t attention_workspace_bytes(int B, int max_M, int Hq, int Hkv, int d);
 int64_t units_below_host(int x, int C);

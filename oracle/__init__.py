@@ -52,9 +52,11 @@ def _load():
             lib.oracle_select_topk.argtypes = [P, P, P, P, i32, P]
             lib.oracle_compact.argtypes = [P, P, P, P, P, i32, i32, P, P, P, P, P, P]
             lib.oracle_gated_attention.argtypes = [P, P, P, P, i32, i32, i32, i32, P, P, P, P, P, f64,
-                                                   P, i64, P, P, i32]
+                                                   P, i64, P, P, i32, i32]
             lib.oracle_masked_gated_attention.argtypes = [P, P, P, P, P, i32, i32, i32, i32, P, P, P, P,
                                                           f64, P, i64, P]
+            if lib.oracle_abi_version() != 2:
+                raise ImportError("oracle/liboracle.so is stale: rebuild it")
             _lib = lib
     return _lib
 
@@ -160,7 +162,10 @@ def compact(hidden_bits, scores_f32, keep, cu_seqlens, span, with_hidden: bool =
 
 def gated_attention(q_bits, k_bits, v_bits, cu_kept, pos, rank, gls_f32, g, c, sm_scale=None,
                     rows=None, tau_on_qk_only: bool = False, want_lse: bool = True):
-    """Token-gated attention.  Returns (out [R, Hq, d] f64, lse [R, Hq] f64 or None)."""
+    """Token-gated attention.  Returns (out [R, Hq, d] f64, lse [R, Hq] f64 or None).
+
+    One gate: gls_f32 [M], g [Hq].  Several gates: gls_f32 [G, M] and g [G, Hq];
+    each gate adds its own bias term to the logits."""
     q, qp = _c(q_bits, np.uint16)
     k, kp = _c(k_bits, np.uint16)
     v, vp_ = _c(v_bits, np.uint16)
@@ -169,8 +174,11 @@ def gated_attention(q_bits, k_bits, v_bits, cu_kept, pos, rank, gls_f32, g, c, s
     cu, cup = _c(cu_kept, np.int32)
     po, pop = _c(pos, np.int32)
     ra, rap = _c(rank, np.int32)
-    gl, glp = _c(gls_f32, np.float32)
-    ga, gap = _c(g, np.float32)
+    gl, glp = _c(np.asarray(gls_f32, dtype=np.float32).reshape(-1, M), np.float32)
+    ga, gap = _c(np.asarray(g, dtype=np.float32).reshape(-1, Hq), np.float32)
+    n_gates = gl.shape[0]
+    if ga.shape[0] != n_gates:
+        raise ValueError("one row of g per gate")
     ca, cap = _c(c, np.float32)
     if sm_scale is None:
         sm_scale = 1.0 / np.sqrt(d)
@@ -184,8 +192,41 @@ def gated_attention(q_bits, k_bits, v_bits, cu_kept, pos, rank, gls_f32, g, c, s
     _load().oracle_gated_attention(qp, kp, vp_, cup, len(cu) - 1, Hq, Hkv, d, pop, rap, glp, gap, cap,
                                    float(sm_scale), rwp, R, out.ctypes.data_as(C.c_void_p),
                                    None if lse is None else lse.ctypes.data_as(C.c_void_p),
-                                   1 if tau_on_qk_only else 0)
+                                   1 if tau_on_qk_only else 0, n_gates)
     return out, lse
+
+
+def next_gate_span(first: dict, cu_seqlens, span) -> np.ndarray:
+    """Prunable span of a second gate, in the first gate's kept order: the kept
+    rows of sequence b that came from its span, found by counting the kept rows
+    whose source lies before the span start and before its end."""
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    sp = np.asarray(span, dtype=np.int64).reshape(-1, 2)
+    cuk = first["cu_kept"].astype(np.int64)
+    src = first["src"].astype(np.int64)
+    out = np.zeros_like(sp)
+    for b in range(len(cu) - 1):
+        rows = src[cuk[b]:cuk[b + 1]] - cu[b]  # positions (0-indexed) of b's kept tokens
+        out[b, 0] = int(np.sum(rows < sp[b, 0]))
+        out[b, 1] = int(np.sum(rows < sp[b, 1]))
+    return out.astype(np.int32)
+
+
+def compose_gates(first: dict, second: dict, first_gls=None) -> dict:
+    """The map of two stacked gates.  `second` is the compaction a second gate
+    made over the rows `first` kept (its `src` indexes those rows).  Positions
+    stay the original ones, ranks are the second gate's, and every gate's
+    logsigmoid follows the surviving rows: gls is [G, M2], the first gate's
+    rows (or `first_gls` [G1, M1] for deeper stacks) then the second gate's."""
+    s2 = second["src"].astype(np.int64)
+    prev = np.asarray(first["gls"] if first_gls is None else first_gls, dtype=np.float64).reshape(-1, len(first["pos"]))
+    return {
+        "cu_kept": second["cu_kept"],
+        "pos": first["pos"][s2].astype(np.int32),
+        "rank": second["rank"].astype(np.int32),
+        "gls": np.concatenate([prev[:, s2], np.asarray(second["gls"], dtype=np.float64)[None, :]], axis=0),
+        "src": first["src"][s2].astype(np.int32),
+    }
 
 
 def masked_gated_attention(q_bits, k_bits, v_bits, cu_seqlens, span, keep, scores_f32, g, c,

@@ -81,7 +81,7 @@ int64_t kept_prunable(int64_t p, int32_t k) { return (k < 0 || k > p) ? p : stat
 
 extern "C" {
 
-int oracle_abi_version() { return 1; }
+int oracle_abi_version() { return 2; }
 
 // Thread count of the parallel loops (one row per iteration; no reduction
 // crosses threads, so results do not depend on it).
@@ -256,10 +256,16 @@ void oracle_compact(const uint16_t* hidden, const float* scores, const uint8_t* 
 // `rows` (n_rows entries) selects which kept rows to compute; rows == nullptr
 // computes all M rows.  out is [n_rows, Hq, d]; lse (natural log of the
 // softmax denominator, max included) is [n_rows, Hq], may be null.
+// Several gate modules (AI summary, "Future Directions": each gate selects
+// from what the lower ones kept and contributes to the token-gated attention
+// above it): gls is [n_gates, M] and g is [n_gates, Hq], and each gate adds
+// its own term softplus(g_i,h) * gls_i,j to the logit.  n_gates = 1 is the
+// single gate of the method.
 void oracle_gated_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* cu_kept,
                             int B, int Hq, int Hkv, int d, const int32_t* pos, const int32_t* rank,
                             const float* gls, const float* g, const float* c, double sm_scale,
-                            const int64_t* rows, int64_t n_rows, double* out, double* lse, int tau_on_qk_only) {
+                            const int64_t* rows, int64_t n_rows, double* out, double* lse, int tau_on_qk_only,
+                            int n_gates) {
     const int64_t M = cu_kept[B];
     if (!rows) n_rows = M;
     const int group = Hq / Hkv;
@@ -273,7 +279,6 @@ void oracle_gated_attention(const uint16_t* q, const uint16_t* k, const uint16_t
         std::vector<double> acc(d);
         for (int h = 0; h < Hq; ++h) {
             const int hk = h / group;
-            const double gain = softplus(static_cast<double>(g[h]));
             const double tau = 1.0 + static_cast<double>(c[h]) *
                                          std::log(static_cast<double>(pos[i]) / static_cast<double>(rank[i]));
             double mx = -INFINITY;
@@ -281,7 +286,9 @@ void oracle_gated_attention(const uint16_t* q, const uint16_t* k, const uint16_t
                 double dot = 0.0;
                 for (int e = 0; e < d; ++e)
                     dot += bf16_to_double(q[(i * Hq + h) * d + e]) * bf16_to_double(k[(j * Hkv + hk) * d + e]);
-                const double bias = gain * static_cast<double>(gls[j]);
+                double bias = 0.0;
+                for (int gi = 0; gi < n_gates; ++gi)
+                    bias += softplus(static_cast<double>(g[gi * Hq + h])) * static_cast<double>(gls[gi * M + j]);
                 const double l = tau_on_qk_only ? (dot * sm_scale / tau + bias) : ((dot * sm_scale + bias) / tau);
                 logit[static_cast<size_t>(j - j0)] = l;
                 mx = std::max(mx, l);
