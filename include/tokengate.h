@@ -45,7 +45,7 @@
  *     error.  No exception crosses the ABI.  tg_last_error_string() describes
  *     the last failure of the calling thread.
  *   - Supported shapes: D a multiple of 64 (<= 8192); I a multiple of 16 in
- *     [16, 256]; head_dim 64 or 128; Hq a multiple of Hkv; sm_100 devices.
+ *     [16, 256]; head_dim 64, 128 or 256; Hq a multiple of Hkv; sm_100 devices.
  */
 #ifndef TOKENGATE_H
 #define TOKENGATE_H

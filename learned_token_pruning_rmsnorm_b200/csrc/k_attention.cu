@@ -12,13 +12,17 @@
 //              through a two-stage ring (128-byte swizzled boxes of 64 cols)
 //   warp 5     MMA issuer (one thread): S_j = Q K_j^T into one of two TMEM
 //              S buffers, then O += P_{j-1} V_{j-1} into the TMEM O accumulator
+//              with P read from TMEM
 //   warps 0-3  softmax: thread r owns query row r (TMEM lane r).  It reads
 //              S_j from TMEM, applies scale, gate bias and temperature in the
 //              log2 domain with one FFMA per element, masks the causal
 //              diagonal, keeps a running max that is only moved (and O only
 //              rescaled in TMEM) when it grows by more than 2^8, writes P_j
-//              as bf16 into a swizzled shared-memory tile for the next MMA,
-//              and at the end normalises O and stores it.
+//              as bf16 pairs over the first 64 columns of its S buffer, and
+//              at the end normalises O and stores it.
+// This kernel serves odd GQA groups and head_dim 256 (two heads of 256 would
+// need 768 TMEM columns); tcgen05 operations of one thread execute in issue
+// order, so S_{j+2} overwrites P_j only after PV_j has read it.
 // The bias and temperature therefore cost one extra FFMA per score element
 // on top of plain attention.
 
@@ -39,20 +43,24 @@ constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: rescale only when the 
 
 template <int HD>
 struct AttnSmem {
+    // K and V tiles are double-buffered up to head_dim 128; at 256 one 64 KB tile of
+    // each fits beside Q (the K tile of j+1 still loads during the softmax of j, and
+    // the V tile of j+1 during S(j+1)).
+    static constexpr int KV_STAGES = HD == 256 ? 1 : 2;
     static constexpr int TILE_Q = BM * HD * 2;
     static constexpr int TILE_KV = BN * HD * 2;
-    static constexpr int TILE_P = BM * BN * 2;
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + TILE_Q;
-    static constexpr int OFF_V = OFF_K + 2 * TILE_KV;
-    static constexpr int OFF_P = OFF_V + 2 * TILE_KV;
-    static constexpr int OFF_BIAS = OFF_P + TILE_P;
+    static constexpr int OFF_V = OFF_K + KV_STAGES * TILE_KV;
+    static constexpr int OFF_BIAS = OFF_V + KV_STAGES * TILE_KV;
     static constexpr int OFF_BAR = OFF_BIAS + 4 * 2 * BN * 4;  // a private bias copy per softmax warp
     static constexpr int NUM_BARS = 16;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int BYTES = OFF_MISC + 16;
     static constexpr int ALLOC = BYTES + 1024;  // slack for 1024-byte alignment
-    static constexpr uint32_t TMEM_COLS = 512;  // S0 | S1 | O
+    static constexpr uint32_t TMEM_COLS = 512;  // S0 | S1 | O (P_j as bf16 over S_(j&1))
+    static_assert(ALLOC <= 227 * 1024, "shared memory");
+    static_assert(2 * BN + HD <= 512, "TMEM columns");
 };
 
 // barrier indices
@@ -176,7 +184,8 @@ gated_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t sQ = sbase + L::OFF_Q, sK0 = sbase + L::OFF_K, sV0 = sbase + L::OFF_V, sP = sbase + L::OFF_P;
+    const uint32_t sQ = sbase + L::OFF_Q, sK0 = sbase + L::OFF_K, sV0 = sbase + L::OFF_V;
+    constexpr int NS = L::KV_STAGES;
     auto bar = [&](int i) { return sbase + L::OFF_BAR + 8u * static_cast<uint32_t>(i); };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
@@ -220,9 +229,9 @@ gated_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 tma_load_2d(sQ + hf * BM * 128, &tmQ, h * HD + hf * 64, seq0 + qt * BM, bar(B_Q_FULL));
             int k_issued[2] = {0, 0}, v_issued[2] = {0, 0};
             for (int j = 0; j < n_kv; ++j) {
-                const int s = j & 1;
-                if (j >= 2 && !mbar_wait(bar(B_K_EMPTY + s), ((j - 2) >> 1) & 1, abort_flag, status,
-                                         TG_WHERE_PRODUCER))
+                const int s = j % NS;
+                if (j >= NS && !mbar_wait(bar(B_K_EMPTY + s), ((j - NS) / NS) & 1, abort_flag, status,
+                                          TG_WHERE_PRODUCER))
                     break;
                 mbar_expect_tx(bar(B_K_FULL + s), BN * HD * 2);
 #pragma unroll
@@ -230,8 +239,8 @@ gated_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     tma_load_2d(sK0 + s * L::TILE_KV + hf * BN * 128, &tmK, hk * HD + hf * 64, seq0 + j * BN,
                                 bar(B_K_FULL + s));
                 ++k_issued[s];
-                if (j >= 2 && !mbar_wait(bar(B_V_EMPTY + s), ((j - 2) >> 1) & 1, abort_flag, status,
-                                         TG_WHERE_PRODUCER))
+                if (j >= NS && !mbar_wait(bar(B_V_EMPTY + s), ((j - NS) / NS) & 1, abort_flag, status,
+                                          TG_WHERE_PRODUCER))
                     break;
                 mbar_expect_tx(bar(B_V_FULL + s), BN * HD * 2);
 #pragma unroll
@@ -243,7 +252,7 @@ gated_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             if (*abort_flag) {
                 // let every copy this thread started land before the CTA exits
                 drain_wait(bar(B_Q_FULL), 0, status);
-                for (int s = 0; s < 2; ++s) {
+                for (int s = 0; s < NS; ++s) {
                     if (k_issued[s]) drain_wait(bar(B_K_FULL + s), (k_issued[s] - 1) & 1, status);
                     if (v_issued[s]) drain_wait(bar(B_V_FULL + s), (v_issued[s] - 1) & 1, status);
                 }
@@ -257,14 +266,14 @@ gated_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             bool ok = mbar_wait(bar(B_Q_FULL), 0, abort_flag, status, TG_WHERE_MMA);
             for (int j = 0; ok && j <= n_kv; ++j) {
                 if (j < n_kv) {
-                    const int s = j & 1;
-                    ok = mbar_wait(bar(B_K_FULL + s), (j >> 1) & 1, abort_flag, status, TG_WHERE_MMA);
+                    const int s = j & 1, ks = j % NS;
+                    ok = mbar_wait(bar(B_K_FULL + ks), (j / NS) & 1, abort_flag, status, TG_WHERE_MMA);
                     if (ok && j >= 2)
                         ok = mbar_wait(bar(B_S_FREE + s), ((j - 2) >> 1) & 1, abort_flag, status, TG_WHERE_MMA);
                     if (!ok) break;
                     tc_fence_after();
                     const uint32_t d = tmem + s * BN;
-                    const uint32_t kb = sK0 + s * L::TILE_KV;
+                    const uint32_t kb = sK0 + ks * L::TILE_KV;
 #pragma unroll
                     for (int kk = 0; kk < HD / 16; ++kk) {
                         const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
@@ -273,24 +282,22 @@ gated_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                                     idesc_qk, kk > 0 ? 1u : 0u);
                     }
                     mma_commit(bar(B_S_FULL + s));
-                    mma_commit(bar(B_K_EMPTY + s));
+                    mma_commit(bar(B_K_EMPTY + ks));
                 }
                 if (j >= 1) {
-                    const int jj = j - 1, s = jj & 1;
+                    const int jj = j - 1, s = jj & 1, vs = jj % NS;
                     ok = mbar_wait(bar(B_P_FULL), jj & 1, abort_flag, status, TG_WHERE_MMA);
-                    if (ok) ok = mbar_wait(bar(B_V_FULL + s), (jj >> 1) & 1, abort_flag, status, TG_WHERE_MMA);
+                    if (ok) ok = mbar_wait(bar(B_V_FULL + vs), (jj / NS) & 1, abort_flag, status, TG_WHERE_MMA);
                     if (!ok) break;
                     tc_fence_after();
-                    const uint32_t vb = sV0 + s * L::TILE_KV;
+                    const uint32_t vb = sV0 + vs * L::TILE_KV;
+                    // A = P_jj from TMEM (16 keys = 8 columns of bf16 pairs per k-step)
 #pragma unroll
-                    for (int kk = 0; kk < BN / 16; ++kk) {
-                        const uint32_t offp = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-                        mma_bf16_ss(tmem_O, smem_desc_sw128(sP + offp, 16, 1024),
-                                    smem_desc_sw128(vb + kk * 16 * 128, BN * 128, 1024), idesc_pv,
-                                    (jj > 0 || kk > 0) ? 1u : 0u);
-                    }
+                    for (int kk = 0; kk < BN / 16; ++kk)
+                        mma_bf16_ts(tmem_O, tmem + s * BN + kk * 8, smem_desc_sw128(vb + kk * 16 * 128, BN * 128, 1024),
+                                    idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
                     mma_commit(bar(B_PV_DONE));
-                    mma_commit(bar(B_V_EMPTY + s));
+                    mma_commit(bar(B_V_EMPTY + vs));
                 }
             }
             // every MMA (and the barrier arrivals its commits trigger) lands before the CTA exits
@@ -390,22 +397,16 @@ gated_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 }
                 tmem_wait_st();
             }
-            // P row r as bf16 into the 128-byte-swizzled K-major tile (two 64-key halves)
+            // P row r as bf16 pairs over the first 64 columns of its S buffer (the A
+            // operand of the PV MMA, read from TMEM)
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
-                uint8_t* rowp = smem + L::OFF_P + hf * (BM * 128) + r * 128;
+                uint32_t pk[32];
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    const float* p = x + hf * 64 + ch * 8;
-                    uint4 v;
-                    v.x = pack_bf16x2(p[0], p[1]);
-                    v.y = pack_bf16x2(p[2], p[3]);
-                    v.z = pack_bf16x2(p[4], p[5]);
-                    v.w = pack_bf16x2(p[6], p[7]);
-                    *reinterpret_cast<uint4*>(rowp + ((ch ^ (r & 7)) << 4)) = v;
-                }
+                for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(x[hf * 64 + 2 * e], x[hf * 64 + 2 * e + 1]);
+                tmem_st32u(tmem + lane_addr + s * BN + hf * 32, pk);
             }
-            fence_proxy_async_smem();
+            tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar(B_P_FULL));
         }
@@ -1189,9 +1190,11 @@ cudaError_t launch_tc(const uint16_t* q, const uint16_t* k, const uint16_t* v, c
         !encode_tmap_2d_bf16(&tv, v, static_cast<uint64_t>(Hkv) * HD, static_cast<uint64_t>(M_total),
                              static_cast<uint64_t>(Hkv) * HD * 2, 64, BN))
         return cudaErrorInvalidValue;
-    if ((Hq / Hkv) % 2 == 0)
-        return launch_gqa2<HD>(tq, tk, tv, cu_kept, B, max_M, Hq, Hkv, pos, rank, gates, c, sm_scale, out, lse, ws,
-                               ws_bytes, st);
+    if constexpr (HD <= 128) {  // two heads of 256 would need 768 TMEM columns
+        if ((Hq / Hkv) % 2 == 0)
+            return launch_gqa2<HD>(tq, tk, tv, cu_kept, B, max_M, Hq, Hkv, pos, rank, gates, c, sm_scale, out, lse,
+                                   ws, ws_bytes, st);
+    }
     int* status = device_status_ptr();
     const int n_qt_max = (max_M + BM - 1) / BM;
     dim3 grid(Hq, n_qt_max, B);
@@ -1219,6 +1222,9 @@ cudaError_t launch_gated_attention(const uint16_t* q, const uint16_t* k, const u
     if (d == 64)
         return launch_tc<64>(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, pos, rank, gates, c, sm_scale, out, lse,
                              ws, ws_bytes, st);
+    if (d == 256)
+        return launch_tc<256>(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, pos, rank, gates, c, sm_scale, out, lse,
+                              ws, ws_bytes, st);
     return launch_tc<128>(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, pos, rank, gates, c, sm_scale, out, lse, ws,
                           ws_bytes, st);
 }
@@ -1247,7 +1253,7 @@ int attention_kv_chunk(int B, int max_M, int Hq, int Hkv, bool have_ws) {
 
 size_t attention_workspace_bytes(int B, int max_M, int Hq, int Hkv, int d) {
     const int n_qt = (max_M + BM - 1) / BM;
-    if (B <= 0 || n_qt < 4 || (Hq / Hkv) % 2 != 0) return 0;
+    if (B <= 0 || n_qt < 4 || (Hq / Hkv) % 2 != 0 || d > 128) return 0;  // only the two-head kernel splits
     const int C = attention_kv_chunk(B, max_M, Hq, Hkv, true);
     if (C >= n_qt) return 0;  // this launch never splits
     const int64_t max_nch = (n_qt + C - 1) / C;

@@ -87,7 +87,7 @@ tg_status check_gate_shape(int D, int I) {
 }
 
 tg_status check_attn_shape(int Hq, int Hkv, int d) {
-    TG_SUPPORT(d == 64 || d == 128, "head_dim %d must be 64 or 128", d);
+    TG_SUPPORT(d == 64 || d == 128 || d == 256, "head_dim %d must be 64, 128 or 256", d);
     TG_REQUIRE(Hq > 0 && Hkv > 0 && Hq % Hkv == 0, "Hq=%d must be a positive multiple of Hkv=%d", Hq, Hkv);
     TG_SUPPORT(Hq <= 256, "Hq=%d above 256", Hq);
     return TG_OK;
@@ -165,7 +165,7 @@ extern "C" {
 
 size_t tg_masked_gated_attention_workspace_size(int B, int64_t T, int64_t M_total, int max_M, int Hq, int Hkv, int d) {
     if (B <= 0 || T <= 0 || M_total < 0 || max_M < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 ||
-        (d != 64 && d != 128))
+        (d != 64 && d != 128 && d != 256))
         return 0;
     return masked_layout(B, T, M_total, max_M, Hq, Hkv, d).total;
 }
@@ -342,7 +342,7 @@ tg_status tg_gated_attention_noalloc(const uint16_t* q, const uint16_t* k, const
 }
 
 size_t tg_gated_attention_workspace_size(int B, int max_M, int Hq, int Hkv, int d) {
-    if (B <= 0 || max_M <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || (d != 64 && d != 128)) return 0;
+    if (B <= 0 || max_M <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || (d != 64 && d != 128 && d != 256)) return 0;
     return tg::attention_workspace_bytes(B, max_M, Hq, Hkv, d);
 }
 

@@ -79,6 +79,11 @@ def test_invalid_shapes_are_refused_before_launch(lib):
     # head_dim 96
     st = lib.tg_gated_attention(P, P, P, P, 1, 10, 10, 4, 2, 96, P, P, P, P, P, 0.1, P, None, None, 0, None)
     assert st == _lib.TG_ERR_UNSUPPORTED
+    # head_dim 256 is supported (an empty batch returns before any device work) and
+    # never needs the causal-split scratch (one query head per CTA)
+    st = lib.tg_gated_attention(P, P, P, P, 0, 0, 0, 8, 2, 256, P, P, P, P, P, 0.1, P, None, None, 0, None)
+    assert st == _lib.TG_OK
+    assert lib.tg_gated_attention_workspace_size(1, 32768, 16, 8, 256) == 0
     # Hq not a multiple of Hkv
     st = lib.tg_gated_attention(P, P, P, P, 1, 10, 10, 6, 4, 64, P, P, P, P, P, 0.1, P, None, None, 0, None)
     assert st == _lib.TG_ERR_INVALID_ARG

@@ -116,6 +116,11 @@ def _build() -> dict:
         note="training-time full-budget gated attention, masked budget")
     cfg["c4_128k"] = _qwen3_17b("c4_128k", [131072], [(128, 130944)], [2000],
                                 note="long context 128k")
+    # head_dim 256 (the pages' key-bias kernel serves it for the Qwen3.5 models; their
+    # head counts are not given: 8 query and 2 KV heads, a small-model GQA layout)
+    cfg["c5_hd256_16k"] = Workload(
+        name="c5_hd256_16k", seqlens=(16384,), spans=((256, 16256),), budgets=(2000,),
+        D=2048, I=256, Hq=8, Hkv=2, d=256, note="head_dim 256 at 16k")
     lens = [8192, 24576, 65536, 131072]
     cfg["c4_varlen"] = _qwen3_17b(
         "c4_varlen", lens, [(128, n - 128) for n in lens], _varlen_budgets(4, 4, 100, 4000),
