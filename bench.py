@@ -37,7 +37,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from workloads import get_config, make_attention_inputs, make_gate_inputs  # noqa: E402
+from workloads import get_config, make_attention_inputs, make_gate_inputs, make_scores  # noqa: E402
 
 METRIC = "gated-prefill layer tokens/s; gated-attn TFLOP/s (% bf16 peak) at N=32k,K=2000"
 UNIT = "tokens/s"
@@ -236,6 +236,136 @@ def workload_config(w, n_layers):
 
 # ------------------------------------------------------------------ GPU arm
 
+def time_device_us(fn, st, flush, reps, warm=3):
+    """Median device time (us) of fn() on stream st, L2 flushed before each rep."""
+    import torch
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    ev = []
+    for i in range(reps):
+        flush.fill_(i)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        fn()
+        b.record(st)
+        ev.append((a, b))
+    torch.cuda.synchronize()
+    return 1e3 * float(np.median([a.elapsed_time(b) for a, b in ev]))
+
+
+def measure_next_rows(tg, dev, st, flush, main, peaks, reps=10):
+    """One measured figure per widened row, each on its own seeded workload:
+    masked full-length attention at a sampled budget, the KV-cache row gather,
+    head_dim 256 attention and four stacked gates.  Each is one C-ABI call with
+    its arguments bound beforehand (device-resident inputs and index arrays);
+    L2 is flushed before every rep."""
+    import ctypes
+    import torch
+    from workloads import masked_budgets
+
+    lib = tg.load()
+    sh = st.cuda_stream
+
+    def bf16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    def i32(a):
+        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(dev)
+
+    def check(fn):
+        def run():
+            assert fn() == 0, lib.tg_last_error_string()
+        return run
+
+    tc_peak, hbm_peak = float(peaks["bf16_tflops"]), float(peaks["hbm_gbs"])
+    res = {}
+    # f1: masked full-length attention (training layout), N=16384, K' sampled log-uniform
+    w = get_config("c3_full_budget_16k")
+    kb = np.asarray(masked_budgets(w, seed=0), np.int32)
+    ai = make_attention_inputs(w, w.T, layer=0)
+    q, k, v = bf16(ai["q"]), bf16(ai["k"]), bf16(ai["v"])
+    g, c = torch.from_numpy(ai["g"]).to(dev), torch.from_numpy(ai["c"]).to(dev)
+    s = torch.from_numpy(make_scores(w.T, std=2.0, seed=w.seed)).to(dev)
+    out = torch.empty((w.T, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
+    keep = torch.empty(w.T, dtype=torch.uint8, device=dev)
+    cu, sp = w.cu_seqlens(), w.span_array()
+    Mm, ck = tg.tg_kept_count(cu, sp, kb)
+    maxm = int(np.max(np.diff(ck)))
+    cu_d, sp_d, kb_d, ck_d = i32(cu), i32(sp), i32(kb), i32(ck)
+    nws = int(lib.tg_masked_gated_attention_workspace_size(w.B, w.T, Mm, maxm, w.Hq, w.Hkv, w.d))
+    mws = torch.zeros(max(nws, 256), dtype=torch.uint8, device=dev)
+    fl, _ = attention_flops(ck, w.Hq, w.d)
+    us = time_device_us(check(lambda: lib.tg_masked_gated_attention(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), s.data_ptr(), cu_d.data_ptr(), sp_d.data_ptr(), kb_d.data_ptr(),
+        ck_d.data_ptr(), w.B, w.T, Mm, maxm, w.Hq, w.Hkv, w.d, g.data_ptr(), c.data_ptr(), 1.0 / math.sqrt(w.d),
+        out.data_ptr(), keep.data_ptr(), mws.data_ptr(), mws.numel(), sh)), st, flush, reps)
+    res["f1_masked_attention"] = {"workload": f"{w.name}: N={w.T}, K'={int(kb[0])} (log-uniform in [1, |P|/2]), M={Mm}",
+                                  "us": us, "kept_pair_tflops": fl / (us * 1e-6) / 1e12,
+                                  "includes": "zero fill of pruned rows + select map + Q/K/V row gather + attention "
+                                              "+ scatter"}
+    del q, k, v, out, s, mws
+    # f2: lower-layer KV cache gathered to the kept tokens (one layer's K cache)
+    wm = main["w"]
+    kcache = torch.randn((wm.T, wm.Hkv, wm.d), device=dev).to(torch.bfloat16)
+    kdst = torch.empty((main["M"], wm.Hkv, wm.d), dtype=torch.bfloat16, device=dev)
+    row_bytes = wm.Hkv * wm.d * 2
+    us = time_device_us(check(lambda: lib.tg_gather_rows(kcache.data_ptr(), wm.T, row_bytes,
+                                                         main["kept_idx"].data_ptr(), main["M"], kdst.data_ptr(), sh)),
+                        st, flush, reps)
+    nbytes = 2 * main["M"] * row_bytes
+    res["f2_kv_gather"] = {"workload": f"{wm.name}: K cache [{wm.T}, {wm.Hkv}, {wm.d}] bf16 -> {main['M']} rows",
+                           "us": us, "bytes": nbytes, "gbs": nbytes / (us * 1e-6) / 1e9,
+                           "frac_of_hbm": nbytes / (us * 1e-6) / 1e9 / hbm_peak}
+    del kcache, kdst
+    # f3: head_dim 256 attention, N=16384, K=2000
+    w = get_config("c5_hd256_16k")
+    cu, sp, kk = w.cu_seqlens(), w.span_array(), w.budget_array()
+    M, ck = tg.tg_kept_count(cu, sp, kk)
+    s = torch.from_numpy(make_scores(w.T, std=2.0, seed=w.seed)).to(dev)
+    _, cmap = tg.tg_select_topk(s, cu, sp, kk, cu_kept=ck, M_total=M)
+    ai = make_attention_inputs(w, M, layer=0)
+    q, k, v = bf16(ai["q"]), bf16(ai["k"]), bf16(ai["v"])
+    g, c = torch.from_numpy(ai["g"]).to(dev), torch.from_numpy(ai["c"]).to(dev)
+    out = torch.empty((M, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
+    ck_d = i32(ck)
+    maxM = int(np.max(np.diff(ck)))
+    fl, _ = attention_flops(ck, w.Hq, w.d)
+    us = time_device_us(check(lambda: lib.tg_gated_attention(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), ck_d.data_ptr(), w.B, M, maxM, w.Hq, w.Hkv, w.d,
+        cmap["pos"].data_ptr(), cmap["rank"].data_ptr(), cmap["gls"].data_ptr(), g.data_ptr(), c.data_ptr(),
+        1.0 / math.sqrt(w.d), out.data_ptr(), None, None, 0, sh)), st, flush, reps)
+    res["f3_hd256_attention"] = {"workload": f"{w.name}: M={M}, Hq={w.Hq}, Hkv={w.Hkv}, d={w.d}", "us": us,
+                                 "tflops": fl / (us * 1e-6) / 1e12,
+                                 "frac_of_bf16_peak": fl / (us * 1e-6) / 1e12 / tc_peak}
+    # f4: four stacked gates on the main workload's attention (same inputs as the step's)
+    L0, wm, bufs = main["layer"], main["w"], main["bufs"]
+    rng = np.random.default_rng(5)
+    extra = [torch.from_numpy(np.where(main["gls_host"] != 0, -np.abs(rng.standard_normal(main["M"])), 0.0)
+                              .astype(np.float32)).to(dev) for _ in range(3)]
+    gains = [L0["g"]] + [torch.from_numpy(rng.standard_normal(wm.Hq).astype(np.float32)).to(dev) for _ in range(3)]
+    gls_arr = (ctypes.c_void_p * 4)(*([bufs.gls.data_ptr()] + [t.data_ptr() for t in extra]))
+    g_arr = (ctypes.c_void_p * 4)(*[t.data_ptr() for t in gains])
+    out = torch.empty((main["M"], wm.Hq, wm.d), dtype=torch.bfloat16, device=dev)
+    ck_d = i32(main["cu_kept"])
+    ws_t = main["ws"]
+    ws_p, ws_n = (None, 0) if ws_t is None else (ws_t.data_ptr(), ws_t.numel())
+    fl, _ = attention_flops(main["cu_kept"], wm.Hq, wm.d)
+    sm = 1.0 / math.sqrt(wm.d)
+    common = (L0["q"].data_ptr(), L0["k"].data_ptr(), L0["v"].data_ptr(), ck_d.data_ptr(), wm.B, main["M"],
+              main["max_M"], wm.Hq, wm.Hkv, wm.d, bufs.pos.data_ptr(), bufs.rank.data_ptr())
+    us = time_device_us(check(lambda: lib.tg_gated_attention_gates(*common, 4, gls_arr, g_arr, L0["c"].data_ptr(), sm,
+                                                                   out.data_ptr(), None, ws_p, ws_n, sh)),
+                        st, flush, reps)
+    us1 = time_device_us(check(lambda: lib.tg_gated_attention(*common, bufs.gls.data_ptr(), L0["g"].data_ptr(),
+                                                              L0["c"].data_ptr(), sm, out.data_ptr(), None, ws_p,
+                                                              ws_n, sh)), st, flush, reps)
+    res["f4_four_gates_attention"] = {"workload": f"{wm.name}: M={main['M']}, 4 gates", "us": us,
+                                      "tflops": fl / (us * 1e-6) / 1e12, "one_gate_us": us1,
+                                      "vs_one_gate": us / us1}
+    return res
+
+
 def run_gpu(args, w):
     import torch
     import torch.distributed as dist
@@ -408,6 +538,12 @@ def run_gpu(args, w):
     s13_bytes = sb["score"] + sb["select"] + sb["gather"]
     s13_us = stage_us["score"] + stage_us["select"] + stage_us["gather"]
 
+    next_rows = None
+    if rank == 0 and not args.no_next_rows:
+        main_ctx = {"w": w, "M": M, "cu_kept": cu_kept, "max_M": call.max_M, "kept_idx": bufs.kept_idx,
+                    "layer": L0, "bufs": bufs, "gls_host": bufs.gls.cpu().numpy(), "ws": call.ws}
+        next_rows = measure_next_rows(tg, dev, st, flush, main_ctx, peaks)
+
     cpu_base = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         import oracle
@@ -430,6 +566,7 @@ def run_gpu(args, w):
                 "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                         "d2h_bytes_per_step": int(d2h)},
                 "gpu_launches": args.steps * (3 + args.layers), "cuda_graph": graph is not None,
+                "next_rows": next_rows,
                 "cpu_baseline": cpu_base, "clocks": clk, "peaks": {"source": peaks["source"],
                                                                    "hbm_gbs": hbm_peak, "bf16_tflops": tc_peak}}
         print(json.dumps(line), flush=True)
@@ -448,6 +585,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="c2_32k_k2000")
     ap.add_argument("--layers", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-next-rows", action="store_true",
+                    help="skip the measurements of masked attention, KV gather, head_dim 256 and stacked gates")
     ap.add_argument("--no-graph", action="store_true", help="launch the step directly instead of a CUDA graph")
     args = ap.parse_args(argv)
     if args.warmup < 3:
