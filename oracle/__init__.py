@@ -55,7 +55,9 @@ def _load():
                                                    P, i64, P, P, i32, i32]
             lib.oracle_masked_gated_attention.argtypes = [P, P, P, P, P, i32, i32, i32, i32, P, P, P, P,
                                                           f64, P, i64, P]
-            if lib.oracle_abi_version() != 2:
+            lib.oracle_gated_attention_backward.argtypes = [P, P, P, P, i32, i32, i32, i32, P, P, P, P, P, f64,
+                                                            P, P, P, P, P, P, P]
+            if lib.oracle_abi_version() != 3:
                 raise ImportError("oracle/liboracle.so is stale: rebuild it")
             _lib = lib
     return _lib
@@ -194,6 +196,33 @@ def gated_attention(q_bits, k_bits, v_bits, cu_kept, pos, rank, gls_f32, g, c, s
                                    None if lse is None else lse.ctypes.data_as(C.c_void_p),
                                    1 if tau_on_qk_only else 0, n_gates)
     return out, lse
+
+
+def gated_attention_backward(q_bits, k_bits, v_bits, cu_kept, pos, rank, gls_f32, g, c, dout, sm_scale=None) -> dict:
+    """Gradients of the token-gated attention (one gate) for the upstream
+    gradient dout [M, Hq, d]: dq [M, Hq, d], dk/dv [M, Hkv, d], dgls [M],
+    dg/dc [Hq], all fp64.  d loss / d score_j = dgls_j * sigmoid(-score_j)."""
+    q, qp = _c(q_bits, np.uint16)
+    k, kp = _c(k_bits, np.uint16)
+    v, vp_ = _c(v_bits, np.uint16)
+    M, Hq, d = q.shape
+    Hkv = k.shape[1]
+    cu, cup = _c(cu_kept, np.int32)
+    po, pop = _c(pos, np.int32)
+    ra, rap = _c(rank, np.int32)
+    gl, glp = _c(gls_f32, np.float32)
+    ga, gap = _c(g, np.float32)
+    ca, cap = _c(c, np.float32)
+    go, gop = _c(np.asarray(dout, dtype=np.float64).reshape(M, Hq, d), np.float64)
+    if sm_scale is None:
+        sm_scale = 1.0 / np.sqrt(d)
+    out = {"dq": np.empty((M, Hq, d)), "dk": np.empty((M, Hkv, d)), "dv": np.empty((M, Hkv, d)),
+           "dgls": np.empty(M), "dg": np.empty(Hq), "dc": np.empty(Hq)}
+    vp = lambda a: a.ctypes.data_as(C.c_void_p)  # noqa: E731
+    _load().oracle_gated_attention_backward(qp, kp, vp_, cup, len(cu) - 1, Hq, Hkv, d, pop, rap, glp, gap, cap,
+                                            float(sm_scale), gop, vp(out["dq"]), vp(out["dk"]), vp(out["dv"]),
+                                            vp(out["dgls"]), vp(out["dg"]), vp(out["dc"]))
+    return out
 
 
 def next_gate_span(first: dict, cu_seqlens, span) -> np.ndarray:

@@ -1,0 +1,129 @@
+"""CPU pins of the oracle's backward of the token-gated attention.
+
+Pinned against things other than its own chain rule: PyTorch fp64 autograd
+through the forward written as library calls (per-row scaled_dot_product_
+attention of the query scaled by sm/tau with additive mask softplus(g) gls / tau -- the
+composition the forward pins already tie to the oracle's forward), central
+differences of the oracle's own forward for g, c and gls, and the closed form
+of uniform values (the output no longer depends on any logit).
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+from workloads import bf16_bits_to_f32, f32_to_bf16_bits
+
+
+def _case(seed, seqlens, Hq, Hkv, d, std=0.8):
+    rng = np.random.default_rng(seed)
+    M = sum(seqlens)
+    q = f32_to_bf16_bits((rng.standard_normal((M, Hq, d)) * std).astype(np.float32))
+    k = f32_to_bf16_bits((rng.standard_normal((M, Hkv, d)) * std).astype(np.float32))
+    v = f32_to_bf16_bits(rng.standard_normal((M, Hkv, d)).astype(np.float32))
+    cu = np.concatenate([[0], np.cumsum(seqlens)]).astype(np.int32)
+    rank = np.concatenate([np.arange(1, n + 1) for n in seqlens]).astype(np.int32)
+    pos = (rank + np.concatenate([np.sort(rng.integers(0, 30, n)) for n in seqlens])).astype(np.int32)
+    gls = -np.abs(rng.standard_normal(M) * 2).astype(np.float32)
+    gls[:3] = 0.0
+    g = rng.standard_normal(Hq).astype(np.float32)
+    c = (0.6 * rng.random(Hq)).astype(np.float32)
+    dout = rng.standard_normal((M, Hq, d))
+    return q, k, v, cu, pos, rank, gls, g, c, dout
+
+
+def _autograd(q, k, v, cu, pos, rank, gls, g, c, dout):
+    Hq, Hkv, d = q.shape[1], k.shape[1], q.shape[2]
+    qt = torch.tensor(bf16_bits_to_f32(q), dtype=torch.float64, requires_grad=True)
+    kt = torch.tensor(bf16_bits_to_f32(k), dtype=torch.float64, requires_grad=True)
+    vt = torch.tensor(bf16_bits_to_f32(v), dtype=torch.float64, requires_grad=True)
+    gl = torch.tensor(gls, dtype=torch.float64, requires_grad=True)
+    gt = torch.tensor(g, dtype=torch.float64, requires_grad=True)
+    ct = torch.tensor(c, dtype=torch.float64, requires_grad=True)
+    sm = 1.0 / math.sqrt(d)
+    outs = []
+    for b in range(len(cu) - 1):
+        for i in range(cu[b], cu[b + 1]):
+            row = []
+            for h in range(Hq):
+                hk = h // (Hq // Hkv)
+                tau = 1 + ct[h] * math.log(pos[i] / rank[i])
+                mask = F.softplus(gt[h]) * gl[cu[b]:i + 1] / tau
+                # SDPA's scale is a plain number: sm / tau enters through the query instead
+                o = F.scaled_dot_product_attention((qt[i, h] * (sm / tau))[None, None, None],
+                                                   kt[cu[b]:i + 1, hk][None, None], vt[cu[b]:i + 1, hk][None, None],
+                                                   attn_mask=mask[None, None, None], scale=1.0)
+                row.append(o[0, 0, 0])
+            outs.append(torch.stack(row))
+    out = torch.stack(outs)
+    (out * torch.from_numpy(dout)).sum().backward()
+    return {"dq": qt.grad.numpy(), "dk": kt.grad.numpy(), "dv": vt.grad.numpy(), "dgls": gl.grad.numpy(),
+            "dg": gt.grad.numpy(), "dc": ct.grad.numpy()}
+
+
+@pytest.mark.parametrize("seed,seqlens,Hq,Hkv,d", [(1, [13, 9], 4, 2, 8), (2, [1, 17], 3, 1, 4),
+                                                   (3, [20], 2, 2, 16)])
+def test_backward_matches_autograd_of_library_forward(oracle_mod, seed, seqlens, Hq, Hkv, d):
+    q, k, v, cu, pos, rank, gls, g, c, dout = _case(seed, seqlens, Hq, Hkv, d)
+    ref = _autograd(q, k, v, cu, pos, rank, gls, g, c, dout)
+    got = oracle_mod.gated_attention_backward(q, k, v, cu, pos, rank, gls, g, c, dout)
+    for key in ("dq", "dk", "dv", "dgls", "dg", "dc"):
+        np.testing.assert_allclose(got[key], ref[key], rtol=1e-9, atol=1e-11, err_msg=key)
+
+
+def _loss(oracle_mod, q, k, v, cu, pos, rank, gls, g, c, dout):
+    out, _ = oracle_mod.gated_attention(q, k, v, cu, pos, rank, gls, g, c)
+    return float(np.sum(out * dout))
+
+
+def test_backward_matches_central_differences(oracle_mod):
+    """Gain, temperature and one logsigmoid perturbed by +-2^-12 (exact in fp32)."""
+    q, k, v, cu, pos, rank, gls, g, c, dout = _case(4, [15, 10], 4, 2, 8)
+    got = oracle_mod.gated_attention_backward(q, k, v, cu, pos, rank, gls, g, c, dout)
+    eps = 2.0 ** -12
+    for h in range(4):
+        gp, gm = g.copy(), g.copy()
+        gp[h] += eps
+        gm[h] -= eps
+        fd = (_loss(oracle_mod, q, k, v, cu, pos, rank, gls, gp, c, dout) -
+              _loss(oracle_mod, q, k, v, cu, pos, rank, gls, gm, c, dout)) / (2 * eps)
+        assert got["dg"][h] == pytest.approx(fd, rel=1e-4, abs=1e-8)
+        cp, cm = c.copy(), c.copy()
+        cp[h] += eps
+        cm[h] -= eps
+        fd = (_loss(oracle_mod, q, k, v, cu, pos, rank, gls, g, cp, dout) -
+              _loss(oracle_mod, q, k, v, cu, pos, rank, gls, g, cm, dout)) / (2 * eps)
+        assert got["dc"][h] == pytest.approx(fd, rel=1e-4, abs=1e-8)
+    for j in (3, 7, 14, 20):
+        lp, lm = gls.copy(), gls.copy()
+        lp[j] += eps
+        lm[j] -= eps
+        fd = (_loss(oracle_mod, q, k, v, cu, pos, rank, lp, g, c, dout) -
+              _loss(oracle_mod, q, k, v, cu, pos, rank, lm, g, c, dout)) / (2 * eps)
+        assert got["dgls"][j] == pytest.approx(fd, rel=1e-4, abs=1e-8)
+
+
+def test_uniform_values_give_no_logit_gradient(oracle_mod):
+    """With every value row equal the output is that row whatever the logits: all
+    gradients through the logits vanish, and the value gradient sums to the
+    output gradient (the weights of each row sum to one)."""
+    q, k, v, cu, pos, rank, gls, g, c, dout = _case(5, [12, 8], 4, 2, 8)
+    v = np.repeat(v[:1], len(v), axis=0)
+    got = oracle_mod.gated_attention_backward(q, k, v, cu, pos, rank, gls, g, c, dout)
+    for key in ("dq", "dk", "dgls", "dg", "dc"):
+        assert np.max(np.abs(got[key])) < 1e-12, key
+    for hk in range(2):
+        want = dout[:, 2 * hk:2 * hk + 2].sum(axis=(0, 1))
+        np.testing.assert_allclose(got["dv"][:, hk].sum(axis=0), want, rtol=1e-12, atol=1e-12)
+
+
+def test_temperature_gradient_vanishes_where_pos_equals_rank(oracle_mod):
+    """ln(pos/rank) = 0 rows carry no temperature gradient: with every pos equal to
+    its rank, dc is exactly 0 while dg is not."""
+    q, k, v, cu, pos, rank, gls, g, c, dout = _case(6, [16], 2, 1, 8)
+    got = oracle_mod.gated_attention_backward(q, k, v, cu, rank.copy(), rank, gls, g, c, dout)
+    assert (got["dc"] == 0).all()
+    assert np.abs(got["dg"]).max() > 1e-6
