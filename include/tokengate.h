@@ -201,6 +201,37 @@ tg_status tg_gated_attention_gates(const uint16_t* q, const uint16_t* k, const u
                                    size_t ws_bytes, tg_stream_t stream);
 
 /*
+ * Backward of tg_gated_attention (one gate): the gradient path that makes the
+ * gate trainable (AI summary, "Key Contributions" 2: the bias on the logits
+ * carries the task loss's gradient back to the scoring network; 3: the gain
+ * and temperature are learned; 4: training runs this attention at full budget
+ * and at a sampled budget).  With l_ij = (sm q_i.k_j + softplus(g_h) gls_j) /
+ * tau_ih and P = softmax(l), for the upstream gradient dout [M, Hq, d] bf16:
+ *   dq [M, Hq, d], dk / dv [M, Hkv, d] bf16 (GQA: dk, dv summed over the
+ *   query heads of each KV head);
+ *   dgls [M] fp32 = d loss / d gls_j (summed over heads);
+ *   dscore [M] fp32 (may be NULL) = dgls_j * sigmoid(-score_j), computed as
+ *   dgls_j * (1 - exp(gls_j)): the gradient reaching the gate's score of kept
+ *   row j (0 for rows the gate cannot prune, whose gls is 0);
+ *   dg, dc [Hq] fp32 = gradients of the gain and temperature parameters.
+ * q, k, v, pos, rank, gls, g, c, cu_kept, sm_scale as passed to the forward;
+ * out [M, Hq, d] bf16 and lse [M, Hq] fp32 are the forward's outputs (call
+ * tg_gated_attention with a non-NULL lse).  head_dim 64 or 128 (else
+ * TG_ERR_UNSUPPORTED).  ws: device scratch, 256-byte aligned, of at least
+ * tg_gated_attention_backward_workspace_size(M_total, Hq) bytes (4 floats per
+ * row and head; no zeroing needed).  Tensor cores, no atomics: the results are
+ * deterministic.
+ */
+size_t tg_gated_attention_backward_workspace_size(int64_t M_total, int Hq);
+tg_status tg_gated_attention_backward(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* out,
+                                      const uint16_t* dout, const float* lse, const int32_t* cu_kept, int B,
+                                      int64_t M_total, int max_M, int Hq, int Hkv, int d, const int32_t* pos,
+                                      const int32_t* rank, const float* gls, const float* g, const float* c,
+                                      float sm_scale, uint16_t* dq, uint16_t* dk, uint16_t* dv, float* dgls,
+                                      float* dscore, float* dg, float* dc, void* ws, size_t ws_bytes,
+                                      tg_stream_t stream);
+
+/*
  * Host only: the prunable span of the NEXT gate, in the kept order of this
  * one.  All tokens before a span are kept, so sequence b's surviving span
  * tokens sit at kept indices [p0_b, p0_b + min(k_b, |P_b|)) (k_b < 0 = all).

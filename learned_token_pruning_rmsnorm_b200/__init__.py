@@ -24,7 +24,7 @@ from ._lib import TokenGateError, load  # noqa: F401
 __all__ = [
     "TokenGateError", "load", "tg_abi_version", "tg_kept_count", "tg_gate_prepare", "tg_score",
     "tg_select_topk", "tg_compact", "tg_gather_kept", "tg_gather_rows", "tg_gated_attention",
-    "tg_gated_attention_gates", "tg_next_gate_span", "tg_masked_gated_attention",
+    "tg_gated_attention_gates", "tg_next_gate_span", "tg_gated_attention_backward", "tg_masked_gated_attention",
     "tg_gated_prefill_layer",
     "tg_device_status", "tg_selftest_bounded_wait",
 ]
@@ -333,6 +333,44 @@ def tg_gated_attention_gates(q, k, v, cu_kept, max_M: int, pos, rank, gls, g, c,
                                                out.data_ptr(), _lib.ptr(lse), _lib.ptr(ws),
                                                0 if ws is None else ws.numel(), _lib.stream_handle(dev)))
     return (out, lse) if want_lse or lse is not None else out
+
+
+def tg_gated_attention_backward(q, k, v, out, dout, lse, cu_kept, max_M: int, pos, rank, gls, g, c,
+                                sm_scale: float | None = None, want_dscore: bool = True):
+    """Gradients of tg_gated_attention for dout: returns a dict with dq, dk, dv
+    (bf16, shaped like q, k, v), dgls [M], dscore [M] (d loss / d score of each
+    kept row; None unless want_dscore), dg [Hq] and dc [Hq] (fp32).  out and lse
+    are the forward's outputs."""
+    M, Hq, d = q.shape
+    Hkv = k.shape[1]
+    dev = q.device
+    _dev(q, torch.bfloat16, "q")
+    _dev(k, torch.bfloat16, "k", (M, Hkv, d))
+    _dev(v, torch.bfloat16, "v", (M, Hkv, d))
+    _dev(out, torch.bfloat16, "out", (M, Hq, d))
+    _dev(dout, torch.bfloat16, "dout", (M, Hq, d))
+    _dev(lse, torch.float32, "lse", (M, Hq))
+    _dev(pos, torch.int32, "pos", (M,))
+    _dev(rank, torch.int32, "rank", (M,))
+    _dev(gls, torch.float32, "gls", (M,))
+    _dev(g, torch.float32, "g", (Hq,))
+    _dev(c, torch.float32, "c", (Hq,))
+    ck = _i32_dev(cu_kept, dev, "cu_kept")
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    res = {"dq": torch.empty_like(q), "dk": torch.empty_like(k), "dv": torch.empty_like(v),
+           "dgls": torch.empty(M, dtype=torch.float32, device=dev),
+           "dscore": torch.empty(M, dtype=torch.float32, device=dev) if want_dscore else None,
+           "dg": torch.empty(Hq, dtype=torch.float32, device=dev), "dc": torch.empty(Hq, dtype=torch.float32, device=dev)}
+    n = int(load().tg_gated_attention_backward_workspace_size(M, Hq))
+    ws = torch.empty(max(n, 256), dtype=torch.uint8, device=dev)
+    _lib.check(load().tg_gated_attention_backward(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(), lse.data_ptr(), ck.data_ptr(),
+        ck.numel() - 1, M, int(max_M), Hq, Hkv, d, pos.data_ptr(), rank.data_ptr(), gls.data_ptr(), g.data_ptr(),
+        c.data_ptr(), float(sm_scale), res["dq"].data_ptr(), res["dk"].data_ptr(), res["dv"].data_ptr(),
+        res["dgls"].data_ptr(), _lib.ptr(res["dscore"]), res["dg"].data_ptr(), res["dc"].data_ptr(), ws.data_ptr(),
+        ws.numel(), _lib.stream_handle(dev)))
+    return res
 
 
 def tg_device_status(clear: bool = True, device=None):

@@ -1,0 +1,794 @@
+// Backward of stage 4, the token-gated causal GQA attention (TokenGate AI
+// summary, "Key Contributions" 2 and 3: the gate bias is what carries the task
+// loss's gradient back to the scoring network, and the gain and temperature
+// are learned).  One gate.  With
+//   l_ij = (sm q_i.k_j + beta_h gls_j) / tau_ih,   beta_h = softplus(g_h),
+//   P = softmax_j(l),   out_i = sum_j P_ij v_j,
+// and the upstream gradient dout:
+//   dP_ij = dout_i.v_j,  D_i = dout_i.out_i,  dl_ij = P_ij (dP_ij - D_i),
+//   G_ij = dl_ij / tau_ih,
+//   dq_i = sm sum_j G_ij k_j,  dk_j = sm sum_i G_ij q_i,  dv_j = sum_i P_ij dout_i,
+//   dgls_j = sum_h beta_h sum_i G_ij,  dbeta_h = sum_ij G_ij gls_j,
+//   dtau_ih = -sum_j dl_ij l_ij / tau_ih,
+//   dg_h = dbeta_h sigmoid(g_h),  dc_h = sum_i dtau_ih ln(pos_i / rank_i),
+//   d score_j = dgls_j sigmoid(-score_j) = dgls_j (1 - exp(gls_j)).
+//
+// Five launches, no atomics (results do not depend on scheduling):
+//   rowdot   D_ih = dout_i.out_i for every (row, head)
+//   dq       (below)
+//   dkv      one CTA per (KV head, 128-key tile): for every query head of the
+//            group and every causal query tile, S^T = K Q^T and dP^T = V dO^T
+//            on the tensor core (TMEM lanes = keys), then P^T and G^T as bf16
+//            over the first 64 columns of S^T and dP^T, and dV += P^T dO,
+//            dK += G^T Q read from TMEM.  The per-key sums of G (the gate
+//            bias's gradient, per head) are sums along each thread's own row.
+//   dq       one CTA per (query head, 128-query tile), the forward's layout:
+//            S = Q K^T and dP = dO V^T, G as bf16 over S, dQ += G K.  The
+//            per-query sums for dbeta and dtau run along each thread's row,
+//            which also yields the exact D'_i = sum_j P_ij dP_ij; it replaces
+//            D for the dkv kernel (launched after dq).
+//   reduce   dgls / d score per key, dg and dc per head.
+// Every row of P is rebuilt from the forward's log-sum-exp.
+
+#include "tg_sm100.cuh"
+
+namespace tg {
+namespace {
+
+using namespace sm100;
+
+constexpr int BT = 128;  // rows of a query or key tile (= TMEM lanes)
+constexpr int BWD_THREADS = 192;
+constexpr float LOG2E_B = 1.4426950408889634f;
+constexpr float LN2_B = 0.6931471805599453f;
+
+__device__ __forceinline__ float softplus_b(float x) { return fmaxf(x, 0.f) + log1pf(expf(-fabsf(x))); }
+
+__device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ bool drain_wait_b(uint32_t bar, uint32_t parity, int* status) {
+    volatile int never = 0;
+    return mbar_wait(bar, parity, &never, status, TG_WHERE_DRAIN);
+}
+
+// ---------------------------------------------------------------------------
+// D_r = dout_r . out_r for each of the M * Hq rows of d elements; one warp per row.
+__global__ void __launch_bounds__(256)
+bwd_rowdot_kernel(const uint16_t* __restrict__ out, const uint16_t* __restrict__ dout, int64_t rows, int d,
+                  float* __restrict__ D) {
+    pdl_wait();
+    pdl_trigger();
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+    for (int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows;
+         r += warps) {
+        const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(out + r * d);
+        const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(dout + r * d);
+        float acc = 0.f;
+        for (int e = lane; e < d / 2; e += 32) {
+            const float2 a = __bfloat1622float2(o2[e]), b = __bfloat1622float2(g2[e]);
+            acc = fmaf(a.x, b.x, fmaf(a.y, b.y, acc));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) D[r] = acc;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// dK, dV and the per-key sums of G: one CTA per (KV head, 128-key tile, sequence).
+//
+// 192 threads: warps 0-3 compute (thread r = key row r of the tile = TMEM lane),
+// warp 4 TMA producer, warp 5 MMA issuer.  The K and V tiles stay resident; the
+// (Q, dO) tiles of every (query head of the group, causal query tile) stream
+// through a two-stage ring.  TMEM (512 columns): S^T | dP^T | dV | dK.  Per step
+// the issuer waits for the compute warps' P^T and G^T of the previous step,
+// accumulates dV += P^T dO and dK += G^T Q from TMEM, then issues the next
+// S^T = K Q^T and dP^T = V dO^T (tcgen05 operations of one thread execute in
+// issue order, so S^T and dP^T are overwritten only after the products that
+// read P^T and G^T).  The compute warps rebuild each element of P^T from the
+// query's log-sum-exp; the per-query factors come from a shared-memory table
+// that the compute threads fill (one query row each) before every step.
+template <int HD>
+struct DkvSmem {
+    static constexpr int TILE = BT * HD * 2;
+    static constexpr int OFF_K = 0;
+    static constexpr int OFF_V = OFF_K + TILE;
+    static constexpr int OFF_Q = OFF_V + TILE;        // [2 stages]
+    static constexpr int OFF_DO = OFF_Q + 2 * TILE;   // [2 stages]
+    static constexpr int OFF_PAR = OFF_DO + 2 * TILE; // [2 stages][5][BT] fp32
+    static constexpr int OFF_BAR = OFF_PAR + 2 * 5 * BT * 4;
+    static constexpr int NUM_BARS = 12;
+    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+    static constexpr int BYTES = OFF_MISC + 16;
+    static constexpr int ALLOC = BYTES + 1024;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static_assert(ALLOC <= 227 * 1024, "shared memory");
+    static_assert(2 * BT + 2 * HD <= 512, "TMEM columns");
+};
+
+enum : int { D_KV_FULL = 0, D_QD_FULL = 1, D_QD_EMPTY = 3, D_SDP_FULL = 5, D_PG_FULL = 6, D_ACC_DONE = 7, D_DRAIN = 8 };
+
+template <int HD>
+__global__ void __launch_bounds__(BWD_THREADS, 1)
+gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                          const int32_t* __restrict__ cu_kept, const int32_t* __restrict__ pos,
+                          const int32_t* __restrict__ rank, const float* __restrict__ gls,
+                          const float* __restrict__ g, const float* __restrict__ c, const float* __restrict__ lse,
+                          const float* __restrict__ Drow, float sm_scale, int Hq, int Hkv, uint16_t* __restrict__ dk,
+                          uint16_t* __restrict__ dv, float* __restrict__ colsum, int* __restrict__ status) {
+    using L = DkvSmem<HD>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int hk = blockIdx.x, kt = blockIdx.y, b = blockIdx.z;
+    pdl_wait();  // global memory is read only from here on
+    pdl_trigger();
+    const int seq0 = cu_kept[b];
+    const int Mb = cu_kept[b + 1] - seq0;
+    if (kt * BT >= Mb) return;
+    const int n_qt = (Mb + BT - 1) / BT;
+    const int grp = Hq / Hkv;
+    const int nq = n_qt - kt;  // causal query tiles per head
+    const int n_steps = grp * nq;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t sK = sbase + L::OFF_K, sV = sbase + L::OFF_V, sQ = sbase + L::OFF_Q, sDO = sbase + L::OFF_DO;
+    auto bar = [&](int i) { return sbase + L::OFF_BAR + 8u * static_cast<uint32_t>(i); };
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(D_KV_FULL), 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar(D_QD_FULL + s), 1);
+            mbar_init(bar(D_QD_EMPTY + s), 1);
+        }
+        mbar_init(bar(D_SDP_FULL), 1);
+        mbar_init(bar(D_PG_FULL), 128);
+        mbar_init(bar(D_ACC_DONE), 1);
+        mbar_init(bar(D_DRAIN), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 4) {
+        tmem_alloc(smem_u32(tmem_slot), L::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tST = tmem, tDPT = tmem + BT, tDV = tmem + 2 * BT, tDK = tmem + 2 * BT + HD;
+
+    if (warp == 4) {
+        // ---------------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            prefetch_tmap(&tmQ);
+            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmV);
+            prefetch_tmap(&tmDO);
+            mbar_expect_tx(bar(D_KV_FULL), 2 * L::TILE);
+#pragma unroll
+            for (int hf = 0; hf < HD / 64; ++hf) {
+                tma_load_2d(sK + hf * BT * 128, &tmK, hk * HD + hf * 64, seq0 + kt * BT, bar(D_KV_FULL));
+                tma_load_2d(sV + hf * BT * 128, &tmV, hk * HD + hf * 64, seq0 + kt * BT, bar(D_KV_FULL));
+            }
+            int issued[2] = {0, 0};
+            for (int t = 0; t < n_steps; ++t) {
+                const int s = t & 1;
+                const int h = hk * grp + t / nq, i = kt + t % nq;
+                if (t >= 2 && !mbar_wait(bar(D_QD_EMPTY + s), ((t - 2) >> 1) & 1, abort_flag, status,
+                                         TG_WHERE_PRODUCER))
+                    break;
+                mbar_expect_tx(bar(D_QD_FULL + s), 2 * L::TILE);
+#pragma unroll
+                for (int hf = 0; hf < HD / 64; ++hf) {
+                    tma_load_2d(sQ + s * L::TILE + hf * BT * 128, &tmQ, h * HD + hf * 64, seq0 + i * BT,
+                                bar(D_QD_FULL + s));
+                    tma_load_2d(sDO + s * L::TILE + hf * BT * 128, &tmDO, h * HD + hf * 64, seq0 + i * BT,
+                                bar(D_QD_FULL + s));
+                }
+                ++issued[s];
+            }
+            if (*abort_flag) {
+                drain_wait_b(bar(D_KV_FULL), 0, status);
+                for (int s = 0; s < 2; ++s)
+                    if (issued[s]) drain_wait_b(bar(D_QD_FULL + s), (issued[s] - 1) & 1, status);
+            }
+        }
+    } else if (warp == 5) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = idesc_bf16_f32(BT, BT, false);
+            constexpr uint32_t idesc_acc = idesc_bf16_f32(BT, HD, true);
+            // dV += P^T dO(t), dK += G^T Q(t): A from TMEM (16 queries = 8 columns per
+            // k-step), B the (query x head_dim) tile read MN-major
+            auto issue_acc = [&](int t) {
+                const int s = t & 1;
+#pragma unroll
+                for (int kk = 0; kk < BT / 16; ++kk)
+                    mma_bf16_ts(tDV, tST + kk * 8, smem_desc_sw128(sDO + s * L::TILE + kk * 16 * 128, BT * 128, 1024),
+                                idesc_acc, (t > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                for (int kk = 0; kk < BT / 16; ++kk)
+                    mma_bf16_ts(tDK, tDPT + kk * 8, smem_desc_sw128(sQ + s * L::TILE + kk * 16 * 128, BT * 128, 1024),
+                                idesc_acc, (t > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(bar(D_QD_EMPTY + s));
+            };
+            bool ok = mbar_wait(bar(D_KV_FULL), 0, abort_flag, status, TG_WHERE_MMA);
+            for (int t = 0; ok && t < n_steps; ++t) {
+                const int s = t & 1;
+                ok = mbar_wait(bar(D_QD_FULL + s), (t >> 1) & 1, abort_flag, status, TG_WHERE_MMA);
+                if (ok && t >= 1) ok = mbar_wait(bar(D_PG_FULL), (t - 1) & 1, abort_flag, status, TG_WHERE_MMA);
+                if (!ok) break;
+                tc_fence_after();
+                if (t >= 1) issue_acc(t - 1);
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * (BT * 128) + (kk & 3) * 32;
+                    mma_bf16_ss(tST, smem_desc_sw128(sK + off, 16, 1024),
+                                smem_desc_sw128(sQ + s * L::TILE + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * (BT * 128) + (kk & 3) * 32;
+                    mma_bf16_ss(tDPT, smem_desc_sw128(sV + off, 16, 1024),
+                                smem_desc_sw128(sDO + s * L::TILE + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(bar(D_SDP_FULL));
+            }
+            if (ok) ok = mbar_wait(bar(D_PG_FULL), (n_steps - 1) & 1, abort_flag, status, TG_WHERE_MMA);
+            if (ok) {
+                tc_fence_after();
+                issue_acc(n_steps - 1);
+                mma_commit(bar(D_ACC_DONE));
+            }
+            mma_commit(bar(D_DRAIN));
+            drain_wait_b(bar(D_DRAIN), 0, status);
+        }
+    } else {
+        // ---------------------------------------------------------------- compute warps 0-3
+        const int r = threadIdx.x;  // key row of the tile == TMEM lane
+        const int key_local = kt * BT + r;
+        const bool valid_key = key_local < Mb;
+        const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+        const float gl = valid_key ? gls[seq0 + key_local] : 0.f;
+        float* par = reinterpret_cast<float*>(smem + L::OFF_PAR);
+        bool ok = true;
+        int t = 0;
+        for (int hh = 0; hh < grp && ok; ++hh) {
+            const int h = hk * grp + hh;
+            const float beta = softplus_b(g[h]);
+            float csum = 0.f;
+            for (int ii = 0; ii < nq; ++ii, ++t) {
+                const int i = kt + ii, s = t & 1;
+                // this thread's query row of tile i fills one column of the factor table
+                const int qrow = i * BT + r;
+                float fa = 0.f, fb = 0.f, fl = 0.f, fd = 0.f, fi = 0.f;
+                if (qrow < Mb) {
+                    const int qg = seq0 + qrow;
+                    fi = 1.0f / (1.0f + c[h] * logf(static_cast<float>(pos[qg]) / static_cast<float>(rank[qg])));
+                    fa = sm_scale * LOG2E_B * fi;
+                    fb = beta * LOG2E_B * fi;
+                    fl = lse[static_cast<size_t>(qg) * Hq + h] * LOG2E_B;
+                    fd = Drow[static_cast<size_t>(qg) * Hq + h];
+                }
+                float* ps = par + s * 5 * BT;
+                ps[0 * BT + r] = fa;
+                ps[1 * BT + r] = fb;
+                ps[2 * BT + r] = fl;
+                ps[3 * BT + r] = fd;
+                ps[4 * BT + r] = fi;
+                const bool okw = mbar_wait_warp(bar(D_SDP_FULL), t & 1, abort_flag, status, TG_WHERE_SOFTMAX);
+                // the table is complete past this barrier, which also makes an abort uniform
+                uint32_t any_abort;
+                asm volatile(
+                    "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, 1, 128, p;\n\t"
+                    "selp.u32 %0, 1, 0, q;\n\t}"
+                    : "=r"(any_abort)
+                    : "r"(static_cast<uint32_t>(!okw))
+                    : "memory");
+                if (any_abort) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const int col_lim = min(BT, Mb - i * BT);  // query columns inside the sequence
+                const bool diag = (i == kt);               // keys above the query are masked there
+#pragma unroll 1
+                for (int half = 0; half < 2; ++half) {
+                    float sx[64], dpx[64];
+                    tmem_ld32(tST + lane_addr + half * 64, sx);
+                    tmem_ld32(tST + lane_addr + half * 64 + 32, sx + 32);
+                    tmem_ld32(tDPT + lane_addr + half * 64, dpx);
+                    tmem_ld32(tDPT + lane_addr + half * 64 + 32, dpx + 32);
+                    tmem_wait_ld();
+                    uint32_t pp[32], gg[32];
+#pragma unroll
+                    for (int cc = 0; cc < 64; cc += 2) {
+                        float pv[2], gv[2];
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int col = half * 64 + cc + e;
+                            const float tt = fmaf(ps[0 * BT + col], sx[cc + e], fmaf(ps[1 * BT + col], gl, -ps[2 * BT + col]));
+                            const bool keep = col < col_lim && !(diag && col < r);
+                            const float p = keep ? ex2_approx(tt) : 0.f;
+                            const float G = p * (dpx[cc + e] - ps[3 * BT + col]) * ps[4 * BT + col];
+                            csum += G;
+                            pv[e] = p;
+                            gv[e] = G;
+                        }
+                        pp[cc / 2] = pack2_bf16(pv[0], pv[1]);
+                        gg[cc / 2] = pack2_bf16(gv[0], gv[1]);
+                    }
+                    // P^T and G^T over the (already read) first 64 columns of S^T and dP^T
+                    tmem_st32u(tST + lane_addr + half * 32, pp);
+                    tmem_st32u(tDPT + lane_addr + half * 32, gg);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar(D_PG_FULL));
+            }
+            if (ok && valid_key) colsum[static_cast<size_t>(seq0 + key_local) * Hq + h] = csum;
+        }
+        // ---------------------------------------------------------------- epilogue
+        if (ok) ok = mbar_wait_warp(bar(D_ACC_DONE), 0, abort_flag, status, TG_WHERE_SOFTMAX);
+        if (ok) {
+            tc_fence_after();
+            const size_t row = (static_cast<size_t>(seq0 + key_local) * Hkv + hk) * HD;
+#pragma unroll 1
+            for (int which = 0; which < 2; ++which) {
+                const uint32_t src = which ? tDK : tDV;
+                const float scale = which ? sm_scale : 1.0f;
+                uint16_t* dst = (which ? dk : dv) + row;
+#pragma unroll
+                for (int ch = 0; ch < HD / 32; ++ch) {
+                    float o[32];
+                    tmem_ld32(src + lane_addr + ch * 32, o);
+                    tmem_wait_ld();
+                    if (valid_key) {
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            uint4 w;
+                            w.x = pack2_bf16(o[q4 * 8 + 0] * scale, o[q4 * 8 + 1] * scale);
+                            w.y = pack2_bf16(o[q4 * 8 + 2] * scale, o[q4 * 8 + 3] * scale);
+                            w.z = pack2_bf16(o[q4 * 8 + 4] * scale, o[q4 * 8 + 5] * scale);
+                            w.w = pack2_bf16(o[q4 * 8 + 6] * scale, o[q4 * 8 + 7] * scale);
+                            *reinterpret_cast<uint4*>(dst + ch * 32 + q4 * 8) = w;
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 4) {
+        tc_fence_after();
+        tmem_dealloc(tmem, L::TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// dQ and the per-query sums: one CTA per (query head, 128-query tile, sequence),
+// heaviest causal tiles first.
+//
+// 192 threads: warps 0-3 compute (thread r = query row r = TMEM lane), warp 4
+// TMA producer (Q and dO once, K/V tiles through a two-stage ring), warp 5 MMA
+// issuer.  TMEM: S | dP | dQ.  Per KV tile j the issuer waits for G(j-1),
+// accumulates dQ += G(j-1) K(j-1) from TMEM and then issues S(j) = Q K(j)^T and
+// dP(j) = dO V(j)^T.  The compute warps rebuild P from the log-sum-exp, form
+// G = P (dP - D) / tau, store it as bf16 over the first 64 columns of S and sum,
+// along their own row, G gls (for dbeta) and dl l (for dtau).
+template <int HD>
+struct DqSmem {
+    static constexpr int TILE = BT * HD * 2;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_DO = OFF_Q + TILE;
+    static constexpr int OFF_K = OFF_DO + TILE;        // [2 stages]
+    static constexpr int OFF_V = OFF_K + 2 * TILE;     // [2 stages]
+    static constexpr int OFF_GLS = OFF_V + 2 * TILE;   // [4 warps][2][BT] fp32, a private copy per warp
+    static constexpr int OFF_BAR = OFF_GLS + 4 * 2 * BT * 4;
+    static constexpr int NUM_BARS = 16;
+    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+    static constexpr int BYTES = OFF_MISC + 16;
+    static constexpr int ALLOC = BYTES + 1024;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static_assert(ALLOC <= 227 * 1024, "shared memory");
+    static_assert(2 * BT + HD <= 512, "TMEM columns");
+};
+
+enum : int {
+    Q_QD_FULL = 0, Q_K_FULL = 1, Q_K_EMPTY = 3, Q_V_FULL = 5, Q_V_EMPTY = 7, Q_SDP_FULL = 9, Q_G_FULL = 10,
+    Q_DQ_DONE = 11, Q_DRAIN = 12
+};
+
+template <int HD>
+__global__ void __launch_bounds__(BWD_THREADS, 1)
+gated_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                         const int32_t* __restrict__ cu_kept, const int32_t* __restrict__ pos,
+                         const int32_t* __restrict__ rank, const float* __restrict__ gls,
+                         const float* __restrict__ g, const float* __restrict__ c, const float* __restrict__ lse,
+                         float* __restrict__ Drow, float sm_scale, int Hq, int Hkv, int n_qt_max,
+                         uint16_t* __restrict__ dq, float* __restrict__ rowE, float* __restrict__ rowT,
+                         int* __restrict__ status) {
+    using L = DqSmem<HD>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int h = blockIdx.x;
+    const int qt = n_qt_max - 1 - static_cast<int>(blockIdx.y);
+    const int b = blockIdx.z;
+    pdl_wait();  // global memory is read only from here on
+    pdl_trigger();
+    const int seq0 = cu_kept[b];
+    const int Mb = cu_kept[b + 1] - seq0;
+    if (qt * BT >= Mb) return;
+    const int n_kv = qt + 1;  // the diagonal tile is the last one
+    const int hk = h / (Hq / Hkv);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t sQ = sbase + L::OFF_Q, sDO = sbase + L::OFF_DO, sK = sbase + L::OFF_K, sV = sbase + L::OFF_V;
+    auto bar = [&](int i) { return sbase + L::OFF_BAR + 8u * static_cast<uint32_t>(i); };
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(Q_QD_FULL), 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar(Q_K_FULL + s), 1);
+            mbar_init(bar(Q_K_EMPTY + s), 1);
+            mbar_init(bar(Q_V_FULL + s), 1);
+            mbar_init(bar(Q_V_EMPTY + s), 1);
+        }
+        mbar_init(bar(Q_SDP_FULL), 1);
+        mbar_init(bar(Q_G_FULL), 128);
+        mbar_init(bar(Q_DQ_DONE), 1);
+        mbar_init(bar(Q_DRAIN), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 4) {
+        tmem_alloc(smem_u32(tmem_slot), L::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tS = tmem, tDP = tmem + BT, tDQ = tmem + 2 * BT;
+
+    if (warp == 4) {
+        // ---------------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            prefetch_tmap(&tmQ);
+            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmV);
+            prefetch_tmap(&tmDO);
+            mbar_expect_tx(bar(Q_QD_FULL), 2 * L::TILE);
+#pragma unroll
+            for (int hf = 0; hf < HD / 64; ++hf) {
+                tma_load_2d(sQ + hf * BT * 128, &tmQ, h * HD + hf * 64, seq0 + qt * BT, bar(Q_QD_FULL));
+                tma_load_2d(sDO + hf * BT * 128, &tmDO, h * HD + hf * 64, seq0 + qt * BT, bar(Q_QD_FULL));
+            }
+            int k_issued[2] = {0, 0}, v_issued[2] = {0, 0};
+            for (int j = 0; j < n_kv; ++j) {
+                const int s = j & 1;
+                if (j >= 2 && !mbar_wait(bar(Q_K_EMPTY + s), ((j - 2) >> 1) & 1, abort_flag, status,
+                                         TG_WHERE_PRODUCER))
+                    break;
+                mbar_expect_tx(bar(Q_K_FULL + s), L::TILE);
+#pragma unroll
+                for (int hf = 0; hf < HD / 64; ++hf)
+                    tma_load_2d(sK + s * L::TILE + hf * BT * 128, &tmK, hk * HD + hf * 64, seq0 + j * BT,
+                                bar(Q_K_FULL + s));
+                ++k_issued[s];
+                if (j >= 2 && !mbar_wait(bar(Q_V_EMPTY + s), ((j - 2) >> 1) & 1, abort_flag, status,
+                                         TG_WHERE_PRODUCER))
+                    break;
+                mbar_expect_tx(bar(Q_V_FULL + s), L::TILE);
+#pragma unroll
+                for (int hf = 0; hf < HD / 64; ++hf)
+                    tma_load_2d(sV + s * L::TILE + hf * BT * 128, &tmV, hk * HD + hf * 64, seq0 + j * BT,
+                                bar(Q_V_FULL + s));
+                ++v_issued[s];
+            }
+            if (*abort_flag) {
+                drain_wait_b(bar(Q_QD_FULL), 0, status);
+                for (int s = 0; s < 2; ++s) {
+                    if (k_issued[s]) drain_wait_b(bar(Q_K_FULL + s), (k_issued[s] - 1) & 1, status);
+                    if (v_issued[s]) drain_wait_b(bar(Q_V_FULL + s), (v_issued[s] - 1) & 1, status);
+                }
+            }
+        }
+    } else if (warp == 5) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = idesc_bf16_f32(BT, BT, false);
+            constexpr uint32_t idesc_acc = idesc_bf16_f32(BT, HD, true);
+            // dQ += G(jj) K(jj): A from TMEM (16 keys = 8 columns per k-step), B the K tile MN-major
+            auto issue_dq = [&](int jj) {
+                const int s = jj & 1;
+#pragma unroll
+                for (int kk = 0; kk < BT / 16; ++kk)
+                    mma_bf16_ts(tDQ, tS + kk * 8, smem_desc_sw128(sK + s * L::TILE + kk * 16 * 128, BT * 128, 1024),
+                                idesc_acc, (jj > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(bar(Q_K_EMPTY + s));
+            };
+            bool ok = mbar_wait(bar(Q_QD_FULL), 0, abort_flag, status, TG_WHERE_MMA);
+            for (int j = 0; ok && j < n_kv; ++j) {
+                const int s = j & 1;
+                ok = mbar_wait(bar(Q_K_FULL + s), (j >> 1) & 1, abort_flag, status, TG_WHERE_MMA);
+                if (ok) ok = mbar_wait(bar(Q_V_FULL + s), (j >> 1) & 1, abort_flag, status, TG_WHERE_MMA);
+                if (ok && j >= 1) ok = mbar_wait(bar(Q_G_FULL), (j - 1) & 1, abort_flag, status, TG_WHERE_MMA);
+                if (!ok) break;
+                tc_fence_after();
+                if (j >= 1) issue_dq(j - 1);
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * (BT * 128) + (kk & 3) * 32;
+                    mma_bf16_ss(tS, smem_desc_sw128(sQ + off, 16, 1024),
+                                smem_desc_sw128(sK + s * L::TILE + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * (BT * 128) + (kk & 3) * 32;
+                    mma_bf16_ss(tDP, smem_desc_sw128(sDO + off, 16, 1024),
+                                smem_desc_sw128(sV + s * L::TILE + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(bar(Q_SDP_FULL));
+                mma_commit(bar(Q_V_EMPTY + s));
+            }
+            if (ok) ok = mbar_wait(bar(Q_G_FULL), (n_kv - 1) & 1, abort_flag, status, TG_WHERE_MMA);
+            if (ok) {
+                tc_fence_after();
+                issue_dq(n_kv - 1);
+                mma_commit(bar(Q_DQ_DONE));
+            }
+            mma_commit(bar(Q_DRAIN));
+            drain_wait_b(bar(Q_DRAIN), 0, status);
+        }
+    } else {
+        // ---------------------------------------------------------------- compute warps 0-3
+        const int r = threadIdx.x;  // query row of the tile == TMEM lane
+        const int q_local = qt * BT + r;
+        const bool valid_row = q_local < Mb;
+        const int qg = seq0 + q_local;
+        const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+        float fa = 0.f, fb = 0.f, fl = 0.f, fd = 0.f, fi = 0.f;
+        if (valid_row) {
+            fi = 1.0f / (1.0f + c[h] * logf(static_cast<float>(pos[qg]) / static_cast<float>(rank[qg])));
+            fa = sm_scale * LOG2E_B * fi;
+            fb = softplus_b(g[h]) * LOG2E_B * fi;
+            fl = lse[static_cast<size_t>(qg) * Hq + h] * LOG2E_B;
+            fd = Drow[static_cast<size_t>(qg) * Hq + h];
+        }
+        float* wgls = reinterpret_cast<float*>(smem + L::OFF_GLS) + warp * (2 * BT);
+        // Row sums for dbeta and dtau, formed with the row's exact D' = sum_j P dP (the
+        // D above comes from the bf16 output; dtau = -sum_j dl l / tau cancels to a small
+        // number and would amplify its rounding):  sum_j dl x = sum P dP x - D' sum P x.
+        float aPdPt = 0.f, aPt = 0.f, aPdP = 0.f, aP = 0.f, aPdPg = 0.f, aPg = 0.f;
+        bool ok = true;
+        for (int j = 0; j < n_kv; ++j) {
+            const int s = j & 1;
+            // the tile's gls into this warp's own copy (only __syncwarp orders it)
+#pragma unroll
+            for (int e = 0; e < BT / 32; ++e) {
+                const int key_local = j * BT + e * 32 + lane;
+                wgls[s * BT + e * 32 + lane] = key_local < Mb ? gls[seq0 + key_local] : 0.f;
+            }
+            __syncwarp();
+            ok = mbar_wait_warp(bar(Q_SDP_FULL), j & 1, abort_flag, status, TG_WHERE_SOFTMAX);
+            if (!ok) break;
+            tc_fence_after();
+            const bool diag = (j == n_kv - 1);
+            const int lim = q_local - j * BT;  // on the diagonal tile, columns > lim are future keys
+            const float* bl = wgls + s * BT;
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                float sx[64], dpx[64];
+                tmem_ld32(tS + lane_addr + half * 64, sx);
+                tmem_ld32(tS + lane_addr + half * 64 + 32, sx + 32);
+                tmem_ld32(tDP + lane_addr + half * 64, dpx);
+                tmem_ld32(tDP + lane_addr + half * 64 + 32, dpx + 32);
+                tmem_wait_ld();
+                uint32_t gg[32];
+#pragma unroll
+                for (int cc = 0; cc < 64; cc += 2) {
+                    float gv[2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int col = half * 64 + cc + e;
+                        const float glj = bl[col];
+                        const float tt = fmaf(fa, sx[cc + e], fmaf(fb, glj, -fl));
+                        const bool keep = valid_row && !(diag && col > lim);
+                        const float p = keep ? ex2_approx(tt) : 0.f;
+                        const float G = p * (dpx[cc + e] - fd) * fi;
+                        if (p > 0.f) {
+                            const float pdp = p * dpx[cc + e];
+                            aPdPt = fmaf(pdp, tt, aPdPt);
+                            aPt = fmaf(p, tt, aPt);
+                            aPdP += pdp;
+                            aP += p;
+                            aPdPg = fmaf(pdp, glj, aPdPg);
+                            aPg = fmaf(p, glj, aPg);
+                        }
+                        gv[e] = G;
+                    }
+                    gg[cc / 2] = pack2_bf16(gv[0], gv[1]);
+                }
+                tmem_st32u(tS + lane_addr + half * 32, gg);  // G over the (already read) first columns of S
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(Q_G_FULL));
+        }
+        // ---------------------------------------------------------------- epilogue
+        if (ok) ok = mbar_wait_warp(bar(Q_DQ_DONE), 0, abort_flag, status, TG_WHERE_SOFTMAX);
+        if (ok) {
+            tc_fence_after();
+            uint16_t* dst = dq + (static_cast<size_t>(qg) * Hq + h) * HD;
+#pragma unroll
+            for (int ch = 0; ch < HD / 32; ++ch) {
+                float o[32];
+                tmem_ld32(tDQ + lane_addr + ch * 32, o);
+                tmem_wait_ld();
+                if (valid_row) {
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        uint4 w;
+                        w.x = pack2_bf16(o[q4 * 8 + 0] * sm_scale, o[q4 * 8 + 1] * sm_scale);
+                        w.y = pack2_bf16(o[q4 * 8 + 2] * sm_scale, o[q4 * 8 + 3] * sm_scale);
+                        w.z = pack2_bf16(o[q4 * 8 + 4] * sm_scale, o[q4 * 8 + 5] * sm_scale);
+                        w.w = pack2_bf16(o[q4 * 8 + 6] * sm_scale, o[q4 * 8 + 7] * sm_scale);
+                        *reinterpret_cast<uint4*>(dst + ch * 32 + q4 * 8) = w;
+                    }
+                }
+            }
+            if (valid_row) {
+                const float Dx = aPdP;
+                // tt = l log2(e) - lse log2(e):  sum dl l = ln2 (sum dl tt + lse log2(e) sum dl)
+                const float sum_dl_t = aPdPt - Dx * aPt + fl * (aPdP - Dx * aP);
+                rowE[static_cast<size_t>(qg) * Hq + h] = fi * (aPdPg - Dx * aPg);  // sum_j G gls_j
+                rowT[static_cast<size_t>(qg) * Hq + h] = -LN2_B * fi * sum_dl_t;   // dtau of the row
+                Drow[static_cast<size_t>(qg) * Hq + h] = Dx;  // the exact D' for the dK/dV kernel
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 4) {
+        tc_fence_after();
+        tmem_dealloc(tmem, L::TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Per key: dgls_j = sum_h softplus(g_h) colsum[j, h]; d score_j = dgls_j (1 - exp(gls_j)).
+__global__ void __launch_bounds__(256)
+bwd_keys_kernel(const float* __restrict__ colsum, const float* __restrict__ gls, const float* __restrict__ g,
+                int64_t M, int Hq, float* __restrict__ dgls, float* __restrict__ dscore) {
+    pdl_wait();
+    pdl_trigger();
+    for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < M;
+         j += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        float acc = 0.f;
+        for (int h = 0; h < Hq; ++h) acc = fmaf(softplus_b(g[h]), colsum[j * Hq + h], acc);
+        dgls[j] = acc;
+        if (dscore) dscore[j] = acc * -expm1f(gls[j]);
+    }
+}
+
+// Per head (one block each): dg_h = sigmoid(g_h) sum_i rowE[i, h];
+// dc_h = sum_i ln(pos_i / rank_i) rowT[i, h].  Fixed summation order.
+__global__ void __launch_bounds__(256)
+bwd_heads_kernel(const float* __restrict__ rowE, const float* __restrict__ rowT, const int32_t* __restrict__ pos,
+                 const int32_t* __restrict__ rank, const float* __restrict__ g, int64_t M, int Hq,
+                 float* __restrict__ dg, float* __restrict__ dc) {
+    pdl_wait();
+    pdl_trigger();
+    __shared__ float sE[256], sT[256];
+    const int h = blockIdx.x;
+    float e = 0.f, t = 0.f;
+    for (int64_t i = threadIdx.x; i < M; i += blockDim.x) {
+        e += rowE[i * Hq + h];
+        t = fmaf(logf(static_cast<float>(pos[i]) / static_cast<float>(rank[i])), rowT[i * Hq + h], t);
+    }
+    sE[threadIdx.x] = e;
+    sT[threadIdx.x] = t;
+    __syncthreads();
+    for (int w = 128; w > 0; w >>= 1) {
+        if (threadIdx.x < w) {
+            sE[threadIdx.x] += sE[threadIdx.x + w];
+            sT[threadIdx.x] += sT[threadIdx.x + w];
+        }
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        dg[h] = sE[0] / (1.0f + expf(-g[h]));
+        dc[h] = sT[0];
+    }
+}
+
+template <int HD>
+cudaError_t launch_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* out,
+                       const uint16_t* dout, const float* lse, const int32_t* cu_kept, int B, int64_t M_total,
+                       int max_M, int Hq, int Hkv, const int32_t* pos, const int32_t* rank, const float* gls,
+                       const float* g, const float* c, float sm_scale, uint16_t* dq, uint16_t* dk, uint16_t* dv,
+                       float* dgls, float* dscore, float* dg, float* dc, void* ws, cudaStream_t st) {
+    static std::atomic<uint64_t> set_dkv{0}, set_dq{0};
+    if (cudaError_t e = ensure_smem_limit(gated_attn_bwd_dkv_kernel<HD>, DkvSmem<HD>::ALLOC, set_dkv);
+        e != cudaSuccess)
+        return e;
+    if (cudaError_t e = ensure_smem_limit(gated_attn_bwd_dq_kernel<HD>, DqSmem<HD>::ALLOC, set_dq); e != cudaSuccess)
+        return e;
+    const size_t rows = static_cast<size_t>(M_total) * Hq;
+    float* Drow = static_cast<float*>(ws);
+    float* colsum = Drow + rows;
+    float* rowE = colsum + rows;
+    float* rowT = rowE + rows;
+    CUtensorMap tq, tk, tv, tdo;
+    if (!encode_tmap_2d_bf16(&tq, q, static_cast<uint64_t>(Hq) * HD, static_cast<uint64_t>(M_total),
+                             static_cast<uint64_t>(Hq) * HD * 2, 64, BT) ||
+        !encode_tmap_2d_bf16(&tdo, dout, static_cast<uint64_t>(Hq) * HD, static_cast<uint64_t>(M_total),
+                             static_cast<uint64_t>(Hq) * HD * 2, 64, BT) ||
+        !encode_tmap_2d_bf16(&tk, k, static_cast<uint64_t>(Hkv) * HD, static_cast<uint64_t>(M_total),
+                             static_cast<uint64_t>(Hkv) * HD * 2, 64, BT) ||
+        !encode_tmap_2d_bf16(&tv, v, static_cast<uint64_t>(Hkv) * HD, static_cast<uint64_t>(M_total),
+                             static_cast<uint64_t>(Hkv) * HD * 2, 64, BT))
+        return cudaErrorInvalidValue;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int* status = device_status_ptr();
+    const int64_t rd_blocks = (static_cast<int64_t>(rows) + 7) / 8;
+    cudaError_t e = launch_pdl(bwd_rowdot_kernel, dim3(static_cast<unsigned>(rd_blocks < sms * 8 ? rd_blocks : sms * 8)),
+                               dim3(256), 0, st, out, dout, static_cast<int64_t>(rows), HD, Drow);
+    if (e != cudaSuccess) return e;
+    const int n_t = (max_M + BT - 1) / BT;
+    // dq first: it replaces each row's D by the exact sum_j P dP, which the dK/dV kernel then uses
+    e = launch_pdl(gated_attn_bwd_dq_kernel<HD>, dim3(Hq, n_t, B), dim3(BWD_THREADS),
+                   static_cast<size_t>(DqSmem<HD>::ALLOC), st, tq, tk, tv, tdo, cu_kept, pos, rank, gls, g, c, lse,
+                   Drow, sm_scale, Hq, Hkv, n_t, dq, rowE, rowT, status);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(gated_attn_bwd_dkv_kernel<HD>, dim3(Hkv, n_t, B), dim3(BWD_THREADS),
+                   static_cast<size_t>(DkvSmem<HD>::ALLOC), st, tq, tk, tv, tdo, cu_kept, pos, rank, gls, g, c, lse,
+                   static_cast<const float*>(Drow), sm_scale, Hq, Hkv, dk, dv, colsum, status);
+    if (e != cudaSuccess) return e;
+    const int64_t kb = (M_total + 255) / 256;
+    e = launch_pdl(bwd_keys_kernel, dim3(static_cast<unsigned>(kb < sms * 4 ? kb : sms * 4)), dim3(256), 0, st,
+                   static_cast<const float*>(colsum), gls, g, M_total, Hq, dgls, dscore);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(bwd_heads_kernel, dim3(Hq), dim3(256), 0, st, static_cast<const float*>(rowE),
+                      static_cast<const float*>(rowT), pos, rank, g, M_total, Hq, dg, dc);
+}
+
+}  // namespace
+
+size_t attention_backward_workspace_bytes(int64_t M_total, int Hq) {
+    return static_cast<size_t>(4) * static_cast<size_t>(M_total) * static_cast<size_t>(Hq) * sizeof(float);
+}
+
+cudaError_t launch_gated_attention_backward(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                            const uint16_t* out, const uint16_t* dout, const float* lse,
+                                            const int32_t* cu_kept, int B, int64_t M_total, int max_M, int Hq,
+                                            int Hkv, int d, const int32_t* pos, const int32_t* rank,
+                                            const float* gls, const float* g, const float* c, float sm_scale,
+                                            uint16_t* dq, uint16_t* dk, uint16_t* dv, float* dgls, float* dscore,
+                                            float* dg, float* dc, void* ws, cudaStream_t st) {
+    if (d == 64)
+        return launch_bwd<64>(q, k, v, out, dout, lse, cu_kept, B, M_total, max_M, Hq, Hkv, pos, rank, gls, g, c,
+                              sm_scale, dq, dk, dv, dgls, dscore, dg, dc, ws, st);
+    return launch_bwd<128>(q, k, v, out, dout, lse, cu_kept, B, M_total, max_M, Hq, Hkv, pos, rank, gls, g, c,
+                           sm_scale, dq, dk, dv, dgls, dscore, dg, dc, ws, st);
+}
+
+}  // namespace tg

@@ -219,7 +219,7 @@ tg_status tg_masked_gated_attention(const uint16_t* q, const uint16_t* k, const 
 }
 
 
-int tg_abi_version(void) { return 3; }
+int tg_abi_version(void) { return 4; }
 
 const char* tg_last_error_string(void) { return g_last_error.c_str(); }
 
@@ -369,6 +369,40 @@ tg_status tg_gated_attention_gates(const uint16_t* q, const uint16_t* k, const u
     }
     return do_attention(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, d, pos, rank, gates, c, sm_scale, out, lse, ws,
                         ws_bytes, stream);
+}
+
+size_t tg_gated_attention_backward_workspace_size(int64_t M_total, int Hq) {
+    if (M_total <= 0 || Hq <= 0) return 0;
+    return tg::attention_backward_workspace_bytes(M_total, Hq);
+}
+
+tg_status tg_gated_attention_backward(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* out,
+                                      const uint16_t* dout, const float* lse, const int32_t* cu_kept, int B,
+                                      int64_t M_total, int max_M, int Hq, int Hkv, int d, const int32_t* pos,
+                                      const int32_t* rank, const float* gls, const float* g, const float* c,
+                                      float sm_scale, uint16_t* dq, uint16_t* dk, uint16_t* dv, float* dgls,
+                                      float* dscore, float* dg, float* dc, void* ws, size_t ws_bytes,
+                                      tg_stream_t stream) {
+    TG_REQUIRE(B >= 0 && M_total >= 0 && max_M >= 0, "negative size");
+    if (tg_status s = check_attn_shape(Hq, Hkv, d)) return s;
+    TG_SUPPORT(d == 64 || d == 128, "the backward supports head_dim 64 and 128, not %d", d);
+    TG_REQUIRE(sm_scale > 0.f, "sm_scale must be positive");
+    if (B == 0 || M_total == 0) return TG_OK;
+    TG_REQUIRE(max_M > 0, "max_M must bound the longest sequence");
+    TG_REQUIRE(q && k && v && out && dout && lse && cu_kept && pos && rank && gls && g && c && dq && dk && dv &&
+                   dgls && dg && dc && ws,
+               "null pointer argument");
+    TG_REQUIRE(aligned16(q) && aligned16(k) && aligned16(v) && aligned16(out) && aligned16(dout) && aligned16(dq) &&
+                   aligned16(dk) && aligned16(dv),
+               "q, k, v, out, dout, dq, dk and dv must be 16-byte aligned");
+    TG_REQUIRE((reinterpret_cast<uintptr_t>(ws) & 255u) == 0, "ws must be 256-byte aligned");
+    const size_t need = tg::attention_backward_workspace_bytes(M_total, Hq);
+    TG_REQUIRE(ws_bytes >= need, "ws holds %zu bytes, the backward needs %zu", ws_bytes, need);
+    if (tg_status s = check_device()) return s;
+    return cuda_status(tg::launch_gated_attention_backward(q, k, v, out, dout, lse, cu_kept, B, M_total, max_M, Hq,
+                                                           Hkv, d, pos, rank, gls, g, c, sm_scale, dq, dk, dv, dgls,
+                                                           dscore, dg, dc, ws, stream),
+                       "tg_gated_attention_backward launch");
 }
 
 tg_status tg_next_gate_span(const int32_t* h_span, const int32_t* h_k, int B, int32_t* h_span_next) {

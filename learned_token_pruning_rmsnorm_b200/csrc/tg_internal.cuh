@@ -135,6 +135,17 @@ cudaError_t launch_gated_attention_noalloc(const uint16_t* q, const uint16_t* k,
                                            const float* c, float sm_scale, uint16_t* out, float* lse,
                                            cudaStream_t st);
 size_t attention_workspace_bytes(int B, int max_M, int Hq, int Hkv, int d);
+
+// Backward of the one-gate attention (head_dim 64 or 128); ws holds
+// attention_backward_workspace_bytes(M_total, Hq) bytes (4 fp32 per row and head).
+size_t attention_backward_workspace_bytes(int64_t M_total, int Hq);
+cudaError_t launch_gated_attention_backward(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                            const uint16_t* out, const uint16_t* dout, const float* lse,
+                                            const int32_t* cu_kept, int B, int64_t M_total, int max_M, int Hq,
+                                            int Hkv, int d, const int32_t* pos, const int32_t* rank,
+                                            const float* gls, const float* g, const float* c, float sm_scale,
+                                            uint16_t* dq, uint16_t* dk, uint16_t* dv, float* dgls, float* dscore,
+                                            float* dg, float* dc, void* ws, cudaStream_t st);
 int64_t units_below_host(int x, int C);
 
 cudaError_t launch_selftest_wait(int64_t timeout_ns, cudaStream_t st);
