@@ -363,6 +363,27 @@ def measure_next_rows(tg, dev, st, flush, main, peaks, reps=10):
     res["f4_four_gates_attention"] = {"workload": f"{wm.name}: M={main['M']}, 4 gates", "us": us,
                                       "tflops": fl / (us * 1e-6) / 1e12, "one_gate_us": us1,
                                       "vs_one_gate": us / us1}
+    # f1 (training): backward of the gated attention on the main workload, from the
+    # forward's output and log-sum-exp
+    lse = torch.empty((main["M"], wm.Hq), dtype=torch.float32, device=dev)
+    assert lib.tg_gated_attention(*common, bufs.gls.data_ptr(), L0["g"].data_ptr(), L0["c"].data_ptr(), sm,
+                                  out.data_ptr(), lse.data_ptr(), ws_p, ws_n, sh) == 0
+    dout = torch.randn((main["M"], wm.Hq, wm.d), device=dev).to(torch.bfloat16)
+    grads = [torch.empty_like(L0["q"]), torch.empty_like(L0["k"]), torch.empty_like(L0["v"])]
+    f32 = [torch.empty(main["M"], dtype=torch.float32, device=dev) for _ in range(2)] + \
+          [torch.empty(wm.Hq, dtype=torch.float32, device=dev) for _ in range(2)]
+    nb = int(lib.tg_gated_attention_backward_workspace_size(main["M"], wm.Hq))
+    bws = torch.empty(nb, dtype=torch.uint8, device=dev)
+    us = time_device_us(check(lambda: lib.tg_gated_attention_backward(
+        L0["q"].data_ptr(), L0["k"].data_ptr(), L0["v"].data_ptr(), out.data_ptr(), dout.data_ptr(), lse.data_ptr(),
+        ck_d.data_ptr(), wm.B, main["M"], main["max_M"], wm.Hq, wm.Hkv, wm.d, bufs.pos.data_ptr(),
+        bufs.rank.data_ptr(), bufs.gls.data_ptr(), L0["g"].data_ptr(), L0["c"].data_ptr(), sm, grads[0].data_ptr(),
+        grads[1].data_ptr(), grads[2].data_ptr(), f32[0].data_ptr(), f32[1].data_ptr(), f32[2].data_ptr(),
+        f32[3].data_ptr(), bws.data_ptr(), bws.numel(), sh)), st, flush, reps)
+    res["f1_attention_backward"] = {"workload": f"{wm.name}: M={main['M']}, Hq={wm.Hq}, Hkv={wm.Hkv}, d={wm.d}",
+                                    "us": us, "tflops": 2.5 * fl / (us * 1e-6) / 1e12,
+                                    "frac_of_bf16_peak": 2.5 * fl / (us * 1e-6) / 1e12 / tc_peak,
+                                    "algorithmic": "2.5x the forward's 4*d*Hq per causal pair (five products)"}
     return res
 
 
