@@ -275,12 +275,15 @@ tg_status tg_gated_attention_noalloc(const uint16_t* q, const uint16_t* k, const
 /*
  * The whole gated prefill at one gate layer: tg_score, tg_select_topk (which
  * also writes the compaction map), the row gather of tg_compact and n_layers
- * gated-attention layers above the gate, with no host synchronisation.  The
- * row gather runs on a library-owned side stream, forked from and joined
- * back into `stream` by events (one pair per device, created on first use),
- * so that it overlaps the attention; everything the call enqueues is
- * ordered before work enqueued on `stream` afterwards, and the call may be
- * captured into a CUDA graph.  Fields mirror
+ * gated-attention layers above the gate, with no host synchronisation, all
+ * on `stream`.  The kernels are chained by programmatic dependent launch:
+ * each attention layer loads its q/k/v while the kernel before it runs, and
+ * the row gathers run last, overlapping the final attention wave.  This
+ * relies on q, k, v, g, c, hidden and cu_kept being complete before the call
+ * (written by work enqueued on `stream` earlier, or already synchronised),
+ * and on no other stream writing them while the call runs.  Everything the
+ * call enqueues is ordered before work enqueued on `stream` afterwards, and
+ * the call may be captured into a CUDA graph.  Fields mirror
  * the stage arguments above; per-layer tensors are arrays of n_layers
  * device pointers (the array itself lives in host memory).  The
  * projections that turn hidden_kept into each layer's q/k/v belong to the

@@ -101,11 +101,14 @@ __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity, int* s
 }
 
 // Global load that stays where it is written (volatile asm is not moved across the
-// other volatile asm statements), so that a prefetch issued a tile ahead is not
-// sunk by the compiler to its first use.
+// other volatile asm statements), so that a prefetch issued a tile ahead is not sunk by the
+// compiler to its first use.  It reads through L2 (.cg), not the read-only path: with
+// programmatic dependent launch the kernel that writes the compaction map may still be
+// running during this kernel's lifetime, and the non-coherent path then returned stale
+// values now and then.
 __device__ __forceinline__ float ldg_early(const float* p) {
     float v;
-    asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v) : "l"(p));
+    asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(v) : "l"(p));
     return v;
 }
 
@@ -311,7 +314,8 @@ gated_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         const bool valid_row = q_local < Mb;
         const int qg = seq0 + q_local;
         float inv_tau = 1.0f;
-        if (valid_row) inv_tau = 1.0f / (1.0f + c[h] * logf(static_cast<float>(pos[qg]) / static_cast<float>(rank[qg])));
+        if (valid_row)
+            inv_tau = 1.0f / (1.0f + c[h] * logf(static_cast<float>(__ldcg(pos + qg)) / static_cast<float>(__ldcg(rank + qg))));
         const float alpha = sm_scale * LOG2E * inv_tau;
         float gscale[kMaxGates];  // per gate: softplus(g_h) in log2 units (0 past the last gate)
 #pragma unroll
@@ -329,10 +333,10 @@ gated_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 const int key_local = j * BN + e * 32 + lane;
                 float bsum = 0.f;
                 if (key_local < Mb) {
-                    bsum = gscale[0] * gates.gls[0][seq0 + key_local];
+                    bsum = gscale[0] * __ldcg(gates.gls[0] + seq0 + key_local);
 #pragma unroll
                     for (int gi = 1; gi < kMaxGates; ++gi)
-                        if (gi < gates.n) bsum += gscale[gi] * gates.gls[gi][seq0 + key_local];
+                        if (gi < gates.n) bsum += gscale[gi] * __ldcg(gates.gls[gi] + seq0 + key_local);
                 }
                 wbias[s * BN + e * 32 + lane] = bsum;
             }
@@ -537,7 +541,7 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                        const int32_t* __restrict__ pos, const int32_t* __restrict__ rank, const GateSet gates,
                        const float* __restrict__ c, float sm_scale, int Hq, int Hkv, int n_qt_max, int kv_chunk,
                        SplitWs ws,
-                       uint16_t* __restrict__ out, float* __restrict__ lse, int* __restrict__ status) {
+                       uint16_t* __restrict__ out, float* __restrict__ lse, int* __restrict__ status, int early) {
     using L = G2Smem<HD>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -547,8 +551,15 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
 #ifdef TG_TRACE
     const unsigned long long trace_t0 = globaltimer();
 #endif
-    pdl_wait();  // global memory is read only from here on
-    pdl_trigger();
+    // `early`: q, k, v, g, c and cu_kept were complete before the preceding kernel started
+    // (the caller's guarantee), so the set-up, Q and the first K/V tiles go ahead while that
+    // kernel runs; only the compaction map (pos, rank, gls) and the split scratch wait for it,
+    // each role executing the wait before its first such access.  Otherwise every global
+    // access waits here.
+    if (!early) {
+        pdl_wait();
+        pdl_trigger();
+    }
     const int seq0 = cu_kept[b];
     const int Mb = cu_kept[b + 1] - seq0;
     const int n_qt = (Mb + BM - 1) / BM;
@@ -622,7 +633,7 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     if (threadIdx.x == 0) {
         mbar_init(bar(G_Q_FULL), 1);
         for (int s = 0; s < 2; ++s) {
-            mbar_init(bar(G_K_FULL + s), 1);
+            mbar_init(bar(G_K_FULL + s), 2);  // the K tile's bytes and the producer's K_ext rows
             mbar_init(bar(G_K_EMPTY + s), 1);
             mbar_init(bar(G_V_FULL + s), 1);
             mbar_init(bar(G_V_EMPTY + s), 1);
@@ -661,6 +672,37 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                                 seq0 + qt * BM, bar(G_Q_FULL));
         }
         int k_issued[2] = {0, 0}, v_issued[2] = {0, 0};
+        auto issue_k = [&](int j) {
+            const int s = j & 1;
+            mbar_expect_tx(bar(G_K_FULL + s), BN * HD * 2);
+#pragma unroll
+            for (int hf = 0; hf < HD / 64; ++hf)
+                tma_load_2d(sK0 + s * L::TILE_KV + hf * BN * 128, &tmK, hk * HD + hf * 64, seq0 + (kv0 + j) * BN,
+                            bar(G_K_FULL + s));
+            ++k_issued[s];
+        };
+        auto issue_v = [&](int j) {
+            const int s = j & 1;
+            mbar_expect_tx(bar(G_V_FULL + s), BN * HD * 2);
+#pragma unroll
+            for (int hf = 0; hf < HD / 64; ++hf)
+                tma_load_2d(sV0 + s * L::TILE_KV + hf * BN * 128, &tmV, hk * HD + hf * 64, seq0 + (kv0 + j) * BN,
+                            bar(G_V_FULL + s));
+            ++v_issued[s];
+        };
+        // tiles whose K and V copies leave before the compaction map is available
+        const int pre = early ? min(n_kv, 2) : 0;
+        if (lane == 0)
+            for (int j = 0; j < pre; ++j) {
+                issue_k(j);
+                issue_v(j);
+            }
+        if (early) {
+            pdl_wait();  // gls (the compaction map) is read from here on
+            // dependents are released only now, once the preceding kernel has completed, so
+            // a following row gather may read the compaction map straight away
+            if (lane == 0) pdl_trigger();
+        }
         float gk[4];  // first gate's gls of this lane's keys of the next tile (0 past the end)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -682,6 +724,7 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             if (j >= 2 && !mbar_wait_warp(bar(G_K_EMPTY + s), ((j - 2) >> 1) & 1, abort_flag, status,
                                           TG_WHERE_PRODUCER))
                 break;
+            if (lane == 0 && j >= pre) issue_k(j);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int r = lane * 4 + i;
@@ -701,32 +744,18 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int r = lane * 4 + i;
-                    const uint32_t hl = bf16_hi_lo(r < valid ? gsrc[r] : 0.f);
+                    const uint32_t hl = bf16_hi_lo(r < valid ? __ldcg(gsrc + r) : 0.f);
                     *reinterpret_cast<uint2*>(kx + (r >> 3) * 256 + (gi >> 1) * 128 + (r & 7) * 16 + (gi & 1) * 8) =
                         make_uint2(__byte_perm(hl, 0u, 0x1010), __byte_perm(hl, 0u, 0x3232));
                 }
             }
             fence_proxy_async_smem();  // K_ext is read by the tensor core (async proxy)
             __syncwarp();
-            if (lane == 0) {
-                mbar_expect_tx(bar(G_K_FULL + s), BN * HD * 2);
-#pragma unroll
-                for (int hf = 0; hf < HD / 64; ++hf)
-                    tma_load_2d(sK0 + s * L::TILE_KV + hf * BN * 128, &tmK, hk * HD + hf * 64,
-                                seq0 + (kv0 + j) * BN, bar(G_K_FULL + s));
-                ++k_issued[s];
-            }
+            if (lane == 0) mbar_arrive(bar(G_K_FULL + s));  // the K_ext half of the stage
             if (j >= 2 && !mbar_wait_warp(bar(G_V_EMPTY + s), ((j - 2) >> 1) & 1, abort_flag, status,
                                           TG_WHERE_PRODUCER))
                 break;
-            if (lane == 0) {
-                mbar_expect_tx(bar(G_V_FULL + s), BN * HD * 2);
-#pragma unroll
-                for (int hf = 0; hf < HD / 64; ++hf)
-                    tma_load_2d(sV0 + s * L::TILE_KV + hf * BN * 128, &tmV, hk * HD + hf * 64,
-                                seq0 + (kv0 + j) * BN, bar(G_V_FULL + s));
-                ++v_issued[s];
-            }
+            if (lane == 0 && j >= pre) issue_v(j);
         }
         if (lane == 0 && *abort_flag) {
             drain_wait(bar(G_Q_FULL), 0, status);
@@ -829,7 +858,10 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         const int q_local = qt * BM + r;
         const bool valid_row = q_local < Mb;
         const int qg = seq0 + q_local;
-        const float ratio_log = valid_row ? logf(static_cast<float>(pos[qg]) / static_cast<float>(rank[qg])) : 0.f;
+        if (early) pdl_wait();  // pos and rank (the compaction map) and the split scratch from here on
+        // (through L2, as ldg_early, since their writer may have run during this kernel's lifetime)
+        const float ratio_log =
+            valid_row ? logf(static_cast<float>(__ldcg(pos + qg)) / static_cast<float>(__ldcg(rank + qg))) : 0.f;
         // per-head values are scalars selected by the head index (no local-memory arrays)
         const float inv_tau0 = valid_row ? 1.0f / (1.0f + c[2 * pair] * ratio_log) : 1.0f;
         const float inv_tau1 = valid_row ? 1.0f / (1.0f + c[2 * pair + 1] * ratio_log) : 1.0f;
@@ -1145,7 +1177,7 @@ template <int HD>
 cudaError_t launch_gqa2(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const int32_t* cu_kept,
                         int B, int max_M, int Hq, int Hkv, const int32_t* pos, const int32_t* rank,
                         const GateSet& gates, const float* c, float sm_scale, uint16_t* out, float* lse, void* ws,
-                        size_t ws_bytes, cudaStream_t st) {
+                        size_t ws_bytes, bool early, cudaStream_t st) {
     using L = G2Smem<HD>;
     static std::atomic<uint64_t> attr_set{0};
     if (cudaError_t e = ensure_smem_limit(gated_attn_gqa2_kernel<HD>, L::ALLOC, attr_set); e != cudaSuccess)
@@ -1170,14 +1202,14 @@ cudaError_t launch_gqa2(const CUtensorMap& tq, const CUtensorMap& tk, const CUte
     dim3 grid(Hq / 2, static_cast<unsigned>(units), B);
     return launch_pdl(gated_attn_gqa2_kernel<HD>, grid, dim3(G2_THREADS), static_cast<size_t>(L::ALLOC), st, tq, tk,
                       tv, cu_kept, pos, rank, gates, c, sm_scale, Hq, Hkv, n_qt_max, C, sw, out, lse,
-                      device_status_ptr());
+                      device_status_ptr(), early ? 1 : 0);
 }
 
 template <int HD>
 cudaError_t launch_tc(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* cu_kept, int B,
                       int64_t M_total, int max_M, int Hq, int Hkv, const int32_t* pos, const int32_t* rank,
                       const GateSet& gates, const float* c, float sm_scale, uint16_t* out, float* lse, void* ws,
-                      size_t ws_bytes, cudaStream_t st) {
+                      size_t ws_bytes, bool early, cudaStream_t st) {
     using L = AttnSmem<HD>;
     static std::atomic<uint64_t> attr_set{0};
     if (cudaError_t e = ensure_smem_limit(gated_attn_tc_kernel<HD>, L::ALLOC, attr_set); e != cudaSuccess)
@@ -1193,7 +1225,7 @@ cudaError_t launch_tc(const uint16_t* q, const uint16_t* k, const uint16_t* v, c
     if constexpr (HD <= 128) {  // two heads of 256 would need 768 TMEM columns
         if ((Hq / Hkv) % 2 == 0)
             return launch_gqa2<HD>(tq, tk, tv, cu_kept, B, max_M, Hq, Hkv, pos, rank, gates, c, sm_scale, out, lse,
-                                   ws, ws_bytes, st);
+                                   ws, ws_bytes, early, st);
     }
     int* status = device_status_ptr();
     const int n_qt_max = (max_M + BM - 1) / BM;
@@ -1216,17 +1248,18 @@ extern "C" int tg_trace_read_attention_ctas(unsigned long long* host) {
 cudaError_t launch_gated_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* cu_kept,
                                    int B, int64_t M_total, int max_M, int Hq, int Hkv, int d, const int32_t* pos,
                                    const int32_t* rank, const GateSet& gates, const float* c, float sm_scale,
-                                   uint16_t* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t st) {
+                                   uint16_t* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t st,
+                                   bool inputs_ready) {
     if (M_total == 0 || B == 0) return cudaSuccess;
     if (gates.n < 1 || gates.n > kMaxGates) return cudaErrorInvalidValue;
     if (d == 64)
         return launch_tc<64>(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, pos, rank, gates, c, sm_scale, out, lse,
-                             ws, ws_bytes, st);
+                             ws, ws_bytes, inputs_ready, st);
     if (d == 256)
         return launch_tc<256>(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, pos, rank, gates, c, sm_scale, out, lse,
-                              ws, ws_bytes, st);
+                              ws, ws_bytes, inputs_ready, st);
     return launch_tc<128>(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, pos, rank, gates, c, sm_scale, out, lse, ws,
-                          ws_bytes, st);
+                          ws_bytes, inputs_ready, st);
 }
 
 int64_t units_below_host(int x, int C) {

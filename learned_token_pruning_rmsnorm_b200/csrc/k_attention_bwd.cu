@@ -257,7 +257,7 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
         const int key_local = kt * BT + r;
         const bool valid_key = key_local < Mb;
         const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
-        const float gl = valid_key ? gls[seq0 + key_local] : 0.f;
+        const float gl = valid_key ? __ldcg(gls + seq0 + key_local) : 0.f;
         float* par = reinterpret_cast<float*>(smem + L::OFF_PAR);
         bool ok = true;
         int t = 0;
@@ -272,11 +272,12 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
                 float fa = 0.f, fb = 0.f, fl = 0.f, fd = 0.f, fi = 0.f;
                 if (qrow < Mb) {
                     const int qg = seq0 + qrow;
-                    fi = 1.0f / (1.0f + c[h] * logf(static_cast<float>(pos[qg]) / static_cast<float>(rank[qg])));
+                    fi = 1.0f / (1.0f + c[h] * logf(static_cast<float>(__ldcg(pos + qg)) /
+                                                    static_cast<float>(__ldcg(rank + qg))));
                     fa = sm_scale * LOG2E_B * fi;
                     fb = beta * LOG2E_B * fi;
                     fl = lse[static_cast<size_t>(qg) * Hq + h] * LOG2E_B;
-                    fd = Drow[static_cast<size_t>(qg) * Hq + h];
+                    fd = __ldcg(Drow + static_cast<size_t>(qg) * Hq + h);
                 }
                 float* ps = par + s * 5 * BT;
                 ps[0 * BT + r] = fa;
@@ -564,11 +565,11 @@ gated_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
         const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
         float fa = 0.f, fb = 0.f, fl = 0.f, fd = 0.f, fi = 0.f;
         if (valid_row) {
-            fi = 1.0f / (1.0f + c[h] * logf(static_cast<float>(pos[qg]) / static_cast<float>(rank[qg])));
+            fi = 1.0f / (1.0f + c[h] * logf(static_cast<float>(__ldcg(pos + qg)) / static_cast<float>(__ldcg(rank + qg))));
             fa = sm_scale * LOG2E_B * fi;
             fb = softplus_b(g[h]) * LOG2E_B * fi;
             fl = lse[static_cast<size_t>(qg) * Hq + h] * LOG2E_B;
-            fd = Drow[static_cast<size_t>(qg) * Hq + h];
+            fd = __ldcg(Drow + static_cast<size_t>(qg) * Hq + h);
         }
         float* wgls = reinterpret_cast<float*>(smem + L::OFF_GLS) + warp * (2 * BT);
         // Row sums for dbeta and dtau, formed with the row's exact D' = sum_j P dP (the
@@ -582,7 +583,7 @@ gated_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
 #pragma unroll
             for (int e = 0; e < BT / 32; ++e) {
                 const int key_local = j * BT + e * 32 + lane;
-                wgls[s * BT + e * 32 + lane] = key_local < Mb ? gls[seq0 + key_local] : 0.f;
+                wgls[s * BT + e * 32 + lane] = key_local < Mb ? __ldcg(gls + seq0 + key_local) : 0.f;
             }
             __syncwarp();
             ok = mbar_wait_warp(bar(Q_SDP_FULL), j & 1, abort_flag, status, TG_WHERE_SOFTMAX);
@@ -681,7 +682,7 @@ bwd_keys_kernel(const float* __restrict__ colsum, const float* __restrict__ gls,
     for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < M;
          j += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         float acc = 0.f;
-        for (int h = 0; h < Hq; ++h) acc = fmaf(softplus_b(g[h]), colsum[j * Hq + h], acc);
+        for (int h = 0; h < Hq; ++h) acc = fmaf(softplus_b(g[h]), __ldcg(colsum + j * Hq + h), acc);
         dgls[j] = acc;
         if (dscore) dscore[j] = acc * -expm1f(gls[j]);
     }
@@ -699,8 +700,8 @@ bwd_heads_kernel(const float* __restrict__ rowE, const float* __restrict__ rowT,
     const int h = blockIdx.x;
     float e = 0.f, t = 0.f;
     for (int64_t i = threadIdx.x; i < M; i += blockDim.x) {
-        e += rowE[i * Hq + h];
-        t = fmaf(logf(static_cast<float>(pos[i]) / static_cast<float>(rank[i])), rowT[i * Hq + h], t);
+        e += __ldcg(rowE + i * Hq + h);
+        t = fmaf(logf(static_cast<float>(pos[i]) / static_cast<float>(rank[i])), __ldcg(rowT + i * Hq + h), t);
     }
     sE[threadIdx.x] = e;
     sT[threadIdx.x] = t;

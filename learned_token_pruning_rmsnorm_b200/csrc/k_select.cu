@@ -157,7 +157,7 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
         uint32_t lmin = 0xFFFFFFFFu, lmax = 0u;
 #pragma unroll 8
         for (int64_t t = k0 + tid; t < k1; t += SEL_THREADS) {
-            const uint32_t key = score_key(__ldg(scores + t));
+            const uint32_t key = score_key(__ldcg(scores + t));
             skeys[t - k0] = key;
             lmin = min(lmin, key);
             lmax = max(lmax, key);
@@ -181,7 +181,7 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
     } else if (do_select) {
         uint32_t lmin = 0xFFFFFFFFu, lmax = 0u;
         for (int64_t t = k0 + tid; t < k1; t += SEL_THREADS) {
-            const uint32_t key = score_key(__ldg(scores + t));
+            const uint32_t key = score_key(__ldcg(scores + t));
             lmin = min(lmin, key);
             lmax = max(lmax, key);
         }
@@ -239,7 +239,7 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
             __syncthreads();
 #pragma unroll 4
             for (int64_t t = k0 + tid; t < k1; t += SEL_THREADS) {
-                const uint32_t key = cached ? skeys[t - k0] : score_key(__ldg(scores + t));
+                const uint32_t key = cached ? skeys[t - k0] : score_key(__ldcg(scores + t));
                 const uint32_t d = key - lo;  // wraps for keys below lo: excluded by the range test
                 if (key >= lo && static_cast<uint64_t>(d) < width) atomicAdd(&hist[d >> sh_bits], 1);
             }
@@ -325,13 +325,13 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
         if (t >= w1) return;
         const bool prun = t >= p0 && t < p1;
         if (mode == 1) {
-            kept = keep_in[t] != 0;
+            kept = __ldcg(keep_in + t) != 0;
         } else if (!prun) {
             kept = true;
         } else if (!do_select) {
             kept = kk > 0;  // kk >= P keeps all, kk == 0 keeps none
         } else {
-            const uint32_t key = cached ? skeys[t - k0] : score_key(__ldg(scores + t));
+            const uint32_t key = cached ? skeys[t - k0] : score_key(__ldcg(scores + t));
             kept = key > thr || (key == thr && all_eq_kept);
             eq = key == thr && !all_eq_kept;
         }
@@ -405,7 +405,7 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
             if (emit && kept && mi < m1) {
                 const bool prun = t >= p0 && t < p1;
                 float g = 0.0f;
-                if (prun) g = logsigmoid_f(cached ? key_to_score(skeys[t - k0]) : __ldg(scores + t));
+                if (prun) g = logsigmoid_f(cached ? key_to_score(skeys[t - k0]) : __ldcg(scores + t));
                 kept_idx[mi] = static_cast<int32_t>(t);
                 pos[mi] = static_cast<int32_t>(t - s0 + 1);
                 rank[mi] = static_cast<int32_t>(mi - m0 + 1);
@@ -424,14 +424,17 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
 template <int VPL>  // 16-byte vectors per lane per row
 __global__ void __launch_bounds__(256)
 gather_rows_kernel(const uint4* __restrict__ hidden, const int32_t* __restrict__ kept_idx, int64_t M, int64_t T,
-                   int vecs_per_row, uint4* __restrict__ out) {
+                   int vecs_per_row, uint4* __restrict__ out, int wait_at_end) {
     const int lane = threadIdx.x & 31;
-    pdl_wait();  // global memory is read only from here on
+    // wait_at_end: the map and rows were complete before the preceding kernel was released,
+    // so only the kernel's completion waits for it (which keeps "this kernel is done" meaning
+    // "everything before it is done" for the work that follows)
+    if (!wait_at_end) pdl_wait();  // global memory is read only from here on
     pdl_trigger();
     const int64_t warps_total = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
     for (int64_t m = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); m < M;
          m += warps_total) {
-        const int64_t src = kept_idx[m];
+        const int64_t src = __ldcg(kept_idx + m);
         if (src < 0 || src >= T) continue;  // an unwritten map entry (inconsistent keep flags) copies nothing
         const uint4* s = hidden + src * vecs_per_row;
         uint4* d = out + m * vecs_per_row;
@@ -449,6 +452,7 @@ gather_rows_kernel(const uint4* __restrict__ hidden, const int32_t* __restrict__
             }
         }
     }
+    if (wait_at_end) pdl_wait();
 }
 
 // Gather of narrow rows (one 4- or 8-byte word each, e.g. a position or a gate's
@@ -456,14 +460,15 @@ gather_rows_kernel(const uint4* __restrict__ hidden, const int32_t* __restrict__
 template <typename W>
 __global__ void __launch_bounds__(256)
 gather_words_kernel(const W* __restrict__ src, const int32_t* __restrict__ kept_idx, int64_t M, int64_t T,
-                    W* __restrict__ out) {
-    pdl_wait();  // global memory is read only from here on
+                    W* __restrict__ out, int wait_at_end) {
+    if (!wait_at_end) pdl_wait();  // as in gather_rows_kernel
     pdl_trigger();
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     for (int64_t m = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; m < M; m += stride) {
-        const int64_t i = kept_idx[m];
-        if (i >= 0 && i < T) out[m] = src[i];
+        const int64_t i = __ldcg(kept_idx + m);
+        if (i >= 0 && i < T) out[m] = __ldcg(src + i);
     }
+    if (wait_at_end) pdl_wait();
 }
 
 // Row scatter out[idx[m], :] = in[m, :] (the inverse of the gather), one warp per
@@ -478,7 +483,7 @@ scatter_rows_kernel(const uint4* __restrict__ in, const int32_t* __restrict__ id
     const int64_t warps_total = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
     for (int64_t m = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); m < M;
          m += warps_total) {
-        const int64_t dst = idx[m];
+        const int64_t dst = __ldcg(idx + m);
         if (dst < 0 || dst >= T) continue;
         const uint4* s = in + m * vecs_per_row;
         uint4* d = out + dst * vecs_per_row;
@@ -487,7 +492,7 @@ scatter_rows_kernel(const uint4* __restrict__ in, const int32_t* __restrict__ id
 #pragma unroll
             for (int e = 0; e < VPL; ++e) {
                 const int c = c0 + e * 32 + lane;
-                if (c < vecs_per_row) r[e] = __ldg(s + c);
+                if (c < vecs_per_row) r[e] = __ldcg(s + c);
             }
 #pragma unroll
             for (int e = 0; e < VPL; ++e) {
@@ -519,7 +524,8 @@ cudaError_t launch_select_scan(int mode, const float* scores, const uint8_t* kee
 }
 
 cudaError_t launch_gather_bytes(const void* src, const int32_t* kept_idx, int64_t M_total, int64_t T,
-                                int64_t row_bytes, void* dst, cudaStream_t st) {
+                                int64_t row_bytes, void* dst, cudaStream_t st, bool wait_at_end) {
+    const int wae = wait_at_end ? 1 : 0;
     if (M_total == 0) return cudaSuccess;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
@@ -529,10 +535,11 @@ cudaError_t launch_gather_bytes(const void* src, const int32_t* kept_idx, int64_
         const int grid = static_cast<int>(need < static_cast<int64_t>(sms) * 8 ? need : sms * 8);
         if (row_bytes == 4)
             return launch_pdl(gather_words_kernel<uint32_t>, dim3(grid), dim3(256), 0, st,
-                              static_cast<const uint32_t*>(src), kept_idx, M_total, T, static_cast<uint32_t*>(dst));
+                              static_cast<const uint32_t*>(src), kept_idx, M_total, T, static_cast<uint32_t*>(dst),
+                              wae);
         return launch_pdl(gather_words_kernel<unsigned long long>, dim3(grid), dim3(256), 0, st,
                           static_cast<const unsigned long long*>(src), kept_idx, M_total, T,
-                          static_cast<unsigned long long*>(dst));
+                          static_cast<unsigned long long*>(dst), wae);
     }
     const int64_t vpr64 = row_bytes / 16;
     if (vpr64 <= 0 || vpr64 * 16 != row_bytes || vpr64 > (int64_t(1) << 30)) return cudaErrorInvalidValue;
@@ -541,8 +548,9 @@ cudaError_t launch_gather_bytes(const void* src, const int32_t* kept_idx, int64_
     const int grid = static_cast<int>(blocks_needed < static_cast<int64_t>(sms) * 8 ? blocks_needed : sms * 8);
     const uint4* h = static_cast<const uint4*>(src);
     uint4* o = static_cast<uint4*>(dst);
-    if (vpr >= 256) return launch_pdl(gather_rows_kernel<8>, dim3(grid), dim3(256), 0, st, h, kept_idx, M_total, T, vpr, o);
-    return launch_pdl(gather_rows_kernel<2>, dim3(grid), dim3(256), 0, st, h, kept_idx, M_total, T, vpr, o);
+    if (vpr >= 256)
+        return launch_pdl(gather_rows_kernel<8>, dim3(grid), dim3(256), 0, st, h, kept_idx, M_total, T, vpr, o, wae);
+    return launch_pdl(gather_rows_kernel<2>, dim3(grid), dim3(256), 0, st, h, kept_idx, M_total, T, vpr, o, wae);
 }
 
 cudaError_t launch_scatter_bytes(const void* src, const int32_t* idx, int64_t M, int64_t T, int64_t row_bytes,
@@ -563,8 +571,9 @@ cudaError_t launch_scatter_bytes(const void* src, const int32_t* idx, int64_t M,
 }
 
 cudaError_t launch_gather_rows(const uint16_t* hidden, const int32_t* kept_idx, int64_t M_total, int64_t T, int D,
-                               uint16_t* hidden_kept, cudaStream_t st) {
-    return launch_gather_bytes(hidden, kept_idx, M_total, T, static_cast<int64_t>(D) * 2, hidden_kept, st);
+                               uint16_t* hidden_kept, cudaStream_t st, bool wait_at_end) {
+    return launch_gather_bytes(hidden, kept_idx, M_total, T, static_cast<int64_t>(D) * 2, hidden_kept, st,
+                               wait_at_end);
 }
 
 }  // namespace tg

@@ -4,7 +4,6 @@
 
 #include <cstdarg>
 #include <cstdio>
-#include <mutex>
 #include <string>
 
 #include "tg_internal.cuh"
@@ -43,32 +42,6 @@ tg_status check_device() {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-// Per device: a second stream and two events with which tg_gated_prefill_layer
-// runs the row gather beside the attention (both only need the compaction
-// map).  Created on first use; the mutex keeps one fork/join pair at a time.
-struct SideStream {
-    cudaStream_t stream = nullptr;
-    cudaEvent_t fork = nullptr, join = nullptr;
-};
-constexpr int kMaxDev = 64;
-SideStream g_side[kMaxDev];
-std::mutex g_side_mu;
-
-cudaError_t side_stream(SideStream** out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
-    SideStream& ss = g_side[dev];
-    if (!ss.stream) {
-        if ((e = cudaStreamCreateWithFlags(&ss.stream, cudaStreamNonBlocking)) != cudaSuccess) return e;
-        if ((e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming)) != cudaSuccess) return e;
-        if ((e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming)) != cudaSuccess) return e;
-    }
-    *out = &ss;
-    return cudaSuccess;
-}
 
 #define TG_REQUIRE(cond, ...)                                   \
     do {                                                        \
@@ -110,7 +83,7 @@ tg_status do_score(const uint16_t* hidden, const int32_t* cu_seqlens, const int3
 tg_status do_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* cu_kept, int B,
                        int64_t M_total, int max_M, int Hq, int Hkv, int d, const int32_t* pos, const int32_t* rank,
                        const tg::GateSet& gates, const float* c, float sm_scale, uint16_t* out, float* lse,
-                       void* ws, size_t ws_bytes, cudaStream_t st) {
+                       void* ws, size_t ws_bytes, cudaStream_t st, bool inputs_ready = false) {
     TG_REQUIRE(B >= 0 && M_total >= 0 && max_M >= 0, "negative size");
     if (tg_status s = check_attn_shape(Hq, Hkv, d)) return s;
     TG_REQUIRE(sm_scale > 0.f, "sm_scale must be positive");
@@ -128,7 +101,7 @@ tg_status do_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
     }
     if (tg_status s = check_device()) return s;
     return cuda_status(tg::launch_gated_attention(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, d, pos, rank, gates,
-                                                  c, sm_scale, out, lse, ws, ws_bytes, st),
+                                                  c, sm_scale, out, lse, ws, ws_bytes, st, inputs_ready),
                        "tg_gated_attention launch");
 }
 
@@ -478,42 +451,35 @@ tg_status tg_gated_prefill_layer(const tg_prefill_layer_args* a, tg_stream_t str
                                   "select launch"))
         return s;
     if (a->M_total == 0) return TG_OK;  // every token pruned: no kept rows, no attention
-    // the row gather (HBM-bound) runs on a side stream beside the attention
-    // layers (tensor-bound); both read only the compaction map
-    std::unique_lock<std::mutex> lk(g_side_mu);
-    SideStream* side = nullptr;
-    const bool gathers = a->hidden_kept || a->n_gather > 0;
-    const bool fork = gathers && a->n_layers > 0;
-    if (fork) {
-        if (tg_status s = cuda_status(side_stream(&side), "side stream")) return s;
-        if (tg_status s = cuda_status(cudaEventRecord(side->fork, st), "fork record")) return s;
-        if (tg_status s = cuda_status(cudaStreamWaitEvent(side->stream, side->fork, 0), "fork wait")) return s;
-    }
-    if (a->hidden_kept) {
-        if (tg_status s = cuda_status(tg::launch_gather_rows(a->hidden, a->kept_idx, a->M_total, a->T, a->D,
-                                                             a->hidden_kept, fork ? side->stream : st),
-                                      "gather launch"))
-            return s;
-    }
-    for (int i = 0; i < a->n_gather; ++i) {
-        if (tg_status s = cuda_status(tg::launch_gather_bytes(a->gather_src[i], a->kept_idx, a->M_total, a->T,
-                                                              a->gather_row_bytes[i], a->gather_dst[i],
-                                                              fork ? side->stream : st),
-                                      "extra gather launch"))
-            return s;
-    }
+    // One stream, kernels chained by programmatic dependent launch:
+    //   score -> select -> attention x n_layers -> row gathers.
+    // Each attention layer loads its Q/K/V while its predecessor runs (they are the
+    // caller's, complete before this call) and releases its dependents only once the
+    // selection has completed; the row gathers (HBM-bound) therefore start during the last
+    // attention layer's final wave and read the compaction map at once, waiting for the
+    // attention only before they exit, so that the call's last kernel completes after all
+    // of its work.
     tg_status result = TG_OK;
     for (int l = 0; l < a->n_layers && result == TG_OK; ++l) {
         float* lse = a->lse ? a->lse[l] : nullptr;
         result = do_attention(a->q[l], a->kk[l], a->v[l], a->cu_kept, a->B, a->M_total, a->max_M, a->Hq, a->Hkv,
                               a->d, a->pos, a->rank, tg::single_gate(a->gls, a->g[l]), a->c[l], a->sm_scale,
-                              a->out[l], lse, a->attn_ws, a->attn_ws_bytes, st);
+                              a->out[l], lse, a->attn_ws, a->attn_ws_bytes, st, true);
     }
-    if (fork) {
-        // join: work queued on `stream` after this call also waits for the gather
-        tg_status s = cuda_status(cudaEventRecord(side->join, side->stream), "join record");
-        if (s == TG_OK) s = cuda_status(cudaStreamWaitEvent(st, side->join, 0), "join wait");
-        if (result == TG_OK) result = s;
+    if (result != TG_OK) return result;
+    const bool after_attention = a->n_layers > 0;
+    if (a->hidden_kept) {
+        if (tg_status s = cuda_status(tg::launch_gather_rows(a->hidden, a->kept_idx, a->M_total, a->T, a->D,
+                                                             a->hidden_kept, st, after_attention),
+                                      "gather launch"))
+            return s;
+    }
+    for (int i = 0; i < a->n_gather; ++i) {
+        if (tg_status s = cuda_status(tg::launch_gather_bytes(a->gather_src[i], a->kept_idx, a->M_total, a->T,
+                                                              a->gather_row_bytes[i], a->gather_dst[i], st,
+                                                              after_attention),
+                                      "extra gather launch"))
+            return s;
     }
     return result;
 }

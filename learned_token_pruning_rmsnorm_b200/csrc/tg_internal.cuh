@@ -96,14 +96,22 @@ cudaError_t launch_select_scan(int mode, const float* scores, const uint8_t* kee
 // dst[m, :] = src[kept_idx[m], :] for rows of row_bytes bytes (4, 8 or a multiple of 16;
 // both pointers aligned to min(row_bytes, 16)); rows whose index lies outside [0, T) are
 // left untouched
+// wait_at_end: kept_idx and src were complete before the preceding kernel released its
+// dependents (an attention launched with inputs_ready does so only once its own wait has
+// returned); the kernel then reads at once and waits for its predecessor only before exiting.
 cudaError_t launch_gather_bytes(const void* src, const int32_t* kept_idx, int64_t M_total, int64_t T,
-                                int64_t row_bytes, void* dst, cudaStream_t st);
+                                int64_t row_bytes, void* dst, cudaStream_t st, bool wait_at_end = false);
 // dst[idx[m], :] = src[m, :] (rows of row_bytes bytes, as for launch_gather_bytes)
 cudaError_t launch_scatter_bytes(const void* src, const int32_t* idx, int64_t M, int64_t T, int64_t row_bytes,
                                  void* dst, cudaStream_t st);
 cudaError_t launch_gather_rows(const uint16_t* hidden, const int32_t* kept_idx, int64_t M_total, int64_t T, int D,
-                               uint16_t* hidden_kept, cudaStream_t st);
+                               uint16_t* hidden_kept, cudaStream_t st, bool wait_at_end = false);
 
+// inputs_ready: q, k, v, g, c and cu_kept were complete before the kernel that precedes the
+// attention on `st` started (so the attention may load them while that kernel runs; only
+// pos, rank, gls and the split scratch wait for it).  Only callers that know the stream's
+// history (tg_gated_prefill_layer) may set it.
+//
 // The gate modules whose biases add up on the attention logits: gate i
 // contributes softplus(g[i][h]) * gls[i][j] (one gate is n = 1).  gls[i] is
 // indexed by kept row, g[i] by query head.
@@ -124,7 +132,8 @@ inline GateSet single_gate(const float* gls, const float* g) {
 cudaError_t launch_gated_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* cu_kept,
                                    int B, int64_t M_total, int max_M, int Hq, int Hkv, int d, const int32_t* pos,
                                    const int32_t* rank, const GateSet& gates, const float* c, float sm_scale,
-                                   uint16_t* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t st);
+                                   uint16_t* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t st,
+                                   bool inputs_ready = false);
 
 // Causal work split of the attention: KV chunk length chosen for a launch,
 // scratch bytes the split needs (0 when it never splits), unit count.
