@@ -14,9 +14,11 @@
 //      concentrated exponents still spread) and sums them into 64 superbins.
 //      One warp per CTA then reads the 8 x 64 superbin sums and the 8 x 32
 //      buckets of the chosen superbin through distributed shared memory and
-//      narrows the range to the bucket holding the K-th key.  At most three
-//      passes reach a single key value: thr, with need_eq = how many keys
-//      equal to thr are kept (the lowest-indexed ones).
+//      narrows the range to the bucket holding the K-th key.  The passes stop
+//      when that bucket is a single key value thr (need_eq = how many keys
+//      equal to thr are kept: the lowest-indexed ones), at most three, or as
+//      soon as every key of the bucket is taken (usually after two): then the
+//      rule is key >= the bucket's lower edge, with no tie to rank.
 //   2. ordered scan: every warp owns a contiguous run of the slice and walks
 //      it 32 tokens at a time; ballots count the kept tokens, one block scan
 //      over the warp totals and one exchange of slice totals across the
@@ -309,7 +311,9 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
             }
             __syncthreads();
             SEL_TRACE(3 + pass);
-            if (sh_bits == 0 || pass >= 3) break;  // the bucket is a single key value
+            // done when the bucket is a single key value, or when every key of the bucket is
+            // taken: then "key >= its lower edge" is the whole rule (thr = lo, all kept below)
+            if (sh_bits == 0 || pass >= 3 || sh.remaining == sh.bin_count) break;
         }
         thr = sh.lo;
         need_eq = sh.remaining;
