@@ -26,7 +26,13 @@
 // The bias and temperature therefore cost one extra FFMA per score element
 // on top of plain attention.
 
+#include <algorithm>
+#include <functional>
+#include <map>
 #include <mutex>
+#include <queue>
+#include <tuple>
+#include <vector>
 
 #include "tg_sm100.cuh"
 
@@ -1267,21 +1273,76 @@ int64_t units_below_host(int x, int C) {
     return C * a * (a + 1) / 2 + r * (a + 1);
 }
 
-// KV chunk length (in 128-key tiles) of the causal work split.  The longest
-// query tile of a head pair needs n_qt KV tiles; the whole launch needs
-// B * pairs * n_qt (n_qt + 1) / 2 of them.  When the longest is well above a
-// fair share per SM, long query tiles are cut in halves; otherwise (many
-// waves) the heaviest-first order alone balances the SMs.
+// KV chunk length (in 128-key tiles) of the causal work split.  Query tile qt
+// of a sequence needs qt + 1 KV tiles; a chunk length C < n_qt cuts the query
+// tiles past C into two units ([0, C) and [C, qt + 1)), C >= ceil(n_qt / 2) so
+// that two always suffice.  A unit costs about F + n_kv tile pairs on one SM,
+// F = 3.1 being the fixed part (set-up, first loads, epilogue: 9.0 us against
+// 2.87 us per tile pair in a per-CTA timeline of the N=32k, K=2000 launch).  The
+// block scheduler hands out units heaviest first, which is longest-processing-
+// time scheduling, so C is the candidate whose LPT makespan over the SMs is
+// smallest (all sequences taken at max_M, the bound the host knows); ties go to
+// the larger C (fewer units).
 int attention_kv_chunk(int B, int max_M, int Hq, int Hkv, bool have_ws) {
     const int n_qt = (max_M + BM - 1) / BM;
     if (!have_ws || (Hq / Hkv) % 2 != 0 || n_qt < 4) return n_qt > 0 ? n_qt : 1;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const double total = static_cast<double>(B) * (Hq / 2) * n_qt * (n_qt + 1) / 2.0;
-    const double share = total / sms;
-    if (n_qt <= 1.3 * share) return n_qt;
-    return (n_qt + 1) / 2;
+    if (sms <= 0) sms = 148;
+    const int64_t tiles = static_cast<int64_t>(B) * (Hq / 2);  // (sequence, head pair) instances
+    // many waves (each SM's share at least twice the longest unit): splitting only adds fixed costs
+    if (static_cast<double>(tiles) * n_qt * (n_qt + 1) / 2.0 >= 2.0 * sms * n_qt) return n_qt;
+    // the choice depends on the shape alone: remember it (a few hundred heap operations
+    // per candidate would otherwise run on every call)
+    static std::mutex mu;
+    static std::map<std::tuple<int, int, int, int>, int> memo;
+    const auto key = std::make_tuple(B, n_qt, Hq / 2, sms);
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        const auto it = memo.find(key);
+        if (it != memo.end()) return it->second;
+    }
+    constexpr double F = 3.1;
+    int best_c = n_qt;
+    double best = 1e300;
+    std::vector<double> cost;
+    std::vector<double> load;
+    for (int C = n_qt; C >= (n_qt + 1) / 2; --C) {
+        cost.clear();
+        for (int qt = 0; qt < n_qt; ++qt) {
+            const int n = qt + 1;
+            if (n <= C) {
+                cost.push_back(F + n);
+            } else {
+                cost.push_back(F + C);
+                cost.push_back(F + (n - C));
+            }
+        }
+        std::sort(cost.begin(), cost.end(), [](double a, double b) { return a > b; });
+        // LPT over `sms` machines of the units of all instances (each instance has the same list)
+        load.assign(static_cast<size_t>(sms), 0.0);
+        std::priority_queue<double, std::vector<double>, std::greater<double>> q(load.begin(), load.end());
+        for (double c : cost)
+            for (int64_t i = 0; i < tiles; ++i) {
+                const double t = q.top();
+                q.pop();
+                q.push(t + c);
+            }
+        double mk = 0.0;
+        while (!q.empty()) {
+            mk = q.top();
+            q.pop();
+        }
+        if (mk < best - 1e-9) {
+            best = mk;
+            best_c = C;
+        }
+    }
+    std::lock_guard<std::mutex> lk(mu);
+    if (memo.size() > 256) memo.clear();
+    memo[key] = best_c;
+    return best_c;
 }
 
 size_t attention_workspace_bytes(int B, int max_M, int Hq, int Hkv, int d) {
