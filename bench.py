@@ -372,7 +372,7 @@ def measure_next_rows(tg, dev, st, flush, main, peaks, reps=10):
     grads = [torch.empty_like(L0["q"]), torch.empty_like(L0["k"]), torch.empty_like(L0["v"])]
     f32 = [torch.empty(main["M"], dtype=torch.float32, device=dev) for _ in range(2)] + \
           [torch.empty(wm.Hq, dtype=torch.float32, device=dev) for _ in range(2)]
-    nb = int(lib.tg_gated_attention_backward_workspace_size(main["M"], wm.Hq))
+    nb = int(lib.tg_gated_attention_backward_workspace_size(main["M"], wm.Hq, wm.Hkv, wm.d))
     bws = torch.empty(nb, dtype=torch.uint8, device=dev)
     us = time_device_us(check(lambda: lib.tg_gated_attention_backward(
         L0["q"].data_ptr(), L0["k"].data_ptr(), L0["v"].data_ptr(), out.data_ptr(), dout.data_ptr(), lse.data_ptr(),

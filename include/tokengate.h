@@ -218,11 +218,12 @@ tg_status tg_gated_attention_gates(const uint16_t* q, const uint16_t* k, const u
  * out [M, Hq, d] bf16 and lse [M, Hq] fp32 are the forward's outputs (call
  * tg_gated_attention with a non-NULL lse).  head_dim 64 or 128 (else
  * TG_ERR_UNSUPPORTED).  ws: device scratch, 256-byte aligned, of at least
- * tg_gated_attention_backward_workspace_size(M_total, Hq) bytes (4 floats per
- * row and head; no zeroing needed).  Tensor cores, no atomics: the results are
- * deterministic.
+ * tg_gated_attention_backward_workspace_size(M_total, Hq, Hkv, d) bytes (4
+ * floats per row and head, plus fp32 partial dk and dv per query head when a
+ * KV head serves two or more; no zeroing needed).  Tensor cores, no atomics:
+ * the results are deterministic.
  */
-size_t tg_gated_attention_backward_workspace_size(int64_t M_total, int Hq);
+size_t tg_gated_attention_backward_workspace_size(int64_t M_total, int Hq, int Hkv, int d);
 tg_status tg_gated_attention_backward(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* out,
                                       const uint16_t* dout, const float* lse, const int32_t* cu_kept, int B,
                                       int64_t M_total, int max_M, int Hq, int Hkv, int d, const int32_t* pos,

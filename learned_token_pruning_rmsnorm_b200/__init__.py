@@ -362,7 +362,7 @@ def tg_gated_attention_backward(q, k, v, out, dout, lse, cu_kept, max_M: int, po
            "dgls": torch.empty(M, dtype=torch.float32, device=dev),
            "dscore": torch.empty(M, dtype=torch.float32, device=dev) if want_dscore else None,
            "dg": torch.empty(Hq, dtype=torch.float32, device=dev), "dc": torch.empty(Hq, dtype=torch.float32, device=dev)}
-    n = int(load().tg_gated_attention_backward_workspace_size(M, Hq))
+    n = int(load().tg_gated_attention_backward_workspace_size(M, Hq, Hkv, d))
     ws = torch.empty(max(n, 256), dtype=torch.uint8, device=dev)
     _lib.check(load().tg_gated_attention_backward(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(), lse.data_ptr(), ck.data_ptr(),

@@ -61,7 +61,7 @@ SIGNATURES = {
     "tg_gated_attention_gates": ([P, P, P, P, i32, i64, i32, i32, i32, i32, P, P, i32, P, P, P, f32, P, P, P,
                                   C.c_size_t, P], i32),
     "tg_next_gate_span": ([P, P, i32, P], i32),
-    "tg_gated_attention_backward_workspace_size": ([i64, i32], C.c_size_t),
+    "tg_gated_attention_backward_workspace_size": ([i64, i32, i32, i32], C.c_size_t),
     "tg_gated_attention_backward": ([P, P, P, P, P, P, P, i32, i64, i32, i32, i32, i32, P, P, P, P, P, f32,
                                      P, P, P, P, P, P, P, P, C.c_size_t, P], i32),
     "tg_gated_attention_workspace_size": ([i32, i32, i32, i32, i32], C.c_size_t),

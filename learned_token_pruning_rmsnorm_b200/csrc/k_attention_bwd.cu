@@ -16,12 +16,14 @@
 // Five launches, no atomics (results do not depend on scheduling):
 //   rowdot   D_ih = dout_i.out_i for every (row, head)
 //   dq       (below)
-//   dkv      one CTA per (KV head, 128-key tile): for every query head of the
-//            group and every causal query tile, S^T = K Q^T and dP^T = V dO^T
+//   dkv      one CTA per (query head, 128-key tile): for every causal query
+//            tile, S^T = K Q^T and dP^T = V dO^T
 //            on the tensor core (TMEM lanes = keys), then P^T and G^T as bf16
 //            over the first 64 columns of S^T and dP^T, and dV += P^T dO,
 //            dK += G^T Q read from TMEM.  The per-key sums of G (the gate
 //            bias's gradient, per head) are sums along each thread's own row.
+//            The query heads of a GQA group leave fp32 partials of dK / dV that
+//            kv_reduce sums in head order (a group of one writes bf16 itself).
 //   dq       one CTA per (query head, 128-query tile), the forward's layout:
 //            S = Q K^T and dP = dO V^T, G as bf16 over S, dQ += G K.  The
 //            per-query sums for dbeta and dtau run along each thread's row,
@@ -119,12 +121,15 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
                           const int32_t* __restrict__ cu_kept, const int32_t* __restrict__ pos,
                           const int32_t* __restrict__ rank, const float* __restrict__ gls,
                           const float* __restrict__ g, const float* __restrict__ c, const float* __restrict__ lse,
-                          const float* __restrict__ Drow, float sm_scale, int Hq, int Hkv, uint16_t* __restrict__ dk,
-                          uint16_t* __restrict__ dv, float* __restrict__ colsum, int* __restrict__ status) {
+                          const float* __restrict__ Drow, float sm_scale, int Hq, int Hkv, int64_t M_total,
+                          uint16_t* __restrict__ dk, uint16_t* __restrict__ dv, float* __restrict__ part_k,
+                          float* __restrict__ part_v, float* __restrict__ colsum, int* __restrict__ status) {
     using L = DkvSmem<HD>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int hk = blockIdx.x, kt = blockIdx.y, b = blockIdx.z;
+    // one query head per CTA: the heads of a GQA group leave partial dK / dV (fp32, summed
+    // in head order by bwd_kv_reduce_kernel); a group of one writes bf16 directly
+    const int h = blockIdx.x, kt = blockIdx.y, b = blockIdx.z;
     pdl_wait();  // global memory is read only from here on
     pdl_trigger();
     const int seq0 = cu_kept[b];
@@ -132,8 +137,9 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
     if (kt * BT >= Mb) return;
     const int n_qt = (Mb + BT - 1) / BT;
     const int grp = Hq / Hkv;
-    const int nq = n_qt - kt;  // causal query tiles per head
-    const int n_steps = grp * nq;
+    const int hk = h / grp, hh = h - hk * grp;
+    const int nq = n_qt - kt;  // causal query tiles
+    const int n_steps = nq;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     const uint32_t sbase = smem_u32(smem);
@@ -181,7 +187,7 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
             int issued[2] = {0, 0};
             for (int t = 0; t < n_steps; ++t) {
                 const int s = t & 1;
-                const int h = hk * grp + t / nq, i = kt + t % nq;
+                const int i = kt + t;
                 if (t >= 2 && !mbar_wait(bar(D_QD_EMPTY + s), ((t - 2) >> 1) & 1, abort_flag, status,
                                          TG_WHERE_PRODUCER))
                     break;
@@ -261,8 +267,7 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
         float* par = reinterpret_cast<float*>(smem + L::OFF_PAR);
         bool ok = true;
         int t = 0;
-        for (int hh = 0; hh < grp && ok; ++hh) {
-            const int h = hk * grp + hh;
+        {
             const float beta = softplus_b(g[h]);
             float csum = 0.f;
             for (int ii = 0; ii < nq; ++ii, ++t) {
@@ -339,7 +344,28 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
         }
         // ---------------------------------------------------------------- epilogue
         if (ok) ok = mbar_wait_warp(bar(D_ACC_DONE), 0, abort_flag, status, TG_WHERE_SOFTMAX);
-        if (ok) {
+        if (ok && part_k) {
+            // partials of this head: [head in group][row][KV head][d] fp32, unscaled
+            tc_fence_after();
+            const size_t row = ((static_cast<size_t>(hh) * M_total + seq0 + key_local) * Hkv + hk) * HD;
+#pragma unroll 1
+            for (int which = 0; which < 2; ++which) {
+                const uint32_t src = which ? tDK : tDV;
+                float* dst = (which ? part_k : part_v) + row;
+#pragma unroll
+                for (int ch = 0; ch < HD / 32; ++ch) {
+                    float o[32];
+                    tmem_ld32(src + lane_addr + ch * 32, o);
+                    tmem_wait_ld();
+                    if (valid_key) {
+#pragma unroll
+                        for (int q4 = 0; q4 < 8; ++q4)
+                            *reinterpret_cast<float4*>(dst + ch * 32 + q4 * 4) =
+                                make_float4(o[q4 * 4], o[q4 * 4 + 1], o[q4 * 4 + 2], o[q4 * 4 + 3]);
+                    }
+                }
+            }
+        } else if (ok) {
             tc_fence_after();
             const size_t row = (static_cast<size_t>(seq0 + key_local) * Hkv + hk) * HD;
 #pragma unroll 1
@@ -673,6 +699,37 @@ gated_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
 }
 
 // ---------------------------------------------------------------------------
+// dK = sm * sum_h part_k[h], dV = sum_h part_v[h] over the query heads of each group, in
+// head order, to bf16 (8 consecutive elements per thread).
+__global__ void __launch_bounds__(256)
+bwd_kv_reduce_kernel(const float* __restrict__ part_k, const float* __restrict__ part_v, int grp, int64_t n,
+                     float sm_scale, uint16_t* __restrict__ dk, uint16_t* __restrict__ dv) {
+    pdl_wait();
+    pdl_trigger();
+    for (int64_t e = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 8; e < n;
+         e += static_cast<int64_t>(gridDim.x) * blockDim.x * 8) {
+#pragma unroll 1
+        for (int which = 0; which < 2; ++which) {
+            const float* src = which ? part_v : part_k;
+            float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            for (int q = 0; q < grp; ++q) {
+                const float4 x = __ldcg(reinterpret_cast<const float4*>(src + q * n + e));
+                const float4 y = __ldcg(reinterpret_cast<const float4*>(src + q * n + e + 4));
+                a[0] += x.x; a[1] += x.y; a[2] += x.z; a[3] += x.w;
+                a[4] += y.x; a[5] += y.y; a[6] += y.z; a[7] += y.w;
+            }
+            const float sc = which ? 1.0f : sm_scale;
+            uint4 w;
+            w.x = pack2_bf16(a[0] * sc, a[1] * sc);
+            w.y = pack2_bf16(a[2] * sc, a[3] * sc);
+            w.z = pack2_bf16(a[4] * sc, a[5] * sc);
+            w.w = pack2_bf16(a[6] * sc, a[7] * sc);
+            *reinterpret_cast<uint4*>((which ? dv : dk) + e) = w;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Per key: dgls_j = sum_h softplus(g_h) colsum[j, h]; d score_j = dgls_j (1 - exp(gls_j)).
 __global__ void __launch_bounds__(256)
 bwd_keys_kernel(const float* __restrict__ colsum, const float* __restrict__ gls, const float* __restrict__ g,
@@ -736,6 +793,10 @@ cudaError_t launch_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
     float* colsum = Drow + rows;
     float* rowE = colsum + rows;
     float* rowT = rowE + rows;
+    const int grp = Hq / Hkv;
+    const int64_t nkv = M_total * Hkv * HD;
+    float* part_k = grp > 1 ? rowT + rows : nullptr;  // [grp][M][Hkv][HD] each
+    float* part_v = grp > 1 ? part_k + grp * nkv : nullptr;
     CUtensorMap tq, tk, tv, tdo;
     if (!encode_tmap_2d_bf16(&tq, q, static_cast<uint64_t>(Hq) * HD, static_cast<uint64_t>(M_total),
                              static_cast<uint64_t>(Hq) * HD * 2, 64, BT) ||
@@ -760,10 +821,18 @@ cudaError_t launch_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
                    static_cast<size_t>(DqSmem<HD>::ALLOC), st, tq, tk, tv, tdo, cu_kept, pos, rank, gls, g, c, lse,
                    Drow, sm_scale, Hq, Hkv, n_t, dq, rowE, rowT, status);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(gated_attn_bwd_dkv_kernel<HD>, dim3(Hkv, n_t, B), dim3(BWD_THREADS),
+    e = launch_pdl(gated_attn_bwd_dkv_kernel<HD>, dim3(Hq, n_t, B), dim3(BWD_THREADS),
                    static_cast<size_t>(DkvSmem<HD>::ALLOC), st, tq, tk, tv, tdo, cu_kept, pos, rank, gls, g, c, lse,
-                   static_cast<const float*>(Drow), sm_scale, Hq, Hkv, dk, dv, colsum, status);
+                   static_cast<const float*>(Drow), sm_scale, Hq, Hkv, M_total, dk, dv, part_k, part_v, colsum,
+                   status);
     if (e != cudaSuccess) return e;
+    if (grp > 1) {
+        const int64_t rb = (nkv / 8 + 255) / 256;
+        e = launch_pdl(bwd_kv_reduce_kernel, dim3(static_cast<unsigned>(rb < sms * 8 ? rb : sms * 8)), dim3(256), 0, st,
+                       static_cast<const float*>(part_k), static_cast<const float*>(part_v), grp, nkv, sm_scale, dk,
+                       dv);
+        if (e != cudaSuccess) return e;
+    }
     const int64_t kb = (M_total + 255) / 256;
     e = launch_pdl(bwd_keys_kernel, dim3(static_cast<unsigned>(kb < sms * 4 ? kb : sms * 4)), dim3(256), 0, st,
                    static_cast<const float*>(colsum), gls, g, M_total, Hq, dgls, dscore);
@@ -774,8 +843,11 @@ cudaError_t launch_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
 
 }  // namespace
 
-size_t attention_backward_workspace_bytes(int64_t M_total, int Hq) {
-    return static_cast<size_t>(4) * static_cast<size_t>(M_total) * static_cast<size_t>(Hq) * sizeof(float);
+size_t attention_backward_workspace_bytes(int64_t M_total, int Hq, int Hkv, int d) {
+    const size_t rows = static_cast<size_t>(4) * static_cast<size_t>(M_total) * static_cast<size_t>(Hq);
+    const int grp = Hkv > 0 ? Hq / Hkv : 1;
+    const size_t parts = grp > 1 ? static_cast<size_t>(2) * grp * static_cast<size_t>(M_total) * Hkv * d : 0;
+    return (rows + parts) * sizeof(float);
 }
 
 cudaError_t launch_gated_attention_backward(const uint16_t* q, const uint16_t* k, const uint16_t* v,

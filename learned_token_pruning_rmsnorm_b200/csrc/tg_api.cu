@@ -192,7 +192,7 @@ tg_status tg_masked_gated_attention(const uint16_t* q, const uint16_t* k, const 
 }
 
 
-int tg_abi_version(void) { return 4; }
+int tg_abi_version(void) { return 5; }
 
 const char* tg_last_error_string(void) { return g_last_error.c_str(); }
 
@@ -344,9 +344,9 @@ tg_status tg_gated_attention_gates(const uint16_t* q, const uint16_t* k, const u
                         ws_bytes, stream);
 }
 
-size_t tg_gated_attention_backward_workspace_size(int64_t M_total, int Hq) {
-    if (M_total <= 0 || Hq <= 0) return 0;
-    return tg::attention_backward_workspace_bytes(M_total, Hq);
+size_t tg_gated_attention_backward_workspace_size(int64_t M_total, int Hq, int Hkv, int d) {
+    if (M_total <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || (d != 64 && d != 128)) return 0;
+    return tg::attention_backward_workspace_bytes(M_total, Hq, Hkv, d);
 }
 
 tg_status tg_gated_attention_backward(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* out,
@@ -369,7 +369,7 @@ tg_status tg_gated_attention_backward(const uint16_t* q, const uint16_t* k, cons
                    aligned16(dk) && aligned16(dv),
                "q, k, v, out, dout, dq, dk and dv must be 16-byte aligned");
     TG_REQUIRE((reinterpret_cast<uintptr_t>(ws) & 255u) == 0, "ws must be 256-byte aligned");
-    const size_t need = tg::attention_backward_workspace_bytes(M_total, Hq);
+    const size_t need = tg::attention_backward_workspace_bytes(M_total, Hq, Hkv, d);
     TG_REQUIRE(ws_bytes >= need, "ws holds %zu bytes, the backward needs %zu", ws_bytes, need);
     if (tg_status s = check_device()) return s;
     return cuda_status(tg::launch_gated_attention_backward(q, k, v, out, dout, lse, cu_kept, B, M_total, max_M, Hq,

@@ -146,8 +146,9 @@ cudaError_t launch_gated_attention_noalloc(const uint16_t* q, const uint16_t* k,
 size_t attention_workspace_bytes(int B, int max_M, int Hq, int Hkv, int d);
 
 // Backward of the one-gate attention (head_dim 64 or 128); ws holds
-// attention_backward_workspace_bytes(M_total, Hq) bytes (4 fp32 per row and head).
-size_t attention_backward_workspace_bytes(int64_t M_total, int Hq);
+// attention_backward_workspace_bytes(M_total, Hq, Hkv, d) bytes (4 fp32 per row and head,
+// plus fp32 partial dK and dV per query head of a GQA group when the group has two or more).
+size_t attention_backward_workspace_bytes(int64_t M_total, int Hq, int Hkv, int d);
 cudaError_t launch_gated_attention_backward(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                             const uint16_t* out, const uint16_t* dout, const float* lse,
                                             const int32_t* cu_kept, int B, int64_t M_total, int max_M, int Hq,

@@ -44,7 +44,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version(lib):
-    assert lib.tg_abi_version() == 4
+    assert lib.tg_abi_version() == 5
 
 
 def test_kept_count_host_helper(lib):
