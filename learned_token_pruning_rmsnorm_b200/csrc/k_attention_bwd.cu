@@ -13,9 +13,8 @@
 //   dg_h = dbeta_h sigmoid(g_h),  dc_h = sum_i dtau_ih ln(pos_i / rank_i),
 //   d score_j = dgls_j sigmoid(-score_j) = dgls_j (1 - exp(gls_j)).
 //
-// Five launches, no atomics (results do not depend on scheduling):
-//   rowdot   D_ih = dout_i.out_i for every (row, head)
-//   dq       (below)
+// Three or four launches, no atomics (results do not depend on scheduling):
+//   dq       (below; it also forms D_ih = dout_i.out_i for its rows)
 //   dkv      one CTA per (query head, 128-key tile): for every causal query
 //            tile, S^T = K Q^T and dP^T = V dO^T
 //            on the tensor core (TMEM lanes = keys), then P^T and G^T as bf16
@@ -29,7 +28,8 @@
 //            per-query sums for dbeta and dtau run along each thread's row,
 //            which also yields the exact D'_i = sum_j P_ij dP_ij; it replaces
 //            D for the dkv kernel (launched after dq).
-//   reduce   dgls / d score per key, dg and dc per head.
+//   finish   dgls / d score per key, dg and dc per head (the dq kernel leaves one
+//            partial sum of the dbeta and dc terms per query tile).
 // Every row of P is rebuilt from the forward's log-sum-exp.
 
 #include "tg_sm100.cuh"
@@ -54,30 +54,6 @@ __device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) {
 __device__ __forceinline__ bool drain_wait_b(uint32_t bar, uint32_t parity, int* status) {
     volatile int never = 0;
     return mbar_wait(bar, parity, &never, status, TG_WHERE_DRAIN);
-}
-
-// ---------------------------------------------------------------------------
-// D_r = dout_r . out_r for each of the M * Hq rows of d elements; one warp per row.
-__global__ void __launch_bounds__(256)
-bwd_rowdot_kernel(const uint16_t* __restrict__ out, const uint16_t* __restrict__ dout, int64_t rows, int d,
-                  float* __restrict__ D) {
-    pdl_wait();
-    pdl_trigger();
-    const int lane = threadIdx.x & 31;
-    const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-    for (int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows;
-         r += warps) {
-        const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(out + r * d);
-        const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(dout + r * d);
-        float acc = 0.f;
-        for (int e = lane; e < d / 2; e += 32) {
-            const float2 a = __bfloat1622float2(o2[e]), b = __bfloat1622float2(g2[e]);
-            acc = fmaf(a.x, b.x, fmaf(a.y, b.y, acc));
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (lane == 0) D[r] = acc;
-    }
 }
 
 // ---------------------------------------------------------------------------
@@ -423,8 +399,8 @@ struct DqSmem {
     static constexpr int OFF_GLS = OFF_V + 2 * TILE;   // [4 warps][2][BT] fp32, a private copy per warp
     static constexpr int OFF_BAR = OFF_GLS + 4 * 2 * BT * 4;
     static constexpr int NUM_BARS = 16;
-    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-    static constexpr int BYTES = OFF_MISC + 16;
+    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;  // tmem slot, abort flag, then 8 fp32
+    static constexpr int BYTES = OFF_MISC + 16 + 32;
     static constexpr int ALLOC = BYTES + 1024;
     static constexpr uint32_t TMEM_COLS = 512;
     static_assert(ALLOC <= 227 * 1024, "shared memory");
@@ -443,9 +419,9 @@ gated_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
                          const int32_t* __restrict__ cu_kept, const int32_t* __restrict__ pos,
                          const int32_t* __restrict__ rank, const float* __restrict__ gls,
                          const float* __restrict__ g, const float* __restrict__ c, const float* __restrict__ lse,
-                         float* __restrict__ Drow, float sm_scale, int Hq, int Hkv, int n_qt_max,
-                         uint16_t* __restrict__ dq, float* __restrict__ rowE, float* __restrict__ rowT,
-                         int* __restrict__ status) {
+                         const uint16_t* __restrict__ out_fwd, float* __restrict__ Drow, float sm_scale, int Hq,
+                         int Hkv, int n_qt_max, uint16_t* __restrict__ dq, float* __restrict__ tileE,
+                         float* __restrict__ tileT, int* __restrict__ status) {
     using L = DqSmem<HD>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -589,21 +565,42 @@ gated_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
         const bool valid_row = q_local < Mb;
         const int qg = seq0 + q_local;
         const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
-        float fa = 0.f, fb = 0.f, fl = 0.f, fd = 0.f, fi = 0.f;
+        float fa = 0.f, fb = 0.f, fl = 0.f, fd = 0.f, fi = 0.f, lr = 0.f;
         if (valid_row) {
-            fi = 1.0f / (1.0f + c[h] * logf(static_cast<float>(__ldcg(pos + qg)) / static_cast<float>(__ldcg(rank + qg))));
+            lr = logf(static_cast<float>(__ldcg(pos + qg)) / static_cast<float>(__ldcg(rank + qg)));
+            fi = 1.0f / (1.0f + c[h] * lr);
             fa = sm_scale * LOG2E_B * fi;
             fb = softplus_b(g[h]) * LOG2E_B * fi;
-            fl = lse[static_cast<size_t>(qg) * Hq + h] * LOG2E_B;
-            fd = __ldcg(Drow + static_cast<size_t>(qg) * Hq + h);
+            fl = __ldcg(lse + static_cast<size_t>(qg) * Hq + h) * LOG2E_B;
+        }
+        // D = dout . out of this row, with dout from the staged tile (128-byte swizzled boxes of
+        // 64 columns) and out, the forward's output, from global memory
+        bool ok = mbar_wait_warp(bar(Q_QD_FULL), 0, abort_flag, status, TG_WHERE_SOFTMAX);
+        if (ok && valid_row) {
+            const uint16_t* orow = out_fwd + (static_cast<size_t>(qg) * Hq + h) * HD;
+            float acc = 0.f;
+#pragma unroll
+            for (int hf = 0; hf < HD / 64; ++hf)
+#pragma unroll
+                for (int cch = 0; cch < 8; ++cch) {
+                    const uint4 dv = *reinterpret_cast<const uint4*>(smem + L::OFF_DO + hf * (BT * 128) + r * 128 +
+                                                                     ((cch ^ (r & 7)) << 4));
+                    const uint4 ov = __ldcg(reinterpret_cast<const uint4*>(orow + hf * 64 + cch * 8));
+                    const uint32_t a[4] = {dv.x, dv.y, dv.z, dv.w}, o4[4] = {ov.x, ov.y, ov.z, ov.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        acc = fmaf(__uint_as_float(a[e] << 16), __uint_as_float(o4[e] << 16), acc);
+                        acc = fmaf(__uint_as_float(a[e] & 0xFFFF0000u), __uint_as_float(o4[e] & 0xFFFF0000u), acc);
+                    }
+                }
+            fd = acc;
         }
         float* wgls = reinterpret_cast<float*>(smem + L::OFF_GLS) + warp * (2 * BT);
         // Row sums for dbeta and dtau, formed with the row's exact D' = sum_j P dP (the
         // D above comes from the bf16 output; dtau = -sum_j dl l / tau cancels to a small
         // number and would amplify its rounding):  sum_j dl x = sum P dP x - D' sum P x.
         float aPdPt = 0.f, aPt = 0.f, aPdP = 0.f, aP = 0.f, aPdPg = 0.f, aPg = 0.f;
-        bool ok = true;
-        for (int j = 0; j < n_kv; ++j) {
+        for (int j = 0; ok && j < n_kv; ++j) {
             const int s = j & 1;
             // the tile's gls into this warp's own copy (only __syncwarp orders it)
 #pragma unroll
@@ -679,14 +676,33 @@ gated_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
                     }
                 }
             }
-            if (valid_row) {
-                const float Dx = aPdP;
-                // tt = l log2(e) - lse log2(e):  sum dl l = ln2 (sum dl tt + lse log2(e) sum dl)
-                const float sum_dl_t = aPdPt - Dx * aPt + fl * (aPdP - Dx * aP);
-                rowE[static_cast<size_t>(qg) * Hq + h] = fi * (aPdPg - Dx * aPg);  // sum_j G gls_j
-                rowT[static_cast<size_t>(qg) * Hq + h] = -LN2_B * fi * sum_dl_t;   // dtau of the row
-                Drow[static_cast<size_t>(qg) * Hq + h] = Dx;  // the exact D' for the dK/dV kernel
-            }
+            if (valid_row) Drow[static_cast<size_t>(qg) * Hq + h] = aPdP;  // the exact D' for the dK/dV kernel
+        }
+        // this tile's terms of dbeta_h (sum_i sum_j G gls_j) and dc_h (sum_i ln(pos/rank) dtau),
+        // summed over its rows in a fixed order and stored at the tile's first row
+        float eE = 0.f, eT = 0.f;
+        if (ok && valid_row) {
+            const float Dx = aPdP;
+            // tt = l log2(e) - lse log2(e):  sum dl l = ln2 (sum dl tt + lse log2(e) sum dl)
+            const float sum_dl_t = aPdPt - Dx * aPt + fl * (aPdP - Dx * aP);
+            eE = fi * (aPdPg - Dx * aPg);
+            eT = lr * (-LN2_B * fi * sum_dl_t);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            eE += __shfl_xor_sync(0xffffffffu, eE, o);
+            eT += __shfl_xor_sync(0xffffffffu, eT, o);
+        }
+        float* red = reinterpret_cast<float*>(smem + L::OFF_MISC + 16);
+        if (lane == 0) {
+            red[warp] = eE;
+            red[4 + warp] = eT;
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");  // the four compute warps, abort or not
+        if (threadIdx.x == 0 && ok) {
+            const size_t slot = (static_cast<size_t>(seq0) + static_cast<size_t>(qt) * BT) * Hq + h;
+            tileE[slot] = (red[0] + red[1]) + (red[2] + red[3]);
+            tileT[slot] = (red[4] + red[5]) + (red[6] + red[7]);
         }
     }
 
@@ -730,49 +746,50 @@ bwd_kv_reduce_kernel(const float* __restrict__ part_k, const float* __restrict__
 }
 
 // ---------------------------------------------------------------------------
-// Per key: dgls_j = sum_h softplus(g_h) colsum[j, h]; d score_j = dgls_j (1 - exp(gls_j)).
+// The last step, one launch:
+//   blocks 0 .. Hq-1, head h:  dg_h = sigmoid(g_h) sum_tiles tileE[., h],
+//                              dc_h = sum_tiles tileT[., h]  (one warp, fixed order);
+//   the other blocks, per key: dgls_j = sum_h softplus(g_h) colsum[j, h] and
+//                              d score_j = dgls_j (1 - exp(gls_j)).
 __global__ void __launch_bounds__(256)
-bwd_keys_kernel(const float* __restrict__ colsum, const float* __restrict__ gls, const float* __restrict__ g,
-                int64_t M, int Hq, float* __restrict__ dgls, float* __restrict__ dscore) {
+bwd_finish_kernel(const float* __restrict__ colsum, const float* __restrict__ tileE, const float* __restrict__ tileT,
+                  const float* __restrict__ gls, const float* __restrict__ g, const int32_t* __restrict__ cu_kept,
+                  int B, int64_t M, int Hq, float* __restrict__ dgls, float* __restrict__ dscore,
+                  float* __restrict__ dg, float* __restrict__ dc) {
     pdl_wait();
     pdl_trigger();
-    for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < M;
-         j += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    if (static_cast<int>(blockIdx.x) < Hq) {
+        const int h = blockIdx.x;
+        if (threadIdx.x >= 32) return;
+        const int lane = threadIdx.x;
+        float e = 0.f, t = 0.f;
+        int k = 0;  // running tile number: lane k % 32 takes tile k
+        for (int b = 0; b < B; ++b) {
+            const int s0 = cu_kept[b], n_qt = (cu_kept[b + 1] - s0 + BT - 1) / BT;
+            for (int qt = 0; qt < n_qt; ++qt, ++k)
+                if ((k & 31) == lane) {
+                    const size_t slot = (static_cast<size_t>(s0) + static_cast<size_t>(qt) * BT) * Hq + h;
+                    e += __ldcg(tileE + slot);
+                    t += __ldcg(tileT + slot);
+                }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            e += __shfl_xor_sync(0xffffffffu, e, o);
+            t += __shfl_xor_sync(0xffffffffu, t, o);
+        }
+        if (lane == 0) {
+            dg[h] = e / (1.0f + expf(-g[h]));
+            dc[h] = t;
+        }
+        return;
+    }
+    const int64_t nb = static_cast<int64_t>(gridDim.x) - Hq;
+    for (int64_t j = static_cast<int64_t>(blockIdx.x - Hq) * blockDim.x + threadIdx.x; j < M; j += nb * blockDim.x) {
         float acc = 0.f;
         for (int h = 0; h < Hq; ++h) acc = fmaf(softplus_b(g[h]), __ldcg(colsum + j * Hq + h), acc);
         dgls[j] = acc;
         if (dscore) dscore[j] = acc * -expm1f(gls[j]);
-    }
-}
-
-// Per head (one block each): dg_h = sigmoid(g_h) sum_i rowE[i, h];
-// dc_h = sum_i ln(pos_i / rank_i) rowT[i, h].  Fixed summation order.
-__global__ void __launch_bounds__(256)
-bwd_heads_kernel(const float* __restrict__ rowE, const float* __restrict__ rowT, const int32_t* __restrict__ pos,
-                 const int32_t* __restrict__ rank, const float* __restrict__ g, int64_t M, int Hq,
-                 float* __restrict__ dg, float* __restrict__ dc) {
-    pdl_wait();
-    pdl_trigger();
-    __shared__ float sE[256], sT[256];
-    const int h = blockIdx.x;
-    float e = 0.f, t = 0.f;
-    for (int64_t i = threadIdx.x; i < M; i += blockDim.x) {
-        e += __ldcg(rowE + i * Hq + h);
-        t = fmaf(logf(static_cast<float>(pos[i]) / static_cast<float>(rank[i])), __ldcg(rowT + i * Hq + h), t);
-    }
-    sE[threadIdx.x] = e;
-    sT[threadIdx.x] = t;
-    __syncthreads();
-    for (int w = 128; w > 0; w >>= 1) {
-        if (threadIdx.x < w) {
-            sE[threadIdx.x] += sE[threadIdx.x + w];
-            sT[threadIdx.x] += sT[threadIdx.x + w];
-        }
-        __syncthreads();
-    }
-    if (threadIdx.x == 0) {
-        dg[h] = sE[0] / (1.0f + expf(-g[h]));
-        dc[h] = sT[0];
     }
 }
 
@@ -791,11 +808,11 @@ cudaError_t launch_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
     const size_t rows = static_cast<size_t>(M_total) * Hq;
     float* Drow = static_cast<float*>(ws);
     float* colsum = Drow + rows;
-    float* rowE = colsum + rows;
-    float* rowT = rowE + rows;
+    float* tileE = colsum + rows;  // per query tile, at its first row
+    float* tileT = tileE + rows;
     const int grp = Hq / Hkv;
     const int64_t nkv = M_total * Hkv * HD;
-    float* part_k = grp > 1 ? rowT + rows : nullptr;  // [grp][M][Hkv][HD] each
+    float* part_k = grp > 1 ? tileT + rows : nullptr;  // [grp][M][Hkv][HD] each
     float* part_v = grp > 1 ? part_k + grp * nkv : nullptr;
     CUtensorMap tq, tk, tv, tdo;
     if (!encode_tmap_2d_bf16(&tq, q, static_cast<uint64_t>(Hq) * HD, static_cast<uint64_t>(M_total),
@@ -811,15 +828,12 @@ cudaError_t launch_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     int* status = device_status_ptr();
-    const int64_t rd_blocks = (static_cast<int64_t>(rows) + 7) / 8;
-    cudaError_t e = launch_pdl(bwd_rowdot_kernel, dim3(static_cast<unsigned>(rd_blocks < sms * 8 ? rd_blocks : sms * 8)),
-                               dim3(256), 0, st, out, dout, static_cast<int64_t>(rows), HD, Drow);
-    if (e != cudaSuccess) return e;
     const int n_t = (max_M + BT - 1) / BT;
-    // dq first: it replaces each row's D by the exact sum_j P dP, which the dK/dV kernel then uses
-    e = launch_pdl(gated_attn_bwd_dq_kernel<HD>, dim3(Hq, n_t, B), dim3(BWD_THREADS),
-                   static_cast<size_t>(DqSmem<HD>::ALLOC), st, tq, tk, tv, tdo, cu_kept, pos, rank, gls, g, c, lse,
-                   Drow, sm_scale, Hq, Hkv, n_t, dq, rowE, rowT, status);
+    // dq first: it forms each row's D = dout . out for its own use and leaves the exact
+    // D' = sum_j P dP for the dK/dV kernel
+    cudaError_t e = launch_pdl(gated_attn_bwd_dq_kernel<HD>, dim3(Hq, n_t, B), dim3(BWD_THREADS),
+                               static_cast<size_t>(DqSmem<HD>::ALLOC), st, tq, tk, tv, tdo, cu_kept, pos, rank, gls, g,
+                               c, lse, out, Drow, sm_scale, Hq, Hkv, n_t, dq, tileE, tileT, status);
     if (e != cudaSuccess) return e;
     e = launch_pdl(gated_attn_bwd_dkv_kernel<HD>, dim3(Hq, n_t, B), dim3(BWD_THREADS),
                    static_cast<size_t>(DkvSmem<HD>::ALLOC), st, tq, tk, tv, tdo, cu_kept, pos, rank, gls, g, c, lse,
@@ -834,11 +848,10 @@ cudaError_t launch_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
         if (e != cudaSuccess) return e;
     }
     const int64_t kb = (M_total + 255) / 256;
-    e = launch_pdl(bwd_keys_kernel, dim3(static_cast<unsigned>(kb < sms * 4 ? kb : sms * 4)), dim3(256), 0, st,
-                   static_cast<const float*>(colsum), gls, g, M_total, Hq, dgls, dscore);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(bwd_heads_kernel, dim3(Hq), dim3(256), 0, st, static_cast<const float*>(rowE),
-                      static_cast<const float*>(rowT), pos, rank, g, M_total, Hq, dg, dc);
+    const int key_blocks = static_cast<int>(kb < sms * 4 ? kb : sms * 4);
+    return launch_pdl(bwd_finish_kernel, dim3(Hq + key_blocks), dim3(256), 0, st, static_cast<const float*>(colsum),
+                      static_cast<const float*>(tileE), static_cast<const float*>(tileT), gls, g, cu_kept, B, M_total,
+                      Hq, dgls, dscore, dg, dc);
 }
 
 }  // namespace
