@@ -237,20 +237,28 @@ def workload_config(w, n_layers):
 # ------------------------------------------------------------------ GPU arm
 
 def time_device_us(fn, st, flush, reps, warm=3):
-    """Median device time (us) of fn() on stream st, L2 flushed before each rep."""
+    """Median device time (us) of fn() on stream st, L2 flushed before each rep.  fn is
+    captured into a CUDA graph and the replays are timed, so that no host work (argument
+    checks, tensor-map encoding) sits between the events."""
     import torch
     for _ in range(warm):
         fn()
+    torch.cuda.synchronize()
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr):
+        fn()
+    gr.replay()
     torch.cuda.synchronize()
     ev = []
     for i in range(reps):
         flush.fill_(i)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(st)
-        fn()
+        gr.replay()
         b.record(st)
         ev.append((a, b))
     torch.cuda.synchronize()
+    del gr
     return 1e3 * float(np.median([a.elapsed_time(b) for a, b in ev]))
 
 
@@ -265,7 +273,9 @@ def measure_next_rows(tg, dev, st, flush, main, peaks, reps=10):
     from workloads import masked_budgets
 
     lib = tg.load()
-    sh = st.cuda_stream
+
+    def sh_now():  # the current stream (the capture stream while a call is recorded)
+        return torch.cuda.current_stream(dev).cuda_stream
 
     def bf16(bits):
         return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
@@ -299,7 +309,7 @@ def measure_next_rows(tg, dev, st, flush, main, peaks, reps=10):
     us = time_device_us(check(lambda: lib.tg_masked_gated_attention(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), s.data_ptr(), cu_d.data_ptr(), sp_d.data_ptr(), kb_d.data_ptr(),
         ck_d.data_ptr(), w.B, w.T, Mm, maxm, w.Hq, w.Hkv, w.d, g.data_ptr(), c.data_ptr(), 1.0 / math.sqrt(w.d),
-        out.data_ptr(), keep.data_ptr(), mws.data_ptr(), mws.numel(), sh)), st, flush, reps)
+        out.data_ptr(), keep.data_ptr(), mws.data_ptr(), mws.numel(), sh_now())), st, flush, reps)
     res["f1_masked_attention"] = {"workload": f"{w.name}: N={w.T}, K'={int(kb[0])} (log-uniform in [1, |P|/2]), M={Mm}",
                                   "us": us, "kept_pair_tflops": fl / (us * 1e-6) / 1e12,
                                   "includes": "zero fill of pruned rows + select map + Q/K/V row gather + attention "
@@ -311,7 +321,7 @@ def measure_next_rows(tg, dev, st, flush, main, peaks, reps=10):
     kdst = torch.empty((main["M"], wm.Hkv, wm.d), dtype=torch.bfloat16, device=dev)
     row_bytes = wm.Hkv * wm.d * 2
     us = time_device_us(check(lambda: lib.tg_gather_rows(kcache.data_ptr(), wm.T, row_bytes,
-                                                         main["kept_idx"].data_ptr(), main["M"], kdst.data_ptr(), sh)),
+                                                         main["kept_idx"].data_ptr(), main["M"], kdst.data_ptr(), sh_now())),
                         st, flush, reps)
     nbytes = 2 * main["M"] * row_bytes
     res["f2_kv_gather"] = {"workload": f"{wm.name}: K cache [{wm.T}, {wm.Hkv}, {wm.d}] bf16 -> {main['M']} rows",
@@ -334,7 +344,7 @@ def measure_next_rows(tg, dev, st, flush, main, peaks, reps=10):
     us = time_device_us(check(lambda: lib.tg_gated_attention(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), ck_d.data_ptr(), w.B, M, maxM, w.Hq, w.Hkv, w.d,
         cmap["pos"].data_ptr(), cmap["rank"].data_ptr(), cmap["gls"].data_ptr(), g.data_ptr(), c.data_ptr(),
-        1.0 / math.sqrt(w.d), out.data_ptr(), None, None, 0, sh)), st, flush, reps)
+        1.0 / math.sqrt(w.d), out.data_ptr(), None, None, 0, sh_now())), st, flush, reps)
     res["f3_hd256_attention"] = {"workload": f"{w.name}: M={M}, Hq={w.Hq}, Hkv={w.Hkv}, d={w.d}", "us": us,
                                  "tflops": fl / (us * 1e-6) / 1e12,
                                  "frac_of_bf16_peak": fl / (us * 1e-6) / 1e12 / tc_peak}
@@ -355,11 +365,11 @@ def measure_next_rows(tg, dev, st, flush, main, peaks, reps=10):
     common = (L0["q"].data_ptr(), L0["k"].data_ptr(), L0["v"].data_ptr(), ck_d.data_ptr(), wm.B, main["M"],
               main["max_M"], wm.Hq, wm.Hkv, wm.d, bufs.pos.data_ptr(), bufs.rank.data_ptr())
     us = time_device_us(check(lambda: lib.tg_gated_attention_gates(*common, 4, gls_arr, g_arr, L0["c"].data_ptr(), sm,
-                                                                   out.data_ptr(), None, ws_p, ws_n, sh)),
+                                                                   out.data_ptr(), None, ws_p, ws_n, sh_now())),
                         st, flush, reps)
     us1 = time_device_us(check(lambda: lib.tg_gated_attention(*common, bufs.gls.data_ptr(), L0["g"].data_ptr(),
                                                               L0["c"].data_ptr(), sm, out.data_ptr(), None, ws_p,
-                                                              ws_n, sh)), st, flush, reps)
+                                                              ws_n, sh_now())), st, flush, reps)
     res["f4_four_gates_attention"] = {"workload": f"{wm.name}: M={main['M']}, 4 gates", "us": us,
                                       "tflops": fl / (us * 1e-6) / 1e12, "one_gate_us": us1,
                                       "vs_one_gate": us / us1}
@@ -367,7 +377,7 @@ def measure_next_rows(tg, dev, st, flush, main, peaks, reps=10):
     # forward's output and log-sum-exp
     lse = torch.empty((main["M"], wm.Hq), dtype=torch.float32, device=dev)
     assert lib.tg_gated_attention(*common, bufs.gls.data_ptr(), L0["g"].data_ptr(), L0["c"].data_ptr(), sm,
-                                  out.data_ptr(), lse.data_ptr(), ws_p, ws_n, sh) == 0
+                                  out.data_ptr(), lse.data_ptr(), ws_p, ws_n, sh_now()) == 0
     dout = torch.randn((main["M"], wm.Hq, wm.d), device=dev).to(torch.bfloat16)
     grads = [torch.empty_like(L0["q"]), torch.empty_like(L0["k"]), torch.empty_like(L0["v"])]
     f32 = [torch.empty(main["M"], dtype=torch.float32, device=dev) for _ in range(2)] + \
@@ -379,7 +389,7 @@ def measure_next_rows(tg, dev, st, flush, main, peaks, reps=10):
         ck_d.data_ptr(), wm.B, main["M"], main["max_M"], wm.Hq, wm.Hkv, wm.d, bufs.pos.data_ptr(),
         bufs.rank.data_ptr(), bufs.gls.data_ptr(), L0["g"].data_ptr(), L0["c"].data_ptr(), sm, grads[0].data_ptr(),
         grads[1].data_ptr(), grads[2].data_ptr(), f32[0].data_ptr(), f32[1].data_ptr(), f32[2].data_ptr(),
-        f32[3].data_ptr(), bws.data_ptr(), bws.numel(), sh)), st, flush, reps)
+        f32[3].data_ptr(), bws.data_ptr(), bws.numel(), sh_now())), st, flush, reps)
     res["f1_attention_backward"] = {"workload": f"{wm.name}: M={main['M']}, Hq={wm.Hq}, Hkv={wm.Hkv}, d={wm.d}",
                                     "us": us, "tflops": 2.5 * fl / (us * 1e-6) / 1e12,
                                     "frac_of_bf16_peak": 2.5 * fl / (us * 1e-6) / 1e12 / tc_peak,
@@ -428,7 +438,10 @@ def run_gpu(args, w):
             dist.barrier()
 
     lib = tg.load()
-    sh = st.cuda_stream
+
+    def sh_now():  # the current stream (a capture stream while a stage graph is recorded)
+        return torch.cuda.current_stream(dev).cuda_stream
+
     B, T, D, I = w.B, w.T, w.D, w.I
     sm_scale = 1.0 / math.sqrt(w.d)
     L0 = layers[0]
@@ -438,18 +451,18 @@ def run_gpu(args, w):
     stage_calls = {
         "score": lambda: lib.tg_score(hidden.data_ptr(), call.cu.data_ptr(), call.sp.data_ptr(), B, T, D,
                                       Wg.data_ptr(), b1.data_ptr(), w2.data_ptr(), float(gi["b2"]), I, float(w.eps),
-                                      bufs.scores.data_ptr(), sh),
+                                      bufs.scores.data_ptr(), sh_now()),
         "select": lambda: lib.tg_select_topk(bufs.scores.data_ptr(), call.cu.data_ptr(), call.sp.data_ptr(),
                                              call.kk.data_ptr(), B, T, bufs.keep.data_ptr(), call.ck.data_ptr(),
                                              bufs.kept_idx.data_ptr(), bufs.pos.data_ptr(), bufs.rank.data_ptr(),
-                                             bufs.gls.data_ptr(), sh),
+                                             bufs.gls.data_ptr(), sh_now()),
         "gather": lambda: lib.tg_compact(hidden.data_ptr(), None, None, None, None, B, T, D, None, M,
-                                         bufs.hidden_kept.data_ptr(), None, None, None, bufs.kept_idx.data_ptr(), sh),
+                                         bufs.hidden_kept.data_ptr(), None, None, None, bufs.kept_idx.data_ptr(), sh_now()),
         "attention": lambda: lib.tg_gated_attention(L0["q"].data_ptr(), L0["k"].data_ptr(), L0["v"].data_ptr(),
                                                     call.ck.data_ptr(), B, M, call.max_M, w.Hq, w.Hkv, w.d,
                                                     bufs.pos.data_ptr(), bufs.rank.data_ptr(), bufs.gls.data_ptr(),
                                                     L0["g"].data_ptr(), L0["c"].data_ptr(), sm_scale,
-                                                    bufs.out[0].data_ptr(), None, _ws_ptr, _ws_n, sh),
+                                                    bufs.out[0].data_ptr(), None, _ws_ptr, _ws_n, sh_now()),
     }
 
     # warm-up (also sets kernel attributes before any capture)
@@ -484,15 +497,26 @@ def run_gpu(args, w):
     barrier()
     step_ms = [a.elapsed_time(b) for a, b in ev]
 
-    # ---------------- per-stage breakdown over K more steps (same stream, same kernels)
+    # ---------------- per-stage breakdown over K more steps (same stream, same kernels); each
+    # stage replays a one-call CUDA graph, so that no host work (argument checks, tensor-map
+    # encoding) sits between the events around it
     names = list(stage_calls)
+    stage_graphs = {}
+    if not args.no_graph:
+        for nm in names:
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr):
+                assert stage_calls[nm]() == 0
+            stage_graphs[nm] = gr
+        torch.cuda.synchronize(dev)
+    run_stage = {nm: (stage_graphs[nm].replay if nm in stage_graphs else stage_calls[nm]) for nm in names}
     sev = {s: [] for s in names}
     for i in range(args.steps):
         flush.fill_(i)
         e = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
         e[0].record(st)
         for n_i, nm in enumerate(names):
-            stage_calls[nm]()
+            run_stage[nm]()
             e[n_i + 1].record(st)
         for n_i, nm in enumerate(names):
             sev[nm].append((e[n_i], e[n_i + 1]))
