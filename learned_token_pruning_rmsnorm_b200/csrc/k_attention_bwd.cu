@@ -245,21 +245,36 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
         int t = 0;
         {
             const float beta = softplus_b(g[h]);
+            const float ch = c[h];
             float csum = 0.f;
+            // this thread's query row of the next tile: pos, rank, lse and D' are loaded one
+            // step ahead (their latency hides behind a step of work)
+            int npos = 1, nrank = 1;
+            float nlse = 0.f, nD = 0.f;
+            auto load_row = [&](int i) {
+                const int qrow = i * BT + r;
+                if (qrow < Mb) {
+                    const int qg = seq0 + qrow;
+                    npos = __ldcg(pos + qg);
+                    nrank = __ldcg(rank + qg);
+                    nlse = __ldcg(lse + static_cast<size_t>(qg) * Hq + h);
+                    nD = __ldcg(Drow + static_cast<size_t>(qg) * Hq + h);
+                }
+            };
+            load_row(kt);
             for (int ii = 0; ii < nq; ++ii, ++t) {
                 const int i = kt + ii, s = t & 1;
                 // this thread's query row of tile i fills one column of the factor table
                 const int qrow = i * BT + r;
                 float fa = 0.f, fb = 0.f, fl = 0.f, fd = 0.f, fi = 0.f;
                 if (qrow < Mb) {
-                    const int qg = seq0 + qrow;
-                    fi = 1.0f / (1.0f + c[h] * logf(static_cast<float>(__ldcg(pos + qg)) /
-                                                    static_cast<float>(__ldcg(rank + qg))));
+                    fi = 1.0f / (1.0f + ch * logf(static_cast<float>(npos) / static_cast<float>(nrank)));
                     fa = sm_scale * LOG2E_B * fi;
                     fb = beta * LOG2E_B * fi;
-                    fl = lse[static_cast<size_t>(qg) * Hq + h] * LOG2E_B;
-                    fd = __ldcg(Drow + static_cast<size_t>(qg) * Hq + h);
+                    fl = nlse * LOG2E_B;
+                    fd = nD;
                 }
+                if (ii + 1 < nq) load_row(i + 1);
                 float* ps = par + s * 5 * BT;
                 ps[0 * BT + r] = fa;
                 ps[1 * BT + r] = fb;
@@ -382,13 +397,15 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
 // dQ and the per-query sums: one CTA per (query head, 128-query tile, sequence),
 // heaviest causal tiles first.
 //
-// 192 threads: warps 0-3 compute (thread r = query row r = TMEM lane), warp 4
-// TMA producer (Q and dO once, K/V tiles through a two-stage ring), warp 5 MMA
-// issuer.  TMEM: S | dP | dQ.  Per KV tile j the issuer waits for G(j-1),
-// accumulates dQ += G(j-1) K(j-1) from TMEM and then issues S(j) = Q K(j)^T and
-// dP(j) = dO V(j)^T.  The compute warps rebuild P from the log-sum-exp, form
-// G = P (dP - D) / tau, store it as bf16 over the first 64 columns of S and sum,
-// along their own row, G gls (for dbeta) and dl l (for dtau).
+// 320 threads: warps 0-7 compute (warps w and w + 4 share query rows 32 w .. + 31,
+// the TMEM lanes of that quarter, and split each half tile's keys), warp 8 TMA
+// producer (Q and dO once, K/V tiles through a two-stage ring), warp 9 MMA issuer.
+// TMEM: two (S | dP) buffers of half a KV tile (64 keys) and dQ.  The issuer puts
+// out S and dP of one half while the compute warps turn the other half into G,
+// then accumulates dQ += G K from TMEM.  The compute warps rebuild P from the
+// log-sum-exp, form tau G = P (dP - D) (1/tau scales dQ's rows at the end), store
+// it as bf16 over the first 32 columns of the half's S and sum, along their own
+// row, G gls (for dbeta) and dl l (for dtau).
 template <int HD>
 struct DqSmem {
     static constexpr int TILE = BT * HD * 2;
@@ -396,8 +413,9 @@ struct DqSmem {
     static constexpr int OFF_DO = OFF_Q + TILE;
     static constexpr int OFF_K = OFF_DO + TILE;        // [2 stages]
     static constexpr int OFF_V = OFF_K + 2 * TILE;     // [2 stages]
-    static constexpr int OFF_GLS = OFF_V + 2 * TILE;   // [4 warps][2][BT] fp32, a private copy per warp
-    static constexpr int OFF_BAR = OFF_GLS + 4 * 2 * BT * 4;
+    static constexpr int OFF_GLS = OFF_V + 2 * TILE;   // [8 warps][2][BT] fp32, a private copy per warp
+    static constexpr int OFF_XCH = OFF_GLS + 8 * 2 * BT * 4;  // [6][BT] fp32: the second column half's row sums
+    static constexpr int OFF_BAR = OFF_XCH + 6 * BT * 4;
     static constexpr int NUM_BARS = 16;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;  // tmem slot, abort flag, then 8 fp32
     static constexpr int BYTES = OFF_MISC + 16 + 32;
@@ -408,12 +426,26 @@ struct DqSmem {
 };
 
 enum : int {
-    Q_QD_FULL = 0, Q_K_FULL = 1, Q_K_EMPTY = 3, Q_V_FULL = 5, Q_V_EMPTY = 7, Q_SDP_FULL = 9, Q_G_FULL = 10,
-    Q_DQ_DONE = 11, Q_DRAIN = 12
+    Q_QD_FULL = 0, Q_K_FULL = 1, Q_K_EMPTY = 3, Q_V_FULL = 5, Q_V_EMPTY = 7, Q_SDP_FULL = 9, Q_G_FULL = 11,
+    Q_DQ_DONE = 13, Q_DRAIN = 14
 };
 
+constexpr int DQ_THREADS = 320;  // warps 0-7 compute, 8 TMA producer, 9 MMA issuer
+
+// bar.red.or over the two compute warps of one row group (named barrier 2 + q4, 64 threads)
+__device__ __forceinline__ bool pair_red_or(int id, bool pred) {
+    uint32_t res;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, %2, 64, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(res)
+        : "r"(static_cast<uint32_t>(pred)), "r"(id)
+        : "memory");
+    return res != 0;
+}
+
 template <int HD>
-__global__ void __launch_bounds__(BWD_THREADS, 1)
+__global__ void __launch_bounds__(DQ_THREADS, 1)
 gated_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                          const int32_t* __restrict__ cu_kept, const int32_t* __restrict__ pos,
@@ -451,14 +483,16 @@ gated_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
             mbar_init(bar(Q_V_FULL + s), 1);
             mbar_init(bar(Q_V_EMPTY + s), 1);
         }
-        mbar_init(bar(Q_SDP_FULL), 1);
-        mbar_init(bar(Q_G_FULL), 128);
+        for (int hb = 0; hb < 2; ++hb) {
+            mbar_init(bar(Q_SDP_FULL + hb), 1);
+            mbar_init(bar(Q_G_FULL + hb), 256);  // every thread of the eight compute warps
+        }
         mbar_init(bar(Q_DQ_DONE), 1);
         mbar_init(bar(Q_DRAIN), 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 4) {
+    if (warp == 8) {
         tmem_alloc(smem_u32(tmem_slot), L::TMEM_COLS);
         tmem_relinquish();
     }
@@ -466,9 +500,11 @@ gated_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS = tmem, tDP = tmem + BT, tDQ = tmem + 2 * BT;
+    // two half-tile buffers: half hb of a KV tile (keys 64 hb .. 64 hb + 63) keeps S at
+    // columns [128 hb, +64) and dP at [128 hb + 64, +64); dQ follows
+    const uint32_t tDQ = tmem + 2 * BT;
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ---------------------------------------------------------------- TMA producer
         if (lane == 0) {
             prefetch_tmap(&tmQ);
@@ -511,60 +547,87 @@ gated_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
                 }
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == 9) {
         // ---------------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc_s = idesc_bf16_f32(BT, BT, false);
+            constexpr uint32_t idesc_s = idesc_bf16_f32(BT, 64, false);
             constexpr uint32_t idesc_acc = idesc_bf16_f32(BT, HD, true);
-            // dQ += G(jj) K(jj): A from TMEM (16 keys = 8 columns per k-step), B the K tile MN-major
-            auto issue_dq = [&](int jj) {
-                const int s = jj & 1;
+            // Half step u: KV tile u >> 1, keys 64 (u & 1) .. +63 (64 rows = 8 KB into each
+            // swizzled box), TMEM buffer u & 1.  S(u) and dP(u) go out before dQ(u - 1), so the
+            // tensor core computes half u while the compute warps turn half u - 1 into G; the
+            // buffer S(u) overwrites last held G(u - 2), which dQ(u - 2) -- issued earlier by this
+            // thread, so executed earlier -- has read.
+            auto issue_sdp = [&](int u) {
+                const int hb = u & 1, s = (u >> 1) & 1;
+                const uint32_t tb = tmem + hb * 128;
 #pragma unroll
-                for (int kk = 0; kk < BT / 16; ++kk)
-                    mma_bf16_ts(tDQ, tS + kk * 8, smem_desc_sw128(sK + s * L::TILE + kk * 16 * 128, BT * 128, 1024),
-                                idesc_acc, (jj > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(bar(Q_K_EMPTY + s));
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * (BT * 128) + (kk & 3) * 32;
+                    mma_bf16_ss(tb, smem_desc_sw128(sQ + off, 16, 1024),
+                                smem_desc_sw128(sK + s * L::TILE + hb * 64 * 128 + off, 16, 1024), idesc_s,
+                                kk > 0 ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * (BT * 128) + (kk & 3) * 32;
+                    mma_bf16_ss(tb + 64, smem_desc_sw128(sDO + off, 16, 1024),
+                                smem_desc_sw128(sV + s * L::TILE + hb * 64 * 128 + off, 16, 1024), idesc_s,
+                                kk > 0 ? 1u : 0u);
+                }
+                mma_commit(bar(Q_SDP_FULL + hb));
+                if (hb == 1) mma_commit(bar(Q_V_EMPTY + s));  // V(tile) is no longer read
             };
+            // dQ += G(u) K(half of u): A from TMEM (16 keys = 8 columns per k-step), B the K rows MN-major
+            auto issue_dq = [&](int u) {
+                const int hb = u & 1, s = (u >> 1) & 1;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16_ts(tDQ, tmem + hb * 128 + kk * 8,
+                                smem_desc_sw128(sK + s * L::TILE + (hb * 64 + kk * 16) * 128, BT * 128, 1024),
+                                idesc_acc, (u > 0 || kk > 0) ? 1u : 0u);
+                if (hb == 1) mma_commit(bar(Q_K_EMPTY + s));  // K(tile) is no longer read
+            };
+            const int n_u = 2 * n_kv;
             bool ok = mbar_wait(bar(Q_QD_FULL), 0, abort_flag, status, TG_WHERE_MMA);
-            for (int j = 0; ok && j < n_kv; ++j) {
-                const int s = j & 1;
-                ok = mbar_wait(bar(Q_K_FULL + s), (j >> 1) & 1, abort_flag, status, TG_WHERE_MMA);
-                if (ok) ok = mbar_wait(bar(Q_V_FULL + s), (j >> 1) & 1, abort_flag, status, TG_WHERE_MMA);
-                if (ok && j >= 1) ok = mbar_wait(bar(Q_G_FULL), (j - 1) & 1, abort_flag, status, TG_WHERE_MMA);
-                if (!ok) break;
+            for (int u = 0; ok && u < n_u; ++u) {
+                const int j = u >> 1, s = j & 1;
+                if ((u & 1) == 0) {
+                    ok = mbar_wait(bar(Q_K_FULL + s), (j >> 1) & 1, abort_flag, status, TG_WHERE_MMA);
+                    if (ok) ok = mbar_wait(bar(Q_V_FULL + s), (j >> 1) & 1, abort_flag, status, TG_WHERE_MMA);
+                    if (!ok) break;
+                }
                 tc_fence_after();
-                if (j >= 1) issue_dq(j - 1);
-#pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * (BT * 128) + (kk & 3) * 32;
-                    mma_bf16_ss(tS, smem_desc_sw128(sQ + off, 16, 1024),
-                                smem_desc_sw128(sK + s * L::TILE + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+                issue_sdp(u);
+                if (u >= 1) {
+                    ok = mbar_wait(bar(Q_G_FULL + ((u - 1) & 1)), ((u - 1) >> 1) & 1, abort_flag, status,
+                                   TG_WHERE_MMA);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_dq(u - 1);
                 }
-#pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * (BT * 128) + (kk & 3) * 32;
-                    mma_bf16_ss(tDP, smem_desc_sw128(sDO + off, 16, 1024),
-                                smem_desc_sw128(sV + s * L::TILE + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
-                }
-                mma_commit(bar(Q_SDP_FULL));
-                mma_commit(bar(Q_V_EMPTY + s));
             }
-            if (ok) ok = mbar_wait(bar(Q_G_FULL), (n_kv - 1) & 1, abort_flag, status, TG_WHERE_MMA);
+            if (ok) ok = mbar_wait(bar(Q_G_FULL + ((n_u - 1) & 1)), ((n_u - 1) >> 1) & 1, abort_flag, status,
+                                   TG_WHERE_MMA);
             if (ok) {
                 tc_fence_after();
-                issue_dq(n_kv - 1);
+                issue_dq(n_u - 1);
                 mma_commit(bar(Q_DQ_DONE));
             }
             mma_commit(bar(Q_DRAIN));
             drain_wait_b(bar(Q_DRAIN), 0, status);
         }
     } else {
-        // ---------------------------------------------------------------- compute warps 0-3
-        const int r = threadIdx.x;  // query row of the tile == TMEM lane
+        // ---------------------------------------------------------------- compute warps 0-7
+        // Warp w owns query rows 32 (w & 3) .. + 31 (TMEM lanes) and the keys
+        // 32 (w >> 2) .. + 31 of each 64-key half step; the two warps of a row group meet
+        // at a 64-thread reducing barrier once per half step (each stores G over S columns
+        // the other reads) and combine their row sums once at the end.
+        const int q4 = warp & 3, cs = warp >> 2;
+        const int r = q4 * 32 + lane;  // query row of the tile == TMEM lane
         const int q_local = qt * BT + r;
         const bool valid_row = q_local < Mb;
         const int qg = seq0 + q_local;
-        const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+        const uint32_t lane_addr = static_cast<uint32_t>(q4 * 32) << 16;
         float fa = 0.f, fb = 0.f, fl = 0.f, fd = 0.f, fi = 0.f, lr = 0.f;
         if (valid_row) {
             lr = logf(static_cast<float>(__ldcg(pos + qg)) / static_cast<float>(__ldcg(rank + qg)));
@@ -573,9 +636,11 @@ gated_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
             fb = softplus_b(g[h]) * LOG2E_B * fi;
             fl = __ldcg(lse + static_cast<size_t>(qg) * Hq + h) * LOG2E_B;
         }
-        // D = dout . out of this row, with dout from the staged tile (128-byte swizzled boxes of
-        // 64 columns) and out, the forward's output, from global memory
+        // D = dout . out of this row (both warps of the row group form it), with dout from the
+        // staged tile (128-byte swizzled boxes of 64 columns) and out, the forward's output,
+        // from global memory
         bool ok = mbar_wait_warp(bar(Q_QD_FULL), 0, abort_flag, status, TG_WHERE_SOFTMAX);
+        ok = !pair_red_or(2 + q4, !ok);
         if (ok && valid_row) {
             const uint16_t* orow = out_fwd + (static_cast<size_t>(qg) * Hq + h) * HD;
             float acc = 0.f;
@@ -600,105 +665,137 @@ gated_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
         // D above comes from the bf16 output; dtau = -sum_j dl l / tau cancels to a small
         // number and would amplify its rounding):  sum_j dl x = sum P dP x - D' sum P x.
         float aPdPt = 0.f, aPt = 0.f, aPdP = 0.f, aP = 0.f, aPdPg = 0.f, aPg = 0.f;
+        // gls of the next KV tile is loaded one tile ahead (its latency hides behind a tile of work)
+        float gnext[BT / 32];
+#pragma unroll
+        for (int e = 0; e < BT / 32; ++e) gnext[e] = e * 32 + lane < Mb ? __ldcg(gls + seq0 + e * 32 + lane) : 0.f;
         for (int j = 0; ok && j < n_kv; ++j) {
             const int s = j & 1;
             // the tile's gls into this warp's own copy (only __syncwarp orders it)
 #pragma unroll
-            for (int e = 0; e < BT / 32; ++e) {
-                const int key_local = j * BT + e * 32 + lane;
-                wgls[s * BT + e * 32 + lane] = key_local < Mb ? __ldcg(gls + seq0 + key_local) : 0.f;
-            }
+            for (int e = 0; e < BT / 32; ++e) wgls[s * BT + e * 32 + lane] = gnext[e];
             __syncwarp();
-            ok = mbar_wait_warp(bar(Q_SDP_FULL), j & 1, abort_flag, status, TG_WHERE_SOFTMAX);
-            if (!ok) break;
-            tc_fence_after();
+            if (j + 1 < n_kv) {
+#pragma unroll
+                for (int e = 0; e < BT / 32; ++e) {
+                    const int key_local = (j + 1) * BT + e * 32 + lane;
+                    gnext[e] = key_local < Mb ? __ldcg(gls + seq0 + key_local) : 0.f;
+                }
+            }
             const bool diag = (j == n_kv - 1);
             const int lim = q_local - j * BT;  // on the diagonal tile, columns > lim are future keys
             const float* bl = wgls + s * BT;
 #pragma unroll 1
             for (int half = 0; half < 2; ++half) {
-                float sx[64], dpx[64];
-                tmem_ld32(tS + lane_addr + half * 64, sx);
-                tmem_ld32(tS + lane_addr + half * 64 + 32, sx + 32);
-                tmem_ld32(tDP + lane_addr + half * 64, dpx);
-                tmem_ld32(tDP + lane_addr + half * 64 + 32, dpx + 32);
-                tmem_wait_ld();
-                uint32_t gg[32];
+                const bool okw = mbar_wait_warp(bar(Q_SDP_FULL + half), j & 1, abort_flag, status, TG_WHERE_SOFTMAX);
+                const uint32_t tb = tmem + lane_addr + half * 128;
+                float sx[32], dpx[32];
+                if (okw) {
+                    tc_fence_after();
+                    tmem_ld32(tb + cs * 32, sx);
+                    tmem_ld32(tb + 64 + cs * 32, dpx);
+                    tmem_wait_ld();
+                }
+                // both warps of the row group have read their columns of S (the G stores below
+                // overwrite some of the partner's); an abort is decided by the pair together
+                if (pair_red_or(2 + q4, !okw)) {
+                    ok = false;
+                    break;
+                }
+                uint32_t gg[16];
 #pragma unroll
-                for (int cc = 0; cc < 64; cc += 2) {
+                for (int cc = 0; cc < 32; cc += 2) {
                     float gv[2];
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
-                        const int col = half * 64 + cc + e;
+                        const int col = half * 64 + cs * 32 + cc + e;
                         const float glj = bl[col];
                         const float tt = fmaf(fa, sx[cc + e], fmaf(fb, glj, -fl));
                         const bool keep = valid_row && !(diag && col > lim);
+                        // masked and padded entries have p = 0 and finite tt, glj: they add nothing
                         const float p = keep ? ex2_approx(tt) : 0.f;
-                        const float G = p * (dpx[cc + e] - fd) * fi;
-                        if (p > 0.f) {
-                            const float pdp = p * dpx[cc + e];
-                            aPdPt = fmaf(pdp, tt, aPdPt);
-                            aPt = fmaf(p, tt, aPt);
-                            aPdP += pdp;
-                            aP += p;
-                            aPdPg = fmaf(pdp, glj, aPdPg);
-                            aPg = fmaf(p, glj, aPg);
-                        }
-                        gv[e] = G;
+                        const float pdp = p * dpx[cc + e];
+                        aPdPt = fmaf(pdp, tt, aPdPt);
+                        aPt = fmaf(p, tt, aPt);
+                        aPdP += pdp;
+                        aP += p;
+                        aPdPg = fmaf(pdp, glj, aPdPg);
+                        aPg = fmaf(p, glj, aPg);
+                        gv[e] = pdp - p * fd;  // G tau = P (dP - D); 1/tau is applied to dQ's rows
                     }
                     gg[cc / 2] = pack2_bf16(gv[0], gv[1]);
                 }
-                tmem_st32u(tS + lane_addr + half * 32, gg);  // G over the (already read) first columns of S
+                tmem_st16u(tb + cs * 16, gg);  // G of these 32 keys as bf16 pairs over S
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar(Q_G_FULL + half));
             }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(bar(Q_G_FULL));
         }
         // ---------------------------------------------------------------- epilogue
         if (ok) ok = mbar_wait_warp(bar(Q_DQ_DONE), 0, abort_flag, status, TG_WHERE_SOFTMAX);
         if (ok) {
             tc_fence_after();
-            uint16_t* dst = dq + (static_cast<size_t>(qg) * Hq + h) * HD;
+            const float rs = sm_scale * fi;
+            uint16_t* dst = dq + (static_cast<size_t>(qg) * Hq + h) * HD + cs * (HD / 2);
 #pragma unroll
-            for (int ch = 0; ch < HD / 32; ++ch) {
+            for (int ch = 0; ch < HD / 64; ++ch) {
                 float o[32];
-                tmem_ld32(tDQ + lane_addr + ch * 32, o);
+                tmem_ld32(tDQ + lane_addr + cs * (HD / 2) + ch * 32, o);
                 tmem_wait_ld();
                 if (valid_row) {
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
+                    for (int q8 = 0; q8 < 4; ++q8) {
                         uint4 w;
-                        w.x = pack2_bf16(o[q4 * 8 + 0] * sm_scale, o[q4 * 8 + 1] * sm_scale);
-                        w.y = pack2_bf16(o[q4 * 8 + 2] * sm_scale, o[q4 * 8 + 3] * sm_scale);
-                        w.z = pack2_bf16(o[q4 * 8 + 4] * sm_scale, o[q4 * 8 + 5] * sm_scale);
-                        w.w = pack2_bf16(o[q4 * 8 + 6] * sm_scale, o[q4 * 8 + 7] * sm_scale);
-                        *reinterpret_cast<uint4*>(dst + ch * 32 + q4 * 8) = w;
+                        w.x = pack2_bf16(o[q8 * 8 + 0] * rs, o[q8 * 8 + 1] * rs);
+                        w.y = pack2_bf16(o[q8 * 8 + 2] * rs, o[q8 * 8 + 3] * rs);
+                        w.z = pack2_bf16(o[q8 * 8 + 4] * rs, o[q8 * 8 + 5] * rs);
+                        w.w = pack2_bf16(o[q8 * 8 + 6] * rs, o[q8 * 8 + 7] * rs);
+                        *reinterpret_cast<uint4*>(dst + ch * 32 + q8 * 8) = w;
                     }
                 }
             }
-            if (valid_row) Drow[static_cast<size_t>(qg) * Hq + h] = aPdP;  // the exact D' for the dK/dV kernel
         }
+        // the second column half's row sums join the first's (all eight warps, abort or not)
+        float* xch = reinterpret_cast<float*>(smem + L::OFF_XCH);
+        if (cs == 1) {
+            xch[0 * BT + r] = aPdPt;
+            xch[1 * BT + r] = aPt;
+            xch[2 * BT + r] = aPdP;
+            xch[3 * BT + r] = aP;
+            xch[4 * BT + r] = aPdPg;
+            xch[5 * BT + r] = aPg;
+        }
+        asm volatile("bar.sync 1, 256;" ::: "memory");
         // this tile's terms of dbeta_h (sum_i sum_j G gls_j) and dc_h (sum_i ln(pos/rank) dtau),
         // summed over its rows in a fixed order and stored at the tile's first row
         float eE = 0.f, eT = 0.f;
-        if (ok && valid_row) {
-            const float Dx = aPdP;
-            // tt = l log2(e) - lse log2(e):  sum dl l = ln2 (sum dl tt + lse log2(e) sum dl)
-            const float sum_dl_t = aPdPt - Dx * aPt + fl * (aPdP - Dx * aP);
-            eE = fi * (aPdPg - Dx * aPg);
-            eT = lr * (-LN2_B * fi * sum_dl_t);
-        }
+        if (cs == 0) {
+            aPdPt += xch[0 * BT + r];
+            aPt += xch[1 * BT + r];
+            aPdP += xch[2 * BT + r];
+            aP += xch[3 * BT + r];
+            aPdPg += xch[4 * BT + r];
+            aPg += xch[5 * BT + r];
+            if (ok && valid_row) {
+                const float Dx = aPdP;
+                // tt = l log2(e) - lse log2(e):  sum dl l = ln2 (sum dl tt + lse log2(e) sum dl)
+                const float sum_dl_t = aPdPt - Dx * aPt + fl * (aPdP - Dx * aP);
+                eE = fi * (aPdPg - Dx * aPg);
+                eT = lr * (-LN2_B * fi * sum_dl_t);
+                Drow[static_cast<size_t>(qg) * Hq + h] = Dx;  // the exact D' for the dK/dV kernel
+            }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            eE += __shfl_xor_sync(0xffffffffu, eE, o);
-            eT += __shfl_xor_sync(0xffffffffu, eT, o);
+            for (int o = 16; o > 0; o >>= 1) {
+                eE += __shfl_xor_sync(0xffffffffu, eE, o);
+                eT += __shfl_xor_sync(0xffffffffu, eT, o);
+            }
         }
         float* red = reinterpret_cast<float*>(smem + L::OFF_MISC + 16);
-        if (lane == 0) {
-            red[warp] = eE;
-            red[4 + warp] = eT;
+        if (cs == 0 && lane == 0) {
+            red[q4] = eE;
+            red[4 + q4] = eT;
         }
-        asm volatile("bar.sync 1, 128;" ::: "memory");  // the four compute warps, abort or not
+        asm volatile("bar.sync 1, 256;" ::: "memory");
         if (threadIdx.x == 0 && ok) {
             const size_t slot = (static_cast<size_t>(seq0) + static_cast<size_t>(qt) * BT) * Hq + h;
             tileE[slot] = (red[0] + red[1]) + (red[2] + red[3]);
@@ -708,7 +805,7 @@ gated_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 4) {
+    if (warp == 8) {
         tc_fence_after();
         tmem_dealloc(tmem, L::TMEM_COLS);
     }
@@ -831,7 +928,7 @@ cudaError_t launch_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
     const int n_t = (max_M + BT - 1) / BT;
     // dq first: it forms each row's D = dout . out for its own use and leaves the exact
     // D' = sum_j P dP for the dK/dV kernel
-    cudaError_t e = launch_pdl(gated_attn_bwd_dq_kernel<HD>, dim3(Hq, n_t, B), dim3(BWD_THREADS),
+    cudaError_t e = launch_pdl(gated_attn_bwd_dq_kernel<HD>, dim3(Hq, n_t, B), dim3(DQ_THREADS),
                                static_cast<size_t>(DqSmem<HD>::ALLOC), st, tq, tk, tv, tdo, cu_kept, pos, rank, gls, g,
                                c, lse, out, Drow, sm_scale, Hq, Hkv, n_t, dq, tileE, tileT, status);
     if (e != cudaSuccess) return e;
