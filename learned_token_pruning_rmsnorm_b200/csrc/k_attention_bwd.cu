@@ -15,10 +15,10 @@
 //
 // Three or four launches, no atomics (results do not depend on scheduling):
 //   dq       (below; it also forms D_ih = dout_i.out_i for its rows)
-//   dkv      one CTA per (query head, 128-key tile): for every causal query
-//            tile, S^T = K Q^T and dP^T = V dO^T
+//   dkv      one CTA per (query head, 128-key tile): for every half (64
+//            queries) of every causal query tile, S^T = K Q^T and dP^T = V dO^T
 //            on the tensor core (TMEM lanes = keys), then P^T and G^T as bf16
-//            over the first 64 columns of S^T and dP^T, and dV += P^T dO,
+//            over the first 32 columns of S^T and dP^T, and dV += P^T dO,
 //            dK += G^T Q read from TMEM.  The per-key sums of G (the gate
 //            bias's gradient, per head) are sums along each thread's own row.
 //            The query heads of a GQA group leave fp32 partials of dK / dV that
@@ -40,7 +40,6 @@ namespace {
 using namespace sm100;
 
 constexpr int BT = 128;  // rows of a query or key tile (= TMEM lanes)
-constexpr int BWD_THREADS = 192;
 constexpr float LOG2E_B = 1.4426950408889634f;
 constexpr float LN2_B = 0.6931471805599453f;
 
@@ -57,28 +56,57 @@ __device__ __forceinline__ bool drain_wait_b(uint32_t bar, uint32_t parity, int*
 }
 
 // ---------------------------------------------------------------------------
-// dK, dV and the per-key sums of G: one CTA per (KV head, 128-key tile, sequence).
+// dK, dV and the per-key sums of G: one CTA per (query head, 128-key tile, sequence).
 //
-// 192 threads: warps 0-3 compute (thread r = key row r of the tile = TMEM lane),
-// warp 4 TMA producer, warp 5 MMA issuer.  The K and V tiles stay resident; the
-// (Q, dO) tiles of every (query head of the group, causal query tile) stream
-// through a two-stage ring.  TMEM (512 columns): S^T | dP^T | dV | dK.  Per step
-// the issuer waits for the compute warps' P^T and G^T of the previous step,
-// accumulates dV += P^T dO and dK += G^T Q from TMEM, then issues the next
-// S^T = K Q^T and dP^T = V dO^T (tcgen05 operations of one thread execute in
-// issue order, so S^T and dP^T are overwritten only after the products that
-// read P^T and G^T).  The compute warps rebuild each element of P^T from the
-// query's log-sum-exp; the per-query factors come from a shared-memory table
-// that the compute threads fill (one query row each) before every step.
+// 320 threads: warps 0-7 compute, warp 8 TMA producer, warp 9 MMA issuer.  The K
+// and V tiles stay resident; the (Q, dO) tiles of the causal query tiles stream
+// through a two-stage ring.  TMEM (512 columns): two (S^T | dP^T) buffers of half a
+// query tile (64 queries, 64 + 64 columns), then dV and dK.  Per half step u the
+// issuer puts out S^T = K Q^T and dP^T = V dO^T into buffer u & 1, then, once the
+// compute warps have turned half u - 1 into P^T and G^T, accumulates dV += P^T dO
+// and dK += G^T Q from TMEM: the tensor core computes one half while the compute
+// warps work on the other (tcgen05 operations of one thread execute in issue
+// order, so a buffer is overwritten only after the products that read it).
+// Warps w and w + 4 share key rows 32 (w & 3) .. + 31 (the TMEM lanes of that
+// quarter) and split each half's 64 queries.  Each element of P^T is rebuilt from
+// the query's log-sum-exp; the per-query factors come from a shared-memory table
+// that warps 0-3 fill (one query row per thread) before every query tile.
+constexpr int DKV_THREADS = 320;
+
+// bar.red.or over the two compute warps of one row group (named barrier 2 + q4, 64 threads)
+__device__ __forceinline__ bool pair_red_or(int id, bool pred) {
+    uint32_t res;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, %2, 64, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(res)
+        : "r"(static_cast<uint32_t>(pred)), "r"(id)
+        : "memory");
+    return res != 0;
+}
+
+// bar.red.or over the eight compute warps (named barrier 1, 256 threads)
+__device__ __forceinline__ bool compute_red_or(bool pred) {
+    uint32_t res;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, 1, 256, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(res)
+        : "r"(static_cast<uint32_t>(pred))
+        : "memory");
+    return res != 0;
+}
+
 template <int HD>
 struct DkvSmem {
     static constexpr int TILE = BT * HD * 2;
     static constexpr int OFF_K = 0;
     static constexpr int OFF_V = OFF_K + TILE;
-    static constexpr int OFF_Q = OFF_V + TILE;        // [2 stages]
-    static constexpr int OFF_DO = OFF_Q + 2 * TILE;   // [2 stages]
-    static constexpr int OFF_PAR = OFF_DO + 2 * TILE; // [2 stages][5][BT] fp32
-    static constexpr int OFF_BAR = OFF_PAR + 2 * 5 * BT * 4;
+    static constexpr int OFF_Q = OFF_V + TILE;         // [2 stages]
+    static constexpr int OFF_DO = OFF_Q + 2 * TILE;    // [2 stages]
+    static constexpr int OFF_PAR = OFF_DO + 2 * TILE;  // [2 stages][5][BT] fp32
+    static constexpr int OFF_XCH = OFF_PAR + 2 * 5 * BT * 4;  // [BT] fp32: the second query half's key sums
+    static constexpr int OFF_BAR = OFF_XCH + BT * 4;
     static constexpr int NUM_BARS = 12;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int BYTES = OFF_MISC + 16;
@@ -88,10 +116,18 @@ struct DkvSmem {
     static_assert(2 * BT + 2 * HD <= 512, "TMEM columns");
 };
 
-enum : int { D_KV_FULL = 0, D_QD_FULL = 1, D_QD_EMPTY = 3, D_SDP_FULL = 5, D_PG_FULL = 6, D_ACC_DONE = 7, D_DRAIN = 8 };
+enum : int {
+    D_KV_FULL = 0,
+    D_QD_FULL = 1,   // [2]
+    D_QD_EMPTY = 3,  // [2]
+    D_SDP_FULL = 5,  // [2]
+    D_PG_FULL = 7,   // [2]
+    D_ACC_DONE = 9,
+    D_DRAIN = 10
+};
 
 template <int HD>
-__global__ void __launch_bounds__(BWD_THREADS, 1)
+__global__ void __launch_bounds__(DKV_THREADS, 1)
 gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                           const int32_t* __restrict__ cu_kept, const int32_t* __restrict__ pos,
@@ -115,7 +151,6 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
     const int grp = Hq / Hkv;
     const int hk = h / grp, hh = h - hk * grp;
     const int nq = n_qt - kt;  // causal query tiles
-    const int n_steps = nq;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     const uint32_t sbase = smem_u32(smem);
@@ -129,15 +164,15 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
         for (int s = 0; s < 2; ++s) {
             mbar_init(bar(D_QD_FULL + s), 1);
             mbar_init(bar(D_QD_EMPTY + s), 1);
+            mbar_init(bar(D_SDP_FULL + s), 1);
+            mbar_init(bar(D_PG_FULL + s), 256);  // every thread of the eight compute warps
         }
-        mbar_init(bar(D_SDP_FULL), 1);
-        mbar_init(bar(D_PG_FULL), 128);
         mbar_init(bar(D_ACC_DONE), 1);
         mbar_init(bar(D_DRAIN), 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 4) {
+    if (warp == 8) {
         tmem_alloc(smem_u32(tmem_slot), L::TMEM_COLS);
         tmem_relinquish();
     }
@@ -145,9 +180,11 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tST = tmem, tDPT = tmem + BT, tDV = tmem + 2 * BT, tDK = tmem + 2 * BT + HD;
+    // half buffer hb: S^T of 64 queries at columns [128 hb, +64), dP^T at [128 hb + 64, +64);
+    // P^T and G^T (bf16 pairs) go over the first 32 columns of each
+    const uint32_t tDV = tmem + 2 * BT, tDK = tmem + 2 * BT + HD;
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ---------------------------------------------------------------- TMA producer
         if (lane == 0) {
             prefetch_tmap(&tmQ);
@@ -161,7 +198,7 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
                 tma_load_2d(sV + hf * BT * 128, &tmV, hk * HD + hf * 64, seq0 + kt * BT, bar(D_KV_FULL));
             }
             int issued[2] = {0, 0};
-            for (int t = 0; t < n_steps; ++t) {
+            for (int t = 0; t < nq; ++t) {
                 const int s = t & 1;
                 const int i = kt + t;
                 if (t >= 2 && !mbar_wait(bar(D_QD_EMPTY + s), ((t - 2) >> 1) & 1, abort_flag, status,
@@ -183,72 +220,93 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
                     if (issued[s]) drain_wait_b(bar(D_QD_FULL + s), (issued[s] - 1) & 1, status);
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == 9) {
         // ---------------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc_s = idesc_bf16_f32(BT, BT, false);
+            constexpr uint32_t idesc_s = idesc_bf16_f32(BT, 64, false);
             constexpr uint32_t idesc_acc = idesc_bf16_f32(BT, HD, true);
-            // dV += P^T dO(t), dK += G^T Q(t): A from TMEM (16 queries = 8 columns per
-            // k-step), B the (query x head_dim) tile read MN-major
-            auto issue_acc = [&](int t) {
-                const int s = t & 1;
+            // Half step u: query tile u >> 1, queries 64 (u & 1) .. +63 (64 rows = 8 KB into
+            // each swizzled box of the stage), TMEM buffer u & 1.
+            auto issue_sdp = [&](int u) {
+                const int hb = u & 1, s = (u >> 1) & 1;
+                const uint32_t tb = tmem + hb * 128;
 #pragma unroll
-                for (int kk = 0; kk < BT / 16; ++kk)
-                    mma_bf16_ts(tDV, tST + kk * 8, smem_desc_sw128(sDO + s * L::TILE + kk * 16 * 128, BT * 128, 1024),
-                                idesc_acc, (t > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * (BT * 128) + (kk & 3) * 32;
+                    mma_bf16_ss(tb, smem_desc_sw128(sK + off, 16, 1024),
+                                smem_desc_sw128(sQ + s * L::TILE + hb * 64 * 128 + off, 16, 1024), idesc_s,
+                                kk > 0 ? 1u : 0u);
+                }
 #pragma unroll
-                for (int kk = 0; kk < BT / 16; ++kk)
-                    mma_bf16_ts(tDK, tDPT + kk * 8, smem_desc_sw128(sQ + s * L::TILE + kk * 16 * 128, BT * 128, 1024),
-                                idesc_acc, (t > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(bar(D_QD_EMPTY + s));
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * (BT * 128) + (kk & 3) * 32;
+                    mma_bf16_ss(tb + 64, smem_desc_sw128(sV + off, 16, 1024),
+                                smem_desc_sw128(sDO + s * L::TILE + hb * 64 * 128 + off, 16, 1024), idesc_s,
+                                kk > 0 ? 1u : 0u);
+                }
+                mma_commit(bar(D_SDP_FULL + hb));
             };
+            // dV += P^T dO(half), dK += G^T Q(half): A from TMEM (16 queries = 8 columns per
+            // k-step), B the (query x head_dim) rows read MN-major
+            auto issue_acc = [&](int u) {
+                const int hb = u & 1, s = (u >> 1) & 1;
+                const uint32_t tb = tmem + hb * 128;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16_ts(tDV, tb + kk * 8,
+                                smem_desc_sw128(sDO + s * L::TILE + (hb * 64 + kk * 16) * 128, BT * 128, 1024),
+                                idesc_acc, (u > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16_ts(tDK, tb + 64 + kk * 8,
+                                smem_desc_sw128(sQ + s * L::TILE + (hb * 64 + kk * 16) * 128, BT * 128, 1024),
+                                idesc_acc, (u > 0 || kk > 0) ? 1u : 0u);
+                if (hb == 1) mma_commit(bar(D_QD_EMPTY + s));  // the stage is no longer read
+            };
+            const int n_u = 2 * nq;
             bool ok = mbar_wait(bar(D_KV_FULL), 0, abort_flag, status, TG_WHERE_MMA);
-            for (int t = 0; ok && t < n_steps; ++t) {
-                const int s = t & 1;
-                ok = mbar_wait(bar(D_QD_FULL + s), (t >> 1) & 1, abort_flag, status, TG_WHERE_MMA);
-                if (ok && t >= 1) ok = mbar_wait(bar(D_PG_FULL), (t - 1) & 1, abort_flag, status, TG_WHERE_MMA);
-                if (!ok) break;
+            for (int u = 0; ok && u < n_u; ++u) {
+                const int t = u >> 1, s = t & 1;
+                if ((u & 1) == 0) {
+                    ok = mbar_wait(bar(D_QD_FULL + s), (t >> 1) & 1, abort_flag, status, TG_WHERE_MMA);
+                    if (!ok) break;
+                }
                 tc_fence_after();
-                if (t >= 1) issue_acc(t - 1);
-#pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * (BT * 128) + (kk & 3) * 32;
-                    mma_bf16_ss(tST, smem_desc_sw128(sK + off, 16, 1024),
-                                smem_desc_sw128(sQ + s * L::TILE + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+                issue_sdp(u);
+                if (u >= 1) {
+                    ok = mbar_wait(bar(D_PG_FULL + ((u - 1) & 1)), ((u - 1) >> 1) & 1, abort_flag, status,
+                                   TG_WHERE_MMA);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_acc(u - 1);
                 }
-#pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * (BT * 128) + (kk & 3) * 32;
-                    mma_bf16_ss(tDPT, smem_desc_sw128(sV + off, 16, 1024),
-                                smem_desc_sw128(sDO + s * L::TILE + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
-                }
-                mma_commit(bar(D_SDP_FULL));
             }
-            if (ok) ok = mbar_wait(bar(D_PG_FULL), (n_steps - 1) & 1, abort_flag, status, TG_WHERE_MMA);
+            if (ok) ok = mbar_wait(bar(D_PG_FULL + ((n_u - 1) & 1)), ((n_u - 1) >> 1) & 1, abort_flag, status,
+                                   TG_WHERE_MMA);
             if (ok) {
                 tc_fence_after();
-                issue_acc(n_steps - 1);
+                issue_acc(n_u - 1);
                 mma_commit(bar(D_ACC_DONE));
             }
             mma_commit(bar(D_DRAIN));
             drain_wait_b(bar(D_DRAIN), 0, status);
         }
     } else {
-        // ---------------------------------------------------------------- compute warps 0-3
-        const int r = threadIdx.x;  // key row of the tile == TMEM lane
+        // ---------------------------------------------------------------- compute warps 0-7
+        const int q4 = warp & 3, cs = warp >> 2;
+        const int r = q4 * 32 + lane;  // key row of the tile == TMEM lane
         const int key_local = kt * BT + r;
         const bool valid_key = key_local < Mb;
-        const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+        const uint32_t lane_addr = static_cast<uint32_t>(q4 * 32) << 16;
         const float gl = valid_key ? __ldcg(gls + seq0 + key_local) : 0.f;
         float* par = reinterpret_cast<float*>(smem + L::OFF_PAR);
         bool ok = true;
-        int t = 0;
+        float csum = 0.f;
         {
             const float beta = softplus_b(g[h]);
             const float ch = c[h];
-            float csum = 0.f;
-            // this thread's query row of the next tile: pos, rank, lse and D' are loaded one
-            // step ahead (their latency hides behind a step of work)
+            // warps 0-3: this thread's query row of the next tile; pos, rank, lse and D' are
+            // loaded one step ahead (their latency hides behind a step of work)
             int npos = 1, nrank = 1;
             float nlse = 0.f, nD = 0.f;
             auto load_row = [&](int i) {
@@ -261,123 +319,146 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
                     nD = __ldcg(Drow + static_cast<size_t>(qg) * Hq + h);
                 }
             };
-            load_row(kt);
-            for (int ii = 0; ii < nq; ++ii, ++t) {
-                const int i = kt + ii, s = t & 1;
-                // this thread's query row of tile i fills one column of the factor table
-                const int qrow = i * BT + r;
-                float fa = 0.f, fb = 0.f, fl = 0.f, fd = 0.f, fi = 0.f;
-                if (qrow < Mb) {
-                    fi = 1.0f / (1.0f + ch * logf(static_cast<float>(npos) / static_cast<float>(nrank)));
-                    fa = sm_scale * LOG2E_B * fi;
-                    fb = beta * LOG2E_B * fi;
-                    fl = nlse * LOG2E_B;
-                    fd = nD;
+            if (cs == 0) load_row(kt);
+            for (int t = 0; t < nq; ++t) {
+                const int i = kt + t, s = t & 1;
+                const float* ps = par + s * 5 * BT;
+                if (cs == 0) {
+                    // column r of the factor table: fa, fb, -fl, fi, -fi D for query row r of tile i
+                    float fa = 0.f, fb = 0.f, nfl = 0.f, fi = 0.f, nfd = 0.f;
+                    if (i * BT + r < Mb) {
+                        fi = 1.0f / (1.0f + ch * logf(static_cast<float>(npos) / static_cast<float>(nrank)));
+                        fa = sm_scale * LOG2E_B * fi;
+                        fb = beta * LOG2E_B * fi;
+                        nfl = -nlse * LOG2E_B;
+                        nfd = -fi * nD;
+                    }
+                    if (t + 1 < nq) load_row(i + 1);
+                    float* pw = par + s * 5 * BT;
+                    pw[0 * BT + r] = fa;
+                    pw[1 * BT + r] = fb;
+                    pw[2 * BT + r] = nfl;
+                    pw[3 * BT + r] = fi;
+                    pw[4 * BT + r] = nfd;
                 }
-                if (ii + 1 < nq) load_row(i + 1);
-                float* ps = par + s * 5 * BT;
-                ps[0 * BT + r] = fa;
-                ps[1 * BT + r] = fb;
-                ps[2 * BT + r] = fl;
-                ps[3 * BT + r] = fd;
-                ps[4 * BT + r] = fi;
-                const bool okw = mbar_wait_warp(bar(D_SDP_FULL), t & 1, abort_flag, status, TG_WHERE_SOFTMAX);
                 // the table is complete past this barrier, which also makes an abort uniform
-                uint32_t any_abort;
-                asm volatile(
-                    "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, 1, 128, p;\n\t"
-                    "selp.u32 %0, 1, 0, q;\n\t}"
-                    : "=r"(any_abort)
-                    : "r"(static_cast<uint32_t>(!okw))
-                    : "memory");
-                if (any_abort) {
+                // (the table of slot s was last read two tiles ago, before the previous barrier)
+                if (compute_red_or(!ok)) {
                     ok = false;
                     break;
                 }
-                tc_fence_after();
                 const int col_lim = min(BT, Mb - i * BT);  // query columns inside the sequence
-                const bool diag = (i == kt);               // keys above the query are masked there
+                const int lo = (i == kt) ? r : 0;          // on the diagonal tile, queries below the key are masked
 #pragma unroll 1
-                for (int half = 0; half < 2; ++half) {
-                    float sx[64], dpx[64];
-                    tmem_ld32(tST + lane_addr + half * 64, sx);
-                    tmem_ld32(tST + lane_addr + half * 64 + 32, sx + 32);
-                    tmem_ld32(tDPT + lane_addr + half * 64, dpx);
-                    tmem_ld32(tDPT + lane_addr + half * 64 + 32, dpx + 32);
-                    tmem_wait_ld();
-                    uint32_t pp[32], gg[32];
-#pragma unroll
-                    for (int cc = 0; cc < 64; cc += 2) {
-                        float pv[2], gv[2];
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int col = half * 64 + cc + e;
-                            const float tt = fmaf(ps[0 * BT + col], sx[cc + e], fmaf(ps[1 * BT + col], gl, -ps[2 * BT + col]));
-                            const bool keep = col < col_lim && !(diag && col < r);
-                            const float p = keep ? ex2_approx(tt) : 0.f;
-                            const float G = p * (dpx[cc + e] - ps[3 * BT + col]) * ps[4 * BT + col];
-                            csum += G;
-                            pv[e] = p;
-                            gv[e] = G;
-                        }
-                        pp[cc / 2] = pack2_bf16(pv[0], pv[1]);
-                        gg[cc / 2] = pack2_bf16(gv[0], gv[1]);
+                for (int hb = 0; hb < 2; ++hb) {
+                    const int c0 = hb * 64 + cs * 32;  // first query column of this warp
+                    const bool okw = mbar_wait_warp(bar(D_SDP_FULL + hb), t & 1, abort_flag, status, TG_WHERE_SOFTMAX);
+                    const uint32_t tb = tmem + lane_addr + hb * 128;
+                    float sx[32], dpx[32];
+                    if (okw) {
+                        tc_fence_after();
+                        tmem_ld32(tb + cs * 32, sx);
+                        tmem_ld32(tb + 64 + cs * 32, dpx);
+                        tmem_wait_ld();
                     }
-                    // P^T and G^T over the (already read) first 64 columns of S^T and dP^T
-                    tmem_st32u(tST + lane_addr + half * 32, pp);
-                    tmem_st32u(tDPT + lane_addr + half * 32, gg);
+                    // both warps of the row group have read their columns (the P^T / G^T stores
+                    // below overwrite some of the partner's); an abort is decided by the pair
+                    if (pair_red_or(2 + q4, !okw)) {
+                        ok = false;
+                        break;
+                    }
+                    // columns c0 + k with lo <= c0 + k < col_lim are live
+                    const int a = lo - c0, e = col_lim - c0;
+                    const uint32_t live = (a >= 32 || e <= 0 || a >= e)
+                                              ? 0u
+                                              : ((e >= 32 ? 0xFFFFFFFFu : ((1u << e) - 1u)) &
+                                                 (a <= 0 ? 0xFFFFFFFFu : ~((1u << a) - 1u)));
+                    uint32_t pp[16], gg[16];
+#pragma unroll
+                    for (int k4 = 0; k4 < 32; k4 += 4) {
+                        const float4 fa4 = *reinterpret_cast<const float4*>(ps + 0 * BT + c0 + k4);
+                        const float4 fb4 = *reinterpret_cast<const float4*>(ps + 1 * BT + c0 + k4);
+                        const float4 fl4 = *reinterpret_cast<const float4*>(ps + 2 * BT + c0 + k4);
+                        const float4 fi4 = *reinterpret_cast<const float4*>(ps + 3 * BT + c0 + k4);
+                        const float4 fd4 = *reinterpret_cast<const float4*>(ps + 4 * BT + c0 + k4);
+                        const float fav[4] = {fa4.x, fa4.y, fa4.z, fa4.w}, fbv[4] = {fb4.x, fb4.y, fb4.z, fb4.w};
+                        const float flv[4] = {fl4.x, fl4.y, fl4.z, fl4.w}, fiv[4] = {fi4.x, fi4.y, fi4.z, fi4.w};
+                        const float fdv[4] = {fd4.x, fd4.y, fd4.z, fd4.w};
+                        float pv[4], gv[4];
+#pragma unroll
+                        for (int x = 0; x < 4; ++x) {
+                            const int k = k4 + x;
+                            const float tt = fmaf(fav[x], sx[k], fmaf(fbv[x], gl, flv[x]));
+                            const float p = (live >> k) & 1u ? ex2_approx(tt) : 0.f;
+                            const float G = p * fmaf(fiv[x], dpx[k], fdv[x]);
+                            csum += G;
+                            pv[x] = p;
+                            gv[x] = G;
+                        }
+                        pp[k4 / 2] = pack2_bf16(pv[0], pv[1]);
+                        pp[k4 / 2 + 1] = pack2_bf16(pv[2], pv[3]);
+                        gg[k4 / 2] = pack2_bf16(gv[0], gv[1]);
+                        gg[k4 / 2 + 1] = pack2_bf16(gv[2], gv[3]);
+                    }
+                    tmem_st16u(tb + cs * 16, pp);       // P^T of these 32 queries over S^T
+                    tmem_st16u(tb + 64 + cs * 16, gg);  // G^T over dP^T
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(bar(D_PG_FULL + hb));
                 }
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(bar(D_PG_FULL));
             }
-            if (ok && valid_key) colsum[static_cast<size_t>(seq0 + key_local) * Hq + h] = csum;
         }
+        // the second query half's key sums join the first's (all eight warps, abort or not)
+        float* xch = reinterpret_cast<float*>(smem + L::OFF_XCH);
+        if (cs == 1) xch[r] = csum;
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        if (cs == 0 && ok && valid_key) colsum[static_cast<size_t>(seq0 + key_local) * Hq + h] = csum + xch[r];
         // ---------------------------------------------------------------- epilogue
         if (ok) ok = mbar_wait_warp(bar(D_ACC_DONE), 0, abort_flag, status, TG_WHERE_SOFTMAX);
         if (ok && part_k) {
-            // partials of this head: [head in group][row][KV head][d] fp32, unscaled
+            // partials of this head: [head in group][row][KV head][d] fp32, unscaled; warp cs
+            // writes head_dim columns cs HD/2 .. + HD/2 - 1 of its rows
             tc_fence_after();
-            const size_t row = ((static_cast<size_t>(hh) * M_total + seq0 + key_local) * Hkv + hk) * HD;
+            const size_t row = ((static_cast<size_t>(hh) * M_total + seq0 + key_local) * Hkv + hk) * HD + cs * (HD / 2);
 #pragma unroll 1
             for (int which = 0; which < 2; ++which) {
-                const uint32_t src = which ? tDK : tDV;
+                const uint32_t src = (which ? tDK : tDV) + cs * (HD / 2);
                 float* dst = (which ? part_k : part_v) + row;
 #pragma unroll
-                for (int ch = 0; ch < HD / 32; ++ch) {
+                for (int ch = 0; ch < HD / 64; ++ch) {
                     float o[32];
                     tmem_ld32(src + lane_addr + ch * 32, o);
                     tmem_wait_ld();
                     if (valid_key) {
 #pragma unroll
-                        for (int q4 = 0; q4 < 8; ++q4)
-                            *reinterpret_cast<float4*>(dst + ch * 32 + q4 * 4) =
-                                make_float4(o[q4 * 4], o[q4 * 4 + 1], o[q4 * 4 + 2], o[q4 * 4 + 3]);
+                        for (int q = 0; q < 8; ++q)
+                            *reinterpret_cast<float4*>(dst + ch * 32 + q * 4) =
+                                make_float4(o[q * 4], o[q * 4 + 1], o[q * 4 + 2], o[q * 4 + 3]);
                     }
                 }
             }
         } else if (ok) {
             tc_fence_after();
-            const size_t row = (static_cast<size_t>(seq0 + key_local) * Hkv + hk) * HD;
+            const size_t row = (static_cast<size_t>(seq0 + key_local) * Hkv + hk) * HD + cs * (HD / 2);
 #pragma unroll 1
             for (int which = 0; which < 2; ++which) {
-                const uint32_t src = which ? tDK : tDV;
+                const uint32_t src = (which ? tDK : tDV) + cs * (HD / 2);
                 const float scale = which ? sm_scale : 1.0f;
                 uint16_t* dst = (which ? dk : dv) + row;
 #pragma unroll
-                for (int ch = 0; ch < HD / 32; ++ch) {
+                for (int ch = 0; ch < HD / 64; ++ch) {
                     float o[32];
                     tmem_ld32(src + lane_addr + ch * 32, o);
                     tmem_wait_ld();
                     if (valid_key) {
 #pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4) {
+                        for (int q = 0; q < 4; ++q) {
                             uint4 w;
-                            w.x = pack2_bf16(o[q4 * 8 + 0] * scale, o[q4 * 8 + 1] * scale);
-                            w.y = pack2_bf16(o[q4 * 8 + 2] * scale, o[q4 * 8 + 3] * scale);
-                            w.z = pack2_bf16(o[q4 * 8 + 4] * scale, o[q4 * 8 + 5] * scale);
-                            w.w = pack2_bf16(o[q4 * 8 + 6] * scale, o[q4 * 8 + 7] * scale);
-                            *reinterpret_cast<uint4*>(dst + ch * 32 + q4 * 8) = w;
+                            w.x = pack2_bf16(o[q * 8 + 0] * scale, o[q * 8 + 1] * scale);
+                            w.y = pack2_bf16(o[q * 8 + 2] * scale, o[q * 8 + 3] * scale);
+                            w.z = pack2_bf16(o[q * 8 + 4] * scale, o[q * 8 + 5] * scale);
+                            w.w = pack2_bf16(o[q * 8 + 6] * scale, o[q * 8 + 7] * scale);
+                            *reinterpret_cast<uint4*>(dst + ch * 32 + q * 8) = w;
                         }
                     }
                 }
@@ -387,7 +468,7 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 4) {
+    if (warp == 8) {
         tc_fence_after();
         tmem_dealloc(tmem, L::TMEM_COLS);
     }
@@ -431,18 +512,6 @@ enum : int {
 };
 
 constexpr int DQ_THREADS = 320;  // warps 0-7 compute, 8 TMA producer, 9 MMA issuer
-
-// bar.red.or over the two compute warps of one row group (named barrier 2 + q4, 64 threads)
-__device__ __forceinline__ bool pair_red_or(int id, bool pred) {
-    uint32_t res;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, %2, 64, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(res)
-        : "r"(static_cast<uint32_t>(pred)), "r"(id)
-        : "memory");
-    return res != 0;
-}
 
 template <int HD>
 __global__ void __launch_bounds__(DQ_THREADS, 1)
@@ -932,7 +1001,7 @@ cudaError_t launch_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
                                static_cast<size_t>(DqSmem<HD>::ALLOC), st, tq, tk, tv, tdo, cu_kept, pos, rank, gls, g,
                                c, lse, out, Drow, sm_scale, Hq, Hkv, n_t, dq, tileE, tileT, status);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(gated_attn_bwd_dkv_kernel<HD>, dim3(Hq, n_t, B), dim3(BWD_THREADS),
+    e = launch_pdl(gated_attn_bwd_dkv_kernel<HD>, dim3(Hq, n_t, B), dim3(DKV_THREADS),
                    static_cast<size_t>(DkvSmem<HD>::ALLOC), st, tq, tk, tv, tdo, cu_kept, pos, rank, gls, g, c, lse,
                    static_cast<const float*>(Drow), sm_scale, Hq, Hkv, M_total, dk, dv, part_k, part_v, colsum,
                    status);
