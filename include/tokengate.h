@@ -218,7 +218,7 @@ tg_status tg_gated_attention_gates(const uint16_t* q, const uint16_t* k, const u
  * out [M, Hq, d] bf16 and lse [M, Hq] fp32 are the forward's outputs (call
  * tg_gated_attention with a non-NULL lse).  head_dim 64 or 128 (else
  * TG_ERR_UNSUPPORTED).  ws: device scratch, 256-byte aligned, of at least
- * tg_gated_attention_backward_workspace_size(M_total, Hq, Hkv, d) bytes (4
+ * tg_gated_attention_backward_workspace_size(M_total, Hq, Hkv, d) bytes (6
  * floats per row and head, plus fp32 partial dk and dv per query head when a
  * KV head serves two or more; no zeroing needed).  Tensor cores, no atomics:
  * the results are deterministic.

@@ -13,23 +13,26 @@
 //   dg_h = dbeta_h sigmoid(g_h),  dc_h = sum_i dtau_ih ln(pos_i / rank_i),
 //   d score_j = dgls_j sigmoid(-score_j) = dgls_j (1 - exp(gls_j)).
 //
-// Three or four launches, no atomics (results do not depend on scheduling):
-//   dq       (below; it also forms D_ih = dout_i.out_i for its rows)
+// Three or four launches in this order, no atomics (results do not depend on
+// scheduling):
+//   dq       one CTA per (query head, 128-query tile), the forward's layout:
+//            S = Q K^T and dP = dO V^T, G as bf16 over S, dQ += G K.  It forms
+//            D_ih = dout_i.out_i for its rows; the per-query sums for dtau run
+//            along each thread's row, which also yields the exact
+//            D'_i = sum_j P_ij dP_ij.  It leaves each row's factors (with D' in
+//            place of D) for the dkv kernel.
 //   dkv      one CTA per (query head, 128-key tile): for every half (64
 //            queries) of every causal query tile, S^T = K Q^T and dP^T = V dO^T
 //            on the tensor core (TMEM lanes = keys), then P^T and G^T as bf16
 //            over the first 32 columns of S^T and dP^T, and dV += P^T dO,
 //            dK += G^T Q read from TMEM.  The per-key sums of G (the gate
 //            bias's gradient, per head) are sums along each thread's own row.
-//            The query heads of a GQA group leave fp32 partials of dK / dV that
-//            kv_reduce sums in head order (a group of one writes bf16 itself).
-//   dq       one CTA per (query head, 128-query tile), the forward's layout:
-//            S = Q K^T and dP = dO V^T, G as bf16 over S, dQ += G K.  The
-//            per-query sums for dbeta and dtau run along each thread's row,
-//            which also yields the exact D'_i = sum_j P_ij dP_ij; it replaces
-//            D for the dkv kernel (launched after dq).
-//   finish   dgls / d score per key, dg and dc per head (the dq kernel leaves one
-//            partial sum of the dbeta and dc terms per query tile).
+//            The query heads of a GQA group leave fp32 partials of dK / dV (a
+//            group of one writes bf16 itself).
+//   kv_reduce sums those partials in head order (groups of two or more only).
+//   finish   dgls / d score per key, dg and dc per head (dbeta from the per-key
+//            sums of G; the dq kernel leaves one partial sum of the dc terms per
+//            query tile).
 // Every row of P is rebuilt from the forward's log-sum-exp.
 
 #include "tg_sm100.cuh"
@@ -69,8 +72,8 @@ __device__ __forceinline__ bool drain_wait_b(uint32_t bar, uint32_t parity, int*
 // order, so a buffer is overwritten only after the products that read it).
 // Warps w and w + 4 share key rows 32 (w & 3) .. + 31 (the TMEM lanes of that
 // quarter) and split each half's 64 queries.  Each element of P^T is rebuilt from
-// the query's log-sum-exp; the per-query factors come from a shared-memory table
-// that warps 0-3 fill (one query row per thread) before every query tile.
+// the query's log-sum-exp; the per-query factors (left by the dQ kernel, one
+// float4 per query row and head) go through a small table of each warp's own.
 constexpr int DKV_THREADS = 320;
 
 // bar.red.or over the two compute warps of one row group (named barrier 2 + q4, 64 threads)
@@ -85,18 +88,6 @@ __device__ __forceinline__ bool pair_red_or(int id, bool pred) {
     return res != 0;
 }
 
-// bar.red.or over the eight compute warps (named barrier 1, 256 threads)
-__device__ __forceinline__ bool compute_red_or(bool pred) {
-    uint32_t res;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, 1, 256, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(res)
-        : "r"(static_cast<uint32_t>(pred))
-        : "memory");
-    return res != 0;
-}
-
 template <int HD>
 struct DkvSmem {
     static constexpr int TILE = BT * HD * 2;
@@ -104,8 +95,8 @@ struct DkvSmem {
     static constexpr int OFF_V = OFF_K + TILE;
     static constexpr int OFF_Q = OFF_V + TILE;         // [2 stages]
     static constexpr int OFF_DO = OFF_Q + 2 * TILE;    // [2 stages]
-    static constexpr int OFF_PAR = OFF_DO + 2 * TILE;  // [2 stages][5][BT] fp32
-    static constexpr int OFF_XCH = OFF_PAR + 2 * 5 * BT * 4;  // [BT] fp32: the second query half's key sums
+    static constexpr int OFF_TAB = OFF_DO + 2 * TILE;  // [8 warps][2][4][32] fp32 query factors
+    static constexpr int OFF_XCH = OFF_TAB + 8 * 2 * 4 * 32 * 4;  // [BT] fp32: the second query half's key sums
     static constexpr int OFF_BAR = OFF_XCH + BT * 4;
     static constexpr int NUM_BARS = 12;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
@@ -130,10 +121,9 @@ template <int HD>
 __global__ void __launch_bounds__(DKV_THREADS, 1)
 gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                          const int32_t* __restrict__ cu_kept, const int32_t* __restrict__ pos,
-                          const int32_t* __restrict__ rank, const float* __restrict__ gls,
-                          const float* __restrict__ g, const float* __restrict__ c, const float* __restrict__ lse,
-                          const float* __restrict__ Drow, float sm_scale, int Hq, int Hkv, int64_t M_total,
+                          const int32_t* __restrict__ cu_kept, const float* __restrict__ gls,
+                          const float* __restrict__ g, const float4* __restrict__ fac, float sm_scale, int Hq,
+                          int Hkv, int64_t M_total,
                           uint16_t* __restrict__ dk, uint16_t* __restrict__ dv, float* __restrict__ part_k,
                           float* __restrict__ part_v, float* __restrict__ colsum, int* __restrict__ status) {
     using L = DkvSmem<HD>;
@@ -298,115 +288,87 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
         const int key_local = kt * BT + r;
         const bool valid_key = key_local < Mb;
         const uint32_t lane_addr = static_cast<uint32_t>(q4 * 32) << 16;
-        const float gl = valid_key ? __ldcg(gls + seq0 + key_local) : 0.f;
-        float* par = reinterpret_cast<float*>(smem + L::OFF_PAR);
+        // kgl = (beta / sm) gls_j, the key's bias in units of the score, so that the log2 of
+        // P is tt = fa (s + kgl) - lse log2(e) with the query's fa = sm log2(e) / tau
+        const float kgl = valid_key ? (softplus_b(g[h]) / sm_scale) * __ldcg(gls + seq0 + key_local) : 0.f;
+        // this warp's own table of its 32 queries' factors (fa, -lse log2(e), 1/tau, -D'/tau),
+        // [2 half steps][4][32]; only __syncwarp orders it
+        float* wtab = reinterpret_cast<float*>(smem + L::OFF_TAB) + warp * (2 * 4 * 32);
         bool ok = true;
         float csum = 0.f;
-        {
-            const float beta = softplus_b(g[h]);
-            const float ch = c[h];
-            // warps 0-3: this thread's query row of the next tile; pos, rank, lse and D' are
-            // loaded one step ahead (their latency hides behind a step of work)
-            int npos = 1, nrank = 1;
-            float nlse = 0.f, nD = 0.f;
-            auto load_row = [&](int i) {
-                const int qrow = i * BT + r;
-                if (qrow < Mb) {
-                    const int qg = seq0 + qrow;
-                    npos = __ldcg(pos + qg);
-                    nrank = __ldcg(rank + qg);
-                    nlse = __ldcg(lse + static_cast<size_t>(qg) * Hq + h);
-                    nD = __ldcg(Drow + static_cast<size_t>(qg) * Hq + h);
-                }
-            };
-            if (cs == 0) load_row(kt);
-            for (int t = 0; t < nq; ++t) {
-                const int i = kt + t, s = t & 1;
-                const float* ps = par + s * 5 * BT;
-                if (cs == 0) {
-                    // column r of the factor table: fa, fb, -fl, fi, -fi D for query row r of tile i
-                    float fa = 0.f, fb = 0.f, nfl = 0.f, fi = 0.f, nfd = 0.f;
-                    if (i * BT + r < Mb) {
-                        fi = 1.0f / (1.0f + ch * logf(static_cast<float>(npos) / static_cast<float>(nrank)));
-                        fa = sm_scale * LOG2E_B * fi;
-                        fb = beta * LOG2E_B * fi;
-                        nfl = -nlse * LOG2E_B;
-                        nfd = -fi * nD;
-                    }
-                    if (t + 1 < nq) load_row(i + 1);
-                    float* pw = par + s * 5 * BT;
-                    pw[0 * BT + r] = fa;
-                    pw[1 * BT + r] = fb;
-                    pw[2 * BT + r] = nfl;
-                    pw[3 * BT + r] = fi;
-                    pw[4 * BT + r] = nfd;
-                }
-                // the table is complete past this barrier, which also makes an abort uniform
-                // (the table of slot s was last read two tiles ago, before the previous barrier)
-                if (compute_red_or(!ok)) {
-                    ok = false;
-                    break;
-                }
-                const int col_lim = min(BT, Mb - i * BT);  // query columns inside the sequence
-                const int lo = (i == kt) ? r : 0;          // on the diagonal tile, queries below the key are masked
-#pragma unroll 1
-                for (int hb = 0; hb < 2; ++hb) {
-                    const int c0 = hb * 64 + cs * 32;  // first query column of this warp
-                    const bool okw = mbar_wait_warp(bar(D_SDP_FULL + hb), t & 1, abort_flag, status, TG_WHERE_SOFTMAX);
-                    const uint32_t tb = tmem + lane_addr + hb * 128;
-                    float sx[32], dpx[32];
-                    if (okw) {
-                        tc_fence_after();
-                        tmem_ld32(tb + cs * 32, sx);
-                        tmem_ld32(tb + 64 + cs * 32, dpx);
-                        tmem_wait_ld();
-                    }
-                    // both warps of the row group have read their columns (the P^T / G^T stores
-                    // below overwrite some of the partner's); an abort is decided by the pair
-                    if (pair_red_or(2 + q4, !okw)) {
-                        ok = false;
-                        break;
-                    }
-                    // columns c0 + k with lo <= c0 + k < col_lim are live
-                    const int a = lo - c0, e = col_lim - c0;
-                    const uint32_t live = (a >= 32 || e <= 0 || a >= e)
-                                              ? 0u
-                                              : ((e >= 32 ? 0xFFFFFFFFu : ((1u << e) - 1u)) &
-                                                 (a <= 0 ? 0xFFFFFFFFu : ~((1u << a) - 1u)));
-                    uint32_t pp[16], gg[16];
-#pragma unroll
-                    for (int k4 = 0; k4 < 32; k4 += 4) {
-                        const float4 fa4 = *reinterpret_cast<const float4*>(ps + 0 * BT + c0 + k4);
-                        const float4 fb4 = *reinterpret_cast<const float4*>(ps + 1 * BT + c0 + k4);
-                        const float4 fl4 = *reinterpret_cast<const float4*>(ps + 2 * BT + c0 + k4);
-                        const float4 fi4 = *reinterpret_cast<const float4*>(ps + 3 * BT + c0 + k4);
-                        const float4 fd4 = *reinterpret_cast<const float4*>(ps + 4 * BT + c0 + k4);
-                        const float fav[4] = {fa4.x, fa4.y, fa4.z, fa4.w}, fbv[4] = {fb4.x, fb4.y, fb4.z, fb4.w};
-                        const float flv[4] = {fl4.x, fl4.y, fl4.z, fl4.w}, fiv[4] = {fi4.x, fi4.y, fi4.z, fi4.w};
-                        const float fdv[4] = {fd4.x, fd4.y, fd4.z, fd4.w};
-                        float pv[4], gv[4];
-#pragma unroll
-                        for (int x = 0; x < 4; ++x) {
-                            const int k = k4 + x;
-                            const float tt = fmaf(fav[x], sx[k], fmaf(fbv[x], gl, flv[x]));
-                            const float p = (live >> k) & 1u ? ex2_approx(tt) : 0.f;
-                            const float G = p * fmaf(fiv[x], dpx[k], fdv[x]);
-                            csum += G;
-                            pv[x] = p;
-                            gv[x] = G;
-                        }
-                        pp[k4 / 2] = pack2_bf16(pv[0], pv[1]);
-                        pp[k4 / 2 + 1] = pack2_bf16(pv[2], pv[3]);
-                        gg[k4 / 2] = pack2_bf16(gv[0], gv[1]);
-                        gg[k4 / 2 + 1] = pack2_bf16(gv[2], gv[3]);
-                    }
-                    tmem_st16u(tb + cs * 16, pp);       // P^T of these 32 queries over S^T
-                    tmem_st16u(tb + 64 + cs * 16, gg);  // G^T over dP^T
-                    tmem_wait_st();
-                    tc_fence_before();
-                    mbar_arrive(bar(D_PG_FULL + hb));
-                }
+        const int n_u = 2 * nq;
+        // lane's query of half step u: query tile kt + (u >> 1), column 64 (u & 1) + 32 cs + lane;
+        // its factors are loaded one half step ahead
+        auto load_fac = [&](int u) {
+            const int qrow = (kt + (u >> 1)) * BT + (u & 1) * 64 + cs * 32 + lane;
+            return qrow < Mb ? __ldcg(fac + static_cast<size_t>(seq0 + qrow) * Hq + h)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+        };
+        float4 fnext = load_fac(0);
+        for (int u = 0; u < n_u; ++u) {
+            const int t = u >> 1, hb = u & 1, i = kt + t;
+            float* tab = wtab + hb * 128;
+            tab[0 * 32 + lane] = fnext.x;
+            tab[1 * 32 + lane] = fnext.y;
+            tab[2 * 32 + lane] = fnext.z;
+            tab[3 * 32 + lane] = fnext.w;
+            __syncwarp();
+            if (u + 1 < n_u) fnext = load_fac(u + 1);
+            const int c0 = hb * 64 + cs * 32;  // first query column of this warp
+            const bool okw = mbar_wait_warp(bar(D_SDP_FULL + hb), t & 1, abort_flag, status, TG_WHERE_SOFTMAX);
+            const uint32_t tb = tmem + lane_addr + hb * 128;
+            float sx[32], dpx[32];
+            if (okw) {
+                tc_fence_after();
+                tmem_ld32(tb + cs * 32, sx);
+                tmem_ld32(tb + 64 + cs * 32, dpx);
+                tmem_wait_ld();
             }
+            // both warps of the row group have read their columns (the P^T / G^T stores
+            // below overwrite some of the partner's); an abort is decided by the pair
+            if (pair_red_or(2 + q4, !okw)) {
+                ok = false;
+                break;
+            }
+            // columns c0 + k with lo <= c0 + k < col_lim are live: inside the sequence and, on
+            // the diagonal tile, not before the key
+            const int col_lim = min(BT, Mb - i * BT);
+            const int lo = (i == kt) ? r : 0;
+            const int a = lo - c0, e = col_lim - c0;
+            const uint32_t live = (a >= 32 || e <= 0 || a >= e)
+                                      ? 0u
+                                      : ((e >= 32 ? 0xFFFFFFFFu : ((1u << e) - 1u)) &
+                                         (a <= 0 ? 0xFFFFFFFFu : ~((1u << a) - 1u)));
+            uint32_t pp[16], gg[16];
+#pragma unroll
+            for (int k4 = 0; k4 < 32; k4 += 4) {
+                const float4 fa4 = *reinterpret_cast<const float4*>(tab + 0 * 32 + k4);
+                const float4 fl4 = *reinterpret_cast<const float4*>(tab + 1 * 32 + k4);
+                const float4 fi4 = *reinterpret_cast<const float4*>(tab + 2 * 32 + k4);
+                const float4 fd4 = *reinterpret_cast<const float4*>(tab + 3 * 32 + k4);
+                const float fav[4] = {fa4.x, fa4.y, fa4.z, fa4.w}, flv[4] = {fl4.x, fl4.y, fl4.z, fl4.w};
+                const float fiv[4] = {fi4.x, fi4.y, fi4.z, fi4.w}, fdv[4] = {fd4.x, fd4.y, fd4.z, fd4.w};
+                float pv[4], gv[4];
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    const int k = k4 + x;
+                    const float tt = fmaf(fav[x], sx[k] + kgl, flv[x]);
+                    const float p = (live >> k) & 1u ? ex2_approx(tt) : 0.f;
+                    const float G = p * fmaf(fiv[x], dpx[k], fdv[x]);
+                    csum += G;
+                    pv[x] = p;
+                    gv[x] = G;
+                }
+                pp[k4 / 2] = pack2_bf16(pv[0], pv[1]);
+                pp[k4 / 2 + 1] = pack2_bf16(pv[2], pv[3]);
+                gg[k4 / 2] = pack2_bf16(gv[0], gv[1]);
+                gg[k4 / 2 + 1] = pack2_bf16(gv[2], gv[3]);
+            }
+            tmem_st16u(tb + cs * 16, pp);       // P^T of these 32 queries over S^T
+            tmem_st16u(tb + 64 + cs * 16, gg);  // G^T over dP^T
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(D_PG_FULL + hb));
         }
         // the second query half's key sums join the first's (all eight warps, abort or not)
         float* xch = reinterpret_cast<float*>(smem + L::OFF_XCH);
@@ -486,7 +448,7 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
 // then accumulates dQ += G K from TMEM.  The compute warps rebuild P from the
 // log-sum-exp, form tau G = P (dP - D) (1/tau scales dQ's rows at the end), store
 // it as bf16 over the first 32 columns of the half's S and sum, along their own
-// row, G gls (for dbeta) and dl l (for dtau).
+// row, dl l (for dtau).
 template <int HD>
 struct DqSmem {
     static constexpr int TILE = BT * HD * 2;
@@ -520,9 +482,9 @@ gated_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
                          const int32_t* __restrict__ cu_kept, const int32_t* __restrict__ pos,
                          const int32_t* __restrict__ rank, const float* __restrict__ gls,
                          const float* __restrict__ g, const float* __restrict__ c, const float* __restrict__ lse,
-                         const uint16_t* __restrict__ out_fwd, float* __restrict__ Drow, float sm_scale, int Hq,
-                         int Hkv, int n_qt_max, uint16_t* __restrict__ dq, float* __restrict__ tileE,
-                         float* __restrict__ tileT, int* __restrict__ status) {
+                         const uint16_t* __restrict__ out_fwd, float4* __restrict__ fac, float sm_scale, int Hq,
+                         int Hkv, int n_qt_max, uint16_t* __restrict__ dq, float* __restrict__ tileT,
+                         int* __restrict__ status) {
     using L = DqSmem<HD>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -697,7 +659,17 @@ gated_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
         const bool valid_row = q_local < Mb;
         const int qg = seq0 + q_local;
         const uint32_t lane_addr = static_cast<uint32_t>(q4 * 32) << 16;
-        float fa = 0.f, fb = 0.f, fl = 0.f, fd = 0.f, fi = 0.f, lr = 0.f;
+        // D = dout . out of this row, each warp of the row group taking half of head_dim:
+        // out (the forward's output) is read from global memory while Q and dout arrive,
+        // dout from the staged tile (128-byte swizzled boxes of 64 columns)
+        constexpr int NCH = HD / 16;  // 8-column chunks per warp
+        uint4 ov[NCH];
+        if (valid_row) {
+            const uint16_t* orow = out_fwd + (static_cast<size_t>(qg) * Hq + h) * HD + cs * (HD / 2);
+#pragma unroll
+            for (int m = 0; m < NCH; ++m) ov[m] = __ldcg(reinterpret_cast<const uint4*>(orow + m * 8));
+        }
+        float fa = 0.f, fb = 0.f, fl = 0.f, fi = 0.f, lr = 0.f;
         if (valid_row) {
             lr = logf(static_cast<float>(__ldcg(pos + qg)) / static_cast<float>(__ldcg(rank + qg)));
             fi = 1.0f / (1.0f + c[h] * lr);
@@ -705,35 +677,34 @@ gated_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
             fb = softplus_b(g[h]) * LOG2E_B * fi;
             fl = __ldcg(lse + static_cast<size_t>(qg) * Hq + h) * LOG2E_B;
         }
-        // D = dout . out of this row (both warps of the row group form it), with dout from the
-        // staged tile (128-byte swizzled boxes of 64 columns) and out, the forward's output,
-        // from global memory
+        float* xch = reinterpret_cast<float*>(smem + L::OFF_XCH);
         bool ok = mbar_wait_warp(bar(Q_QD_FULL), 0, abort_flag, status, TG_WHERE_SOFTMAX);
-        ok = !pair_red_or(2 + q4, !ok);
-        if (ok && valid_row) {
-            const uint16_t* orow = out_fwd + (static_cast<size_t>(qg) * Hq + h) * HD;
+        {
             float acc = 0.f;
+            if (ok && valid_row) {
 #pragma unroll
-            for (int hf = 0; hf < HD / 64; ++hf)
-#pragma unroll
-                for (int cch = 0; cch < 8; ++cch) {
+                for (int m = 0; m < NCH; ++m) {
+                    const int col = cs * (HD / 2) + m * 8;  // first head_dim column of the chunk
+                    const int hf = col / 64, cch = (col % 64) / 8;
                     const uint4 dv = *reinterpret_cast<const uint4*>(smem + L::OFF_DO + hf * (BT * 128) + r * 128 +
                                                                      ((cch ^ (r & 7)) << 4));
-                    const uint4 ov = __ldcg(reinterpret_cast<const uint4*>(orow + hf * 64 + cch * 8));
-                    const uint32_t a[4] = {dv.x, dv.y, dv.z, dv.w}, o4[4] = {ov.x, ov.y, ov.z, ov.w};
+                    const uint32_t a[4] = {dv.x, dv.y, dv.z, dv.w}, o4[4] = {ov[m].x, ov[m].y, ov[m].z, ov[m].w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         acc = fmaf(__uint_as_float(a[e] << 16), __uint_as_float(o4[e] << 16), acc);
                         acc = fmaf(__uint_as_float(a[e] & 0xFFFF0000u), __uint_as_float(o4[e] & 0xFFFF0000u), acc);
                     }
                 }
-            fd = acc;
+            }
+            xch[(4 + cs) * BT + r] = acc;
         }
+        ok = !pair_red_or(2 + q4, !ok);
+        const float fd = xch[4 * BT + r] + xch[5 * BT + r];  // the same order in both warps
         float* wgls = reinterpret_cast<float*>(smem + L::OFF_GLS) + warp * (2 * BT);
-        // Row sums for dbeta and dtau, formed with the row's exact D' = sum_j P dP (the
-        // D above comes from the bf16 output; dtau = -sum_j dl l / tau cancels to a small
-        // number and would amplify its rounding):  sum_j dl x = sum P dP x - D' sum P x.
-        float aPdPt = 0.f, aPt = 0.f, aPdP = 0.f, aP = 0.f, aPdPg = 0.f, aPg = 0.f;
+        // Row sums for dtau, formed with the row's exact D' = sum_j P dP (the D above comes
+        // from the bf16 output; dtau = -sum_j dl l / tau cancels to a small number and would
+        // amplify its rounding):  sum_j dl x = sum P dP x - D' sum P x.
+        float aPdPt = 0.f, aPt = 0.f, aPdP = 0.f, aP = 0.f;
         // gls of the next KV tile is loaded one tile ahead (its latency hides behind a tile of work)
         float gnext[BT / 32];
 #pragma unroll
@@ -753,9 +724,9 @@ gated_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
             }
             const bool diag = (j == n_kv - 1);
             const int lim = q_local - j * BT;  // on the diagonal tile, columns > lim are future keys
-            const float* bl = wgls + s * BT;
 #pragma unroll 1
             for (int half = 0; half < 2; ++half) {
+                const int c0 = half * 64 + cs * 32;  // first key column of this warp
                 const bool okw = mbar_wait_warp(bar(Q_SDP_FULL + half), j & 1, abort_flag, status, TG_WHERE_SOFTMAX);
                 const uint32_t tb = tmem + lane_addr + half * 128;
                 float sx[32], dpx[32];
@@ -771,28 +742,31 @@ gated_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
                     ok = false;
                     break;
                 }
+                // live columns c0 + k: the row exists and, on the diagonal tile, c0 + k <= lim
+                const int nlive = diag ? lim - c0 + 1 : 32;
+                const uint32_t live = !valid_row || nlive <= 0 ? 0u : (nlive >= 32 ? 0xFFFFFFFFu : (1u << nlive) - 1u);
+                const float* bl = wgls + s * BT + c0;
                 uint32_t gg[16];
 #pragma unroll
-                for (int cc = 0; cc < 32; cc += 2) {
-                    float gv[2];
+                for (int k4 = 0; k4 < 32; k4 += 4) {
+                    const float4 g4 = *reinterpret_cast<const float4*>(bl + k4);
+                    const float glv[4] = {g4.x, g4.y, g4.z, g4.w};
+                    float gv[4];
 #pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int col = half * 64 + cs * 32 + cc + e;
-                        const float glj = bl[col];
-                        const float tt = fmaf(fa, sx[cc + e], fmaf(fb, glj, -fl));
-                        const bool keep = valid_row && !(diag && col > lim);
-                        // masked and padded entries have p = 0 and finite tt, glj: they add nothing
-                        const float p = keep ? ex2_approx(tt) : 0.f;
-                        const float pdp = p * dpx[cc + e];
+                    for (int x = 0; x < 4; ++x) {
+                        const int k = k4 + x;
+                        const float tt = fmaf(fa, sx[k], fmaf(fb, glv[x], -fl));
+                        // masked and padded entries have p = 0 and finite tt: they add nothing
+                        const float p = (live >> k) & 1u ? ex2_approx(tt) : 0.f;
+                        const float pdp = p * dpx[k];
                         aPdPt = fmaf(pdp, tt, aPdPt);
                         aPt = fmaf(p, tt, aPt);
                         aPdP += pdp;
                         aP += p;
-                        aPdPg = fmaf(pdp, glj, aPdPg);
-                        aPg = fmaf(p, glj, aPg);
-                        gv[e] = pdp - p * fd;  // G tau = P (dP - D); 1/tau is applied to dQ's rows
+                        gv[x] = fmaf(-p, fd, pdp);  // G tau = P (dP - D); 1/tau is applied to dQ's rows
                     }
-                    gg[cc / 2] = pack2_bf16(gv[0], gv[1]);
+                    gg[k4 / 2] = pack2_bf16(gv[0], gv[1]);
+                    gg[k4 / 2 + 1] = pack2_bf16(gv[2], gv[3]);
                 }
                 tmem_st16u(tb + cs * 16, gg);  // G of these 32 keys as bf16 pairs over S
                 tmem_wait_st();
@@ -825,50 +799,38 @@ gated_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
             }
         }
         // the second column half's row sums join the first's (all eight warps, abort or not)
-        float* xch = reinterpret_cast<float*>(smem + L::OFF_XCH);
         if (cs == 1) {
             xch[0 * BT + r] = aPdPt;
             xch[1 * BT + r] = aPt;
             xch[2 * BT + r] = aPdP;
             xch[3 * BT + r] = aP;
-            xch[4 * BT + r] = aPdPg;
-            xch[5 * BT + r] = aPg;
         }
         asm volatile("bar.sync 1, 256;" ::: "memory");
-        // this tile's terms of dbeta_h (sum_i sum_j G gls_j) and dc_h (sum_i ln(pos/rank) dtau),
-        // summed over its rows in a fixed order and stored at the tile's first row
-        float eE = 0.f, eT = 0.f;
+        // this tile's terms of dc_h (sum_i ln(pos/rank) dtau), summed over its rows in a fixed
+        // order and stored at the tile's first row
+        float eT = 0.f;
         if (cs == 0) {
             aPdPt += xch[0 * BT + r];
             aPt += xch[1 * BT + r];
             aPdP += xch[2 * BT + r];
             aP += xch[3 * BT + r];
-            aPdPg += xch[4 * BT + r];
-            aPg += xch[5 * BT + r];
             if (ok && valid_row) {
                 const float Dx = aPdP;
                 // tt = l log2(e) - lse log2(e):  sum dl l = ln2 (sum dl tt + lse log2(e) sum dl)
                 const float sum_dl_t = aPdPt - Dx * aPt + fl * (aPdP - Dx * aP);
-                eE = fi * (aPdPg - Dx * aPg);
                 eT = lr * (-LN2_B * fi * sum_dl_t);
-                Drow[static_cast<size_t>(qg) * Hq + h] = Dx;  // the exact D' for the dK/dV kernel
+                // the row's factors for the dK/dV kernel, with the exact D'
+                fac[static_cast<size_t>(qg) * Hq + h] = make_float4(fa, -fl, fi, -fi * Dx);
             }
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                eE += __shfl_xor_sync(0xffffffffu, eE, o);
-                eT += __shfl_xor_sync(0xffffffffu, eT, o);
-            }
+            for (int o = 16; o > 0; o >>= 1) eT += __shfl_xor_sync(0xffffffffu, eT, o);
         }
         float* red = reinterpret_cast<float*>(smem + L::OFF_MISC + 16);
-        if (cs == 0 && lane == 0) {
-            red[q4] = eE;
-            red[4 + q4] = eT;
-        }
+        if (cs == 0 && lane == 0) red[q4] = eT;
         asm volatile("bar.sync 1, 256;" ::: "memory");
         if (threadIdx.x == 0 && ok) {
             const size_t slot = (static_cast<size_t>(seq0) + static_cast<size_t>(qt) * BT) * Hq + h;
-            tileE[slot] = (red[0] + red[1]) + (red[2] + red[3]);
-            tileT[slot] = (red[4] + red[5]) + (red[6] + red[7]);
+            tileT[slot] = (red[0] + red[1]) + (red[2] + red[3]);
         }
     }
 
@@ -913,40 +875,49 @@ bwd_kv_reduce_kernel(const float* __restrict__ part_k, const float* __restrict__
 
 // ---------------------------------------------------------------------------
 // The last step, one launch:
-//   blocks 0 .. Hq-1, head h:  dg_h = sigmoid(g_h) sum_tiles tileE[., h],
-//                              dc_h = sum_tiles tileT[., h]  (one warp, fixed order);
+//   blocks 0 .. Hq-1, head h:  dg_h = sigmoid(g_h) sum_j gls_j colsum[j, h]  (dbeta_h
+//                              = sum_ij G_ij gls_j, by keys) and
+//                              dc_h = sum_tiles tileT[., h]  (fixed order);
 //   the other blocks, per key: dgls_j = sum_h softplus(g_h) colsum[j, h] and
 //                              d score_j = dgls_j (1 - exp(gls_j)).
 __global__ void __launch_bounds__(256)
-bwd_finish_kernel(const float* __restrict__ colsum, const float* __restrict__ tileE, const float* __restrict__ tileT,
-                  const float* __restrict__ gls, const float* __restrict__ g, const int32_t* __restrict__ cu_kept,
-                  int B, int64_t M, int Hq, float* __restrict__ dgls, float* __restrict__ dscore,
-                  float* __restrict__ dg, float* __restrict__ dc) {
+bwd_finish_kernel(const float* __restrict__ colsum, const float* __restrict__ tileT, const float* __restrict__ gls,
+                  const float* __restrict__ g, const int32_t* __restrict__ cu_kept, int B, int64_t M, int Hq,
+                  float* __restrict__ dgls, float* __restrict__ dscore, float* __restrict__ dg,
+                  float* __restrict__ dc) {
     pdl_wait();
     pdl_trigger();
     if (static_cast<int>(blockIdx.x) < Hq) {
         const int h = blockIdx.x;
-        if (threadIdx.x >= 32) return;
-        const int lane = threadIdx.x;
         float e = 0.f, t = 0.f;
-        int k = 0;  // running tile number: lane k % 32 takes tile k
+        // thread x takes keys x, x + 256, ... and tiles x, x + 256, ... (running tile number)
+        for (int64_t j = threadIdx.x; j < M; j += 256) e = fmaf(__ldcg(gls + j), __ldcg(colsum + j * Hq + h), e);
+        int k = 0;
         for (int b = 0; b < B; ++b) {
             const int s0 = cu_kept[b], n_qt = (cu_kept[b + 1] - s0 + BT - 1) / BT;
             for (int qt = 0; qt < n_qt; ++qt, ++k)
-                if ((k & 31) == lane) {
-                    const size_t slot = (static_cast<size_t>(s0) + static_cast<size_t>(qt) * BT) * Hq + h;
-                    e += __ldcg(tileE + slot);
-                    t += __ldcg(tileT + slot);
-                }
+                if ((k & 255) == static_cast<int>(threadIdx.x))
+                    t += __ldcg(tileT + (static_cast<size_t>(s0) + static_cast<size_t>(qt) * BT) * Hq + h);
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
             e += __shfl_xor_sync(0xffffffffu, e, o);
             t += __shfl_xor_sync(0xffffffffu, t, o);
         }
-        if (lane == 0) {
-            dg[h] = e / (1.0f + expf(-g[h]));
-            dc[h] = t;
+        __shared__ float red[2][8];
+        const int w = threadIdx.x >> 5;
+        if ((threadIdx.x & 31) == 0) {
+            red[0][w] = e;
+            red[1][w] = t;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            const float se = ((red[0][0] + red[0][1]) + (red[0][2] + red[0][3])) +
+                             ((red[0][4] + red[0][5]) + (red[0][6] + red[0][7]));
+            const float st = ((red[1][0] + red[1][1]) + (red[1][2] + red[1][3])) +
+                             ((red[1][4] + red[1][5]) + (red[1][6] + red[1][7]));
+            dg[h] = se / (1.0f + expf(-g[h]));
+            dc[h] = st;
         }
         return;
     }
@@ -972,13 +943,14 @@ cudaError_t launch_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
     if (cudaError_t e = ensure_smem_limit(gated_attn_bwd_dq_kernel<HD>, DqSmem<HD>::ALLOC, set_dq); e != cudaSuccess)
         return e;
     const size_t rows = static_cast<size_t>(M_total) * Hq;
-    float* Drow = static_cast<float*>(ws);
-    float* colsum = Drow + rows;
-    float* tileE = colsum + rows;  // per query tile, at its first row
-    float* tileT = tileE + rows;
+    // every section starts on a 16-byte boundary (the partials are written as float4)
+    const size_t rows4 = (rows + 3) & ~static_cast<size_t>(3);
+    float4* fac = static_cast<float4*>(ws);  // per query row and head: fa, -lse log2(e), 1/tau, -D'/tau
+    float* colsum = reinterpret_cast<float*>(fac + rows);
+    float* tileT = colsum + rows4;  // per query tile, at its first row
     const int grp = Hq / Hkv;
     const int64_t nkv = M_total * Hkv * HD;
-    float* part_k = grp > 1 ? tileT + rows : nullptr;  // [grp][M][Hkv][HD] each
+    float* part_k = grp > 1 ? tileT + rows4 : nullptr;  // [grp][M][Hkv][HD] each
     float* part_v = grp > 1 ? part_k + grp * nkv : nullptr;
     CUtensorMap tq, tk, tv, tdo;
     if (!encode_tmap_2d_bf16(&tq, q, static_cast<uint64_t>(Hq) * HD, static_cast<uint64_t>(M_total),
@@ -999,11 +971,11 @@ cudaError_t launch_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
     // D' = sum_j P dP for the dK/dV kernel
     cudaError_t e = launch_pdl(gated_attn_bwd_dq_kernel<HD>, dim3(Hq, n_t, B), dim3(DQ_THREADS),
                                static_cast<size_t>(DqSmem<HD>::ALLOC), st, tq, tk, tv, tdo, cu_kept, pos, rank, gls, g,
-                               c, lse, out, Drow, sm_scale, Hq, Hkv, n_t, dq, tileE, tileT, status);
+                               c, lse, out, fac, sm_scale, Hq, Hkv, n_t, dq, tileT, status);
     if (e != cudaSuccess) return e;
     e = launch_pdl(gated_attn_bwd_dkv_kernel<HD>, dim3(Hq, n_t, B), dim3(DKV_THREADS),
-                   static_cast<size_t>(DkvSmem<HD>::ALLOC), st, tq, tk, tv, tdo, cu_kept, pos, rank, gls, g, c, lse,
-                   static_cast<const float*>(Drow), sm_scale, Hq, Hkv, M_total, dk, dv, part_k, part_v, colsum,
+                   static_cast<size_t>(DkvSmem<HD>::ALLOC), st, tq, tk, tv, tdo, cu_kept, gls, g,
+                   static_cast<const float4*>(fac), sm_scale, Hq, Hkv, M_total, dk, dv, part_k, part_v, colsum,
                    status);
     if (e != cudaSuccess) return e;
     if (grp > 1) {
@@ -1016,14 +988,16 @@ cudaError_t launch_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
     const int64_t kb = (M_total + 255) / 256;
     const int key_blocks = static_cast<int>(kb < sms * 4 ? kb : sms * 4);
     return launch_pdl(bwd_finish_kernel, dim3(Hq + key_blocks), dim3(256), 0, st, static_cast<const float*>(colsum),
-                      static_cast<const float*>(tileE), static_cast<const float*>(tileT), gls, g, cu_kept, B, M_total,
-                      Hq, dgls, dscore, dg, dc);
+                      static_cast<const float*>(tileT), gls, g, cu_kept, B, M_total, Hq, dgls, dscore, dg, dc);
 }
 
 }  // namespace
 
 size_t attention_backward_workspace_bytes(int64_t M_total, int Hq, int Hkv, int d) {
-    const size_t rows = static_cast<size_t>(4) * static_cast<size_t>(M_total) * static_cast<size_t>(Hq);
+    // a float4 of factors, the key sum of G and a tile sum per row and head, each
+    // section padded to 16 bytes
+    const size_t mh = static_cast<size_t>(M_total) * static_cast<size_t>(Hq);
+    const size_t rows = 4 * mh + 2 * ((mh + 3) & ~static_cast<size_t>(3));
     const int grp = Hkv > 0 ? Hq / Hkv : 1;
     const size_t parts = grp > 1 ? static_cast<size_t>(2) * grp * static_cast<size_t>(M_total) * Hkv * d : 0;
     return (rows + parts) * sizeof(float);
