@@ -74,12 +74,14 @@ def test_score_parity(tg, name):
     assert (s[~m] == 0).all(), "non-prunable entries must be left untouched"
 
 
-def test_score_ragged_spans(tg):
-    """Spans that start at 0, end at N, are empty, or hold one token; D=256."""
+@pytest.mark.parametrize("I", [64, 48])
+def test_score_ragged_spans(tg, I):
+    """Spans that start at 0, end at N, are empty, or hold one token; D=256; I = 48
+    leaves a 16-column tail in the epilogue."""
     rng = np.random.default_rng(5)
     seqlens = [1, 130, 257, 64, 300]
     spans = [(0, 1), (0, 130), (3, 200), (10, 10), (299, 300)]
-    D, I = 256, 64
+    D = 256
     T = sum(seqlens)
     from workloads import f32_to_bf16_bits
     hidden = f32_to_bf16_bits(rng.standard_normal((T, D)).astype(np.float32))
@@ -96,6 +98,33 @@ def test_score_ragged_spans(tg):
     m = ~np.isnan(s_ref)
     assert m.sum() == 1 + 130 + 197 + 0 + 1
     assert H.score_error(s[m], s_ref[m]) <= H.SCORE_REL
+
+
+@pytest.mark.parametrize("D,I", [(512, 128), (256, 256), (256, 48)])
+def test_score_ragged_spans_above_one_tile_per_sm(tg, D, I):
+    """More 128-row tiles than SMs (256-row tiles on a 148-SM part): four sequences
+    with spans that are ragged, empty, one token long and whole; I = 48 leaves a
+    16-column tail in the epilogue."""
+    rng = np.random.default_rng(6 + I)
+    seqlens = [7000, 1, 9000, 5000]
+    spans = [(17, 6999), (0, 1), (0, 9000), (2500, 2500)]
+    T = sum(seqlens)
+    from workloads import f32_to_bf16_bits
+    hidden = f32_to_bf16_bits(rng.standard_normal((T, D)).astype(np.float32))
+    gamma = f32_to_bf16_bits((1 + 0.1 * rng.standard_normal(D)).astype(np.float32))
+    W1 = f32_to_bf16_bits((rng.standard_normal((D, I)) / np.sqrt(D)).astype(np.float32))
+    b1 = (0.1 * rng.standard_normal(I)).astype(np.float32)
+    w2 = (rng.standard_normal(I) / np.sqrt(I)).astype(np.float32)
+    cu = np.concatenate([[0], np.cumsum(seqlens)]).astype(np.int32)
+    span = np.array(spans, np.int32)
+    Wg = oracle.gate_fold(gamma, W1)
+    s_ref = oracle.score(hidden, cu, span, Wg, b1, w2, -0.2, 1e-6)
+    s = tg.tg_score(H.bf16_dev(hidden), cu, span, H.bf16_dev(Wg), H.f32_dev(b1), H.f32_dev(w2), -0.2,
+                    1e-6).cpu().numpy()
+    m = ~np.isnan(s_ref)
+    assert m.sum() == 6982 + 1 + 9000 + 0
+    assert H.score_error(s[m], s_ref[m]) <= H.SCORE_REL
+    assert (s[~m] == 0).all(), "non-prunable entries must be left untouched"
 
 
 # ------------------------------------------------------------------ stage 2 + 3
