@@ -279,14 +279,20 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
             tc_fence_after();
             const float rr = rsqrtf(ss / static_cast<float>(D) + eps);
             float acc_s = 0.f;
-            for (int c0 = 0; c0 < I; c0 += 32) {
-                const int nq = min(32, I - c0);  // 16 or 32: I is a multiple of 16
+            const int I32 = I & ~31;
+            for (int c0 = 0; c0 < I32; c0 += 32) {
                 float z[32];
                 tmem_ld32(tmem + a * 256 + lane_addr + c0, z);
                 tmem_wait_ld();
 #pragma unroll
-                for (int q = 0; q < 32; ++q)
-                    if (q < nq) acc_s = fmaf(s_w2[c0 + q], silu_f(fmaf(rr, z[q], s_b1[c0 + q])), acc_s);
+                for (int q = 0; q < 32; ++q) acc_s = fmaf(s_w2[c0 + q], silu_f(fmaf(rr, z[q], s_b1[c0 + q])), acc_s);
+            }
+            if (I32 < I) {  // the last 16 columns when I is 16 mod 32
+                float z[32];
+                tmem_ld32(tmem + a * 256 + lane_addr + I32, z);
+                tmem_wait_ld();
+#pragma unroll
+                for (int q = 0; q < 16; ++q) acc_s = fmaf(s_w2[I32 + q], silu_f(fmaf(rr, z[q], s_b1[I32 + q])), acc_s);
             }
             tc_fence_before();
             __syncwarp();
