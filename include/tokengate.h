@@ -220,7 +220,8 @@ tg_status tg_gated_attention_gates(const uint16_t* q, const uint16_t* k, const u
  * TG_ERR_UNSUPPORTED).  ws: device scratch, 256-byte aligned, of at least
  * tg_gated_attention_backward_workspace_size(M_total, Hq, Hkv, d) bytes (6
  * floats per row and head, plus fp32 partial dk and dv per query head when a
- * KV head serves two or more; no zeroing needed).  Tensor cores, no atomics:
+ * KV head serves 3, 5, 6, 7 or more than 8 query heads; groups of 2, 4 and 8
+ * add theirs inside a thread-block cluster; no zeroing needed).  Tensor cores, no atomics:
  * the results are deterministic.
  */
 size_t tg_gated_attention_backward_workspace_size(int64_t M_total, int Hq, int Hkv, int d);

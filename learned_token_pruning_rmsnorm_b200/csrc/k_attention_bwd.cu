@@ -125,12 +125,17 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
                           const float* __restrict__ g, const float4* __restrict__ fac, float sm_scale, int Hq,
                           int Hkv, int64_t M_total,
                           uint16_t* __restrict__ dk, uint16_t* __restrict__ dv, float* __restrict__ part_k,
-                          float* __restrict__ part_v, float* __restrict__ colsum, int* __restrict__ status) {
+                          float* __restrict__ part_v, float* __restrict__ colsum, int* __restrict__ status,
+                          int cl) {
     using L = DkvSmem<HD>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    // one query head per CTA: the heads of a GQA group leave partial dK / dV (fp32, summed
-    // in head order by bwd_kv_reduce_kernel); a group of one writes bf16 directly
+    // One query head per CTA.  The heads of a GQA group of 2, 4 or 8 run as one cluster
+    // (cl = the group size, cluster rank = head within the group): at the end the other
+    // heads' fp32 dK / dV go into their own shared memory and rank 0 adds them in head
+    // order and writes bf16.  Other groups of two or more leave fp32 partials that
+    // bwd_kv_reduce_kernel sums in head order; a group of one writes bf16 directly.  A
+    // cluster's CTAs share kt and b, so they return here together or not at all.
     const int h = blockIdx.x, kt = blockIdx.y, b = blockIdx.z;
     pdl_wait();  // global memory is read only from here on
     pdl_trigger();
@@ -174,6 +179,7 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
     // P^T and G^T (bf16 pairs) go over the first 32 columns of each
     const uint32_t tDV = tmem + 2 * BT, tDK = tmem + 2 * BT + HD;
 
+    bool epi_ok = false;  // a compute thread's accumulators are complete
     if (warp == 8) {
         // ---------------------------------------------------------------- TMA producer
         if (lane == 0) {
@@ -377,7 +383,29 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
         if (cs == 0 && ok && valid_key) colsum[static_cast<size_t>(seq0 + key_local) * Hq + h] = csum + xch[r];
         // ---------------------------------------------------------------- epilogue
         if (ok) ok = mbar_wait_warp(bar(D_ACC_DONE), 0, abort_flag, status, TG_WHERE_SOFTMAX);
-        if (ok && part_k) {
+        epi_ok = ok;
+        if (cl > 1) {
+            // heads 1 .. cl-1 of the group: this head's fp32 dV and dK into the exchange area
+            // (the Q/dO stages, idle now), [dV|dK][HD/4 column quads][128 rows] float4s
+            if (ok && hh != 0) {
+                tc_fence_after();
+                float4* xa = reinterpret_cast<float4*>(smem + L::OFF_Q);
+#pragma unroll 1
+                for (int which = 0; which < 2; ++which) {
+#pragma unroll
+                    for (int ch = 0; ch < HD / 64; ++ch) {
+                        float o[32];
+                        tmem_ld32((which ? tDK : tDV) + cs * (HD / 2) + lane_addr + ch * 32, o);
+                        tmem_wait_ld();
+                        const int c4 = (cs * (HD / 2) + ch * 32) / 4;
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            xa[(which * (HD / 4) + c4 + q) * BT + r] =
+                                make_float4(o[q * 4], o[q * 4 + 1], o[q * 4 + 2], o[q * 4 + 3]);
+                    }
+                }
+            }
+        } else if (ok && part_k) {
             // partials of this head: [head in group][row][KV head][d] fp32, unscaled; warp cs
             // writes head_dim columns cs HD/2 .. + HD/2 - 1 of its rows
             tc_fence_after();
@@ -430,6 +458,55 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
 
     tc_fence_before();
     __syncthreads();
+    if (cl > 1) {
+        // every thread of the cluster, abort or not
+        cluster_sync_all();  // the other heads' copies are in their shared memory
+        if (hh == 0 && warp < 8 && epi_ok) {
+            // rank 0: dK = sm (dK_0 + dK_1 + ...), dV = dV_0 + dV_1 + ... in head order, to bf16
+            tc_fence_after();
+            const int q4 = warp & 3, cs = warp >> 2;
+            const int r = q4 * 32 + lane;
+            const int key_local = kt * BT + r;
+            const uint32_t lane_addr = static_cast<uint32_t>(q4 * 32) << 16;
+            const uint32_t xa_local = sbase + L::OFF_Q;
+            const size_t row = (static_cast<size_t>(seq0 + key_local) * Hkv + hk) * HD + cs * (HD / 2);
+#pragma unroll 1
+            for (int which = 0; which < 2; ++which) {
+                const float scale = which ? sm_scale : 1.0f;
+                uint16_t* dst = (which ? dk : dv) + row;
+#pragma unroll 1
+                for (int ch = 0; ch < HD / 64; ++ch) {
+                    float o[32];
+                    tmem_ld32((which ? tDK : tDV) + cs * (HD / 2) + lane_addr + ch * 32, o);
+                    tmem_wait_ld();
+                    const int c4 = (cs * (HD / 2) + ch * 32) / 4;
+                    for (int rk = 1; rk < cl; ++rk) {
+                        const uint32_t base = mapa_shared(xa_local, static_cast<uint32_t>(rk));
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const float4 v = ld_dsmem_f4(base + static_cast<uint32_t>(((which * (HD / 4) + c4 + q) * BT + r) * 16));
+                            o[q * 4] += v.x;
+                            o[q * 4 + 1] += v.y;
+                            o[q * 4 + 2] += v.z;
+                            o[q * 4 + 3] += v.w;
+                        }
+                    }
+                    if (key_local < Mb) {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            uint4 w;
+                            w.x = pack2_bf16(o[q * 8 + 0] * scale, o[q * 8 + 1] * scale);
+                            w.y = pack2_bf16(o[q * 8 + 2] * scale, o[q * 8 + 3] * scale);
+                            w.z = pack2_bf16(o[q * 8 + 4] * scale, o[q * 8 + 5] * scale);
+                            w.w = pack2_bf16(o[q * 8 + 6] * scale, o[q * 8 + 7] * scale);
+                            *reinterpret_cast<uint4*>(dst + ch * 32 + q * 8) = w;
+                        }
+                    }
+                }
+            }
+        }
+        cluster_sync_all();  // rank 0 has read the other heads' shared memory
+    }
     if (warp == 8) {
         tc_fence_after();
         tmem_dealloc(tmem, L::TMEM_COLS);
@@ -930,6 +1007,9 @@ bwd_finish_kernel(const float* __restrict__ colsum, const float* __restrict__ ti
     }
 }
 
+// GQA groups of 2, 4 or 8 heads run their dK/dV CTAs as one cluster (portable sizes).
+inline int bwd_cluster_size(int grp) { return grp == 2 || grp == 4 || grp == 8 ? grp : 0; }
+
 template <int HD>
 cudaError_t launch_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* out,
                        const uint16_t* dout, const float* lse, const int32_t* cu_kept, int B, int64_t M_total,
@@ -949,9 +1029,10 @@ cudaError_t launch_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
     float* colsum = reinterpret_cast<float*>(fac + rows);
     float* tileT = colsum + rows4;  // per query tile, at its first row
     const int grp = Hq / Hkv;
+    const int cl = bwd_cluster_size(grp);  // the group's heads as one cluster, else partials
     const int64_t nkv = M_total * Hkv * HD;
-    float* part_k = grp > 1 ? tileT + rows4 : nullptr;  // [grp][M][Hkv][HD] each
-    float* part_v = grp > 1 ? part_k + grp * nkv : nullptr;
+    float* part_k = grp > 1 && cl == 0 ? tileT + rows4 : nullptr;  // [grp][M][Hkv][HD] each
+    float* part_v = part_k ? part_k + grp * nkv : nullptr;
     CUtensorMap tq, tk, tv, tdo;
     if (!encode_tmap_2d_bf16(&tq, q, static_cast<uint64_t>(Hq) * HD, static_cast<uint64_t>(M_total),
                              static_cast<uint64_t>(Hq) * HD * 2, 64, BT) ||
@@ -973,12 +1054,18 @@ cudaError_t launch_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
                                static_cast<size_t>(DqSmem<HD>::ALLOC), st, tq, tk, tv, tdo, cu_kept, pos, rank, gls, g,
                                c, lse, out, fac, sm_scale, Hq, Hkv, n_t, dq, tileT, status);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(gated_attn_bwd_dkv_kernel<HD>, dim3(Hq, n_t, B), dim3(DKV_THREADS),
-                   static_cast<size_t>(DkvSmem<HD>::ALLOC), st, tq, tk, tv, tdo, cu_kept, gls, g,
-                   static_cast<const float4*>(fac), sm_scale, Hq, Hkv, M_total, dk, dv, part_k, part_v, colsum,
-                   status);
+    if (cl > 1)
+        e = launch_pdl_cluster(gated_attn_bwd_dkv_kernel<HD>, dim3(Hq, n_t, B), dim3(DKV_THREADS),
+                               static_cast<size_t>(DkvSmem<HD>::ALLOC), st, static_cast<unsigned>(cl), tq, tk, tv, tdo,
+                               cu_kept, gls, g, static_cast<const float4*>(fac), sm_scale, Hq, Hkv, M_total, dk, dv,
+                               part_k, part_v, colsum, status, cl);
+    else
+        e = launch_pdl(gated_attn_bwd_dkv_kernel<HD>, dim3(Hq, n_t, B), dim3(DKV_THREADS),
+                       static_cast<size_t>(DkvSmem<HD>::ALLOC), st, tq, tk, tv, tdo, cu_kept, gls, g,
+                       static_cast<const float4*>(fac), sm_scale, Hq, Hkv, M_total, dk, dv, part_k, part_v, colsum,
+                       status, 0);
     if (e != cudaSuccess) return e;
-    if (grp > 1) {
+    if (part_k) {
         const int64_t rb = (nkv / 8 + 255) / 256;
         e = launch_pdl(bwd_kv_reduce_kernel, dim3(static_cast<unsigned>(rb < sms * 8 ? rb : sms * 8)), dim3(256), 0, st,
                        static_cast<const float*>(part_k), static_cast<const float*>(part_v), grp, nkv, sm_scale, dk,
@@ -999,7 +1086,8 @@ size_t attention_backward_workspace_bytes(int64_t M_total, int Hq, int Hkv, int 
     const size_t mh = static_cast<size_t>(M_total) * static_cast<size_t>(Hq);
     const size_t rows = 4 * mh + 2 * ((mh + 3) & ~static_cast<size_t>(3));
     const int grp = Hkv > 0 ? Hq / Hkv : 1;
-    const size_t parts = grp > 1 ? static_cast<size_t>(2) * grp * static_cast<size_t>(M_total) * Hkv * d : 0;
+    const size_t parts =
+        grp > 1 && bwd_cluster_size(grp) == 0 ? static_cast<size_t>(2) * grp * static_cast<size_t>(M_total) * Hkv * d : 0;
     return (rows + parts) * sizeof(float);
 }
 
