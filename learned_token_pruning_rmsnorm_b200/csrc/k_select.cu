@@ -552,8 +552,11 @@ cudaError_t launch_gather_bytes(const void* src, const int32_t* kept_idx, int64_
     const int grid = static_cast<int>(blocks_needed < static_cast<int64_t>(sms) * 8 ? blocks_needed : sms * 8);
     const uint4* h = static_cast<const uint4*>(src);
     uint4* o = static_cast<uint4*>(dst);
+    // one round trip per row where it fits: all of a 4 KB or 2 KB row's loads in flight before its stores
     if (vpr >= 256)
         return launch_pdl(gather_rows_kernel<8>, dim3(grid), dim3(256), 0, st, h, kept_idx, M_total, T, vpr, o, wae);
+    if (vpr >= 128)
+        return launch_pdl(gather_rows_kernel<4>, dim3(grid), dim3(256), 0, st, h, kept_idx, M_total, T, vpr, o, wae);
     return launch_pdl(gather_rows_kernel<2>, dim3(grid), dim3(256), 0, st, h, kept_idx, M_total, T, vpr, o, wae);
 }
 

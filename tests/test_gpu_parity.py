@@ -343,7 +343,7 @@ def test_prefill_layer_end_to_end(tg, name):
 
 # ------------------------------------------------------------------ KV-cache gather (next row f2)
 
-@pytest.mark.parametrize("row_shape", [(8, 128), (2, 64), (8,), (24,), (1, 2056)])
+@pytest.mark.parametrize("row_shape", [(8, 128), (2, 64), (8,), (24,), (1, 2056), (1, 1544)])
 def test_gather_rows_matches_oracle_gather(tg, row_shape):
     """dst[m] = src[kept_idx[m]] for rows of any width that is a multiple of 16 bytes
     (the [T, Hkv, d] K/V cache of a layer below the gate among them), bit-exact against
