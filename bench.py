@@ -64,6 +64,22 @@ def dist_env():
     return ws, rank, local
 
 
+def max_over_ranks(vals, ws, device):
+    """Element-wise max of per-rank device timings over all ranks of the process group
+    (a no-op on one rank): the job's time is its slowest rank's."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
+    if ws > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
+def job_rate(ws, units_per_rank_step, steps, t_total_ms):
+    """Whole-job throughput: the units every rank processed over the (slowest rank's) time."""
+    return ws * units_per_rank_step * steps / (t_total_ms / 1e3)
+
+
 def attention_flops(cu_kept, Hq, d):
     m = np.diff(np.asarray(cu_kept, np.int64))
     pairs = int(np.sum(m * (m + 1) // 2))
@@ -548,15 +564,11 @@ def run_gpu(args, w):
     e2e_ms = float(np.sum([a.elapsed_time(b) for a, b in e2e_ev]))
 
     # ---------------- max over ranks
-    t_total_ms = float(np.sum(step_ms))
-    vals = torch.tensor([t_total_ms, e2e_ms], dtype=torch.float64, device=dev)
-    if ws > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    t_total_ms, e2e_ms = float(vals[0]), float(vals[1])
+    t_total_ms, e2e_ms = max_over_ranks([float(np.sum(step_ms)), e2e_ms], ws, dev)
 
     ms_per_step = t_total_ms / args.steps
-    value = ws * w.T * args.steps / (t_total_ms / 1e3)
-    e2e_value = ws * w.T * args.steps / (e2e_ms / 1e3)
+    value = job_rate(ws, w.T, args.steps, t_total_ms)
+    e2e_value = job_rate(ws, w.T, args.steps, e2e_ms)
 
     flops, pairs = attention_flops(cu_kept, w.Hq, w.d)
     attn_tflops = flops / (stage_us["attention"] * 1e-6) / 1e12
