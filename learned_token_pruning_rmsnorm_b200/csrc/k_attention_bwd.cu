@@ -534,7 +534,7 @@ struct DqSmem {
     static constexpr int OFF_K = OFF_DO + TILE;        // [2 stages]
     static constexpr int OFF_V = OFF_K + 2 * TILE;     // [2 stages]
     static constexpr int OFF_GLS = OFF_V + 2 * TILE;   // [8 warps][2][BT] fp32, a private copy per warp
-    static constexpr int OFF_XCH = OFF_GLS + 8 * 2 * BT * 4;  // [6][BT] fp32: the second column half's row sums
+    static constexpr int OFF_XCH = OFF_GLS + 8 * 2 * BT * 4;  // [6][BT] fp32: row sums [0..3], D halves [4..5]
     static constexpr int OFF_BAR = OFF_XCH + 6 * BT * 4;
     static constexpr int NUM_BARS = 16;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;  // tmem slot, abort flag, then 8 fp32
