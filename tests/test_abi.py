@@ -43,6 +43,49 @@ def test_library_exports_every_declared_symbol(lib):
         assert n in _lib.SIGNATURES, f"{n} has no binding signature"
 
 
+_C_PROGRAM = r"""
+#include "tokengate.h"
+#include <stdio.h>
+#include <string.h>
+
+int main(void) {
+    int32_t span[4] = {2, 8, 0, 15}, k[2] = {3, -1}, next[4];
+    tg_status st;
+    if (tg_abi_version() != 5) return 1;
+    /* host-only helper: the next gate's span in this gate's kept order */
+    if (tg_next_gate_span(span, k, 2, next) != TG_OK) return 2;
+    if (next[0] != 2 || next[1] != 5 || next[2] != 0 || next[3] != 15) return 3;
+    /* refused before any device work: D = 100 is not a multiple of 64 */
+    st = tg_score(NULL, NULL, NULL, 1, 128, 100, NULL, NULL, NULL, 0.0f, 64, 1e-6f, NULL, NULL);
+    if (st != TG_ERR_UNSUPPORTED) return 4;
+    if (strstr(tg_last_error_string(), "D=100") == NULL) return 5;
+    if (tg_gated_attention_backward_workspace_size(7, 3, 1, 64) != (size_t)(132 + 2688) * 4) return 6;
+    printf("ok\n");
+    return 0;
+}
+"""
+
+
+def test_header_compiles_as_c_and_the_library_links(lib, tmp_path):
+    """The header is plain C (C11, warnings as errors) and a C program links the
+    library and calls it without PyTorch (host-side entry points only)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no gcc")
+    pkg = os.path.join(ROOT, "learned_token_pruning_rmsnorm_b200")
+    src = tmp_path / "prog.c"
+    src.write_text(_C_PROGRAM)
+    exe = tmp_path / "prog"
+    cmd = [gcc, "-std=c11", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+           str(src), "-L", pkg, "-ltokengate", "-Wl,-rpath," + pkg, "-o", str(exe)]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
+
+
 def test_abi_version(lib):
     assert lib.tg_abi_version() == 5
 
