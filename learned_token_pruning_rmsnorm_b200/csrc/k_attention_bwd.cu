@@ -137,7 +137,10 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
     // bwd_kv_reduce_kernel sums in head order; a group of one writes bf16 directly.  A
     // cluster's CTAs share kt and b, so they return here together or not at all.
     const int h = blockIdx.x, kt = blockIdx.y, b = blockIdx.z;
-    pdl_wait();  // global memory is read only from here on
+    // Early start: every input but the dQ kernel's factor records was complete before the dQ
+    // kernel (this kernel's predecessor) passed its own wait, and this kernel starts only
+    // after that, so the set-up and the tile loads go ahead while the dQ kernel drains; only
+    // the compute warps wait, before their first factor record.
     pdl_trigger();
     const int seq0 = cu_kept[b];
     const int Mb = cu_kept[b + 1] - seq0;
@@ -310,6 +313,7 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
             return qrow < Mb ? __ldcg(fac + static_cast<size_t>(seq0 + qrow) * Hq + h)
                              : make_float4(0.f, 0.f, 0.f, 0.f);
         };
+        pdl_wait();  // the dQ kernel's factor records are complete from here on
         float4 fnext = load_fac(0);
         for (int u = 0; u < n_u; ++u) {
             const int t = u >> 1, hb = u & 1, i = kt + t;
