@@ -198,10 +198,19 @@ def gated_attention(q_bits, k_bits, v_bits, cu_kept, pos, rank, gls_f32, g, c, s
     return out, lse
 
 
-def gated_attention_backward(q_bits, k_bits, v_bits, cu_kept, pos, rank, gls_f32, g, c, dout, sm_scale=None) -> dict:
+def gated_attention_backward(q_bits, k_bits, v_bits, cu_kept, pos, rank, gls_f32, g, c, dout, sm_scale=None,
+                             scores=None, prunable=None) -> dict:
     """Gradients of the token-gated attention (one gate) for the upstream
     gradient dout [M, Hq, d]: dq [M, Hq, d], dk/dv [M, Hkv, d], dgls [M],
-    dg/dc [Hq], all fp64.  d loss / d score_j = dgls_j * sigmoid(-score_j)."""
+    dg/dc [Hq], all fp64.
+
+    With the kept rows' gate scores (scores [M] fp32, the s_j whose
+    logsigmoid is gls_j) and the rows the gate could prune (prunable [M]
+    bool), it also returns dscore [M]: the gradient that reaches the gate's
+    score through the bias (AI summary, "Key Contributions" 2: the bias on
+    the logits carries the task loss back to the scoring network).  Since
+    gls_j = logsigmoid(s_j), d gls_j / d s_j = sigmoid(-s_j), taken here from
+    the score itself; rows the gate cannot prune carry no bias and get 0."""
     q, qp = _c(q_bits, np.uint16)
     k, kp = _c(k_bits, np.uint16)
     v, vp_ = _c(v_bits, np.uint16)
@@ -222,6 +231,12 @@ def gated_attention_backward(q_bits, k_bits, v_bits, cu_kept, pos, rank, gls_f32
     _load().oracle_gated_attention_backward(qp, kp, vp_, cup, len(cu) - 1, Hq, Hkv, d, pop, rap, glp, gap, cap,
                                             float(sm_scale), gop, vp(out["dq"]), vp(out["dk"]), vp(out["dv"]),
                                             vp(out["dgls"]), vp(out["dg"]), vp(out["dc"]))
+    if scores is not None:
+        s64 = np.asarray(scores, dtype=np.float64).reshape(M)
+        mask = np.ones(M, dtype=bool) if prunable is None else np.asarray(prunable, dtype=bool).reshape(M)
+        # sigmoid(-s) = exp(-log(1 + e^s)), finite for every s
+        sig_neg = np.exp(-np.logaddexp(0.0, np.where(mask, s64, 0.0)))
+        out["dscore"] = np.where(mask, out["dgls"] * sig_neg, 0.0)
     return out
 
 

@@ -4,8 +4,10 @@ oracle, through the C ABI.
 Bars, relative to each gradient's own scale (the tensor cores take P and G as
 bf16 operands, 2^-9 relative, and dq/dk/dv are returned in bf16):
   dq, dk, dv      max-abs <= 3e-2 * max|ref|, mean-abs <= 6e-3 * mean|ref|
-  dgls            max-abs <= 1e-2 * max|ref|
+  dgls, dscore    max-abs <= 1e-2 * max|ref|
   dg, dc          max-abs <= 1e-2 * max|ref|
+dscore is compared with the oracle's, which takes it from the kept rows' gate
+scores themselves (sigmoid(-s) times d gls), not from the kernel's identity.
 """
 
 import functools
@@ -44,12 +46,14 @@ def _rand_case(seed, seqlens, Hq, Hkv, d, std=0.5):
     rank = np.concatenate([np.arange(1, n + 1) for n in seqlens]).astype(np.int32)
     pos = (rank + np.concatenate([np.sort(rng.integers(0, 400, n)) for n in seqlens])).astype(np.int32)
     s = (2 * rng.standard_normal(M)).astype(np.float32)
-    gls = (np.minimum(s, 0) - np.log1p(np.exp(-np.abs(s.astype(np.float64))))).astype(np.float32)
-    gls[:24] = 0.0  # rows the gate cannot prune
+    prunable = np.arange(M) >= 24  # the first 24 rows are ones the gate cannot prune
+    gls = np.where(prunable, np.minimum(s, 0) - np.log1p(np.exp(-np.abs(s.astype(np.float64)))), 0.0)
+    gls = gls.astype(np.float32)
     g = rng.standard_normal(Hq).astype(np.float32)
     c = (0.5 * rng.random(Hq)).astype(np.float32)
     dout = f32_to_bf16_bits(rng.standard_normal((M, Hq, d)).astype(np.float32))
-    return {"q": q, "k": k, "v": v, "cu": cu, "pos": pos, "rank": rank, "gls": gls, "g": g, "c": c, "dout": dout}
+    return {"q": q, "k": k, "v": v, "cu": cu, "pos": pos, "rank": rank, "gls": gls, "g": g, "c": c, "dout": dout,
+            "s": s, "prunable": prunable}
 
 
 def _gpu_backward(tg, cs):
@@ -70,17 +74,23 @@ def _check(got, ref, cs, what):
         scale = np.abs(ref[key])
         assert err.max() <= GRAD_MAX_REL * scale.max(), f"{what} {key}: max {err.max():.3e} vs {scale.max():.3e}"
         assert err.mean() <= GRAD_MEAN_REL * scale.mean(), f"{what} {key}: mean {err.mean():.3e} vs {scale.mean():.3e}"
-    for key in ("dgls", "dg", "dc"):
+    for key in ("dgls", "dscore", "dg", "dc"):
         err = np.abs(got[key] - ref[key])
         assert err.max() <= SUM_MAX_REL * np.abs(ref[key]).max(), f"{what} {key}: {err.max():.3e}"
-    want = ref["dgls"] * -np.expm1(cs["gls"].astype(np.float64))
-    assert np.abs(got["dscore"] - want).max() <= SUM_MAX_REL * np.abs(want).max() + 1e-30
-    assert (got["dscore"][cs["gls"] == 0] == 0).all()
+    assert (got["dscore"][~cs["prunable"]] == 0).all()
+
+
+def _in_span(src, cu, span):
+    """Kept rows whose source token lies in its sequence's prunable span."""
+    b = np.searchsorted(cu, src, side="right") - 1
+    local = src - cu[b]
+    return (local >= span[b, 0]) & (local < span[b, 1])
 
 
 def _oracle_backward(cs):
     return oracle.gated_attention_backward(cs["q"], cs["k"], cs["v"], cs["cu"], cs["pos"], cs["rank"], cs["gls"],
-                                           cs["g"], cs["c"], bf16_bits_to_f32(cs["dout"]).astype(np.float64))
+                                           cs["g"], cs["c"], bf16_bits_to_f32(cs["dout"]).astype(np.float64),
+                                           scores=cs["s"], prunable=cs["prunable"])
 
 
 # GQA groups of 2, 4 and 8 heads reduce dK / dV inside a thread-block cluster; a group of 3
@@ -108,7 +118,8 @@ def test_backward_at_the_bench_workload(tg):
     rng = np.random.default_rng(8)
     cs = {"q": ai["q"], "k": ai["k"], "v": ai["v"], "cu": comp["cu_kept"], "pos": comp["pos"], "rank": comp["rank"],
           "gls": comp["gls"].astype(np.float32), "g": ai["g"], "c": ai["c"],
-          "dout": f32_to_bf16_bits(rng.standard_normal((M, w.Hq, w.d)).astype(np.float32))}
+          "dout": f32_to_bf16_bits(rng.standard_normal((M, w.Hq, w.d)).astype(np.float32)),
+          "s": s[comp["src"]], "prunable": _in_span(comp["src"], cu, span)}
     got = _gpu_backward(tg, cs)
     ref = _oracle_backward(cs)
     _check(got, ref, cs, "c2_32k_k2000")

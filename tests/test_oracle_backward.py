@@ -127,3 +127,36 @@ def test_temperature_gradient_vanishes_where_pos_equals_rank(oracle_mod):
     got = oracle_mod.gated_attention_backward(q, k, v, cu, rank.copy(), rank, gls, g, c, dout)
     assert (got["dc"] == 0).all()
     assert np.abs(got["dg"]).max() > 1e-6
+
+
+def _logsigmoid(s):
+    s = np.asarray(s, dtype=np.float64)
+    return np.minimum(s, 0.0) - np.log1p(np.exp(-np.abs(s)))
+
+
+def test_score_gradient_matches_central_differences(oracle_mod):
+    """d loss / d s_j, pinned by differencing the oracle's forward in the gate score
+    itself: s_j is moved by +-2^-6 and gls_j = logsigmoid(s_j) recomputed, so a sign,
+    a missing factor or sigmoid(s) in place of sigmoid(-s) in dscore fails by O(1).
+    Rows the gate cannot prune (gls = 0, no bias) get 0."""
+    q, k, v, cu, pos, rank, gls, g, c, dout = _case(7, [14, 11], 4, 2, 8)
+    rng = np.random.default_rng(70)
+    s = (2.0 * rng.standard_normal(len(gls))).astype(np.float32)
+    s[[5, 12]] = [9.0, -9.0]  # saturated ends of the sigmoid
+    prunable = np.ones(len(gls), dtype=bool)
+    prunable[:3] = False
+    gls = np.where(prunable, _logsigmoid(s), 0.0).astype(np.float32)
+    got = oracle_mod.gated_attention_backward(q, k, v, cu, pos, rank, gls, g, c, dout, scores=s, prunable=prunable)
+    assert (got["dscore"][~prunable] == 0).all()
+    eps = 2.0 ** -6
+    for j in (3, 5, 8, 12, 16, 24):
+        sp, sm = s.astype(np.float64), s.astype(np.float64)
+        sp = sp.copy()
+        sm = sm.copy()
+        sp[j] += eps
+        sm[j] -= eps
+        lp = np.where(prunable, _logsigmoid(sp), 0.0).astype(np.float32)
+        lm = np.where(prunable, _logsigmoid(sm), 0.0).astype(np.float32)
+        fd = (_loss(oracle_mod, q, k, v, cu, pos, rank, lp, g, c, dout) -
+              _loss(oracle_mod, q, k, v, cu, pos, rank, lm, g, c, dout)) / (2 * eps)
+        assert got["dscore"][j] == pytest.approx(fd, rel=2e-3, abs=1e-7), j
