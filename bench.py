@@ -109,8 +109,8 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv") \
-            if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else f"/tmp/tg_clocks_{os.getpid()}.csv"
+        import tempfile
+        self.path = os.path.join(tempfile.gettempdir(), f"tg_clocks_{os.getpid()}_gpu{gpu_index}.csv")
 
     def start(self):
         try:

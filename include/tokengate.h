@@ -53,6 +53,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+/* The library is built with hidden visibility; every declaration below is
+   its exported interface. */
+#if defined(__GNUC__)
+#pragma GCC visibility push(default)
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -275,7 +281,10 @@ tg_status tg_gated_attention_noalloc(const uint16_t* q, const uint16_t* k, const
                                      float sm_scale, uint16_t* out, float* lse, tg_stream_t stream);
 
 /*
- * The whole gated prefill at one gate layer: tg_score, tg_select_topk (which
+ * The whole gated prefill at one gate layer (AI summary, "Methodology in
+ * Plain English": the layers below the gate run on every token, the gate
+ * scores and keeps the top-K at layer L, and the layers above run on the kept
+ * tokens only; README copy, "How it works"): tg_score, tg_select_topk (which
  * also writes the compaction map), the row gather of tg_compact and n_layers
  * gated-attention layers above the gate, with no host synchronisation, all
  * on `stream`.  The kernels are chained by programmatic dependent launch:
@@ -375,7 +384,9 @@ tg_status tg_masked_gated_attention(const uint16_t* q, const uint16_t* k, const 
  * layers' KV cache to the kept tokens on a separate stream (AI summary,
  * "Methodology in Plain English"): with src the [T, Hkv, d] K or V cache of
  * a layer below L (row_bytes = 2 * Hkv * d for bf16) this is that gather.
- * Entries of kept_idx outside [0, T) leave their row unwritten.
+ * Entries of kept_idx outside [0, T) leave their row unwritten.  src
+ * ([T, row_bytes]) and dst ([M, row_bytes]) must not overlap: an in-place or
+ * overlapping call is refused with TG_ERR_INVALID_ARG.
  * tg_gated_prefill_layer runs the same gather for args->gather_* beside the
  * attention.  With 4-byte rows it composes the maps of two gates: the
  * original positions of the tokens the second gate keeps are
@@ -409,6 +420,10 @@ tg_status tg_selftest_bounded_wait(int64_t timeout_ns, tg_stream_t stream);
 
 #ifdef __cplusplus
 }
+#endif
+
+#if defined(__GNUC__)
+#pragma GCC visibility pop
 #endif
 
 #endif /* TOKENGATE_H */

@@ -5,7 +5,13 @@
 Each csrc/*.cu compiles to an object under _build/ (in parallel), then one
 shared library is linked next to this file.  The CUDA runtime is linked
 statically, so the library does not depend on which libcudart the host
-process (for example PyTorch) has loaded.
+process (for example PyTorch) has loaded.  Only the C ABI (tg_*) is exported
+(csrc/tokengate.map); all other symbols are hidden.
+
+    TG_DEBUG=1 python -m learned_token_pruning_rmsnorm_b200.build --force
+builds the checking variant: every kernel checks the indices it derives from
+its inputs and records a violation in the device status word (read with
+tg_device_status) instead of accessing memory out of bounds.
 """
 
 from __future__ import annotations
@@ -25,8 +31,13 @@ BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libtokengate.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
-              "-Xptxas", "-warn-spills"]
+NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
+              "--expt-relaxed-constexpr", "-Xptxas", "-warn-spills"]
+EXPORTS = os.path.join(CSRC, "tokengate.map")
+
+
+def _debug() -> bool:
+    return os.environ.get("TG_DEBUG", "0") not in ("", "0")
 
 
 def _nvcc() -> str:
@@ -41,7 +52,7 @@ def _sources():
 
 
 def _headers():
-    return sorted(glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h")))
+    return sorted(glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h")) + [EXPORTS])
 
 
 def _stale(target: str, deps) -> bool:
@@ -53,16 +64,19 @@ def _stale(target: str, deps) -> bool:
 
 def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
     nvcc = _nvcc()
-    os.makedirs(BUILD, exist_ok=True)
+    # objects of the checking variant live apart, so that switching variants rebuilds
+    build_dir = BUILD + ("_debug" if _debug() else "")
+    os.makedirs(build_dir, exist_ok=True)
+    flags = NVCC_FLAGS + (["-DTG_DEBUG=1"] if _debug() else [])
     srcs = _sources()
     hdrs = _headers()
     objs = []
     jobs = []
     for s in srcs:
-        o = os.path.join(BUILD, os.path.basename(s)[:-3] + ".o")
+        o = os.path.join(build_dir, os.path.basename(s)[:-3] + ".o")
         objs.append(o)
         if force or _stale(o, [s] + hdrs):
-            cmd = [nvcc, *ARCH, *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-c", s, "-o", o]
+            cmd = [nvcc, *ARCH, *flags, "-I", INCLUDE, "-I", CSRC, "-c", s, "-o", o]
             if ptxas_info:
                 cmd += ["-Xptxas", "-v"]
             jobs.append(cmd)
@@ -80,9 +94,10 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
     if jobs:
         with ThreadPoolExecutor(max_workers=min(8, len(jobs))) as ex:
             list(ex.map(run, jobs))
-    if force or jobs or _stale(LIB, objs):
+    if force or jobs or _stale(LIB, objs + [EXPORTS]):
         tmp = LIB + f".tmp{os.getpid()}"
-        run([nvcc, *ARCH, "-shared", "-Xcompiler", "-fPIC", "-o", tmp, *objs])
+        run([nvcc, *ARCH, "-shared", "-Xcompiler", "-fPIC", "-Xlinker", f"--version-script={EXPORTS}", "-o", tmp,
+             *objs])
         os.replace(tmp, LIB)
     return LIB
 

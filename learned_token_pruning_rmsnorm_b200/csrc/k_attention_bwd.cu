@@ -313,7 +313,12 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
             return qrow < Mb ? __ldcg(fac + static_cast<size_t>(seq0 + qrow) * Hq + h)
                              : make_float4(0.f, 0.f, 0.f, 0.f);
         };
-        pdl_wait();  // the dQ kernel's factor records are complete from here on
+        // The dQ kernel's factor records are complete from here on.  This wait must stay
+        // unconditional for every CTA with work: bwd_finish_kernel waits only for this grid
+        // (its direct predecessor) and reads tileT, which the dQ kernel writes, so it is
+        // ordered after the dQ kernel only through these waits (a non-empty batch always
+        // has key tile 0 of some sequence with work).
+        pdl_wait();
         float4 fnext = load_fac(0);
         for (int u = 0; u < n_u; ++u) {
             const int t = u >> 1, hb = u & 1, i = kt + t;
@@ -966,6 +971,9 @@ bwd_finish_kernel(const float* __restrict__ colsum, const float* __restrict__ ti
                   const float* __restrict__ g, const int32_t* __restrict__ cu_kept, int B, int64_t M, int Hq,
                   float* __restrict__ dgls, float* __restrict__ dscore, float* __restrict__ dg,
                   float* __restrict__ dc) {
+    // Waits for the dK/dV grid (colsum).  tileT comes from the dQ kernel, one launch
+    // earlier: it is complete because every dK/dV CTA with work waits for the dQ kernel
+    // before it finishes, and a non-empty batch has at least one such CTA.
     pdl_wait();
     pdl_trigger();
     if (static_cast<int>(blockIdx.x) < Hq) {

@@ -286,6 +286,14 @@ tg_status tg_gather_rows(const void* src, int64_t T, int64_t row_bytes, const in
     const uintptr_t amask = static_cast<uintptr_t>(row_bytes < 16 ? row_bytes : 16) - 1;
     TG_REQUIRE(((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & amask) == 0,
                "src and dst must be aligned to %d bytes", static_cast<int>(amask + 1));
+    // the kernels read src and write dst through restrict pointers, all of a row's loads
+    // before its stores: an in-place or overlapping gather would return wrong rows
+    {
+        const uintptr_t s0 = reinterpret_cast<uintptr_t>(src), d0 = reinterpret_cast<uintptr_t>(dst);
+        const uintptr_t s1 = s0 + static_cast<uintptr_t>(T) * static_cast<uintptr_t>(row_bytes);
+        const uintptr_t d1 = d0 + static_cast<uintptr_t>(M) * static_cast<uintptr_t>(row_bytes);
+        TG_REQUIRE(s0 == d0 ? false : (s1 <= d0 || d1 <= s0), "src [T rows] and dst [M rows] must not overlap");
+    }
     if (tg_status s = check_device()) return s;
     return cuda_status(tg::launch_gather_bytes(src, kept_idx, M, T, row_bytes, dst, stream), "tg_gather_rows launch");
 }

@@ -189,3 +189,33 @@ def test_gather_rows_refuses_bad_rows_before_launch(lib):
     st = lib.tg_gather_rows(C.c_void_p(8), 10, 32, P, 4, P, None)  # misaligned source
     assert st == _lib.TG_ERR_INVALID_ARG
     assert lib.tg_gather_rows(None, 0, 32, None, 0, None, None) == _lib.TG_OK  # nothing to gather
+
+
+def test_gather_rows_refuses_overlapping_buffers(lib):
+    """The gather reads src and writes dst through restrict pointers (all of a row's loads
+    before its stores), so in-place and overlapping calls are refused before any launch."""
+    from learned_token_pruning_rmsnorm_b200 import _lib
+    P = C.c_void_p(1 << 20)  # never dereferenced: validation fails first
+    st = lib.tg_gather_rows(P, 100, 64, C.c_void_p(16), 10, P, None)  # src == dst
+    assert st == _lib.TG_ERR_INVALID_ARG
+    assert b"overlap" in lib.tg_last_error_string()
+    # dst starts inside src's 100 rows of 64 bytes; src starts inside dst's 10 rows
+    assert lib.tg_gather_rows(P, 100, 64, C.c_void_p(16), 10, C.c_void_p((1 << 20) + 99 * 64), None) == \
+        _lib.TG_ERR_INVALID_ARG
+    assert lib.tg_gather_rows(C.c_void_p((1 << 20) + 9 * 64), 100, 64, C.c_void_p(16), 10, P, None) == \
+        _lib.TG_ERR_INVALID_ARG
+
+
+def test_library_exports_only_the_c_abi(lib):
+    """Only the tg_* entry points of tokengate.h are dynamic symbols: the launchers, the
+    statically linked CUDA runtime and every C++ instance stay local, so two copies of the
+    library in one process cannot bind to each other's internals."""
+    import shutil
+    import subprocess
+    from learned_token_pruning_rmsnorm_b200 import _lib
+    nm = shutil.which("nm")
+    if nm is None:
+        pytest.skip("no nm")
+    r = subprocess.run([nm, "-D", "--defined-only", _lib.LIB_PATH], capture_output=True, text=True, check=True)
+    names = sorted(line.split()[-1] for line in r.stdout.splitlines() if line.strip())
+    assert names == _declared_functions()

@@ -80,17 +80,23 @@ def test_noalloc_matches_workspace_entry_point(lib, name):
 
 
 def test_noalloc_scratch_bounds_the_split_on_this_device(lib):
-    """The causal split only triggers while (n_qt + 1) < 2 * SMs / (1.3 * B * Hq/2),
-    which keeps its scratch near 30 MB for head_dim 128 on 148 SMs: every size
-    then fits the fixed array.  (Larger needs, possible on devices with more
-    SMs, are refused by the entry point with TG_ERR_UNSUPPORTED.)"""
+    """The causal split is only considered while tiles * (n_qt + 1) < 4 * SMs, where
+    tiles = B * Hq / 2 is the number of (sequence, head pair) instances and n_qt the
+    number of 128-row query tiles (beyond that every SM's share is at least twice the
+    longest unit and no tile is split).  Every such shape is checked here against the
+    fixed array, for the SM count of this device; on 148 SMs the largest need is about
+    18 MB (head_dim 128, one head pair, n_qt = 144).  Larger needs, possible on devices
+    with more SMs, are refused by the entry point with TG_ERR_UNSUPPORTED."""
+    import math
     limit = 32 * 1024 * 1024
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
     worst = 0
     for d in (64, 128):
-        for Hq, Hkv in ((16, 8), (2, 1), (4, 2)):
+        for Hq, Hkv in ((2, 1), (4, 2), (16, 8), (8, 2)):
             for B in (1, 2, 4):
-                for max_M in range(128, 16384 + 1, 128):
-                    need = lib.tg_gated_attention_workspace_size(B, max_M, Hq, Hkv, d)
+                tiles = B * (Hq // 2)
+                for n_qt in range(1, math.ceil(4 * sms / tiles) + 2):
+                    need = lib.tg_gated_attention_workspace_size(B, 128 * n_qt, Hq, Hkv, d)
                     worst = max(worst, need)
-                    assert need <= limit, (d, Hq, Hkv, B, max_M, need)
+                    assert need <= limit, (d, Hq, Hkv, B, n_qt, need)
     assert worst > 0
