@@ -17,8 +17,9 @@ Under torchrun (N>1) every rank runs an independent replica of the workload
 (the path is single-GPU; no collective on the data path), the value is the
 tokens of all ranks divided by the slowest rank's time, and scaling is weak.
 
---impl reference times the fp64 CPU oracle on a bounded sample of the same
-workload, extrapolated to the whole workload; it is a slow program by design.
+--impl reference times the fp64 CPU oracle on whole steps of the same workload
+(every prunable row scored, every kept row attended); it is a slow program by
+design (about 1.5 s per step at the default workload on 16 host threads).
 """
 
 from __future__ import annotations
@@ -177,41 +178,45 @@ KERNEL_FILES = {"score": "k_gate.cu", "select": "k_select.cu", "gather": "k_sele
 
 # ------------------------------------------------------------------ oracle (CPU baseline / reference arm)
 
-def oracle_sample_pass(w, gi, Wg_bits, layer, score_rows=1024, attn_rows=48):
-    """One bounded pass of the fp64 oracle over a sample of the workload,
-    extrapolated to the whole workload.  Returns (est_seconds, sample_desc)."""
+def oracle_step(w, gi, Wg_bits, layers):
+    """One whole step of the fp64 oracle over the workload: the gate score of every
+    prunable row, top-K selection, compaction, and the gated-attention layers (one per
+    entry of `layers`) over every kept row.  Returns (seconds, description, per-part
+    seconds)."""
     import oracle
     cu, span, k = w.cu_seqlens(), w.span_array(), w.budget_array()
     n_prun = int(sum(p1 - p0 for p0, p1 in w.spans))
-    # gate scores on the first `score_rows` prunable rows of sequence 0
-    sub_span = span.copy()
-    sub_span[:, 1] = np.minimum(span[:, 1], span[:, 0] + score_rows)
-    sub_span[1:, 1] = sub_span[1:, 0]
     t0 = time.perf_counter()
-    s = oracle.score(gi["hidden"], cu, sub_span, Wg_bits, gi["b1"], gi["w2"], gi["b2"], w.eps)
-    t_score = (time.perf_counter() - t0) * n_prun / max(1, int(np.sum(sub_span[:, 1] - sub_span[:, 0])))
-    # selection + compaction on full-length scores (the oracle's real cost)
+    s = oracle.score(gi["hidden"], cu, span, Wg_bits, gi["b1"], gi["w2"], gi["b2"], w.eps)
+    t1 = time.perf_counter()
     s32 = np.nan_to_num(s, nan=0.0).astype(np.float32)
-    t0 = time.perf_counter()
     keep = oracle.select_topk(s32, cu, span, k)
     comp = oracle.compact(gi["hidden"], s32, keep, cu, span)
-    t_sel = time.perf_counter() - t0
-    # attention on evenly spaced query rows; cost of a row is proportional to its causal length
+    t2 = time.perf_counter()
     cu_kept = comp["cu_kept"]
     M = int(cu_kept[-1])
-    rows = np.linspace(0, M - 1, attn_rows).astype(np.int64)
-    t0 = time.perf_counter()
-    oracle.gated_attention(layer["q"], layer["k"], layer["v"], cu_kept, comp["pos"], comp["rank"],
-                           comp["gls"].astype(np.float32), layer["g"], layer["c"], rows=rows, want_lse=False)
-    t_attn_sample = time.perf_counter() - t0
-    b_of = np.searchsorted(cu_kept, rows, side="right") - 1
-    sampled_pairs = float(np.sum(rows - cu_kept[b_of] + 1))
+    for layer in layers:
+        oracle.gated_attention(layer["q"], layer["k"], layer["v"], cu_kept, comp["pos"], comp["rank"],
+                               comp["gls"].astype(np.float32), layer["g"], layer["c"], want_lse=False)
+    t3 = time.perf_counter()
     _, pairs = attention_flops(cu_kept, w.Hq, w.d)
-    t_attn = t_attn_sample * pairs / sampled_pairs
-    desc = (f"oracle fp64: gate on {int(np.sum(sub_span[:, 1] - sub_span[:, 0]))} of {n_prun} prunable rows, "
-            f"full select+compact, attention on {attn_rows} of {M} query rows ({int(sampled_pairs)} of {pairs} "
-            f"causal pairs); times scaled to the whole workload")
-    return t_score + t_sel + t_attn, desc, {"score_s": t_score, "select_compact_s": t_sel, "attention_s": t_attn}
+    desc = (f"oracle fp64, whole step: gate score of all {n_prun} prunable rows, select + compact, "
+            f"{len(layers)} attention layer(s) over all {M} kept rows x {w.Hq} heads ({pairs} causal pairs "
+            f"each); nothing extrapolated")
+    return t3 - t0, desc, {"score_s": t1 - t0, "select_compact_s": t2 - t1, "attention_s": t3 - t2}
+
+
+def oracle_baseline(w, gi, Wg_bits, layers, min_seconds=10.0, max_steps=8):
+    """The oracle timed on whole steps (at least two, until about `min_seconds` of CPU
+    work): the cpu_baseline leg of the GPU arm."""
+    import oracle
+    times, desc, parts = [], "", None
+    while len(times) < 2 or (sum(times) < min_seconds and len(times) < max_steps):
+        t, desc, parts = oracle_step(w, gi, Wg_bits, layers)
+        times.append(t)
+    t = float(np.mean(times))
+    return {"value": w.T / t, "unit": UNIT, "cores": oracle.get_threads(), "kind": "oracle",
+            "sample": f"{len(times)} whole steps; {desc}", "seconds_per_step": t, "parts_s": parts}
 
 
 def run_reference(args, w):
@@ -222,11 +227,11 @@ def run_reference(args, w):
     gi = make_gate_inputs(w)
     Wg = oracle.gate_fold(gi["gamma"], gi["W1"])
     M = int(w.cu_kept()[-1])
-    layer = make_attention_inputs(w, M, layer=0)
+    layers = [make_attention_inputs(w, M, layer=l) for l in range(args.layers)]
     times = []
     desc = ""
     for it in range(args.warmup + args.steps):
-        t, desc, _ = oracle_sample_pass(w, gi, Wg, layer, score_rows=1024, attn_rows=64)
+        t, desc, _ = oracle_step(w, gi, Wg, layers)
         if it >= args.warmup:
             times.append(t)
     t = float(np.mean(times))
@@ -236,7 +241,7 @@ def run_reference(args, w):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
             "config": workload_config(w, args.layers),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.get_threads(), "kind": "oracle",
-                             "sample": desc},
+                             "sample": f"{args.steps} timed whole steps after {args.warmup} warm-up; {desc}"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -410,6 +415,155 @@ def measure_next_rows(tg, dev, st, flush, main, peaks, reps=10):
                                     "us": us, "tflops": 2.5 * fl / (us * 1e-6) / 1e12,
                                     "frac_of_bf16_peak": 2.5 * fl / (us * 1e-6) / 1e12 / tc_peak,
                                     "algorithmic": "2.5x the forward's 4*d*Hq per causal pair (five products)"}
+    return res
+
+
+def device_gate_inputs(tg, w, dev):
+    """Gate weights from the seeded workload generator; the hidden rows are drawn on the
+    device from a seeded generator with the same distribution (N(0, 1), the workload's
+    outlier channels x8), which keeps the largest workloads' set-up to milliseconds."""
+    import torch
+    from workloads import make_gate_weights
+    gw = make_gate_weights(w)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(7919 * (w.seed + 1) + w.T)
+    hidden = torch.randn((w.T, w.D), generator=gen, device=dev, dtype=torch.float32)
+    if len(gw["outlier_channels"]):
+        hidden[:, torch.from_numpy(gw["outlier_channels"]).to(dev)] *= w.outlier_scale
+    hidden = hidden.to(torch.bfloat16)
+
+    def bf16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    Wg = tg.tg_gate_prepare(bf16(gw["gamma"]), bf16(gw["W1"]))
+    return hidden, Wg, torch.from_numpy(gw["b1"]).to(dev), torch.from_numpy(gw["w2"]).to(dev), gw["b2"]
+
+
+def device_attention_inputs(w, M, n_layers, dev, seed=0):
+    """Per-layer q, k, v (N(0, 1) x the workload's std, bf16), g ~ N(0, 0.5), c ~ U(0, 0.5),
+    drawn on the device from a seeded generator."""
+    import torch
+    gen = torch.Generator(device=dev)
+    out = []
+    for l in range(n_layers):
+        gen.manual_seed(104729 * (seed + 1) + 31 * l + M)
+        rnd = lambda *shape: torch.randn(shape, generator=gen, device=dev, dtype=torch.float32)  # noqa: E731
+        out.append({"q": (rnd(M, w.Hq, w.d) * w.qkv_std).to(torch.bfloat16),
+                    "k": (rnd(M, w.Hkv, w.d) * w.qkv_std).to(torch.bfloat16),
+                    "v": (rnd(M, w.Hkv, w.d) * w.qkv_std).to(torch.bfloat16),
+                    "g": rnd(w.Hq) * w.g_std,
+                    "c": torch.rand((w.Hq,), generator=gen, device=dev) * w.c_high})
+    return out
+
+
+def measure_workload(tg, dev, st, flush, peaks, w, n_layers=1, reps=10, stages=True):
+    """One gated-prefill call (score, select + compaction map, n_layers attention layers,
+    row gather) on workload w, replayed as a CUDA graph after an L2 flush; median of reps.
+    With `stages`, the attention and the stages 1-3 are also timed alone for their
+    roofline fractions."""
+    import torch
+    from learned_token_pruning_rmsnorm_b200 import PrefillBuffers, PrefillCall
+    lib = tg.load()
+    hidden, Wg, b1, w2, b2 = device_gate_inputs(tg, w, dev)
+    cu, span, k = w.cu_seqlens(), w.span_array(), w.budget_array()
+    M, cu_kept = tg.tg_kept_count(cu, span, k)
+    layers = device_attention_inputs(w, M, n_layers, dev, seed=w.seed)
+    bufs = PrefillBuffers(w.T, w.D, M, n_layers, w.Hq, w.d, dev, with_hidden=True)
+    call = PrefillCall(hidden, cu, span, k, Wg, b1, w2, b2, w.eps, layers, bufs, w.Hq, w.Hkv, w.d)
+    step_us = time_device_us(call, st, flush, reps)
+    flops, pairs = attention_flops(cu_kept, w.Hq, w.d)
+    tc_peak, hbm_peak = float(peaks["bf16_tflops"]), float(peaks["hbm_gbs"])
+    res = {"N": list(w.seqlens) if w.B > 1 else w.seqlens[0], "K": list(w.budgets) if w.B > 1 else w.budgets[0],
+           "M": M, "attn_layers": n_layers, "step_us": step_us, "tokens_per_s": w.T / (step_us * 1e-6),
+           "attn_flops_per_layer": flops}
+    if not stages:
+        return res, call
+    sh = lambda: torch.cuda.current_stream(dev).cuda_stream  # noqa: E731
+    L0 = layers[0]
+    ws_p, ws_n = (None, 0) if call.ws is None else (call.ws.data_ptr(), call.ws.numel())
+    sm = 1.0 / math.sqrt(w.d)
+
+    def ok(rc):
+        assert rc == 0, lib.tg_last_error_string()
+
+    attn = lambda: ok(lib.tg_gated_attention(  # noqa: E731
+        L0["q"].data_ptr(), L0["k"].data_ptr(), L0["v"].data_ptr(), call.ck.data_ptr(), w.B, M, call.max_M, w.Hq,
+        w.Hkv, w.d, bufs.pos.data_ptr(), bufs.rank.data_ptr(), bufs.gls.data_ptr(), L0["g"].data_ptr(),
+        L0["c"].data_ptr(), sm, bufs.out[0].data_ptr(), None, ws_p, ws_n, sh()))
+    score = lambda: ok(lib.tg_score(  # noqa: E731
+        hidden.data_ptr(), call.cu.data_ptr(), call.sp.data_ptr(), w.B, w.T, w.D, Wg.data_ptr(), b1.data_ptr(),
+        w2.data_ptr(), float(b2), w.I, float(w.eps), bufs.scores.data_ptr(), sh()))
+    select = lambda: ok(lib.tg_select_topk(  # noqa: E731
+        bufs.scores.data_ptr(), call.cu.data_ptr(), call.sp.data_ptr(), call.kk.data_ptr(), w.B, w.T,
+        bufs.keep.data_ptr(), call.ck.data_ptr(), bufs.kept_idx.data_ptr(), bufs.pos.data_ptr(),
+        bufs.rank.data_ptr(), bufs.gls.data_ptr(), sh()))
+    gather = lambda: ok(lib.tg_compact(  # noqa: E731
+        hidden.data_ptr(), None, None, None, None, w.B, w.T, w.D, None, M, bufs.hidden_kept.data_ptr(), None, None,
+        None, bufs.kept_idx.data_ptr(), sh()))
+    a_us = time_device_us(attn, st, flush, reps)
+    s_us = [time_device_us(f, st, flush, reps) for f in (score, select, gather)]
+    sb = stage_bytes(w, M)
+    s13_bytes = sb["score"] + sb["select"] + sb["gather"]
+    s13_us = sum(s_us)
+    res.update({"attn_us": a_us, "attn_tflops": flops / (a_us * 1e-6) / 1e12,
+                "attn_frac_of_bf16_peak": flops / (a_us * 1e-6) / 1e12 / tc_peak,
+                "stage_us": {"score": s_us[0], "select": s_us[1], "gather": s_us[2]},
+                "score_frac_of_hbm": sb["score"] / (s_us[0] * 1e-6) / 1e9 / hbm_peak,
+                "score_select_compact_gbs": s13_bytes / (s13_us * 1e-6) / 1e9,
+                "score_select_compact_frac_of_hbm": s13_bytes / (s13_us * 1e-6) / 1e9 / hbm_peak})
+    return res, call
+
+
+def measure_workload_sweep(tg, dev, st, flush, peaks, main_step_us):
+    """Every seeded workload besides the headline one, each on its own prefill call: the
+    K sweep at 32k, 16k, 128k and the varlen batch; the 14-layer stack of the 32k, K=2000
+    workload; and dense causal attention over all 16384 tokens (config 3's comparison:
+    no pruning, bias 0 and temperature 1)."""
+    import torch
+    res = {}
+    for name in ("c1_16k", "c2_32k_k100", "c2_32k_k500", "c2_32k_kall", "c4_128k", "c4_varlen"):
+        w = get_config(name)
+        r, call = measure_workload(tg, dev, st, flush, peaks, w, reps=5 if name == "c2_32k_kall" else 10)
+        res[name] = r
+        del call
+        torch.cuda.empty_cache()
+    # the stack: one call with 14 attention layers (each its own q, k, v, g, c)
+    w = get_config("c2_32k_k2000")
+    r14, call = measure_workload(tg, dev, st, flush, peaks, w, n_layers=14, stages=False)
+    r1, call1 = measure_workload(tg, dev, st, flush, peaks, w, n_layers=1, stages=False)
+    per_layer = (r14["step_us"] - r1["step_us"]) / 13.0
+    r14.update({"one_layer_step_us": r1["step_us"], "marginal_attn_layer_us": per_layer,
+                "marginal_attn_tflops": r14["attn_flops_per_layer"] / (per_layer * 1e-6) / 1e12,
+                "marginal_attn_frac_of_bf16_peak": r14["attn_flops_per_layer"] / (per_layer * 1e-6) / 1e12
+                / float(peaks["bf16_tflops"])})
+    res["c2_32k_k2000_stack14"] = r14
+    del call, call1
+    torch.cuda.empty_cache()
+    # dense causal attention over the whole 16k sequence (no compaction; gls = 0, c = 0)
+    w = get_config("c3_full_budget_16k")
+    lib = tg.load()
+    N = w.T
+    L = device_attention_inputs(w, N, 1, dev, seed=3)[0]
+    zeros = torch.zeros(N, dtype=torch.float32, device=dev)
+    c0 = torch.zeros(w.Hq, dtype=torch.float32, device=dev)
+    ar = torch.arange(1, N + 1, dtype=torch.int32, device=dev)
+    ck = torch.tensor([0, N], dtype=torch.int32, device=dev)
+    out = torch.empty((N, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
+    ws = tg.attention_workspace(1, N, w.Hq, w.Hkv, w.d, dev)
+    ws_p, ws_n = (None, 0) if ws is None else (ws.data_ptr(), ws.numel())
+    flops, _ = attention_flops(np.array([0, N]), w.Hq, w.d)
+
+    def dense():
+        assert lib.tg_gated_attention(L["q"].data_ptr(), L["k"].data_ptr(), L["v"].data_ptr(), ck.data_ptr(), 1, N, N,
+                                      w.Hq, w.Hkv, w.d, ar.data_ptr(), ar.data_ptr(), zeros.data_ptr(),
+                                      L["g"].data_ptr(), c0.data_ptr(), 1.0 / math.sqrt(w.d), out.data_ptr(), None,
+                                      ws_p, ws_n, torch.cuda.current_stream(dev).cuda_stream) == 0
+    us = time_device_us(dense, st, flush, 5)
+    res["c3_dense_causal_16k"] = {"N": N, "us": us, "flops": flops, "tflops": flops / (us * 1e-6) / 1e12,
+                                  "frac_of_bf16_peak": flops / (us * 1e-6) / 1e12 / float(peaks["bf16_tflops"]),
+                                  "note": "unpruned causal attention, N=16384, 16/8 heads, d=128 (gls = 0, c = 0)"}
+    del L, out, ws
+    torch.cuda.empty_cache()
     return res
 
 
@@ -601,13 +755,15 @@ def run_gpu(args, w):
                     "layer": L0, "bufs": bufs, "gls_host": bufs.gls.cpu().numpy(), "ws": call.ws}
         next_rows = measure_next_rows(tg, dev, st, flush, main_ctx, peaks)
 
+    sweep = None
+    if rank == 0 and not args.no_sweep:
+        sweep = measure_workload_sweep(tg, dev, st, flush, peaks, ms_per_step * 1e3)
+
     cpu_base = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         import oracle
         Wg_bits = oracle.gate_fold(gi["gamma"], gi["W1"])
-        t_est, desc, parts = oracle_sample_pass(w, gi, Wg_bits, layers_np[0], score_rows=8192, attn_rows=512)
-        cpu_base = {"value": w.T / t_est, "unit": UNIT, "cores": oracle.get_threads(), "kind": "oracle",
-                    "sample": desc, "est_seconds_per_step": t_est, "parts_s": parts}
+        cpu_base = oracle_baseline(w, gi, Wg_bits, layers_np)
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
@@ -623,7 +779,7 @@ def run_gpu(args, w):
                 "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                         "d2h_bytes_per_step": int(d2h)},
                 "gpu_launches": args.steps * (3 + args.layers), "cuda_graph": graph is not None,
-                "next_rows": next_rows,
+                "next_rows": next_rows, "workloads": sweep,
                 "cpu_baseline": cpu_base, "clocks": clk, "peaks": {"source": peaks["source"],
                                                                    "hbm_gbs": hbm_peak, "bf16_tflops": tc_peak}}
         print(json.dumps(line), flush=True)
@@ -645,6 +801,8 @@ def main(argv=None):
     ap.add_argument("--no-next-rows", action="store_true",
                     help="skip the measurements of masked attention, KV gather, head_dim 256 and stacked gates")
     ap.add_argument("--no-graph", action="store_true", help="launch the step directly instead of a CUDA graph")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the other workloads (K sweep, 16k, 128k, varlen, 14-layer stack, dense 16k)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

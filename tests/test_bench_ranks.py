@@ -71,7 +71,10 @@ def test_reference_arm_prints_the_contract_line(monkeypatch, capsys):
     import json
     monkeypatch.delenv("RANK", raising=False)
     monkeypatch.delenv("WORLD_SIZE", raising=False)
-    assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "3", "--workload", "c0_tiny"]) == 0
+    import time
+    t0 = time.perf_counter()
+    assert bench.main(["--impl", "reference", "--steps", "2", "--warmup", "3", "--workload", "c0_tiny"]) == 0
+    wall = time.perf_counter() - t0
     lines = [ln for ln in capsys.readouterr().out.splitlines() if ln.strip()]
     assert len(lines) == 1
     d = json.loads(lines[0])
@@ -82,3 +85,6 @@ def test_reference_arm_prints_the_contract_line(monkeypatch, capsys):
     assert d["config"]["workload"] == "c0_tiny"
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    # whole steps are timed, nothing is extrapolated: the claimed timed region fits in the run
+    assert d["ms_per_step"] * d["steps"] / 1e3 <= wall
+    assert "nothing extrapolated" in d["cpu_baseline"]["sample"]

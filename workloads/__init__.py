@@ -12,5 +12,6 @@ from .gen import (  # noqa: F401
     f32_to_bf16_bits,
     make_attention_inputs,
     make_gate_inputs,
+    make_gate_weights,
     make_scores,
 )

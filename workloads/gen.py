@@ -68,29 +68,39 @@ def _normal_bf16(rng: np.random.Generator, shape, std: float, chunk_rows: int = 
     return out
 
 
-def make_gate_inputs(w, seed: int | None = None) -> dict:
-    """Hidden states at the gate layer plus the gate's parameters."""
+def make_gate_weights(w, seed: int | None = None) -> dict:
+    """The gate's parameters and the hidden states' outlier channels (the small part of
+    make_gate_inputs, drawn from the same streams)."""
     seed = w.seed if seed is None else seed
-    T, D, I = w.T, w.D, w.I
-    hidden = np.empty((T, D), dtype=np.uint16)
-    rng = _rng(seed, "hidden")
+    D, I = w.D, w.I
     orng = _rng(seed, "outliers")
     outl = np.sort(orng.choice(D, size=w.n_outlier_channels, replace=False)) \
         if w.n_outlier_channels > 0 else np.zeros(0, dtype=np.int64)
-    scale = np.ones(D, dtype=np.float32)
-    scale[outl] = np.float32(w.outlier_scale)
-    for r0 in range(0, T, 8192):
-        r1 = min(T, r0 + 8192)
-        x = rng.standard_normal((r1 - r0, D), dtype=np.float32)
-        x *= scale[None, :]
-        hidden[r0:r1] = f32_to_bf16_bits(x)
     gamma = f32_to_bf16_bits(1.0 + 0.1 * _rng(seed, "gamma").standard_normal(D).astype(np.float32))
     W1 = _normal_bf16(_rng(seed, "W1"), (D, I), 1.0 / np.sqrt(D))
     b1 = (0.1 * _rng(seed, "b1").standard_normal(I)).astype(np.float32)
     w2 = (_rng(seed, "w2").standard_normal(I) / np.sqrt(I)).astype(np.float32)
     b2 = np.float32(0.1 * _rng(seed, "b2").standard_normal())
-    return {"hidden": hidden, "gamma": gamma, "W1": W1, "b1": b1, "w2": w2,
-            "b2": float(b2), "outlier_channels": outl.astype(np.int64)}
+    return {"gamma": gamma, "W1": W1, "b1": b1, "w2": w2, "b2": float(b2),
+            "outlier_channels": outl.astype(np.int64)}
+
+
+def make_gate_inputs(w, seed: int | None = None) -> dict:
+    """Hidden states at the gate layer plus the gate's parameters."""
+    seed = w.seed if seed is None else seed
+    T, D = w.T, w.D
+    out = make_gate_weights(w, seed)
+    hidden = np.empty((T, D), dtype=np.uint16)
+    rng = _rng(seed, "hidden")
+    scale = np.ones(D, dtype=np.float32)
+    scale[out["outlier_channels"]] = np.float32(w.outlier_scale)
+    for r0 in range(0, T, 8192):
+        r1 = min(T, r0 + 8192)
+        x = rng.standard_normal((r1 - r0, D), dtype=np.float32)
+        x *= scale[None, :]
+        hidden[r0:r1] = f32_to_bf16_bits(x)
+    out["hidden"] = hidden
+    return out
 
 
 def make_attention_inputs(w, M: int, layer: int = 0, seed: int | None = None,
