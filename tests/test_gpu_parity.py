@@ -74,6 +74,32 @@ def test_score_parity(tg, name):
     assert (s[~m] == 0).all(), "non-prunable entries must be left untouched"
 
 
+@pytest.mark.parametrize("name", ["c4_128k", "c4_varlen"])
+def test_score_parity_long_context_sampled_rows(tg, name):
+    """128k tokens (130,816 prunable rows, about 3.5 tiles of 256 rows per CTA of the
+    persistent kernel) and the varlen batch (four spans, tiles crossing no sequence).
+    The score of a row depends on that row alone, so the oracle scores a sample: every
+    64th prunable row plus the first and last 256 rows of each span."""
+    w = CONFIGS[name]
+    gi = make_gate_inputs(w)
+    Wg_ref = oracle.gate_fold(gi["gamma"], gi["W1"])
+    s = tg.tg_score(H.bf16_dev(gi["hidden"]), w.cu_seqlens(), w.span_array(), H.bf16_dev(Wg_ref),
+                    H.f32_dev(gi["b1"]), H.f32_dev(gi["w2"]), gi["b2"], w.eps).cpu().numpy()
+    cu = w.cu_seqlens()
+    rows = []
+    for b, (p0, p1) in enumerate(w.spans):
+        r = np.arange(cu[b] + p0, cu[b] + p1)
+        rows.append(np.concatenate([r[:256], r[::64], r[-256:]]))
+    rows = np.unique(np.concatenate(rows))
+    n = len(rows)
+    s_ref = oracle.score(gi["hidden"][rows], np.array([0, n], np.int32), np.array([[0, n]], np.int32), Wg_ref,
+                         gi["b1"], gi["w2"], gi["b2"], w.eps)
+    err = H.score_error(s[rows], s_ref)
+    assert err <= H.SCORE_REL, f"{name}: score error {err:.3e} over {n} sampled rows"
+    m = H.prunable_mask(w)
+    assert (s[~m] == 0).all(), "non-prunable entries must be left untouched"
+
+
 @pytest.mark.parametrize("I", [64, 48])
 def test_score_ragged_spans(tg, I):
     """Spans that start at 0, end at N, are empty, or hold one token; D=256; I = 48
