@@ -34,18 +34,15 @@
 #include <tuple>
 #include <vector>
 
-#include "tg_sm100.cuh"
+#include "tg_attn_util.cuh"
 
 namespace tg {
 namespace {
 
 using namespace sm100;
+using namespace attn;
 
-constexpr int BM = 128;           // query rows per tile (TMEM lanes)
-constexpr int BN = 128;           // keys per tile
 constexpr int NUM_THREADS = 192;
-constexpr float LOG2E = 1.4426950408889634f;
-constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: rescale only when the max grows by > 2^8
 
 template <int HD>
 struct AttnSmem {
@@ -98,76 +95,6 @@ __device__ unsigned long long g_attn_cta[4096 * 12];  // per CTA: phase stamps (
     do {                      \
     } while (0)
 #endif
-
-__device__ __forceinline__ float softplus_f(float x) { return fmaxf(x, 0.f) + log1pf(expf(-fabsf(x))); }
-
-__device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity, int* status) {
-    volatile int never = 0;
-    return mbar_wait(bar, parity, &never, status, TG_WHERE_DRAIN);
-}
-
-// Global load that stays where it is written (volatile asm is not moved across the
-// other volatile asm statements), so that a prefetch issued a tile ahead is not sunk by the
-// compiler to its first use.  It reads through L2 (.cg), not the read-only path: with
-// programmatic dependent launch the kernel that writes the compaction map may still be
-// running during this kernel's lifetime, and the non-coherent path then returned stale
-// values now and then.
-__device__ __forceinline__ float ldg_early(const float* p) {
-    float v;
-    asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(v) : "l"(p));
-    return v;
-}
-
-// max of three floats (one instruction on sm_100)
-__device__ __forceinline__ float max3f(float a, float b, float c) {
-    float d;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-    return d;
-}
-
-// Packed fp32 pairs (lo in bits 0-31): two FMAs or adds per instruction on sm_100.
-__device__ __forceinline__ uint64_t f32x2_pack(float lo, float hi) {
-    return static_cast<uint64_t>(__float_as_uint(lo)) | (static_cast<uint64_t>(__float_as_uint(hi)) << 32);
-}
-__device__ __forceinline__ float f32x2_lo(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v)); }
-__device__ __forceinline__ float f32x2_hi(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
-__device__ __forceinline__ uint64_t f32x2_fma(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-__device__ __forceinline__ uint64_t f32x2_add(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-
-// Named barrier `id` over `n` threads that also returns the OR of `pred` over them.
-__device__ __forceinline__ bool bar_red_or(int id, int n, bool pred) {
-    uint32_t res;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, %2, %3, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(res)
-        : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(n)
-        : "memory");
-    return res != 0;
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&v);
-}
-
-// (high, low) bf16 split of v packed as a pair: high = bf16(v), low = bf16(v - high).
-// Infinities are clamped to the largest finite magnitude so that products with a zero
-// low part of the other operand stay finite (the sum still overflows to infinity).
-__device__ __forceinline__ uint32_t bf16_hi_lo(float v) {
-    const float c = fminf(fmaxf(v, -3.0e38f), 3.0e38f);  // NaN stays NaN
-    const __nv_bfloat16 hi = __float2bfloat16_rn(isnan(v) ? v : c);
-    const float lo = (isnan(v) ? v : c) - __bfloat162float(hi);
-    return pack_bf16x2(__bfloat162float(hi), lo);
-}
 
 template <int HD>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -499,27 +426,6 @@ struct G2Smem {
 enum : int {
     G_Q_FULL = 0, G_K_FULL = 1, G_K_EMPTY = 3, G_V_FULL = 5, G_V_EMPTY = 7, G_S_FULL = 9, G_P_FULL = 11,
     G_O_FULL = 13, G_DRAIN = 14
-};
-
-// Causal work split.  Query tile qt of a sequence needs KV tiles 0..qt.  With
-// a chunk length C, it is cut into ceil((qt+1)/C) units of at most C KV
-// tiles; units are numbered heaviest query tile first, so the block
-// scheduler hands out long units first.  units_below(x) counts the units of
-// query tiles 0..x-1:  sum_{L=1..x} ceil(L/C) = C*a*(a+1)/2 + r*(a+1), x = a*C + r.
-__device__ __forceinline__ int64_t units_below(int x, int C) {
-    const int64_t a = x / C, r = x % C;
-    return C * a * (a + 1) / 2 + r * (a + 1);
-}
-
-// Scratch of the KV split, per split query tile (qt >= C) of each (sequence,
-// head pair): nch partial results (O / l in fp32 and m + log2 l per row and
-// head) and one arrival counter that the merging CTA resets to zero.
-struct SplitWs {
-    float* o;       // [slots][max_nch][2][HD/2][BM] bf16 column pairs (sized for fp32; half is used)
-    float* lse2;    // [slots][max_nch][2][BM]
-    int* cnt;       // [slots]
-    int max_nch;
-    int slots_per_pair;  // n_qt_max - C (query tiles that may be split)
 };
 
 // Q_ext columns 4..15 (gates 2..n) of both heads' rows, out of line so that the
@@ -1189,20 +1095,18 @@ cudaError_t launch_gqa2(const CUtensorMap& tq, const CUtensorMap& tk, const CUte
     if (cudaError_t e = ensure_smem_limit(gated_attn_gqa2_kernel<HD>, L::ALLOC, attr_set); e != cudaSuccess)
         return e;
     const int n_qt_max = (max_M + BM - 1) / BM;
-    const int C = attention_kv_chunk(B, max_M, Hq, Hkv, ws != nullptr);
+    int C = n_qt_max > 0 ? n_qt_max : 1;
     SplitWs sw{};
-    if (C < n_qt_max) {
-        const size_t need = attention_workspace_bytes(B, max_M, Hq, Hkv, HD);
-        if (ws_bytes < need) return cudaErrorInvalidValue;
-        sw.max_nch = (n_qt_max + C - 1) / C;
-        sw.slots_per_pair = n_qt_max - C;
-        const int64_t slots = static_cast<int64_t>(B) * (Hq / 2) * sw.slots_per_pair;
+    if (ws != nullptr) {
+        const AttnWsLayout lay = attention_ws_layout(B, max_M, Hq, Hkv, HD);
+        if (ws_bytes < lay.total) return cudaErrorInvalidValue;
+        C = lay.C;
         uint8_t* p = static_cast<uint8_t*>(ws);
-        sw.o = reinterpret_cast<float*>(p);
-        p += slots * sw.max_nch * 2 * BM * HD * sizeof(float);
-        sw.lse2 = reinterpret_cast<float*>(p);
-        p += slots * sw.max_nch * 2 * BM * sizeof(float);
-        sw.cnt = reinterpret_cast<int*>(p);
+        sw.cnt = reinterpret_cast<int*>(p + lay.cnt_off);
+        sw.o = reinterpret_cast<float*>(p + lay.o_off);
+        sw.lse2 = reinterpret_cast<float*>(p + lay.lse_off);
+        sw.max_nch = lay.max_nch;
+        sw.slots_per_pair = lay.slots_per_pair;
     }
     const int64_t units = units_below_host(n_qt_max, C);
     dim3 grid(Hq / 2, static_cast<unsigned>(units), B);
@@ -1229,10 +1133,20 @@ cudaError_t launch_tc(const uint16_t* q, const uint16_t* k, const uint16_t* v, c
                              static_cast<uint64_t>(Hkv) * HD * 2, 64, BN))
         return cudaErrorInvalidValue;
     if constexpr (HD <= 128) {  // two heads of 256 would need 768 TMEM columns
-        if ((Hq / Hkv) % 2 == 0)
+        if ((Hq / Hkv) % 2 == 0) {
+            // the persistent kernel (one gate or none) needs the workspace for its unit counter
+            if (ws != nullptr && gates.n <= 1) {
+                const cudaError_t e = launch_attention_persistent(
+                    tq, tk, tv, cu_kept, B, max_M, Hq, Hkv, HD, pos, rank, gates.n ? gates.gls[0] : nullptr,
+                    gates.n ? gates.g[0] : nullptr, gates.n ? c : nullptr, sm_scale, out, lse, ws, ws_bytes, early, st);
+                if (e != cudaErrorNotSupported || gates.n == 0) return e;
+            }
+            if (gates.n == 0) return cudaErrorNotSupported;
             return launch_gqa2<HD>(tq, tk, tv, cu_kept, B, max_M, Hq, Hkv, pos, rank, gates, c, sm_scale, out, lse,
                                    ws, ws_bytes, early, st);
+        }
     }
+    if (gates.n == 0) return cudaErrorNotSupported;
     int* status = device_status_ptr();
     const int n_qt_max = (max_M + BM - 1) / BM;
     dim3 grid(Hq, n_qt_max, B);
@@ -1257,7 +1171,7 @@ cudaError_t launch_gated_attention(const uint16_t* q, const uint16_t* k, const u
                                    uint16_t* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t st,
                                    bool inputs_ready) {
     if (M_total == 0 || B == 0) return cudaSuccess;
-    if (gates.n < 1 || gates.n > kMaxGates) return cudaErrorInvalidValue;
+    if (gates.n < 0 || gates.n > kMaxGates) return cudaErrorInvalidValue;  // 0: no gate (plain attention)
     if (d == 64)
         return launch_tc<64>(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, pos, rank, gates, c, sm_scale, out, lse,
                              ws, ws_bytes, inputs_ready, st);
@@ -1345,15 +1259,29 @@ int attention_kv_chunk(int B, int max_M, int Hq, int Hkv, bool have_ws) {
     return best_c;
 }
 
-size_t attention_workspace_bytes(int B, int max_M, int Hq, int Hkv, int d) {
+AttnWsLayout attention_ws_layout(int B, int max_M, int Hq, int Hkv, int d) {
+    AttnWsLayout L;
     const int n_qt = (max_M + BM - 1) / BM;
-    if (B <= 0 || n_qt < 4 || (Hq / Hkv) % 2 != 0 || d > 128) return 0;  // only the two-head kernel splits
-    const int C = attention_kv_chunk(B, max_M, Hq, Hkv, true);
-    if (C >= n_qt) return 0;  // this launch never splits
-    const int64_t max_nch = (n_qt + C - 1) / C;
-    const int64_t slots = static_cast<int64_t>(B) * (Hq / 2) * (n_qt - C);
-    return static_cast<size_t>(slots * max_nch * 2 * BM * (static_cast<int64_t>(d) + 1) * sizeof(float) +
-                               slots * sizeof(int));
+    L.C = n_qt > 0 ? n_qt : 1;
+    if (B <= 0 || n_qt <= 0 || Hkv <= 0 || (Hq / Hkv) % 2 != 0 || d > 128) return L;  // one-head kernel: none
+    auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+    L.C = attention_kv_chunk(B, max_M, Hq, Hkv, true);
+    L.total = 256;  // the unit counters of the persistent kernel
+    if (L.C < n_qt) {
+        L.max_nch = (n_qt + L.C - 1) / L.C;
+        L.slots_per_pair = n_qt - L.C;
+        L.slots = static_cast<int64_t>(B) * (Hq / 2) * L.slots_per_pair;
+        L.cnt_off = 256;
+        L.o_off = al(L.cnt_off + static_cast<size_t>(L.slots) * 2 * sizeof(int));
+        L.lse_off = L.o_off + static_cast<size_t>(L.slots) * L.max_nch * 2 * BM * d * sizeof(float);
+        L.total = L.lse_off + static_cast<size_t>(L.slots) * L.max_nch * 2 * BM * sizeof(float);
+        L.zero_bytes = L.o_off;
+    }
+    return L;
+}
+
+size_t attention_workspace_bytes(int B, int max_M, int Hq, int Hkv, int d) {
+    return attention_ws_layout(B, max_M, Hq, Hkv, d).total;
 }
 
 // ---------------------------------------------------------------------------
@@ -1404,12 +1332,8 @@ cudaError_t launch_gated_attention_noalloc(const uint16_t* q, const uint16_t* k,
     cudaError_t e = noalloc_attention_scratch(&ws);
     if (e != cudaSuccess) return e;
     if (need > 0) {
-        // the arrival counters must start at zero: the last call may have stopped early
-        const int n_qt = (max_M + BM - 1) / BM;
-        const int C = attention_kv_chunk(B, max_M, Hq, Hkv, true);
-        const int64_t slots = static_cast<int64_t>(B) * (Hq / 2) * (n_qt - C);
-        const size_t cnt_bytes = static_cast<size_t>(slots) * sizeof(int);
-        e = cudaMemsetAsync(static_cast<uint8_t*>(ws) + (need - cnt_bytes), 0, cnt_bytes, st);
+        // the counters must start at zero: the last call may have stopped early
+        e = cudaMemsetAsync(ws, 0, attention_ws_layout(B, max_M, Hq, Hkv, d).zero_bytes, st);
         if (e != cudaSuccess) return e;
     }
     return launch_gated_attention(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, d, pos, rank, gates, c, sm_scale,

@@ -87,11 +87,19 @@ tg_status do_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
     TG_REQUIRE(B >= 0 && M_total >= 0 && max_M >= 0, "negative size");
     if (tg_status s = check_attn_shape(Hq, Hkv, d)) return s;
     TG_REQUIRE(sm_scale > 0.f, "sm_scale must be positive");
-    TG_SUPPORT(gates.n >= 1 && gates.n <= tg::kMaxGates, "n_gates=%d must be in [1, %d]", gates.n, tg::kMaxGates);
+    TG_SUPPORT(gates.n >= 0 && gates.n <= tg::kMaxGates, "n_gates=%d must be in [0, %d]", gates.n, tg::kMaxGates);
+    if (gates.n == 0) {
+        // no gate: ordinary causal attention (bias 0, tau 1) on the persistent kernel
+        TG_SUPPORT(d <= 128 && (Hq / Hkv) % 2 == 0,
+                   "attention without a gate needs head_dim 64 or 128 and an even GQA group (Hq/Hkv=%d, d=%d)",
+                   Hq / Hkv, d);
+        TG_REQUIRE(ws != nullptr, "attention without a gate needs ws (tg_gated_attention_workspace_size bytes)");
+    }
     if (B == 0 || M_total == 0) return TG_OK;
     TG_REQUIRE(max_M > 0, "max_M must bound the longest sequence");
     for (int i = 0; i < gates.n; ++i) TG_REQUIRE(gates.gls[i] && gates.g[i], "null gls or g of gate %d", i);
-    TG_REQUIRE(q && k && v && cu_kept && pos && rank && c && out, "null pointer argument");
+    TG_REQUIRE(q && k && v && cu_kept && out, "null pointer argument");
+    TG_REQUIRE(gates.n == 0 || (pos && rank && c), "null pos, rank or c");
     TG_REQUIRE(aligned16(q) && aligned16(k) && aligned16(v) && aligned16(out),
                "q, k, v and out must be 16-byte aligned");
     if (ws) {
@@ -331,8 +339,10 @@ tg_status tg_gated_attention(const uint16_t* q, const uint16_t* k, const uint16_
                              int64_t M_total, int max_M, int Hq, int Hkv, int d, const int32_t* pos,
                              const int32_t* rank, const float* gls, const float* g, const float* c, float sm_scale,
                              uint16_t* out, float* lse, void* ws, size_t ws_bytes, tg_stream_t stream) {
-    return do_attention(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, d, pos, rank, tg::single_gate(gls, g), c,
-                        sm_scale, out, lse, ws, ws_bytes, stream);
+    tg::GateSet gates = tg::single_gate(gls, g);
+    if (!gls && !g && !c) gates.n = 0;  // no gate: ordinary causal attention
+    return do_attention(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, d, pos, rank, gates, c, sm_scale, out, lse, ws,
+                        ws_bytes, stream);
 }
 
 tg_status tg_gated_attention_gates(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* cu_kept,

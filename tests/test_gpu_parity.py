@@ -500,3 +500,72 @@ def test_attention_is_deterministic_with_the_causal_split(tg):
     outs = [_run_attention(tg, w, comp, ai, gls32) for _ in range(3)]
     for o, l in outs[1:]:
         assert np.array_equal(o, outs[0][0]) and np.array_equal(l, outs[0][1])
+
+
+def _raw_attention(tg, w, comp, ai, gls32, c, ws_mode, g=None):
+    """tg_gated_attention through the C ABI with explicit pointers: gls/g/c may be None (no
+    gate); ws_mode "auto" passes the sized workspace, None passes no workspace."""
+    from learned_token_pruning_rmsnorm_b200 import _lib
+    lib = _lib.load()
+    ck = comp["cu_kept"]
+    M, max_M = int(ck[-1]), int(np.max(np.diff(ck)))
+    keep = [H.bf16_dev(ai["q"]), H.bf16_dev(ai["k"]), H.bf16_dev(ai["v"]), H.i32_dev(ck), H.i32_dev(comp["pos"]),
+            H.i32_dev(comp["rank"])]
+    gl = None if gls32 is None else H.f32_dev(gls32)
+    gg = None if g is None else H.f32_dev(g)
+    cc = None if c is None else H.f32_dev(c)
+    ws = None
+    if ws_mode == "auto":
+        n = int(lib.tg_gated_attention_workspace_size(w.B, max_M, w.Hq, w.Hkv, w.d))
+        ws = torch.zeros(max(n, 256), dtype=torch.uint8, device="cuda")
+    out = torch.empty((M, w.Hq, w.d), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((M, w.Hq), dtype=torch.float32, device="cuda")
+    p = lambda t: None if t is None else t.data_ptr()  # noqa: E731
+    _lib.check(lib.tg_gated_attention(p(keep[0]), p(keep[1]), p(keep[2]), p(keep[3]), w.B, M, max_M, w.Hq, w.Hkv,
+                                      w.d, p(keep[4]), p(keep[5]), p(gl), p(gg), p(cc), 1.0 / math.sqrt(w.d),
+                                      p(out), p(lse), p(ws), 0 if ws is None else ws.numel(), None))
+    torch.cuda.synchronize()
+    return out.float().cpu().numpy(), lse.cpu().numpy()
+
+
+@pytest.mark.parametrize("name", ["c0_tiny", "c1_16k", "c2_32k_k2000"])
+def test_attention_without_gate_is_the_zero_gate_bit_for_bit(tg, name):
+    """gls = g = c = NULL is ordinary causal attention (bias 0, tau 1): the kernel then
+    skips the bias k-step, whose products with gls = 0 add exact zeros, and tau = 1 + 0 is
+    exactly 1; so it equals the gated call with gls = 0 and c = 0 bit for bit, and it is
+    within the parity bars of the oracle's gated attention with zero bias."""
+    w, comp, ai, gls32, _, _, _ = attn_case(name)
+    zeros = np.zeros_like(gls32)
+    plain, plain_lse = _raw_attention(tg, w, comp, ai, None, None, "auto")
+    gated0, gated0_lse = _raw_attention(tg, w, comp, ai, zeros, np.zeros_like(ai["c"]), "auto", g=ai["g"])
+    np.testing.assert_array_equal(plain, gated0)
+    np.testing.assert_array_equal(plain_lse, gated0_lse)
+    ck = comp["cu_kept"]
+    rows = np.unique(np.concatenate([np.arange(0, int(ck[-1]), 13), [int(ck[-1]) - 1]])).astype(np.int64)
+    ref, ref_lse = oracle.gated_attention(ai["q"], ai["k"], ai["v"], ck, comp["pos"], comp["rank"], zeros, ai["g"],
+                                          np.zeros_like(ai["c"]), rows=rows)
+    H.assert_attention_close(plain[rows], ref, name + " no gate")
+    assert np.max(np.abs(plain_lse[rows] - ref_lse)) <= H.LSE_ABS
+
+
+def test_attention_without_gate_needs_a_workspace(tg):
+    from learned_token_pruning_rmsnorm_b200 import TokenGateError
+    w, comp, ai, gls32, _, _, _ = attn_case("c0_tiny")
+    with pytest.raises(TokenGateError):
+        _raw_attention(tg, w, comp, ai, None, None, None)
+
+
+@pytest.mark.parametrize("name", ["c1_16k", "c2_32k_k2000", "c4_varlen"])
+def test_persistent_and_per_unit_kernels_agree(tg, name):
+    """With a workspace the attention runs persistent CTAs that take units from a counter;
+    without one, one CTA per unit.  Same arithmetic per row (the row maximum, the
+    exponentials, the bf16 P), so the outputs agree within the parity bars and both match
+    the oracle's rows."""
+    w, comp, ai, gls32, rows, out_ref, lse_ref = attn_case(name, rows_step=7 if name == "c4_varlen" else None)
+    a, a_lse = _raw_attention(tg, w, comp, ai, gls32, ai["c"], "auto", g=ai["g"])
+    b, b_lse = _raw_attention(tg, w, comp, ai, gls32, ai["c"], None, g=ai["g"])
+    H.assert_attention_close(a, b.astype(np.float64), name + " persistent vs per-unit")
+    sel = slice(None) if rows is None else rows
+    H.assert_attention_close(a[sel], out_ref, name + " persistent")
+    H.assert_attention_close(b[sel], out_ref, name + " per-unit")
+    assert np.max(np.abs(a_lse[sel] - lse_ref)) <= H.LSE_ABS
