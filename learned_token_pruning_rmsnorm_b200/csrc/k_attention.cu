@@ -1134,11 +1134,11 @@ cudaError_t launch_tc(const uint16_t* q, const uint16_t* k, const uint16_t* v, c
         return cudaErrorInvalidValue;
     if constexpr (HD <= 128) {  // two heads of 256 would need 768 TMEM columns
         if ((Hq / Hkv) % 2 == 0) {
-            // the persistent kernel (one gate or none) needs the workspace for its unit counter
-            if (ws != nullptr && gates.n <= 1) {
-                const cudaError_t e = launch_attention_persistent(
-                    tq, tk, tv, cu_kept, B, max_M, Hq, Hkv, HD, pos, rank, gates.n ? gates.gls[0] : nullptr,
-                    gates.n ? gates.g[0] : nullptr, gates.n ? c : nullptr, sm_scale, out, lse, ws, ws_bytes, early, st);
+            // the persistent kernel needs the workspace for its unit counter
+            if (ws != nullptr) {
+                const cudaError_t e = launch_attention_persistent(tq, tk, tv, cu_kept, B, max_M, Hq, Hkv, HD, pos,
+                                                                  rank, gates, c, sm_scale, out, lse, ws, ws_bytes,
+                                                                  early, st);
                 if (e != cudaErrorNotSupported || gates.n == 0) return e;
             }
             if (gates.n == 0) return cudaErrorNotSupported;

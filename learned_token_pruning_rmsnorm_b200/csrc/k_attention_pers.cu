@@ -118,9 +118,9 @@ template <int HD, bool GATED>
 __global__ void __launch_bounds__(PT_THREADS, 1)
 gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const int32_t* __restrict__ cu_kept,
-                       const int32_t* __restrict__ pos, const int32_t* __restrict__ rank,
-                       const float* __restrict__ gls, const float* __restrict__ g, const float* __restrict__ c,
-                       float sm_scale, int Hq, int Hkv, int B, int kv_chunk, int64_t total_units, SplitWs ws,
+                       const int32_t* __restrict__ pos, const int32_t* __restrict__ rank, const GateSet gates,
+                       const float* __restrict__ c, float sm_scale, int Hq, int Hkv, int B, int kv_chunk,
+                       int64_t total_units, SplitWs ws,
                        int* __restrict__ sched, uint16_t* __restrict__ out, float* __restrict__ lse,
                        int* __restrict__ status, int early) {
     using L = PtSmem<HD>;
@@ -148,8 +148,9 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     volatile int* ring = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 16);  // [PT_RING]
 
     if (GATED) {
-        // K cores 8..15 (columns 8..15) of the four bias operand tiles stay zero; the
-        // producer writes columns 0..7 (the gate's four products, then zeros)
+        // Gate i owns columns 4i..4i+3 of the bias k-step; the producer writes columns 0..7
+        // (gates 0 and 1, zeros for an absent gate 1) and, with three or four gates, columns
+        // 8..15, which otherwise stay the zeros written here
         for (int i = threadIdx.x; i < 4 * (BM / 8) * 8; i += blockDim.x) {
             const int tile = i / ((BM / 8) * 8), rem = i % ((BM / 8) * 8);
             *reinterpret_cast<uint4*>(smem + L::OFF_QX + tile * L::EXT + (rem >> 3) * 256 + 128 + (rem & 7) * 16) =
@@ -244,16 +245,23 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 ++q_issued;
             }
             if (GATED) {
-                // Q_ext row = (bh, bl, bh, bl, 0, ...): the bf16 high and low parts of
-                // softplus(g_h) / sm_scale; lane l writes rows 4l..4l+3 of both heads
+                // Q_ext row of head h: gate i's columns hold (bh, bl, bh, bl), the bf16 high
+                // and low parts of softplus(g_i[h]) / sm_scale; lane l writes rows 4l..4l+3
+                // of both heads
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
-                    const uint32_t hl = bf16_hi_lo(softplus_f(__ldg(g + 2 * U.pair + hh)) / sm_scale);
+                    const int hq = 2 * U.pair + hh;
+                    auto hl_of = [&](const float* gp) { return bf16_hi_lo(softplus_f(__ldg(gp + hq)) / sm_scale); };
+                    const uint32_t h0 = hl_of(gates.g[0]);
+                    const uint32_t h1 = gates.n > 1 ? hl_of(gates.g[1]) : 0u;
+                    const uint32_t h2 = gates.n > 2 ? hl_of(gates.g[2]) : 0u;
+                    const uint32_t h3 = gates.n > 3 ? hl_of(gates.g[3]) : 0u;
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         const int r = lane * 4 + i;
-                        *reinterpret_cast<uint4*>(smem + L::OFF_QX + hh * L::EXT + (r >> 3) * 256 + (r & 7) * 16) =
-                            make_uint4(hl, hl, 0u, 0u);
+                        uint8_t* row = smem + L::OFF_QX + hh * L::EXT + (r >> 3) * 256 + (r & 7) * 16;
+                        *reinterpret_cast<uint4*>(row) = make_uint4(h0, h0, h1, h1);
+                        if (gates.n > 2) *reinterpret_cast<uint4*>(row + 128) = make_uint4(h2, h2, h3, h3);
                     }
                 }
                 fence_proxy_async_smem();
@@ -297,16 +305,27 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 }
                 if (GATED) {
                     wait_inputs();  // gls (the compaction map) from here on
-                    // K_ext row of key k = (gh, gh, gl, gl, 0, ...): the bf16 high and low
-                    // parts of gls_k (0 past the sequence end); lane l writes keys 4l..4l+3
+                    // K_ext row of key k: gate i's columns hold (gh, gh, gl, gl), the bf16 high
+                    // and low parts of gls_i[k] (0 past the sequence end); lane l writes keys
+                    // 4l..4l+3
+                    const int key0 = (U.kv0 + j) * BN + lane * 4;
+                    auto kx_of = [&](const float* gp, int i) {
+                        const float gv = key0 + i < U.Mb ? ldg_early(gp + U.seq0 + key0 + i) : 0.f;
+                        const uint32_t hl = bf16_hi_lo(gv);
+                        return make_uint2(__byte_perm(hl, 0u, 0x1010), __byte_perm(hl, 0u, 0x3232));
+                    };
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         const int r = lane * 4 + i;
-                        const int key_local = (U.kv0 + j) * BN + r;
-                        const float gv = key_local < U.Mb ? ldg_early(gls + U.seq0 + key_local) : 0.f;
-                        const uint32_t hl = bf16_hi_lo(gv);
-                        *reinterpret_cast<uint4*>(smem + L::OFF_KX + s * L::EXT + (r >> 3) * 256 + (r & 7) * 16) =
-                            make_uint4(__byte_perm(hl, 0u, 0x1010), __byte_perm(hl, 0u, 0x3232), 0u, 0u);
+                        uint8_t* row = smem + L::OFF_KX + s * L::EXT + (r >> 3) * 256 + (r & 7) * 16;
+                        const uint2 k0 = kx_of(gates.gls[0], i);
+                        const uint2 k1 = gates.n > 1 ? kx_of(gates.gls[1], i) : make_uint2(0u, 0u);
+                        *reinterpret_cast<uint4*>(row) = make_uint4(k0.x, k0.y, k1.x, k1.y);
+                        if (gates.n > 2) {
+                            const uint2 k2 = kx_of(gates.gls[2], i);
+                            const uint2 k3 = gates.n > 3 ? kx_of(gates.gls[3], i) : make_uint2(0u, 0u);
+                            *reinterpret_cast<uint4*>(row + 128) = make_uint4(k2.x, k2.y, k3.x, k3.y);
+                        }
                     }
                     fence_proxy_async_smem();  // K_ext is read by the tensor core (async proxy)
                     __syncwarp();
@@ -696,8 +715,8 @@ static int pers_launch_regs() {
 template <int HD, bool GATED>
 static cudaError_t launch_pers_impl(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                     const int32_t* cu_kept, int B, int max_M, int Hq, int Hkv, const int32_t* pos,
-                                    const int32_t* rank, const float* gls, const float* g, const float* c,
-                                    float sm_scale, uint16_t* out, float* lse, void* ws, size_t ws_bytes, bool early,
+                                    const int32_t* rank, const GateSet& gates, const float* c, float sm_scale,
+                                    uint16_t* out, float* lse, void* ws, size_t ws_bytes, bool early,
                                     cudaStream_t st) {
     using L = PtSmem<HD>;
     static std::atomic<uint64_t> attr_set{0};
@@ -723,25 +742,25 @@ static cudaError_t launch_pers_impl(const CUtensorMap& tq, const CUtensorMap& tk
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const unsigned grid = static_cast<unsigned>(total < sms ? total : sms);
     return launch_pdl(gated_attn_pers_kernel<HD, GATED>, dim3(grid), dim3(PT_THREADS), static_cast<size_t>(L::ALLOC),
-                      st, tq, tk, tv, cu_kept, pos, rank, gls, g, c, sm_scale, Hq, Hkv, B, lay.C, total, sw,
+                      st, tq, tk, tv, cu_kept, pos, rank, gates, c, sm_scale, Hq, Hkv, B, lay.C, total, sw,
                       reinterpret_cast<int*>(base), out, lse, device_status_ptr(), early ? 1 : 0);
 }
 
 cudaError_t launch_attention_persistent(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                         const int32_t* cu_kept, int B, int max_M, int Hq, int Hkv, int d,
-                                        const int32_t* pos, const int32_t* rank, const float* gls, const float* g,
-                                        const float* c, float sm_scale, uint16_t* out, float* lse, void* ws,
-                                        size_t ws_bytes, bool early, cudaStream_t st) {
-    const bool gated = gls != nullptr;
+                                        const int32_t* pos, const int32_t* rank, const GateSet& gates, const float* c,
+                                        float sm_scale, uint16_t* out, float* lse, void* ws, size_t ws_bytes,
+                                        bool early, cudaStream_t st) {
+    const bool gated = gates.n > 0;
     if (d == 64)
-        return gated ? launch_pers_impl<64, true>(tq, tk, tv, cu_kept, B, max_M, Hq, Hkv, pos, rank, gls, g, c,
+        return gated ? launch_pers_impl<64, true>(tq, tk, tv, cu_kept, B, max_M, Hq, Hkv, pos, rank, gates, c,
                                                   sm_scale, out, lse, ws, ws_bytes, early, st)
-                     : launch_pers_impl<64, false>(tq, tk, tv, cu_kept, B, max_M, Hq, Hkv, pos, rank, gls, g, c,
+                     : launch_pers_impl<64, false>(tq, tk, tv, cu_kept, B, max_M, Hq, Hkv, pos, rank, gates, c,
                                                    sm_scale, out, lse, ws, ws_bytes, early, st);
     if (d == 128)
-        return gated ? launch_pers_impl<128, true>(tq, tk, tv, cu_kept, B, max_M, Hq, Hkv, pos, rank, gls, g, c,
+        return gated ? launch_pers_impl<128, true>(tq, tk, tv, cu_kept, B, max_M, Hq, Hkv, pos, rank, gates, c,
                                                    sm_scale, out, lse, ws, ws_bytes, early, st)
-                     : launch_pers_impl<128, false>(tq, tk, tv, cu_kept, B, max_M, Hq, Hkv, pos, rank, gls, g, c,
+                     : launch_pers_impl<128, false>(tq, tk, tv, cu_kept, B, max_M, Hq, Hkv, pos, rank, gates, c,
                                                     sm_scale, out, lse, ws, ws_bytes, early, st);
     return cudaErrorNotSupported;
 }

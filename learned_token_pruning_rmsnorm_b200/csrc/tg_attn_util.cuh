@@ -160,12 +160,12 @@ struct AttnWsLayout {
 attn::AttnWsLayout attention_ws_layout(int B, int max_M, int Hq, int Hkv, int d);
 
 // The persistent attention (k_attention_pers.cu): head_dim 64 or 128, GQA groups of
-// even size, one gate (gls, g, c) or none (gls == g == c == nullptr: bias 0, tau 1).
+// even size, 1 to kMaxGates gates, or none (gates.n == 0: bias 0, tau 1, c unused).
 // Needs the workspace (its unit counter); returns cudaErrorNotSupported when it cannot
 // run on this build or device, so that the caller can fall back.
 cudaError_t launch_attention_persistent(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                         const int32_t* cu_kept, int B, int max_M, int Hq, int Hkv, int d,
-                                        const int32_t* pos, const int32_t* rank, const float* gls, const float* g,
-                                        const float* c, float sm_scale, uint16_t* out, float* lse, void* ws,
-                                        size_t ws_bytes, bool early, cudaStream_t st);
+                                        const int32_t* pos, const int32_t* rank, const GateSet& gates, const float* c,
+                                        float sm_scale, uint16_t* out, float* lse, void* ws, size_t ws_bytes,
+                                        bool early, cudaStream_t st);
 }  // namespace tg
