@@ -73,6 +73,7 @@ SIGNATURES = {
                                    C.c_size_t, P], i32),
     "tg_device_status": ([P, i32, P], i32),
     "tg_selftest_bounded_wait": ([i64, P], i32),
+    "tg_selftest_exp2": ([P, P, i64, P], i32),
 }
 
 

@@ -1157,10 +1157,10 @@ cudaError_t launch_tc(const uint16_t* q, const uint16_t* k, const uint16_t* v, c
 }  // namespace
 
 #ifdef TG_TRACE
-extern "C" int tg_trace_read_attention(unsigned long long* host) {
+extern "C" __attribute__((visibility("default"))) int tg_trace_read_attention(unsigned long long* host) {
     return cudaMemcpyFromSymbol(host, g_attn_trace, sizeof(g_attn_trace)) == cudaSuccess ? 0 : 1;
 }
-extern "C" int tg_trace_read_attention_ctas(unsigned long long* host) {
+extern "C" __attribute__((visibility("default"))) int tg_trace_read_attention_ctas(unsigned long long* host) {
     return cudaMemcpyFromSymbol(host, g_attn_cta, sizeof(g_attn_cta)) == cudaSuccess ? 0 : 1;
 }
 #endif

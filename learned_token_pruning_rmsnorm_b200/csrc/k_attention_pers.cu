@@ -47,6 +47,14 @@ constexpr int PT_LAUNCH_REGS = 168;   // registers per thread at launch (65536 /
 constexpr int PT_SOFTMAX_REGS = 200;  // after the hand-over: 256 x 200 + 128 x 104 = 384 x 168
 constexpr int PT_OTHER_REGS = 104;
 constexpr int PT_RING = 8;            // unit numbers in flight between the producer and the consumers
+// Of every 32 columns of a tile, the first 4 * PT_POLY_QUADS take their exponentials on the
+// FMA pipe (exp2_poly_x2) instead of the special-function unit, except in the diagonal tile,
+// whose masked elements must come out exactly 0.
+#ifndef TG_EXP2_POLY_QUADS
+#define TG_EXP2_POLY_QUADS 3
+#endif
+constexpr int PT_POLY_QUADS = TG_EXP2_POLY_QUADS;
+static_assert(PT_POLY_QUADS >= 0 && PT_POLY_QUADS <= 8, "quads of 4 columns per 32");
 static_assert(256 * PT_SOFTMAX_REGS + 128 * PT_OTHER_REGS <= PT_THREADS * PT_LAUNCH_REGS, "register hand-over");
 
 template <int HD>
@@ -114,6 +122,20 @@ __device__ __forceinline__ void named_bar_sync(int id, int n) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
+// Optional device trace (builds with -DTG_TRACE only): per-CTA globaltimer stamps of the
+// hand-offs of the first unit and of the whole CTA, with the SM id and the unit count.
+#ifdef TG_TRACE
+__device__ unsigned long long g_pers_trace[1024 * 16];
+#define PT_STAMP(slot, cond)                                                             \
+    do {                                                                                 \
+        if ((cond) && blockIdx.x < 1024) g_pers_trace[blockIdx.x * 16 + (slot)] = globaltimer(); \
+    } while (0)
+#else
+#define PT_STAMP(slot, cond) \
+    do {                     \
+    } while (0)
+#endif
+
 template <int HD, bool GATED>
 __global__ void __launch_bounds__(PT_THREADS, 1)
 gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -129,6 +151,7 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int pairs = Hq / 2;
     const int group = Hq / Hkv;
+    PT_STAMP(0, threadIdx.x == 0);
     // `early`: q, k, v, g, c and cu_kept were complete before the preceding kernel started
     // (the caller's guarantee), so set-up, Q and the first K/V tiles go ahead while that
     // kernel runs; gls, pos, rank, the scratch and the unit counter are touched only after
@@ -183,6 +206,7 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    PT_STAMP(1, threadIdx.x == 0);
 
     // The producer / MMA warpgroup hands most of its registers to the softmax warpgroups;
     // each role's code sits inside the branch that set its register budget.
@@ -243,6 +267,7 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                         tma_load_2d(sQ + hh * L::TILE_Q + hf * BM * 128, &tmQ, (2 * U.pair + hh) * HD + hf * 64,
                                     U.seq0 + U.qt * BM, bar(T_Q_FULL));
                 ++q_issued;
+                PT_STAMP(2, uc == 0);
             }
             if (GATED) {
                 // Q_ext row of head h: gate i's columns hold (bh, bl, bh, bl), the bf16 high
@@ -391,8 +416,10 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 if (unit < 0) break;
                 Unit U{};
                 decode_unit(unit, pairs, B, cu_kept, kv_chunk, &U);
-                ok = mbar_wait(bar(T_Q_FULL), uc & 1, abort_flag, status, TG_WHERE_MMA) &&
-                     mbar_wait(bar(T_K_FULL + (t & 1)), (t >> 1) & 1, abort_flag, status, TG_WHERE_MMA);
+                ok = mbar_wait(bar(T_Q_FULL), uc & 1, abort_flag, status, TG_WHERE_MMA);
+                PT_STAMP(3, uc == 0);
+                ok = ok && mbar_wait(bar(T_K_FULL + (t & 1)), (t >> 1) & 1, abort_flag, status, TG_WHERE_MMA);
+                PT_STAMP(4, uc == 0);
                 if (!ok) break;
                 tc_fence_after();
                 // S_h(0) of this unit: S_h's last reader (PV_h of the previous unit's last tile)
@@ -499,6 +526,7 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     ok = false;
                     break;
                 }
+                PT_STAMP(5, uc == 0 && j == 0 && threadIdx.x == 0);
                 tc_fence_after();
                 float x[BN];
 #pragma unroll
@@ -524,6 +552,7 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     rescale_o = j > 0;
                 }
                 const uint64_t nm2 = f32x2_pack(-m_run, -m_run);
+                const bool poly_ok = jt != U.qt;  // no masked element in this tile
                 uint64_t sp[4] = {0ull, 0ull, 0ull, 0ull};
                 // P row r as bf16 pairs over the first 64 columns of S_h (the A operand of the
                 // PV product, read from TMEM); every S value is in registers already
@@ -535,12 +564,18 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                         const int cc = c32 * 32 + 4 * e;
                         const uint64_t a0 = f32x2_fma(al2, f32x2_pack(x[cc], x[cc + 1]), nm2);
                         const uint64_t a1 = f32x2_fma(al2, f32x2_pack(x[cc + 2], x[cc + 3]), nm2);
-                        const float p0 = ex2_approx(f32x2_lo(a0)), p1 = ex2_approx(f32x2_hi(a0));
-                        const float p2 = ex2_approx(f32x2_lo(a1)), p3 = ex2_approx(f32x2_hi(a1));
-                        sp[(2 * e) & 3] = f32x2_add(sp[(2 * e) & 3], f32x2_pack(p0, p1));
-                        sp[(2 * e + 1) & 3] = f32x2_add(sp[(2 * e + 1) & 3], f32x2_pack(p2, p3));
-                        pk[2 * e] = pack_bf16x2(p0, p1);
-                        pk[2 * e + 1] = pack_bf16x2(p2, p3);
+                        uint64_t e0, e1;
+                        if (e < PT_POLY_QUADS && poly_ok) {
+                            e0 = exp2_poly_x2(a0);
+                            e1 = exp2_poly_x2(a1);
+                        } else {
+                            e0 = f32x2_pack(ex2_approx(f32x2_lo(a0)), ex2_approx(f32x2_hi(a0)));
+                            e1 = f32x2_pack(ex2_approx(f32x2_lo(a1)), ex2_approx(f32x2_hi(a1)));
+                        }
+                        sp[(2 * e) & 3] = f32x2_add(sp[(2 * e) & 3], e0);
+                        sp[(2 * e + 1) & 3] = f32x2_add(sp[(2 * e + 1) & 3], e1);
+                        pk[2 * e] = pack_bf16x2(f32x2_lo(e0), f32x2_hi(e0));
+                        pk[2 * e + 1] = pack_bf16x2(f32x2_lo(e1), f32x2_hi(e1));
                     }
                     tmem_st16u(tS + c32 * 16, pk);
                 }
@@ -566,7 +601,9 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 if (lane == 0) mbar_arrive(bar(T_P_FULL + h));
             }
             // ---------------------------------------------------------------- epilogue
+            PT_STAMP(6, uc == 0 && threadIdx.x == 0);
             if (ok) ok = mbar_wait_warp(bar(T_O_FULL + h), uc & 1, abort_flag, status, TG_WHERE_SOFTMAX);
+            PT_STAMP(7, uc == 0 && threadIdx.x == 0);
             if (bar_red_or(bid, 128, !ok)) break;
             tc_fence_after();
             const float inv_l = 1.0f / l_run;
@@ -680,8 +717,17 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             // the O reads are complete before the next unit's first PV_h overwrites O_h
             // (that product waits for this warpgroup's next P arrival)
             tc_fence_before();
+            PT_STAMP(8, uc == 0 && threadIdx.x == 0);
             ++uc;
         }
+#ifdef TG_TRACE
+        if (threadIdx.x == 0 && blockIdx.x < 1024) {
+            unsigned smid;
+            asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+            g_pers_trace[blockIdx.x * 16 + 9] = globaltimer();
+            g_pers_trace[blockIdx.x * 16 + 11] = smid | (static_cast<unsigned long long>(uc) << 32);
+        }
+#endif
     }
 
     tc_fence_before();
@@ -690,6 +736,7 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
+    PT_STAMP(10, threadIdx.x == 0);
     if (threadIdx.x == 0) {
         // the last CTA to finish resets the unit counter for the next launch
         __threadfence();
@@ -701,7 +748,30 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     }
 }
 
+__global__ void exp2_poly_selftest_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n) {
+    for (int64_t i = 2 * (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x); i < n;
+         i += 2 * static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const float a = x[i], b = i + 1 < n ? x[i + 1] : 0.f;
+        const uint64_t r = exp2_poly_x2(f32x2_pack(a, b));
+        y[i] = f32x2_lo(r);
+        if (i + 1 < n) y[i + 1] = f32x2_hi(r);
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_exp2_poly_selftest(const float* x, float* y, int64_t n, cudaStream_t st) {
+    if (n <= 0) return cudaSuccess;
+    const int64_t blocks = (n + 511) / 512;
+    exp2_poly_selftest_kernel<<<static_cast<unsigned>(blocks < 1024 ? blocks : 1024), 256, 0, st>>>(x, y, n);
+    return cudaGetLastError();
+}
+
+#ifdef TG_TRACE
+extern "C" __attribute__((visibility("default"))) int tg_trace_read_attention_pers(unsigned long long* host) {
+    return cudaMemcpyFromSymbol(host, g_pers_trace, sizeof(g_pers_trace)) == cudaSuccess ? 0 : 1;
+}
+#endif
 
 // Registers per thread the persistent kernel was built with, or 0 if it cannot run (its
 // register hand-over needs exactly the launch budget).

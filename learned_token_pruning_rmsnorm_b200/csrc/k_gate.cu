@@ -337,7 +337,7 @@ cudaError_t launch_score_tc(const uint16_t* hidden, const int32_t* cu_seqlens, c
 }  // namespace
 
 #ifdef TG_TRACE
-extern "C" int tg_trace_read_score(unsigned long long* pipe, unsigned long long* ctas) {
+extern "C" __attribute__((visibility("default"))) int tg_trace_read_score(unsigned long long* pipe, unsigned long long* ctas) {
     if (cudaMemcpyFromSymbol(pipe, g_score_trace, sizeof(g_score_trace)) != cudaSuccess) return 1;
     return cudaMemcpyFromSymbol(ctas, g_score_cta, sizeof(g_score_cta)) == cudaSuccess ? 0 : 1;
 }

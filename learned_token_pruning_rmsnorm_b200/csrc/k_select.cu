@@ -510,7 +510,7 @@ scatter_rows_kernel(const uint4* __restrict__ in, const int32_t* __restrict__ id
 }  // namespace
 
 #ifdef TG_TRACE
-extern "C" int tg_trace_read_select(unsigned long long* host) {
+extern "C" __attribute__((visibility("default"))) int tg_trace_read_select(unsigned long long* host) {
     return cudaMemcpyFromSymbol(host, g_sel_trace, sizeof(g_sel_trace)) == cudaSuccess ? 0 : 1;
 }
 #endif

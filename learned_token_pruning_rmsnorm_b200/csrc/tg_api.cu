@@ -6,9 +6,21 @@
 #include <cstdio>
 #include <string>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "tg_internal.cuh"
 
 namespace {
+
+// NVTX range over one entry point (host side: argument checks and the launches it
+// enqueues), named after the call, so that a profiler's timeline shows each stage.  The
+// NVTX calls are no-ops unless a profiling tool is attached.
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 thread_local std::string g_last_error;
 
@@ -156,6 +168,7 @@ tg_status tg_masked_gated_attention(const uint16_t* q, const uint16_t* k, const 
                                     const int32_t* cu_kept, int B, int64_t T, int64_t M_total, int max_M, int Hq,
                                     int Hkv, int d, const float* g, const float* c, float sm_scale, uint16_t* out,
                                     uint8_t* keep_out, void* ws, size_t ws_bytes, tg_stream_t stream) {
+    NvtxRange nvtx_range("tg_masked_gated_attention");
     TG_REQUIRE(B >= 0 && T >= 0 && M_total >= 0 && M_total <= T && max_M >= 0, "bad sizes");
     if (tg_status s = check_attn_shape(Hq, Hkv, d)) return s;
     TG_REQUIRE(sm_scale > 0.f, "sm_scale must be positive");
@@ -233,6 +246,7 @@ int64_t tg_kept_count(const int32_t* h_cu_seqlens, const int32_t* h_span, const 
 }
 
 tg_status tg_gate_prepare(const uint16_t* gamma, const uint16_t* W1, int D, int I, uint16_t* Wg, tg_stream_t stream) {
+    NvtxRange nvtx_range("tg_gate_prepare");
     if (tg_status s = check_gate_shape(D, I)) return s;
     TG_REQUIRE(gamma && W1 && Wg, "null pointer argument");
     if (tg_status s = check_device()) return s;
@@ -242,12 +256,14 @@ tg_status tg_gate_prepare(const uint16_t* gamma, const uint16_t* W1, int D, int 
 tg_status tg_score(const uint16_t* hidden, const int32_t* cu_seqlens, const int32_t* span, int B, int64_t T, int D,
                    const uint16_t* Wg, const float* b1, const float* w2, float b2, int I, float eps, float* scores,
                    tg_stream_t stream) {
+    NvtxRange nvtx_range("tg_score");
     return do_score(hidden, cu_seqlens, span, B, T, D, Wg, b1, w2, b2, I, eps, scores, stream);
 }
 
 tg_status tg_select_topk(const float* scores, const int32_t* cu_seqlens, const int32_t* span, const int32_t* k, int B,
                          int64_t T, uint8_t* keep, const int32_t* cu_kept, int32_t* kept_idx, int32_t* pos,
                          int32_t* rank, float* gls, tg_stream_t stream) {
+    NvtxRange nvtx_range("tg_select_topk");
     TG_REQUIRE(B >= 0 && T >= 0, "negative size");
     if (B == 0 || T == 0) return TG_OK;
     TG_REQUIRE(scores && cu_seqlens && span && k && keep, "null pointer argument");
@@ -263,6 +279,7 @@ tg_status tg_compact(const uint16_t* hidden, const float* scores, const uint8_t*
                      const int32_t* span, int B, int64_t T, int D, const int32_t* cu_kept, int64_t M_total,
                      uint16_t* hidden_kept, int32_t* pos, int32_t* rank, float* gls, int32_t* kept_idx,
                      tg_stream_t stream) {
+    NvtxRange nvtx_range("tg_compact");
     TG_REQUIRE(B >= 0 && T >= 0 && M_total >= 0 && M_total <= T, "bad sizes (B=%d T=%lld M=%lld)", B, (long long)T,
                (long long)M_total);
     if (B == 0 || T == 0 || M_total == 0) return TG_OK;  // nothing is kept: no output to write
@@ -286,6 +303,7 @@ tg_status tg_compact(const uint16_t* hidden, const float* scores, const uint8_t*
 
 tg_status tg_gather_rows(const void* src, int64_t T, int64_t row_bytes, const int32_t* kept_idx, int64_t M, void* dst,
                          tg_stream_t stream) {
+    NvtxRange nvtx_range("tg_gather_rows");
     TG_REQUIRE(T >= 0 && M >= 0 && row_bytes >= 0, "negative size");
     if (M == 0 || row_bytes == 0) return TG_OK;
     TG_REQUIRE(src && kept_idx && dst, "null pointer argument");
@@ -310,6 +328,7 @@ tg_status tg_gated_attention_noalloc(const uint16_t* q, const uint16_t* k, const
                                      int B, int64_t M_total, int max_M, int Hq, int Hkv, int d, const int32_t* pos,
                                      const int32_t* rank, const float* gls, const float* g, const float* c,
                                      float sm_scale, uint16_t* out, float* lse, tg_stream_t stream) {
+    NvtxRange nvtx_range("tg_gated_attention_noalloc");
     TG_REQUIRE(B >= 0 && M_total >= 0 && max_M >= 0, "negative size");
     if (tg_status s = check_attn_shape(Hq, Hkv, d)) return s;
     TG_REQUIRE(sm_scale > 0.f, "sm_scale must be positive");
@@ -339,6 +358,7 @@ tg_status tg_gated_attention(const uint16_t* q, const uint16_t* k, const uint16_
                              int64_t M_total, int max_M, int Hq, int Hkv, int d, const int32_t* pos,
                              const int32_t* rank, const float* gls, const float* g, const float* c, float sm_scale,
                              uint16_t* out, float* lse, void* ws, size_t ws_bytes, tg_stream_t stream) {
+    NvtxRange nvtx_range("tg_gated_attention");
     tg::GateSet gates = tg::single_gate(gls, g);
     if (!gls && !g && !c) gates.n = 0;  // no gate: ordinary causal attention
     return do_attention(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, d, pos, rank, gates, c, sm_scale, out, lse, ws,
@@ -350,6 +370,7 @@ tg_status tg_gated_attention_gates(const uint16_t* q, const uint16_t* k, const u
                                    const int32_t* rank, int n_gates, const float* const* gls, const float* const* g,
                                    const float* c, float sm_scale, uint16_t* out, float* lse, void* ws,
                                    size_t ws_bytes, tg_stream_t stream) {
+    NvtxRange nvtx_range("tg_gated_attention_gates");
     TG_SUPPORT(n_gates >= 1 && n_gates <= tg::kMaxGates, "n_gates=%d must be in [1, %d]", n_gates, tg::kMaxGates);
     TG_REQUIRE(gls && g, "null gate arrays");
     tg::GateSet gates{};
@@ -374,6 +395,7 @@ tg_status tg_gated_attention_backward(const uint16_t* q, const uint16_t* k, cons
                                       float sm_scale, uint16_t* dq, uint16_t* dk, uint16_t* dv, float* dgls,
                                       float* dscore, float* dg, float* dc, void* ws, size_t ws_bytes,
                                       tg_stream_t stream) {
+    NvtxRange nvtx_range("tg_gated_attention_backward");
     TG_REQUIRE(B >= 0 && M_total >= 0 && max_M >= 0, "negative size");
     if (tg_status s = check_attn_shape(Hq, Hkv, d)) return s;
     TG_SUPPORT(d == 64 || d == 128, "the backward supports head_dim 64 and 128, not %d", d);
@@ -428,7 +450,16 @@ tg_status tg_selftest_bounded_wait(int64_t timeout_ns, tg_stream_t stream) {
     return cuda_status(tg::launch_selftest_wait(timeout_ns, stream), "tg_selftest_bounded_wait launch");
 }
 
+tg_status tg_selftest_exp2(const float* x, float* y, int64_t n, tg_stream_t stream) {
+    TG_REQUIRE(n >= 0, "negative n");
+    if (n == 0) return TG_OK;
+    TG_REQUIRE(x && y, "null pointer argument");
+    if (tg_status s = check_device()) return s;
+    return cuda_status(tg::launch_exp2_poly_selftest(x, y, n, stream), "tg_selftest_exp2 launch");
+}
+
 tg_status tg_gated_prefill_layer(const tg_prefill_layer_args* a, tg_stream_t stream) {
+    NvtxRange nvtx_range("tg_gated_prefill_layer");
     TG_REQUIRE(a != nullptr, "null args");
     TG_REQUIRE(a->B >= 0 && a->T >= 0 && a->M_total >= 0 && a->M_total <= a->T && a->n_layers >= 0, "bad sizes");
     if (tg_status s = check_gate_shape(a->D, a->I)) return s;

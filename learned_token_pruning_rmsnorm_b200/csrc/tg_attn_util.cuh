@@ -59,6 +59,33 @@ __device__ __forceinline__ uint64_t f32x2_add(uint64_t a, uint64_t b) {
     return d;
 }
 
+// 2^x of a pair of fp32 values on the FMA pipe, to share the exponentials of the softmax
+// with the special-function unit.  Cody-Waite style range reduction: adding and removing
+// 1.5 * 2^23 rounds x to an integer n (exactly, for |x| < 2^22), f = x - n lies in
+// [-0.5, 0.5]; 2^f comes from a degree-3 polynomial whose coefficients were fitted for this
+// library (Lawson's iteratively reweighted least squares towards the minimax relative
+// error over [-0.5, 0.5]: 7.5e-5 at most, evaluated in fp32), and 2^n is added into the
+// exponent field.  Inputs are clamped to >= -126 first (below that the result is a tiny
+// number of at most 2^-126 instead of 0; the softmax only passes x <= 0 and sends its
+// masked elements to the special-function unit).
+constexpr float EXP2_C0 = 0.9999280571937561f;
+constexpr float EXP2_C1 = 0.6932609677314758f;
+constexpr float EXP2_C2 = 0.24261116981506348f;
+constexpr float EXP2_C3 = 0.05517167970538139f;
+__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x2) {
+    const uint64_t xc = f32x2_pack(fmaxf(f32x2_lo(x2), -126.0f), fmaxf(f32x2_hi(x2), -126.0f));
+    const uint64_t j = f32x2_add(xc, f32x2_pack(12582912.0f, 12582912.0f));  // 1.5 * 2^23 + round(x)
+    const uint64_t n = f32x2_add(j, f32x2_pack(-12582912.0f, -12582912.0f));
+    const uint64_t f = f32x2_fma(n, f32x2_pack(-1.0f, -1.0f), xc);
+    uint64_t p = f32x2_fma(f, f32x2_pack(EXP2_C3, EXP2_C3), f32x2_pack(EXP2_C2, EXP2_C2));
+    p = f32x2_fma(p, f, f32x2_pack(EXP2_C1, EXP2_C1));
+    p = f32x2_fma(p, f, f32x2_pack(EXP2_C0, EXP2_C0));
+    // the low bits of j hold n (two's complement): n << 23 moves it into the exponent field
+    const uint32_t r0 = static_cast<uint32_t>(p) + (static_cast<uint32_t>(j) << 23);
+    const uint32_t r1 = static_cast<uint32_t>(p >> 32) + (static_cast<uint32_t>(j >> 32) << 23);
+    return static_cast<uint64_t>(r0) | (static_cast<uint64_t>(r1) << 32);
+}
+
 // Named barrier `id` over `n` threads that also returns the OR of `pred` over them.
 __device__ __forceinline__ bool bar_red_or(int id, int n, bool pred) {
     uint32_t res;

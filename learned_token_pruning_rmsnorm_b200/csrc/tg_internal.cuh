@@ -181,6 +181,9 @@ int64_t units_below_host(int x, int C);
 
 cudaError_t launch_selftest_wait(int64_t timeout_ns, cudaStream_t st);
 
+// y[i] = the attention softmax's FMA-pipe 2^x (exp2_poly_x2) of x[i], device arrays of n floats.
+cudaError_t launch_exp2_poly_selftest(const float* x, float* y, int64_t n, cudaStream_t st);
+
 cudaError_t read_device_status(int32_t* word, bool clear, cudaStream_t st);
 
 }  // namespace tg
