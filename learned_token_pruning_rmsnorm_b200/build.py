@@ -29,6 +29,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libtokengate.so")
+LIB_DEBUG = os.path.join(PKG, "libtokengate_debug.so")  # the TG_DEBUG variant (index checks)
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
@@ -62,12 +63,16 @@ def _stale(target: str, deps) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
+def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False, debug: bool | None = None) -> str:
+    """Build libtokengate.so (or, with debug / TG_DEBUG=1, libtokengate_debug.so) and
+    return its path."""
     nvcc = _nvcc()
-    # objects of the checking variant live apart, so that switching variants rebuilds
-    build_dir = BUILD + ("_debug" if _debug() else "")
+    debug = _debug() if debug is None else debug
+    # the checking variant has objects and a library of its own
+    build_dir = BUILD + ("_debug" if debug else "")
+    lib_path = LIB_DEBUG if debug else LIB
     os.makedirs(build_dir, exist_ok=True)
-    flags = NVCC_FLAGS + (["-DTG_DEBUG=1"] if _debug() else [])
+    flags = NVCC_FLAGS + (["-DTG_DEBUG=1"] if debug else [])
     srcs = _sources()
     hdrs = _headers()
     objs = []
@@ -94,14 +99,13 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
     if jobs:
         with ThreadPoolExecutor(max_workers=min(8, len(jobs))) as ex:
             list(ex.map(run, jobs))
-    if force or jobs or _stale(LIB, objs + [EXPORTS]):
-        tmp = LIB + f".tmp{os.getpid()}"
+    if force or jobs or _stale(lib_path, objs + [EXPORTS]):
+        tmp = lib_path + f".tmp{os.getpid()}"
         run([nvcc, *ARCH, "-shared", "-Xcompiler", "-fPIC", "-Xlinker", f"--version-script={EXPORTS}", "-o", tmp,
              *objs])
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib_path)
+    return lib_path
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose="-v" in sys.argv, ptxas_info="--ptxas" in sys.argv)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, ptxas_info="--ptxas" in sys.argv))

@@ -1136,9 +1136,9 @@ cudaError_t launch_tc(const uint16_t* q, const uint16_t* k, const uint16_t* v, c
         if ((Hq / Hkv) % 2 == 0) {
             // the persistent kernel needs the workspace for its unit counter
             if (ws != nullptr) {
-                const cudaError_t e = launch_attention_persistent(tq, tk, tv, cu_kept, B, max_M, Hq, Hkv, HD, pos,
-                                                                  rank, gates, c, sm_scale, out, lse, ws, ws_bytes,
-                                                                  early, st);
+                const cudaError_t e = launch_attention_persistent(tq, tk, tv, cu_kept, B, M_total, max_M, Hq, Hkv,
+                                                                  HD, pos, rank, gates, c, sm_scale, out, lse, ws,
+                                                                  ws_bytes, early, st);
                 if (e != cudaErrorNotSupported || gates.n == 0) return e;
             }
             if (gates.n == 0) return cudaErrorNotSupported;

@@ -92,8 +92,10 @@ struct Unit {
 // with fewer units than the longest).  Numbering: u = (v * B + b) * pairs + pair, v the
 // unit's place in its sequence's decreasing-cost order, so all sequences' heaviest
 // units come first.
+// In TG_DEBUG builds a sequence whose rows [cu_kept[b], cu_kept[b+1]) do not lie inside
+// [0, M_total) is recorded in the status word and skipped (every role decodes the same way).
 __device__ __forceinline__ bool decode_unit(int64_t u, int pairs, int B, const int32_t* cu_kept, int C_all,
-                                            Unit* U) {
+                                            Unit* U, int64_t M_total, int* status) {
     const int pair = static_cast<int>(u % pairs);
     const int64_t t = u / pairs;
     const int b = static_cast<int>(t % B);
@@ -102,6 +104,8 @@ __device__ __forceinline__ bool decode_unit(int64_t u, int pairs, int B, const i
     const int Mb = cu_kept[b + 1] - seq0;
     const int n_qt = (Mb + BM - 1) / BM;
     if (n_qt <= 0) return false;
+    if (!TG_DEBUG_CHECK(seq0 >= 0 && static_cast<int64_t>(seq0) + Mb <= M_total, status, TG_WHERE_ATTENTION))
+        return false;
     const int C = min(C_all, n_qt);
     if (v >= units_below(n_qt, C)) return false;
     int qt, chunk;
@@ -141,8 +145,8 @@ __global__ void __launch_bounds__(PT_THREADS, 1)
 gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const int32_t* __restrict__ cu_kept,
                        const int32_t* __restrict__ pos, const int32_t* __restrict__ rank, const GateSet gates,
-                       const float* __restrict__ c, float sm_scale, int Hq, int Hkv, int B, int kv_chunk,
-                       int64_t total_units, SplitWs ws,
+                       const float* __restrict__ c, float sm_scale, int Hq, int Hkv, int B, int64_t M_total,
+                       int kv_chunk, int64_t total_units, SplitWs ws,
                        int* __restrict__ sched, uint16_t* __restrict__ out, float* __restrict__ lse,
                        int* __restrict__ status, int early) {
     using L = PtSmem<HD>;
@@ -237,7 +241,7 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             Unit U{};
             bool have = false;
             while (unit < total_units) {
-                if (decode_unit(unit, pairs, B, cu_kept, kv_chunk, &U)) {
+                if (decode_unit(unit, pairs, B, cu_kept, kv_chunk, &U, M_total, status)) {
                     have = true;
                     break;
                 }
@@ -415,7 +419,7 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 const int unit = ring[uc % PT_RING];
                 if (unit < 0) break;
                 Unit U{};
-                decode_unit(unit, pairs, B, cu_kept, kv_chunk, &U);
+                decode_unit(unit, pairs, B, cu_kept, kv_chunk, &U, M_total, status);
                 ok = mbar_wait(bar(T_Q_FULL), uc & 1, abort_flag, status, TG_WHERE_MMA);
                 PT_STAMP(3, uc == 0);
                 ok = ok && mbar_wait(bar(T_K_FULL + (t & 1)), (t >> 1) & 1, abort_flag, status, TG_WHERE_MMA);
@@ -496,7 +500,7 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             if (unit < 0) break;
             bool ok = true;
             Unit U{};
-            decode_unit(unit, pairs, B, cu_kept, kv_chunk, &U);
+            decode_unit(unit, pairs, B, cu_kept, kv_chunk, &U, M_total, status);
             const int q_local = U.qt * BM + r;
             const bool valid_row = q_local < U.Mb;
             const int64_t qg = static_cast<int64_t>(U.seq0) + q_local;
@@ -784,7 +788,8 @@ static int pers_launch_regs() {
 
 template <int HD, bool GATED>
 static cudaError_t launch_pers_impl(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                                    const int32_t* cu_kept, int B, int max_M, int Hq, int Hkv, const int32_t* pos,
+                                    const int32_t* cu_kept, int B, int64_t M_total, int max_M, int Hq, int Hkv,
+                                    const int32_t* pos,
                                     const int32_t* rank, const GateSet& gates, const float* c, float sm_scale,
                                     uint16_t* out, float* lse, void* ws, size_t ws_bytes, bool early,
                                     cudaStream_t st) {
@@ -812,25 +817,25 @@ static cudaError_t launch_pers_impl(const CUtensorMap& tq, const CUtensorMap& tk
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const unsigned grid = static_cast<unsigned>(total < sms ? total : sms);
     return launch_pdl(gated_attn_pers_kernel<HD, GATED>, dim3(grid), dim3(PT_THREADS), static_cast<size_t>(L::ALLOC),
-                      st, tq, tk, tv, cu_kept, pos, rank, gates, c, sm_scale, Hq, Hkv, B, lay.C, total, sw,
+                      st, tq, tk, tv, cu_kept, pos, rank, gates, c, sm_scale, Hq, Hkv, B, M_total, lay.C, total, sw,
                       reinterpret_cast<int*>(base), out, lse, device_status_ptr(), early ? 1 : 0);
 }
 
 cudaError_t launch_attention_persistent(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                                        const int32_t* cu_kept, int B, int max_M, int Hq, int Hkv, int d,
-                                        const int32_t* pos, const int32_t* rank, const GateSet& gates, const float* c,
-                                        float sm_scale, uint16_t* out, float* lse, void* ws, size_t ws_bytes,
-                                        bool early, cudaStream_t st) {
+                                        const int32_t* cu_kept, int B, int64_t M_total, int max_M, int Hq,
+                                        int Hkv, int d, const int32_t* pos, const int32_t* rank,
+                                        const GateSet& gates, const float* c, float sm_scale, uint16_t* out,
+                                        float* lse, void* ws, size_t ws_bytes, bool early, cudaStream_t st) {
     const bool gated = gates.n > 0;
     if (d == 64)
-        return gated ? launch_pers_impl<64, true>(tq, tk, tv, cu_kept, B, max_M, Hq, Hkv, pos, rank, gates, c,
+        return gated ? launch_pers_impl<64, true>(tq, tk, tv, cu_kept, B, M_total, max_M, Hq, Hkv, pos, rank, gates, c,
                                                   sm_scale, out, lse, ws, ws_bytes, early, st)
-                     : launch_pers_impl<64, false>(tq, tk, tv, cu_kept, B, max_M, Hq, Hkv, pos, rank, gates, c,
+                     : launch_pers_impl<64, false>(tq, tk, tv, cu_kept, B, M_total, max_M, Hq, Hkv, pos, rank, gates, c,
                                                    sm_scale, out, lse, ws, ws_bytes, early, st);
     if (d == 128)
-        return gated ? launch_pers_impl<128, true>(tq, tk, tv, cu_kept, B, max_M, Hq, Hkv, pos, rank, gates, c,
+        return gated ? launch_pers_impl<128, true>(tq, tk, tv, cu_kept, B, M_total, max_M, Hq, Hkv, pos, rank, gates, c,
                                                    sm_scale, out, lse, ws, ws_bytes, early, st)
-                     : launch_pers_impl<128, false>(tq, tk, tv, cu_kept, B, max_M, Hq, Hkv, pos, rank, gates, c,
+                     : launch_pers_impl<128, false>(tq, tk, tv, cu_kept, B, M_total, max_M, Hq, Hkv, pos, rank, gates, c,
                                                     sm_scale, out, lse, ws, ws_bytes, early, st);
     return cudaErrorNotSupported;
 }

@@ -108,7 +108,7 @@ __global__ void __launch_bounds__(ScoreCfg<NACC>::THREADS, 1)
 score_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                 const int32_t* __restrict__ cu_seqlens, const int32_t* __restrict__ span, int B, int D, int I,
                 const float* __restrict__ b1, const float* __restrict__ w2, float b2, float eps,
-                float* __restrict__ scores, int* __restrict__ status) {
+                float* __restrict__ scores, int64_t T, int* __restrict__ status) {
     using C = ScoreCfg<NACC>;
     constexpr int STAGES = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
@@ -298,7 +298,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
             __syncwarp();
             if (lane == 0) mbar_arrive(acc_empty);
             const int64_t row = row0 + a * 128 + r;
-            if (row < row_end) scores[row] = acc_s + b2;
+            if (row < row_end && TG_DEBUG_CHECK(row >= 0 && row < T, status, TG_WHERE_SCORE)) scores[row] = acc_s + b2;
         }
     }
 
@@ -329,7 +329,7 @@ cudaError_t launch_score_tc(const uint16_t* hidden, const int32_t* cu_seqlens, c
     const int grid = static_cast<int>(tiles_bound < sms ? tiles_bound : sms);
     const cudaError_t le = launch_pdl(score_tc_kernel<NACC>, dim3(grid), dim3(C::THREADS),
                                       static_cast<size_t>(score_smem_bytes<NACC>(I)), st, tx, tw, cu_seqlens, span, B,
-                                      D, I, b1, w2, b2, eps, scores, device_status_ptr());
+                                      D, I, b1, w2, b2, eps, scores, T, device_status_ptr());
     if (le != cudaSuccess) return le;
     return cudaGetLastError();
 }

@@ -441,6 +441,9 @@ tg_status tg_device_status(int32_t* h_word, int clear, tg_stream_t stream) {
     if (tg_status s = cuda_status(tg::read_device_status(&w, clear != 0, stream), "tg_device_status")) return s;
     if (h_word) *h_word = w;
     if (w & tg::TG_DEVICE_TIMEOUT) return fail(TG_ERR_TIMEOUT, "a bounded device wait gave up (status word 0x%x)", w);
+    if (w & tg::TG_DEVICE_BAD_INDEX)
+        return fail(TG_ERR_INVALID_ARG, "a kernel found an input-derived index outside its array (status word 0x%x)",
+                    w);
     return TG_OK;
 }
 

@@ -191,8 +191,8 @@ attn::AttnWsLayout attention_ws_layout(int B, int max_M, int Hq, int Hkv, int d)
 // Needs the workspace (its unit counter); returns cudaErrorNotSupported when it cannot
 // run on this build or device, so that the caller can fall back.
 cudaError_t launch_attention_persistent(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                                        const int32_t* cu_kept, int B, int max_M, int Hq, int Hkv, int d,
-                                        const int32_t* pos, const int32_t* rank, const GateSet& gates, const float* c,
-                                        float sm_scale, uint16_t* out, float* lse, void* ws, size_t ws_bytes,
-                                        bool early, cudaStream_t st);
+                                        const int32_t* cu_kept, int B, int64_t M_total, int max_M, int Hq,
+                                        int Hkv, int d, const int32_t* pos, const int32_t* rank,
+                                        const GateSet& gates, const float* c, float sm_scale, uint16_t* out,
+                                        float* lse, void* ws, size_t ws_bytes, bool early, cudaStream_t st);
 }  // namespace tg

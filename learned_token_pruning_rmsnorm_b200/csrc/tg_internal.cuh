@@ -79,6 +79,20 @@ constexpr int TG_WHERE_PRODUCER = 1 << 0;    // ... in the TMA producer
 constexpr int TG_WHERE_MMA = 1 << 1;         // ... in the MMA issuer
 constexpr int TG_WHERE_SOFTMAX = 1 << 2;     // ... in the softmax / epilogue warps
 constexpr int TG_WHERE_DRAIN = 1 << 3;       // ... while draining after an abort
+constexpr int TG_DEVICE_BAD_INDEX = 1 << 17;  // (TG_DEBUG builds) an index derived from the inputs
+                                              // fell outside its array; the access was skipped
+constexpr int TG_WHERE_ATTENTION = 1 << 4;    // ... in an attention kernel (cu_kept vs M_total)
+constexpr int TG_WHERE_SCORE = 1 << 5;        // ... in the score kernel (cu_seqlens / span vs T)
+
+// TG_DEBUG builds: evaluate `cond` (an index bound derived from the caller's inputs); when
+// it fails, record TG_DEVICE_BAD_INDEX | where in the status word and yield false, so that
+// the caller skips the access.  Release builds trust the documented contract: always true.
+#ifdef TG_DEBUG
+#define TG_DEBUG_CHECK(cond, status, where) \
+    ((cond) ? true : ((status) ? (atomicOr((status), ::tg::TG_DEVICE_BAD_INDEX | (where)), false) : false))
+#else
+#define TG_DEBUG_CHECK(cond, status, where) true
+#endif
 
 // ------------------------------------------------------------------ device helpers
 
