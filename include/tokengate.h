@@ -423,7 +423,7 @@ tg_status tg_selftest_bounded_wait(int64_t timeout_ns, tg_stream_t stream);
  * exponential (the share of the softmax's exponentials that does not go to
  * the special-function unit): Cody-Waite range reduction to f in [-0.5, 0.5]
  * and a degree-3 polynomial fitted for this library (relative error at most
- * 7.5e-5 for -126 <= x <= 0; x below -126 is clamped to -126).  x, y are
+ * 7.5e-5 for -125 <= x <= 0; x below -125 is clamped to -125).  x, y are
  * device arrays of n floats.  Used to test that exponential against exp2.
  */
 tg_status tg_selftest_exp2(const float* x, float* y, int64_t n, tg_stream_t stream);

@@ -1217,7 +1217,10 @@ int attention_kv_chunk(int B, int max_M, int Hq, int Hkv, bool have_ws) {
         const auto it = memo.find(key);
         if (it != memo.end()) return it->second;
     }
-    constexpr double F = 3.1;
+#ifndef TG_LPT_FIXED_COST
+#define TG_LPT_FIXED_COST 3.1
+#endif
+    constexpr double F = TG_LPT_FIXED_COST;
     int best_c = n_qt;
     double best = 1e300;
     std::vector<double> cost;

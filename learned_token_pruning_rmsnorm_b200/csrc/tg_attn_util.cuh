@@ -65,15 +65,15 @@ __device__ __forceinline__ uint64_t f32x2_add(uint64_t a, uint64_t b) {
 // [-0.5, 0.5]; 2^f comes from a degree-3 polynomial whose coefficients were fitted for this
 // library (Lawson's iteratively reweighted least squares towards the minimax relative
 // error over [-0.5, 0.5]: 7.5e-5 at most, evaluated in fp32), and 2^n is added into the
-// exponent field.  Inputs are clamped to >= -126 first (below that the result is a tiny
-// number of at most 2^-126 instead of 0; the softmax only passes x <= 0 and sends its
-// masked elements to the special-function unit).
+// exponent field.  Inputs are clamped to >= -125 first, so that the result stays a normal
+// number (below that it is a tiny number of at most 2^-124 instead of 0; the softmax only
+// passes x <= 0 and sends its masked elements to the special-function unit).
 constexpr float EXP2_C0 = 0.9999280571937561f;
 constexpr float EXP2_C1 = 0.6932609677314758f;
 constexpr float EXP2_C2 = 0.24261116981506348f;
 constexpr float EXP2_C3 = 0.05517167970538139f;
 __device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x2) {
-    const uint64_t xc = f32x2_pack(fmaxf(f32x2_lo(x2), -126.0f), fmaxf(f32x2_hi(x2), -126.0f));
+    const uint64_t xc = f32x2_pack(fmaxf(f32x2_lo(x2), -125.0f), fmaxf(f32x2_hi(x2), -125.0f));
     const uint64_t j = f32x2_add(xc, f32x2_pack(12582912.0f, 12582912.0f));  // 1.5 * 2^23 + round(x)
     const uint64_t n = f32x2_add(j, f32x2_pack(-12582912.0f, -12582912.0f));
     const uint64_t f = f32x2_fma(n, f32x2_pack(-1.0f, -1.0f), xc);
