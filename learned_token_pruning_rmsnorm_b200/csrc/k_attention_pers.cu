@@ -51,7 +51,7 @@ constexpr int PT_RING = 8;            // unit numbers in flight between the prod
 // FMA pipe (exp2_poly_x2) instead of the special-function unit, except in the diagonal tile,
 // whose masked elements must come out exactly 0.
 #ifndef TG_EXP2_POLY_QUADS
-#define TG_EXP2_POLY_QUADS 3
+#define TG_EXP2_POLY_QUADS 0
 #endif
 constexpr int PT_POLY_QUADS = TG_EXP2_POLY_QUADS;
 static_assert(PT_POLY_QUADS >= 0 && PT_POLY_QUADS <= 8, "quads of 4 columns per 32");
@@ -129,6 +129,11 @@ __device__ __forceinline__ void named_bar_sync(int id, int n) {
 // Optional device trace (builds with -DTG_TRACE only): per-CTA globaltimer stamps of the
 // hand-offs of the first unit and of the whole CTA, with the SM id and the unit count.
 #ifdef TG_TRACE
+__device__ unsigned long long g_pers_pipe[16 * 64];  // clock64 of pipeline points of CTA 0, first 64 tiles
+#define PT_PIPE(point, j)                                                                      \
+    do {                                                                                       \
+        if (blockIdx.x == 0 && (j) < 64) g_pers_pipe[(point) * 64 + (j)] = clock64();         \
+    } while (0)
 __device__ unsigned long long g_pers_trace[1024 * 16];
 #define PT_STAMP(slot, cond)                                                             \
     do {                                                                                 \
@@ -137,6 +142,9 @@ __device__ unsigned long long g_pers_trace[1024 * 16];
 #else
 #define PT_STAMP(slot, cond) \
     do {                     \
+    } while (0)
+#define PT_PIPE(point, j) \
+    do {                  \
     } while (0)
 #endif
 
@@ -389,27 +397,33 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, HD, true);
+            // Matrix descriptors are built once; a k-step's operand is the same descriptor with
+            // its byte offset / 16 added to the start-address field (the offsets stay inside
+            // shared memory, so the 14-bit field never carries).  One thread issues every MMA,
+            // and building each descriptor from scratch would slow it below the tensor pipe.
+            const uint64_t qdesc[2] = {smem_desc_sw128(sQ, 16, 1024), smem_desc_sw128(sQ + L::TILE_Q, 16, 1024)};
+            const uint64_t kdesc[2] = {smem_desc_sw128(sK0, 16, 1024), smem_desc_sw128(sK0 + L::TILE_KV, 16, 1024)};
+            const uint64_t vdesc[2] = {smem_desc_sw128(sV0, BN * 128, 1024),
+                                       smem_desc_sw128(sV0 + L::TILE_KV, BN * 128, 1024)};
+            const uint64_t qxdesc = smem_desc_noswz(sQX, 128, 256), kxdesc = smem_desc_noswz(sKX, 128, 256);
             auto issue_s = [&](int hh, int s) {
-                const uint32_t kb = sK0 + s * L::TILE_KV;
-                const uint32_t qb = sQ + hh * L::TILE_Q;
+                const uint64_t qd = qdesc[hh], kd = kdesc[s];
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk) {
                     const uint32_t off_q = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
                     const uint32_t off_k = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
-                    mma_bf16_ss(tmem + hh * BN, smem_desc_sw128(qb + off_q, 16, 1024),
-                                smem_desc_sw128(kb + off_k, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+                    mma_bf16_ss(tmem + hh * BN, qd + (off_q >> 4), kd + (off_k >> 4), idesc_qk, kk > 0 ? 1u : 0u);
                 }
                 if (GATED)  // + bscale_h * gls_j: the bias k-step (no-swizzle tiles, K cores 128 B apart)
-                    mma_bf16_ss(tmem + hh * BN, smem_desc_noswz(sQX + hh * L::EXT, 128, 256),
-                                smem_desc_noswz(sKX + s * L::EXT, 128, 256), idesc_qk, 1u);
+                    mma_bf16_ss(tmem + hh * BN, qxdesc + ((hh * L::EXT) >> 4), kxdesc + ((s * L::EXT) >> 4), idesc_qk,
+                                1u);
             };
             auto issue_pv = [&](int hh, int s, bool acc) {
-                const uint32_t vb = sV0 + s * L::TILE_KV;
+                const uint64_t vd = vdesc[s];
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk)
-                    mma_bf16_ts(tmem + 2 * BN + hh * HD, tmem + hh * BN + kk * 8,
-                                smem_desc_sw128(vb + kk * 16 * 128, BN * 128, 1024), idesc_pv,
-                                (acc || kk > 0) ? 1u : 0u);
+                    mma_bf16_ts(tmem + 2 * BN + hh * HD, tmem + hh * BN + kk * 8, vd + ((kk * 16 * 128) >> 4),
+                                idesc_pv, (acc || kk > 0) ? 1u : 0u);
             };
             int uc = 0, t = 0, it = 0;
             bool ok = true;
@@ -441,11 +455,13 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                          mbar_wait(bar(T_P_FULL + 0), it & 1, abort_flag, status, TG_WHERE_MMA);
                     if (!ok) break;
                     tc_fence_after();
+                    PT_PIPE(0, it);
                     issue_pv(0, s, j > 0);
                     if (more) {
                         ok = mbar_wait(bar(T_K_FULL + (s ^ 1)), ((t + 1) >> 1) & 1, abort_flag, status, TG_WHERE_MMA);
                         if (!ok) break;
                         tc_fence_after();
+                        PT_PIPE(2, it);
                         issue_s(0, s ^ 1);
                         mma_commit(bar(T_S_FULL + 0));
                     } else {
@@ -454,6 +470,7 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     ok = mbar_wait(bar(T_P_FULL + 1), it & 1, abort_flag, status, TG_WHERE_MMA);
                     if (!ok) break;
                     tc_fence_after();
+                    PT_PIPE(1, it);
                     issue_pv(1, s, j > 0);
                     mma_commit(bar(T_V_EMPTY + s));
                     if (more) {
@@ -531,11 +548,13 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     break;
                 }
                 PT_STAMP(5, uc == 0 && j == 0 && threadIdx.x == 0);
+                if (r == 0) PT_PIPE(4 + h, it);
                 tc_fence_after();
                 float x[BN];
 #pragma unroll
                 for (int cc = 0; cc < BN / 32; ++cc) tmem_ld32(tS + cc * 32, x + cc * 32);
                 tmem_wait_ld();
+                if (r == 0) PT_PIPE(6 + h, it);
                 if (jt == U.qt) {
                     const int lim = q_local - jt * BN;  // keys with column > lim lie in the causal future
 #pragma unroll
@@ -556,6 +575,7 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     rescale_o = j > 0;
                 }
                 const uint64_t nm2 = f32x2_pack(-m_run, -m_run);
+                if (r == 0) PT_PIPE(8 + h, it);
                 const bool poly_ok = jt != U.qt;  // no masked element in this tile
                 uint64_t sp[4] = {0ull, 0ull, 0ull, 0ull};
                 // P row r as bf16 pairs over the first 64 columns of S_h (the A operand of the
@@ -602,6 +622,7 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();  // every lane's P and O stores are complete and fenced
+                if (r == 0) PT_PIPE(10 + h, it);
                 if (lane == 0) mbar_arrive(bar(T_P_FULL + h));
             }
             // ---------------------------------------------------------------- epilogue
@@ -774,6 +795,9 @@ cudaError_t launch_exp2_poly_selftest(const float* x, float* y, int64_t n, cudaS
 #ifdef TG_TRACE
 extern "C" __attribute__((visibility("default"))) int tg_trace_read_attention_pers(unsigned long long* host) {
     return cudaMemcpyFromSymbol(host, g_pers_trace, sizeof(g_pers_trace)) == cudaSuccess ? 0 : 1;
+}
+extern "C" __attribute__((visibility("default"))) int tg_trace_read_attention_pers_pipe(unsigned long long* host) {
+    return cudaMemcpyFromSymbol(host, g_pers_pipe, sizeof(g_pers_pipe)) == cudaSuccess ? 0 : 1;
 }
 #endif
 

@@ -214,13 +214,16 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                     }
                     tc_fence_after();
                     SC_TRACE(1, it);
+                    // one descriptor per operand of the stage; a k-step adds its byte offset / 16
+                    // to the start-address field (no carry: offsets stay inside shared memory)
                     const uint32_t st = sbase + s * stage_bytes;
+                    const uint64_t bdesc0 = smem_desc_sw128(st + NACC * TILE_A, 16, 1024);
+                    const uint64_t adesc0 = smem_desc_sw128(st, 16, 1024);
 #pragma unroll
                     for (int kk = 0; kk < KB / 16; ++kk) {
-                        const uint64_t bdesc = smem_desc_sw128(st + NACC * TILE_A + kk * 32, 16, 1024);
 #pragma unroll
                         for (int a = 0; a < NACC; ++a)
-                            mma_bf16_ss(tmem + a * 256, smem_desc_sw128(st + a * TILE_A + kk * 32, 16, 1024), bdesc,
+                            mma_bf16_ss(tmem + a * 256, adesc0 + ((a * TILE_A + kk * 32) >> 4), bdesc0 + ((kk * 32) >> 4),
                                         idesc, (kb | kk) != 0 ? 1u : 0u);
                     }
                     mma_commit(empty(s));
