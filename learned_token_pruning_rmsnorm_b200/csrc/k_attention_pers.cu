@@ -25,11 +25,10 @@
 //   warp 8      TMA producer: Q of both heads once per unit, K/V tiles of 128
 //               keys through a two-stage ring, the gate-bias operand rows, the
 //               next unit's number
-//   warps 9, 10 MMA issuers, one thread each, warp 9 + h for head h:
-//               S_h(0) | PV_h(0) S_h(1) | PV_h(1) S_h(2) | ...   (P_h is read
-//               from TMEM, written by the softmax as bf16 over the first 64
-//               columns of S_h)
-//   warp 11     idle (it completes the producer/MMA warpgroup, whose
+//   warp 9      MMA issuer (one thread):  S0(j) S1(j) | PV0(j) S0(j+1) |
+//               PV1(j) S1(j+1) | ...   (P_h is read from TMEM, written by the
+//               softmax as bf16 over the first 64 columns of S_h)
+//   warps 10-11 idle (they complete the producer/MMA warpgroup, whose
 //               registers are handed to the softmax warpgroups)
 // TMEM (512 columns): S0 | S1 | O0 | O1.  Each head's epilogue reads its O
 // from TMEM and writes its rows while the other head still computes and the
@@ -81,7 +80,7 @@ enum : int {
     T_Q_FULL = 0, T_Q_EMPTY = 1, T_K_FULL = 2, T_K_EMPTY = 4, T_V_FULL = 6, T_V_EMPTY = 8, T_S_FULL = 10,
     T_P_FULL = 12, T_O_FULL = 14, T_UNIT = 16, T_DRAIN = 16 + PT_RING
 };
-static_assert(T_DRAIN + 1 < PtSmem<128>::NUM_BARS, "barrier slots");
+static_assert(T_DRAIN < PtSmem<128>::NUM_BARS, "barrier slots");
 
 // One unit of work: (sequence b, head pair, query tile, KV chunk).
 struct Unit {
@@ -196,19 +195,18 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     }
     if (threadIdx.x == 0) {
         mbar_init(bar(T_Q_FULL), GATED ? 2 : 1);  // the Q bytes (+ the producer's bias operand rows)
-        mbar_init(bar(T_Q_EMPTY), 2);  // both MMA issuers
+        mbar_init(bar(T_Q_EMPTY), 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(bar(T_K_FULL + s), GATED ? 2 : 1);  // the K bytes (+ the K_ext rows)
-            mbar_init(bar(T_K_EMPTY + s), 2);  // both MMA issuers
+            mbar_init(bar(T_K_EMPTY + s), 1);
             mbar_init(bar(T_V_FULL + s), 1);
-            mbar_init(bar(T_V_EMPTY + s), 2);
+            mbar_init(bar(T_V_EMPTY + s), 1);
             mbar_init(bar(T_S_FULL + s), 1);
             mbar_init(bar(T_P_FULL + s), 4);  // one arrival per softmax warp of the head
             mbar_init(bar(T_O_FULL + s), 1);
         }
         for (int i = 0; i < PT_RING; ++i) mbar_init(bar(T_UNIT + i), 1);
-        mbar_init(bar(T_DRAIN + 0), 1);
-        mbar_init(bar(T_DRAIN + 1), 1);
+        mbar_init(bar(T_DRAIN), 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -394,43 +392,38 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 if (v_issued[s]) drain_wait(bar(T_V_FULL + s), (v_issued[s] - 1) & 1, status);
             }
         }
-    } else if (warp == 9 || warp == 10) {
-        // ---------------------------------------------------------------- MMA issuers
-        // Warp 9 issues head 0's products, warp 10 head 1's: one thread issues a tcgen05.mma
-        // only every ~100 cycles, more slowly than the tensor pipe runs a 128 x 128 x 16
-        // product, so two issuers keep it busier.  Each head's S_h(j+1) follows PV_h(j) from the
-        // same thread (tcgen05 operations of one thread execute in order), and the stage and
-        // Q releases count both issuers' commits.
-        const int hh = warp - 9;
+    } else if (warp == 9) {
+        // ---------------------------------------------------------------- MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, HD, true);
             // Matrix descriptors are built once; a k-step's operand is the same descriptor with
             // its byte offset / 16 added to the start-address field (the offsets stay inside
-            // shared memory, so the 14-bit field never carries).
-            const uint64_t qdesc = smem_desc_sw128(sQ + hh * L::TILE_Q, 16, 1024);
-            const uint64_t kdesc0 = smem_desc_sw128(sK0, 16, 1024), kdesc1 = smem_desc_sw128(sK0 + L::TILE_KV, 16, 1024);
-            const uint64_t vdesc0 = smem_desc_sw128(sV0, BN * 128, 1024);
-            const uint64_t vdesc1 = smem_desc_sw128(sV0 + L::TILE_KV, BN * 128, 1024);
-            const uint64_t qxdesc = smem_desc_noswz(sQX + hh * L::EXT, 128, 256);
-            const uint64_t kxdesc = smem_desc_noswz(sKX, 128, 256);
-            const uint32_t tS = tmem + hh * BN, tO = tmem + 2 * BN + hh * HD;
-            auto issue_s = [&](int s) {
-                const uint64_t kd = s ? kdesc1 : kdesc0;
+            // shared memory, so the 14-bit field never carries).  One thread issues every MMA,
+            // and building each descriptor from scratch would slow it below the tensor pipe.
+            const uint64_t qdesc[2] = {smem_desc_sw128(sQ, 16, 1024), smem_desc_sw128(sQ + L::TILE_Q, 16, 1024)};
+            const uint64_t kdesc[2] = {smem_desc_sw128(sK0, 16, 1024), smem_desc_sw128(sK0 + L::TILE_KV, 16, 1024)};
+            const uint64_t vdesc[2] = {smem_desc_sw128(sV0, BN * 128, 1024),
+                                       smem_desc_sw128(sV0 + L::TILE_KV, BN * 128, 1024)};
+            const uint64_t qxdesc = smem_desc_noswz(sQX, 128, 256), kxdesc = smem_desc_noswz(sKX, 128, 256);
+            auto issue_s = [&](int hh, int s) {
+                const uint64_t qd = qdesc[hh], kd = kdesc[s];
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk) {
                     const uint32_t off_q = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
                     const uint32_t off_k = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
-                    mma_bf16_ss(tS, qdesc + (off_q >> 4), kd + (off_k >> 4), idesc_qk, kk > 0 ? 1u : 0u);
+                    mma_bf16_ss(tmem + hh * BN, qd + (off_q >> 4), kd + (off_k >> 4), idesc_qk, kk > 0 ? 1u : 0u);
                 }
                 if (GATED)  // + bscale_h * gls_j: the bias k-step (no-swizzle tiles, K cores 128 B apart)
-                    mma_bf16_ss(tS, qxdesc, kxdesc + ((s * L::EXT) >> 4), idesc_qk, 1u);
+                    mma_bf16_ss(tmem + hh * BN, qxdesc + ((hh * L::EXT) >> 4), kxdesc + ((s * L::EXT) >> 4), idesc_qk,
+                                1u);
             };
-            auto issue_pv = [&](int s, bool acc) {
-                const uint64_t vd = s ? vdesc1 : vdesc0;
+            auto issue_pv = [&](int hh, int s, bool acc) {
+                const uint64_t vd = vdesc[s];
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk)
-                    mma_bf16_ts(tO, tS + kk * 8, vd + ((kk * 16 * 128) >> 4), idesc_pv, (acc || kk > 0) ? 1u : 0u);
+                    mma_bf16_ts(tmem + 2 * BN + hh * HD, tmem + hh * BN + kk * 8, vd + ((kk * 16 * 128) >> 4),
+                                idesc_pv, (acc || kk > 0) ? 1u : 0u);
             };
             int uc = 0, t = 0, it = 0;
             bool ok = true;
@@ -442,38 +435,51 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 Unit U{};
                 decode_unit(unit, pairs, B, cu_kept, kv_chunk, &U, M_total, status);
                 ok = mbar_wait(bar(T_Q_FULL), uc & 1, abort_flag, status, TG_WHERE_MMA);
-                if (hh == 0) PT_STAMP(3, uc == 0);
+                PT_STAMP(3, uc == 0);
                 ok = ok && mbar_wait(bar(T_K_FULL + (t & 1)), (t >> 1) & 1, abort_flag, status, TG_WHERE_MMA);
-                if (hh == 0) PT_STAMP(4, uc == 0);
+                PT_STAMP(4, uc == 0);
                 if (!ok) break;
                 tc_fence_after();
                 // S_h(0) of this unit: S_h's last reader (PV_h of the previous unit's last tile)
-                // was issued before by this thread
-                issue_s(t & 1);
-                mma_commit(bar(T_S_FULL + hh));
+                // was issued before by this thread, and tcgen05 operations execute in order
+                issue_s(0, t & 1);
+                mma_commit(bar(T_S_FULL + 0));
+                issue_s(1, t & 1);
+                mma_commit(bar(T_S_FULL + 1));
                 mma_commit(bar(T_K_EMPTY + (t & 1)));
                 if (U.n_kv == 1) mma_commit(bar(T_Q_EMPTY));
                 for (int j = 0; j < U.n_kv; ++j) {
                     const int s = t & 1;
                     const bool more = j + 1 < U.n_kv;
                     ok = mbar_wait(bar(T_V_FULL + s), (t >> 1) & 1, abort_flag, status, TG_WHERE_MMA) &&
-                         mbar_wait(bar(T_P_FULL + hh), it & 1, abort_flag, status, TG_WHERE_MMA);
+                         mbar_wait(bar(T_P_FULL + 0), it & 1, abort_flag, status, TG_WHERE_MMA);
                     if (!ok) break;
                     tc_fence_after();
-                    PT_PIPE(hh, it);
-                    issue_pv(s, j > 0);
-                    mma_commit(bar(T_V_EMPTY + s));
+                    PT_PIPE(0, it);
+                    issue_pv(0, s, j > 0);
                     if (more) {
                         ok = mbar_wait(bar(T_K_FULL + (s ^ 1)), ((t + 1) >> 1) & 1, abort_flag, status, TG_WHERE_MMA);
                         if (!ok) break;
                         tc_fence_after();
-                        if (hh == 0) PT_PIPE(2, it);
-                        issue_s(s ^ 1);
-                        mma_commit(bar(T_S_FULL + hh));
+                        PT_PIPE(2, it);
+                        issue_s(0, s ^ 1);
+                        mma_commit(bar(T_S_FULL + 0));
+                    } else {
+                        mma_commit(bar(T_O_FULL + 0));
+                    }
+                    ok = mbar_wait(bar(T_P_FULL + 1), it & 1, abort_flag, status, TG_WHERE_MMA);
+                    if (!ok) break;
+                    tc_fence_after();
+                    PT_PIPE(1, it);
+                    issue_pv(1, s, j > 0);
+                    mma_commit(bar(T_V_EMPTY + s));
+                    if (more) {
+                        issue_s(1, s ^ 1);
+                        mma_commit(bar(T_S_FULL + 1));
                         mma_commit(bar(T_K_EMPTY + (s ^ 1)));
                         if (j + 2 == U.n_kv) mma_commit(bar(T_Q_EMPTY));  // the unit's last S products
                     } else {
-                        mma_commit(bar(T_O_FULL + hh));
+                        mma_commit(bar(T_O_FULL + 1));
                     }
                     ++t;
                     ++it;
@@ -481,8 +487,8 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 ++uc;
             }
             // every MMA (and the barrier arrivals its commits trigger) lands before the CTA exits
-            mma_commit(bar(T_DRAIN + hh));
-            drain_wait(bar(T_DRAIN + hh), 0, status);
+            mma_commit(bar(T_DRAIN));
+            drain_wait(bar(T_DRAIN), 0, status);
         }
     }
     } else {
