@@ -1191,12 +1191,14 @@ int64_t units_below_host(int x, int C) {
 // of a sequence needs qt + 1 KV tiles; a chunk length C < n_qt cuts the query
 // tiles past C into two units ([0, C) and [C, qt + 1)), C >= ceil(n_qt / 2) so
 // that two always suffice.  A unit costs about F + n_kv tile pairs on one SM,
-// F = 3.1 being the fixed part (set-up, first loads, epilogue: 9.0 us against
-// 2.87 us per tile pair in a per-CTA timeline of the N=32k, K=2000 launch).  The
-// block scheduler hands out units heaviest first, which is longest-processing-
-// time scheduling, so C is the candidate whose LPT makespan over the SMs is
-// smallest (all sequences taken at max_M, the bound the host knows); ties go to
-// the larger C (fewer units).
+// F being the part a unit adds beyond its tiles.  With the persistent kernel
+// (the split only runs there) a CTA loads the next unit while it finishes the
+// current one, so F is about one tile pair (the epilogue and the merge); the
+// one-CTA-per-unit kernel paid F = 3.1 (9 us of set-up, first loads and
+// epilogue against 2.87 us per tile pair).  Units are taken heaviest first,
+// which is longest-processing-time scheduling, so C is the candidate whose LPT
+// makespan over the SMs is smallest (all sequences taken at max_M, the bound the
+// host knows); ties go to the larger C (fewer units).
 int attention_kv_chunk(int B, int max_M, int Hq, int Hkv, bool have_ws) {
     const int n_qt = (max_M + BM - 1) / BM;
     if (!have_ws || (Hq / Hkv) % 2 != 0 || n_qt < 4) return n_qt > 0 ? n_qt : 1;
@@ -1218,7 +1220,7 @@ int attention_kv_chunk(int B, int max_M, int Hq, int Hkv, bool have_ws) {
         if (it != memo.end()) return it->second;
     }
 #ifndef TG_LPT_FIXED_COST
-#define TG_LPT_FIXED_COST 3.1
+#define TG_LPT_FIXED_COST 1.0
 #endif
     constexpr double F = TG_LPT_FIXED_COST;
     int best_c = n_qt;
