@@ -135,6 +135,12 @@ __device__ unsigned long long g_pers_pipe[16 * 64];  // clock64 of pipeline poin
         if (blockIdx.x == 0 && (j) < 64) g_pers_pipe[(point) * 64 + (j)] = clock64();         \
     } while (0)
 __device__ unsigned long long g_pers_trace[1024 * 16];
+__device__ unsigned long long g_pers_units[1024 * 4 * 4];  // per CTA, first 4 units: start, loop end, epi end, info
+#define PT_UNIT(uc, slot, val)                                                                  \
+    do {                                                                                        \
+        if (threadIdx.x == 0 && blockIdx.x < 1024 && (uc) < 4)                                  \
+            g_pers_units[(blockIdx.x * 4 + (uc)) * 4 + (slot)] = (val);                         \
+    } while (0)
 #define PT_STAMP(slot, cond)                                                             \
     do {                                                                                 \
         if ((cond) && blockIdx.x < 1024) g_pers_trace[blockIdx.x * 16 + (slot)] = globaltimer(); \
@@ -146,6 +152,9 @@ __device__ unsigned long long g_pers_trace[1024 * 16];
 #define PT_PIPE(point, j) \
     do {                  \
     } while (0)
+#define PT_UNIT(uc, slot, val) \
+    do {                       \
+    } while (0)
 #endif
 
 template <int HD, bool GATED>
@@ -156,7 +165,7 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                        const float* __restrict__ c, float sm_scale, int Hq, int Hkv, int B, int64_t M_total,
                        int kv_chunk, int64_t total_units, SplitWs ws,
                        int* __restrict__ sched, uint16_t* __restrict__ out, float* __restrict__ lse,
-                       int* __restrict__ status, int early) {
+                       int* __restrict__ status, int early, int wide_out) {
     using L = PtSmem<HD>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -518,6 +527,11 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             bool ok = true;
             Unit U{};
             decode_unit(unit, pairs, B, cu_kept, kv_chunk, &U, M_total, status);
+            PT_UNIT(uc, 0, globaltimer());
+            PT_UNIT(uc, 3, static_cast<unsigned long long>(U.n_kv) | (static_cast<unsigned long long>(U.split) << 8) |
+                               (static_cast<unsigned long long>(U.qt) << 24) |
+                               (static_cast<unsigned long long>(U.chunk) << 40) |
+                               (static_cast<unsigned long long>(U.pair) << 48));
             const int q_local = U.qt * BM + r;
             const bool valid_row = q_local < U.Mb;
             const int64_t qg = static_cast<int64_t>(U.seq0) + q_local;
@@ -548,6 +562,10 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     break;
                 }
                 PT_STAMP(5, uc == 0 && j == 0 && threadIdx.x == 0);
+#ifdef TG_TRACE
+                if (uc == 0 && j == 0 && threadIdx.x == 0 && blockIdx.x < 1024)
+                    g_pers_trace[blockIdx.x * 16 + 13] = U.n_kv | (U.split ? 1000 : 0) | (U.qt << 16);
+#endif
                 if (r == 0) PT_PIPE(4 + h, it);
                 tc_fence_after();
                 float x[BN];
@@ -627,22 +645,39 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             }
             // ---------------------------------------------------------------- epilogue
             PT_STAMP(6, uc == 0 && threadIdx.x == 0);
+            PT_UNIT(uc, 1, globaltimer());
             if (ok) ok = mbar_wait_warp(bar(T_O_FULL + h), uc & 1, abort_flag, status, TG_WHERE_SOFTMAX);
             PT_STAMP(7, uc == 0 && threadIdx.x == 0);
             if (bar_red_or(bid, 128, !ok)) break;
             tc_fence_after();
             const float inv_l = 1.0f / l_run;
             uint16_t* orow = out + (qg * Hq + hw) * HD;
+            // A thread writes its own row; a warp's stores go to 32 different rows, so wider
+            // stores mean fewer of them: 32 bytes (one whole sector) when `out` is 32-byte
+            // aligned, else 16.
             auto store_chunk = [&](int ch, const float* o32, float w) {  // 32 columns from 32 ch
                 if (!valid_row) return;
+                if (wide_out) {
 #pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4) {
-                    uint4 v;
-                    v.x = pack_bf16x2(o32[k4 * 8 + 0] * w, o32[k4 * 8 + 1] * w);
-                    v.y = pack_bf16x2(o32[k4 * 8 + 2] * w, o32[k4 * 8 + 3] * w);
-                    v.z = pack_bf16x2(o32[k4 * 8 + 4] * w, o32[k4 * 8 + 5] * w);
-                    v.w = pack_bf16x2(o32[k4 * 8 + 6] * w, o32[k4 * 8 + 7] * w);
-                    *reinterpret_cast<uint4*>(orow + ch * 32 + k4 * 8) = v;
+                    for (int k8 = 0; k8 < 2; ++k8) {
+                        const float* p = o32 + k8 * 16;
+                        asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(orow + ch * 32 + k8 * 16),
+                                     "r"(pack_bf16x2(p[0] * w, p[1] * w)), "r"(pack_bf16x2(p[2] * w, p[3] * w)),
+                                     "r"(pack_bf16x2(p[4] * w, p[5] * w)), "r"(pack_bf16x2(p[6] * w, p[7] * w)),
+                                     "r"(pack_bf16x2(p[8] * w, p[9] * w)), "r"(pack_bf16x2(p[10] * w, p[11] * w)),
+                                     "r"(pack_bf16x2(p[12] * w, p[13] * w)), "r"(pack_bf16x2(p[14] * w, p[15] * w))
+                                     : "memory");
+                    }
+                } else {
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        uint4 v;
+                        v.x = pack_bf16x2(o32[k4 * 8 + 0] * w, o32[k4 * 8 + 1] * w);
+                        v.y = pack_bf16x2(o32[k4 * 8 + 2] * w, o32[k4 * 8 + 3] * w);
+                        v.z = pack_bf16x2(o32[k4 * 8 + 4] * w, o32[k4 * 8 + 5] * w);
+                        v.w = pack_bf16x2(o32[k4 * 8 + 6] * w, o32[k4 * 8 + 7] * w);
+                        *reinterpret_cast<uint4*>(orow + ch * 32 + k4 * 8) = v;
+                    }
                 }
             };
             if (!U.split) {
@@ -743,6 +778,7 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             // (that product waits for this warpgroup's next P arrival)
             tc_fence_before();
             PT_STAMP(8, uc == 0 && threadIdx.x == 0);
+            PT_UNIT(uc, 2, globaltimer() | (static_cast<unsigned long long>(U.split ? s_arr[h] + 1 : 0) << 60));
             ++uc;
         }
 #ifdef TG_TRACE
@@ -751,6 +787,7 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
             g_pers_trace[blockIdx.x * 16 + 9] = globaltimer();
             g_pers_trace[blockIdx.x * 16 + 11] = smid | (static_cast<unsigned long long>(uc) << 32);
+            g_pers_trace[blockIdx.x * 16 + 12] = it;  // tiles this CTA processed
         }
 #endif
     }
@@ -795,6 +832,9 @@ cudaError_t launch_exp2_poly_selftest(const float* x, float* y, int64_t n, cudaS
 #ifdef TG_TRACE
 extern "C" __attribute__((visibility("default"))) int tg_trace_read_attention_pers(unsigned long long* host) {
     return cudaMemcpyFromSymbol(host, g_pers_trace, sizeof(g_pers_trace)) == cudaSuccess ? 0 : 1;
+}
+extern "C" __attribute__((visibility("default"))) int tg_trace_read_attention_pers_units(unsigned long long* host) {
+    return cudaMemcpyFromSymbol(host, g_pers_units, sizeof(g_pers_units)) == cudaSuccess ? 0 : 1;
 }
 extern "C" __attribute__((visibility("default"))) int tg_trace_read_attention_pers_pipe(unsigned long long* host) {
     return cudaMemcpyFromSymbol(host, g_pers_pipe, sizeof(g_pers_pipe)) == cudaSuccess ? 0 : 1;
@@ -842,7 +882,8 @@ static cudaError_t launch_pers_impl(const CUtensorMap& tq, const CUtensorMap& tk
     const unsigned grid = static_cast<unsigned>(total < sms ? total : sms);
     return launch_pdl(gated_attn_pers_kernel<HD, GATED>, dim3(grid), dim3(PT_THREADS), static_cast<size_t>(L::ALLOC),
                       st, tq, tk, tv, cu_kept, pos, rank, gates, c, sm_scale, Hq, Hkv, B, M_total, lay.C, total, sw,
-                      reinterpret_cast<int*>(base), out, lse, device_status_ptr(), early ? 1 : 0);
+                      reinterpret_cast<int*>(base), out, lse, device_status_ptr(), early ? 1 : 0,
+                      (reinterpret_cast<uintptr_t>(out) & 31u) == 0 ? 1 : 0);
 }
 
 cudaError_t launch_attention_persistent(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,

@@ -569,3 +569,28 @@ def test_persistent_and_per_unit_kernels_agree(tg, name):
     H.assert_attention_close(a[sel], out_ref, name + " persistent")
     H.assert_attention_close(b[sel], out_ref, name + " per-unit")
     assert np.max(np.abs(a_lse[sel] - lse_ref)) <= H.LSE_ABS
+
+
+def test_attention_output_only_16_byte_aligned(tg):
+    """`out` needs 16-byte alignment only: a buffer that is 16- but not 32-byte aligned
+    takes the 16-byte row stores and gives the same bits as an aligned one."""
+    from learned_token_pruning_rmsnorm_b200 import _lib
+    lib = _lib.load()
+    w, comp, ai, gls32, _, _, _ = attn_case("c1_16k")
+    ck = comp["cu_kept"]
+    M, max_M = int(ck[-1]), int(np.max(np.diff(ck)))
+    t = [H.bf16_dev(ai["q"]), H.bf16_dev(ai["k"]), H.bf16_dev(ai["v"]), H.i32_dev(ck), H.i32_dev(comp["pos"]),
+         H.i32_dev(comp["rank"]), H.f32_dev(gls32), H.f32_dev(ai["g"]), H.f32_dev(ai["c"])]
+    n = int(lib.tg_gated_attention_workspace_size(w.B, max_M, w.Hq, w.Hkv, w.d))
+    ws = torch.zeros(max(n, 256), dtype=torch.uint8, device="cuda")
+    outs = []
+    for shift in (0, 8):  # 8 bf16 = 16 bytes
+        flat = torch.zeros(M * w.Hq * w.d + 16, dtype=torch.bfloat16, device="cuda")
+        out = flat[shift:shift + M * w.Hq * w.d]
+        assert (out.data_ptr() % 32 == 0) == (shift == 0) and out.data_ptr() % 16 == 0
+        _lib.check(lib.tg_gated_attention(*[x.data_ptr() for x in t[:4]], w.B, M, max_M, w.Hq, w.Hkv, w.d,
+                                          *[x.data_ptr() for x in t[4:]], 1.0 / math.sqrt(w.d), out.data_ptr(), None,
+                                          ws.data_ptr(), ws.numel(), None))
+        torch.cuda.synchronize()
+        outs.append(H.bf16_host_bits(out))
+    np.testing.assert_array_equal(outs[0], outs[1])
