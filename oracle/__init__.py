@@ -56,8 +56,8 @@ def _load():
             lib.oracle_masked_gated_attention.argtypes = [P, P, P, P, P, i32, i32, i32, i32, P, P, P, P,
                                                           f64, P, i64, P]
             lib.oracle_gated_attention_backward.argtypes = [P, P, P, P, i32, i32, i32, i32, P, P, P, P, P, f64,
-                                                            P, P, P, P, P, P, P]
-            if lib.oracle_abi_version() != 3:
+                                                            P, P, P, P, P, P, P, i32]
+            if lib.oracle_abi_version() != 4:
                 raise ImportError("oracle/liboracle.so is stale: rebuild it")
             _lib = lib
     return _lib
@@ -200,17 +200,20 @@ def gated_attention(q_bits, k_bits, v_bits, cu_kept, pos, rank, gls_f32, g, c, s
 
 def gated_attention_backward(q_bits, k_bits, v_bits, cu_kept, pos, rank, gls_f32, g, c, dout, sm_scale=None,
                              scores=None, prunable=None) -> dict:
-    """Gradients of the token-gated attention (one gate) for the upstream
-    gradient dout [M, Hq, d]: dq [M, Hq, d], dk/dv [M, Hkv, d], dgls [M],
-    dg/dc [Hq], all fp64.
+    """Gradients of the token-gated attention for the upstream gradient dout
+    [M, Hq, d]: dq [M, Hq, d], dk/dv [M, Hkv, d], dgls, dg, dc [Hq], all fp64.
+
+    One gate: gls_f32 [M] and g [Hq] give dgls [M] and dg [Hq].  Several gates
+    (AI summary, "Future Directions"): gls_f32 [G, M] and g [G, Hq] give dgls
+    [G, M] and dg [G, Hq], gate i's bias term being softplus(g[i, h]) gls[i, j].
 
     With the kept rows' gate scores (scores [M] fp32, the s_j whose
     logsigmoid is gls_j) and the rows the gate could prune (prunable [M]
-    bool), it also returns dscore [M]: the gradient that reaches the gate's
-    score through the bias (AI summary, "Key Contributions" 2: the bias on
-    the logits carries the task loss back to the scoring network).  Since
-    gls_j = logsigmoid(s_j), d gls_j / d s_j = sigmoid(-s_j), taken here from
-    the score itself; rows the gate cannot prune carry no bias and get 0."""
+    bool), the one-gate form also returns dscore [M]: the gradient that reaches
+    the gate's score through the bias (AI summary, "Key Contributions" 2: the
+    bias on the logits carries the task loss back to the scoring network).
+    Since gls_j = logsigmoid(s_j), d gls_j / d s_j = sigmoid(-s_j), taken here
+    from the score itself; rows the gate cannot prune carry no bias and get 0."""
     q, qp = _c(q_bits, np.uint16)
     k, kp = _c(k_bits, np.uint16)
     v, vp_ = _c(v_bits, np.uint16)
@@ -219,19 +222,25 @@ def gated_attention_backward(q_bits, k_bits, v_bits, cu_kept, pos, rank, gls_f32
     cu, cup = _c(cu_kept, np.int32)
     po, pop = _c(pos, np.int32)
     ra, rap = _c(rank, np.int32)
-    gl, glp = _c(gls_f32, np.float32)
-    ga, gap = _c(g, np.float32)
+    one_gate = np.ndim(gls_f32) == 1
+    gl, glp = _c(np.asarray(gls_f32, dtype=np.float32).reshape(-1, M), np.float32)
+    ga, gap = _c(np.asarray(g, dtype=np.float32).reshape(-1, Hq), np.float32)
+    G = gl.shape[0]
+    if ga.shape[0] != G:
+        raise ValueError("one row of g per gate")
     ca, cap = _c(c, np.float32)
     go, gop = _c(np.asarray(dout, dtype=np.float64).reshape(M, Hq, d), np.float64)
     if sm_scale is None:
         sm_scale = 1.0 / np.sqrt(d)
     out = {"dq": np.empty((M, Hq, d)), "dk": np.empty((M, Hkv, d)), "dv": np.empty((M, Hkv, d)),
-           "dgls": np.empty(M), "dg": np.empty(Hq), "dc": np.empty(Hq)}
+           "dgls": np.empty((G, M)), "dg": np.empty((G, Hq)), "dc": np.empty(Hq)}
     vp = lambda a: a.ctypes.data_as(C.c_void_p)  # noqa: E731
     _load().oracle_gated_attention_backward(qp, kp, vp_, cup, len(cu) - 1, Hq, Hkv, d, pop, rap, glp, gap, cap,
                                             float(sm_scale), gop, vp(out["dq"]), vp(out["dk"]), vp(out["dv"]),
-                                            vp(out["dgls"]), vp(out["dg"]), vp(out["dc"]))
-    if scores is not None:
+                                            vp(out["dgls"]), vp(out["dg"]), vp(out["dc"]), G)
+    if one_gate:
+        out["dgls"], out["dg"] = out["dgls"][0], out["dg"][0]
+    if scores is not None and one_gate:
         s64 = np.asarray(scores, dtype=np.float64).reshape(M)
         mask = np.ones(M, dtype=bool) if prunable is None else np.asarray(prunable, dtype=bool).reshape(M)
         # sigmoid(-s) = exp(-log(1 + e^s)), finite for every s

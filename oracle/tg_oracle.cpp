@@ -81,7 +81,7 @@ int64_t kept_prunable(int64_t p, int32_t k) { return (k < 0 || k > p) ? p : stat
 
 extern "C" {
 
-int oracle_abi_version() { return 3; }
+int oracle_abi_version() { return 4; }
 
 // Thread count of the parallel loops (one row per iteration; no reduction
 // crosses threads, so results do not depend on it).
@@ -377,37 +377,40 @@ void oracle_masked_gated_attention(const uint16_t* q, const uint16_t* k, const u
 // lacks: AI summary, "Key Contributions" 2 -- the bias carries the task loss's
 // gradient to the scoring network -- and 3 -- the gain and temperature are
 // learned).  One gate.  Given dL/d out, every derivative follows the forward
-// definitions by the chain rule, per (query i, head h, causal key j):
-//   l_ij   = (sm * q_i.k_j + beta_h * gls_j) / tau_ih,  beta_h = softplus(g_h)
+// definitions by the chain rule, per (query i, head h, causal key j), for n_gates gate
+// modules (gate i with logsigmoids gls_i and gains g_i; one gate is n_gates = 1):
+//   l_ij   = (sm * q_i.k_j + sum_i beta_ih * gls_ij) / tau_ih,  beta_ih = softplus(g_ih)
 //   P_ij   = softmax_j(l_ij),  out_i = sum_j P_ij v_j
 //   dP_ij  = dout_i . v_j,  D_i = sum_j P_ij dP_ij,  dl_ij = P_ij (dP_ij - D_i)
 //   dq_i  += sm dl_ij / tau * k_j,   dk_j += sm dl_ij / tau * q_i
-//   dv_j  += P_ij dout_i,            dgls_j += beta_h dl_ij / tau
-//   dbeta_h += dl_ij gls_j / tau,    dtau_ih = -sum_j dl_ij l_ij / tau
-//   dg_h = dbeta_h * sigmoid(g_h),   dc_h = sum_i dtau_ih ln(pos_i / rank_i)
-// dout is [M, Hq, d] fp64; dq [M, Hq, d], dk/dv [M, Hkv, d], dgls [M] and
-// dg/dc [Hq] are fp64 outputs.  Heads run in parallel, each into its own
-// partial sums, added in head order (results do not depend on the threads).
+//   dv_j  += P_ij dout_i,            dgls_ij += beta_ih dl_ij / tau
+//   dbeta_ih += dl_ij gls_ij / tau,  dtau_ih = -sum_j dl_ij l_ij / tau
+//   dg_ih = dbeta_ih * sigmoid(g_ih),   dc_h = sum_i dtau_ih ln(pos_i / rank_i)
+// dout is [M, Hq, d] fp64; dq [M, Hq, d], dk/dv [M, Hkv, d], dgls [n_gates, M], dg
+// [n_gates, Hq] and dc [Hq] are fp64 outputs; gls is [n_gates, M], g [n_gates, Hq].
+// Heads run in parallel, each into its own partial sums, added in head order (results do
+// not depend on the threads).
 void oracle_gated_attention_backward(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* cu_kept,
                                      int B, int Hq, int Hkv, int d, const int32_t* pos, const int32_t* rank,
                                      const float* gls, const float* g, const float* c, double sm_scale,
                                      const double* dout, double* dq, double* dk, double* dv, double* dgls, double* dg,
-                                     double* dc) {
+                                     double* dc, int n_gates) {
     const int64_t M = cu_kept[B];
     const int group = Hq / Hkv;
+    const int G = n_gates;
     const size_t kv = static_cast<size_t>(M) * Hkv * d;
     std::vector<double> dk_h(static_cast<size_t>(Hq) * kv, 0.0), dv_h(static_cast<size_t>(Hq) * kv, 0.0);
-    std::vector<double> dgls_h(static_cast<size_t>(Hq) * M, 0.0);
+    std::vector<double> dgls_h(static_cast<size_t>(Hq) * G * M, 0.0);
     std::fill(dq, dq + static_cast<size_t>(M) * Hq * d, 0.0);
 #pragma omp parallel for schedule(dynamic, 1)
     for (int h = 0; h < Hq; ++h) {
         const int hk = h / group;
-        const double gh = static_cast<double>(g[h]);
-        const double beta = softplus(gh);
-        double dbeta = 0.0, dcs = 0.0;
+        std::vector<double> beta(G), dbeta(G, 0.0);
+        for (int gi = 0; gi < G; ++gi) beta[gi] = softplus(static_cast<double>(g[gi * Hq + h]));
+        double dcs = 0.0;
         double* dkp = dk_h.data() + static_cast<size_t>(h) * kv;
         double* dvp = dv_h.data() + static_cast<size_t>(h) * kv;
-        double* dglp = dgls_h.data() + static_cast<size_t>(h) * M;
+        double* dglp = dgls_h.data() + static_cast<size_t>(h) * G * M;
         std::vector<double> logit, p, dp;
         for (int b = 0; b < B; ++b) {
             for (int64_t i = cu_kept[b]; i < cu_kept[b + 1]; ++i) {
@@ -424,7 +427,9 @@ void oracle_gated_attention_backward(const uint16_t* q, const uint16_t* k, const
                     double dot = 0.0;
                     for (int e = 0; e < d; ++e)
                         dot += bf16_to_double(q[(i * Hq + h) * d + e]) * bf16_to_double(k[(j * Hkv + hk) * d + e]);
-                    const double l = (dot * sm_scale + beta * static_cast<double>(gls[j])) / tau;
+                    double bias = 0.0;
+                    for (int gi = 0; gi < G; ++gi) bias += beta[gi] * static_cast<double>(gls[gi * M + j]);
+                    const double l = (dot * sm_scale + bias) / tau;
                     logit[static_cast<size_t>(j - j0)] = l;
                     mx = std::max(mx, l);
                 }
@@ -446,31 +451,34 @@ void oracle_gated_attention_backward(const uint16_t* q, const uint16_t* k, const
                 for (int64_t j = j0; j <= i; ++j) {
                     const size_t t = static_cast<size_t>(j - j0);
                     const double dl = p[t] * (dp[t] - D);
-                    const double G = dl / tau;
+                    const double Gq = dl / tau;
                     for (int e = 0; e < d; ++e) {
-                        dq[(i * Hq + h) * d + e] += sm_scale * G * bf16_to_double(k[(j * Hkv + hk) * d + e]);
-                        dkp[(j * Hkv + hk) * d + e] += sm_scale * G * bf16_to_double(q[(i * Hq + h) * d + e]);
+                        dq[(i * Hq + h) * d + e] += sm_scale * Gq * bf16_to_double(k[(j * Hkv + hk) * d + e]);
+                        dkp[(j * Hkv + hk) * d + e] += sm_scale * Gq * bf16_to_double(q[(i * Hq + h) * d + e]);
                         dvp[(j * Hkv + hk) * d + e] += p[t] * go[e];
                     }
-                    dglp[j] += beta * G;
-                    dbeta += G * static_cast<double>(gls[j]);
+                    for (int gi = 0; gi < G; ++gi) {
+                        dglp[gi * M + j] += beta[gi] * Gq;
+                        dbeta[gi] += Gq * static_cast<double>(gls[gi * M + j]);
+                    }
                     if (dl != 0.0) dtau -= dl * logit[t] / tau;
                 }
                 dcs += dtau * lr;
             }
         }
-        dg[h] = dbeta / (1.0 + std::exp(-gh));
+        for (int gi = 0; gi < G; ++gi)
+            dg[gi * Hq + h] = dbeta[gi] / (1.0 + std::exp(-static_cast<double>(g[gi * Hq + h])));
         dc[h] = dcs;
     }
     std::fill(dk, dk + kv, 0.0);
     std::fill(dv, dv + kv, 0.0);
-    std::fill(dgls, dgls + M, 0.0);
+    std::fill(dgls, dgls + static_cast<size_t>(G) * M, 0.0);
     for (int h = 0; h < Hq; ++h) {
         for (size_t e = 0; e < kv; ++e) {
             dk[e] += dk_h[static_cast<size_t>(h) * kv + e];
             dv[e] += dv_h[static_cast<size_t>(h) * kv + e];
         }
-        for (int64_t j = 0; j < M; ++j) dgls[j] += dgls_h[static_cast<size_t>(h) * M + j];
+        for (size_t e = 0; e < static_cast<size_t>(G) * M; ++e) dgls[e] += dgls_h[static_cast<size_t>(h) * G * M + e];
     }
 }
 

@@ -160,3 +160,49 @@ def test_score_gradient_matches_central_differences(oracle_mod):
         fd = (_loss(oracle_mod, q, k, v, cu, pos, rank, lp, g, c, dout) -
               _loss(oracle_mod, q, k, v, cu, pos, rank, lm, g, c, dout)) / (2 * eps)
         assert got["dscore"][j] == pytest.approx(fd, rel=2e-3, abs=1e-7), j
+
+
+def test_two_gate_backward_matches_central_differences(oracle_mod):
+    """Several gates: each gate's logsigmoids and gains, perturbed by +-2^-12 in the
+    oracle's two-gate forward, give its dgls and dg."""
+    q, k, v, cu, pos, rank, gls, g, c, dout = _case(8, [12, 9], 4, 2, 8)
+    rng = np.random.default_rng(80)
+    gls2 = np.stack([gls, -np.abs(rng.standard_normal(len(gls)) * 1.5).astype(np.float32)])
+    gls2[1, :2] = 0.0
+    g2 = np.stack([g, rng.standard_normal(4).astype(np.float32)])
+    got = oracle_mod.gated_attention_backward(q, k, v, cu, pos, rank, gls2, g2, c, dout)
+    assert got["dgls"].shape == (2, len(gls)) and got["dg"].shape == (2, 4)
+    eps = 2.0 ** -12
+    for gi in range(2):
+        for j in (2, 6, 15, 20):
+            lp, lm = gls2.copy(), gls2.copy()
+            lp[gi, j] += eps
+            lm[gi, j] -= eps
+            fd = (_loss(oracle_mod, q, k, v, cu, pos, rank, lp, g2, c, dout) -
+                  _loss(oracle_mod, q, k, v, cu, pos, rank, lm, g2, c, dout)) / (2 * eps)
+            assert got["dgls"][gi, j] == pytest.approx(fd, rel=1e-4, abs=1e-8), (gi, j)
+        for h in range(4):
+            gp, gm = g2.copy(), g2.copy()
+            gp[gi, h] += eps
+            gm[gi, h] -= eps
+            fd = (_loss(oracle_mod, q, k, v, cu, pos, rank, gls2, gp, c, dout) -
+                  _loss(oracle_mod, q, k, v, cu, pos, rank, gls2, gm, c, dout)) / (2 * eps)
+            assert got["dg"][gi, h] == pytest.approx(fd, rel=1e-4, abs=1e-8), (gi, h)
+
+
+def test_split_gate_backward_equals_one_gate(oracle_mod):
+    """Two gates with the same gains whose logsigmoids add up to one gate's give that
+    gate's dq, dk, dv, dc; each of them gets the one gate's dgls (same gain), and their
+    dg add up to the one gate's."""
+    q, k, v, cu, pos, rank, gls, g, c, dout = _case(9, [10, 7], 2, 1, 8)
+    # a keeps the top 12 significand bits of gls, b the rest: both exact, a + b == gls in fp32
+    a = (gls.view(np.uint32) & np.uint32(0xFFFFF800)).view(np.float32)
+    b = (gls - a).astype(np.float32)
+    assert np.array_equal(a + b, gls) and np.abs(b).max() > 0
+    one = oracle_mod.gated_attention_backward(q, k, v, cu, pos, rank, a + b, g, c, dout)
+    two = oracle_mod.gated_attention_backward(q, k, v, cu, pos, rank, np.stack([a, b]), np.stack([g, g]), c, dout)
+    for key in ("dq", "dk", "dv", "dc"):
+        np.testing.assert_allclose(two[key], one[key], rtol=1e-9, atol=1e-12, err_msg=key)
+    for gi in range(2):
+        np.testing.assert_allclose(two["dgls"][gi], one["dgls"], rtol=1e-9, atol=1e-12)
+    np.testing.assert_allclose(two["dg"].sum(axis=0), one["dg"], rtol=1e-9, atol=1e-12)
