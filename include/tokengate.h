@@ -240,6 +240,25 @@ tg_status tg_gated_attention_backward(const uint16_t* q, const uint16_t* k, cons
                                       tg_stream_t stream);
 
 /*
+ * Backward of tg_gated_attention_gates: several gate modules (AI summary,
+ * "Future Directions"), the logits carrying sum_i softplus(g[i][h]) gls[i][j].
+ * Same arguments and outputs as tg_gated_attention_backward, with per-gate
+ * HOST arrays of DEVICE pointers: gls[i] [M] and g[i] [Hq] in; dgls[i] [M]
+ * (d loss / d gls_i) and dg[i] [Hq] out; dscore (may be NULL, as may any of
+ * its entries) gets dscore[i][j] = dgls[i][j] * (1 - exp(gls[i][j])).
+ * 1 <= n_gates <= 4, else TG_ERR_UNSUPPORTED; n_gates = 1 is
+ * tg_gated_attention_backward.  Same workspace size.
+ */
+tg_status tg_gated_attention_backward_gates(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                            const uint16_t* out, const uint16_t* dout, const float* lse,
+                                            const int32_t* cu_kept, int B, int64_t M_total, int max_M, int Hq,
+                                            int Hkv, int d, const int32_t* pos, const int32_t* rank, int n_gates,
+                                            const float* const* gls, const float* const* g, const float* c,
+                                            float sm_scale, uint16_t* dq, uint16_t* dk, uint16_t* dv,
+                                            float* const* dgls, float* const* dscore, float* const* dg, float* dc,
+                                            void* ws, size_t ws_bytes, tg_stream_t stream);
+
+/*
  * Host only: the prunable span of the NEXT gate, in the kept order of this
  * one.  All tokens before a span are kept, so sequence b's surviving span
  * tokens sit at kept indices [p0_b, p0_b + min(k_b, |P_b|)) (k_b < 0 = all).

@@ -373,6 +373,50 @@ def tg_gated_attention_backward(q, k, v, out, dout, lse, cu_kept, max_M: int, po
     return res
 
 
+def tg_gated_attention_backward_gates(q, k, v, out, dout, lse, cu_kept, max_M: int, pos, rank, gls, g, c,
+                                      sm_scale: float | None = None, want_dscore: bool = True):
+    """Gradients of tg_gated_attention_gates for dout: gls and g are lists with one
+    tensor per gate ([M] and [Hq] fp32).  Returns a dict with dq, dk, dv, dc as for one
+    gate, and lists dgls, dscore (or None), dg with one tensor per gate."""
+    M, Hq, d = q.shape
+    Hkv = k.shape[1]
+    dev = q.device
+    n = len(gls)
+    if n != len(g):
+        raise ValueError("one gain tensor per gate")
+    _dev(q, torch.bfloat16, "q")
+    _dev(k, torch.bfloat16, "k", (M, Hkv, d))
+    _dev(v, torch.bfloat16, "v", (M, Hkv, d))
+    _dev(out, torch.bfloat16, "out", (M, Hq, d))
+    _dev(dout, torch.bfloat16, "dout", (M, Hq, d))
+    _dev(lse, torch.float32, "lse", (M, Hq))
+    _dev(pos, torch.int32, "pos", (M,))
+    _dev(rank, torch.int32, "rank", (M,))
+    for i in range(n):
+        _dev(gls[i], torch.float32, f"gls[{i}]", (M,))
+        _dev(g[i], torch.float32, f"g[{i}]", (Hq,))
+    _dev(c, torch.float32, "c", (Hq,))
+    ck = _i32_dev(cu_kept, dev, "cu_kept")
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    res = {"dq": torch.empty_like(q), "dk": torch.empty_like(k), "dv": torch.empty_like(v),
+           "dgls": [torch.empty(M, dtype=torch.float32, device=dev) for _ in range(n)],
+           "dscore": [torch.empty(M, dtype=torch.float32, device=dev) for _ in range(n)] if want_dscore else None,
+           "dg": [torch.empty(Hq, dtype=torch.float32, device=dev) for _ in range(n)],
+           "dc": torch.empty(Hq, dtype=torch.float32, device=dev)}
+    arr = lambda ts: (C.c_void_p * n)(*[t.data_ptr() for t in ts])  # noqa: E731
+    gls_a, g_a, dgls_a, dg_a = arr(gls), arr(g), arr(res["dgls"]), arr(res["dg"])
+    dsc_a = arr(res["dscore"]) if want_dscore else None
+    nb = int(load().tg_gated_attention_backward_workspace_size(M, Hq, Hkv, d))
+    ws = torch.empty(max(nb, 256), dtype=torch.uint8, device=dev)
+    _lib.check(load().tg_gated_attention_backward_gates(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(), lse.data_ptr(), ck.data_ptr(),
+        ck.numel() - 1, M, int(max_M), Hq, Hkv, d, pos.data_ptr(), rank.data_ptr(), n, gls_a, g_a, c.data_ptr(),
+        float(sm_scale), res["dq"].data_ptr(), res["dk"].data_ptr(), res["dv"].data_ptr(), dgls_a, dsc_a, dg_a,
+        res["dc"].data_ptr(), ws.data_ptr(), ws.numel(), _lib.stream_handle(dev)))
+    return res
+
+
 def tg_device_status(clear: bool = True, device=None):
     """(status, word): the device status word of the current device; status is
     TG_OK or TG_ERR_TIMEOUT.  Synchronises the current stream."""

@@ -48,6 +48,28 @@ constexpr float LN2_B = 0.6931471805599453f;
 
 __device__ __forceinline__ float softplus_b(float x) { return fmaxf(x, 0.f) + log1pf(expf(-fabsf(x))); }
 
+// The gains beta_i = softplus(g_i[h]) of every gate for query head h (0 past the last gate).
+struct GateGains {
+    float b0, b1, b2, b3;
+};
+__device__ __forceinline__ GateGains gate_gains(const GateSet& gs, int h) {
+    GateGains r;
+    r.b0 = softplus_b(gs.g[0][h]);
+    r.b1 = gs.n > 1 ? softplus_b(gs.g[1][h]) : 0.f;
+    r.b2 = gs.n > 2 ? softplus_b(gs.g[2][h]) : 0.f;
+    r.b3 = gs.n > 3 ? softplus_b(gs.g[3][h]) : 0.f;
+    return r;
+}
+// The bias of kept row `row` for that head: sum_i beta_i gls_i[row] (loads through L2: the
+// compaction map may have been written during this kernel's lifetime).
+__device__ __forceinline__ float gate_bias(const GateSet& gs, const GateGains& w, int64_t row) {
+    float acc = w.b0 * __ldcg(gs.gls[0] + row);
+    if (gs.n > 1) acc = fmaf(w.b1, __ldcg(gs.gls[1] + row), acc);
+    if (gs.n > 2) acc = fmaf(w.b2, __ldcg(gs.gls[2] + row), acc);
+    if (gs.n > 3) acc = fmaf(w.b3, __ldcg(gs.gls[3] + row), acc);
+    return acc;
+}
+
 __device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
@@ -121,8 +143,8 @@ template <int HD>
 __global__ void __launch_bounds__(DKV_THREADS, 1)
 gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                          const int32_t* __restrict__ cu_kept, const float* __restrict__ gls,
-                          const float* __restrict__ g, const float4* __restrict__ fac, float sm_scale, int Hq,
+                          const int32_t* __restrict__ cu_kept, const GateSet gates,
+                          const float4* __restrict__ fac, float sm_scale, int Hq,
                           int Hkv, int64_t M_total,
                           uint16_t* __restrict__ dk, uint16_t* __restrict__ dv, float* __restrict__ part_k,
                           float* __restrict__ part_v, float* __restrict__ colsum, int* __restrict__ status,
@@ -297,9 +319,9 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
         const int key_local = kt * BT + r;
         const bool valid_key = key_local < Mb;
         const uint32_t lane_addr = static_cast<uint32_t>(q4 * 32) << 16;
-        // kgl = (beta / sm) gls_j, the key's bias in units of the score, so that the log2 of
-        // P is tt = fa (s + kgl) - lse log2(e) with the query's fa = sm log2(e) / tau
-        const float kgl = valid_key ? (softplus_b(g[h]) / sm_scale) * __ldcg(gls + seq0 + key_local) : 0.f;
+        // kgl = (sum_i beta_i gls_ij) / sm, the key's bias in units of the score, so that the
+        // log2 of P is tt = fa (s + kgl) - lse log2(e) with the query's fa = sm log2(e) / tau
+        const float kgl = valid_key ? gate_bias(gates, gate_gains(gates, h), seq0 + key_local) / sm_scale : 0.f;
         // this warp's own table of its 32 queries' factors (fa, -lse log2(e), 1/tau, -D'/tau),
         // [2 half steps][4][32]; only __syncwarp orders it
         float* wtab = reinterpret_cast<float*>(smem + L::OFF_TAB) + warp * (2 * 4 * 32);
@@ -566,8 +588,8 @@ __global__ void __launch_bounds__(DQ_THREADS, 1)
 gated_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                          const int32_t* __restrict__ cu_kept, const int32_t* __restrict__ pos,
-                         const int32_t* __restrict__ rank, const float* __restrict__ gls,
-                         const float* __restrict__ g, const float* __restrict__ c, const float* __restrict__ lse,
+                         const int32_t* __restrict__ rank, const GateSet gates,
+                         const float* __restrict__ c, const float* __restrict__ lse,
                          const uint16_t* __restrict__ out_fwd, float4* __restrict__ fac, float sm_scale, int Hq,
                          int Hkv, int n_qt_max, uint16_t* __restrict__ dq, float* __restrict__ tileT,
                          int* __restrict__ status) {
@@ -760,7 +782,7 @@ gated_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
             lr = logf(static_cast<float>(__ldcg(pos + qg)) / static_cast<float>(__ldcg(rank + qg)));
             fi = 1.0f / (1.0f + c[h] * lr);
             fa = sm_scale * LOG2E_B * fi;
-            fb = softplus_b(g[h]) * LOG2E_B * fi;
+            fb = LOG2E_B * fi;  // multiplies the key's whole bias sum_i beta_i gls_ij
             fl = __ldcg(lse + static_cast<size_t>(qg) * Hq + h) * LOG2E_B;
         }
         float* xch = reinterpret_cast<float*>(smem + L::OFF_XCH);
@@ -791,10 +813,12 @@ gated_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
         // from the bf16 output; dtau = -sum_j dl l / tau cancels to a small number and would
         // amplify its rounding):  sum_j dl x = sum P dP x - D' sum P x.
         float aPdPt = 0.f, aPt = 0.f, aPdP = 0.f, aP = 0.f;
-        // gls of the next KV tile is loaded one tile ahead (its latency hides behind a tile of work)
+        // the bias sum_i beta_i gls_ij of the next KV tile's keys is loaded one tile ahead (its
+        // latency hides behind a tile of work)
+        const GateGains gw = gate_gains(gates, h);
         float gnext[BT / 32];
 #pragma unroll
-        for (int e = 0; e < BT / 32; ++e) gnext[e] = e * 32 + lane < Mb ? __ldcg(gls + seq0 + e * 32 + lane) : 0.f;
+        for (int e = 0; e < BT / 32; ++e) gnext[e] = e * 32 + lane < Mb ? gate_bias(gates, gw, seq0 + e * 32 + lane) : 0.f;
         for (int j = 0; ok && j < n_kv; ++j) {
             const int s = j & 1;
             // the tile's gls into this warp's own copy (only __syncwarp orders it)
@@ -805,7 +829,7 @@ gated_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
 #pragma unroll
                 for (int e = 0; e < BT / 32; ++e) {
                     const int key_local = (j + 1) * BT + e * 32 + lane;
-                    gnext[e] = key_local < Mb ? __ldcg(gls + seq0 + key_local) : 0.f;
+                    gnext[e] = key_local < Mb ? gate_bias(gates, gw, seq0 + key_local) : 0.f;
                 }
             }
             const bool diag = (j == n_kv - 1);
@@ -960,33 +984,46 @@ bwd_kv_reduce_kernel(const float* __restrict__ part_k, const float* __restrict__
 }
 
 // ---------------------------------------------------------------------------
-// The last step, one launch:
-//   blocks 0 .. Hq-1, head h:  dg_h = sigmoid(g_h) sum_j gls_j colsum[j, h]  (dbeta_h
-//                              = sum_ij G_ij gls_j, by keys) and
-//                              dc_h = sum_tiles tileT[., h]  (fixed order);
-//   the other blocks, per key: dgls_j = sum_h softplus(g_h) colsum[j, h] and
-//                              d score_j = dgls_j (1 - exp(gls_j)).
+// The last step, one launch, for gates i < n:
+//   blocks (i, h), i * Hq + h:  dg_ih = sigmoid(g_ih) sum_j gls_ij colsum[j, h]  (dbeta_ih
+//                               = sum_qj G_qj gls_ij, by keys); the blocks of gate 0 also
+//                               dc_h = sum_tiles tileT[., h]  (fixed order);
+//   the other blocks, per key:  dgls_ij = sum_h softplus(g_ih) colsum[j, h] and
+//                               d score_ij = dgls_ij (1 - exp(gls_ij)).
+struct BwdGateOut {
+    float* dgls[kMaxGates];
+    float* dscore[kMaxGates];  // entries may be null
+    float* dg[kMaxGates];
+};
+
 __global__ void __launch_bounds__(256)
-bwd_finish_kernel(const float* __restrict__ colsum, const float* __restrict__ tileT, const float* __restrict__ gls,
-                  const float* __restrict__ g, const int32_t* __restrict__ cu_kept, int B, int64_t M, int Hq,
-                  float* __restrict__ dgls, float* __restrict__ dscore, float* __restrict__ dg,
+bwd_finish_kernel(const float* __restrict__ colsum, const float* __restrict__ tileT, const GateSet gates,
+                  const int32_t* __restrict__ cu_kept, int B, int64_t M, int Hq, const BwdGateOut go,
                   float* __restrict__ dc) {
     // Waits for the dK/dV grid (colsum).  tileT comes from the dQ kernel, one launch
     // earlier: it is complete because every dK/dV CTA with work waits for the dQ kernel
     // before it finishes, and a non-empty batch has at least one such CTA.
     pdl_wait();
     pdl_trigger();
-    if (static_cast<int>(blockIdx.x) < Hq) {
-        const int h = blockIdx.x;
+    const int n = gates.n;
+    if (static_cast<int>(blockIdx.x) < n * Hq) {
+        const int gi = static_cast<int>(blockIdx.x) / Hq, h = static_cast<int>(blockIdx.x) % Hq;
+        // (a select chain, not gates.gls[gi]: a run-time index into the parameter block would
+        // copy it to local memory)
+        const float* gls = gi == 0 ? gates.gls[0] : (gi == 1 ? gates.gls[1] : (gi == 2 ? gates.gls[2] : gates.gls[3]));
+        const float* g = gi == 0 ? gates.g[0] : (gi == 1 ? gates.g[1] : (gi == 2 ? gates.g[2] : gates.g[3]));
+        float* dg = gi == 0 ? go.dg[0] : (gi == 1 ? go.dg[1] : (gi == 2 ? go.dg[2] : go.dg[3]));
         float e = 0.f, t = 0.f;
         // thread x takes keys x, x + 256, ... and tiles x, x + 256, ... (running tile number)
         for (int64_t j = threadIdx.x; j < M; j += 256) e = fmaf(__ldcg(gls + j), __ldcg(colsum + j * Hq + h), e);
-        int k = 0;
-        for (int b = 0; b < B; ++b) {
-            const int s0 = cu_kept[b], n_qt = (cu_kept[b + 1] - s0 + BT - 1) / BT;
-            for (int qt = 0; qt < n_qt; ++qt, ++k)
-                if ((k & 255) == static_cast<int>(threadIdx.x))
-                    t += __ldcg(tileT + (static_cast<size_t>(s0) + static_cast<size_t>(qt) * BT) * Hq + h);
+        if (gi == 0) {
+            int k = 0;
+            for (int b = 0; b < B; ++b) {
+                const int s0 = cu_kept[b], n_qt = (cu_kept[b + 1] - s0 + BT - 1) / BT;
+                for (int qt = 0; qt < n_qt; ++qt, ++k)
+                    if ((k & 255) == static_cast<int>(threadIdx.x))
+                        t += __ldcg(tileT + (static_cast<size_t>(s0) + static_cast<size_t>(qt) * BT) * Hq + h);
+            }
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
@@ -1006,16 +1043,25 @@ bwd_finish_kernel(const float* __restrict__ colsum, const float* __restrict__ ti
             const float st = ((red[1][0] + red[1][1]) + (red[1][2] + red[1][3])) +
                              ((red[1][4] + red[1][5]) + (red[1][6] + red[1][7]));
             dg[h] = se / (1.0f + expf(-g[h]));
-            dc[h] = st;
+            if (gi == 0) dc[h] = st;
         }
         return;
     }
-    const int64_t nb = static_cast<int64_t>(gridDim.x) - Hq;
-    for (int64_t j = static_cast<int64_t>(blockIdx.x - Hq) * blockDim.x + threadIdx.x; j < M; j += nb * blockDim.x) {
-        float acc = 0.f;
-        for (int h = 0; h < Hq; ++h) acc = fmaf(softplus_b(g[h]), __ldcg(colsum + j * Hq + h), acc);
-        dgls[j] = acc;
-        if (dscore) dscore[j] = acc * -expm1f(gls[j]);
+    const int64_t nb = static_cast<int64_t>(gridDim.x) - n * Hq;
+    for (int64_t j = static_cast<int64_t>(blockIdx.x - n * Hq) * blockDim.x + threadIdx.x; j < M;
+         j += nb * blockDim.x) {
+#pragma unroll 1
+        for (int gi = 0; gi < n; ++gi) {
+            const float* gls = gi == 0 ? gates.gls[0] : (gi == 1 ? gates.gls[1] : (gi == 2 ? gates.gls[2] : gates.gls[3]));
+            const float* g = gi == 0 ? gates.g[0] : (gi == 1 ? gates.g[1] : (gi == 2 ? gates.g[2] : gates.g[3]));
+            float* dgls = gi == 0 ? go.dgls[0] : (gi == 1 ? go.dgls[1] : (gi == 2 ? go.dgls[2] : go.dgls[3]));
+            float* dscore =
+                gi == 0 ? go.dscore[0] : (gi == 1 ? go.dscore[1] : (gi == 2 ? go.dscore[2] : go.dscore[3]));
+            float acc = 0.f;
+            for (int h = 0; h < Hq; ++h) acc = fmaf(softplus_b(g[h]), __ldcg(colsum + j * Hq + h), acc);
+            dgls[j] = acc;
+            if (dscore) dscore[j] = acc * -expm1f(__ldcg(gls + j));
+        }
     }
 }
 
@@ -1025,9 +1071,9 @@ inline int bwd_cluster_size(int grp) { return grp == 2 || grp == 4 || grp == 8 ?
 template <int HD>
 cudaError_t launch_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* out,
                        const uint16_t* dout, const float* lse, const int32_t* cu_kept, int B, int64_t M_total,
-                       int max_M, int Hq, int Hkv, const int32_t* pos, const int32_t* rank, const float* gls,
-                       const float* g, const float* c, float sm_scale, uint16_t* dq, uint16_t* dk, uint16_t* dv,
-                       float* dgls, float* dscore, float* dg, float* dc, void* ws, cudaStream_t st) {
+                       int max_M, int Hq, int Hkv, const int32_t* pos, const int32_t* rank, const GateSet& gates,
+                       const float* c, float sm_scale, uint16_t* dq, uint16_t* dk, uint16_t* dv,
+                       const BwdGateOut& gout, float* dc, void* ws, cudaStream_t st) {
     static std::atomic<uint64_t> set_dkv{0}, set_dq{0};
     if (cudaError_t e = ensure_smem_limit(gated_attn_bwd_dkv_kernel<HD>, DkvSmem<HD>::ALLOC, set_dkv);
         e != cudaSuccess)
@@ -1063,17 +1109,17 @@ cudaError_t launch_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
     // dq first: it forms each row's D = dout . out for its own use and leaves the exact
     // D' = sum_j P dP for the dK/dV kernel
     cudaError_t e = launch_pdl(gated_attn_bwd_dq_kernel<HD>, dim3(Hq, n_t, B), dim3(DQ_THREADS),
-                               static_cast<size_t>(DqSmem<HD>::ALLOC), st, tq, tk, tv, tdo, cu_kept, pos, rank, gls, g,
+                               static_cast<size_t>(DqSmem<HD>::ALLOC), st, tq, tk, tv, tdo, cu_kept, pos, rank, gates,
                                c, lse, out, fac, sm_scale, Hq, Hkv, n_t, dq, tileT, status);
     if (e != cudaSuccess) return e;
     if (cl > 1)
         e = launch_pdl_cluster(gated_attn_bwd_dkv_kernel<HD>, dim3(Hq, n_t, B), dim3(DKV_THREADS),
                                static_cast<size_t>(DkvSmem<HD>::ALLOC), st, static_cast<unsigned>(cl), tq, tk, tv, tdo,
-                               cu_kept, gls, g, static_cast<const float4*>(fac), sm_scale, Hq, Hkv, M_total, dk, dv,
+                               cu_kept, gates, static_cast<const float4*>(fac), sm_scale, Hq, Hkv, M_total, dk, dv,
                                part_k, part_v, colsum, status, cl);
     else
         e = launch_pdl(gated_attn_bwd_dkv_kernel<HD>, dim3(Hq, n_t, B), dim3(DKV_THREADS),
-                       static_cast<size_t>(DkvSmem<HD>::ALLOC), st, tq, tk, tv, tdo, cu_kept, gls, g,
+                       static_cast<size_t>(DkvSmem<HD>::ALLOC), st, tq, tk, tv, tdo, cu_kept, gates,
                        static_cast<const float4*>(fac), sm_scale, Hq, Hkv, M_total, dk, dv, part_k, part_v, colsum,
                        status, 0);
     if (e != cudaSuccess) return e;
@@ -1086,8 +1132,9 @@ cudaError_t launch_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
     }
     const int64_t kb = (M_total + 255) / 256;
     const int key_blocks = static_cast<int>(kb < sms * 4 ? kb : sms * 4);
-    return launch_pdl(bwd_finish_kernel, dim3(Hq + key_blocks), dim3(256), 0, st, static_cast<const float*>(colsum),
-                      static_cast<const float*>(tileT), gls, g, cu_kept, B, M_total, Hq, dgls, dscore, dg, dc);
+    return launch_pdl(bwd_finish_kernel, dim3(gates.n * Hq + key_blocks), dim3(256), 0, st,
+                      static_cast<const float*>(colsum), static_cast<const float*>(tileT), gates, cu_kept, B, M_total,
+                      Hq, gout, dc);
 }
 
 }  // namespace
@@ -1107,14 +1154,21 @@ cudaError_t launch_gated_attention_backward(const uint16_t* q, const uint16_t* k
                                             const uint16_t* out, const uint16_t* dout, const float* lse,
                                             const int32_t* cu_kept, int B, int64_t M_total, int max_M, int Hq,
                                             int Hkv, int d, const int32_t* pos, const int32_t* rank,
-                                            const float* gls, const float* g, const float* c, float sm_scale,
-                                            uint16_t* dq, uint16_t* dk, uint16_t* dv, float* dgls, float* dscore,
-                                            float* dg, float* dc, void* ws, cudaStream_t st) {
+                                            const GateSet& gates, const float* c, float sm_scale, uint16_t* dq,
+                                            uint16_t* dk, uint16_t* dv, float* const* dgls, float* const* dscore,
+                                            float* const* dg, float* dc, void* ws, cudaStream_t st) {
+    if (gates.n < 1 || gates.n > kMaxGates) return cudaErrorInvalidValue;
+    BwdGateOut go{};
+    for (int i = 0; i < gates.n; ++i) {
+        go.dgls[i] = dgls[i];
+        go.dscore[i] = dscore ? dscore[i] : nullptr;
+        go.dg[i] = dg[i];
+    }
     if (d == 64)
-        return launch_bwd<64>(q, k, v, out, dout, lse, cu_kept, B, M_total, max_M, Hq, Hkv, pos, rank, gls, g, c,
-                              sm_scale, dq, dk, dv, dgls, dscore, dg, dc, ws, st);
-    return launch_bwd<128>(q, k, v, out, dout, lse, cu_kept, B, M_total, max_M, Hq, Hkv, pos, rank, gls, g, c,
-                           sm_scale, dq, dk, dv, dgls, dscore, dg, dc, ws, st);
+        return launch_bwd<64>(q, k, v, out, dout, lse, cu_kept, B, M_total, max_M, Hq, Hkv, pos, rank, gates, c,
+                              sm_scale, dq, dk, dv, go, dc, ws, st);
+    return launch_bwd<128>(q, k, v, out, dout, lse, cu_kept, B, M_total, max_M, Hq, Hkv, pos, rank, gates, c,
+                           sm_scale, dq, dk, dv, go, dc, ws, st);
 }
 
 }  // namespace tg

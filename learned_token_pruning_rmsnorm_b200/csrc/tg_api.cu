@@ -388,23 +388,28 @@ size_t tg_gated_attention_backward_workspace_size(int64_t M_total, int Hq, int H
     return tg::attention_backward_workspace_bytes(M_total, Hq, Hkv, d);
 }
 
-tg_status tg_gated_attention_backward(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* out,
-                                      const uint16_t* dout, const float* lse, const int32_t* cu_kept, int B,
-                                      int64_t M_total, int max_M, int Hq, int Hkv, int d, const int32_t* pos,
-                                      const int32_t* rank, const float* gls, const float* g, const float* c,
-                                      float sm_scale, uint16_t* dq, uint16_t* dk, uint16_t* dv, float* dgls,
-                                      float* dscore, float* dg, float* dc, void* ws, size_t ws_bytes,
-                                      tg_stream_t stream) {
-    NvtxRange nvtx_range("tg_gated_attention_backward");
+}  // extern "C"
+
+namespace {
+
+tg_status do_backward(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* out,
+                      const uint16_t* dout, const float* lse, const int32_t* cu_kept, int B, int64_t M_total, int max_M,
+                      int Hq, int Hkv, int d, const int32_t* pos, const int32_t* rank, const tg::GateSet& gates,
+                      const float* c, float sm_scale, uint16_t* dq, uint16_t* dk, uint16_t* dv, float* const* dgls,
+                      float* const* dscore, float* const* dg, float* dc, void* ws, size_t ws_bytes,
+                      cudaStream_t stream) {
     TG_REQUIRE(B >= 0 && M_total >= 0 && max_M >= 0, "negative size");
     if (tg_status s = check_attn_shape(Hq, Hkv, d)) return s;
     TG_SUPPORT(d == 64 || d == 128, "the backward supports head_dim 64 and 128, not %d", d);
     TG_REQUIRE(sm_scale > 0.f, "sm_scale must be positive");
+    TG_SUPPORT(gates.n >= 1 && gates.n <= tg::kMaxGates, "n_gates=%d must be in [1, %d]", gates.n, tg::kMaxGates);
     if (B == 0 || M_total == 0) return TG_OK;
     TG_REQUIRE(max_M > 0, "max_M must bound the longest sequence");
-    TG_REQUIRE(q && k && v && out && dout && lse && cu_kept && pos && rank && gls && g && c && dq && dk && dv &&
-                   dgls && dg && dc && ws,
+    TG_REQUIRE(q && k && v && out && dout && lse && cu_kept && pos && rank && c && dq && dk && dv && dgls && dg &&
+                   dc && ws,
                "null pointer argument");
+    for (int i = 0; i < gates.n; ++i)
+        TG_REQUIRE(gates.gls[i] && gates.g[i] && dgls[i] && dg[i], "null gls, g, dgls or dg of gate %d", i);
     TG_REQUIRE(aligned16(q) && aligned16(k) && aligned16(v) && aligned16(out) && aligned16(dout) && aligned16(dq) &&
                    aligned16(dk) && aligned16(dv),
                "q, k, v, out, dout, dq, dk and dv must be 16-byte aligned");
@@ -413,9 +418,49 @@ tg_status tg_gated_attention_backward(const uint16_t* q, const uint16_t* k, cons
     TG_REQUIRE(ws_bytes >= need, "ws holds %zu bytes, the backward needs %zu", ws_bytes, need);
     if (tg_status s = check_device()) return s;
     return cuda_status(tg::launch_gated_attention_backward(q, k, v, out, dout, lse, cu_kept, B, M_total, max_M, Hq,
-                                                           Hkv, d, pos, rank, gls, g, c, sm_scale, dq, dk, dv, dgls,
+                                                           Hkv, d, pos, rank, gates, c, sm_scale, dq, dk, dv, dgls,
                                                            dscore, dg, dc, ws, stream),
                        "tg_gated_attention_backward launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+tg_status tg_gated_attention_backward(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* out,
+                                      const uint16_t* dout, const float* lse, const int32_t* cu_kept, int B,
+                                      int64_t M_total, int max_M, int Hq, int Hkv, int d, const int32_t* pos,
+                                      const int32_t* rank, const float* gls, const float* g, const float* c,
+                                      float sm_scale, uint16_t* dq, uint16_t* dk, uint16_t* dv, float* dgls,
+                                      float* dscore, float* dg, float* dc, void* ws, size_t ws_bytes,
+                                      tg_stream_t stream) {
+    NvtxRange nvtx_range("tg_gated_attention_backward");
+    float* dgl[1] = {dgls};
+    float* dsc[1] = {dscore};
+    float* dgg[1] = {dg};
+    return do_backward(q, k, v, out, dout, lse, cu_kept, B, M_total, max_M, Hq, Hkv, d, pos, rank,
+                       tg::single_gate(gls, g), c, sm_scale, dq, dk, dv, dgl, dsc, dgg, dc, ws, ws_bytes, stream);
+}
+
+tg_status tg_gated_attention_backward_gates(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                            const uint16_t* out, const uint16_t* dout, const float* lse,
+                                            const int32_t* cu_kept, int B, int64_t M_total, int max_M, int Hq,
+                                            int Hkv, int d, const int32_t* pos, const int32_t* rank, int n_gates,
+                                            const float* const* gls, const float* const* g, const float* c,
+                                            float sm_scale, uint16_t* dq, uint16_t* dk, uint16_t* dv,
+                                            float* const* dgls, float* const* dscore, float* const* dg, float* dc,
+                                            void* ws, size_t ws_bytes, tg_stream_t stream) {
+    NvtxRange nvtx_range("tg_gated_attention_backward_gates");
+    TG_SUPPORT(n_gates >= 1 && n_gates <= tg::kMaxGates, "n_gates=%d must be in [1, %d]", n_gates, tg::kMaxGates);
+    TG_REQUIRE(gls && g && dgls && dg, "null gate arrays");
+    tg::GateSet gates{};
+    gates.n = n_gates;
+    for (int i = 0; i < n_gates; ++i) {
+        gates.gls[i] = gls[i];
+        gates.g[i] = g[i];
+    }
+    return do_backward(q, k, v, out, dout, lse, cu_kept, B, M_total, max_M, Hq, Hkv, d, pos, rank, gates, c,
+                       sm_scale, dq, dk, dv, dgls, dscore, dg, dc, ws, ws_bytes, stream);
 }
 
 tg_status tg_next_gate_span(const int32_t* h_span, const int32_t* h_k, int B, int32_t* h_span_next) {

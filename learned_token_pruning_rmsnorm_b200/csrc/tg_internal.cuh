@@ -184,13 +184,15 @@ size_t attention_workspace_bytes(int B, int max_M, int Hq, int Hkv, int d);
 // attention_backward_workspace_bytes(M_total, Hq, Hkv, d) bytes (4 fp32 per row and head,
 // plus fp32 partial dK and dV per query head of a GQA group when the group has two or more).
 size_t attention_backward_workspace_bytes(int64_t M_total, int Hq, int Hkv, int d);
+// gates.n (1..kMaxGates) gates: dgls[i], dg[i] per gate (device arrays), dscore may be a
+// null array or hold null entries.
 cudaError_t launch_gated_attention_backward(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                             const uint16_t* out, const uint16_t* dout, const float* lse,
                                             const int32_t* cu_kept, int B, int64_t M_total, int max_M, int Hq,
                                             int Hkv, int d, const int32_t* pos, const int32_t* rank,
-                                            const float* gls, const float* g, const float* c, float sm_scale,
-                                            uint16_t* dq, uint16_t* dk, uint16_t* dv, float* dgls, float* dscore,
-                                            float* dg, float* dc, void* ws, cudaStream_t st);
+                                            const GateSet& gates, const float* c, float sm_scale, uint16_t* dq,
+                                            uint16_t* dk, uint16_t* dv, float* const* dgls, float* const* dscore,
+                                            float* const* dg, float* dc, void* ws, cudaStream_t st);
 int64_t units_below_host(int x, int C);
 
 cudaError_t launch_selftest_wait(int64_t timeout_ns, cudaStream_t st);

@@ -207,10 +207,10 @@ def gated_attention_backward(q_bits, k_bits, v_bits, cu_kept, pos, rank, gls_f32
     (AI summary, "Future Directions"): gls_f32 [G, M] and g [G, Hq] give dgls
     [G, M] and dg [G, Hq], gate i's bias term being softplus(g[i, h]) gls[i, j].
 
-    With the kept rows' gate scores (scores [M] fp32, the s_j whose
-    logsigmoid is gls_j) and the rows the gate could prune (prunable [M]
-    bool), the one-gate form also returns dscore [M]: the gradient that reaches
-    the gate's score through the bias (AI summary, "Key Contributions" 2: the
+    With the kept rows' gate scores (scores [M] or [G, M] fp32, the s_j whose
+    logsigmoid is gls_j) and the rows the gates could prune (prunable [M]
+    bool), it also returns dscore ([M] or [G, M]): the gradient that reaches
+    each gate's score through the bias (AI summary, "Key Contributions" 2: the
     bias on the logits carries the task loss back to the scoring network).
     Since gls_j = logsigmoid(s_j), d gls_j / d s_j = sigmoid(-s_j), taken here
     from the score itself; rows the gate cannot prune carry no bias and get 0."""
@@ -238,14 +238,16 @@ def gated_attention_backward(q_bits, k_bits, v_bits, cu_kept, pos, rank, gls_f32
     _load().oracle_gated_attention_backward(qp, kp, vp_, cup, len(cu) - 1, Hq, Hkv, d, pop, rap, glp, gap, cap,
                                             float(sm_scale), gop, vp(out["dq"]), vp(out["dk"]), vp(out["dv"]),
                                             vp(out["dgls"]), vp(out["dg"]), vp(out["dc"]), G)
-    if one_gate:
-        out["dgls"], out["dg"] = out["dgls"][0], out["dg"][0]
-    if scores is not None and one_gate:
-        s64 = np.asarray(scores, dtype=np.float64).reshape(M)
+    if scores is not None:
+        s64 = np.asarray(scores, dtype=np.float64).reshape(G, M)
         mask = np.ones(M, dtype=bool) if prunable is None else np.asarray(prunable, dtype=bool).reshape(M)
         # sigmoid(-s) = exp(-log(1 + e^s)), finite for every s
-        sig_neg = np.exp(-np.logaddexp(0.0, np.where(mask, s64, 0.0)))
-        out["dscore"] = np.where(mask, out["dgls"] * sig_neg, 0.0)
+        sig_neg = np.exp(-np.logaddexp(0.0, np.where(mask[None, :], s64, 0.0)))
+        out["dscore"] = np.where(mask[None, :], out["dgls"] * sig_neg, 0.0)
+    if one_gate:
+        out["dgls"], out["dg"] = out["dgls"][0], out["dg"][0]
+        if "dscore" in out:
+            out["dscore"] = out["dscore"][0]
     return out
 
 

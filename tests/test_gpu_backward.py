@@ -137,3 +137,44 @@ def test_backward_refuses_head_dim_256(tg):
     cs = _rand_case(10, [64], 2, 1, 256)
     with pytest.raises(tg.TokenGateError):
         _gpu_backward(tg, cs)
+
+
+@pytest.mark.parametrize("seed,seqlens,Hq,Hkv,d,n_gates", [(11, [300, 129], 4, 2, 128, 2), (12, [260], 8, 2, 64, 4),
+                                                           (13, [200, 77], 3, 1, 64, 3)])
+def test_backward_with_several_gates_matches_oracle(tg, seed, seqlens, Hq, Hkv, d, n_gates):
+    """Several gate modules: the forward's logits carry sum_i softplus(g_i) gls_i; the
+    backward returns each gate's dgls, dscore and dg (R24 bars per gate) and the same dq,
+    dk, dv, dc bars as one gate."""
+    cs = _rand_case(seed, seqlens, Hq, Hkv, d)
+    rng = np.random.default_rng(seed + 100)
+    M = sum(seqlens)
+    scores, gls = [cs["s"]], [cs["gls"]]
+    for _ in range(n_gates - 1):
+        sc = (2 * rng.standard_normal(M)).astype(np.float32)
+        x = np.where(cs["prunable"], np.minimum(sc, 0) - np.log1p(np.exp(-np.abs(sc.astype(np.float64)))), 0.0)
+        scores.append(sc)
+        gls.append(x.astype(np.float32))
+    gains = [cs["g"]] + [rng.standard_normal(Hq).astype(np.float32) for _ in range(n_gates - 1)]
+    cu = cs["cu"]
+    max_M = int(np.max(np.diff(cu)))
+    q, k, v = H.bf16_dev(cs["q"]), H.bf16_dev(cs["k"]), H.bf16_dev(cs["v"])
+    pos, rank = H.i32_dev(cs["pos"]), H.i32_dev(cs["rank"])
+    gls_d, g_d, c = [H.f32_dev(x) for x in gls], [H.f32_dev(x) for x in gains], H.f32_dev(cs["c"])
+    out, lse = tg.tg_gated_attention_gates(q, k, v, cu, max_M, pos, rank, gls_d, g_d, c, want_lse=True)
+    res = tg.tg_gated_attention_backward_gates(q, k, v, out, H.bf16_dev(cs["dout"]), lse, cu, max_M, pos, rank,
+                                               gls_d, g_d, c)
+    torch.cuda.synchronize()
+    ref = oracle.gated_attention_backward(cs["q"], cs["k"], cs["v"], cu, cs["pos"], cs["rank"], np.stack(gls),
+                                          np.stack(gains), cs["c"], bf16_bits_to_f32(cs["dout"]).astype(np.float64),
+                                          scores=np.stack(scores), prunable=cs["prunable"])
+    for key in ("dq", "dk", "dv"):
+        got = res[key].float().cpu().numpy()
+        err, scale = np.abs(got - ref[key]), np.abs(ref[key])
+        assert err.max() <= GRAD_MAX_REL * scale.max(), key
+        assert err.mean() <= GRAD_MEAN_REL * scale.mean(), key
+    got_dc = res["dc"].cpu().numpy()
+    assert np.abs(got_dc - ref["dc"]).max() <= SUM_MAX_REL * np.abs(ref["dc"]).max()
+    for i in range(n_gates):
+        for key in ("dgls", "dscore", "dg"):
+            got = res[key][i].cpu().numpy()
+            assert np.abs(got - ref[key][i]).max() <= SUM_MAX_REL * np.abs(ref[key][i]).max(), (key, i)
