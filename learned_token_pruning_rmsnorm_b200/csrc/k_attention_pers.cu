@@ -135,11 +135,12 @@ __device__ unsigned long long g_pers_pipe[16 * 64];  // clock64 of pipeline poin
         if (blockIdx.x == 0 && (j) < 64) g_pers_pipe[(point) * 64 + (j)] = clock64();         \
     } while (0)
 __device__ unsigned long long g_pers_trace[1024 * 16];
-__device__ unsigned long long g_pers_units[1024 * 4 * 4];  // per CTA, first 4 units: start, loop end, epi end, info
+// per CTA, first 4 units: ring read, loop end, O full, epilogue end, info, arrival, S0 seen
+__device__ unsigned long long g_pers_units[1024 * 4 * 8];
 #define PT_UNIT(uc, slot, val)                                                                  \
     do {                                                                                        \
         if (threadIdx.x == 0 && blockIdx.x < 1024 && (uc) < 4)                                  \
-            g_pers_units[(blockIdx.x * 4 + (uc)) * 4 + (slot)] = (val);                         \
+            g_pers_units[(blockIdx.x * 4 + (uc)) * 8 + (slot)] = (val);                         \
     } while (0)
 #define PT_STAMP(slot, cond)                                                             \
     do {                                                                                 \
@@ -528,7 +529,7 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             Unit U{};
             decode_unit(unit, pairs, B, cu_kept, kv_chunk, &U, M_total, status);
             PT_UNIT(uc, 0, globaltimer());
-            PT_UNIT(uc, 3, static_cast<unsigned long long>(U.n_kv) | (static_cast<unsigned long long>(U.split) << 8) |
+            PT_UNIT(uc, 4, static_cast<unsigned long long>(U.n_kv) | (static_cast<unsigned long long>(U.split) << 8) |
                                (static_cast<unsigned long long>(U.qt) << 24) |
                                (static_cast<unsigned long long>(U.chunk) << 40) |
                                (static_cast<unsigned long long>(U.pair) << 48));
@@ -562,6 +563,7 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     break;
                 }
                 PT_STAMP(5, uc == 0 && j == 0 && threadIdx.x == 0);
+                if (j == 0) PT_UNIT(uc, 6, globaltimer());
 #ifdef TG_TRACE
                 if (uc == 0 && j == 0 && threadIdx.x == 0 && blockIdx.x < 1024)
                     g_pers_trace[blockIdx.x * 16 + 13] = U.n_kv | (U.split ? 1000 : 0) | (U.qt << 16);
@@ -648,6 +650,7 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             PT_UNIT(uc, 1, globaltimer());
             if (ok) ok = mbar_wait_warp(bar(T_O_FULL + h), uc & 1, abort_flag, status, TG_WHERE_SOFTMAX);
             PT_STAMP(7, uc == 0 && threadIdx.x == 0);
+            PT_UNIT(uc, 2, globaltimer());
             if (bar_red_or(bid, 128, !ok)) break;
             tc_fence_after();
             const float inv_l = 1.0f / l_run;
@@ -778,7 +781,8 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             // (that product waits for this warpgroup's next P arrival)
             tc_fence_before();
             PT_STAMP(8, uc == 0 && threadIdx.x == 0);
-            PT_UNIT(uc, 2, globaltimer() | (static_cast<unsigned long long>(U.split ? s_arr[h] + 1 : 0) << 60));
+            PT_UNIT(uc, 3, globaltimer());
+            PT_UNIT(uc, 5, static_cast<unsigned long long>(U.split ? s_arr[h] + 1 : 0));
             ++uc;
         }
 #ifdef TG_TRACE
