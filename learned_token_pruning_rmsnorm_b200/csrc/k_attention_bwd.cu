@@ -246,24 +246,31 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
         if (lane == 0) {
             constexpr uint32_t idesc_s = idesc_bf16_f32(BT, 64, false);
             constexpr uint32_t idesc_acc = idesc_bf16_f32(BT, HD, true);
+            // Matrix descriptors are built once per stage; an operand at a byte offset is the
+            // same descriptor with offset / 16 added to its start-address field (shared-memory
+            // addresses stay below 2^18, so the 14-bit field never carries).
+            const uint64_t kd = smem_desc_sw128(sK, 16, 1024), vd = smem_desc_sw128(sV, 16, 1024);
+            const uint64_t qd0 = smem_desc_sw128(sQ, 16, 1024), qd1 = smem_desc_sw128(sQ + L::TILE, 16, 1024);
+            const uint64_t dd0 = smem_desc_sw128(sDO, 16, 1024), dd1 = smem_desc_sw128(sDO + L::TILE, 16, 1024);
+            const uint64_t qm0 = smem_desc_sw128(sQ, BT * 128, 1024), qm1 = smem_desc_sw128(sQ + L::TILE, BT * 128, 1024);
+            const uint64_t dm0 = smem_desc_sw128(sDO, BT * 128, 1024),
+                           dm1 = smem_desc_sw128(sDO + L::TILE, BT * 128, 1024);
             // Half step u: query tile u >> 1, queries 64 (u & 1) .. +63 (64 rows = 8 KB into
             // each swizzled box of the stage), TMEM buffer u & 1.
             auto issue_sdp = [&](int u) {
                 const int hb = u & 1, s = (u >> 1) & 1;
                 const uint32_t tb = tmem + hb * 128;
+                const uint64_t qb = (s ? qd1 : qd0) + ((hb * 64 * 128) >> 4);
+                const uint64_t db = (s ? dd1 : dd0) + ((hb * 64 * 128) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * (BT * 128) + (kk & 3) * 32;
-                    mma_bf16_ss(tb, smem_desc_sw128(sK + off, 16, 1024),
-                                smem_desc_sw128(sQ + s * L::TILE + hb * 64 * 128 + off, 16, 1024), idesc_s,
-                                kk > 0 ? 1u : 0u);
+                    const uint32_t off = ((kk >> 2) * (BT * 128) + (kk & 3) * 32) >> 4;
+                    mma_bf16_ss(tb, kd + off, qb + off, idesc_s, kk > 0 ? 1u : 0u);
                 }
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * (BT * 128) + (kk & 3) * 32;
-                    mma_bf16_ss(tb + 64, smem_desc_sw128(sV + off, 16, 1024),
-                                smem_desc_sw128(sDO + s * L::TILE + hb * 64 * 128 + off, 16, 1024), idesc_s,
-                                kk > 0 ? 1u : 0u);
+                    const uint32_t off = ((kk >> 2) * (BT * 128) + (kk & 3) * 32) >> 4;
+                    mma_bf16_ss(tb + 64, vd + off, db + off, idesc_s, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(bar(D_SDP_FULL + hb));
             };
@@ -272,16 +279,16 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
             auto issue_acc = [&](int u) {
                 const int hb = u & 1, s = (u >> 1) & 1;
                 const uint32_t tb = tmem + hb * 128;
+                const uint64_t db = (s ? dm1 : dm0) + ((hb * 64 * 128) >> 4);
+                const uint64_t qb = (s ? qm1 : qm0) + ((hb * 64 * 128) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16_ts(tDV, tb + kk * 8,
-                                smem_desc_sw128(sDO + s * L::TILE + (hb * 64 + kk * 16) * 128, BT * 128, 1024),
-                                idesc_acc, (u > 0 || kk > 0) ? 1u : 0u);
+                    mma_bf16_ts(tDV, tb + kk * 8, db + ((kk * 16 * 128) >> 4), idesc_acc,
+                                (u > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16_ts(tDK, tb + 64 + kk * 8,
-                                smem_desc_sw128(sQ + s * L::TILE + (hb * 64 + kk * 16) * 128, BT * 128, 1024),
-                                idesc_acc, (u > 0 || kk > 0) ? 1u : 0u);
+                    mma_bf16_ts(tDK, tb + 64 + kk * 8, qb + ((kk * 16 * 128) >> 4), idesc_acc,
+                                (u > 0 || kk > 0) ? 1u : 0u);
                 if (hb == 1) mma_commit(bar(D_QD_EMPTY + s));  // the stage is no longer read
             };
             const int n_u = 2 * nq;
@@ -696,22 +703,25 @@ gated_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
             // tensor core computes half u while the compute warps turn half u - 1 into G; the
             // buffer S(u) overwrites last held G(u - 2), which dQ(u - 2) -- issued earlier by this
             // thread, so executed earlier -- has read.
+            // Descriptors built once, as in the dK/dV kernel.
+            const uint64_t qd = smem_desc_sw128(sQ, 16, 1024), dd = smem_desc_sw128(sDO, 16, 1024);
+            const uint64_t kd0 = smem_desc_sw128(sK, 16, 1024), kd1 = smem_desc_sw128(sK + L::TILE, 16, 1024);
+            const uint64_t vd0 = smem_desc_sw128(sV, 16, 1024), vd1 = smem_desc_sw128(sV + L::TILE, 16, 1024);
+            const uint64_t km0 = smem_desc_sw128(sK, BT * 128, 1024), km1 = smem_desc_sw128(sK + L::TILE, BT * 128, 1024);
             auto issue_sdp = [&](int u) {
                 const int hb = u & 1, s = (u >> 1) & 1;
                 const uint32_t tb = tmem + hb * 128;
+                const uint64_t kb = (s ? kd1 : kd0) + ((hb * 64 * 128) >> 4);
+                const uint64_t vb = (s ? vd1 : vd0) + ((hb * 64 * 128) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * (BT * 128) + (kk & 3) * 32;
-                    mma_bf16_ss(tb, smem_desc_sw128(sQ + off, 16, 1024),
-                                smem_desc_sw128(sK + s * L::TILE + hb * 64 * 128 + off, 16, 1024), idesc_s,
-                                kk > 0 ? 1u : 0u);
+                    const uint32_t off = ((kk >> 2) * (BT * 128) + (kk & 3) * 32) >> 4;
+                    mma_bf16_ss(tb, qd + off, kb + off, idesc_s, kk > 0 ? 1u : 0u);
                 }
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * (BT * 128) + (kk & 3) * 32;
-                    mma_bf16_ss(tb + 64, smem_desc_sw128(sDO + off, 16, 1024),
-                                smem_desc_sw128(sV + s * L::TILE + hb * 64 * 128 + off, 16, 1024), idesc_s,
-                                kk > 0 ? 1u : 0u);
+                    const uint32_t off = ((kk >> 2) * (BT * 128) + (kk & 3) * 32) >> 4;
+                    mma_bf16_ss(tb + 64, dd + off, vb + off, idesc_s, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(bar(Q_SDP_FULL + hb));
                 if (hb == 1) mma_commit(bar(Q_V_EMPTY + s));  // V(tile) is no longer read
@@ -719,11 +729,11 @@ gated_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
             // dQ += G(u) K(half of u): A from TMEM (16 keys = 8 columns per k-step), B the K rows MN-major
             auto issue_dq = [&](int u) {
                 const int hb = u & 1, s = (u >> 1) & 1;
+                const uint64_t kb = (s ? km1 : km0) + ((hb * 64 * 128) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16_ts(tDQ, tmem + hb * 128 + kk * 8,
-                                smem_desc_sw128(sK + s * L::TILE + (hb * 64 + kk * 16) * 128, BT * 128, 1024),
-                                idesc_acc, (u > 0 || kk > 0) ? 1u : 0u);
+                    mma_bf16_ts(tDQ, tmem + hb * 128 + kk * 8, kb + ((kk * 16 * 128) >> 4), idesc_acc,
+                                (u > 0 || kk > 0) ? 1u : 0u);
                 if (hb == 1) mma_commit(bar(Q_K_EMPTY + s));  // K(tile) is no longer read
             };
             const int n_u = 2 * n_kv;
