@@ -725,20 +725,20 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                         atomicAdd(cnt, 1);  // publish
                     }
                 } else {
+                    // The acquire load (thread 0; the others follow through the barrier) makes
+                    // the other chunk's partial visible; it returns at once when that chunk had
+                    // published before this one arrived (arrival value 2).
                     if (r == 0) {
                         int ready = 1;
-                        if (arr == 1) {
-                            const uint64_t t0 = globaltimer();
-                            while (*reinterpret_cast<volatile int*>(cnt) < 3) {
-                                if (globaltimer() - t0 > TG_WAIT_TIMEOUT_NS) {
-                                    *abort_flag = 1;
-                                    atomicOr(status, TG_DEVICE_TIMEOUT | TG_WHERE_SOFTMAX);
-                                    ready = 0;
-                                    break;
-                                }
+                        const uint64_t t0 = globaltimer();
+                        while (ld_acquire_gpu(cnt) < 3) {
+                            if (globaltimer() - t0 > TG_WAIT_TIMEOUT_NS) {
+                                *abort_flag = 1;
+                                atomicOr(status, TG_DEVICE_TIMEOUT | TG_WHERE_SOFTMAX);
+                                ready = 0;
+                                break;
                             }
                         }
-                        asm volatile("fence.acq_rel.gpu;" ::: "memory");
                         s_arr[h] = ready;
                     }
                     named_bar_sync(bid, 128);
@@ -754,15 +754,32 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     const float e_me = ex2_approx(my_lse - mx), e_ot = ex2_approx(other_lse - mx);
                     const float inv_w = 1.0f / (e_me + e_ot);
                     const float w_me = e_me * inv_w, w_ot = e_ot * inv_w;
+                    // The other partial's next 32 columns are loaded while this 32 are merged, so
+                    // the loads' round trips to L2 overlap (head_dim 128; at 64 each chunk loads
+                    // its own, which keeps that instance free of spills).
+                    constexpr bool kAhead = HD > 64;
+                    uint32_t pw[16], pn[16];
+                    if (kAhead && ready) {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) pn[e] = __ldcg(pt + e * BM);
+                    }
 #pragma unroll
                     for (int ch = 0; ch < HD / 32; ++ch) {
+                        if (kAhead) {
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) pw[e] = pn[e];
+                            if (ready && ch + 1 < HD / 32) {
+#pragma unroll
+                                for (int e = 0; e < 16; ++e) pn[e] = __ldcg(pt + ((ch + 1) * 16 + e) * BM);
+                            }
+                        }
                         float o[32];
                         tmem_ld32(tO + ch * 32, o);
                         tmem_wait_ld();
                         if (ready) {
 #pragma unroll
                             for (int e = 0; e < 16; ++e) {
-                                const uint32_t w = __ldcg(pt + (ch * 16 + e) * BM);
+                                const uint32_t w = kAhead ? pw[e] : __ldcg(pt + (ch * 16 + e) * BM);
                                 const uint32_t mine = pack_bf16x2(o[2 * e] * inv_l, o[2 * e + 1] * inv_l);
                                 o[2 * e] = __fadd_rn(__fmul_rn(w_me, __uint_as_float(mine << 16)),
                                                      __fmul_rn(w_ot, __uint_as_float(w << 16)));

@@ -36,6 +36,14 @@ __device__ __forceinline__ float ldg_early(const float* p) {
 }
 
 // max of three floats (one instruction on sm_100)
+// Load with acquire semantics at GPU scope: reads that follow it (in this thread, and in
+// threads that pass a CTA barrier after it) see every write released before the value read.
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 __device__ __forceinline__ float max3f(float a, float b, float c) {
     float d;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
