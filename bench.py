@@ -394,6 +394,27 @@ def measure_next_rows(tg, dev, st, flush, main, peaks, reps=10):
     res["f4_four_gates_attention"] = {"workload": f"{wm.name}: M={main['M']}, 4 gates", "us": us,
                                       "tflops": fl / (us * 1e-6) / 1e12, "one_gate_us": us1,
                                       "vs_one_gate": us / us1}
+    # the key bias's cost: the same attention with gls = g = c = NULL (ordinary causal
+    # attention, no bias k-step, tau = 1), against the gated call in the same kernel (the
+    # persistent one, which serves both) and against the default gated call
+    us_plain = time_device_us(check(lambda: lib.tg_gated_attention(*common, None, None, None, sm, out.data_ptr(),
+                                                                   None, ws_p, ws_n, sh_now())), st, flush, reps)
+    old_env = os.environ.get("TG_ATTENTION_KERNEL")
+    os.environ["TG_ATTENTION_KERNEL"] = "persistent"
+    try:
+        nws = int(lib.tg_gated_attention_workspace_size(wm.B, main["max_M"], wm.Hq, wm.Hkv, wm.d))
+        assert nws <= ws_n
+        us_gp = time_device_us(check(lambda: lib.tg_gated_attention(*common, bufs.gls.data_ptr(), L0["g"].data_ptr(),
+                                                                    L0["c"].data_ptr(), sm, out.data_ptr(), None,
+                                                                    ws_p, ws_n, sh_now())), st, flush, reps)
+    finally:
+        if old_env is None:
+            os.environ.pop("TG_ATTENTION_KERNEL", None)
+        else:
+            os.environ["TG_ATTENTION_KERNEL"] = old_env
+    res["m6_key_bias_overhead"] = {"workload": f"{wm.name}: M={main['M']}, one gate vs none",
+                                   "plain_us": us_plain, "gated_same_kernel_us": us_gp, "gated_default_us": us1,
+                                   "same_kernel_ratio": us_gp / us_plain, "default_ratio": us1 / us_plain}
     # f1 (training): backward of the gated attention on the main workload, from the
     # forward's output and log-sum-exp
     lse = torch.empty((main["M"], wm.Hq), dtype=torch.float32, device=dev)

@@ -178,6 +178,11 @@ tg_status tg_compact(const uint16_t* hidden, const float* scores, const uint8_t*
  * zero-filled before its first use; every call leaves it zero-filled again.
  * Calls that share one ws must not run concurrently.  With ws == NULL the
  * attention runs unsplit (same results, less balanced for small M).
+ * Kernel choice (even GQA groups, d <= 128, ws given): one CTA per unit of
+ * work for a single sequence (B == 1), persistent CTAs that take units from
+ * a counter in ws for a batch; the environment variable TG_ATTENTION_KERNEL
+ * set to "persistent" or "per_unit" overrides it per call (the two give the
+ * same results within rounding; the workspace size may change with it).
  */
 tg_status tg_gated_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* cu_kept,
                              int B, int64_t M_total, int max_M, int Hq, int Hkv, int d, const int32_t* pos,

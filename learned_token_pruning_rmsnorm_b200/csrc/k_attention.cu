@@ -27,6 +27,8 @@
 // on top of plain attention.
 
 #include <algorithm>
+#include <cstdlib>
+#include <cstring>
 #include <functional>
 #include <map>
 #include <mutex>
@@ -997,20 +999,20 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     atomicAdd(cnt, 1);  // publish
                 }
             } else if (arr > 0) {
+                // The acquire load (thread 0; the others follow through the barrier) makes the
+                // other chunk's partial visible; it returns at once when that chunk had published
+                // before this one arrived (arrival value 2).
                 if (threadIdx.x == 0) {
                     int ready = 1;
-                    if (arr == 1) {
-                        const uint64_t t0 = globaltimer();
-                        while (*reinterpret_cast<volatile int*>(cnt) < 3) {
-                            if (globaltimer() - t0 > TG_WAIT_TIMEOUT_NS) {
-                                *abort_flag = 1;
-                                atomicOr(status, TG_DEVICE_TIMEOUT | TG_WHERE_SOFTMAX);
-                                ready = 0;
-                                break;
-                            }
+                    const uint64_t t0 = globaltimer();
+                    while (ld_acquire_gpu(cnt) < 3) {
+                        if (globaltimer() - t0 > TG_WAIT_TIMEOUT_NS) {
+                            *abort_flag = 1;
+                            atomicOr(status, TG_DEVICE_TIMEOUT | TG_WHERE_SOFTMAX);
+                            ready = 0;
+                            break;
                         }
                     }
-                    asm volatile("fence.acq_rel.gpu;" ::: "memory");
                     *s_last = ready;
                 }
                 asm volatile("bar.sync 1, 256;" ::: "memory");
@@ -1098,7 +1100,7 @@ cudaError_t launch_gqa2(const CUtensorMap& tq, const CUtensorMap& tk, const CUte
     int C = n_qt_max > 0 ? n_qt_max : 1;
     SplitWs sw{};
     if (ws != nullptr) {
-        const AttnWsLayout lay = attention_ws_layout(B, max_M, Hq, Hkv, HD);
+        const AttnWsLayout lay = attention_ws_layout(B, max_M, Hq, Hkv, HD, true);
         if (ws_bytes < lay.total) return cudaErrorInvalidValue;
         C = lay.C;
         uint8_t* p = static_cast<uint8_t*>(ws);
@@ -1135,7 +1137,7 @@ cudaError_t launch_tc(const uint16_t* q, const uint16_t* k, const uint16_t* v, c
     if constexpr (HD <= 128) {  // two heads of 256 would need 768 TMEM columns
         if ((Hq / Hkv) % 2 == 0) {
             // the persistent kernel needs the workspace for its unit counter
-            if (ws != nullptr) {
+            if (ws != nullptr && !attention_per_unit_kernel(B, gates.n)) {
                 const cudaError_t e = launch_attention_persistent(tq, tk, tv, cu_kept, B, M_total, max_M, Hq, Hkv,
                                                                   HD, pos, rank, gates, c, sm_scale, out, lse, ws,
                                                                   ws_bytes, early, st);
@@ -1182,6 +1184,24 @@ cudaError_t launch_gated_attention(const uint16_t* q, const uint16_t* k, const u
                           ws_bytes, inputs_ready, st);
 }
 
+namespace {
+// 0: by the batch, 1: persistent, 2: one CTA per unit (read on every call, so that a process
+// may switch between calls)
+int attention_kernel_override() {
+    const char* e = std::getenv("TG_ATTENTION_KERNEL");
+    if (e == nullptr) return 0;
+    if (std::strcmp(e, "persistent") == 0) return 1;
+    if (std::strcmp(e, "per_unit") == 0) return 2;
+    return 0;
+}
+}  // namespace
+
+bool attention_per_unit_kernel(int B, int n_gates) {
+    const int choice = attention_kernel_override();
+    if (n_gates <= 0 || choice == 1) return false;
+    return choice == 2 || B == 1;
+}
+
 int64_t units_below_host(int x, int C) {
     const int64_t a = x / C, r = x % C;
     return C * a * (a + 1) / 2 + r * (a + 1);
@@ -1192,14 +1212,14 @@ int64_t units_below_host(int x, int C) {
 // tiles past C into two units ([0, C) and [C, qt + 1)), C >= ceil(n_qt / 2) so
 // that two always suffice.  A unit costs about F + n_kv tile pairs on one SM,
 // F being the part a unit adds beyond its tiles.  With the persistent kernel
-// (the split only runs there) a CTA loads the next unit while it finishes the
-// current one, so F is about one tile pair (the epilogue and the merge); the
-// one-CTA-per-unit kernel paid F = 3.1 (9 us of set-up, first loads and
-// epilogue against 2.87 us per tile pair).  Units are taken heaviest first,
+// a CTA loads the next unit while it finishes the current one, so F is about
+// one tile pair (the epilogue and the merge); the one-CTA-per-unit kernel pays
+// F = 3.1 (9 us of set-up, first loads and epilogue against 2.87 us per tile
+// pair).  Units are taken heaviest first,
 // which is longest-processing-time scheduling, so C is the candidate whose LPT
 // makespan over the SMs is smallest (all sequences taken at max_M, the bound the
 // host knows); ties go to the larger C (fewer units).
-int attention_kv_chunk(int B, int max_M, int Hq, int Hkv, bool have_ws) {
+int attention_kv_chunk(int B, int max_M, int Hq, int Hkv, bool have_ws, bool per_unit) {
     const int n_qt = (max_M + BM - 1) / BM;
     if (!have_ws || (Hq / Hkv) % 2 != 0 || n_qt < 4) return n_qt > 0 ? n_qt : 1;
     int dev = 0, sms = 148;
@@ -1212,17 +1232,14 @@ int attention_kv_chunk(int B, int max_M, int Hq, int Hkv, bool have_ws) {
     // the choice depends on the shape alone: remember it (a few hundred heap operations
     // per candidate would otherwise run on every call)
     static std::mutex mu;
-    static std::map<std::tuple<int, int, int, int>, int> memo;
-    const auto key = std::make_tuple(B, n_qt, Hq / 2, sms);
+    static std::map<std::tuple<int, int, int, int, int>, int> memo;
+    const double F = per_unit ? 3.1 : 1.0;
+    const auto key = std::make_tuple(B, n_qt, Hq / 2, sms, F > 2.0 ? 1 : 0);
     {
         std::lock_guard<std::mutex> lk(mu);
         const auto it = memo.find(key);
         if (it != memo.end()) return it->second;
     }
-#ifndef TG_LPT_FIXED_COST
-#define TG_LPT_FIXED_COST 1.0
-#endif
-    constexpr double F = TG_LPT_FIXED_COST;
     int best_c = n_qt;
     double best = 1e300;
     std::vector<double> cost;
@@ -1264,13 +1281,13 @@ int attention_kv_chunk(int B, int max_M, int Hq, int Hkv, bool have_ws) {
     return best_c;
 }
 
-AttnWsLayout attention_ws_layout(int B, int max_M, int Hq, int Hkv, int d) {
+AttnWsLayout attention_ws_layout(int B, int max_M, int Hq, int Hkv, int d, bool per_unit) {
     AttnWsLayout L;
     const int n_qt = (max_M + BM - 1) / BM;
     L.C = n_qt > 0 ? n_qt : 1;
     if (B <= 0 || n_qt <= 0 || Hkv <= 0 || (Hq / Hkv) % 2 != 0 || d > 128) return L;  // one-head kernel: none
     auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
-    L.C = attention_kv_chunk(B, max_M, Hq, Hkv, true);
+    L.C = attention_kv_chunk(B, max_M, Hq, Hkv, true, per_unit);
     L.total = 256;  // the unit counters of the persistent kernel
     if (L.C < n_qt) {
         L.max_nch = (n_qt + L.C - 1) / L.C;
@@ -1285,8 +1302,10 @@ AttnWsLayout attention_ws_layout(int B, int max_M, int Hq, int Hkv, int d) {
     return L;
 }
 
+// The workspace serves either two-head kernel (their chunk choices differ): the larger need.
 size_t attention_workspace_bytes(int B, int max_M, int Hq, int Hkv, int d) {
-    return attention_ws_layout(B, max_M, Hq, Hkv, d).total;
+    return std::max(attention_ws_layout(B, max_M, Hq, Hkv, d, false).total,
+                    attention_ws_layout(B, max_M, Hq, Hkv, d, true).total);
 }
 
 // ---------------------------------------------------------------------------
@@ -1338,7 +1357,10 @@ cudaError_t launch_gated_attention_noalloc(const uint16_t* q, const uint16_t* k,
     if (e != cudaSuccess) return e;
     if (need > 0) {
         // the counters must start at zero: the last call may have stopped early
-        e = cudaMemsetAsync(ws, 0, attention_ws_layout(B, max_M, Hq, Hkv, d).zero_bytes, st);
+        e = cudaMemsetAsync(ws, 0,
+                            std::max(attention_ws_layout(B, max_M, Hq, Hkv, d, false).zero_bytes,
+                                     attention_ws_layout(B, max_M, Hq, Hkv, d, true).zero_bytes),
+                            st);
         if (e != cudaSuccess) return e;
     }
     return launch_gated_attention(q, k, v, cu_kept, B, M_total, max_M, Hq, Hkv, d, pos, rank, gates, c, sm_scale,

@@ -886,7 +886,7 @@ static cudaError_t launch_pers_impl(const CUtensorMap& tq, const CUtensorMap& tk
     if (regs.load() != PT_LAUNCH_REGS) return cudaErrorNotSupported;
     if (cudaError_t e = ensure_smem_limit(gated_attn_pers_kernel<HD, GATED>, L::ALLOC, attr_set); e != cudaSuccess)
         return e;
-    const AttnWsLayout lay = attention_ws_layout(B, max_M, Hq, Hkv, HD);
+    const AttnWsLayout lay = attention_ws_layout(B, max_M, Hq, Hkv, HD, false);
     if (ws == nullptr || ws_bytes < lay.total) return cudaErrorInvalidValue;
     uint8_t* base = static_cast<uint8_t*>(ws);
     SplitWs sw{};

@@ -192,7 +192,8 @@ struct AttnWsLayout {
 
 // Workspace layout of the forward attention for these sizes (host side; the kernels get
 // the pointers it describes).
-attn::AttnWsLayout attention_ws_layout(int B, int max_M, int Hq, int Hkv, int d);
+// per_unit: the layout for the one-CTA-per-unit kernel's chunk choice, else the persistent kernel's
+attn::AttnWsLayout attention_ws_layout(int B, int max_M, int Hq, int Hkv, int d, bool per_unit);
 
 // The persistent attention (k_attention_pers.cu): head_dim 64 or 128, GQA groups of
 // even size, 1 to kMaxGates gates, or none (gates.n == 0: bias 0, tau 1, c unused).

@@ -172,7 +172,15 @@ cudaError_t launch_gated_attention(const uint16_t* q, const uint16_t* k, const u
 
 // Causal work split of the attention: KV chunk length chosen for a launch,
 // scratch bytes the split needs (0 when it never splits), unit count.
-int attention_kv_chunk(int B, int max_M, int Hq, int Hkv, bool have_ws);
+int attention_kv_chunk(int B, int max_M, int Hq, int Hkv, bool have_ws, bool per_unit);
+// Which two-head kernel a call with a workspace runs (even GQA groups, head_dim <= 128): the
+// one-CTA-per-unit kernel for a gated call over one sequence, the persistent kernel otherwise.
+// Measured on B200: one CTA per unit is faster on one sequence (46.9 against 50.5 us at 32k
+// tokens, K = 2000; 4.13 against 4.57 ms with every token kept), persistent CTAs on a batch of
+// unequal sequences (73.7 against 86.0 us on a four-sequence batch).  The environment variable
+// TG_ATTENTION_KERNEL = persistent | per_unit overrides the choice (per_unit applies to gated
+// calls only: the plain, ungated attention runs persistent CTAs in every case).
+bool attention_per_unit_kernel(int B, int n_gates);
 cudaError_t launch_gated_attention_noalloc(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                            const int32_t* cu_kept, int B, int64_t M_total, int max_M, int Hq, int Hkv,
                                            int d, const int32_t* pos, const int32_t* rank, const GateSet& gates,

@@ -2,6 +2,9 @@
 
 from __future__ import annotations
 
+import contextlib
+import os
+
 import numpy as np
 import torch
 
@@ -65,3 +68,20 @@ def check_selection_swaps(keep_gpu: np.ndarray, keep_ref: np.ndarray, s_ref: np.
         tol = NEAR_TIE_REL * max(1.0, abs(float(s_ref[i])))
         assert np.any(np.abs(s_ref[only_gpu] - s_ref[i]) <= tol), f"token {i} swapped without a near-tie"
     return len(only_ref)
+
+
+@contextlib.contextmanager
+def attention_kernel(name):
+    """Run the enclosed calls with TG_ATTENTION_KERNEL = name ("persistent" or "per_unit";
+    None leaves the library's own choice); the previous setting is restored after."""
+    old = os.environ.get("TG_ATTENTION_KERNEL")
+    if name is not None:
+        os.environ["TG_ATTENTION_KERNEL"] = name
+    try:
+        yield
+    finally:
+        if name is not None:
+            if old is None:
+                os.environ.pop("TG_ATTENTION_KERNEL", None)
+            else:
+                os.environ["TG_ATTENTION_KERNEL"] = old

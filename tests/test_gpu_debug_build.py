@@ -49,12 +49,14 @@ def _attend(lib, w, comp, ai, M, cu_kept, max_M):
     t = [H.bf16_dev(ai["q"]), H.bf16_dev(ai["k"]), H.bf16_dev(ai["v"]), H.i32_dev(cu_kept),
          H.i32_dev(comp["pos"]), H.i32_dev(comp["rank"]), H.f32_dev(comp["gls"]), H.f32_dev(ai["g"]),
          H.f32_dev(ai["c"])]
-    n = int(lib.tg_gated_attention_workspace_size(w.B, max_M, w.Hq, w.Hkv, w.d))
-    ws = torch.zeros(max(n, 256), dtype=torch.uint8, device="cuda")
     out = torch.zeros((M, w.Hq, w.d), dtype=torch.bfloat16, device="cuda")
-    st = lib.tg_gated_attention(*[x.data_ptr() for x in t[:4]], w.B, M, max_M, w.Hq, w.Hkv, w.d,
-                                *[x.data_ptr() for x in t[4:]], 1.0 / math.sqrt(w.d), out.data_ptr(), None,
-                                ws.data_ptr(), ws.numel(), None)
+    # the persistent kernel is the one whose debug build checks cu_kept against M_total
+    with H.attention_kernel("persistent"):
+        n = int(lib.tg_gated_attention_workspace_size(w.B, max_M, w.Hq, w.Hkv, w.d))
+        ws = torch.zeros(max(n, 256), dtype=torch.uint8, device="cuda")
+        st = lib.tg_gated_attention(*[x.data_ptr() for x in t[:4]], w.B, M, max_M, w.Hq, w.Hkv, w.d,
+                                    *[x.data_ptr() for x in t[4:]], 1.0 / math.sqrt(w.d), out.data_ptr(), None,
+                                    ws.data_ptr(), ws.numel(), None)
     assert st == 0, lib.tg_last_error_string()
     torch.cuda.synchronize()
     return out

@@ -211,6 +211,26 @@ def test_select_ties_signed_zero_nan_inf(tg, seed):
         _select_and_compact(tg, [0, n], [[0, n]], [k], s)
 
 
+@pytest.mark.parametrize("n", [20000, 40000])
+def test_select_degenerate_score_ranges(tg, n):
+    """Score sets whose value range is degenerate for a bucket search: all equal, a range
+    as wide as fp32, denormals only, only infinities and NaN, a few distinct values under
+    heavy ties, one outlier far above the rest; each at two span lengths."""
+    rng = np.random.default_rng(7 + n)
+    cases = {
+        "all equal": np.full(n, 1.5, np.float32),
+        "fp32-wide": rng.choice(np.array([-3.0e38, 3.0e38, 0.0, 1.0, -1.0], np.float32), size=n),
+        "denormal": (rng.integers(1, 1000, size=n) * np.float32(1.4e-45)).astype(np.float32),
+        "non-finite": rng.choice(np.array([np.inf, -np.inf, np.nan], np.float32), size=n),
+        "few values": np.round(rng.standard_normal(n) * 3).astype(np.float32),
+        "one outlier": np.concatenate([np.full(n - 1, -2.0, np.float32), np.array([1e30], np.float32)]),
+    }
+    for what, s in cases.items():
+        s = s.astype(np.float32)
+        for k in (0, 1, n // 3, n - 1, -1):
+            _select_and_compact(tg, [0, n], [[0, n]], [k], s)
+
+
 def test_select_large_span_uncached_path(tg):
     """A span longer than the shared-memory key cache (global re-reads)."""
     n = 131072
@@ -502,11 +522,16 @@ def test_attention_is_deterministic_with_the_causal_split(tg):
         assert np.array_equal(o, outs[0][0]) and np.array_equal(l, outs[0][1])
 
 
-def _raw_attention(tg, w, comp, ai, gls32, c, ws_mode, g=None):
+def _raw_attention(tg, w, comp, ai, gls32, c, ws_mode, g=None, kernel=None):
     """tg_gated_attention through the C ABI with explicit pointers: gls/g/c may be None (no
-    gate); ws_mode "auto" passes the sized workspace, None passes no workspace."""
+    gate); ws_mode "auto" passes the sized workspace, None passes no workspace; kernel
+    ("persistent" / "per_unit") sets TG_ATTENTION_KERNEL for this call."""
     from learned_token_pruning_rmsnorm_b200 import _lib
-    lib = _lib.load()
+    with H.attention_kernel(kernel):
+        return _raw_attention_call(_lib.load(), _lib, w, comp, ai, gls32, c, ws_mode, g)
+
+
+def _raw_attention_call(lib, _lib, w, comp, ai, gls32, c, ws_mode, g):
     ck = comp["cu_kept"]
     M, max_M = int(ck[-1]), int(np.max(np.diff(ck)))
     keep = [H.bf16_dev(ai["q"]), H.bf16_dev(ai["k"]), H.bf16_dev(ai["v"]), H.i32_dev(ck), H.i32_dev(comp["pos"]),
@@ -537,7 +562,8 @@ def test_attention_without_gate_is_the_zero_gate_bit_for_bit(tg, name):
     w, comp, ai, gls32, _, _, _ = attn_case(name)
     zeros = np.zeros_like(gls32)
     plain, plain_lse = _raw_attention(tg, w, comp, ai, None, None, "auto")
-    gated0, gated0_lse = _raw_attention(tg, w, comp, ai, zeros, np.zeros_like(ai["c"]), "auto", g=ai["g"])
+    gated0, gated0_lse = _raw_attention(tg, w, comp, ai, zeros, np.zeros_like(ai["c"]), "auto", g=ai["g"],
+                                        kernel="persistent")
     np.testing.assert_array_equal(plain, gated0)
     np.testing.assert_array_equal(plain_lse, gated0_lse)
     ck = comp["cu_kept"]
@@ -557,18 +583,27 @@ def test_attention_without_gate_needs_a_workspace(tg):
 
 @pytest.mark.parametrize("name", ["c1_16k", "c2_32k_k2000", "c4_varlen"])
 def test_persistent_and_per_unit_kernels_agree(tg, name):
-    """With a workspace the attention runs persistent CTAs that take units from a counter;
-    without one, one CTA per unit.  Same arithmetic per row (the row maximum, the
-    exponentials, the bf16 P), so the outputs agree within the parity bars and both match
-    the oracle's rows."""
+    """Both two-head kernels on the same inputs: persistent CTAs that take units from a
+    counter, one CTA per unit with the causal split (both with a workspace, forced through
+    TG_ATTENTION_KERNEL) and one CTA per unit unsplit (no workspace).  Same arithmetic per
+    row (the row maximum, the exponentials, the bf16 P), so the outputs agree within the
+    parity bars and all match the oracle's rows; the default choice equals one of them bit
+    for bit (one CTA per unit for one sequence, persistent CTAs for a batch)."""
     w, comp, ai, gls32, rows, out_ref, lse_ref = attn_case(name, rows_step=7 if name == "c4_varlen" else None)
-    a, a_lse = _raw_attention(tg, w, comp, ai, gls32, ai["c"], "auto", g=ai["g"])
+    a, a_lse = _raw_attention(tg, w, comp, ai, gls32, ai["c"], "auto", g=ai["g"], kernel="persistent")
+    s, s_lse = _raw_attention(tg, w, comp, ai, gls32, ai["c"], "auto", g=ai["g"], kernel="per_unit")
     b, b_lse = _raw_attention(tg, w, comp, ai, gls32, ai["c"], None, g=ai["g"])
+    d, d_lse = _raw_attention(tg, w, comp, ai, gls32, ai["c"], "auto", g=ai["g"])
     H.assert_attention_close(a, b.astype(np.float64), name + " persistent vs per-unit")
+    H.assert_attention_close(a, s.astype(np.float64), name + " persistent vs per-unit split")
     sel = slice(None) if rows is None else rows
     H.assert_attention_close(a[sel], out_ref, name + " persistent")
+    H.assert_attention_close(s[sel], out_ref, name + " per-unit split")
     H.assert_attention_close(b[sel], out_ref, name + " per-unit")
-    assert np.max(np.abs(a_lse[sel] - lse_ref)) <= H.LSE_ABS
+    for lse_x in (a_lse, s_lse, b_lse):
+        assert np.max(np.abs(lse_x[sel] - lse_ref)) <= H.LSE_ABS
+    np.testing.assert_array_equal(d, s if w.B == 1 else a)
+    np.testing.assert_array_equal(d_lse, s_lse if w.B == 1 else a_lse)
 
 
 def test_attention_output_only_16_byte_aligned(tg):
