@@ -173,7 +173,7 @@ def source_sha(kernel_file: str) -> str:
 
 
 KERNEL_FILES = {"score": "k_gate.cu", "select": "k_select.cu", "gather": "k_select.cu",
-                "attention": "k_attention_pers.cu"}
+                "attention": "k_attention.cu"}
 
 
 # ------------------------------------------------------------------ oracle (CPU baseline / reference arm)
