@@ -8,10 +8,10 @@
 // Design: one cluster of SEL_CL CTAs per sequence.  CTA i owns a contiguous
 // slice of the sequence's tokens and caches the order-preserving uint32 keys
 // of its prunable tokens in shared memory.
-//   1. bucket select: the cluster agrees on the span's [min, max] key range,
-//      then each pass histograms the keys of the current range into <= 2048
-//      buckets of width 2^s (buckets span the data's actual range, so
-//      concentrated exponents still spread) and sums them into 64 superbins.
+//   1. bucket select: each pass histograms the keys of the current range into
+//      <= 2048 buckets of width 2^s (the first pass the whole key range by its
+//      top 11 bits, the next ones the chosen bucket by the following 11 and 10
+//      bits) and sums them into 64 superbins.
 //      One warp per CTA then reads the 8 x 64 superbin sums and the 8 x 32
 //      buckets of the chosen superbin through distributed shared memory and
 //      narrows the range to the bucket holding the K-th key.  The passes stop
@@ -60,7 +60,6 @@ constexpr int SEL_SUPER = SEL_BINS / 32;      // superbins of 32 buckets
 constexpr int SEL_SMEM_BYTES = SEL_CACHE_KEYS * 4 + 2 * SEL_BINS * 4;
 
 struct SelShared {
-    uint32_t kmin, kmax;
     int coarse[2][SEL_SUPER];  // per pass parity: bucket counts summed over each superbin
     int xchg[2];               // slice totals published to the cluster: kept, tie-ranked
     int warp_kept[SEL_WARPS];  // exclusive prefix over the warps of this CTA
@@ -156,78 +155,24 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
     // ------------------------------------------------ cache keys (for the selection and for gls)
     const bool need_gls = emit && kk > 0;  // some prunable token is kept: its logsigmoid is emitted
     if (cached && (do_select || need_gls)) {
-        uint32_t lmin = 0xFFFFFFFFu, lmax = 0u;
 #pragma unroll 8
-        for (int64_t t = k0 + tid; t < k1; t += SEL_THREADS) {
-            const uint32_t key = score_key(__ldcg(scores + t));
-            skeys[t - k0] = key;
-            lmin = min(lmin, key);
-            lmax = max(lmax, key);
-        }
-        if (do_select) {
-#pragma unroll
-            for (int off = 16; off; off >>= 1) {
-                lmin = min(lmin, __shfl_xor_sync(0xffffffffu, lmin, off));
-                lmax = max(lmax, __shfl_xor_sync(0xffffffffu, lmax, off));
-            }
-            if (tid == 0) {
-                sh.kmin = 0xFFFFFFFFu;
-                sh.kmax = 0u;
-            }
-            __syncthreads();
-            if (lane == 0) {
-                atomicMin(&sh.kmin, lmin);
-                atomicMax(&sh.kmax, lmax);
-            }
-        }
-    } else if (do_select) {
-        uint32_t lmin = 0xFFFFFFFFu, lmax = 0u;
-        for (int64_t t = k0 + tid; t < k1; t += SEL_THREADS) {
-            const uint32_t key = score_key(__ldcg(scores + t));
-            lmin = min(lmin, key);
-            lmax = max(lmax, key);
-        }
-#pragma unroll
-        for (int off = 16; off; off >>= 1) {
-            lmin = min(lmin, __shfl_xor_sync(0xffffffffu, lmin, off));
-            lmax = max(lmax, __shfl_xor_sync(0xffffffffu, lmax, off));
-        }
-        if (tid == 0) {
-            sh.kmin = 0xFFFFFFFFu;
-            sh.kmax = 0u;
-        }
-        __syncthreads();
-        if (lane == 0) {
-            atomicMin(&sh.kmin, lmin);
-            atomicMax(&sh.kmax, lmax);
-        }
+        for (int64_t t = k0 + tid; t < k1; t += SEL_THREADS) skeys[t - k0] = score_key(__ldcg(scores + t));
     }
     SEL_TRACE(1);
 
     if (do_select) {  // uniform over the cluster: it depends on the sequence only
-        cl.sync();  // every CTA's slice min/max is published
-        SEL_TRACE(2);
-        if (warp == 0) {
-            // lane r < SEL_CL reads CTA r's range; a warp reduction combines them
-            uint32_t gmin = 0xFFFFFFFFu, gmax = 0u;
-            if (lane < SEL_CL) {
-                const SelShared* o = cl.map_shared_rank(&sh, lane);
-                gmin = o->kmin;
-                gmax = o->kmax;
-            }
-#pragma unroll
-            for (int off = 16; off; off >>= 1) {
-                gmin = min(gmin, __shfl_xor_sync(0xffffffffu, gmin, off));
-                gmax = max(gmax, __shfl_xor_sync(0xffffffffu, gmax, off));
-            }
-            if (lane == 0) {
-                sh.lo = gmin;
-                sh.width = static_cast<uint64_t>(gmax) - gmin + 1;
-                sh.remaining = static_cast<int>(kk);
-                sh.bin_count = 0;
-            }
+        // The first pass buckets the whole key range by the top 11 bits (sign, exponent and two
+        // mantissa bits of the score), each later pass the chosen bucket by the next 11 and then
+        // 10 bits, so three passes resolve any key and no agreement on the keys' range is
+        // needed before the first.
+        if (tid == 0) {
+            sh.lo = 0u;
+            sh.width = static_cast<uint64_t>(1) << 32;
+            sh.remaining = static_cast<int>(kk);
+            sh.bin_count = 0;
         }
-        __syncthreads();
+        __syncthreads();  // the key cache and the range are in place
+        SEL_TRACE(2);
         // ------------------------------------------------ bucket passes
         for (int pass = 0;; ++pass) {
             const uint32_t lo = sh.lo;
