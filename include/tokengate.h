@@ -360,7 +360,7 @@ typedef struct tg_prefill_layer_args {
     const float* const* c;      /* n_layers x [Hq] */
     uint16_t* const* out;       /* n_layers x [M, Hq, d] out */
     float* const* lse;          /* n_layers x [M, Hq] out, array or entries may be NULL */
-    void* attn_ws;              /* scratch of tg_gated_attention, shared by the layers (may be NULL) */
+    void* attn_ws;              /* scratch shared by the layers (may be NULL): see below */
     size_t attn_ws_bytes;
     /* optional: more row-major arrays gathered by the same map beside the attention, e.g. the
        KV cache of the layers below L (see tg_gather_rows); n_gather = 0 for none */
@@ -371,6 +371,21 @@ typedef struct tg_prefill_layer_args {
 } tg_prefill_layer_args;
 
 tg_status tg_gated_prefill_layer(const tg_prefill_layer_args* args, tg_stream_t stream);
+
+/*
+ * Bytes of args->attn_ws with which tg_gated_prefill_layer also runs the
+ * selection's first bucket pass inside the score kernel: after the attention's
+ * scratch (tg_gated_attention_workspace_size, rounded up to 256 bytes) the
+ * workspace holds a [B][2048] int32 histogram of the top 11 bits of every
+ * scored row's order-preserving key, which the score kernel fills with atomic
+ * adds and the selection reads (saving a pass over the keys and a cluster
+ * round trip) and zeroes again.  The same zero-on-entry contract as the
+ * attention's scratch holds: zero-fill attn_ws before its first use; every
+ * call leaves it zero-filled.  A smaller attn_ws (at least the attention's
+ * size) runs every pass in the selection; results are identical.
+ * n_layers = 0: the histogram alone.  Returns 0 for B <= 0.
+ */
+size_t tg_gated_prefill_workspace_size(int B, int max_M, int Hq, int Hkv, int d, int n_layers);
 
 /*
  * Full-length (training-time) token-gated attention for a sampled budget.

@@ -194,6 +194,21 @@ def tg_compact(hidden, scores, keep, cu_seqlens, span, cu_kept, M_total: int, wi
 _WS_CACHE = {}
 
 
+def prefill_workspace(B: int, max_M: int, Hq: int, Hkv: int, d: int, n_layers: int, device) -> torch.Tensor | None:
+    """Zero-filled scratch for tg_gated_prefill_layer: the attention's causal-split scratch
+    and the selection's first-pass histogram (one per device and size, reused; calls sharing
+    it must not run concurrently)."""
+    n = int(load().tg_gated_prefill_workspace_size(B, max_M, Hq, Hkv, d, n_layers))
+    if n == 0:
+        return None
+    key = (torch.device(device), n, "prefill")
+    ws = _WS_CACHE.get(key)
+    if ws is None:
+        ws = torch.zeros(n, dtype=torch.uint8, device=device)
+        _WS_CACHE[key] = ws
+    return ws
+
+
 def attention_workspace(B: int, max_M: int, Hq: int, Hkv: int, d: int, device) -> torch.Tensor | None:
     """Zero-filled scratch for tg_gated_attention's causal work split (one per
     device and size, reused; calls sharing it must not run concurrently)."""
@@ -494,7 +509,7 @@ class PrefillCall:
         a.q, a.kk, a.v, a.g, a.c, a.out = (cast(self._q), cast(self._k), cast(self._v), cast(self._g),
                                            cast(self._c), cast(self._o))
         a.lse = cast(self._lse)
-        self.ws = attention_workspace(a.B, self.max_M, Hq, Hkv, d, dev) if nl > 0 else None
+        self.ws = prefill_workspace(a.B, self.max_M, Hq, Hkv, d, nl, dev)
         a.attn_ws = _lib.ptr(self.ws)
         a.attn_ws_bytes = 0 if self.ws is None else self.ws.numel()
         gathers = list(gathers)

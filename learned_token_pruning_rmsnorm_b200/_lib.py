@@ -67,6 +67,7 @@ SIGNATURES = {
     "tg_gated_attention_backward_gates": ([P, P, P, P, P, P, P, i32, i64, i32, i32, i32, i32, P, P, i32, P, P, P,
                                            f32, P, P, P, P, P, P, P, P, C.c_size_t, P], i32),
     "tg_gated_attention_workspace_size": ([i32, i32, i32, i32, i32], C.c_size_t),
+    "tg_gated_prefill_workspace_size": ([i32, i32, i32, i32, i32, i32], C.c_size_t),
     "tg_gated_attention_noalloc": ([P, P, P, P, i32, i64, i32, i32, i32, i32, P, P, P, P, P, f32, P, P, P], i32),
     "tg_gated_prefill_layer": ([C.POINTER(PrefillLayerArgs), P], i32),
     "tg_gather_rows": ([P, i64, i64, P, i64, P, P], i32),

@@ -98,9 +98,9 @@ __device__ __forceinline__ float silu_f(float z) {
     return z * r;
 }
 
-// Tile t of the concatenated per-sequence tile lists -> (first row, end of span).
+// Tile t of the concatenated per-sequence tile lists -> (first row, end of span, sequence).
 __device__ __forceinline__ bool map_tile(int64_t t, int rows, const int32_t* cu_seqlens, const int32_t* span, int B,
-                                         int64_t* row0, int64_t* row_end) {
+                                         int64_t* row0, int64_t* row_end, int* seq = nullptr) {
     for (int b = 0; b < B; ++b) {
         const int64_t s0 = cu_seqlens[b], n = cu_seqlens[b + 1] - s0;
         const int64_t p0 = s0 + min(max(static_cast<int64_t>(span[2 * b]), int64_t(0)), n);
@@ -109,6 +109,7 @@ __device__ __forceinline__ bool map_tile(int64_t t, int rows, const int32_t* cu_
         if (t < nt) {
             *row0 = p0 + t * rows;
             *row_end = p1;
+            if (seq) *seq = b;
             return true;
         }
         t -= nt;
@@ -121,7 +122,7 @@ __global__ void __launch_bounds__(ScoreCfg<NACC>::THREADS, 1)
 score_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                 const int32_t* __restrict__ cu_seqlens, const int32_t* __restrict__ span, int B, int D, int I,
                 const float* __restrict__ b1, const float* __restrict__ w2, float b2, float eps,
-                float* __restrict__ scores, int64_t T, int* __restrict__ status) {
+                float* __restrict__ scores, int64_t T, int* __restrict__ status, int* __restrict__ key_hist) {
     using C = ScoreCfg<NACC>;
     constexpr int STAGES = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
@@ -261,7 +262,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
         bool ok = true;
         for (int64_t t = blockIdx.x; ok; t += gridDim.x, ++tcount) {
             int64_t row0, row_end;
-            if (!map_tile(t, C::ROWS, cu_seqlens, span, B, &row0, &row_end)) break;
+            int seq = 0;
+            if (!map_tile(t, C::ROWS, cu_seqlens, span, B, &row0, &row_end, &seq)) break;
             float ss = 0.f;
             for (int kb = 0; kb < nkb; ++kb, ++it) {
                 const int s = static_cast<int>(it % STAGES);
@@ -314,7 +316,15 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
             __syncwarp();
             if (lane == 0) mbar_arrive(acc_empty);
             const int64_t row = row0 + a * 128 + r;
-            if (row < row_end && TG_DEBUG_CHECK(row >= 0 && row < T, status, TG_WHERE_SCORE)) scores[row] = acc_s + b2;
+            const bool valid = row < row_end && TG_DEBUG_CHECK(row >= 0 && row < T, status, TG_WHERE_SCORE);
+            if (valid) scores[row] = acc_s + b2;
+            if (key_hist != nullptr) {
+                // the selection's first pass: this sequence's scores counted by the top 11 bits of
+                // their order-preserving key, one atomic per distinct bucket of the warp
+                const int bin = valid ? seq * 2048 + static_cast<int>(score_key(acc_s + b2) >> 21) : -1;
+                const unsigned same = __match_any_sync(0xffffffffu, bin);
+                if (valid && lane == __ffs(same) - 1) atomicAdd(key_hist + bin, __popc(same));
+            }
         }
     }
 
@@ -330,7 +340,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
 template <int NACC>
 cudaError_t launch_score_tc(const uint16_t* hidden, const int32_t* cu_seqlens, const int32_t* span, int B, int64_t T,
                             int D, const uint16_t* Wg, const float* b1, const float* w2, float b2, int I, float eps,
-                            float* scores, int sms, cudaStream_t st) {
+                            float* scores, int* key_hist, int sms, cudaStream_t st) {
     using C = ScoreCfg<NACC>;
     static std::atomic<uint64_t> attr_set{0};
     if (cudaError_t e = ensure_smem_limit(score_tc_kernel<NACC>, score_smem_bytes<NACC>(256), attr_set); e != cudaSuccess)
@@ -345,7 +355,7 @@ cudaError_t launch_score_tc(const uint16_t* hidden, const int32_t* cu_seqlens, c
     const int grid = static_cast<int>(tiles_bound < sms ? tiles_bound : sms);
     const cudaError_t le = launch_pdl(score_tc_kernel<NACC>, dim3(grid), dim3(C::THREADS),
                                       static_cast<size_t>(score_smem_bytes<NACC>(I)), st, tx, tw, cu_seqlens, span, B,
-                                      D, I, b1, w2, b2, eps, scores, T, device_status_ptr());
+                                      D, I, b1, w2, b2, eps, scores, T, device_status_ptr(), key_hist);
     if (le != cudaSuccess) return le;
     return cudaGetLastError();
 }
@@ -369,7 +379,7 @@ cudaError_t launch_gate_prepare(const uint16_t* gamma, const uint16_t* W1, int D
 
 cudaError_t launch_score(const uint16_t* hidden, const int32_t* cu_seqlens, const int32_t* span, int B,
                          int64_t T, int D, const uint16_t* Wg, const float* b1, const float* w2, float b2, int I,
-                         float eps, float* scores, cudaStream_t st) {
+                         float eps, float* scores, cudaStream_t st, int* key_hist) {
     if (T == 0 || B == 0) return cudaSuccess;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
@@ -377,8 +387,9 @@ cudaError_t launch_score(const uint16_t* hidden, const int32_t* cu_seqlens, cons
     // 256-row tiles halve the gate-weight traffic from L2 once there are more
     // 128-row tiles than SMs; below that, 128-row tiles spread the rows wider.
     if ((T + 127) / 128 > sms)
-        return launch_score_tc<2>(hidden, cu_seqlens, span, B, T, D, Wg, b1, w2, b2, I, eps, scores, sms, st);
-    return launch_score_tc<1>(hidden, cu_seqlens, span, B, T, D, Wg, b1, w2, b2, I, eps, scores, sms, st);
+        return launch_score_tc<2>(hidden, cu_seqlens, span, B, T, D, Wg, b1, w2, b2, I, eps, scores, key_hist, sms,
+                                  st);
+    return launch_score_tc<1>(hidden, cu_seqlens, span, B, T, D, Wg, b1, w2, b2, I, eps, scores, key_hist, sms, st);
 }
 
 }  // namespace tg

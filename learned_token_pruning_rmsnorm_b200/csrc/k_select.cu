@@ -62,6 +62,7 @@ constexpr int SEL_SMEM_BYTES = SEL_CACHE_KEYS * 4 + 2 * SEL_BINS * 4;
 struct SelShared {
     int coarse[2][SEL_SUPER];  // per pass parity: bucket counts summed over each superbin
     int xchg[2];               // slice totals published to the cluster: kept, tie-ranked
+    int wsum[SEL_WARPS];       // a first-pass histogram summed over each warp's 64 buckets
     int warp_kept[SEL_WARPS];  // exclusive prefix over the warps of this CTA
     int warp_eq[SEL_WARPS];
     uint32_t lo;               // current key range [lo, lo + width)
@@ -109,7 +110,7 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
                    const int32_t* __restrict__ cu_seqlens, const int32_t* __restrict__ span,
                    const int32_t* __restrict__ kbud, const int32_t* __restrict__ cu_kept,
                    uint8_t* __restrict__ keep_out, int32_t* __restrict__ kept_idx, int32_t* __restrict__ pos,
-                   int32_t* __restrict__ rank, float* __restrict__ gls) {
+                   int32_t* __restrict__ rank, float* __restrict__ gls, int* __restrict__ key_hist) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     uint32_t* skeys = reinterpret_cast<uint32_t*>(smem_raw);
     int* hist_buf = reinterpret_cast<int*>(smem_raw + SEL_CACHE_KEYS * 4);  // [2][SEL_BINS]
@@ -171,10 +172,49 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
             sh.remaining = static_cast<int>(kk);
             sh.bin_count = 0;
         }
+        if (key_hist != nullptr) {
+            // The score kernel took the first pass (the top 11 bits of every key of this
+            // sequence): every CTA reads the same counts and finds the same bucket itself, the
+            // K-th key from the top (its 64-bucket warp segment, then the bucket), with no
+            // cluster round trip.
+            const int* kh = key_hist + static_cast<int64_t>(b) * SEL_BINS;
+            int* hist0 = hist_buf;  // free until the passes below
+            const int v0 = __ldcg(kh + 2 * tid), v1 = __ldcg(kh + 2 * tid + 1);
+            hist0[2 * tid] = v0;
+            hist0[2 * tid + 1] = v1;
+            const int wsum = warp_sum(v0 + v1);
+            if (lane == 0) sh.wsum[warp] = wsum;
+            __syncthreads();
+            if (warp == 0) {
+                const int rem = static_cast<int>(kk);
+                const int v = sh.wsum[SEL_WARPS - 1 - lane];
+                const int incl = warp_inclusive_scan(v);
+                const unsigned hit = __ballot_sync(0xffffffffu, incl - v < rem && incl >= rem);
+                if (hit != 0u) {  // else (counts inconsistent with the span) the full passes run
+                    const int L = __ffs(hit) - 1;
+                    const int rem1 = rem - __shfl_sync(0xffffffffu, incl - v, L);
+                    const int base = 64 * (SEL_WARPS - 1 - L);
+                    const int hi = hist0[base + 63 - 2 * lane], lo2 = hist0[base + 62 - 2 * lane];
+                    const int incl2 = warp_inclusive_scan(hi + lo2);
+                    const int excl2 = incl2 - hi - lo2;
+                    if (excl2 < rem1 && incl2 >= rem1) {
+                        const bool upper = excl2 + hi >= rem1;
+                        const int bin = upper ? base + 63 - 2 * lane : base + 62 - 2 * lane;
+                        sh.lo = static_cast<uint32_t>(bin) << 21;
+                        sh.width = static_cast<uint64_t>(1) << 21;
+                        sh.remaining = upper ? rem1 - excl2 : rem1 - excl2 - hi;
+                        sh.bin_count = upper ? hi : lo2;
+                    }
+                }
+            }
+        }
         __syncthreads();  // the key cache and the range are in place
         SEL_TRACE(2);
         // ------------------------------------------------ bucket passes
-        for (int pass = 0;; ++pass) {
+        // (none when the score kernel's first pass already ends the search: every key of the
+        // chosen bucket is taken)
+        for (int pass = 0; !(key_hist != nullptr && sh.remaining == sh.bin_count && sh.width < (1ull << 32));
+             ++pass) {
             const uint32_t lo = sh.lo;
             const uint64_t width = sh.width;
             const int sh_bits = max(0, bit_length(width - 1) - 11);  // bucket width 2^sh_bits, <= 2048 buckets
@@ -314,6 +354,10 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
     SEL_TRACE(8);
     cl.sync();  // slice totals published; also orders the key cache before the emission
     SEL_TRACE(9);
+    // every CTA read the score kernel's counts before the barrier above: zero them for the next
+    // call, each CTA its eighth
+    if (key_hist != nullptr && tid < SEL_BINS / SEL_CL)
+        key_hist[static_cast<int64_t>(b) * SEL_BINS + crank * (SEL_BINS / SEL_CL) + tid] = 0;
     int64_t kept_before = sh.warp_kept[warp], eq_before = sh.warp_eq[warp];
     {
         int vk[SEL_CL], ve[SEL_CL];
@@ -463,13 +507,14 @@ extern "C" __attribute__((visibility("default"))) int tg_trace_read_select(unsig
 cudaError_t launch_select_scan(int mode, const float* scores, const uint8_t* keep_in, const int32_t* cu_seqlens,
                                const int32_t* span, const int32_t* k, const int32_t* cu_kept, int B, int64_t T,
                                uint8_t* keep_out, int32_t* kept_idx, int32_t* pos, int32_t* rank, float* gls,
-                               cudaStream_t st) {
+                               cudaStream_t st, int* key_hist) {
     static std::atomic<uint64_t> attr_set{0};
     if (cudaError_t e = ensure_smem_limit(select_scan_kernel, SEL_SMEM_BYTES, attr_set); e != cudaSuccess)
         return e;
     if (B == 0) return cudaSuccess;
     return launch_pdl(select_scan_kernel, dim3(SEL_CL, B), dim3(SEL_THREADS), static_cast<size_t>(SEL_SMEM_BYTES), st,
-                      mode, scores, keep_in, cu_seqlens, span, k, cu_kept, keep_out, kept_idx, pos, rank, gls);
+                      mode, scores, keep_in, cu_seqlens, span, k, cu_kept, keep_out, kept_idx, pos, rank, gls,
+                      key_hist);
 }
 
 cudaError_t launch_gather_bytes(const void* src, const int32_t* kept_idx, int64_t M_total, int64_t T,

@@ -125,6 +125,15 @@ tg_status do_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
                        "tg_gated_attention launch");
 }
 
+// The prefill layer's workspace: the attention's scratch, then (256-byte aligned) the
+// selection's first-pass histogram, [B][2048] int32, which the score kernel fills and the
+// selection reads and zeroes again.
+size_t prefill_key_hist_offset(int B, int max_M, int Hq, int Hkv, int d, int n_layers) {
+    const size_t attn = n_layers > 0 ? tg_gated_attention_workspace_size(B, max_M, Hq, Hkv, d) : 0;
+    return (attn + 255) & ~static_cast<size_t>(255);
+}
+size_t prefill_key_hist_bytes(int B) { return static_cast<size_t>(B) * 2048 * sizeof(int32_t); }
+
 // Scratch of tg_masked_gated_attention: keep flags, compaction map, the gathered
 // Q/K/V rows, the compacted output and the attention's own split scratch, each
 // 256-byte aligned.
@@ -354,6 +363,11 @@ size_t tg_gated_attention_workspace_size(int B, int max_M, int Hq, int Hkv, int 
     return tg::attention_workspace_bytes(B, max_M, Hq, Hkv, d);
 }
 
+size_t tg_gated_prefill_workspace_size(int B, int max_M, int Hq, int Hkv, int d, int n_layers) {
+    if (B <= 0) return 0;
+    return prefill_key_hist_offset(B, max_M, Hq, Hkv, d, n_layers) + prefill_key_hist_bytes(B);
+}
+
 tg_status tg_gated_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* cu_kept, int B,
                              int64_t M_total, int max_M, int Hq, int Hkv, int d, const int32_t* pos,
                              const int32_t* rank, const float* gls, const float* g, const float* c, float sm_scale,
@@ -537,14 +551,25 @@ tg_status tg_gated_prefill_layer(const tg_prefill_layer_args* a, tg_stream_t str
                        "gather %d: tensors must be 16-byte aligned", i);
         }
     }
+    TG_REQUIRE(a->eps >= 0.f, "eps must be >= 0");
+    if (a->attn_ws) TG_REQUIRE((reinterpret_cast<uintptr_t>(a->attn_ws) & 255u) == 0, "attn_ws must be 256-byte aligned");
     if (tg_status s = check_device()) return s;
     cudaStream_t st = stream;
-    if (tg_status s = do_score(a->hidden, a->cu_seqlens, a->span, a->B, a->T, a->D, a->Wg, a->b1, a->w2, a->b2, a->I,
-                               a->eps, a->scores, st))
+    // A workspace of tg_gated_prefill_workspace_size bytes also holds the selection's
+    // first-pass histogram, which the score kernel then fills (the selection skips that pass).
+    int* key_hist = nullptr;
+    {
+        const size_t off = prefill_key_hist_offset(a->B, a->max_M, a->Hq, a->Hkv, a->d, a->n_layers);
+        if (a->attn_ws && a->attn_ws_bytes >= off + prefill_key_hist_bytes(a->B))
+            key_hist = reinterpret_cast<int*>(static_cast<uint8_t*>(a->attn_ws) + off);
+    }
+    if (tg_status s = cuda_status(tg::launch_score(a->hidden, a->cu_seqlens, a->span, a->B, a->T, a->D, a->Wg, a->b1,
+                                                   a->w2, a->b2, a->I, a->eps, a->scores, st, key_hist),
+                                  "score launch"))
         return s;
     if (tg_status s = cuda_status(tg::launch_select_scan(0, a->scores, nullptr, a->cu_seqlens, a->span, a->k,
                                                          a->cu_kept, a->B, a->T, a->keep, a->kept_idx, a->pos, a->rank,
-                                                         a->gls, st),
+                                                         a->gls, st, key_hist),
                                   "select launch"))
         return s;
     if (a->M_total == 0) return TG_OK;  // every token pruned: no kept rows, no attention

@@ -117,16 +117,21 @@ __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
 cudaError_t launch_gate_prepare(const uint16_t* gamma, const uint16_t* W1, int D, int I, uint16_t* Wg,
                                 cudaStream_t st);
 
+// key_hist (may be NULL): [B][2048] int32, zero on entry; the kernel adds each scored row to
+// bin (score_key(score) >> 21) of its sequence, the selection's first pass (select_scan with
+// the same key_hist uses it and leaves it zero again).
 cudaError_t launch_score(const uint16_t* hidden, const int32_t* cu_seqlens, const int32_t* span, int B,
                          int64_t T, int D, const uint16_t* Wg, const float* b1, const float* w2, float b2, int I,
-                         float eps, float* scores, cudaStream_t st);
+                         float eps, float* scores, cudaStream_t st, int* key_hist = nullptr);
 
 // mode 0: select by score (writes keep; the compaction outputs if non-null)
 // mode 1: compaction scan from caller-given keep flags
+// key_hist (may be NULL): the score kernel's first-pass histogram of these scores; the
+// selection then starts from its second pass and zeroes key_hist before it exits.
 cudaError_t launch_select_scan(int mode, const float* scores, const uint8_t* keep_in, const int32_t* cu_seqlens,
                                const int32_t* span, const int32_t* k, const int32_t* cu_kept, int B, int64_t T,
                                uint8_t* keep_out, int32_t* kept_idx, int32_t* pos, int32_t* rank, float* gls,
-                               cudaStream_t st);
+                               cudaStream_t st, int* key_hist = nullptr);
 
 // dst[m, :] = src[kept_idx[m], :] for rows of row_bytes bytes (4, 8 or a multiple of 16;
 // both pointers aligned to min(row_bytes, 16)); rows whose index lies outside [0, T) are

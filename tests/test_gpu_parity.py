@@ -387,6 +387,48 @@ def test_prefill_layer_end_to_end(tg, name):
     assert math.isfinite(float(s[m].sum()))
 
 
+@pytest.mark.parametrize("name", ["c0_tiny", "c2_32k_k2000", "c4_varlen"])
+def test_prefill_first_pass_in_the_score_kernel(tg, name):
+    """With a workspace of tg_gated_prefill_workspace_size bytes the score kernel builds the
+    selection's first-pass histogram and the selection starts from it; with only the
+    attention's workspace the selection runs every pass.  Both give the same bits
+    everywhere, and the histogram region is zero again after the call."""
+    from learned_token_pruning_rmsnorm_b200 import PrefillBuffers, PrefillCall, _lib
+    w = CONFIGS[name]
+    gi = make_gate_inputs(w)
+    cu, span, k = w.cu_seqlens(), w.span_array(), w.budget_array()
+    M, cu_kept = tg.tg_kept_count(cu, span, k)
+    layers_np = [make_attention_inputs(w, M, layer=0)]
+    layers = [{"q": H.bf16_dev(a["q"]), "k": H.bf16_dev(a["k"]), "v": H.bf16_dev(a["v"]),
+               "g": H.f32_dev(a["g"]), "c": H.f32_dev(a["c"])} for a in layers_np]
+    hid = H.bf16_dev(gi["hidden"])
+    Wg = H.bf16_dev(oracle.gate_fold(gi["gamma"], gi["W1"]))
+    b1, w2 = H.f32_dev(gi["b1"]), H.f32_dev(gi["w2"])
+    lib = _lib.load()
+    max_M = int(np.max(np.diff(cu_kept)))
+    attn_bytes = int(lib.tg_gated_attention_workspace_size(w.B, max_M, w.Hq, w.Hkv, w.d))
+    full_bytes = int(lib.tg_gated_prefill_workspace_size(w.B, max_M, w.Hq, w.Hkv, w.d, 1))
+    hist_off = (attn_bytes + 255) // 256 * 256
+    assert full_bytes == hist_off + w.B * 2048 * 4
+    outs = []
+    for fused in (True, False, True):
+        bufs = PrefillBuffers(w.T, w.D, M, 1, w.Hq, w.d, hid.device, True, True)
+        call = PrefillCall(hid, cu, span, k, Wg, b1, w2, gi["b2"], w.eps, layers, bufs, w.Hq, w.Hkv, w.d)
+        assert call.ws.numel() == full_bytes
+        if not fused:
+            call.args.attn_ws_bytes = attn_bytes
+        call()
+        torch.cuda.synchronize()
+        assert int(torch.count_nonzero(call.ws[hist_off:]).item()) == 0, "histogram left zero"
+        outs.append([x.cpu().numpy() for x in (bufs.scores, bufs.keep, bufs.kept_idx, bufs.pos, bufs.rank,
+                                                bufs.gls, bufs.out[0].view(torch.int16), bufs.lse[0],
+                                                bufs.hidden_kept.view(torch.int16))])
+    for a, b_ in zip(outs[0], outs[1]):
+        np.testing.assert_array_equal(a, b_)
+    for a, b_ in zip(outs[0], outs[2]):
+        np.testing.assert_array_equal(a, b_)
+
+
 # ------------------------------------------------------------------ KV-cache gather (next row f2)
 
 @pytest.mark.parametrize("row_shape", [(8, 128), (2, 64), (8,), (24,), (1, 2056), (1, 1544)])
