@@ -227,13 +227,16 @@ tg_status tg_gated_attention_gates(const uint16_t* q, const uint16_t* k, const u
  *   dg, dc [Hq] fp32 = gradients of the gain and temperature parameters.
  * q, k, v, pos, rank, gls, g, c, cu_kept, sm_scale as passed to the forward;
  * out [M, Hq, d] bf16 and lse [M, Hq] fp32 are the forward's outputs (call
- * tg_gated_attention with a non-NULL lse).  head_dim 64 or 128 (else
- * TG_ERR_UNSUPPORTED).  ws: device scratch, 256-byte aligned, of at least
+ * tg_gated_attention with a non-NULL lse).  head_dim 64, 128 or 256.
+ * ws: device scratch, 256-byte aligned, of at least
  * tg_gated_attention_backward_workspace_size(M_total, Hq, Hkv, d) bytes (6
  * floats per row and head, plus fp32 partial dk and dv per query head when a
- * KV head serves 3, 5, 6, 7 or more than 8 query heads; groups of 2, 4 and 8
- * add theirs inside a thread-block cluster; no zeroing needed).  Tensor cores, no atomics:
- * the results are deterministic.
+ * KV head serves 3, 5, 6, 7 or more than 8 query heads, or any group of two
+ * or more at head_dim 256; groups of 2, 4 and 8 at head_dim 64 and 128 add
+ * theirs inside a thread-block cluster; no zeroing needed).  At head_dim 256
+ * dv and dk are accumulated by two launches over the same keys (the two fp32
+ * accumulators would not fit tensor memory together).  Tensor cores, no
+ * atomics: the results are deterministic.
  */
 size_t tg_gated_attention_backward_workspace_size(int64_t M_total, int Hq, int Hkv, int d);
 tg_status tg_gated_attention_backward(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* out,

@@ -110,14 +110,24 @@ __device__ __forceinline__ bool pair_red_or(int id, bool pred) {
     return res != 0;
 }
 
-template <int HD>
+// PASS 0 computes dV and dK together (head_dim <= 128).  At head_dim 256 the two fp32
+// accumulators alone would fill TMEM, so the work runs as two launches over the same keys:
+// PASS 1 forms P^T and accumulates dV = P^T dO, PASS 2 forms G^T and accumulates dK = G^T Q
+// (and the per-key sums of G); there the (Q, dO) rows stream as half query tiles (64 rows),
+// in two stages for PASS 1 (no V needed) and one for PASS 2 (K and V resident).
+template <int HD, int PASS = 0>
 struct DkvSmem {
+    static constexpr bool QD_HALF = PASS != 0;
+    static constexpr bool HAS_V = PASS != 1;  // dP^T = V dO^T is not needed for dV alone
     static constexpr int TILE = BT * HD * 2;
+    static constexpr int QD_ROWS = QD_HALF ? 64 : BT;
+    static constexpr int QD_STAGE = QD_ROWS * HD * 2;  // the Q (or dO) rows of one stage
+    static constexpr int QD_STAGES = PASS == 2 ? 1 : 2;
     static constexpr int OFF_K = 0;
     static constexpr int OFF_V = OFF_K + TILE;
-    static constexpr int OFF_Q = OFF_V + TILE;         // [2 stages]
-    static constexpr int OFF_DO = OFF_Q + 2 * TILE;    // [2 stages]
-    static constexpr int OFF_TAB = OFF_DO + 2 * TILE;  // [8 warps][2][4][32] fp32 query factors
+    static constexpr int OFF_Q = OFF_V + (HAS_V ? TILE : 0);          // [QD_STAGES]
+    static constexpr int OFF_DO = OFF_Q + QD_STAGES * QD_STAGE;        // [QD_STAGES]
+    static constexpr int OFF_TAB = OFF_DO + QD_STAGES * QD_STAGE;      // [8 warps][2][4][32] fp32 query factors
     static constexpr int OFF_XCH = OFF_TAB + 8 * 2 * 4 * 32 * 4;  // [BT] fp32: the second query half's key sums
     static constexpr int OFF_BAR = OFF_XCH + BT * 4;
     static constexpr int NUM_BARS = 12;
@@ -126,7 +136,8 @@ struct DkvSmem {
     static constexpr int ALLOC = BYTES + 1024;
     static constexpr uint32_t TMEM_COLS = 512;
     static_assert(ALLOC <= 227 * 1024, "shared memory");
-    static_assert(2 * BT + 2 * HD <= 512, "TMEM columns");
+    static_assert(2 * BT + (PASS == 0 ? 2 : 1) * HD <= 512, "TMEM columns");
+    static_assert(PASS != 0 || HD <= 128, "head_dim 256 runs as two passes");
 };
 
 enum : int {
@@ -139,7 +150,7 @@ enum : int {
     D_DRAIN = 10
 };
 
-template <int HD>
+template <int HD, int PASS = 0>
 __global__ void __launch_bounds__(DKV_THREADS, 1)
 gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -149,7 +160,8 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
                           uint16_t* __restrict__ dk, uint16_t* __restrict__ dv, float* __restrict__ part_k,
                           float* __restrict__ part_v, float* __restrict__ colsum, int* __restrict__ status,
                           int cl) {
-    using L = DkvSmem<HD>;
+    using L = DkvSmem<HD, PASS>;
+    constexpr bool DO_DV = PASS != 2, DO_DK = PASS != 1;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     // One query head per CTA.  The heads of a GQA group of 2, 4 or 8 run as one cluster
@@ -202,7 +214,7 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
     const uint32_t tmem = *tmem_slot;
     // half buffer hb: S^T of 64 queries at columns [128 hb, +64), dP^T at [128 hb + 64, +64);
     // P^T and G^T (bf16 pairs) go over the first 32 columns of each
-    const uint32_t tDV = tmem + 2 * BT, tDK = tmem + 2 * BT + HD;
+    const uint32_t tDV = tmem + 2 * BT, tDK = tmem + 2 * BT + (PASS == 0 ? HD : 0);
 
     bool epi_ok = false;  // a compute thread's accumulators are complete
     if (warp == 8) {
@@ -212,28 +224,50 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
             prefetch_tmap(&tmK);
             prefetch_tmap(&tmV);
             prefetch_tmap(&tmDO);
-            mbar_expect_tx(bar(D_KV_FULL), 2 * L::TILE);
+            mbar_expect_tx(bar(D_KV_FULL), (L::HAS_V ? 2 : 1) * L::TILE);
 #pragma unroll
             for (int hf = 0; hf < HD / 64; ++hf) {
                 tma_load_2d(sK + hf * BT * 128, &tmK, hk * HD + hf * 64, seq0 + kt * BT, bar(D_KV_FULL));
-                tma_load_2d(sV + hf * BT * 128, &tmV, hk * HD + hf * 64, seq0 + kt * BT, bar(D_KV_FULL));
+                if (L::HAS_V)
+                    tma_load_2d(sV + hf * BT * 128, &tmV, hk * HD + hf * 64, seq0 + kt * BT, bar(D_KV_FULL));
             }
             int issued[2] = {0, 0};
-            for (int t = 0; t < nq; ++t) {
-                const int s = t & 1;
-                const int i = kt + t;
-                if (t >= 2 && !mbar_wait(bar(D_QD_EMPTY + s), ((t - 2) >> 1) & 1, abort_flag, status,
-                                         TG_WHERE_PRODUCER))
-                    break;
-                mbar_expect_tx(bar(D_QD_FULL + s), 2 * L::TILE);
+            if constexpr (L::QD_HALF) {
+                // half query tile u (64 rows: tile kt + u / 2, rows 64 (u & 1) ..) into stage u % S
+                constexpr int S = L::QD_STAGES;
+                for (int u = 0; u < 2 * nq; ++u) {
+                    const int s = u % S;
+                    if (u >= S && !mbar_wait(bar(D_QD_EMPTY + s), ((u / S) - 1) & 1, abort_flag, status,
+                                             TG_WHERE_PRODUCER))
+                        break;
+                    mbar_expect_tx(bar(D_QD_FULL + s), 2 * L::QD_STAGE);
+                    const int row = seq0 + kt * BT + u * 64;
 #pragma unroll
-                for (int hf = 0; hf < HD / 64; ++hf) {
-                    tma_load_2d(sQ + s * L::TILE + hf * BT * 128, &tmQ, h * HD + hf * 64, seq0 + i * BT,
-                                bar(D_QD_FULL + s));
-                    tma_load_2d(sDO + s * L::TILE + hf * BT * 128, &tmDO, h * HD + hf * 64, seq0 + i * BT,
-                                bar(D_QD_FULL + s));
+                    for (int hf = 0; hf < HD / 64; ++hf) {
+                        tma_load_2d(sQ + s * L::QD_STAGE + hf * 64 * 128, &tmQ, h * HD + hf * 64, row,
+                                    bar(D_QD_FULL + s));
+                        tma_load_2d(sDO + s * L::QD_STAGE + hf * 64 * 128, &tmDO, h * HD + hf * 64, row,
+                                    bar(D_QD_FULL + s));
+                    }
+                    ++issued[s];
                 }
-                ++issued[s];
+            } else {
+                for (int t = 0; t < nq; ++t) {
+                    const int s = t & 1;
+                    const int i = kt + t;
+                    if (t >= 2 && !mbar_wait(bar(D_QD_EMPTY + s), ((t - 2) >> 1) & 1, abort_flag, status,
+                                             TG_WHERE_PRODUCER))
+                        break;
+                    mbar_expect_tx(bar(D_QD_FULL + s), 2 * L::TILE);
+#pragma unroll
+                    for (int hf = 0; hf < HD / 64; ++hf) {
+                        tma_load_2d(sQ + s * L::TILE + hf * BT * 128, &tmQ, h * HD + hf * 64, seq0 + i * BT,
+                                    bar(D_QD_FULL + s));
+                        tma_load_2d(sDO + s * L::TILE + hf * BT * 128, &tmDO, h * HD + hf * 64, seq0 + i * BT,
+                                    bar(D_QD_FULL + s));
+                    }
+                    ++issued[s];
+                }
             }
             if (*abort_flag) {
                 drain_wait_b(bar(D_KV_FULL), 0, status);
@@ -249,64 +283,96 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
             // Matrix descriptors are built once per stage; an operand at a byte offset is the
             // same descriptor with offset / 16 added to its start-address field (shared-memory
             // addresses stay below 2^18, so the 14-bit field never carries).
+            // (half-tile stages hold only half u: no offset for hb, and the rows' 64-column boxes
+            // are QD_ROWS * 128 bytes apart)
+            constexpr int QS = L::QD_HALF ? L::QD_STAGE : L::TILE;  // bytes between stages
+            constexpr uint32_t QBOX = L::QD_ROWS * 128;
             const uint64_t kd = smem_desc_sw128(sK, 16, 1024), vd = smem_desc_sw128(sV, 16, 1024);
-            const uint64_t qd0 = smem_desc_sw128(sQ, 16, 1024), qd1 = smem_desc_sw128(sQ + L::TILE, 16, 1024);
-            const uint64_t dd0 = smem_desc_sw128(sDO, 16, 1024), dd1 = smem_desc_sw128(sDO + L::TILE, 16, 1024);
-            const uint64_t qm0 = smem_desc_sw128(sQ, BT * 128, 1024), qm1 = smem_desc_sw128(sQ + L::TILE, BT * 128, 1024);
-            const uint64_t dm0 = smem_desc_sw128(sDO, BT * 128, 1024),
-                           dm1 = smem_desc_sw128(sDO + L::TILE, BT * 128, 1024);
+            const uint64_t qd0 = smem_desc_sw128(sQ, 16, 1024), qd1 = smem_desc_sw128(sQ + QS, 16, 1024);
+            const uint64_t dd0 = smem_desc_sw128(sDO, 16, 1024), dd1 = smem_desc_sw128(sDO + QS, 16, 1024);
+            const uint64_t qm0 = smem_desc_sw128(sQ, QBOX, 1024), qm1 = smem_desc_sw128(sQ + QS, QBOX, 1024);
+            const uint64_t dm0 = smem_desc_sw128(sDO, QBOX, 1024), dm1 = smem_desc_sw128(sDO + QS, QBOX, 1024);
+            auto stage_of = [&](int u) { return L::QD_HALF ? u % L::QD_STAGES : (u >> 1) & 1; };
+            auto hoff_of = [&](int u) {
+                return L::QD_HALF ? 0u : static_cast<uint32_t>(((u & 1) * 64 * 128) >> 4);
+            };
             // Half step u: query tile u >> 1, queries 64 (u & 1) .. +63 (64 rows = 8 KB into
             // each swizzled box of the stage), TMEM buffer u & 1.
             auto issue_sdp = [&](int u) {
-                const int hb = u & 1, s = (u >> 1) & 1;
+                const int hb = u & 1, s = stage_of(u);
                 const uint32_t tb = tmem + hb * 128;
-                const uint64_t qb = (s ? qd1 : qd0) + ((hb * 64 * 128) >> 4);
-                const uint64_t db = (s ? dd1 : dd0) + ((hb * 64 * 128) >> 4);
+                const uint64_t qb = (s ? qd1 : qd0) + hoff_of(u);
+                const uint64_t db = (s ? dd1 : dd0) + hoff_of(u);
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk) {
                     const uint32_t off = ((kk >> 2) * (BT * 128) + (kk & 3) * 32) >> 4;
-                    mma_bf16_ss(tb, kd + off, qb + off, idesc_s, kk > 0 ? 1u : 0u);
+                    const uint32_t offq = ((kk >> 2) * QBOX + (kk & 3) * 32) >> 4;
+                    mma_bf16_ss(tb, kd + off, qb + offq, idesc_s, kk > 0 ? 1u : 0u);
                 }
+                if (DO_DK) {
 #pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk) {
-                    const uint32_t off = ((kk >> 2) * (BT * 128) + (kk & 3) * 32) >> 4;
-                    mma_bf16_ss(tb + 64, vd + off, db + off, idesc_s, kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < HD / 16; ++kk) {
+                        const uint32_t off = ((kk >> 2) * (BT * 128) + (kk & 3) * 32) >> 4;
+                        const uint32_t offq = ((kk >> 2) * QBOX + (kk & 3) * 32) >> 4;
+                        mma_bf16_ss(tb + 64, vd + off, db + offq, idesc_s, kk > 0 ? 1u : 0u);
+                    }
                 }
                 mma_commit(bar(D_SDP_FULL + hb));
             };
             // dV += P^T dO(half), dK += G^T Q(half): A from TMEM (16 queries = 8 columns per
             // k-step), B the (query x head_dim) rows read MN-major
             auto issue_acc = [&](int u) {
-                const int hb = u & 1, s = (u >> 1) & 1;
+                const int hb = u & 1, s = stage_of(u);
                 const uint32_t tb = tmem + hb * 128;
-                const uint64_t db = (s ? dm1 : dm0) + ((hb * 64 * 128) >> 4);
-                const uint64_t qb = (s ? qm1 : qm0) + ((hb * 64 * 128) >> 4);
+                const uint64_t db = (s ? dm1 : dm0) + hoff_of(u);
+                const uint64_t qb = (s ? qm1 : qm0) + hoff_of(u);
+                if (DO_DV) {
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16_ts(tDV, tb + kk * 8, db + ((kk * 16 * 128) >> 4), idesc_acc,
-                                (u > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16_ts(tDV, tb + kk * 8, db + ((kk * 16 * 128) >> 4), idesc_acc,
+                                    (u > 0 || kk > 0) ? 1u : 0u);
+                }
+                if (DO_DK) {
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16_ts(tDK, tb + 64 + kk * 8, qb + ((kk * 16 * 128) >> 4), idesc_acc,
-                                (u > 0 || kk > 0) ? 1u : 0u);
-                if (hb == 1) mma_commit(bar(D_QD_EMPTY + s));  // the stage is no longer read
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16_ts(tDK, tb + 64 + kk * 8, qb + ((kk * 16 * 128) >> 4), idesc_acc,
+                                    (u > 0 || kk > 0) ? 1u : 0u);
+                }
+                if (L::QD_HALF || hb == 1) mma_commit(bar(D_QD_EMPTY + s));  // the stage is no longer read
             };
             const int n_u = 2 * nq;
             bool ok = mbar_wait(bar(D_KV_FULL), 0, abort_flag, status, TG_WHERE_MMA);
             for (int u = 0; ok && u < n_u; ++u) {
-                const int t = u >> 1, s = t & 1;
-                if ((u & 1) == 0) {
-                    ok = mbar_wait(bar(D_QD_FULL + s), (t >> 1) & 1, abort_flag, status, TG_WHERE_MMA);
-                    if (!ok) break;
-                }
-                tc_fence_after();
-                issue_sdp(u);
-                if (u >= 1) {
-                    ok = mbar_wait(bar(D_PG_FULL + ((u - 1) & 1)), ((u - 1) >> 1) & 1, abort_flag, status,
-                                   TG_WHERE_MMA);
+                if constexpr (L::QD_HALF && L::QD_STAGES == 1) {
+                    // one stage: the products of half u - 1 read it and must go out (releasing it)
+                    // before half u can land, so they precede S(u) here
+                    if (u >= 1) {
+                        ok = mbar_wait(bar(D_PG_FULL + ((u - 1) & 1)), ((u - 1) >> 1) & 1, abort_flag, status,
+                                       TG_WHERE_MMA);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_acc(u - 1);
+                    }
+                    ok = mbar_wait(bar(D_QD_FULL), u & 1, abort_flag, status, TG_WHERE_MMA);
                     if (!ok) break;
                     tc_fence_after();
-                    issue_acc(u - 1);
+                    issue_sdp(u);
+                } else {
+                    if (L::QD_HALF || (u & 1) == 0) {
+                        const int s = stage_of(u);
+                        const int use = L::QD_HALF ? u / L::QD_STAGES : u >> 2;
+                        ok = mbar_wait(bar(D_QD_FULL + s), use & 1, abort_flag, status, TG_WHERE_MMA);
+                        if (!ok) break;
+                    }
+                    tc_fence_after();
+                    issue_sdp(u);
+                    if (u >= 1) {
+                        ok = mbar_wait(bar(D_PG_FULL + ((u - 1) & 1)), ((u - 1) >> 1) & 1, abort_flag, status,
+                                       TG_WHERE_MMA);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_acc(u - 1);
+                    }
                 }
             }
             if (ok) ok = mbar_wait(bar(D_PG_FULL + ((n_u - 1) & 1)), ((n_u - 1) >> 1) & 1, abort_flag, status,
@@ -365,8 +431,12 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
             if (okw) {
                 tc_fence_after();
                 tmem_ld32(tb + cs * 32, sx);
-                tmem_ld32(tb + 64 + cs * 32, dpx);
+                if (DO_DK) tmem_ld32(tb + 64 + cs * 32, dpx);
                 tmem_wait_ld();
+            }
+            if (!DO_DK) {
+#pragma unroll
+                for (int x = 0; x < 32; ++x) dpx[x] = 0.f;  // (not used: the dV pass forms no G)
             }
             // both warps of the row group have read their columns (the P^T / G^T stores
             // below overwrite some of the partner's); an abort is decided by the pair
@@ -398,8 +468,8 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
                     const int k = k4 + x;
                     const float tt = fmaf(fav[x], sx[k] + kgl, flv[x]);
                     const float p = (live >> k) & 1u ? ex2_approx(tt) : 0.f;
-                    const float G = p * fmaf(fiv[x], dpx[k], fdv[x]);
-                    csum += G;
+                    const float G = DO_DK ? p * fmaf(fiv[x], dpx[k], fdv[x]) : 0.f;
+                    if (DO_DK) csum += G;
                     pv[x] = p;
                     gv[x] = G;
                 }
@@ -408,8 +478,8 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
                 gg[k4 / 2] = pack2_bf16(gv[0], gv[1]);
                 gg[k4 / 2 + 1] = pack2_bf16(gv[2], gv[3]);
             }
-            tmem_st16u(tb + cs * 16, pp);       // P^T of these 32 queries over S^T
-            tmem_st16u(tb + 64 + cs * 16, gg);  // G^T over dP^T
+            if (DO_DV) tmem_st16u(tb + cs * 16, pp);       // P^T of these 32 queries over S^T
+            if (DO_DK) tmem_st16u(tb + 64 + cs * 16, gg);  // G^T over dP^T
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar(D_PG_FULL + hb));
@@ -418,11 +488,11 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
         float* xch = reinterpret_cast<float*>(smem + L::OFF_XCH);
         if (cs == 1) xch[r] = csum;
         asm volatile("bar.sync 1, 256;" ::: "memory");
-        if (cs == 0 && ok && valid_key) colsum[static_cast<size_t>(seq0 + key_local) * Hq + h] = csum + xch[r];
+        if (DO_DK && cs == 0 && ok && valid_key) colsum[static_cast<size_t>(seq0 + key_local) * Hq + h] = csum + xch[r];
         // ---------------------------------------------------------------- epilogue
         if (ok) ok = mbar_wait_warp(bar(D_ACC_DONE), 0, abort_flag, status, TG_WHERE_SOFTMAX);
         epi_ok = ok;
-        if (cl > 1) {
+        if (PASS == 0 && cl > 1) {
             // heads 1 .. cl-1 of the group: this head's fp32 dV and dK into the exchange area
             // (the Q/dO stages, idle now), [dV|dK][HD/4 column quads][128 rows] float4s
             if (ok && hh != 0) {
@@ -449,7 +519,7 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
             tc_fence_after();
             const size_t row = ((static_cast<size_t>(hh) * M_total + seq0 + key_local) * Hkv + hk) * HD + cs * (HD / 2);
 #pragma unroll 1
-            for (int which = 0; which < 2; ++which) {
+            for (int which = DO_DV ? 0 : 1; which < (DO_DK ? 2 : 1); ++which) {
                 const uint32_t src = (which ? tDK : tDV) + cs * (HD / 2);
                 float* dst = (which ? part_k : part_v) + row;
 #pragma unroll
@@ -469,7 +539,7 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
             tc_fence_after();
             const size_t row = (static_cast<size_t>(seq0 + key_local) * Hkv + hk) * HD + cs * (HD / 2);
 #pragma unroll 1
-            for (int which = 0; which < 2; ++which) {
+            for (int which = DO_DV ? 0 : 1; which < (DO_DK ? 2 : 1); ++which) {
                 const uint32_t src = (which ? tDK : tDV) + cs * (HD / 2);
                 const float scale = which ? sm_scale : 1.0f;
                 uint16_t* dst = (which ? dk : dv) + row;
@@ -496,7 +566,7 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
 
     tc_fence_before();
     __syncthreads();
-    if (cl > 1) {
+    if (PASS == 0 && cl > 1) {
         // every thread of the cluster, abort or not
         cluster_sync_all();  // the other heads' copies are in their shared memory
         if (hh == 0 && warp < 8 && epi_ok) {
@@ -566,12 +636,18 @@ gated_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_
 // row, dl l (for dtau).
 template <int HD>
 struct DqSmem {
+    // head_dim 256: K and V stream as single-buffered half tiles (64 keys), so that they fit
+    // beside the resident Q and dO; otherwise whole tiles in two stages
+    static constexpr bool KV_HALF = HD > 128;
     static constexpr int TILE = BT * HD * 2;
+    static constexpr int KV_ROWS = KV_HALF ? 64 : BT;
+    static constexpr int KV_STAGE = KV_ROWS * HD * 2;
+    static constexpr int KV_STAGES = KV_HALF ? 1 : 2;
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_DO = OFF_Q + TILE;
-    static constexpr int OFF_K = OFF_DO + TILE;        // [2 stages]
-    static constexpr int OFF_V = OFF_K + 2 * TILE;     // [2 stages]
-    static constexpr int OFF_GLS = OFF_V + 2 * TILE;   // [8 warps][2][BT] fp32, a private copy per warp
+    static constexpr int OFF_K = OFF_DO + TILE;                     // [KV_STAGES]
+    static constexpr int OFF_V = OFF_K + KV_STAGES * KV_STAGE;      // [KV_STAGES]
+    static constexpr int OFF_GLS = OFF_V + KV_STAGES * KV_STAGE;    // [8 warps][2][BT] fp32, a private copy per warp
     static constexpr int OFF_XCH = OFF_GLS + 8 * 2 * BT * 4;  // [6][BT] fp32: row sums [0..3], D halves [4..5]
     static constexpr int OFF_BAR = OFF_XCH + 6 * BT * 4;
     static constexpr int NUM_BARS = 16;
@@ -664,26 +740,47 @@ gated_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
                 tma_load_2d(sDO + hf * BT * 128, &tmDO, h * HD + hf * 64, seq0 + qt * BT, bar(Q_QD_FULL));
             }
             int k_issued[2] = {0, 0}, v_issued[2] = {0, 0};
-            for (int j = 0; j < n_kv; ++j) {
-                const int s = j & 1;
-                if (j >= 2 && !mbar_wait(bar(Q_K_EMPTY + s), ((j - 2) >> 1) & 1, abort_flag, status,
-                                         TG_WHERE_PRODUCER))
-                    break;
-                mbar_expect_tx(bar(Q_K_FULL + s), L::TILE);
+            if constexpr (L::KV_HALF) {
+                // one half tile (64 keys) per step u, one stage: the next half's K loads once the
+                // previous half's dQ product has read K, its V once that half's dP has read V
+                for (int u = 0; u < 2 * n_kv; ++u) {
+                    if (u >= 1 && !mbar_wait(bar(Q_K_EMPTY), (u - 1) & 1, abort_flag, status, TG_WHERE_PRODUCER))
+                        break;
+                    mbar_expect_tx(bar(Q_K_FULL), L::KV_STAGE);
 #pragma unroll
-                for (int hf = 0; hf < HD / 64; ++hf)
-                    tma_load_2d(sK + s * L::TILE + hf * BT * 128, &tmK, hk * HD + hf * 64, seq0 + j * BT,
-                                bar(Q_K_FULL + s));
-                ++k_issued[s];
-                if (j >= 2 && !mbar_wait(bar(Q_V_EMPTY + s), ((j - 2) >> 1) & 1, abort_flag, status,
-                                         TG_WHERE_PRODUCER))
-                    break;
-                mbar_expect_tx(bar(Q_V_FULL + s), L::TILE);
+                    for (int hf = 0; hf < HD / 64; ++hf)
+                        tma_load_2d(sK + hf * 64 * 128, &tmK, hk * HD + hf * 64, seq0 + u * 64, bar(Q_K_FULL));
+                    ++k_issued[0];
+                    if (u >= 1 && !mbar_wait(bar(Q_V_EMPTY), (u - 1) & 1, abort_flag, status, TG_WHERE_PRODUCER))
+                        break;
+                    mbar_expect_tx(bar(Q_V_FULL), L::KV_STAGE);
 #pragma unroll
-                for (int hf = 0; hf < HD / 64; ++hf)
-                    tma_load_2d(sV + s * L::TILE + hf * BT * 128, &tmV, hk * HD + hf * 64, seq0 + j * BT,
-                                bar(Q_V_FULL + s));
-                ++v_issued[s];
+                    for (int hf = 0; hf < HD / 64; ++hf)
+                        tma_load_2d(sV + hf * 64 * 128, &tmV, hk * HD + hf * 64, seq0 + u * 64, bar(Q_V_FULL));
+                    ++v_issued[0];
+                }
+            } else {
+                for (int j = 0; j < n_kv; ++j) {
+                    const int s = j & 1;
+                    if (j >= 2 && !mbar_wait(bar(Q_K_EMPTY + s), ((j - 2) >> 1) & 1, abort_flag, status,
+                                             TG_WHERE_PRODUCER))
+                        break;
+                    mbar_expect_tx(bar(Q_K_FULL + s), L::TILE);
+#pragma unroll
+                    for (int hf = 0; hf < HD / 64; ++hf)
+                        tma_load_2d(sK + s * L::TILE + hf * BT * 128, &tmK, hk * HD + hf * 64, seq0 + j * BT,
+                                    bar(Q_K_FULL + s));
+                    ++k_issued[s];
+                    if (j >= 2 && !mbar_wait(bar(Q_V_EMPTY + s), ((j - 2) >> 1) & 1, abort_flag, status,
+                                             TG_WHERE_PRODUCER))
+                        break;
+                    mbar_expect_tx(bar(Q_V_FULL + s), L::TILE);
+#pragma unroll
+                    for (int hf = 0; hf < HD / 64; ++hf)
+                        tma_load_2d(sV + s * L::TILE + hf * BT * 128, &tmV, hk * HD + hf * 64, seq0 + j * BT,
+                                    bar(Q_V_FULL + s));
+                    ++v_issued[s];
+                }
             }
             if (*abort_flag) {
                 drain_wait_b(bar(Q_QD_FULL), 0, status);
@@ -705,54 +802,78 @@ gated_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
             // thread, so executed earlier -- has read.
             // Descriptors built once, as in the dK/dV kernel.
             const uint64_t qd = smem_desc_sw128(sQ, 16, 1024), dd = smem_desc_sw128(sDO, 16, 1024);
-            const uint64_t kd0 = smem_desc_sw128(sK, 16, 1024), kd1 = smem_desc_sw128(sK + L::TILE, 16, 1024);
-            const uint64_t vd0 = smem_desc_sw128(sV, 16, 1024), vd1 = smem_desc_sw128(sV + L::TILE, 16, 1024);
-            const uint64_t km0 = smem_desc_sw128(sK, BT * 128, 1024), km1 = smem_desc_sw128(sK + L::TILE, BT * 128, 1024);
+            const uint64_t kd0 = smem_desc_sw128(sK, 16, 1024), kd1 = smem_desc_sw128(sK + L::KV_STAGE, 16, 1024);
+            const uint64_t vd0 = smem_desc_sw128(sV, 16, 1024), vd1 = smem_desc_sw128(sV + L::KV_STAGE, 16, 1024);
+            const uint64_t km0 = smem_desc_sw128(sK, L::KV_ROWS * 128, 1024),
+                           km1 = smem_desc_sw128(sK + L::KV_STAGE, L::KV_ROWS * 128, 1024);
+            // (with half-tile stages the K/V stage holds only half u, so there is no offset for hb,
+            // and the K/V rows' 64-column boxes are KV_ROWS * 128 bytes apart instead of BT * 128)
             auto issue_sdp = [&](int u) {
-                const int hb = u & 1, s = (u >> 1) & 1;
+                const int hb = u & 1, s = L::KV_HALF ? 0 : (u >> 1) & 1;
                 const uint32_t tb = tmem + hb * 128;
-                const uint64_t kb = (s ? kd1 : kd0) + ((hb * 64 * 128) >> 4);
-                const uint64_t vb = (s ? vd1 : vd0) + ((hb * 64 * 128) >> 4);
+                const uint32_t hoff = L::KV_HALF ? 0u : static_cast<uint32_t>((hb * 64 * 128) >> 4);
+                const uint64_t kb = (s ? kd1 : kd0) + hoff;
+                const uint64_t vb = (s ? vd1 : vd0) + hoff;
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk) {
                     const uint32_t off = ((kk >> 2) * (BT * 128) + (kk & 3) * 32) >> 4;
-                    mma_bf16_ss(tb, qd + off, kb + off, idesc_s, kk > 0 ? 1u : 0u);
+                    const uint32_t offk = ((kk >> 2) * (L::KV_ROWS * 128) + (kk & 3) * 32) >> 4;
+                    mma_bf16_ss(tb, qd + off, kb + offk, idesc_s, kk > 0 ? 1u : 0u);
                 }
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk) {
                     const uint32_t off = ((kk >> 2) * (BT * 128) + (kk & 3) * 32) >> 4;
-                    mma_bf16_ss(tb + 64, dd + off, vb + off, idesc_s, kk > 0 ? 1u : 0u);
+                    const uint32_t offk = ((kk >> 2) * (L::KV_ROWS * 128) + (kk & 3) * 32) >> 4;
+                    mma_bf16_ss(tb + 64, dd + off, vb + offk, idesc_s, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(bar(Q_SDP_FULL + hb));
-                if (hb == 1) mma_commit(bar(Q_V_EMPTY + s));  // V(tile) is no longer read
+                if (L::KV_HALF || hb == 1) mma_commit(bar(Q_V_EMPTY + s));  // V of this stage is no longer read
             };
             // dQ += G(u) K(half of u): A from TMEM (16 keys = 8 columns per k-step), B the K rows MN-major
             auto issue_dq = [&](int u) {
-                const int hb = u & 1, s = (u >> 1) & 1;
-                const uint64_t kb = (s ? km1 : km0) + ((hb * 64 * 128) >> 4);
+                const int hb = u & 1, s = L::KV_HALF ? 0 : (u >> 1) & 1;
+                const uint32_t hoff = L::KV_HALF ? 0u : static_cast<uint32_t>((hb * 64 * 128) >> 4);
+                const uint64_t kb = (s ? km1 : km0) + hoff;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     mma_bf16_ts(tDQ, tmem + hb * 128 + kk * 8, kb + ((kk * 16 * 128) >> 4), idesc_acc,
                                 (u > 0 || kk > 0) ? 1u : 0u);
-                if (hb == 1) mma_commit(bar(Q_K_EMPTY + s));  // K(tile) is no longer read
+                if (L::KV_HALF || hb == 1) mma_commit(bar(Q_K_EMPTY + s));  // K of this stage is no longer read
             };
             const int n_u = 2 * n_kv;
             bool ok = mbar_wait(bar(Q_QD_FULL), 0, abort_flag, status, TG_WHERE_MMA);
             for (int u = 0; ok && u < n_u; ++u) {
                 const int j = u >> 1, s = j & 1;
-                if ((u & 1) == 0) {
-                    ok = mbar_wait(bar(Q_K_FULL + s), (j >> 1) & 1, abort_flag, status, TG_WHERE_MMA);
-                    if (ok) ok = mbar_wait(bar(Q_V_FULL + s), (j >> 1) & 1, abort_flag, status, TG_WHERE_MMA);
-                    if (!ok) break;
-                }
-                tc_fence_after();
-                issue_sdp(u);
-                if (u >= 1) {
-                    ok = mbar_wait(bar(Q_G_FULL + ((u - 1) & 1)), ((u - 1) >> 1) & 1, abort_flag, status,
-                                   TG_WHERE_MMA);
+                if constexpr (L::KV_HALF) {
+                    // one stage: dQ(u - 1) reads K(u - 1) and must go out (releasing the stage)
+                    // before K(u) can land, so it precedes S(u) here
+                    if (u >= 1) {
+                        ok = mbar_wait(bar(Q_G_FULL + ((u - 1) & 1)), ((u - 1) >> 1) & 1, abort_flag, status,
+                                       TG_WHERE_MMA);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_dq(u - 1);
+                    }
+                    ok = mbar_wait(bar(Q_K_FULL), u & 1, abort_flag, status, TG_WHERE_MMA);
+                    if (ok) ok = mbar_wait(bar(Q_V_FULL), u & 1, abort_flag, status, TG_WHERE_MMA);
                     if (!ok) break;
                     tc_fence_after();
-                    issue_dq(u - 1);
+                    issue_sdp(u);
+                } else {
+                    if ((u & 1) == 0) {
+                        ok = mbar_wait(bar(Q_K_FULL + s), (j >> 1) & 1, abort_flag, status, TG_WHERE_MMA);
+                        if (ok) ok = mbar_wait(bar(Q_V_FULL + s), (j >> 1) & 1, abort_flag, status, TG_WHERE_MMA);
+                        if (!ok) break;
+                    }
+                    tc_fence_after();
+                    issue_sdp(u);
+                    if (u >= 1) {
+                        ok = mbar_wait(bar(Q_G_FULL + ((u - 1) & 1)), ((u - 1) >> 1) & 1, abort_flag, status,
+                                       TG_WHERE_MMA);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_dq(u - 1);
+                    }
                 }
             }
             if (ok) ok = mbar_wait(bar(Q_G_FULL + ((n_u - 1) & 1)), ((n_u - 1) >> 1) & 1, abort_flag, status,
@@ -1084,10 +1205,17 @@ cudaError_t launch_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
                        int max_M, int Hq, int Hkv, const int32_t* pos, const int32_t* rank, const GateSet& gates,
                        const float* c, float sm_scale, uint16_t* dq, uint16_t* dk, uint16_t* dv,
                        const BwdGateOut& gout, float* dc, void* ws, cudaStream_t st) {
-    static std::atomic<uint64_t> set_dkv{0}, set_dq{0};
-    if (cudaError_t e = ensure_smem_limit(gated_attn_bwd_dkv_kernel<HD>, DkvSmem<HD>::ALLOC, set_dkv);
+    constexpr bool TWO_PASS = HD > 128;  // dV and dK in two launches (see DkvSmem)
+    constexpr int P1 = TWO_PASS ? 1 : 0;
+    static std::atomic<uint64_t> set_dkv{0}, set_dkv2{0}, set_dq{0};
+    if (cudaError_t e = ensure_smem_limit(gated_attn_bwd_dkv_kernel<HD, P1>, DkvSmem<HD, P1>::ALLOC, set_dkv);
         e != cudaSuccess)
         return e;
+    if constexpr (TWO_PASS) {
+        if (cudaError_t e = ensure_smem_limit(gated_attn_bwd_dkv_kernel<HD, 2>, DkvSmem<HD, 2>::ALLOC, set_dkv2);
+            e != cudaSuccess)
+            return e;
+    }
     if (cudaError_t e = ensure_smem_limit(gated_attn_bwd_dq_kernel<HD>, DqSmem<HD>::ALLOC, set_dq); e != cudaSuccess)
         return e;
     const size_t rows = static_cast<size_t>(M_total) * Hq;
@@ -1097,19 +1225,22 @@ cudaError_t launch_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
     float* colsum = reinterpret_cast<float*>(fac + rows);
     float* tileT = colsum + rows4;  // per query tile, at its first row
     const int grp = Hq / Hkv;
-    const int cl = bwd_cluster_size(grp);  // the group's heads as one cluster, else partials
+    // the group's heads as one cluster (its exchange area holds a head's fp32 dV and dK only at
+    // head_dim <= 128), else partials
+    const int cl = TWO_PASS ? 0 : bwd_cluster_size(grp);
     const int64_t nkv = M_total * Hkv * HD;
     float* part_k = grp > 1 && cl == 0 ? tileT + rows4 : nullptr;  // [grp][M][Hkv][HD] each
     float* part_v = part_k ? part_k + grp * nkv : nullptr;
-    CUtensorMap tq, tk, tv, tdo;
-    if (!encode_tmap_2d_bf16(&tq, q, static_cast<uint64_t>(Hq) * HD, static_cast<uint64_t>(M_total),
-                             static_cast<uint64_t>(Hq) * HD * 2, 64, BT) ||
-        !encode_tmap_2d_bf16(&tdo, dout, static_cast<uint64_t>(Hq) * HD, static_cast<uint64_t>(M_total),
-                             static_cast<uint64_t>(Hq) * HD * 2, 64, BT) ||
-        !encode_tmap_2d_bf16(&tk, k, static_cast<uint64_t>(Hkv) * HD, static_cast<uint64_t>(M_total),
-                             static_cast<uint64_t>(Hkv) * HD * 2, 64, BT) ||
-        !encode_tmap_2d_bf16(&tv, v, static_cast<uint64_t>(Hkv) * HD, static_cast<uint64_t>(M_total),
-                             static_cast<uint64_t>(Hkv) * HD * 2, 64, BT))
+    // tensor maps: whole 128-row tiles, and (head_dim 256) 64-row half tiles for the rows
+    // that stream: K/V in the dQ kernel, Q/dO in the dK/dV passes
+    constexpr uint32_t HR = TWO_PASS ? 64 : BT;
+    CUtensorMap tq, tk, tv, tdo, tq_s, tk_s, tv_s, tdo_s;
+    auto enc = [&](CUtensorMap* m, const uint16_t* p, int H, uint32_t rows) {
+        return encode_tmap_2d_bf16(m, p, static_cast<uint64_t>(H) * HD, static_cast<uint64_t>(M_total),
+                                   static_cast<uint64_t>(H) * HD * 2, 64, rows);
+    };
+    if (!enc(&tq, q, Hq, BT) || !enc(&tdo, dout, Hq, BT) || !enc(&tk, k, Hkv, BT) || !enc(&tv, v, Hkv, BT) ||
+        !enc(&tq_s, q, Hq, HR) || !enc(&tdo_s, dout, Hq, HR) || !enc(&tk_s, k, Hkv, HR) || !enc(&tv_s, v, Hkv, HR))
         return cudaErrorInvalidValue;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
@@ -1119,10 +1250,20 @@ cudaError_t launch_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
     // dq first: it forms each row's D = dout . out for its own use and leaves the exact
     // D' = sum_j P dP for the dK/dV kernel
     cudaError_t e = launch_pdl(gated_attn_bwd_dq_kernel<HD>, dim3(Hq, n_t, B), dim3(DQ_THREADS),
-                               static_cast<size_t>(DqSmem<HD>::ALLOC), st, tq, tk, tv, tdo, cu_kept, pos, rank, gates,
-                               c, lse, out, fac, sm_scale, Hq, Hkv, n_t, dq, tileT, status);
+                               static_cast<size_t>(DqSmem<HD>::ALLOC), st, tq, tk_s, tv_s, tdo, cu_kept, pos, rank,
+                               gates, c, lse, out, fac, sm_scale, Hq, Hkv, n_t, dq, tileT, status);
     if (e != cudaSuccess) return e;
-    if (cl > 1)
+    if constexpr (TWO_PASS) {
+        e = launch_pdl(gated_attn_bwd_dkv_kernel<HD, 1>, dim3(Hq, n_t, B), dim3(DKV_THREADS),
+                       static_cast<size_t>(DkvSmem<HD, 1>::ALLOC), st, tq_s, tk, tv, tdo_s, cu_kept, gates,
+                       static_cast<const float4*>(fac), sm_scale, Hq, Hkv, M_total, dk, dv, part_k, part_v, colsum,
+                       status, 0);
+        if (e == cudaSuccess)
+            e = launch_pdl(gated_attn_bwd_dkv_kernel<HD, 2>, dim3(Hq, n_t, B), dim3(DKV_THREADS),
+                           static_cast<size_t>(DkvSmem<HD, 2>::ALLOC), st, tq_s, tk, tv, tdo_s, cu_kept, gates,
+                           static_cast<const float4*>(fac), sm_scale, Hq, Hkv, M_total, dk, dv, part_k, part_v,
+                           colsum, status, 0);
+    } else if (cl > 1)
         e = launch_pdl_cluster(gated_attn_bwd_dkv_kernel<HD>, dim3(Hq, n_t, B), dim3(DKV_THREADS),
                                static_cast<size_t>(DkvSmem<HD>::ALLOC), st, static_cast<unsigned>(cl), tq, tk, tv, tdo,
                                cu_kept, gates, static_cast<const float4*>(fac), sm_scale, Hq, Hkv, M_total, dk, dv,
@@ -1155,8 +1296,9 @@ size_t attention_backward_workspace_bytes(int64_t M_total, int Hq, int Hkv, int 
     const size_t mh = static_cast<size_t>(M_total) * static_cast<size_t>(Hq);
     const size_t rows = 4 * mh + 2 * ((mh + 3) & ~static_cast<size_t>(3));
     const int grp = Hkv > 0 ? Hq / Hkv : 1;
-    const size_t parts =
-        grp > 1 && bwd_cluster_size(grp) == 0 ? static_cast<size_t>(2) * grp * static_cast<size_t>(M_total) * Hkv * d : 0;
+    // head_dim 256 always reduces the group's heads through partials
+    const bool parts_needed = grp > 1 && (d > 128 || bwd_cluster_size(grp) == 0);
+    const size_t parts = parts_needed ? static_cast<size_t>(2) * grp * static_cast<size_t>(M_total) * Hkv * d : 0;
     return (rows + parts) * sizeof(float);
 }
 
@@ -1177,6 +1319,9 @@ cudaError_t launch_gated_attention_backward(const uint16_t* q, const uint16_t* k
     if (d == 64)
         return launch_bwd<64>(q, k, v, out, dout, lse, cu_kept, B, M_total, max_M, Hq, Hkv, pos, rank, gates, c,
                               sm_scale, dq, dk, dv, go, dc, ws, st);
+    if (d == 256)
+        return launch_bwd<256>(q, k, v, out, dout, lse, cu_kept, B, M_total, max_M, Hq, Hkv, pos, rank, gates, c,
+                               sm_scale, dq, dk, dv, go, dc, ws, st);
     return launch_bwd<128>(q, k, v, out, dout, lse, cu_kept, B, M_total, max_M, Hq, Hkv, pos, rank, gates, c,
                            sm_scale, dq, dk, dv, go, dc, ws, st);
 }

@@ -398,7 +398,7 @@ tg_status tg_gated_attention_gates(const uint16_t* q, const uint16_t* k, const u
 }
 
 size_t tg_gated_attention_backward_workspace_size(int64_t M_total, int Hq, int Hkv, int d) {
-    if (M_total <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || (d != 64 && d != 128)) return 0;
+    if (M_total <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || (d != 64 && d != 128 && d != 256)) return 0;
     return tg::attention_backward_workspace_bytes(M_total, Hq, Hkv, d);
 }
 
@@ -414,7 +414,6 @@ tg_status do_backward(const uint16_t* q, const uint16_t* k, const uint16_t* v, c
                       cudaStream_t stream) {
     TG_REQUIRE(B >= 0 && M_total >= 0 && max_M >= 0, "negative size");
     if (tg_status s = check_attn_shape(Hq, Hkv, d)) return s;
-    TG_SUPPORT(d == 64 || d == 128, "the backward supports head_dim 64 and 128, not %d", d);
     TG_REQUIRE(sm_scale > 0.f, "sm_scale must be positive");
     TG_SUPPORT(gates.n >= 1 && gates.n <= tg::kMaxGates, "n_gates=%d must be in [1, %d]", gates.n, tg::kMaxGates);
     if (B == 0 || M_total == 0) return TG_OK;

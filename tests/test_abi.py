@@ -143,16 +143,17 @@ def test_invalid_shapes_are_refused_before_launch(lib):
 
 def test_backward_workspace_size_matches_its_documentation(lib):
     """6 floats per (row, head), each of the three sections padded to 16 bytes, plus fp32
-    partial dk and dv per query head only for GQA groups outside 1, 2, 4 and 8 (those
-    reduce inside a thread-block cluster or need no reduction)."""
+    partial dk and dv per query head for GQA groups outside 1, 2, 4 and 8 (those reduce
+    inside a thread-block cluster or need no reduction), and for every group of two or more
+    at head_dim 256 (no cluster reduction there)."""
     def expect(M, Hq, Hkv, d):
         mh = M * Hq
         rows = 4 * mh + 2 * ((mh + 3) // 4 * 4)
         grp = Hq // Hkv
-        parts = 2 * grp * M * Hkv * d if grp > 1 and grp not in (2, 4, 8) else 0
+        parts = 2 * grp * M * Hkv * d if grp > 1 and (d == 256 or grp not in (2, 4, 8)) else 0
         return (rows + parts) * 4
     for M, Hq, Hkv, d in [(2256, 16, 8, 128), (7, 3, 1, 64), (10, 8, 1, 64), (5, 4, 4, 128), (9, 6, 1, 128),
-                          (1, 8, 2, 64), (33, 12, 1, 64)]:
+                          (1, 8, 2, 64), (33, 12, 1, 64), (2384, 8, 2, 256), (7, 3, 3, 256), (9, 6, 1, 256)]:
         assert lib.tg_gated_attention_backward_workspace_size(M, Hq, Hkv, d) == expect(M, Hq, Hkv, d), (M, Hq, Hkv, d)
 
 

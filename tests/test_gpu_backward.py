@@ -133,14 +133,48 @@ def test_backward_is_deterministic(tg):
         np.testing.assert_array_equal(a[key], b[key], err_msg=key)
 
 
-def test_backward_refuses_head_dim_256(tg):
-    cs = _rand_case(10, [64], 2, 1, 256)
-    with pytest.raises(tg.TokenGateError):
-        _gpu_backward(tg, cs)
+@pytest.mark.parametrize("seed,seqlens,Hq,Hkv", [(10, [64], 2, 1), (14, [300, 129], 4, 2), (15, [257], 2, 2),
+                                                (16, [513], 8, 2), (17, [200, 77], 3, 1)])
+def test_backward_head_dim_256_matches_oracle(tg, seed, seqlens, Hq, Hkv):
+    """head_dim 256: the dQ kernel streams K/V as single-buffered 64-key half tiles, and dV
+    and dK come from two launches over the same keys (P^T then G^T), reduced over the
+    group's query heads through fp32 partials (a group of one writes bf16 directly).
+    Ragged sequences, a partial query tile, several tiles, odd and even groups."""
+    cs = _rand_case(seed, seqlens, Hq, Hkv, 256)
+    got = _gpu_backward(tg, cs)
+    ref = _oracle_backward(cs)
+    _check(got, ref, cs, f"d=256 seed {seed}")
+
+
+def test_backward_head_dim_256_at_c5(tg):
+    """The head_dim-256 workload: N=16384, K=2000 (M=2384), 8 query / 2 KV heads."""
+    w = CONFIGS["c5_hd256_16k"]
+    cu, span, kb = w.cu_seqlens(), w.span_array(), w.budget_array()
+    s = make_scores(w.T, std=2.0, seed=w.seed)
+    keep = oracle.select_topk(s, cu, span, kb)
+    comp = oracle.compact(None, s, keep, cu, span)
+    M = int(comp["cu_kept"][-1])
+    ai = make_attention_inputs(w, M, layer=0, qkv_std=0.5)
+    rng = np.random.default_rng(18)
+    cs = {"q": ai["q"], "k": ai["k"], "v": ai["v"], "cu": comp["cu_kept"], "pos": comp["pos"], "rank": comp["rank"],
+          "gls": comp["gls"].astype(np.float32), "g": ai["g"], "c": ai["c"],
+          "dout": f32_to_bf16_bits(rng.standard_normal((M, w.Hq, w.d)).astype(np.float32)),
+          "s": s[comp["src"]], "prunable": _in_span(comp["src"], cu, span)}
+    got = _gpu_backward(tg, cs)
+    ref = _oracle_backward(cs)
+    _check(got, ref, cs, "c5_hd256_16k")
+
+
+def test_backward_head_dim_256_is_deterministic(tg):
+    cs = _rand_case(19, [400, 150], 4, 2, 256)
+    a = _gpu_backward(tg, cs)
+    b = _gpu_backward(tg, cs)
+    for key in a:
+        np.testing.assert_array_equal(a[key], b[key], err_msg=key)
 
 
 @pytest.mark.parametrize("seed,seqlens,Hq,Hkv,d,n_gates", [(11, [300, 129], 4, 2, 128, 2), (12, [260], 8, 2, 64, 4),
-                                                           (13, [200, 77], 3, 1, 64, 3)])
+                                                           (13, [200, 77], 3, 1, 64, 3), (20, [300], 4, 2, 256, 2)])
 def test_backward_with_several_gates_matches_oracle(tg, seed, seqlens, Hq, Hkv, d, n_gates):
     """Several gate modules: the forward's logits carry sum_i softplus(g_i) gls_i; the
     backward returns each gate's dgls, dscore and dg (R24 bars per gate) and the same dq,
