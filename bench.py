@@ -369,6 +369,29 @@ def measure_next_rows(tg, dev, st, flush, main, peaks, reps=10):
     res["f3_hd256_attention"] = {"workload": f"{w.name}: M={M}, Hq={w.Hq}, Hkv={w.Hkv}, d={w.d}", "us": us,
                                  "tflops": fl / (us * 1e-6) / 1e12,
                                  "frac_of_bf16_peak": fl / (us * 1e-6) / 1e12 / tc_peak}
+    # f1 x f3: the backward at head_dim 256 on the same workload, from the forward's output and lse
+    lse5 = torch.empty((M, w.Hq), dtype=torch.float32, device=dev)
+    assert lib.tg_gated_attention(q.data_ptr(), k.data_ptr(), v.data_ptr(), ck_d.data_ptr(), w.B, M, maxM, w.Hq,
+                                  w.Hkv, w.d, cmap["pos"].data_ptr(), cmap["rank"].data_ptr(), cmap["gls"].data_ptr(),
+                                  g.data_ptr(), c.data_ptr(), 1.0 / math.sqrt(w.d), out.data_ptr(), lse5.data_ptr(),
+                                  None, 0, sh_now()) == 0
+    dout5 = torch.randn((M, w.Hq, w.d), device=dev).to(torch.bfloat16)
+    gr5 = [torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)]
+    f5 = [torch.empty(M, dtype=torch.float32, device=dev) for _ in range(2)] + \
+         [torch.empty(w.Hq, dtype=torch.float32, device=dev) for _ in range(2)]
+    nb5 = int(lib.tg_gated_attention_backward_workspace_size(M, w.Hq, w.Hkv, w.d))
+    bws5 = torch.empty(nb5, dtype=torch.uint8, device=dev)
+    us = time_device_us(check(lambda: lib.tg_gated_attention_backward(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout5.data_ptr(), lse5.data_ptr(), ck_d.data_ptr(),
+        w.B, M, maxM, w.Hq, w.Hkv, w.d, cmap["pos"].data_ptr(), cmap["rank"].data_ptr(), cmap["gls"].data_ptr(),
+        g.data_ptr(), c.data_ptr(), 1.0 / math.sqrt(w.d), gr5[0].data_ptr(), gr5[1].data_ptr(), gr5[2].data_ptr(),
+        f5[0].data_ptr(), f5[1].data_ptr(), f5[2].data_ptr(), f5[3].data_ptr(), bws5.data_ptr(), bws5.numel(),
+        sh_now())), st, flush, reps)
+    res["f1_attention_backward_hd256"] = {"workload": f"{w.name}: M={M}, Hq={w.Hq}, Hkv={w.Hkv}, d={w.d}",
+                                          "us": us, "tflops": 2.5 * fl / (us * 1e-6) / 1e12,
+                                          "frac_of_bf16_peak": 2.5 * fl / (us * 1e-6) / 1e12 / tc_peak,
+                                          "algorithmic": "2.5x the forward's 4*d*Hq per causal pair"}
+    del lse5, dout5, gr5, f5, bws5
     # f4: four stacked gates on the main workload's attention (same inputs as the step's)
     L0, wm, bufs = main["layer"], main["w"], main["bufs"]
     rng = np.random.default_rng(5)
