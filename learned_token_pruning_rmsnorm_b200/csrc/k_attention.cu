@@ -1214,11 +1214,12 @@ int64_t units_below_host(int x, int C) {
 // F being the part a unit adds beyond its tiles.  With the persistent kernel
 // a CTA loads the next unit while it finishes the current one, so F is about
 // one tile pair (the epilogue and the merge); the one-CTA-per-unit kernel pays
-// F = 3.1 (9 us of set-up, first loads and epilogue against 2.87 us per tile
-// pair).  Units are taken heaviest first,
-// which is longest-processing-time scheduling, so C is the candidate whose LPT
-// makespan over the SMs is smallest (all sequences taken at max_M, the bound the
-// host knows); ties go to the larger C (fewer units).
+// about 9 us of set-up, first loads and epilogue against 2.6-2.9 us per tile
+// pair, plus the merge of a split tile: F = 4.0, the value that measured best
+// among 2.0, 2.5, 3.1, 4.0 and 5.0 at 32k tokens, K = 2000.  Units are taken
+// heaviest first, which is longest-processing-time scheduling, so C is the
+// candidate whose LPT makespan over the SMs is smallest (all sequences taken
+// at max_M, the bound the host knows); ties go to the larger C (fewer units).
 int attention_kv_chunk(int B, int max_M, int Hq, int Hkv, bool have_ws, bool per_unit) {
     const int n_qt = (max_M + BM - 1) / BM;
     if (!have_ws || (Hq / Hkv) % 2 != 0 || n_qt < 4) return n_qt > 0 ? n_qt : 1;
@@ -1233,7 +1234,7 @@ int attention_kv_chunk(int B, int max_M, int Hq, int Hkv, bool have_ws, bool per
     // per candidate would otherwise run on every call)
     static std::mutex mu;
     static std::map<std::tuple<int, int, int, int, int>, int> memo;
-    const double F = per_unit ? 3.1 : 1.0;
+    const double F = per_unit ? 4.0 : 1.0;
     const auto key = std::make_tuple(B, n_qt, Hq / 2, sms, F > 2.0 ? 1 : 0);
     {
         std::lock_guard<std::mutex> lk(mu);
