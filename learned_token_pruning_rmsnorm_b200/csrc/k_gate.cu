@@ -65,22 +65,40 @@ __device__ unsigned long long g_score_cta[512 * 2];
 constexpr int KB = 64;                // channels per pipeline stage (one 128-byte swizzle row)
 constexpr int TILE_A = 128 * KB * 2;  // one 128-row slice: 16 KB
 
+// Two epilogue warps per (accumulator, TMEM lane group): each sums the squares of half of a
+// row's channels in every slice and runs the gate MLP's epilogue over half of its columns;
+// the pair adds its halves through shared memory in a fixed order.
 template <int NACC>
 struct ScoreCfg {
     static constexpr int STAGES = NACC == 2 ? 3 : 4;
-    static constexpr int EPI_WARPS = 4 * NACC;
+    static constexpr int EPI_COMBOS = 4 * NACC;  // (accumulator, lane group)
+    static constexpr int EPI_WARPS = 2 * EPI_COMBOS;
     static constexpr int THREADS = 64 + 32 * EPI_WARPS;
     static constexpr uint32_t TMEM_COLS = NACC == 2 ? 512 : 256;
     static constexpr int ROWS = 128 * NACC;
 };
 
+// bar.red.or over the epilogue warps (named barrier 1): every one learns whether any gave up
+__device__ __forceinline__ bool epi_red_or(int nthreads, bool pred) {
+    uint32_t res;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, 1, %2, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(res)
+        : "r"(static_cast<uint32_t>(pred)), "r"(nthreads)
+        : "memory");
+    return res != 0;
+}
+
 template <int NACC>
 __host__ __device__ constexpr int score_stage_bytes(int I) { return NACC * TILE_A + I * 128; }
 
-// stages x (NACC row slices + one Wg slice of I rows), b1, w2, 16 barriers, tmem slot + abort flag
+// stages x (NACC row slices + one Wg slice of I rows), b1, w2, 16 barriers, tmem slot + abort
+// flag, the epilogue pairs' exchange ([2][NACC * 128] sums of squares, the same for the dots)
 template <int NACC>
 __host__ __device__ constexpr int score_smem_bytes(int I) {
-    return ScoreCfg<NACC>::STAGES * score_stage_bytes<NACC>(I) + 2 * 256 * 4 + 16 * 8 + 16 + 1024;
+    return ScoreCfg<NACC>::STAGES * score_stage_bytes<NACC>(I) + 2 * 256 * 4 + 16 * 8 + 16 +
+           4 * NACC * 128 * 4 + 1024;
 }
 
 // SiLU(z) = z / (1 + e^-z).  e^-z takes one special-function-unit operation; the
@@ -139,6 +157,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
     const uint32_t drain = bar0 + 8u * (2 * STAGES + 2);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + STAGES * stage_bytes + 2 * 256 * 4 + 16 * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    float* xss = reinterpret_cast<float*>(smem + STAGES * stage_bytes + 2 * 256 * 4 + 16 * 8 + 16);  // [2][NACC*128]
+    float* xac = xss + 2 * NACC * 128;                                                                 // [2][NACC*128]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nkb = D / KB;
@@ -252,11 +272,20 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
         }
     } else {
         // ---------------------------------------------------------------- sum of squares + epilogue
-        const int e = warp - 2;          // 0 .. EPI_WARPS-1
-        const int a = e >> 2;            // accumulator of this warp
-        const int lg = warp & 3;         // TMEM lane group this warp may access
-        const int r = lg * 32 + lane;    // row within the 128-row slice == TMEM lane
+        const int e = warp - 2;                 // 0 .. EPI_WARPS-1
+        const int hs = e / C::EPI_COMBOS;       // which half of the channels and columns
+        const int a = (e % C::EPI_COMBOS) >> 2; // accumulator of this warp
+        const int lg = warp & 3;                // TMEM lane group this warp may access
+        const int r = lg * 32 + lane;           // row within the 128-row slice == TMEM lane
         const uint32_t lane_addr = static_cast<uint32_t>(lg * 32) << 16;
+        const int xi = a * 128 + r;             // this row's slot in the pair exchange
+        constexpr int EPI_T = 32 * C::EPI_WARPS;
+        // columns of this warp: the first or second half of the 32-column chunks (the 16-column
+        // tail, when I is 16 mod 32, goes with the second half)
+        const int I32 = I & ~31;
+        const int nfull = I32 / 32;
+        const int c_begin = hs ? (nfull / 2) * 32 : 0, c_end = hs ? I32 : (nfull / 2) * 32;
+        const bool tail = hs == 1 && I32 < I;
         int64_t it = 0;
         int tcount = 0;
         bool ok = true;
@@ -272,14 +301,14 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                     ok = false;
                     break;
                 }
-                // the row's 64 channels of this slice.  Lane r starts at physical chunk
-                // (r & 7): the 128-byte swizzle then spreads a warp's 32 rows over all
-                // banks (4 wavefronts per 512-byte access, the minimum); chunk order is
-                // irrelevant for a sum of squares.
+                // half of the row's 64 channels of this slice (logical 16-byte chunks 4 hs ..
+                // 4 hs + 3).  Lane r reads physical chunk (c ^ (r & 7)): the 128-byte swizzle then
+                // spreads a warp's 32 rows over all banks; chunk order is irrelevant for a sum of
+                // squares.
                 const uint8_t* rowp = smem + s * stage_bytes + a * TILE_A + r * 128;
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    const uint4 v = *reinterpret_cast<const uint4*>(rowp + ((ch ^ (r & 7)) << 4));
+                for (int ch = 0; ch < 4; ++ch) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(rowp + (((4 * hs + ch) ^ (r & 7)) << 4));
                     const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
@@ -292,20 +321,25 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
                 if (lane == 0) mbar_arrive(empty(s));
                 if (warp == 2 && lane == 0) SC_TRACE(3, it);
             }
-            if (!ok) break;
-            if (!mbar_wait_warp(acc_full, tcount & 1, abort_flag, status, TG_WHERE_SOFTMAX)) break;
+            xss[hs * (NACC * 128) + xi] = ss;
+            const bool okw = ok && mbar_wait_warp(acc_full, tcount & 1, abort_flag, status, TG_WHERE_SOFTMAX);
+            // every epilogue warp leaves together (the pairs meet at the barriers below)
+            if (epi_red_or(EPI_T, !okw)) {
+                ok = false;
+                break;
+            }
             tc_fence_after();
-            const float rr = rsqrtf(ss / static_cast<float>(D) + eps);
+            const float sst = xss[xi] + xss[NACC * 128 + xi];  // the same order in both warps of the pair
+            const float rr = rsqrtf(sst / static_cast<float>(D) + eps);
             float acc_s = 0.f;
-            const int I32 = I & ~31;
-            for (int c0 = 0; c0 < I32; c0 += 32) {
+            for (int c0 = c_begin; c0 < c_end; c0 += 32) {
                 float z[32];
                 tmem_ld32(tmem + a * 256 + lane_addr + c0, z);
                 tmem_wait_ld();
 #pragma unroll
                 for (int q = 0; q < 32; ++q) acc_s = fmaf(s_w2[c0 + q], silu_f(fmaf(rr, z[q], s_b1[c0 + q])), acc_s);
             }
-            if (I32 < I) {  // the last 16 columns when I is 16 mod 32
+            if (tail) {  // the last 16 columns when I is 16 mod 32
                 float z[32];
                 tmem_ld32(tmem + a * 256 + lane_addr + I32, z);
                 tmem_wait_ld();
@@ -315,15 +349,20 @@ score_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(acc_empty);
-            const int64_t row = row0 + a * 128 + r;
-            const bool valid = row < row_end && TG_DEBUG_CHECK(row >= 0 && row < T, status, TG_WHERE_SCORE);
-            if (valid) scores[row] = acc_s + b2;
-            if (key_hist != nullptr) {
-                // the selection's first pass: this sequence's scores counted by the top 11 bits of
-                // their order-preserving key, one atomic per distinct bucket of the warp
-                const int bin = valid ? seq * 2048 + static_cast<int>(score_key(acc_s + b2) >> 21) : -1;
-                const unsigned same = __match_any_sync(0xffffffffu, bin);
-                if (valid && lane == __ffs(same) - 1) atomicAdd(key_hist + bin, __popc(same));
+            xac[hs * (NACC * 128) + xi] = acc_s;
+            asm volatile("bar.sync 1, %0;" ::"r"(EPI_T) : "memory");  // both halves of every row are in
+            if (hs == 0) {
+                const float score = xac[xi] + xac[NACC * 128 + xi] + b2;
+                const int64_t row = row0 + a * 128 + r;
+                const bool valid = row < row_end && TG_DEBUG_CHECK(row >= 0 && row < T, status, TG_WHERE_SCORE);
+                if (valid) scores[row] = score;
+                if (key_hist != nullptr) {
+                    // the selection's first pass: this sequence's scores counted by the top 11 bits
+                    // of their order-preserving key, one atomic per distinct bucket of the warp
+                    const int bin = valid ? seq * 2048 + static_cast<int>(score_key(score) >> 21) : -1;
+                    const unsigned same = __match_any_sync(0xffffffffu, bin);
+                    if (valid && lane == __ffs(same) - 1) atomicAdd(key_hist + bin, __popc(same));
+                }
             }
         }
     }
