@@ -604,8 +604,10 @@ gated_attn_gqa2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                             bar(G_V_FULL + s));
             ++v_issued[s];
         };
-        // tiles whose K and V copies leave before the compaction map is available
-        const int pre = early ? min(n_kv, 2) : 0;
+        // The first two tiles' K and V copies leave at once (their stages are free): before the
+        // compaction map is available in an early launch, and before the first gls loads (which
+        // the K_ext rows wait for) in every launch.
+        const int pre = min(n_kv, 2);
         if (lane == 0)
             for (int j = 0; j < pre; ++j) {
                 issue_k(j);

@@ -331,10 +331,10 @@ gated_attn_pers_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                                 U.seq0 + (U.kv0 + j) * BN, bar(T_V_FULL + s));
                 ++v_issued[s];
             };
-            // K/V tiles through the two-stage ring (t counts tiles over all units).  In the
-            // first unit of an early launch the first two tiles' copies leave before the wait
-            // (t < 2: their stages are free).
-            const int pre = waited ? 0 : min(U.n_kv, 2);
+            // K/V tiles through the two-stage ring (t counts tiles over all units).  The CTA's
+            // first two tiles' copies leave at once (t = 0: both stages are free): before the
+            // wait in an early launch, and before the first bias loads in every launch.
+            const int pre = t == 0 ? min(U.n_kv, 2) : 0;
             if (lane == 0)
                 for (int j = 0; j < pre; ++j) {
                     load_k((t + j) & 1, j);
