@@ -157,6 +157,34 @@ def test_backward_workspace_size_matches_its_documentation(lib):
         assert lib.tg_gated_attention_backward_workspace_size(M, Hq, Hkv, d) == expect(M, Hq, Hkv, d), (M, Hq, Hkv, d)
 
 
+def test_prefill_workspace_size_matches_its_documentation(lib):
+    """tg_gated_prefill_workspace_size: the attention's scratch rounded up to 256 bytes, then
+    the selection's [B][2048] int32 first-pass histogram; the histogram alone without
+    attention layers; 0 for an empty batch."""
+    for B, max_M, Hq, Hkv, d in [(1, 2256, 16, 8, 128), (4, 65536, 16, 8, 128), (1, 2384, 8, 2, 256),
+                                 (3, 700, 6, 3, 64), (2, 100, 8, 8, 128)]:
+        attn = lib.tg_gated_attention_workspace_size(B, max_M, Hq, Hkv, d)
+        want = (attn + 255) // 256 * 256 + B * 2048 * 4
+        assert lib.tg_gated_prefill_workspace_size(B, max_M, Hq, Hkv, d, 1) == want, (B, max_M, Hq, Hkv, d)
+        assert lib.tg_gated_prefill_workspace_size(B, max_M, Hq, Hkv, d, 0) == B * 2048 * 4
+    assert lib.tg_gated_prefill_workspace_size(0, 100, 8, 8, 128, 1) == 0
+
+
+def test_attention_workspace_covers_both_kernels(lib, monkeypatch):
+    """The workspace size does not depend on which two-head kernel runs
+    (TG_ATTENTION_KERNEL): it is the larger of the two kernels' causal-split needs."""
+    sizes = {}
+    for choice in (None, "persistent", "per_unit"):
+        if choice is None:
+            monkeypatch.delenv("TG_ATTENTION_KERNEL", raising=False)
+        else:
+            monkeypatch.setenv("TG_ATTENTION_KERNEL", choice)
+        sizes[choice] = [lib.tg_gated_attention_workspace_size(B, M, 16, 8, 128)
+                         for B, M in [(1, 2256), (1, 16384), (2, 9000), (4, 40000)]]
+    assert sizes[None] == sizes["persistent"] == sizes["per_unit"]
+    assert all(n > 0 for n in sizes[None][:1])
+
+
 def test_empty_batches_are_no_ops(lib):
     from learned_token_pruning_rmsnorm_b200 import _lib
     assert lib.tg_select_topk(None, None, None, None, 0, 0, None, None, None, None, None, None, None) == _lib.TG_OK
