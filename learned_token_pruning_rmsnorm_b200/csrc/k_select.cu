@@ -7,24 +7,30 @@
 //
 // Design: one cluster of SEL_CL CTAs per sequence.  CTA i owns a contiguous
 // slice of the sequence's tokens and caches the order-preserving uint32 keys
-// of its prunable tokens in shared memory.
+// of its prunable tokens in shared memory, by their offset in the slice.
 //   1. bucket select: each pass histograms the keys of the current range into
 //      <= 2048 buckets of width 2^s (the first pass the whole key range by its
 //      top 11 bits, the next ones the chosen bucket by the following 11 and 10
-//      bits) and sums them into 64 superbins.
-//      One warp per CTA then reads the 8 x 64 superbin sums and the 8 x 32
-//      buckets of the chosen superbin through distributed shared memory and
-//      narrows the range to the bucket holding the K-th key.  The passes stop
-//      when that bucket is a single key value thr (need_eq = how many keys
-//      equal to thr are kept: the lowest-indexed ones), at most three, or as
-//      soon as every key of the bucket is taken (usually after two): then the
-//      rule is key >= the bucket's lower edge, with no tie to rank.
+//      bits) and sums them into 64 superbins; it also counts the keys above
+//      the range.  One warp per CTA then reads the 8 x 64 superbin sums, the
+//      counts above and the 8 x 32 buckets of the chosen superbin through
+//      distributed shared memory and narrows the range to the bucket holding
+//      the K-th key.  The passes stop when that bucket is a single key value
+//      thr (need_eq = how many keys equal to thr are kept: the lowest-indexed
+//      ones), at most three, or as soon as every key of the bucket is taken
+//      (usually after two): then the rule is key >= the bucket's lower edge,
+//      with no tie to rank.  The same counts give every slice's number of
+//      kept tokens, so the CTAs need no further exchange.
 //   2. ordered scan: every warp owns a contiguous run of the slice and walks
-//      it 32 tokens at a time; ballots count the kept tokens, one block scan
-//      over the warp totals and one exchange of slice totals across the
-//      cluster number them, and each kept token writes its compaction-map
-//      entry (kept_idx, pos, rank, logsigmoid of its score) in coalesced
-//      stores with no further barrier.
+//      it 128 tokens at a time, 4 consecutive tokens per lane (one 16-byte
+//      load of cached keys); ballots of each of the 4 token positions number
+//      the kept tokens after one block scan over the warp totals.  The kept
+//      tokens of up to 4096 consecutive entries are listed in shared memory,
+//      and the threads then write those compaction-map entries (kept_idx,
+//      pos, rank, logsigmoid of the score) densely.  When the counts did not
+//      come from the last pass (caller-given keep flags, a search the score
+//      kernel's first pass already ended) the slice totals are exchanged once
+//      through distributed shared memory.
 // Everything is deterministic: atomics only build counts.
 
 #include <cooperative_groups.h>
@@ -36,14 +42,17 @@ namespace cg = cooperative_groups;
 namespace tg {
 namespace {
 
-// Optional device trace (builds with -DTG_TRACE only): clock64 stamps of the
-// phases of the first CTA of the first sequence.
+// Optional device trace (builds with -DTG_TRACE only): globaltimer stamps (ns) of the
+// phases of every CTA of the first sequence, 16 points per CTA.
 #ifdef TG_TRACE
-__device__ unsigned long long g_sel_trace[32];
+__device__ unsigned long long g_sel_trace[8 * 16];
 #define SEL_TRACE(point)                                                                         \
     do {                                                                                         \
-        if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)                              \
-            g_sel_trace[(point)] = static_cast<unsigned long long>(clock64());                   \
+        if (blockIdx.y == 0 && blockIdx.x < 8 && threadIdx.x == 0) {                             \
+            unsigned long long t_;                                                               \
+            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                               \
+            g_sel_trace[blockIdx.x * 16 + (point)] = t_;                                         \
+        }                                                                                        \
     } while (0)
 #else
 #define SEL_TRACE(point) \
@@ -57,25 +66,26 @@ constexpr int SEL_WARPS = SEL_THREADS / 32;
 constexpr int SEL_CACHE_KEYS = 32768;         // keys cached per CTA (128 KB)
 constexpr int SEL_BINS = 2048;
 constexpr int SEL_SUPER = SEL_BINS / 32;      // superbins of 32 buckets
-constexpr int SEL_SMEM_BYTES = SEL_CACHE_KEYS * 4 + 2 * SEL_BINS * 4;
+constexpr int SEL_LIST = 4096;                // compaction-map entries emitted per round
+constexpr int SEL_SMEM_BYTES = SEL_CACHE_KEYS * 4 + 2 * SEL_BINS * 4 + SEL_LIST * 4;
 
 struct SelShared {
     int coarse[2][SEL_SUPER];  // per pass parity: bucket counts summed over each superbin
+    int above[2];              // per pass parity: this CTA's keys above the pass's range
     int xchg[2];               // slice totals published to the cluster: kept, tie-ranked
     int wsum[SEL_WARPS];       // a first-pass histogram summed over each warp's 64 buckets
     int warp_kept[SEL_WARPS];  // exclusive prefix over the warps of this CTA
     int warp_eq[SEL_WARPS];
+    int cta_kept;              // kept tokens of the slices before this one (tie-ranked keys excluded)
+    int cta_eq;                // tie-ranked keys of the slices before this one
+    int counts_known;          // cta_kept / cta_eq came from the last pass (no exchange needed)
     uint32_t lo;               // current key range [lo, lo + width)
     uint64_t width;
     int remaining;             // keys still to take from the current range, counted from its top
     int bin_count;
 };
 
-__device__ __forceinline__ int warp_sum(int v) {
-#pragma unroll
-    for (int off = 16; off; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-    return v;
-}
+__device__ __forceinline__ int warp_sum(int v) { return __reduce_add_sync(0xffffffffu, v); }
 
 __device__ __forceinline__ int warp_inclusive_scan(int v) {
     const int lane = threadIdx.x & 31;
@@ -105,8 +115,17 @@ __device__ __forceinline__ void cluster_wait_acquire() {
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// Token slice [a0, a1) of cluster rank r: SEL_CL slices of `per` tokens (a multiple of
+// SEL_THREADS), the last ones shorter or empty.  Token indices fit in 32 bits (cu_seqlens is
+// int32); the products are formed in 64 bits so that no intermediate overflows.
+__device__ __forceinline__ void slice_of(int r, int s0, int s1, int per, int& a0, int& a1) {
+    const int64_t x0 = min(static_cast<int64_t>(s1), static_cast<int64_t>(s0) + static_cast<int64_t>(per) * r);
+    a0 = static_cast<int>(x0);
+    a1 = static_cast<int>(min(static_cast<int64_t>(s1), x0 + per));
+}
+
 __global__ void __cluster_dims__(SEL_CL, 1, 1) __launch_bounds__(SEL_THREADS, 1)
-select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __restrict__ keep_in,
+select_scan_kernel(int mode, int early, const float* __restrict__ scores, const uint8_t* __restrict__ keep_in,
                    const int32_t* __restrict__ cu_seqlens, const int32_t* __restrict__ span,
                    const int32_t* __restrict__ kbud, const int32_t* __restrict__ cu_kept,
                    uint8_t* __restrict__ keep_out, int32_t* __restrict__ kept_idx, int32_t* __restrict__ pos,
@@ -114,50 +133,89 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
     extern __shared__ __align__(16) unsigned char smem_raw[];
     uint32_t* skeys = reinterpret_cast<uint32_t*>(smem_raw);
     int* hist_buf = reinterpret_cast<int*>(smem_raw + SEL_CACHE_KEYS * 4);  // [2][SEL_BINS]
+    int* list = hist_buf + 2 * SEL_BINS;  // [SEL_LIST]
     __shared__ SelShared sh;
     cg::cluster_group cl = cg::this_cluster();
 
     const int crank = static_cast<int>(cl.block_rank());
-    SEL_TRACE(0);
-    pdl_wait();  // global memory is read only from here on
-    pdl_trigger();
     const int b = blockIdx.y;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t s0 = cu_seqlens[b], s1 = cu_seqlens[b + 1];
-    // spans are clamped into the sequence so that a malformed span cannot index outside it
-    const int64_t p0 = s0 + min(max(static_cast<int64_t>(span[2 * b]), int64_t(0)), s1 - s0);
-    const int64_t p1 = max(p0, s0 + min(static_cast<int64_t>(span[2 * b + 1]), s1 - s0));
-    const int64_t P = p1 - p0;
     const bool emit = kept_idx != nullptr;  // cu_kept is only read when emitting
-    const int64_t m0 = emit ? cu_kept[b] : 0, m1 = emit ? cu_kept[b + 1] : 0;
+    // The sequence's bounds, span, budget and output range.  Inside the prefill layer they are
+    // the caller's, complete before the call (`early`), and are read before the wait for the
+    // score kernel; otherwise after it.
+    int s0 = 0, s1 = 0, sp0 = 0, sp1 = 0, kb = -1, m0 = 0, m1 = 0;
+    auto load_meta = [&]() {
+        s0 = cu_seqlens[b];
+        s1 = cu_seqlens[b + 1];
+        sp0 = span[2 * b];
+        sp1 = span[2 * b + 1];
+        if (mode == 0) kb = kbud[b];
+        if (emit) {
+            m0 = cu_kept[b];
+            m1 = cu_kept[b + 1];
+        }
+    };
+    if (early) load_meta();
+    SEL_TRACE(0);
+    pdl_wait();  // the scores (and the first-pass counts) are read only from here on
+    SEL_TRACE(12);
+    pdl_trigger();
+    if (!early) load_meta();
+    // spans are clamped into the sequence so that a malformed span cannot index outside it
+    const int n = s1 - s0;
+    const int p0 = s0 + min(max(sp0, 0), n);
+    const int p1 = max(p0, s0 + min(sp1, n));
+    const int P = p1 - p0;
 
-    // this CTA's token slice [t0, t1) (a multiple of 1024 tokens long), split
-    // into one contiguous run per warp
-    const int64_t n = s1 - s0;
-    const int64_t per = ((n + SEL_CL - 1) / SEL_CL + SEL_THREADS - 1) / SEL_THREADS * SEL_THREADS;
-    const int64_t t0 = min(s1, s0 + per * crank), t1 = min(s1, t0 + per);
-    const int64_t per_warp = per / SEL_WARPS;
-    const int64_t w0 = min(t1, t0 + per_warp * warp), w1 = min(t1, w0 + per_warp);
-    // prunable part of the slice [k0, k1) and whether its keys fit the cache
-    const int64_t k0 = max(t0, p0), k1 = max(k0, min(t1, p1));
-    const bool cached = (k1 - k0) <= SEL_CACHE_KEYS;
+    // this CTA's token slice [t0, t1), split into one contiguous run per warp
+    const int per = static_cast<int>(((static_cast<int64_t>(n) + SEL_CL - 1) / SEL_CL + SEL_THREADS - 1) /
+                                     SEL_THREADS * SEL_THREADS);
+    int t0, t1;
+    slice_of(crank, s0, s1, per, t0, t1);
+    const int per_warp = per / SEL_WARPS;  // a multiple of 32
+    const int w0 = static_cast<int>(min(static_cast<int64_t>(t1), static_cast<int64_t>(t0) + static_cast<int64_t>(per_warp) * warp));
+    const int w1 = static_cast<int>(min(static_cast<int64_t>(t1), static_cast<int64_t>(w0) + per_warp));
+    // prunable part of the slice [k0, k1); the keys are cached by their offset from t0 when
+    // the slice fits the cache (uniform over the cluster), so that a lane's 4 consecutive
+    // tokens (offset a multiple of 4) are one 16-byte shared-memory load
+    const int k0 = max(t0, p0), k1 = max(k0, min(t1, p1));
+    const int nk = k1 - k0;
+    const bool cached = per <= SEL_CACHE_KEYS;
 
-    int64_t kk = P;
-    if (mode == 0) {
-        const int32_t kb = kbud[b];
-        kk = (kb < 0 || static_cast<int64_t>(kb) > P) ? P : static_cast<int64_t>(kb);
-    }
+    int kk = P;
+    if (mode == 0) kk = (kb < 0 || kb > P) ? P : kb;
     const bool do_select = (mode == 0) && kk > 0 && kk < P;
+    const bool use_hist = do_select && key_hist != nullptr;
 
     uint32_t thr = 0;        // the K-th largest key
-    int64_t need_eq = 0;     // keys equal to thr that are kept
+    int need_eq = 0;         // keys equal to thr that are kept
     bool all_eq_kept = true; // every key equal to thr is kept: no tie ranking needed
 
+    if (tid == 0) sh.counts_known = 0;
     // ------------------------------------------------ cache keys (for the selection and for gls)
+    // the score kernel's first-pass counts are loaded together with the keys (one round trip)
+    int hv0 = 0, hv1 = 0;
+    if (use_hist) {
+        const int* kh = key_hist + static_cast<int64_t>(b) * SEL_BINS;
+        hv0 = __ldcg(kh + 2 * tid);
+        hv1 = __ldcg(kh + 2 * tid + 1);
+    }
     const bool need_gls = emit && kk > 0;  // some prunable token is kept: its logsigmoid is emitted
     if (cached && (do_select || need_gls)) {
-#pragma unroll 8
-        for (int64_t t = k0 + tid; t < k1; t += SEL_THREADS) skeys[t - k0] = score_key(__ldcg(scores + t));
+        for (int c = 0; c < nk; c += 4 * SEL_THREADS) {
+            uint32_t v[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int o = c + i * SEL_THREADS + tid;
+                v[i] = o < nk ? score_key(__ldcg(scores + k0 + o)) : 0u;
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int o = c + i * SEL_THREADS + tid;
+                if (o < nk) skeys[k0 - t0 + o] = v[i];
+            }
+        }
     }
     SEL_TRACE(1);
 
@@ -169,24 +227,22 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
         if (tid == 0) {
             sh.lo = 0u;
             sh.width = static_cast<uint64_t>(1) << 32;
-            sh.remaining = static_cast<int>(kk);
+            sh.remaining = kk;
             sh.bin_count = 0;
         }
-        if (key_hist != nullptr) {
+        if (use_hist) {
             // The score kernel took the first pass (the top 11 bits of every key of this
             // sequence): every CTA reads the same counts and finds the same bucket itself, the
             // K-th key from the top (its 64-bucket warp segment, then the bucket), with no
             // cluster round trip.
-            const int* kh = key_hist + static_cast<int64_t>(b) * SEL_BINS;
             int* hist0 = hist_buf;  // free until the passes below
-            const int v0 = __ldcg(kh + 2 * tid), v1 = __ldcg(kh + 2 * tid + 1);
-            hist0[2 * tid] = v0;
-            hist0[2 * tid + 1] = v1;
-            const int wsum = warp_sum(v0 + v1);
+            hist0[2 * tid] = hv0;
+            hist0[2 * tid + 1] = hv1;
+            const int wsum = warp_sum(hv0 + hv1);
             if (lane == 0) sh.wsum[warp] = wsum;
             __syncthreads();
             if (warp == 0) {
-                const int rem = static_cast<int>(kk);
+                const int rem = kk;
                 const int v = sh.wsum[SEL_WARPS - 1 - lane];
                 const int incl = warp_inclusive_scan(v);
                 const unsigned hit = __ballot_sync(0xffffffffu, incl - v < rem && incl >= rem);
@@ -213,24 +269,48 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
         // ------------------------------------------------ bucket passes
         // (none when the score kernel's first pass already ends the search: every key of the
         // chosen bucket is taken)
-        for (int pass = 0; !(key_hist != nullptr && sh.remaining == sh.bin_count && sh.width < (1ull << 32));
-             ++pass) {
+        for (int pass = 0; !(use_hist && sh.remaining == sh.bin_count && sh.width < (1ull << 32)); ++pass) {
             const uint32_t lo = sh.lo;
             const uint64_t width = sh.width;
+            const uint64_t range_end = static_cast<uint64_t>(lo) + width;  // keys >= range_end lie above
             const int sh_bits = max(0, bit_length(width - 1) - 11);  // bucket width 2^sh_bits, <= 2048 buckets
             // both buffers alternate by pass: another CTA may still read the previous pass's
             int* hist = hist_buf + (pass & 1) * SEL_BINS;
             int* coarse = sh.coarse[pass & 1];
             hist[tid] = 0;
             hist[tid + SEL_THREADS] = 0;
+            if (tid == 0) sh.above[pass & 1] = 0;
             __syncthreads();
-#pragma unroll 4
-            for (int64_t t = k0 + tid; t < k1; t += SEL_THREADS) {
-                const uint32_t key = cached ? skeys[t - k0] : score_key(__ldcg(scores + t));
+            int my_above = 0;
+            auto count_key = [&](uint32_t key) {
                 const uint32_t d = key - lo;  // wraps for keys below lo: excluded by the range test
                 if (key >= lo && static_cast<uint64_t>(d) < width) atomicAdd(&hist[d >> sh_bits], 1);
+                my_above += static_cast<uint64_t>(key) >= range_end ? 1 : 0;
+            };
+            if (cached) {  // 4 keys per load, offsets [k0 - t0, k1 - t0) of the cache
+                const int c0 = k0 - t0, c1 = k1 - t0;
+                for (int o = (c0 & ~3) + 4 * tid; o < c1; o += 4 * SEL_THREADS) {
+                    const uint4 q = *reinterpret_cast<const uint4*>(skeys + o);
+                    if (o >= c0 && o + 4 <= c1) {
+                        count_key(q.x);
+                        count_key(q.y);
+                        count_key(q.z);
+                        count_key(q.w);
+                    } else {
+                        const uint32_t kv[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            if (o + i >= c0 && o + i < c1) count_key(kv[i]);
+                    }
+                }
+            } else {
+#pragma unroll 4
+                for (int t = k0 + tid; t < k1; t += SEL_THREADS) count_key(score_key(__ldcg(scores + t)));
             }
+            my_above = warp_sum(my_above);
+            if (lane == 0 && my_above != 0) atomicAdd(&sh.above[pass & 1], my_above);
             __syncthreads();
+            if (pass == 0) SEL_TRACE(13);
             {   // superbin sums: warp w sums buckets [64w, 64w + 64)
                 const int a = warp_sum(hist[64 * warp + lane]);
                 const int c = warp_sum(hist[64 * warp + 32 + lane]);
@@ -239,30 +319,32 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
                     coarse[2 * warp + 1] = c;
                 }
             }
-            cl.sync();  // every CTA's histogram and superbin sums of this pass are complete
+            cl.sync();  // every CTA's histogram, superbin sums and count above of this pass are complete
+            if (pass == 0) SEL_TRACE(14);
             if (warp == 0) {
                 // the rem-th key from the top: first its superbin (lane l owns superbins
                 // 63 - 2l and 62 - 2l of all CTAs), then its bucket (lane l owns bucket
                 // 32 S + 31 - l of all CTAs); every CTA finds the same bucket
                 const int rem = sh.remaining;
+                int vh[SEL_CL], vl[SEL_CL];
                 int hi = 0, lo2 = 0;
-                {
-                    int vh[SEL_CL], vl[SEL_CL];
 #pragma unroll
-                    for (int r = 0; r < SEL_CL; ++r) {
-                        const int* cr = cl.map_shared_rank(coarse, r);
-                        vh[r] = cr[SEL_SUPER - 1 - 2 * lane];
-                        vl[r] = cr[SEL_SUPER - 2 - 2 * lane];
-                    }
+                for (int r = 0; r < SEL_CL; ++r) {
+                    const int* cr = cl.map_shared_rank(coarse, r);
+                    vh[r] = cr[SEL_SUPER - 1 - 2 * lane];
+                    vl[r] = cr[SEL_SUPER - 2 - 2 * lane];
+                }
+                // lane r < SEL_CL: slice r's keys above the range
+                const int ab = lane < SEL_CL ? *cl.map_shared_rank(&sh.above[pass & 1], lane) : 0;
 #pragma unroll
-                    for (int r = 0; r < SEL_CL; ++r) {
-                        hi += vh[r];
-                        lo2 += vl[r];
-                    }
+                for (int r = 0; r < SEL_CL; ++r) {
+                    hi += vh[r];
+                    lo2 += vl[r];
                 }
                 const int incl = warp_inclusive_scan(hi + lo2);
                 const int excl = incl - hi - lo2;
                 const unsigned hit = __ballot_sync(0xffffffffu, excl < rem && incl >= rem);
+                bool decided = false;
                 if (hit != 0u) {
                     const int L = __ffs(hit) - 1;
                     const int excl_L = __shfl_sync(0xffffffffu, excl, L);
@@ -279,15 +361,53 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
                     for (int r = 0; r < SEL_CL; ++r) cnt += v[r];
                     const int incl2 = warp_inclusive_scan(cnt);
                     const int excl2 = incl2 - cnt;
-                    if (excl2 < rem2 && incl2 >= rem2) {
-                        const uint64_t new_lo = static_cast<uint64_t>(lo) + (static_cast<uint64_t>(bin) << sh_bits);
-                        const uint64_t end = static_cast<uint64_t>(lo) + width;
-                        sh.lo = static_cast<uint32_t>(new_lo);
-                        sh.width = min(static_cast<uint64_t>(1) << sh_bits, end - new_lo);
-                        sh.remaining = rem2 - excl2;
-                        sh.bin_count = cnt;
+                    const unsigned hit2 = __ballot_sync(0xffffffffu, excl2 < rem2 && incl2 >= rem2);
+                    if (hit2 != 0u) {
+                        decided = true;
+                        const int Lb = __ffs(hit2) - 1;
+                        const int remaining = rem2 - __shfl_sync(0xffffffffu, excl2, Lb);
+                        const int bin_count = __shfl_sync(0xffffffffu, cnt, Lb);
+                        if (lane == Lb) {
+                            const uint64_t new_lo = static_cast<uint64_t>(lo) + (static_cast<uint64_t>(bin) << sh_bits);
+                            sh.lo = static_cast<uint32_t>(new_lo);
+                            sh.width = min(static_cast<uint64_t>(1) << sh_bits, range_end - new_lo);
+                            sh.remaining = remaining;
+                            sh.bin_count = bin_count;
+                        }
+                        if (sh_bits == 0 || pass >= 3 || remaining == bin_count) {
+                            // The search ends here, so every slice's count of kept keys follows
+                            // from this pass's counts: the keys above the range, the superbins
+                            // above S, the buckets of S above the chosen one and, when all of it
+                            // is taken, the chosen bucket (else its keys are ranked by index).
+                            const bool all_kept = remaining == bin_count;
+                            int kept_r = 0, eq_r = 0;  // lane r < SEL_CL: slice r's
+#pragma unroll
+                            for (int r = 0; r < SEL_CL; ++r) {
+                                const int sup = lane < L ? vh[r] + vl[r] : (lane == L && !upper ? vh[r] : 0);
+                                const int above_bin = warp_sum(sup + (lane < Lb ? v[r] : 0));
+                                const int in_bin = __shfl_sync(0xffffffffu, v[r], Lb);
+                                if (lane == r) {
+                                    kept_r = ab + above_bin + (all_kept ? in_bin : 0);
+                                    eq_r = all_kept ? 0 : in_bin;
+                                }
+                            }
+                            if (lane < SEL_CL) {
+                                int a0, a1;
+                                slice_of(lane, s0, s1, per, a0, a1);
+                                const int b0 = max(a0, p0), b1 = max(b0, min(a1, p1));
+                                kept_r += (a1 - a0) - (b1 - b0);  // tokens outside the span are kept
+                            }
+                            const int ik = warp_inclusive_scan(lane < SEL_CL ? kept_r : 0);
+                            const int ie = warp_inclusive_scan(lane < SEL_CL ? eq_r : 0);
+                            if (lane == crank) {
+                                sh.cta_kept = ik - kept_r;
+                                sh.cta_eq = ie - eq_r;
+                                sh.counts_known = 1;
+                            }
+                        }
                     }
-                } else if (lane == 0) {
+                }
+                if (!decided && lane == 0) {
                     // unreachable while the range holds >= rem keys; end the search on lo
                     sh.width = 1;
                     sh.remaining = 0;
@@ -303,39 +423,77 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
         thr = sh.lo;
         need_eq = sh.remaining;
         all_eq_kept = need_eq == sh.bin_count;
+    } else if (mode == 0 && warp == 0) {
+        // no selection: every token outside the span is kept, and every prunable one if kk > 0
+        __syncwarp();  // after tid 0 cleared counts_known
+        int kept_r = 0;
+        if (lane < SEL_CL) {
+            int a0, a1;
+            slice_of(lane, s0, s1, per, a0, a1);
+            const int b0 = max(a0, p0), b1 = max(b0, min(a1, p1));
+            kept_r = kk > 0 ? a1 - a0 : (a1 - a0) - (b1 - b0);
+        }
+        const int ik = warp_inclusive_scan(kept_r);
+        if (lane == crank) {
+            sh.cta_kept = ik - kept_r;
+            sh.cta_eq = 0;
+            sh.counts_known = 1;
+        }
     }
 
     // ---------------------------------------------------------------- ordered scan
-    // kept flag of token t; eq marks a key equal to thr that is ranked by index
-    // when only some of them are kept
-    auto flags = [&](int64_t t, bool& kept, bool& eq) {
-        kept = false;
-        eq = false;
-        if (t >= w1) return;
-        const bool prun = t >= p0 && t < p1;
-        if (mode == 1) {
-            kept = __ldcg(keep_in + t) != 0;
-        } else if (!prun) {
-            kept = true;
-        } else if (!do_select) {
-            kept = kk > 0;  // kk >= P keeps all, kk == 0 keeps none
-        } else {
-            const uint32_t key = cached ? skeys[t - k0] : score_key(__ldcg(scores + t));
-            kept = key > thr || (key == thr && all_eq_kept);
-            eq = key == thr && !all_eq_kept;
+    // Each lane takes 4 consecutive tokens of its warp's run (128 per warp and step).  flags4
+    // sets bit i of kmask when token t + i is kept and of emask when it is a key equal to thr
+    // ranked by index (only some of those are kept); t - t0 is a multiple of 4.
+    auto flags4 = [&](int t, unsigned& kmask, unsigned& emask) {
+        kmask = 0u;
+        emask = 0u;
+        uint32_t key[4] = {0u, 0u, 0u, 0u};
+        if (do_select) {
+            if (cached) {
+                const uint4 q = *reinterpret_cast<const uint4*>(skeys + (t - t0));
+                key[0] = q.x;
+                key[1] = q.y;
+                key[2] = q.z;
+                key[3] = q.w;
+            } else {
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    if (t + i < w1 && t + i >= p0 && t + i < p1) key[i] = score_key(__ldcg(scores + t + i));
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int ti = t + i;
+            if (ti >= w1) break;
+            const bool prun = ti >= p0 && ti < p1;
+            bool kept, eq = false;
+            if (mode == 1) {
+                kept = __ldcg(keep_in + ti) != 0;
+            } else if (!prun) {
+                kept = true;
+            } else if (!do_select) {
+                kept = kk > 0;  // kk >= P keeps all, kk == 0 keeps none
+            } else {
+                kept = key[i] > thr || (key[i] == thr && all_eq_kept);
+                eq = key[i] == thr && !all_eq_kept;
+            }
+            kmask |= (kept ? 1u : 0u) << i;
+            emask |= (eq ? 1u : 0u) << i;
         }
     };
     const unsigned lt_mask = (1u << lane) - 1u;
 
     // warp totals: kept tokens and (for the tie ranking) keys equal to thr
     int my_kept = 0, my_eq = 0;
-#pragma unroll 4
-    for (int64_t base = w0; base < w1; base += 32) {
-        bool kept, eq;
-        flags(base + lane, kept, eq);
-        my_kept += __popc(__ballot_sync(0xffffffffu, kept));
-        my_eq += __popc(__ballot_sync(0xffffffffu, eq));
+    for (int base = w0; base < w1; base += 128) {
+        unsigned km, em;
+        flags4(base + 4 * lane, km, em);
+        my_kept += __popc(km);
+        my_eq += __popc(em);
     }
+    my_kept = warp_sum(my_kept);
+    my_eq = warp_sum(my_eq);
     if (lane == 0) {
         sh.warp_kept[warp] = my_kept;
         sh.warp_eq[warp] = my_eq;
@@ -352,14 +510,16 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
         }
     }
     SEL_TRACE(8);
-    cl.sync();  // slice totals published; also orders the key cache before the emission
-    SEL_TRACE(9);
-    // every CTA read the score kernel's counts before the barrier above: zero them for the next
-    // call, each CTA its eighth
-    if (key_hist != nullptr && tid < SEL_BINS / SEL_CL)
-        key_hist[static_cast<int64_t>(b) * SEL_BINS + crank * (SEL_BINS / SEL_CL) + tid] = 0;
-    int64_t kept_before = sh.warp_kept[warp], eq_before = sh.warp_eq[warp];
-    {
+    const bool counts_known = sh.counts_known != 0;  // uniform over the cluster
+    int cta_kept, cta_eq;
+    if (counts_known) {
+        __syncthreads();  // the warp prefixes and this CTA's totals are in place
+        cta_kept = sh.cta_kept;
+        cta_eq = sh.cta_eq;
+    } else {
+        cl.sync();  // slice totals published
+        cta_kept = 0;
+        cta_eq = 0;
         int vk[SEL_CL], ve[SEL_CL];
 #pragma unroll
         for (int r = 0; r < SEL_CL; ++r) {
@@ -370,42 +530,102 @@ select_scan_kernel(int mode, const float* __restrict__ scores, const uint8_t* __
 #pragma unroll
         for (int r = 0; r < SEL_CL; ++r) {
             if (r < crank) {
-                kept_before += vk[r];
-                eq_before += ve[r];
+                cta_kept += vk[r];
+                cta_eq += ve[r];
             }
         }
     }
-    SEL_TRACE(6);
+    SEL_TRACE(9);
     cluster_arrive_release();  // no remote reads after this point
+    // every CTA read the score kernel's counts before a cluster barrier above (the first pass's,
+    // or the exchange's): zero them for the next call, each CTA its eighth
+    if (key_hist != nullptr && tid < SEL_BINS / SEL_CL)
+        key_hist[static_cast<int64_t>(b) * SEL_BINS + crank * (SEL_BINS / SEL_CL) + tid] = 0;
     SEL_TRACE(7);
+
     // kept_before counts the tie-ranked keys as not kept; min(eq_before, need_eq) of
     // those before this warp's run are kept
-    int64_t m = m0 + kept_before + (all_eq_kept ? 0 : min(eq_before, need_eq));
-    int64_t eq_seen = eq_before;
-    for (int64_t base = w0; base < w1; base += 32) {
-        const int64_t t = base + lane;
-        bool kept, eq;
-        flags(t, kept, eq);
-        const unsigned eq_ball = __ballot_sync(0xffffffffu, eq);
-        if (eq && eq_seen + __popc(eq_ball & lt_mask) < need_eq) kept = true;
-        eq_seen += __popc(eq_ball);
-        const unsigned kept_ball = __ballot_sync(0xffffffffu, kept);
-        if (t < w1) {
-            if (mode == 0) keep_out[t] = kept ? 1 : 0;
-            const int64_t mi = m + __popc(kept_ball & lt_mask);
-            // a caller-given keep vector that disagrees with cu_kept must not
-            // write outside [m0, m1)
-            if (emit && kept && mi < m1) {
+    const int kept_before = cta_kept + sh.warp_kept[warp], eq_before = cta_eq + sh.warp_eq[warp];
+    const int m_cta = m0 + cta_kept + (all_eq_kept ? 0 : min(cta_eq, need_eq));  // this slice's first entry
+    const int n_cta = sh.xchg[0] + (all_eq_kept ? 0 : min(cta_eq + sh.xchg[1], need_eq) - min(cta_eq, need_eq));
+    const int m_warp = m0 + kept_before + (all_eq_kept ? 0 : min(eq_before, need_eq));
+
+    // Emission: a walk over the chunks numbers the kept tokens (and writes the keep flags in
+    // its first round); each round lists the tokens of up to SEL_LIST consecutive entries in
+    // shared memory, and the threads then write those entries of the map densely.
+    const int rounds = max(emit ? (n_cta + SEL_LIST - 1) / SEL_LIST : 0, mode == 0 ? 1 : 0);
+    // a lane's 4 tokens start at an offset from s0 that is a multiple of 4
+    const bool keep_words = ((reinterpret_cast<uintptr_t>(keep_out) + static_cast<uintptr_t>(s0)) & 3u) == 0;
+    for (int round = 0; round < rounds; ++round) {
+        const int j_lo = round * SEL_LIST;
+        int m = m_warp - m_cta;  // this slice's entry index of the warp's next kept token
+        int eq_seen = eq_before;
+        for (int base = w0; base < w1; base += 128) {
+            const int t = base + 4 * lane;
+            unsigned km, em;
+            flags4(t, km, em);
+            if (!all_eq_kept) {  // the first need_eq keys equal to thr, by index, are kept
+                unsigned eb[4];
+                int before = eq_seen;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    eb[i] = __ballot_sync(0xffffffffu, (em >> i) & 1u);
+                    before += __popc(eb[i] & lt_mask);
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    if (((em >> i) & 1u) && before + __popc(em & ((1u << i) - 1u)) < need_eq) km |= 1u << i;
+                eq_seen += __popc(eb[0]) + __popc(eb[1]) + __popc(eb[2]) + __popc(eb[3]);
+            }
+            int j = m - j_lo, step = 0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const unsigned kb_ = __ballot_sync(0xffffffffu, (km >> i) & 1u);
+                j += __popc(kb_ & lt_mask);
+                step += __popc(kb_);
+            }
+            if (mode == 0 && round == 0) {
+                if (keep_words && t + 3 < w1) {  // the 4 flags as one 4-byte store
+                    *reinterpret_cast<uint32_t*>(keep_out + t) =
+                        (km & 1u) | ((km & 2u) << 7) | ((km & 4u) << 14) | ((km & 8u) << 21);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        if (t + i < w1) keep_out[t + i] = (km >> i) & 1u;
+                }
+            }
+            if (emit) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    if ((km >> i) & 1u) {  // kept tokens lie below w1
+                        if (j >= 0 && j < SEL_LIST) list[j] = t + i;
+                        ++j;
+                    }
+                }
+            }
+            m += step;
+        }
+        if (round == 0) SEL_TRACE(6);
+        if (!emit) break;
+        __syncthreads();  // the round's list is complete
+        if (round == 0) SEL_TRACE(15);
+        const int n_round = min(SEL_LIST, n_cta - j_lo);
+        for (int j = tid; j < n_round; j += SEL_THREADS) {
+            const int t = list[j];
+            const int mi = m_cta + j_lo + j;
+            // a caller-given keep vector that disagrees with cu_kept must not write
+            // outside [m0, m1)
+            if (mi < m1) {
                 const bool prun = t >= p0 && t < p1;
                 float g = 0.0f;
-                if (prun) g = logsigmoid_f(cached ? key_to_score(skeys[t - k0]) : __ldcg(scores + t));
-                kept_idx[mi] = static_cast<int32_t>(t);
-                pos[mi] = static_cast<int32_t>(t - s0 + 1);
-                rank[mi] = static_cast<int32_t>(mi - m0 + 1);
+                if (prun) g = logsigmoid_f(cached ? key_to_score(skeys[t - t0]) : __ldcg(scores + t));
+                kept_idx[mi] = t;
+                pos[mi] = t - s0 + 1;
+                rank[mi] = mi - m0 + 1;
                 gls[mi] = g;
             }
         }
-        m += __popc(kept_ball);
+        __syncthreads();  // the list is read before the next round writes it
     }
     SEL_TRACE(10);
     cluster_wait_acquire();
@@ -507,13 +727,13 @@ extern "C" __attribute__((visibility("default"))) int tg_trace_read_select(unsig
 cudaError_t launch_select_scan(int mode, const float* scores, const uint8_t* keep_in, const int32_t* cu_seqlens,
                                const int32_t* span, const int32_t* k, const int32_t* cu_kept, int B, int64_t T,
                                uint8_t* keep_out, int32_t* kept_idx, int32_t* pos, int32_t* rank, float* gls,
-                               cudaStream_t st, int* key_hist) {
+                               cudaStream_t st, int* key_hist, bool early) {
     static std::atomic<uint64_t> attr_set{0};
     if (cudaError_t e = ensure_smem_limit(select_scan_kernel, SEL_SMEM_BYTES, attr_set); e != cudaSuccess)
         return e;
     if (B == 0) return cudaSuccess;
     return launch_pdl(select_scan_kernel, dim3(SEL_CL, B), dim3(SEL_THREADS), static_cast<size_t>(SEL_SMEM_BYTES), st,
-                      mode, scores, keep_in, cu_seqlens, span, k, cu_kept, keep_out, kept_idx, pos, rank, gls,
+                      mode, early ? 1 : 0, scores, keep_in, cu_seqlens, span, k, cu_kept, keep_out, kept_idx, pos, rank, gls,
                       key_hist);
 }
 

@@ -568,7 +568,7 @@ tg_status tg_gated_prefill_layer(const tg_prefill_layer_args* a, tg_stream_t str
         return s;
     if (tg_status s = cuda_status(tg::launch_select_scan(0, a->scores, nullptr, a->cu_seqlens, a->span, a->k,
                                                          a->cu_kept, a->B, a->T, a->keep, a->kept_idx, a->pos, a->rank,
-                                                         a->gls, st, key_hist),
+                                                         a->gls, st, key_hist, true),
                                   "select launch"))
         return s;
     if (a->M_total == 0) return TG_OK;  // every token pruned: no kept rows, no attention

@@ -128,10 +128,13 @@ cudaError_t launch_score(const uint16_t* hidden, const int32_t* cu_seqlens, cons
 // mode 1: compaction scan from caller-given keep flags
 // key_hist (may be NULL): the score kernel's first-pass histogram of these scores; the
 // selection then starts from its second pass and zeroes key_hist before it exits.
+// early: cu_seqlens, span, k and cu_kept are complete before the kernel's predecessor
+// releases it (the caller's, behind a predecessor that waits for the caller's work before it
+// releases its dependents), so the kernel reads them before its own wait.
 cudaError_t launch_select_scan(int mode, const float* scores, const uint8_t* keep_in, const int32_t* cu_seqlens,
                                const int32_t* span, const int32_t* k, const int32_t* cu_kept, int B, int64_t T,
                                uint8_t* keep_out, int32_t* kept_idx, int32_t* pos, int32_t* rank, float* gls,
-                               cudaStream_t st, int* key_hist = nullptr);
+                               cudaStream_t st, int* key_hist = nullptr, bool early = false);
 
 // dst[m, :] = src[kept_idx[m], :] for rows of row_bytes bytes (4, 8 or a multiple of 16;
 // both pointers aligned to min(row_bytes, 16)); rows whose index lies outside [0, T) are

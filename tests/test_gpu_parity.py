@@ -231,12 +231,15 @@ def test_select_degenerate_score_ranges(tg, n):
             _select_and_compact(tg, [0, n], [[0, n]], [k], s)
 
 
-def test_select_large_span_uncached_path(tg):
-    """A span longer than the shared-memory key cache (global re-reads)."""
-    n = 131072
+@pytest.mark.parametrize("n", [131072, 300000])
+def test_select_large_spans(tg, n):
+    """Long spans: 16k tokens per CTA (a CTA that keeps most of them writes its compaction
+    map in several rounds of 4096 entries), and 37.9k tokens per CTA, more than the shared-
+    memory key cache holds (keys re-read from global memory, chunk ballots recomputed)."""
     s = make_scores(n, std=2.0, seed=9)
     s[::7] = s[3]                      # plant ties at the threshold neighbourhood
-    _select_and_compact(tg, [0, n], [[128, n - 128]], [2000], s)
+    for k in (2000, n // 2, -1):
+        _select_and_compact(tg, [0, n], [[128, n - 128]], [k], s)
 
 
 def test_select_varlen_edge_sequences(tg):
@@ -427,6 +430,78 @@ def test_prefill_first_pass_in_the_score_kernel(tg, name):
         np.testing.assert_array_equal(a, b_)
     for a, b_ in zip(outs[0], outs[2]):
         np.testing.assert_array_equal(a, b_)
+
+
+def _score_key_bucket(x):
+    """Top 11 bits of the order-preserving uint32 key of fp32 scores (the selection's
+    first-pass bucket)."""
+    u = np.asarray(x, np.float32).view(np.uint32).astype(np.uint64)
+    key = np.where(u & 0x80000000, ~u & 0xFFFFFFFF, u | 0x80000000)
+    return key >> 21
+
+
+def test_prefill_selection_when_the_first_pass_ends_the_search(tg):
+    """Hidden rows of two kinds whose scores a > b lie in different first-pass buckets (their
+    magnitudes differ by more than 2x, or their signs), with K the number of a-rows in the
+    span: the score kernel's histogram alone ends the search (every key of the chosen bucket
+    is taken), so the selection runs no bucket pass and exchanges the slice totals across the
+    cluster.  The kinds are interleaved at random over 16k tokens, so every CTA's slice keeps
+    some tokens and drops others.  Keep flags and compaction map equal the oracle's on the
+    oracle's scores, with the first-pass histogram and without it."""
+    from learned_token_pruning_rmsnorm_b200 import PrefillBuffers, PrefillCall, _lib
+    from workloads.configs import Workload
+    T, span = 16384, (100, 16300)
+    base = Workload(name="two_kinds_16k", seqlens=(T,), spans=(span,), budgets=(0,), D=256, I=64, Hq=4, Hkv=2,
+                    d=64, seed=21)
+    gi = make_gate_inputs(base)
+    Wg_ref = oracle.gate_fold(gi["gamma"], gi["W1"])
+    cand = gi["hidden"][:16]
+    sc = oracle.score(cand, np.array([0, 16], np.int32), np.array([[0, 16]], np.int32), Wg_ref, gi["b1"],
+                      gi["w2"], gi["b2"], base.eps)
+    pair = None
+    for i in range(16):
+        for j in range(16):
+            a, b_ = sc[i], sc[j]
+            if a > b_ and min(abs(a), abs(b_)) > 1e-3 and (np.sign(a) != np.sign(b_) or
+                                                             max(abs(a), abs(b_)) > 2.5 * min(abs(a), abs(b_))):
+                pair = (i, j)
+                break
+        if pair:
+            break
+    assert pair is not None
+    assert _score_key_bucket(sc[pair[0]]) != _score_key_bucket(sc[pair[1]])
+    kind_a = np.random.default_rng(5).random(T) < 0.1
+    hidden = np.where(kind_a[:, None], cand[pair[0]], cand[pair[1]]).astype(np.uint16)
+    K = int(kind_a[span[0]:span[1]].sum())
+    w = Workload(name="two_kinds_16k", seqlens=(T,), spans=(span,), budgets=(K,), D=256, I=64, Hq=4, Hkv=2,
+                 d=64, seed=21)
+    cu, spans, k = w.cu_seqlens(), w.span_array(), w.budget_array()
+    s_ref = oracle.score(hidden, cu, spans, Wg_ref, gi["b1"], gi["w2"], gi["b2"], w.eps)
+    s_ref32 = np.where(np.isnan(s_ref), 0.0, s_ref).astype(np.float32)
+    keep_ref = oracle.select_topk(s_ref32, cu, spans, k)
+    comp_ref = oracle.compact(hidden, s_ref32, keep_ref, cu, spans)
+    M = int(comp_ref["cu_kept"][-1])
+    assert M == T - (span[1] - span[0]) + K
+    a = make_attention_inputs(w, M, layer=0)
+    layers = [{"q": H.bf16_dev(a["q"]), "k": H.bf16_dev(a["k"]), "v": H.bf16_dev(a["v"]),
+               "g": H.f32_dev(a["g"]), "c": H.f32_dev(a["c"])}]
+    hid = H.bf16_dev(hidden)
+    lib = _lib.load()
+    attn_bytes = int(lib.tg_gated_attention_workspace_size(1, M, w.Hq, w.Hkv, w.d))
+    for fused in (True, False):
+        bufs = PrefillBuffers(w.T, w.D, M, 1, w.Hq, w.d, hid.device, True, True)
+        call = PrefillCall(hid, cu, spans, k, H.bf16_dev(Wg_ref), H.f32_dev(gi["b1"]), H.f32_dev(gi["w2"]),
+                           gi["b2"], w.eps, layers, bufs, w.Hq, w.Hkv, w.d)
+        if not fused:
+            call.args.attn_ws_bytes = attn_bytes
+        call()
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(bufs.keep.cpu().numpy(), keep_ref)
+        np.testing.assert_array_equal(bufs.kept_idx.cpu().numpy(), comp_ref["src"])
+        np.testing.assert_array_equal(bufs.pos.cpu().numpy(), comp_ref["pos"])
+        np.testing.assert_array_equal(bufs.rank.cpu().numpy(), comp_ref["rank"])
+        np.testing.assert_array_equal(H.bf16_host_bits(bufs.hidden_kept), comp_ref["hidden_kept"])
+        assert np.max(np.abs(bufs.gls.cpu().numpy() - comp_ref["gls"])) <= 1e-5
 
 
 # ------------------------------------------------------------------ KV-cache gather (next row f2)
