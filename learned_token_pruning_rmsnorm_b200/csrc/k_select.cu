@@ -106,13 +106,15 @@ __device__ __forceinline__ float key_to_score(uint32_t key) {
 
 __device__ __forceinline__ int bit_length(uint64_t v) { return v ? 64 - __clzll(static_cast<long long>(v)) : 0; }
 
-// split cluster barrier: arrive once this CTA reads no more remote shared
-// memory, wait before leaving so that no CTA exits while another reads it
-__device__ __forceinline__ void cluster_arrive_release() {
-    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+// split cluster barrier: arrive once this CTA reads no more remote shared memory, wait
+// before leaving so that no CTA exits while another reads it.  The arrive is relaxed: every
+// value read remotely has been consumed before it, and no CTA reads what this one writes
+// after it, so it needs no memory fence.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 }
-__device__ __forceinline__ void cluster_wait_acquire() {
-    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+__device__ __forceinline__ void cluster_wait() {
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
 }
 
 // Token slice [a0, a1) of cluster rank r: SEL_CL slices of `per` tokens (a multiple of
@@ -536,7 +538,7 @@ select_scan_kernel(int mode, int early, const float* __restrict__ scores, const 
         }
     }
     SEL_TRACE(9);
-    cluster_arrive_release();  // no remote reads after this point
+    cluster_arrive_relaxed();  // no remote reads after this point
     // every CTA read the score kernel's counts before a cluster barrier above (the first pass's,
     // or the exchange's): zero them for the next call, each CTA its eighth
     if (key_hist != nullptr && tid < SEL_BINS / SEL_CL)
@@ -628,7 +630,7 @@ select_scan_kernel(int mode, int early, const float* __restrict__ scores, const 
         __syncthreads();  // the list is read before the next round writes it
     }
     SEL_TRACE(10);
-    cluster_wait_acquire();
+    cluster_wait();
     SEL_TRACE(11);
 }
 
