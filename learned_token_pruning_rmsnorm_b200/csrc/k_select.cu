@@ -552,7 +552,7 @@ select_scan_kernel(int mode, int early, const float* __restrict__ scores, const 
     const int n_cta = sh.xchg[0] + (all_eq_kept ? 0 : min(cta_eq + sh.xchg[1], need_eq) - min(cta_eq, need_eq));
     const int m_warp = m0 + kept_before + (all_eq_kept ? 0 : min(eq_before, need_eq));
 
-    // Emission: a walk over the chunks numbers the kept tokens (and writes the keep flags in
+    // Emission: a walk over each warp's run numbers the kept tokens (and writes the keep flags in
     // its first round); each round lists the tokens of up to SEL_LIST consecutive entries in
     // shared memory, and the threads then write those entries of the map densely.
     const int rounds = max(emit ? (n_cta + SEL_LIST - 1) / SEL_LIST : 0, mode == 0 ? 1 : 0);

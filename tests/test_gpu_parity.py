@@ -235,7 +235,7 @@ def test_select_degenerate_score_ranges(tg, n):
 def test_select_large_spans(tg, n):
     """Long spans: 16k tokens per CTA (a CTA that keeps most of them writes its compaction
     map in several rounds of 4096 entries), and 37.9k tokens per CTA, more than the shared-
-    memory key cache holds (keys re-read from global memory, chunk ballots recomputed)."""
+    memory key cache holds (keys re-read from global memory)."""
     s = make_scores(n, std=2.0, seed=9)
     s[::7] = s[3]                      # plant ties at the threshold neighbourhood
     for k in (2000, n // 2, -1):
