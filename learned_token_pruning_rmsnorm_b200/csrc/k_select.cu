@@ -453,6 +453,10 @@ select_scan_kernel(int mode, int early, const float* __restrict__ scores, const 
         uint32_t key[4] = {0u, 0u, 0u, 0u};
         if (do_select) {
             if (cached) {
+                // In bounds: a warp's last step overruns its run by less than 128 tokens, so
+                // t - t0 + 3 < SEL_CACHE_KEYS for every t a lane reaches (per <= SEL_CACHE_KEYS,
+                // a multiple of 1024).  Slots of tokens outside [k0, k1) hold stale values, read
+                // only for tokens that ignore their key (outside the span or past the run).
                 const uint4 q = *reinterpret_cast<const uint4*>(skeys + (t - t0));
                 key[0] = q.x;
                 key[1] = q.y;
